@@ -21,6 +21,8 @@ Definition (all integer arithmetic modulo 2^64):
       z = mix(base_t + gamma * (e + 1))
       S = sum of the four 16-bit fields of z            (0 <= S <= 262140)
       w = fp64(S - 131070) * K,   K = (init_std * 1.7320508075688772) / 65536
+  with init_std taken as its fp32 value (the type of the config field in
+  the library's C ABI) and K evaluated in fp64, left to right.
 
   S/65536 - 2 is the Irwin-Hall sum of four uniforms on (0, 1) minus its
   mean (variance 1/3), so w has mean 0 and standard deviation init_std,
@@ -114,7 +116,7 @@ def round_fp32_to_bf16(x32: np.ndarray) -> np.ndarray:
 def draw_tensor(seed: int, t: int, numel: int, init_std: float, dtype: str,
                 chunk: int = 1 << 22) -> np.ndarray:
     """Values of tensor t as float32 (already rounded to the storage precision)."""
-    K = (init_std * SQRT3) / 65536.0
+    K = (float(np.float32(init_std)) * SQRT3) / 65536.0
     with np.errstate(over="ignore"):
         base = mix64(np.uint64(seed) + GAMMA * np.uint64(t + 1))
     out = np.empty(numel, dtype=np.float32)
