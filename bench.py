@@ -1,0 +1,409 @@
+"""PHOTON RecGen decode benchmark on B200 (one process per GPU).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload c2] [--impl reference]
+
+One bench step is one pass of the whole hot path over one batch: the
+hierarchical prefill of the workload's prompts (RecGen mode) followed by the
+workload's RecGen decode (512 tokens per sequence for the 600M-class batch-64
+workload = 32 top-level chunks).  Inputs are synthetic (seeded weights,
+Zipf(1.1) prompts) and already resident in HBM when the timed region starts.
+
+Reported (rank 0, one JSON line):
+  value        RecGen decode tokens/s of the whole job: decoded tokens of all
+               ranks / (max over ranks of the summed decode time of the K
+               timed steps), CUDA events on the launching stream;
+  tpm          value / GiB of resident weights + KV (and KV only);
+  prefill      prefill tokens/s over the same steps;
+  e2e          the same metric through the public API with host buffers:
+               prompt copied from pinned host memory and every chunk's tokens
+               read back each decode step, copies inside the timed region;
+  roofline     the dominant decode kernel's achieved bandwidth against the
+               measured HBM copy peak;
+  cpu_baseline the CPU oracle timed on a bounded sample on the host cores.
+Between timed steps nothing is flushed: the step's working set (0.66 GB of
+decoder+top weights streamed per chunk, 0.9 GB of top KV) exceeds the 126 MB L2.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from synth_inputs import WEIGHT_SEED, WORKLOADS, model_shape, prompt_tokens  # noqa: E402
+
+METRIC = "RecGen decode tok/s and tok/s/GiB (TPM) on 1 B200; % of HBM roofline"
+UNIT = "tok/s"
+
+
+def _peaks() -> tuple[dict, str]:
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        return json.load(open(p)), "measured"
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+            "sm_max_mhz": 1965.0}, "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi samples (200 ms) while the timed region runs."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.idx = gpu_index
+        self.proc = None
+        self.lines: list[str] = []
+        self.t = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.idx}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except (OSError, ValueError):
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self) -> dict:
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            f = [x.strip() for x in ln.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx = float(f[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def run_gpu(args) -> None:
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+
+    import hierarchical_autoregressive_lm_b200 as hal
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        from datetime import timedelta
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=timedelta(seconds=300),
+                                device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(0)
+    dev = torch.device("cuda", torch.cuda.current_device())
+
+    wl = WORKLOADS[args.workload]
+    shape = model_shape(args.workload)
+    B, T = wl["batch"], wl["prompt_len"]
+    model = hal.Model(shape, WEIGHT_SEED)
+    C = model.C
+    chunks = wl["decode_tokens"] // C
+    # data parallel over sequences: every rank decodes its own batch of B
+    # sequences (weak scaling); rank r takes rows [r*B, (r+1)*B) of a
+    # world-sized prompt set, so no two ranks hold the same prompt.
+    toks_all = prompt_tokens(args.workload) if world == 1 else None
+    if toks_all is None:
+        from synth_inputs import zipf_tokens
+        toks_all = zipf_tokens(B * world, T, wl["vocab"], wl["prompt_seed"])
+    toks_host = torch.from_numpy(np.ascontiguousarray(toks_all[rank * B:(rank + 1) * B]))
+    toks = toks_host.to(dev)
+    out = torch.empty(B, chunks * C, dtype=torch.int32, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def one_step(ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        cache = model.prefill(toks, hal.MODE_REC, chunks)
+        if ev is not None:
+            ev[1].record(stream)
+        for s in range(chunks):
+            cache.step_rec(out[:, s * C:(s + 1) * C])
+        if ev is not None:
+            ev[2].record(stream)
+        return cache
+
+    # warm-up (also settles the stream-ordered allocator)
+    for _ in range(args.warmup):
+        one_step().free()
+    torch.cuda.synchronize()
+
+    # resident memory during decode: weights now on the device + this cache's KV
+    probe = one_step()
+    torch.cuda.synchronize()
+    cinfo, minfo = probe.info(), model.info()
+    probe.free()
+    resident = minfo["resident_bytes"] + cinfo["kv_bytes"]
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    caches = []
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(dev.index) as clk:
+        t0 = torch.cuda.Event(enable_timing=True)
+        t1 = torch.cuda.Event(enable_timing=True)
+        t0.record(stream)
+        for k in range(args.steps):
+            caches.append(one_step(evs[k]))
+            if len(caches) > 1:          # keep at most two caches alive
+                caches.pop(0).free()
+        t1.record(stream)
+        torch.cuda.synchronize()
+    for c in caches:
+        c.free()
+    if world > 1:
+        dist.barrier()
+    total_ms = t0.elapsed_time(t1)
+    prefill_ms = sum(e[0].elapsed_time(e[1]) for e in evs)
+    decode_ms = sum(e[1].elapsed_time(e[2]) for e in evs)
+
+    # ---- end to end through the public API with host buffers
+    pin_in = toks_host.pin_memory()
+    pin_out = torch.empty(B, chunks * C, dtype=torch.int32).pin_memory()
+    dev_in = torch.empty_like(toks)
+    e2e_steps = max(1, min(args.steps, 3))
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        dev_in.copy_(pin_in, non_blocking=True)
+        cache = model.prefill(dev_in, hal.MODE_REC, chunks)
+        for s in range(chunks):
+            sl = out[:, s * C:(s + 1) * C]
+            cache.step_rec(sl)
+            pin_out[:, s * C:(s + 1) * C].copy_(sl, non_blocking=True)
+        cache.free()     # synchronises
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1)
+
+    # ---- dominant decode kernel alone, same shapes and launch configuration
+    roof = measure_roofline(model, wl, dev, stream)
+
+    times = torch.tensor([total_ms, prefill_ms, decode_ms, e2e_ms], device=dev, dtype=torch.float64)
+    if world > 1:
+        dist.all_reduce(times, op=dist.ReduceOp.MAX)
+    total_ms, prefill_ms, decode_ms, e2e_ms = times.tolist()
+
+    dec_tokens = world * B * chunks * C * args.steps
+    value = dec_tokens / (decode_ms / 1e3)
+    gib = resident / 2 ** 30
+    line = {
+        "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(total_ms / args.steps, 3), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": shape["dtype"],
+        "data": "synthetic: seeded N(0,0.02)-like weights (SplitMix64 + Irwin-Hall), Zipf(1.1) prompt ids",
+        "config": {"workload": f"{args.workload}: PHOTON 600M-class L=2 C1=C2={shape['C1']}, "
+                               f"B={B} per GPU, prompt {T}, RecGen decode {chunks * C} tokens",
+                   "batch_per_gpu": B, "prompt_len": T, "decode_tokens": chunks * C,
+                   "parallelism": f"dp{world}", "l2": "working set > L2 (no flush)"},
+        "decode_ms_per_step": round(decode_ms / args.steps, 3),
+        "decode_ms_per_chunk": round(decode_ms / args.steps / chunks, 4),
+        "prefill_tok_s": round(world * B * T * args.steps / (prefill_ms / 1e3), 1),
+        "job_tok_s": round(dec_tokens / (total_ms / 1e3), 1),
+        "tpm": {"tok_s_per_gib": round(value / world / gib, 1), "resident_gib": round(gib, 4),
+                "weights_gib": round(minfo["resident_bytes"] / 2 ** 30, 4),
+                "kv_gib": round(cinfo["kv_bytes"] / 2 ** 30, 4),
+                "tok_s_per_gib_kv_only": round(value / world / (cinfo["kv_bytes"] / 2 ** 30), 1),
+                "per_gpu": True},
+        "e2e": {"value": round(world * B * chunks * C * e2e_steps / (e2e_ms / 1e3), 1), "unit": UNIT,
+                "h2d_bytes_per_step": int(B * T * 4), "d2h_bytes_per_step": int(B * chunks * C * 4),
+                "covers": "H2D prompt + prefill + RecGen decode + per-chunk D2H of tokens"},
+        "gpu_launches": launch_count(model, wl, B) * args.steps,
+        "roofline": roof,
+        "clocks": clk.summary(),
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(args.workload, budget_s=args.cpu_budget)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    model.free()
+    if world > 1:
+        dist.destroy_process_group()
+
+
+def launch_count(model, wl, B) -> int:
+    """Kernels the library launches for one prefill + the decode chunks
+    (counted from the launch sequences in runtime.cu)."""
+    s = model.shape
+    C1, C2, chunks = s["C1"], s["C2"], wl["decode_tokens"] // (s["C1"] * s["C2"])
+    M = B  # rows of the smallest GEMMs; split-K adds one reduction launch per split GEMM
+    per_block = 8            # 2 norms + 4 GEMMs + attention (+ combine) ~ 8 launches
+    prefill = 3 + per_block * (s["L1"] + s["Ltop"]) + 2
+    dec = (1 + per_block * s["Ld2"] + 1 + 1 + per_block * s["Ld1"] + 3
+           + (C1 - 1) * (1 + per_block * s["Ld1"] + 3) + 1 + per_block * s["Ltop"] + 1)
+    del M
+    return prefill + chunks * dec
+
+
+def measure_roofline(model, wl, dev, stream) -> dict:
+    """Times the split-K decode attention of the top encoder alone at the
+    decode's shapes (B sequences, H heads, N top entries averaged over the
+    decode, all Ltop layers in turn so the 0.9 GB working set exceeds L2)."""
+    import torch
+    import hierarchical_autoregressive_lm_b200 as hal
+    s = model.shape
+    B, H, dh = wl["batch"], s["n_heads"], s["head_dim"]
+    C = s["C1"] * s["C2"]
+    chunks = wl["decode_tokens"] // C
+    N0 = wl["prompt_len"] // C
+    cap = N0 + chunks
+    n_mid = N0 + chunks // 2          # keys seen by the middle decode step
+    L = s["Ltop"]
+    dt = torch.bfloat16 if s["dtype"] == "bf16" else torch.float32
+    g = torch.Generator(device=dev).manual_seed(7)
+    K = [torch.randn(B, H, cap, dh, device=dev, generator=g).to(dt) for _ in range(L)]
+    V = [torch.randn(B, H, cap, dh, device=dev, generator=g).to(dt) for _ in range(L)]
+    q = torch.randn(B, H * dh, device=dev, generator=g).to(dt)
+    o = torch.empty_like(q)
+    for l in range(L):                                    # warm-up
+        hal.attn_decode(q, K[l], V[l], 1, n_mid - 1, o)
+    torch.cuda.synchronize()
+    reps = 20
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for r in range(reps):
+        for l in range(L):
+            hal.attn_decode(q, K[l], V[l], 1, n_mid - 1, o)
+    b.record(stream)
+    torch.cuda.synchronize()
+    ms = a.elapsed_time(b) / (reps * L)
+    es = 2 if dt == torch.bfloat16 else 4
+    algo = 2 * B * H * n_mid * dh * es + 2 * B * H * dh * es   # K,V rows read + q read + o write
+    peaks, src = _peaks()
+    achieved = algo / (ms / 1e3) / 1e9
+    return {"kernel": "k_attn_decode (top-encoder split-K decode attention, with its combine)",
+            "bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"],
+            "unit": "GB/s", "frac": round(achieved / peaks["hbm_gbs"], 4),
+            "peak_source": f"{src} (STREAM-style copy)", "traffic": None,
+            "bytes_per_launch": algo, "us_per_launch": round(ms * 1e3, 3),
+            "shape": f"B={B} H={H} dh={dh} keys={n_mid}"}
+
+
+def cpu_baseline(workload: str, budget_s: float = 20.0) -> dict:
+    """The fp64 oracle, as it stands, on the host cores: RecGen decode of one
+    sequence of the workload after its prefill; decode steps are timed until
+    the budget is spent (prefill and weight generation are not timed)."""
+    import numpy as np
+    from oracle import Config, PhotonOracle
+    shape = model_shape(workload)
+    cfg = Config.from_dict(shape)
+    orc = PhotonOracle(cfg, WEIGHT_SEED)
+    toks = prompt_tokens(workload, batch=1)[0]
+    st = orc.prefill(toks, "rec")
+    n, t0 = 0, time.perf_counter()
+    chunks = WORKLOADS[workload]["decode_tokens"] // cfg.C
+    while n < chunks:
+        orc.decode_step(st, "rec")
+        n += 1
+        if time.perf_counter() - t0 > budget_s:
+            break
+    dt = time.perf_counter() - t0
+    cores = len(os.sched_getaffinity(0))
+    del np
+    return {"value": round(n * cfg.C / dt, 3), "unit": UNIT, "cores": cores, "kind": "oracle",
+            "sample": f"{workload}: 1 sequence, {n} RecGen chunks ({n * cfg.C} tokens) after its "
+                      f"prefill, fp64 NumPy, BLAS threads = {cores}"}
+
+
+def run_reference(args) -> None:
+    """The CPU oracle as the reference arm: same metric and config, a bounded sample."""
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    wl = WORKLOADS[args.workload]
+    from oracle import Config, PhotonOracle
+    shape = model_shape(args.workload)
+    cfg = Config.from_dict(shape)
+    orc = PhotonOracle(cfg, WEIGHT_SEED)
+    toks = prompt_tokens(args.workload, batch=1)[0]
+    st = orc.prefill(toks, "rec")
+    for _ in range(min(args.warmup, 1)):
+        orc.decode_step(st, "rec")
+    per = []
+    for _ in range(args.steps):
+        t0 = time.perf_counter()
+        orc.decode_step(st, "rec")
+        per.append(time.perf_counter() - t0)
+        if sum(per) > args.cpu_budget:
+            break
+    secs = sum(per)
+    value = len(per) * cfg.C / secs
+    cores = len(os.sched_getaffinity(0))
+    sample = (f"{args.workload}: 1 of {wl['batch']} sequences, {len(per)} RecGen chunks "
+              f"({len(per) * cfg.C} tokens) after its prefill, fp64 NumPy oracle")
+    print(json.dumps({
+        "impl": "reference", "metric": METRIC, "value": round(value, 3), "unit": UNIT,
+        "n_gpus": world, "steps": len(per), "warmup": args.warmup,
+        "ms_per_step": round(1e3 * secs / len(per), 3), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": args.workload, "batch_per_gpu": wl["batch"],
+                   "prompt_len": wl["prompt_len"], "decode_tokens": wl["decode_tokens"],
+                   "parallelism": "none (host cores)"},
+        "cpu_baseline": {"value": round(value, 3), "unit": UNIT, "cores": cores, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": round(value, 3), "unit": UNIT, "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }), flush=True)
+
+
+def main() -> None:
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=5)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--workload", default="c2", choices=["c2", "c3", "c4"])
+    ap.add_argument("--impl", default="photon", choices=["photon", "reference"])
+    ap.add_argument("--cpu-budget", type=float, default=20.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3 and args.impl != "reference":
+        args.warmup = 3
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_gpu(args)
+
+
+if __name__ == "__main__":
+    main()

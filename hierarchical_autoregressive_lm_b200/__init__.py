@@ -1,0 +1,252 @@
+"""B200-native PHOTON inference: hierarchical prefill, HierGen and RecGen decode.
+
+This package is a thin ctypes binding over the C ABI of libphoton.so
+(declared in include/photon.h): it marshals torch tensors' device pointers,
+CUDA streams and config structs, and raises PhotonError on a non-zero status.
+Every step of the computation runs in the library's CUDA kernels; there is
+no Python or CPU fallback -- importing works without a GPU, but any call
+needs the built library and a CUDA device.
+
+Build the library with `python -m hierarchical_autoregressive_lm_b200.build`.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+__all__ = ["PhotonError", "Model", "Cache", "load_library", "LIB_PATH", "MODE_HIER",
+           "MODE_REC", "STATE", "gemm", "attn_decode", "config_struct", "EXPORTED"]
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libphoton.so")
+
+MODE_HIER, MODE_REC = 0, 1
+STATE = {"top_k": 0, "top_v": 1, "l1_k": 2, "l1_v": 3, "pending_o": 4, "a_hat": 5, "a": 6}
+_DTYPES = {"fp32": 0, "bf16": 1}
+_ERRORS = {-1: "PHOTON_ERR_ARG", -2: "PHOTON_ERR_OOM", -3: "PHOTON_ERR_CUDA",
+           -4: "PHOTON_ERR_CAPACITY", -5: "PHOTON_ERR_MODE", -6: "PHOTON_ERR_DEVICE_CHECK"}
+
+# Every entry point of include/photon.h (checked against the header by the tests).
+EXPORTED = ("photon_init_weights", "photon_free_model", "photon_prefill",
+            "photon_decode_step_hier", "photon_decode_step_rec", "photon_decode_step_ex",
+            "photon_free_cache", "photon_cache_info", "photon_model_info",
+            "photon_export_weight", "photon_export_state", "photon_gemm",
+            "photon_attn_decode", "photon_last_error")
+
+
+class PhotonError(RuntimeError):
+    def __init__(self, code: int, msg: str):
+        super().__init__(f"{_ERRORS.get(code, code)}: {msg}")
+        self.code = code
+
+
+class photon_config(ctypes.Structure):
+    _fields_ = [("vocab", ctypes.c_int32), ("d_model", ctypes.c_int32),
+                ("n_heads", ctypes.c_int32), ("head_dim", ctypes.c_int32),
+                ("levels", ctypes.c_int32), ("chunk", ctypes.c_int32 * 2),
+                ("enc_layers", ctypes.c_int32 * 2), ("dec_layers", ctypes.c_int32 * 2),
+                ("mlp_mult", ctypes.c_int32), ("conv_kernel", ctypes.c_int32),
+                ("dtype", ctypes.c_int32), ("init_std", ctypes.c_float),
+                ("rope_theta", ctypes.c_float), ("norm_eps", ctypes.c_float)]
+
+
+class photon_cache_stats(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_int32) for n in
+                ("B", "T", "mode", "N", "N1", "n_prefix", "n1_prefix", "capacity", "steps",
+                 "max_new_chunks", "device_error", "l1_resident")] + \
+               [("kv_bytes", ctypes.c_uint64), ("workspace_bytes", ctypes.c_uint64)]
+
+
+class photon_model_stats(ctypes.Structure):
+    _fields_ = [("param_count", ctypes.c_uint64), ("resident_bytes", ctypes.c_uint64),
+                ("encoder_bytes", ctypes.c_uint64), ("encoder_resident", ctypes.c_int32),
+                ("n_tensors", ctypes.c_int32), ("live_caches", ctypes.c_int32),
+                ("tcgen05_gemm", ctypes.c_int32)]
+
+
+_lib: Optional[ctypes.CDLL] = None
+
+
+def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
+    """Loads libphoton.so (once) and declares the C signatures."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(path):
+        raise ImportError(f"{path} is missing: build it with "
+                          "`python -m hierarchical_autoregressive_lm_b200.build`")
+    L = ctypes.CDLL(path)
+    P, I32, I64, U64, SZ = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_uint64, ctypes.c_size_t
+    sig = {
+        "photon_init_weights": [ctypes.POINTER(photon_config), U64, ctypes.POINTER(P)],
+        "photon_free_model": [P],
+        "photon_prefill": [P, P, P, I32, I32, I32, I32, P, ctypes.POINTER(P)],
+        "photon_decode_step_hier": [P, P, P, P, P],
+        "photon_decode_step_rec": [P, P, P, P, P],
+        "photon_decode_step_ex": [P, P, I32, P, P, P, P, P],
+        "photon_free_cache": [P],
+        "photon_cache_info": [P, ctypes.POINTER(photon_cache_stats)],
+        "photon_model_info": [P, ctypes.POINTER(photon_model_stats)],
+        "photon_export_weight": [P, I32, P, SZ, ctypes.POINTER(SZ), P],
+        "photon_export_state": [P, I32, I32, P, SZ, ctypes.POINTER(SZ), P],
+        "photon_gemm": [I32, P, I64, P, I64, I32, I32, I32, P, I64, I32, I32, I32, P],
+        "photon_attn_decode": [I32, P, P, P, I32, I32, I32, I32, I32, I32, P, P],
+    }
+    for name, args in sig.items():
+        fn = getattr(L, name)
+        fn.argtypes = args
+        fn.restype = ctypes.c_int
+    L.photon_last_error.argtypes = []
+    L.photon_last_error.restype = ctypes.c_char_p
+    _lib = L
+    return L
+
+
+def _check(rc: int) -> None:
+    if rc != 0:
+        msg = load_library().photon_last_error().decode(errors="replace")
+        raise PhotonError(rc, msg)
+
+
+def _stream(stream) -> int:
+    import torch
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def _ptr(t) -> Optional[int]:
+    return None if t is None else t.data_ptr()
+
+
+def config_struct(shape: dict) -> photon_config:
+    """photon_config from a plain shape dict (keys of synth_inputs.MODEL_KEYS)."""
+    c = photon_config()
+    c.vocab, c.d_model = shape["vocab"], shape["d_model"]
+    c.n_heads, c.head_dim = shape["n_heads"], shape["head_dim"]
+    c.levels = 2
+    c.chunk[0], c.chunk[1] = shape["C1"], shape["C2"]
+    c.enc_layers[0], c.enc_layers[1] = shape["L1"], shape["Ltop"]
+    c.dec_layers[0], c.dec_layers[1] = shape["Ld1"], shape["Ld2"]
+    c.mlp_mult = shape.get("mlp_mult", 4)
+    c.conv_kernel = shape.get("conv_kernel", 0)
+    c.dtype = _DTYPES[shape["dtype"]]
+    c.init_std = shape.get("init_std", 0.02)
+    c.rope_theta = shape.get("rope_theta", 10000.0)
+    c.norm_eps = shape.get("norm_eps", 1e-6)
+    return c
+
+
+class Model:
+    """A PHOTON model on the current CUDA device (weights drawn from `seed`)."""
+
+    def __init__(self, shape: dict, seed: int):
+        L = load_library()
+        self.shape = dict(shape)
+        self.cfg = config_struct(shape)
+        h = ctypes.c_void_p()
+        _check(L.photon_init_weights(ctypes.byref(self.cfg), seed, ctypes.byref(h)))
+        self._h = h
+        self.C1, self.C2 = shape["C1"], shape["C2"]
+        self.C = self.C1 * self.C2
+        self.vocab, self.d_model = shape["vocab"], shape["d_model"]
+
+    @property
+    def torch_dtype(self):
+        import torch
+        return torch.float32 if self.cfg.dtype == 0 else torch.bfloat16
+
+    def info(self) -> dict:
+        st = photon_model_stats()
+        _check(load_library().photon_model_info(self._h, ctypes.byref(st)))
+        return {n: getattr(st, n) for n, _ in st._fields_}
+
+    def export_weight(self, index: int, stream=None):
+        """Stored values of parameter tensor `index` (generator order) as a flat tensor."""
+        import torch
+        L = load_library()
+        n = ctypes.c_size_t()
+        _check(L.photon_export_weight(self._h, index, None, 0, ctypes.byref(n), _stream(stream)))
+        buf = torch.empty(n.value, dtype=torch.uint8, device="cuda")
+        _check(L.photon_export_weight(self._h, index, _ptr(buf), n.value, None, _stream(stream)))
+        return buf
+
+    def prefill(self, tokens, mode: int, max_new_chunks: int, prefix: "Cache" = None,
+                stream=None) -> "Cache":
+        """tokens: CUDA int32 tensor [B, T] (contiguous)."""
+        assert tokens.is_cuda and tokens.dtype.itemsize == 4 and tokens.is_contiguous()
+        B, T = tokens.shape
+        h = ctypes.c_void_p()
+        _check(load_library().photon_prefill(self._h, None if prefix is None else prefix._h,
+                                             _ptr(tokens), B, T, mode, max_new_chunks,
+                                             _stream(stream), ctypes.byref(h)))
+        return Cache(self, h, B, prefix)
+
+    def free(self) -> None:
+        if self._h:
+            _check(load_library().photon_free_model(self._h))
+            self._h = None
+
+
+class Cache:
+    """Per-batch decode state (top KV, level-1 KV in HierGen mode, pending output)."""
+
+    def __init__(self, model: Model, handle, B: int, prefix: "Cache" = None):
+        self.model, self._h, self.B, self.prefix = model, handle, B, prefix
+
+    def decode_step(self, mode: int, out_tokens, out_logits=None, force_tokens=None,
+                    force_a=None, stream=None) -> None:
+        """One top-level chunk: out_tokens CUDA int32 [B, C1*C2]; optional fp32
+        logits [B, C1*C2, vocab]; optional teacher-forced tokens / forced A."""
+        _check(load_library().photon_decode_step_ex(
+            self.model._h, self._h, mode, _ptr(out_tokens), _ptr(out_logits),
+            _ptr(force_tokens), _ptr(force_a), _stream(stream)))
+
+    def step_rec(self, out_tokens, out_logits=None, stream=None) -> None:
+        _check(load_library().photon_decode_step_rec(self.model._h, self._h, _ptr(out_tokens),
+                                                     _ptr(out_logits), _stream(stream)))
+
+    def step_hier(self, out_tokens, out_logits=None, stream=None) -> None:
+        _check(load_library().photon_decode_step_hier(self.model._h, self._h, _ptr(out_tokens),
+                                                      _ptr(out_logits), _stream(stream)))
+
+    def info(self) -> dict:
+        st = photon_cache_stats()
+        _check(load_library().photon_cache_info(self._h, ctypes.byref(st)))
+        return {n: getattr(st, n) for n, _ in st._fields_}
+
+    def export_state(self, which: str, layer: int = 0, stream=None):
+        """Raw bytes of a piece of cache state (see PHOTON_STATE_* in photon.h)."""
+        import torch
+        L = load_library()
+        n = ctypes.c_size_t()
+        _check(L.photon_export_state(self._h, STATE[which], layer, None, 0, ctypes.byref(n),
+                                     _stream(stream)))
+        buf = torch.empty(max(1, n.value), dtype=torch.uint8, device="cuda")
+        _check(L.photon_export_state(self._h, STATE[which], layer, _ptr(buf), n.value, None,
+                                     _stream(stream)))
+        return buf[:n.value]
+
+    def free(self) -> None:
+        if self._h:
+            _check(load_library().photon_free_cache(self._h))
+            self._h = None
+
+
+def gemm(A, W, C, path: int = 0, splits: int = 0, swap: int = -1, stream=None) -> None:
+    """C[M, N] (fp32) = A[M, K] @ W[N, K]^T through the library's GEMM kernels."""
+    import torch
+    dt = 0 if A.dtype == torch.float32 else 1
+    M, K = A.shape
+    N = W.shape[0]
+    _check(load_library().photon_gemm(dt, _ptr(A), A.stride(0), _ptr(W), W.stride(0), M, N, K,
+                                      _ptr(C), C.stride(0), path, splits, swap, _stream(stream)))
+
+
+def attn_decode(q, k, v, q_len: int, p0: int, out, stream=None) -> None:
+    """Split-K decode attention: k, v [G, H, cap, dh]; q, out [G*q_len, H*dh]."""
+    import torch
+    dt = 0 if q.dtype == torch.float32 else 1
+    G, H, cap, dh = k.shape
+    _check(load_library().photon_attn_decode(dt, _ptr(q), _ptr(k), _ptr(v), G, H, dh, cap, q_len,
+                                             p0, _ptr(out), _stream(stream)))

@@ -1,0 +1,319 @@
+// Tensor-core GEMM for sm_100a: C = A[M,K] * W[N,K]^T, bf16 in, fp32
+// accumulate in tensor memory, fused epilogue.
+//
+// One CTA computes a 128 x BN accumulator tile D = Amma * Bmma^T:
+//   * normal orientation: Amma = activations (128 rows), Bmma = weights;
+//   * swapped orientation (few tokens, decode): Amma = weights (128 output
+//     features), Bmma = the M <= 256 token rows, so the weight matrix is
+//     streamed by many CTAs even when M is small.
+// Roles inside the 128-thread CTA: thread 0 issues TMA loads of 64-wide K
+// slices into a STAGES-deep ring (128-byte swizzle), thread 32 issues
+// tcgen05.mma (M=128, N=BN, K=16, four per slice) and commits each slice back
+// to the ring; then all four warps read the accumulator out of TMEM
+// (warp w owns TMEM lanes 32w..32w+31), stage it in shared memory as an
+// output-row-major tile and apply the epilogue with coalesced stores.
+// With split-K (grid.z > 1) each CTA covers a contiguous run of K slices and
+// writes its fp32 partial tile; a separate kernel sums the partials in a
+// fixed order and applies the epilogue, so results are deterministic.
+#include <cuda.h>
+
+#include <mutex>
+
+#include "common.cuh"
+#include "epilogue.cuh"
+#include "kernels.h"
+#include "ptx_sm100.cuh"
+
+namespace photon {
+
+namespace {
+
+constexpr int kBM = 128;           // MMA M (TMEM lanes)
+constexpr int kBK = 64;            // K slice per stage: 64 bf16 = 128 bytes per row
+constexpr int kATileBytes = kBM * kBK * 2;
+
+template <int BN, int STAGES>
+struct TcCfg {
+  static constexpr int kBTileBytes = BN * kBK * 2;
+  static constexpr int kStageBytes = kATileBytes + kBTileBytes;
+  static constexpr int kRingBytes = STAGES * kStageBytes;
+  static constexpr int kStagingBytes = 128 * (BN + 1) * 4 > BN * (128 + 1) * 4
+                                           ? 128 * (BN + 1) * 4
+                                           : BN * (128 + 1) * 4;
+  static_assert(kStagingBytes <= kRingBytes, "epilogue staging must fit in the ring");
+  static constexpr int kSmemBytes = kRingBytes + 256 + 1024;  // + barriers + alignment slack
+  static constexpr uint32_t kTmemCols = BN < 32 ? 32 : BN;
+};
+
+template <int BN, int STAGES, bool SWAP>
+__global__ void __launch_bounds__(128, 1)
+    k_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+              int M, int N, int nkb, int kb_per_split, Epilogue ep, float* __restrict__ part,
+              int* err) {
+  using Cfg = TcCfg<BN, STAGES>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Cfg::kRingBytes);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * STAGES + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int a0 = blockIdx.x * kBM;  // rows of Amma
+  const int b0 = blockIdx.y * BN;   // rows of Bmma
+  const int z = blockIdx.z;
+  const int kb0 = z * kb_per_split;
+  const int kb1 = min(nkb, kb0 + kb_per_split);
+  const int nk = kb1 - kb0;
+
+  auto full_bar = [&](int s) { return ptx::smem_u32(bars + s); };
+  auto empty_bar = [&](int s) { return ptx::smem_u32(bars + STAGES + s); };
+  const uint32_t done_bar = ptx::smem_u32(bars + 2 * STAGES);
+  auto a_tile = [&](int s) { return ptx::smem_u32(smem + s * Cfg::kStageBytes); };
+  auto b_tile = [&](int s) { return ptx::smem_u32(smem + s * Cfg::kStageBytes + kATileBytes); };
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      ptx::mbar_init(full_bar(s), 1);
+      ptx::mbar_init(empty_bar(s), 1);
+    }
+    ptx::mbar_init(done_bar, 1);
+    *abort_flag = 0;
+    ptx::fence_barrier_init();
+    ptx::prefetch_tmap(&tmA);
+    ptx::prefetch_tmap(&tmB);
+  }
+  __syncwarp();
+  if (warp == 0) {
+    ptx::tmem_alloc(ptx::smem_u32(tmem_slot), Cfg::kTmemCols);
+    ptx::tmem_relinquish();
+  }
+  ptx::tc_fence_before();
+  __syncthreads();
+  ptx::tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (threadIdx.x == 0) {
+    // ---- TMA producer
+    for (int it = 0; it < nk; ++it) {
+      const int s = it % STAGES;
+      const uint32_t ph = (uint32_t)(it / STAGES) & 1u;
+      if (!ptx::mbar_wait(empty_bar(s), ph ^ 1u, abort_flag)) {
+        report_error(err, DEV_WAIT_TIMEOUT_PRODUCER);
+        *abort_flag = 1;
+        break;
+      }
+      ptx::mbar_arrive_expect_tx(full_bar(s), (uint32_t)Cfg::kStageBytes);
+      ptx::tma_load_2d(a_tile(s), &tmA, (kb0 + it) * kBK, a0, full_bar(s));
+      ptx::tma_load_2d(b_tile(s), &tmB, (kb0 + it) * kBK, b0, full_bar(s));
+    }
+  } else if (threadIdx.x == 32) {
+    // ---- MMA issuer
+    constexpr uint32_t idesc = ptx::idesc_bf16_f32(kBM, BN);
+    for (int it = 0; it < nk; ++it) {
+      const int s = it % STAGES;
+      const uint32_t ph = (uint32_t)(it / STAGES) & 1u;
+      if (!ptx::mbar_wait(full_bar(s), ph, abort_flag)) {
+        report_error(err, DEV_WAIT_TIMEOUT_MMA);
+        *abort_flag = 1;
+        break;
+      }
+      ptx::tc_fence_after();
+      const uint64_t ad = ptx::sdesc_kmajor_sw128(a_tile(s));
+      const uint64_t bd = ptx::sdesc_kmajor_sw128(b_tile(s));
+#pragma unroll
+      for (int k = 0; k < kBK / 16; ++k)  // +32 bytes along K = +2 in the address field
+        ptx::mma_bf16(tmem, ad + 2 * k, bd + 2 * k, idesc, (it > 0 || k > 0) ? 1u : 0u);
+      ptx::mma_commit(empty_bar(s));
+    }
+    ptx::mma_commit(done_bar);  // completes once every issued MMA has finished
+  }
+  __syncwarp();
+
+  // ---- epilogue: TMEM -> shared staging tile (output-row-major)
+  if (!ptx::mbar_wait(done_bar, 0, abort_flag)) {
+    report_error(err, DEV_WAIT_TIMEOUT_EPILOGUE);
+    *abort_flag = 1;
+  }
+  __syncthreads();
+  const bool ok = (*abort_flag == 0);  // CTA-uniform: the TMEM loads below need whole warps
+  ptx::tc_fence_after();
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+  float* tile = reinterpret_cast<float*>(smem);
+  constexpr int R = SWAP ? BN : kBM;     // output rows in the tile (tokens)
+  constexpr int CC = SWAP ? kBM : BN;    // output columns in the tile (features)
+  constexpr int LD = CC + 1;
+  if (ok) {
+    const int tl = warp * 32 + lane;     // this thread's TMEM lane
+#pragma unroll 1
+    for (int j0 = 0; j0 < BN; j0 += 32) {
+      float v[32];
+      ptx::tmem_ld32(tmem + ((uint32_t)(warp * 32) << 16) + (uint32_t)j0, v);
+#pragma unroll
+      for (int i = 0; i < 32; ++i) {
+        if (SWAP)
+          tile[(j0 + i) * LD + tl] = v[i];
+        else
+          tile[tl * LD + j0 + i] = v[i];
+      }
+    }
+  }
+  ptx::tc_fence_before();
+  __syncthreads();
+  if (warp == 0) ptx::tmem_dealloc(tmem, Cfg::kTmemCols);
+  if (!ok || nk <= 0) return;
+
+  const int row_base = SWAP ? b0 : a0;
+  const int col_base = SWAP ? a0 : b0;
+  const long long plane = (long long)M * N;
+#pragma unroll 1
+  for (int r = warp; r < R; r += 4) {
+    const long long grow = row_base + r;
+    if (grow >= M) break;
+#pragma unroll 1
+    for (int seg = 0; seg < CC / 64; ++seg) {
+      if (col_base + seg * 64 >= N) break;  // N is a multiple of 64
+      const int c0 = seg * 64 + lane;
+      const int gc0 = col_base + c0;
+      const float v0 = tile[r * LD + c0];
+      const float v1 = tile[r * LD + c0 + 32];
+      if (part) {
+        float* p = part + (long long)z * plane + grow * N + gc0;
+        p[0] = v0;
+        p[32] = v1;
+      } else {
+        epi_pair<bf16>(ep, grow, gc0, v0, gc0 + 32, v1);
+      }
+    }
+  }
+}
+
+// ------------------------------------------------------------------ host side
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// 2-D bf16 map over a row-major [rows, K] matrix with leading dimension ld
+// (elements); box = 64 (K) x box_rows, 128-byte swizzle, zero fill.
+bool make_map(CUtensorMap* m, const void* ptr, long long rows, int K, long long ld, int box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)ld * 2};
+  cuuint32_t box[2] = {(cuuint32_t)kBK, (cuuint32_t)box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides, box,
+            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int BN, int STAGES, bool SWAP>
+void run_tc(const CUtensorMap& ma, const CUtensorMap& mb, int grid_a, int grid_b, int splits,
+            int M, int N, int nkb, int kbs, const Epilogue& ep, float* part, int* err,
+            cudaStream_t s) {
+  using Cfg = TcCfg<BN, STAGES>;
+  static bool configured = false;
+  if (!configured) {
+    cudaFuncSetAttribute(k_gemm_tc<BN, STAGES, SWAP>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         Cfg::kSmemBytes);
+    configured = true;
+  }
+  dim3 grid(grid_a, grid_b, splits);
+  k_gemm_tc<BN, STAGES, SWAP><<<grid, 128, Cfg::kSmemBytes, s>>>(ma, mb, M, N, nkb, kbs, ep, part,
+                                                                 err);
+}
+
+struct Plan {
+  bool swap;
+  int bn;
+  int splits;
+  int kbs;
+};
+
+Plan plan_for(int M, int N, int K, int force_splits, int force_swap) {
+  Plan p;
+  const int nkb = K / kBK;
+  p.swap = force_swap >= 0 ? (force_swap != 0) : (M <= 256);
+  if (p.swap)
+    p.bn = M <= 64 ? 64 : (M <= 128 ? 128 : 256);
+  else
+    p.bn = (N % 256 == 0 && M >= 4096) ? 256 : 128;
+  const int ga = p.swap ? (N + kBM - 1) / kBM : (M + kBM - 1) / kBM;
+  const int gb = p.swap ? 1 : (N + p.bn - 1) / p.bn;
+  const int tiles = ga * gb;
+  int splits = 1;
+  if (force_splits > 0)
+    splits = force_splits;
+  else if (tiles < 148)
+    splits = (148 + tiles - 1) / tiles;
+  if (splits > nkb) splits = nkb;
+  if (splits < 1) splits = 1;
+  p.kbs = (nkb + splits - 1) / splits;
+  p.splits = (nkb + p.kbs - 1) / p.kbs;  // no empty split
+  return p;
+}
+
+}  // namespace
+
+bool tma_available() { return encode_fn() != nullptr; }
+
+size_t gemm_tc_workspace_bytes(int M, int N, int K) {
+  const Plan p = plan_for(M, N, K, 0, -1);
+  return p.splits > 1 ? (size_t)p.splits * M * N * sizeof(float) : 0;
+}
+
+bool launch_gemm_tc(const GemmArgs& a, const GemmWorkspace& ws, int* err, cudaStream_t s,
+                    int force_splits, int force_swap) {
+  const int M = a.M, N = a.N, K = a.K;
+  if (M <= 0 || N <= 0 || K <= 0) return false;
+  if (K % kBK || N % 64) return false;
+  if (a.ep.kind == EPI_QKV && a.ep.dh != 64) return false;
+  if ((a.lda * 2) % 16 || (a.ldw * 2) % 16) return false;
+  if (reinterpret_cast<uintptr_t>(a.A) % 16 || reinterpret_cast<uintptr_t>(a.W) % 16) return false;
+  const Plan p = plan_for(M, N, K, force_splits, force_swap);
+  float* part = nullptr;
+  if (p.splits > 1) {
+    const size_t need = (size_t)p.splits * M * N * sizeof(float);
+    if (!ws.part || ws.bytes < need) return false;
+    part = ws.part;
+  }
+  CUtensorMap ma, mb;
+  const int nkb = K / kBK;
+  if (p.swap) {
+    if (!make_map(&ma, a.W, N, K, a.ldw, kBM) || !make_map(&mb, a.A, M, K, a.lda, p.bn)) return false;
+    const int ga = (N + kBM - 1) / kBM;
+    if (p.bn == 64)
+      run_tc<64, 6, true>(ma, mb, ga, 1, p.splits, M, N, nkb, p.kbs, a.ep, part, err, s);
+    else if (p.bn == 128)
+      run_tc<128, 4, true>(ma, mb, ga, 1, p.splits, M, N, nkb, p.kbs, a.ep, part, err, s);
+    else
+      run_tc<256, 4, true>(ma, mb, ga, 1, p.splits, M, N, nkb, p.kbs, a.ep, part, err, s);
+  } else {
+    if (!make_map(&ma, a.A, M, K, a.lda, kBM) || !make_map(&mb, a.W, N, K, a.ldw, p.bn)) return false;
+    const int ga = (M + kBM - 1) / kBM, gb = (N + p.bn - 1) / p.bn;
+    if (p.bn == 256)
+      run_tc<256, 4, false>(ma, mb, ga, gb, p.splits, M, N, nkb, p.kbs, a.ep, part, err, s);
+    else
+      run_tc<128, 4, false>(ma, mb, ga, gb, p.splits, M, N, nkb, p.kbs, a.ep, part, err, s);
+  }
+  if (p.splits > 1) launch_splitk_reduce(DT_BF16, part, p.splits, M, N, a.ep, s);
+  return true;
+}
+
+}  // namespace photon

@@ -1,0 +1,268 @@
+// Weight generation, embeddings, RMSNorm, greedy argmax and the split-K
+// reduction.  All memory-bound row kernels.
+#include "common.cuh"
+#include "epilogue.cuh"
+#include "kernels.h"
+
+namespace photon {
+
+// ------------------------------------------------------------------ weights
+// Counter-based draw, defined independently of any other implementation:
+// z = SplitMix64 output for counter (e + 1) of the tensor's stream; S = sum
+// of the four 16-bit fields of z; w = fp64(S - 131070) * K (an Irwin-Hall(4)
+// sum of uniforms, centred; K = init_std * sqrt(3) / 65536 so std = init_std),
+// rounded to fp32 (nearest even) and then to the storage type.
+__device__ __forceinline__ uint64_t splitmix_mix(uint64_t z) {
+  z ^= z >> 30;
+  z *= 0xBF58476D1CE4E5B9ull;
+  z ^= z >> 27;
+  z *= 0x94D049BB133111EBull;
+  z ^= z >> 31;
+  return z;
+}
+static uint64_t splitmix_mix_host(uint64_t z) {
+  z ^= z >> 30;
+  z *= 0xBF58476D1CE4E5B9ull;
+  z ^= z >> 27;
+  z *= 0x94D049BB133111EBull;
+  z ^= z >> 31;
+  return z;
+}
+constexpr uint64_t kGamma = 0x9E3779B97F4A7C15ull;
+
+template <typename T>
+__global__ void k_init_normal(T* __restrict__ dst, long long n, uint64_t base, double K) {
+  for (long long e = blockIdx.x * (long long)blockDim.x + threadIdx.x; e < n;
+       e += (long long)gridDim.x * blockDim.x) {
+    const uint64_t z = splitmix_mix(base + kGamma * (uint64_t)(e + 1));
+    const int S = (int)(z & 0xFFFFu) + (int)((z >> 16) & 0xFFFFu) + (int)((z >> 32) & 0xFFFFu) +
+                  (int)(z >> 48);
+    const double w = (double)(S - 131070) * K;
+    st_f(dst + e, __double2float_rn(w));
+  }
+}
+
+void launch_init_normal(int dt, void* dst, long long numel, uint64_t seed, int tensor_index,
+                        double K, cudaStream_t s) {
+  const uint64_t base = splitmix_mix_host(seed + kGamma * (uint64_t)(tensor_index + 1));
+  const int threads = 256;
+  long long blocks = (numel + threads - 1) / threads;
+  if (blocks > 148 * 64) blocks = 148 * 64;
+  if (blocks < 1) blocks = 1;
+  if (dt == DT_F32)
+    k_init_normal<float><<<(int)blocks, threads, 0, s>>>((float*)dst, numel, base, K);
+  else
+    k_init_normal<bf16><<<(int)blocks, threads, 0, s>>>((bf16*)dst, numel, base, K);
+}
+
+__global__ void k_fill_f32(float* dst, long long n, float v) {
+  for (long long e = blockIdx.x * (long long)blockDim.x + threadIdx.x; e < n;
+       e += (long long)gridDim.x * blockDim.x)
+    dst[e] = v;
+}
+void launch_fill_f32(float* dst, long long n, float v, cudaStream_t s) {
+  long long blocks = (n + 255) / 256;
+  if (blocks > 148 * 16) blocks = 148 * 16;
+  if (blocks < 1) blocks = 1;
+  k_fill_f32<<<(int)blocks, 256, 0, s>>>(dst, n, v);
+}
+
+template <typename T>
+__global__ void k_to_f32(const T* src, float* dst, long long n) {
+  for (long long e = blockIdx.x * (long long)blockDim.x + threadIdx.x; e < n;
+       e += (long long)gridDim.x * blockDim.x)
+    dst[e] = ld_f(src + e);
+}
+void launch_to_f32(int dt, const void* src, float* dst, long long n, cudaStream_t s) {
+  long long blocks = (n + 255) / 256;
+  if (blocks > 148 * 16) blocks = 148 * 16;
+  if (blocks < 1) blocks = 1;
+  if (dt == DT_F32)
+    k_to_f32<float><<<(int)blocks, 256, 0, s>>>((const float*)src, dst, n);
+  else
+    k_to_f32<bf16><<<(int)blocks, 256, 0, s>>>((const bf16*)src, dst, n);
+}
+
+// ------------------------------------------------------------------ embedding
+// One warp per row; 16-byte vector copies (d * sizeof(T) is a multiple of 16).
+template <typename T>
+__global__ void k_embed(const int32_t* __restrict__ ids, const T* __restrict__ E, T* __restrict__ out,
+                        int rows, int d, int vocab, int* err) {
+  const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  if (warp >= rows) return;
+  int id = ids[warp];
+  if (id < 0 || id >= vocab) {
+    if (lane == 0) report_error(err, DEV_BAD_TOKEN);
+    id = 0;
+  }
+  const uint4* src = reinterpret_cast<const uint4*>(E + (long long)id * d);
+  uint4* dst = reinterpret_cast<uint4*>(out + (long long)warp * d);
+  const int nv = d * (int)sizeof(T) / 16;
+  for (int v = lane; v < nv; v += 32) dst[v] = __ldg(src + v);
+}
+void launch_embed(int dt, const int32_t* ids, const void* E, void* out, int rows, int d, int vocab,
+                  int* err, cudaStream_t s) {
+  if (rows <= 0) return;
+  const int threads = 256;
+  const int blocks = (rows * 32 + threads - 1) / threads;
+  if (dt == DT_F32)
+    k_embed<float><<<blocks, threads, 0, s>>>(ids, (const float*)E, (float*)out, rows, d, vocab, err);
+  else
+    k_embed<bf16><<<blocks, threads, 0, s>>>(ids, (const bf16*)E, (bf16*)out, rows, d, vocab, err);
+}
+
+template <typename T>
+__global__ void k_embed_f32(const int32_t* __restrict__ ids, const T* __restrict__ E,
+                            float* __restrict__ x, int rows, int d, int vocab, int* err) {
+  const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  if (warp >= rows) return;
+  int id = ids[warp];
+  if (id < 0 || id >= vocab) {
+    if (lane == 0) report_error(err, DEV_BAD_TOKEN);
+    id = 0;
+  }
+  const T* src = E + (long long)id * d;
+  float* dst = x + (long long)warp * d;
+  for (int c = lane; c < d; c += 32) dst[c] = ld_f(src + c);
+}
+void launch_embed_f32(int dt, const int32_t* ids, const void* E, float* x, int rows, int d,
+                      int vocab, int* err, cudaStream_t s) {
+  if (rows <= 0) return;
+  const int threads = 256;
+  const int blocks = (rows * 32 + threads - 1) / threads;
+  if (dt == DT_F32)
+    k_embed_f32<float><<<blocks, threads, 0, s>>>(ids, (const float*)E, x, rows, d, vocab, err);
+  else
+    k_embed_f32<bf16><<<blocks, threads, 0, s>>>(ids, (const bf16*)E, x, rows, d, vocab, err);
+}
+
+// ------------------------------------------------------------------ RMSNorm
+// One warp per output row: out = x / sqrt(mean(x^2) + eps) * g.
+template <typename T>
+__global__ void k_rmsnorm(const float* __restrict__ x, const float* __restrict__ g,
+                          T* __restrict__ out, int rows, int d, int in_step, int in_off, float eps) {
+  const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  if (warp >= rows) return;
+  const float* xr = x + ((long long)warp * in_step + in_off) * d;
+  float ss = 0.f;
+  for (int c = lane * 4; c < d; c += 128) {
+    const float4 v = *reinterpret_cast<const float4*>(xr + c);
+    ss += v.x * v.x + v.y * v.y + v.z * v.z + v.w * v.w;
+  }
+  ss = warp_sum(ss);
+  const float r = 1.0f / sqrtf(ss / (float)d + eps);
+  T* o = out + (long long)warp * d;
+  for (int c = lane * 4; c < d; c += 128) {
+    const float4 v = *reinterpret_cast<const float4*>(xr + c);
+    const float4 gg = *reinterpret_cast<const float4*>(g + c);
+    st_f(o + c + 0, v.x * r * gg.x);
+    st_f(o + c + 1, v.y * r * gg.y);
+    st_f(o + c + 2, v.z * r * gg.z);
+    st_f(o + c + 3, v.w * r * gg.w);
+  }
+}
+void launch_rmsnorm(int dt, const float* x, const float* g, void* out, int rows, int d, int in_step,
+                    int in_off, float eps, cudaStream_t s) {
+  if (rows <= 0) return;
+  const int threads = 256;
+  const int blocks = (rows * 32 + threads - 1) / threads;
+  if (dt == DT_F32)
+    k_rmsnorm<float><<<blocks, threads, 0, s>>>(x, g, (float*)out, rows, d, in_step, in_off, eps);
+  else
+    k_rmsnorm<bf16><<<blocks, threads, 0, s>>>(x, g, (bf16*)out, rows, d, in_step, in_off, eps);
+}
+
+// ------------------------------------------------------------------ argmax
+__device__ __forceinline__ void better(float& bv, int& bi, float v, int i) {
+  if (v > bv || (v == bv && i < bi)) {
+    bv = v;
+    bi = i;
+  }
+}
+__global__ void k_argmax(const float* __restrict__ logits, long long ld, int rows, int V, int step,
+                         int C1, const int32_t* __restrict__ force, int32_t* own, int32_t* used,
+                         int32_t* next_ids, int* err) {
+  const int row = blockIdx.x;
+  if (row >= rows) return;
+  const float* lr = logits + (long long)row * ld;
+  float bv = -INFINITY;
+  int bi = 0x7fffffff;
+  for (int c = threadIdx.x; c < V; c += blockDim.x) better(bv, bi, lr[c], c);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+    const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
+    better(bv, bi, ov, oi);
+  }
+  __shared__ float sv[32];
+  __shared__ int si[32];
+  const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (lane == 0) {
+    sv[w] = bv;
+    si[w] = bi;
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    for (int k = 1; k < (int)(blockDim.x >> 5); ++k) better(bv, bi, sv[k], si[k]);
+    if (bi < 0 || bi >= V) {  // only if every logit is NaN
+      report_error(err, DEV_BAD_TOKEN);
+      bi = 0;
+    }
+    const long long slot = (long long)row * C1 + step;
+    int u = bi;
+    if (force) {
+      const int f = force[slot];
+      if (f >= 0) u = (f < V) ? f : 0;
+      if (f >= V) report_error(err, DEV_BAD_TOKEN);
+    }
+    if (own) own[slot] = bi;
+    if (used) used[slot] = u;
+    if (next_ids) next_ids[row] = u;
+  }
+}
+void launch_argmax(const float* logits, long long ld, int rows, int V, int i, int C1,
+                   const int32_t* force, int32_t* own, int32_t* used, int32_t* next_ids, int* err,
+                   cudaStream_t s) {
+  if (rows <= 0) return;
+  k_argmax<<<rows, 256, 0, s>>>(logits, ld, rows, V, i, C1, force, own, used, next_ids, err);
+}
+
+// ------------------------------------------------------------------ split-K reduce
+// Sums split partials in a fixed order (deterministic) and applies the
+// epilogue.  part is [splits][M][N] fp32; one thread per RoPE-compatible
+// column pair (c, c + 32) of a 64-column segment.
+template <typename T>
+__global__ void k_splitk_reduce(const float* __restrict__ part, int splits, int M, int N,
+                                Epilogue ep) {
+  const long long t = blockIdx.x * (long long)blockDim.x + threadIdx.x;
+  const int segs = N >> 6;
+  const long long total = (long long)M * segs * 32;
+  if (t >= total) return;
+  const int l = (int)(t & 31);
+  const long long rs = t >> 5;
+  const int seg = (int)(rs % segs);
+  const long long row = rs / segs;
+  const int c0 = seg * 64 + l, c1 = c0 + 32;
+  float v0 = 0.f, v1 = 0.f;
+  const long long plane = (long long)M * N;
+  for (int s = 0; s < splits; ++s) {
+    v0 += part[s * plane + row * N + c0];
+    v1 += part[s * plane + row * N + c1];
+  }
+  epi_pair<T>(ep, row, c0, v0, c1, v1);
+}
+void launch_splitk_reduce(int dt, const float* part, int splits, int M, int N, const Epilogue& ep,
+                          cudaStream_t s) {
+  const long long total = (long long)M * (N >> 6) * 32;
+  const int threads = 256;
+  const long long blocks = (total + threads - 1) / threads;
+  if (dt == DT_F32)
+    k_splitk_reduce<float><<<(int)blocks, threads, 0, s>>>(part, splits, M, N, ep);
+  else
+    k_splitk_reduce<bf16><<<(int)blocks, threads, 0, s>>>(part, splits, M, N, ep);
+}
+
+}  // namespace photon

@@ -1,0 +1,123 @@
+// Internal launch API of the PHOTON kernels (host side).  Not part of the
+// public C ABI; the runtime in runtime.cu is the only caller.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace photon {
+
+enum DType : int { DT_F32 = 0, DT_BF16 = 1 };
+inline size_t dtype_size(int dt) { return dt == DT_F32 ? 4 : 2; }
+
+// What a GEMM does with each accumulator value acc(row, col).
+enum EpiKind : int {
+  EPI_STORE_T = 0,    // out[row, col] = T(acc)
+  EPI_STORE_F32 = 1,  // out[row, col] = acc (fp32)
+  EPI_ADD_F32 = 2,    // out[row, col] += acc (fp32 residual stream)
+  EPI_GELU_T = 3,     // out[row, col] = T(gelu(acc))
+  EPI_QKV = 4,        // fused q/k/v split + RoPE + KV-cache write (see below)
+};
+
+// Epilogue parameters.  For EPI_QKV the GEMM output has 3*d columns
+// (q | k | v).  Row r belongs to group g = r / q_len (a sequence, or a
+// decoder sub-chunk) and sits at stream position pos = p0 + r % q_len.
+// q and k are rotated (rotate-half RoPE with the table `rope`, float2
+// (cos, sin) per [pos][i], i < dh/2); q goes to q_out[r, :d]; k and v go to
+// the caches laid out [G][H][cap][dh] at slot pos - kv_off.
+struct Epilogue {
+  int kind = EPI_STORE_T;
+  void* out = nullptr;
+  long long ldo = 0;
+  void* q_out = nullptr;
+  void* k_cache = nullptr;
+  void* v_cache = nullptr;
+  int d = 0, H = 0, dh = 0, cap = 0, q_len = 1, p0 = 0, kv_off = 0;
+  const float2* rope = nullptr;
+};
+
+// C = A[M, K] * W[N, K]^T with A, W of the storage type, fp32 accumulation.
+struct GemmArgs {
+  const void* A = nullptr;
+  long long lda = 0;
+  const void* W = nullptr;
+  long long ldw = 0;
+  int M = 0, N = 0, K = 0;
+  Epilogue ep;
+};
+
+// Scratch the GEMM may use for split-K partial tiles (fp32).
+struct GemmWorkspace {
+  float* part = nullptr;
+  size_t bytes = 0;
+};
+
+// Attention of q_len new queries per group over a key/value cache.
+// Query i of group g sits at absolute position p0 + i and sees keys at
+// positions 0..p0+i.  Keys at positions < n_pre come from a shared prefix
+// cache Kp/Vp ([H][cap_pre][dh], the same for every group); keys at
+// positions >= n_pre come from the group's own cache K/V ([G][H][cap][dh])
+// at slot pos - n_pre.  Q rows are [G*q_len, q_ld] (head h at column h*dh),
+// outputs O the same layout.
+struct AttnArgs {
+  const void* Q = nullptr;
+  long long q_ld = 0;
+  const void* K = nullptr;
+  const void* V = nullptr;
+  int cap = 0;
+  const void* Kp = nullptr;
+  const void* Vp = nullptr;
+  int cap_pre = 0, n_pre = 0;
+  int G = 0, H = 0, dh = 0, q_len = 1, p0 = 0;
+  void* O = nullptr;
+  long long o_ld = 0;
+  float scale = 1.0f;
+};
+
+// ---- weights -----------------------------------------------------------
+void launch_init_normal(int dt, void* dst, long long numel, uint64_t seed, int tensor_index,
+                        double K, cudaStream_t s);
+void launch_fill_f32(float* dst, long long n, float v, cudaStream_t s);
+void launch_to_f32(int dt, const void* src, float* dst, long long n, cudaStream_t s);
+
+// ---- elementwise / rows -------------------------------------------------
+// out[r, :] = E[ids[r], :] (storage type).  Invalid ids set *err.
+void launch_embed(int dt, const int32_t* ids, const void* E, void* out, int rows, int d, int vocab,
+                  int* err, cudaStream_t s);
+// x[r, :] = fp32(E[ids[r], :]).
+void launch_embed_f32(int dt, const int32_t* ids, const void* E, float* x, int rows, int d,
+                      int vocab, int* err, cudaStream_t s);
+// out[r, :] = T(rmsnorm(x[r*in_step + in_off, :]) * g).
+void launch_rmsnorm(int dt, const float* x, const float* g, void* out, int rows, int d,
+                    int in_step, int in_off, float eps, cudaStream_t s);
+// Greedy token for row g of logits (lowest index among maxima).  Writes the
+// own choice to own[g*C1 + i]; the token fed back (force[g*C1+i] if >= 0,
+// else the own choice) to used[g*C1 + i] and next_ids[g].
+void launch_argmax(const float* logits, long long ld, int rows, int V, int i, int C1,
+                   const int32_t* force, int32_t* own, int32_t* used, int32_t* next_ids, int* err,
+                   cudaStream_t s);
+
+// ---- GEMM ----------------------------------------------------------------
+void launch_gemm(int dt, const GemmArgs& a, const GemmWorkspace& ws, int* err, cudaStream_t s);
+void launch_gemm_simt(int dt, const GemmArgs& a, cudaStream_t s);
+// tcgen05 path (bf16): returns false if the shape is not supported.
+bool launch_gemm_tc(const GemmArgs& a, const GemmWorkspace& ws, int* err, cudaStream_t s,
+                    int force_splits = 0, int force_swap = -1);
+size_t gemm_tc_workspace_bytes(int M, int N, int K);
+void launch_splitk_reduce(int dt, const float* part, int splits, int M, int N, const Epilogue& ep,
+                          cudaStream_t s);
+
+// ---- attention ------------------------------------------------------------
+// Split-K decode attention (q_len <= 8).  `part` is fp32 scratch for the
+// split partials; attn_decode_workspace_bytes gives its size.
+size_t attn_decode_workspace_bytes(const AttnArgs& a);
+// Returns false (nothing launched) for unsupported shapes or too little scratch.
+bool launch_attn_decode(int dt, const AttnArgs& a, float* part, size_t part_bytes, int* err,
+                        cudaStream_t s);
+// Causal attention for many new queries per group (prefill).
+void launch_attn_prefill(int dt, const AttnArgs& a, cudaStream_t s);
+
+// ---- TMA descriptors -----------------------------------------------------
+bool tma_available();
+
+}  // namespace photon

@@ -1,0 +1,1035 @@
+// Host runtime of the PHOTON library: model weights and their residency,
+// KV caches and workspaces, and the launch sequences of prefill, HierGen and
+// RecGen.  Implements the C ABI declared in include/photon.h.
+//
+// Procedure sources (PHOTON pages): module table of the explainer's
+// architecture section (Chunker, Encoder, Converter, Decoder), the RecGen
+// section (HierGen's three stages, RecGen's direct A-hat feed, top-only cache
+// retention, decoder-only weight residency) and the 475x section (decoder
+// attention confined to the chunk).
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <string>
+#include <vector>
+
+#include "kernels.h"
+#include "photon.h"
+
+using namespace photon;
+
+// ============================================================== errors
+static thread_local std::string g_err;
+
+static int fail(int code, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  g_err = buf;
+  return code;
+}
+
+#define CK(call)                                                                   \
+  do {                                                                             \
+    cudaError_t e_ = (call);                                                       \
+    if (e_ != cudaSuccess) {                                                       \
+      if (e_ == cudaErrorMemoryAllocation) {                                       \
+        cudaGetLastError();                                                        \
+        return fail(PHOTON_ERR_OOM, "%s: out of device memory", #call);            \
+      }                                                                            \
+      return fail(PHOTON_ERR_CUDA, "%s: %s", #call, cudaGetErrorString(e_));       \
+    }                                                                              \
+  } while (0)
+
+#define RET(x)                     \
+  do {                             \
+    int r_ = (x);                  \
+    if (r_ != PHOTON_OK) return r_; \
+  } while (0)
+
+// ============================================================== model
+enum Group { G_EMB = 0, G_ENC1 = 1, G_TOP = 2, G_DEC = 3, G_COUNT = 4 };
+
+struct TensorRec {
+  std::string name;
+  int group;
+  size_t offset;  // bytes inside the group buffer
+  long long numel;
+  bool gain;      // RMSNorm gain: fp32, value 1
+};
+
+struct BlockW {
+  const float* g_attn;
+  const void* wqkv;  // [3d, d]: wq, wk, wv stored back to back
+  const void* wo;
+  const float* g_mlp;
+  const void* w1;
+  const void* w2;
+};
+
+struct photon_model {
+  photon_config cfg;
+  int dt;
+  size_t es;
+  uint64_t seed;
+  int d, H, dh, V, C1, C2, C, f, L1, Ltop, Ld1, Ld2;
+  std::vector<TensorRec> t;
+  size_t group_bytes[G_COUNT] = {0, 0, 0, 0};
+  char* group_ptr[G_COUNT] = {nullptr, nullptr, nullptr, nullptr};
+  // first tensor index of each piece
+  int i_embed, i_ch1, i_enc1, i_enc1_g, i_ch2, i_top, i_top_g, i_cv2, i_dec2, i_dec2_g, i_cv1,
+      i_dec1, i_dec1_g, i_head;
+  int live_caches = 0;
+  int hier_caches = 0;
+  bool use_tc = false;
+
+  const void* ptr(int idx) const { return group_ptr[t[idx].group] + t[idx].offset; }
+  BlockW block(int first, int l) const {
+    const int b = first + 8 * l;
+    return BlockW{(const float*)ptr(b), ptr(b + 1), ptr(b + 4), (const float*)ptr(b + 5),
+                  ptr(b + 6), ptr(b + 7)};
+  }
+};
+
+static int check_config(const photon_config* c) {
+  if (!c) return fail(PHOTON_ERR_ARG, "config is NULL");
+  if (c->levels != 2) return fail(PHOTON_ERR_ARG, "only L = 2 levels are supported");
+  if (c->vocab <= 0 || c->d_model <= 0 || c->n_heads <= 0 || c->head_dim <= 0)
+    return fail(PHOTON_ERR_ARG, "non-positive model dimension");
+  if (c->d_model != c->n_heads * c->head_dim)
+    return fail(PHOTON_ERR_ARG, "d_model must equal n_heads * head_dim");
+  if (c->head_dim != 32 && c->head_dim != 64) return fail(PHOTON_ERR_ARG, "head_dim must be 32 or 64");
+  if (c->d_model % 64) return fail(PHOTON_ERR_ARG, "d_model must be a multiple of 64");
+  for (int l = 0; l < 2; ++l) {
+    if (c->chunk[l] < 1 || c->chunk[l] > 4) return fail(PHOTON_ERR_ARG, "chunk sizes must be 1..4");
+    if (c->enc_layers[l] < 1 || c->dec_layers[l] < 1) return fail(PHOTON_ERR_ARG, "layer counts must be >= 1");
+  }
+  if (c->conv_kernel != 0 && (c->conv_kernel != c->chunk[0] || c->conv_kernel != c->chunk[1]))
+    return fail(PHOTON_ERR_ARG, "conv_kernel must equal C1 and C2 (kernel = stride = C)");
+  if (c->mlp_mult < 1) return fail(PHOTON_ERR_ARG, "mlp_mult must be >= 1");
+  if (c->dtype != 0 && c->dtype != 1) return fail(PHOTON_ERR_ARG, "dtype must be 0 (fp32) or 1 (bf16)");
+  if (!(c->norm_eps > 0.f) || !(c->rope_theta > 0.f) || !(c->init_std > 0.f))
+    return fail(PHOTON_ERR_ARG, "eps, theta and init_std must be positive");
+  return PHOTON_OK;
+}
+
+static void build_specs(photon_model* m) {
+  const long long d = m->d, V = m->V, f = m->f;
+  auto add = [&](const std::string& n, int g, long long numel, bool gain) {
+    m->t.push_back(TensorRec{n, g, 0, numel, gain});
+  };
+  auto blocks = [&](const char* p, int n, int g) {
+    for (int l = 0; l < n; ++l) {
+      const std::string s = std::string(p) + "." + std::to_string(l) + ".";
+      add(s + "g_attn", g, d, true);
+      add(s + "wq", g, d * d, false);
+      add(s + "wk", g, d * d, false);
+      add(s + "wv", g, d * d, false);
+      add(s + "wo", g, d * d, false);
+      add(s + "g_mlp", g, d, true);
+      add(s + "w1", g, f * d, false);
+      add(s + "w2", g, d * f, false);
+    }
+  };
+  m->i_embed = (int)m->t.size();
+  add("embed", G_EMB, V * d, false);
+  m->i_ch1 = (int)m->t.size();
+  add("chunker1", G_ENC1, d * m->C1 * d, false);
+  m->i_enc1 = (int)m->t.size();
+  blocks("enc1", m->L1, G_ENC1);
+  m->i_enc1_g = (int)m->t.size();
+  add("enc1.g_final", G_ENC1, d, true);
+  m->i_ch2 = (int)m->t.size();
+  add("chunker2", G_TOP, d * m->C2 * d, false);
+  m->i_top = (int)m->t.size();
+  blocks("top", m->Ltop, G_TOP);
+  m->i_top_g = (int)m->t.size();
+  add("top.g_final", G_TOP, d, true);
+  m->i_cv2 = (int)m->t.size();
+  add("converter2", G_DEC, m->C2 * d * d, false);
+  m->i_dec2 = (int)m->t.size();
+  blocks("dec2", m->Ld2, G_DEC);
+  m->i_dec2_g = (int)m->t.size();
+  add("dec2.g_final", G_DEC, d, true);
+  m->i_cv1 = (int)m->t.size();
+  add("converter1", G_DEC, m->C1 * d * d, false);
+  m->i_dec1 = (int)m->t.size();
+  blocks("dec1", m->Ld1, G_DEC);
+  m->i_dec1_g = (int)m->t.size();
+  add("dec1.g_final", G_DEC, d, true);
+  m->i_head = (int)m->t.size();
+  add("head", G_DEC, V * d, false);
+  for (auto& r : m->t) {
+    const size_t bytes = (size_t)r.numel * (r.gain ? 4 : m->es);
+    r.offset = m->group_bytes[r.group];
+    m->group_bytes[r.group] += (bytes + 255) & ~size_t(255);
+  }
+}
+
+// Draws (or fills) every tensor of one group into its buffer.
+static void generate_group(photon_model* m, int g, cudaStream_t s) {
+  const double K = ((double)m->cfg.init_std * 1.7320508075688772) / 65536.0;
+  for (size_t i = 0; i < m->t.size(); ++i) {
+    const TensorRec& r = m->t[i];
+    if (r.group != g) continue;
+    void* p = m->group_ptr[g] + r.offset;
+    if (r.gain)
+      launch_fill_f32((float*)p, r.numel, 1.0f, s);
+    else
+      launch_init_normal(m->dt, p, r.numel, m->seed, (int)i, K, s);
+  }
+}
+
+// Level-1 encoder + chunker-1 weights are needed only by prefill and HierGen
+// (RecGen section: during RecGen decode the encoder hierarchy is never
+// called).  They are released after a RecGen prefill when no HierGen cache
+// is alive, and regenerated from the seed when needed again.
+static int ensure_encoder(photon_model* m, cudaStream_t s) {
+  if (m->group_ptr[G_ENC1]) return PHOTON_OK;
+  CK(cudaMallocAsync((void**)&m->group_ptr[G_ENC1], m->group_bytes[G_ENC1], s));
+  generate_group(m, G_ENC1, s);
+  CK(cudaGetLastError());
+  return PHOTON_OK;
+}
+static int release_encoder(photon_model* m, cudaStream_t s) {
+  if (!m->group_ptr[G_ENC1]) return PHOTON_OK;
+  CK(cudaFreeAsync(m->group_ptr[G_ENC1], s));
+  m->group_ptr[G_ENC1] = nullptr;
+  return PHOTON_OK;
+}
+
+// ============================================================== cache
+struct Bufs {
+  void* xn;
+  void* q;
+  void* att;
+  void* hid;
+  const float2* rope;
+  float* gemm_ws;
+  size_t gemm_ws_bytes;
+  float* attn_ws;
+  size_t attn_ws_bytes;
+  int* err;
+};
+
+struct photon_cache {
+  photon_model* m = nullptr;
+  const photon_cache* prefix = nullptr;
+  mutable int dependents = 0;
+  int B = 0, T = 0, mode = 0, max_new = 0;
+  int N = 0, N1 = 0, n_pre = 0, n1_pre = 0;
+  int Ncap = 0, N1cap = 0;
+  int steps = 0;
+  cudaStream_t stream = nullptr;
+  char *top_k = nullptr, *top_v = nullptr;
+  size_t top_layer = 0;
+  char *l1_k = nullptr, *l1_v = nullptr;
+  size_t l1_layer = 0;
+  void* o = nullptr;
+  float2* rope = nullptr;
+  // decode workspace
+  float *xd = nullptr, *xs = nullptr, *xt = nullptr, *x1 = nullptr, *logits = nullptr;
+  void *xn = nullptr, *q = nullptr, *att = nullptr, *hid = nullptr;
+  void *a_hat = nullptr, *a = nullptr, *embd = nullptr, *hn = nullptr;
+  char *d2k = nullptr, *d2v = nullptr, *d1k = nullptr, *d1v = nullptr;
+  size_t d2_layer = 0, d1_layer = 0;
+  int32_t *next_ids = nullptr, *used = nullptr;
+  float* gemm_ws = nullptr;
+  size_t gemm_ws_bytes = 0;
+  float* attn_ws = nullptr;
+  size_t attn_ws_bytes = 0;
+  int* d_err = nullptr;
+  std::vector<void*> allocs;
+  size_t kv_bytes = 0, ws_bytes = 0;
+  bool has_a_hat = false, has_a = false;
+};
+
+struct Allocator {
+  cudaStream_t s;
+  std::vector<void*>* list;
+  size_t* counter;
+  cudaError_t err = cudaSuccess;
+  template <typename P>
+  P* get(size_t bytes) {
+    if (bytes == 0 || err != cudaSuccess) return nullptr;
+    void* p = nullptr;
+    err = cudaMallocAsync(&p, (bytes + 255) & ~size_t(255), s);
+    if (err != cudaSuccess) return nullptr;
+    list->push_back(p);
+    if (counter) *counter += bytes;
+    return reinterpret_cast<P*>(p);
+  }
+};
+
+static void free_list(std::vector<void*>& l, cudaStream_t s) {
+  for (void* p : l) cudaFreeAsync(p, s);
+  l.clear();
+}
+
+// One stack invocation: group/position layout and the caches it writes/reads.
+struct StackRun {
+  int G = 0, q_len = 1, p0 = 0, kv_off = 0;
+  char* kc = nullptr;
+  char* vc = nullptr;
+  size_t layer_bytes = 0;
+  int cap = 0;
+  const char* kp = nullptr;
+  const char* vp = nullptr;
+  size_t pre_layer_bytes = 0;
+  int cap_pre = 0, n_pre = 0;
+};
+
+static void gemm(photon_model* m, const Bufs& b, const void* A, long long lda, const void* W,
+                 long long ldw, int M, int N, int K, const Epilogue& ep, cudaStream_t s) {
+  GemmArgs g;
+  g.A = A;
+  g.lda = lda;
+  g.W = W;
+  g.ldw = ldw;
+  g.M = M;
+  g.N = N;
+  g.K = K;
+  g.ep = ep;
+  GemmWorkspace ws{b.gemm_ws, b.gemm_ws_bytes};
+  if (m->use_tc)
+    launch_gemm(m->dt, g, ws, b.err, s);
+  else
+    launch_gemm_simt(m->dt, g, s);
+}
+
+static Epilogue epi(int kind, void* out, long long ldo) {
+  Epilogue e;
+  e.kind = kind;
+  e.out = out;
+  e.ldo = ldo;
+  return e;
+}
+
+// Pre-norm block (reading R8-R11): x += Attn(RMSNorm(x)); x += MLP(RMSNorm(x)).
+static void run_block(photon_model* m, const BlockW& w, float* x, const StackRun& r, int layer,
+                      const Bufs& b, cudaStream_t s) {
+  const int d = m->d, rows = r.G * r.q_len;
+  const float eps = m->cfg.norm_eps;
+  launch_rmsnorm(m->dt, x, w.g_attn, b.xn, rows, d, 1, 0, eps, s);
+  Epilogue e;
+  e.kind = EPI_QKV;
+  e.q_out = b.q;
+  e.k_cache = r.kc + layer * r.layer_bytes;
+  e.v_cache = r.vc + layer * r.layer_bytes;
+  e.d = d;
+  e.H = m->H;
+  e.dh = m->dh;
+  e.cap = r.cap;
+  e.q_len = r.q_len;
+  e.p0 = r.p0;
+  e.kv_off = r.kv_off;
+  e.rope = b.rope;
+  gemm(m, b, b.xn, d, w.wqkv, d, rows, 3 * d, d, e, s);
+
+  AttnArgs a;
+  a.Q = b.q;
+  a.q_ld = d;
+  a.K = e.k_cache;
+  a.V = e.v_cache;
+  a.cap = r.cap;
+  if (r.kp) {
+    a.Kp = r.kp + layer * r.pre_layer_bytes;
+    a.Vp = r.vp + layer * r.pre_layer_bytes;
+    a.cap_pre = r.cap_pre;
+    a.n_pre = r.n_pre;
+  }
+  a.G = r.G;
+  a.H = m->H;
+  a.dh = m->dh;
+  a.q_len = r.q_len;
+  a.p0 = r.p0;
+  a.O = b.att;
+  a.o_ld = d;
+  a.scale = 1.0f / sqrtf((float)m->dh);
+  bool done = false;
+  if (r.q_len <= 4) done = launch_attn_decode(m->dt, a, b.attn_ws, b.attn_ws_bytes, b.err, s);
+  if (!done) launch_attn_prefill(m->dt, a, s);
+
+  gemm(m, b, b.att, d, w.wo, d, rows, d, d, epi(EPI_ADD_F32, x, d), s);
+  launch_rmsnorm(m->dt, x, w.g_mlp, b.xn, rows, d, 1, 0, eps, s);
+  gemm(m, b, b.xn, d, w.w1, d, rows, m->f, d, epi(EPI_GELU_T, b.hid, m->f), s);
+  gemm(m, b, b.hid, m->f, w.w2, m->f, rows, d, m->f, epi(EPI_ADD_F32, x, d), s);
+}
+
+static void run_stack(photon_model* m, int first, int n_layers, float* x, const StackRun& r,
+                      const Bufs& b, cudaStream_t s) {
+  for (int l = 0; l < n_layers; ++l) run_block(m, m->block(first, l), x, r, l, b, s);
+}
+
+static size_t gemm_ws_need(const photon_model* m, int M, int N, int K) {
+  if (!m->use_tc) return 0;
+  return gemm_tc_workspace_bytes(M, N, K);
+}
+static size_t block_ws_need(const photon_model* m, int rows) {
+  size_t w = 0;
+  w = std::max(w, gemm_ws_need(m, rows, 3 * m->d, m->d));
+  w = std::max(w, gemm_ws_need(m, rows, m->d, m->d));
+  w = std::max(w, gemm_ws_need(m, rows, m->f, m->d));
+  w = std::max(w, gemm_ws_need(m, rows, m->d, m->f));
+  return w;
+}
+static size_t attn_ws_need(int G, int H, int dh, int q_len, int n_max) {
+  size_t w = 0;
+  AttnArgs a;
+  a.G = G;
+  a.H = H;
+  a.dh = dh;
+  a.q_len = q_len;
+  for (int n = q_len; n <= n_max; ++n) {
+    a.p0 = n - q_len;
+    w = std::max(w, attn_decode_workspace_bytes(a));
+  }
+  return w;
+}
+
+// cos/sin table: entry [pos][i] = (cos, sin)(pos * theta^(-2i/dh)), computed in fp64.
+static int upload_rope(photon_model* m, photon_cache* c, Allocator& al, int positions) {
+  const int half = m->dh / 2;
+  std::vector<float2> host((size_t)positions * half);
+  for (int p = 0; p < positions; ++p)
+    for (int i = 0; i < half; ++i) {
+      const double inv = std::pow((double)m->cfg.rope_theta, -2.0 * i / m->dh);
+      const double ang = (double)p * inv;
+      host[(size_t)p * half + i] = make_float2((float)std::cos(ang), (float)std::sin(ang));
+    }
+  c->rope = al.get<float2>(host.size() * sizeof(float2));
+  if (!c->rope) return PHOTON_ERR_OOM;
+  CK(cudaMemcpyAsync(c->rope, host.data(), host.size() * sizeof(float2), cudaMemcpyHostToDevice,
+                     al.s));
+  return PHOTON_OK;
+}
+
+static Bufs decode_bufs(photon_cache* c) {
+  Bufs b;
+  b.xn = c->xn;
+  b.q = c->q;
+  b.att = c->att;
+  b.hid = c->hid;
+  b.rope = c->rope;
+  b.gemm_ws = c->gemm_ws;
+  b.gemm_ws_bytes = c->gemm_ws_bytes;
+  b.attn_ws = c->attn_ws;
+  b.attn_ws_bytes = c->attn_ws_bytes;
+  b.err = c->d_err;
+  return b;
+}
+
+// ============================================================== C ABI
+extern "C" {
+
+const char* photon_last_error(void) { return g_err.c_str(); }
+
+int photon_init_weights(const photon_config* cfg, uint64_t seed, photon_model** out) {
+  g_err.clear();
+  if (!out) return fail(PHOTON_ERR_ARG, "out is NULL");
+  *out = nullptr;
+  RET(check_config(cfg));
+  int dev = 0;
+  CK(cudaGetDevice(&dev));
+  photon_model* m = new photon_model();
+  m->cfg = *cfg;
+  m->dt = cfg->dtype;
+  m->es = dtype_size(m->dt);
+  m->seed = seed;
+  m->d = cfg->d_model;
+  m->H = cfg->n_heads;
+  m->dh = cfg->head_dim;
+  m->V = cfg->vocab;
+  m->C1 = cfg->chunk[0];
+  m->C2 = cfg->chunk[1];
+  m->C = m->C1 * m->C2;
+  m->f = cfg->mlp_mult * cfg->d_model;
+  m->L1 = cfg->enc_layers[0];
+  m->Ltop = cfg->enc_layers[1];
+  m->Ld1 = cfg->dec_layers[0];
+  m->Ld2 = cfg->dec_layers[1];
+  m->use_tc = (m->dt == DT_BF16) && tma_available();
+  build_specs(m);
+  cudaStream_t s = nullptr;
+  for (int g = 0; g < G_COUNT; ++g) {
+    cudaError_t e = cudaMalloc((void**)&m->group_ptr[g], m->group_bytes[g]);
+    if (e != cudaSuccess) {
+      cudaGetLastError();
+      for (int k = 0; k < g; ++k) cudaFree(m->group_ptr[k]);
+      delete m;
+      return fail(e == cudaErrorMemoryAllocation ? PHOTON_ERR_OOM : PHOTON_ERR_CUDA,
+                  "weight allocation failed: %s", cudaGetErrorString(e));
+    }
+    generate_group(m, g, s);
+  }
+  cudaError_t e = cudaStreamSynchronize(s);
+  if (e == cudaSuccess) e = cudaGetLastError();
+  if (e != cudaSuccess) {
+    for (int g = 0; g < G_COUNT; ++g) cudaFree(m->group_ptr[g]);
+    delete m;
+    return fail(PHOTON_ERR_CUDA, "weight generation failed: %s", cudaGetErrorString(e));
+  }
+  *out = m;
+  return PHOTON_OK;
+}
+
+int photon_free_model(photon_model* m) {
+  g_err.clear();
+  if (!m) return fail(PHOTON_ERR_ARG, "model is NULL");
+  if (m->live_caches) return fail(PHOTON_ERR_ARG, "%d caches still use this model", m->live_caches);
+  CK(cudaDeviceSynchronize());
+  for (int g = 0; g < G_COUNT; ++g)
+    if (m->group_ptr[g]) cudaFree(m->group_ptr[g]);
+  delete m;
+  return PHOTON_OK;
+}
+
+int photon_model_info(const photon_model* m, photon_model_stats* out) {
+  g_err.clear();
+  if (!m || !out) return fail(PHOTON_ERR_ARG, "NULL argument");
+  memset(out, 0, sizeof(*out));
+  for (const auto& r : m->t) out->param_count += (uint64_t)r.numel;
+  for (int g = 0; g < G_COUNT; ++g) {
+    uint64_t bytes = 0;
+    for (const auto& r : m->t)
+      if (r.group == g) bytes += (uint64_t)r.numel * (r.gain ? 4 : m->es);
+    if (g == G_ENC1) out->encoder_bytes = bytes;
+    if (m->group_ptr[g]) out->resident_bytes += bytes;
+  }
+  out->encoder_resident = m->group_ptr[G_ENC1] != nullptr;
+  out->n_tensors = (int32_t)m->t.size();
+  out->live_caches = m->live_caches;
+  out->tcgen05_gemm = m->use_tc ? 1 : 0;
+  return PHOTON_OK;
+}
+
+int photon_export_weight(photon_model* m, int32_t index, void* d_dst, size_t dst_bytes,
+                         size_t* out_bytes, void* stream) {
+  g_err.clear();
+  if (!m) return fail(PHOTON_ERR_ARG, "model is NULL");
+  if (index < 0 || index >= (int)m->t.size()) return fail(PHOTON_ERR_ARG, "tensor index out of range");
+  const TensorRec& r = m->t[index];
+  const size_t bytes = (size_t)r.numel * (r.gain ? 4 : m->es);
+  if (out_bytes) *out_bytes = bytes;
+  if (!d_dst) return PHOTON_OK;
+  if (dst_bytes < bytes) return fail(PHOTON_ERR_ARG, "destination holds %zu bytes, need %zu", dst_bytes, bytes);
+  cudaStream_t s = (cudaStream_t)stream;
+  if (r.group == G_ENC1) RET(ensure_encoder(m, s));
+  CK(cudaMemcpyAsync(d_dst, m->ptr(index), bytes, cudaMemcpyDeviceToDevice, s));
+  return PHOTON_OK;
+}
+
+int photon_prefill(photon_model* m, const photon_cache* prefix, const int32_t* d_tokens, int32_t B,
+                   int32_t T, int32_t mode, int32_t max_new_chunks, void* stream, photon_cache** out) {
+  g_err.clear();
+  if (!m || !out) return fail(PHOTON_ERR_ARG, "NULL model or out");
+  *out = nullptr;
+  if (!d_tokens) return fail(PHOTON_ERR_ARG, "tokens pointer is NULL");
+  if (B <= 0) return fail(PHOTON_ERR_ARG, "batch must be positive");
+  if (T <= 0 || T % m->C) return fail(PHOTON_ERR_ARG, "T = %d is not a positive multiple of C1*C2 = %d", T, m->C);
+  if (mode != PHOTON_MODE_HIER && mode != PHOTON_MODE_REC) return fail(PHOTON_ERR_ARG, "unknown mode %d", mode);
+  if (max_new_chunks < 0) return fail(PHOTON_ERR_ARG, "max_new_chunks must be >= 0");
+  if (prefix) {
+    if (prefix->m != m) return fail(PHOTON_ERR_ARG, "prefix belongs to another model");
+    if (prefix->mode != PHOTON_MODE_HIER || !prefix->l1_k)
+      return fail(PHOTON_ERR_ARG, "prefix must be prefilled in HIER mode");
+    if (prefix->B != 1) return fail(PHOTON_ERR_ARG, "prefix batch must be 1");
+    if (prefix->prefix) return fail(PHOTON_ERR_ARG, "nested prefixes are not supported");
+  }
+  const long long rows0 = (long long)B * T;
+  if (rows0 > (1ll << 31) / 4) return fail(PHOTON_ERR_ARG, "B*T too large");
+  cudaStream_t s = (cudaStream_t)stream;
+  const int d = m->d, C1 = m->C1, C2 = m->C2, C = m->C;
+
+  photon_cache* c = new photon_cache();
+  c->m = m;
+  c->prefix = prefix;
+  c->B = B;
+  c->T = T;
+  c->mode = mode;
+  c->max_new = max_new_chunks;
+  c->stream = s;
+  c->n_pre = prefix ? prefix->N : 0;
+  c->n1_pre = prefix ? prefix->N1 : 0;
+  const int N_own = T / C, N1_own = T / C1;
+  c->Ncap = N_own + max_new_chunks;
+  c->N1cap = N1_own + (mode == PHOTON_MODE_HIER ? C2 * max_new_chunks : 0);
+
+  Allocator al{s, &c->allocs, &c->kv_bytes};
+  auto bail = [&](int code) {
+    cudaGetLastError();
+    free_list(c->allocs, s);
+    cudaStreamSynchronize(s);
+    delete c;
+    return code == PHOTON_ERR_OOM ? fail(code, "device allocation failed during prefill") : code;
+  };
+  int rc = ensure_encoder(m, s);
+  if (rc) return bail(rc);
+
+  const size_t hd = (size_t)m->H * m->dh;
+  c->top_layer = (size_t)B * hd * c->Ncap * m->es;
+  c->top_k = al.get<char>(c->top_layer * m->Ltop);
+  c->top_v = al.get<char>(c->top_layer * m->Ltop);
+  c->l1_layer = (size_t)B * hd * c->N1cap * m->es;
+  c->l1_k = al.get<char>(c->l1_layer * m->L1);
+  c->l1_v = al.get<char>(c->l1_layer * m->L1);
+  if (al.err != cudaSuccess) return bail(PHOTON_ERR_OOM);
+
+  // decode workspace (kept for the cache's lifetime)
+  al.counter = &c->ws_bytes;
+  const int rows_c = B * C, rows_g = B * C2;
+  const size_t es = m->es;
+  c->xd = al.get<float>((size_t)rows_c * d * 4);
+  c->xs = al.get<float>((size_t)rows_g * d * 4);
+  c->xt = al.get<float>((size_t)B * d * 4);
+  c->x1 = al.get<float>((size_t)rows_g * d * 4);
+  c->xn = al.get<void>((size_t)rows_c * d * es);
+  c->q = al.get<void>((size_t)rows_c * d * es);
+  c->att = al.get<void>((size_t)rows_c * d * es);
+  c->hid = al.get<void>((size_t)rows_c * m->f * es);
+  c->a_hat = al.get<void>((size_t)rows_g * d * es);
+  c->a = al.get<void>((size_t)rows_g * d * es);
+  c->embd = al.get<void>((size_t)rows_c * d * es);
+  c->hn = al.get<void>((size_t)rows_g * d * es);
+  c->o = al.get<void>((size_t)B * d * es);
+  c->logits = al.get<float>((size_t)rows_g * m->V * 4);
+  c->d2_layer = (size_t)B * hd * C2 * es;
+  c->d2k = al.get<char>(c->d2_layer * m->Ld2);
+  c->d2v = al.get<char>(c->d2_layer * m->Ld2);
+  c->d1_layer = (size_t)rows_g * hd * (2 * C1) * es;
+  c->d1k = al.get<char>(c->d1_layer * m->Ld1);
+  c->d1v = al.get<char>(c->d1_layer * m->Ld1);
+  c->next_ids = al.get<int32_t>((size_t)rows_g * 4);
+  c->used = al.get<int32_t>((size_t)rows_c * 4);
+  c->d_err = al.get<int>(16);
+  size_t gw = 0;
+  gw = std::max(gw, block_ws_need(m, B));
+  gw = std::max(gw, block_ws_need(m, rows_g));
+  gw = std::max(gw, block_ws_need(m, rows_c));
+  gw = std::max(gw, gemm_ws_need(m, B, C2 * d, d));
+  gw = std::max(gw, gemm_ws_need(m, rows_g, C1 * d, d));
+  gw = std::max(gw, gemm_ws_need(m, B, d, C2 * d));
+  gw = std::max(gw, gemm_ws_need(m, rows_g, d, C1 * d));
+  gw = std::max(gw, gemm_ws_need(m, rows_g, m->V, d));
+  c->gemm_ws_bytes = gw;
+  c->gemm_ws = al.get<float>(gw);
+  size_t aw = attn_ws_need(B, m->H, m->dh, 1, c->n_pre + c->Ncap);
+  if (mode == PHOTON_MODE_HIER)
+    aw = std::max(aw, attn_ws_need(B, m->H, m->dh, C2, c->n1_pre + c->N1cap));
+  aw = std::max(aw, attn_ws_need(B, m->H, m->dh, C2, C2));
+  aw = std::max(aw, attn_ws_need(rows_g, m->H, m->dh, C1, 2 * C1));
+  c->attn_ws_bytes = aw;
+  c->attn_ws = al.get<float>(aw);
+  const int positions =
+      std::max(std::max(c->n_pre + c->Ncap, c->n1_pre + N1_own + C2 * max_new_chunks), 2 * C1 + C2) + 1;
+  rc = upload_rope(m, c, al, positions);
+  if (al.err != cudaSuccess || rc) return bail(PHOTON_ERR_OOM);
+  if (cudaMemsetAsync(c->d_err, 0, 16, s) != cudaSuccess) return bail(PHOTON_ERR_CUDA);
+
+  // prefill workspace (released at the end of this call)
+  std::vector<void*> tmp;
+  size_t tmp_bytes = 0;
+  Allocator at{s, &tmp, &tmp_bytes};
+  const long long rows1 = rows0 / C1, rows2 = rows0 / C;
+  void* emb = at.get<void>((size_t)rows0 * d * es);
+  float* x = at.get<float>((size_t)rows1 * d * 4);
+  void* xn = at.get<void>((size_t)rows1 * d * es);
+  void* q = at.get<void>((size_t)rows1 * d * es);
+  void* att = at.get<void>((size_t)rows1 * d * es);
+  void* hid = at.get<void>((size_t)rows1 * m->f * es);
+  size_t pgw = std::max(block_ws_need(m, (int)rows1), block_ws_need(m, (int)rows2));
+  pgw = std::max(pgw, gemm_ws_need(m, (int)rows1, d, C1 * d));
+  pgw = std::max(pgw, gemm_ws_need(m, (int)rows2, d, C2 * d));
+  float* pws = at.get<float>(pgw);
+  if (at.err != cudaSuccess) {
+    free_list(tmp, s);
+    return bail(PHOTON_ERR_OOM);
+  }
+  Bufs pb{xn, q, att, hid, c->rope, pws, pgw, nullptr, 0, c->d_err};
+
+  // a1: embedding; a2: Chunker_1 (concatenate C1 states, linear C1*d -> d)
+  launch_embed(m->dt, d_tokens, m->ptr(m->i_embed), emb, (int)rows0, d, m->V, c->d_err, s);
+  gemm(m, pb, emb, (long long)C1 * d, m->ptr(m->i_ch1), (long long)C1 * d, (int)rows1, d, C1 * d,
+       epi(EPI_STORE_F32, x, d), s);
+  // a3: level-1 encoder over T/C1 positions per sequence, writing the level-1 KV
+  StackRun r1;
+  r1.G = B;
+  r1.q_len = N1_own;
+  r1.p0 = c->n1_pre;
+  r1.kv_off = c->n1_pre;
+  r1.kc = c->l1_k;
+  r1.vc = c->l1_v;
+  r1.layer_bytes = c->l1_layer;
+  r1.cap = c->N1cap;
+  if (prefix) {
+    r1.kp = prefix->l1_k;
+    r1.vp = prefix->l1_v;
+    r1.pre_layer_bytes = prefix->l1_layer;
+    r1.cap_pre = prefix->N1cap;
+    r1.n_pre = c->n1_pre;
+  }
+  run_stack(m, m->i_enc1, m->L1, x, r1, pb, s);
+  launch_rmsnorm(m->dt, x, (const float*)m->ptr(m->i_enc1_g), xn, (int)rows1, d, 1, 0,
+                 m->cfg.norm_eps, s);
+  // a4: Chunker_2 on the level-1 states (x is reused for the top stream)
+  gemm(m, pb, xn, (long long)C2 * d, m->ptr(m->i_ch2), (long long)C2 * d, (int)rows2, d, C2 * d,
+       epi(EPI_STORE_F32, x, d), s);
+  // a5: top encoder over T/C positions, writing the top KV
+  StackRun rt;
+  rt.G = B;
+  rt.q_len = N_own;
+  rt.p0 = c->n_pre;
+  rt.kv_off = c->n_pre;
+  rt.kc = c->top_k;
+  rt.vc = c->top_v;
+  rt.layer_bytes = c->top_layer;
+  rt.cap = c->Ncap;
+  if (prefix) {
+    rt.kp = prefix->top_k;
+    rt.vp = prefix->top_v;
+    rt.pre_layer_bytes = prefix->top_layer;
+    rt.cap_pre = prefix->Ncap;
+    rt.n_pre = c->n_pre;
+  }
+  run_stack(m, m->i_top, m->Ltop, x, rt, pb, s);
+  // pending output: final norm of the last top position of each sequence
+  launch_rmsnorm(m->dt, x, (const float*)m->ptr(m->i_top_g), c->o, B, d, N_own, N_own - 1,
+                 m->cfg.norm_eps, s);
+  cudaError_t le = cudaGetLastError();
+  free_list(tmp, s);
+  if (le != cudaSuccess) {
+    return bail(fail(PHOTON_ERR_CUDA, "prefill launch failed: %s", cudaGetErrorString(le)));
+  }
+
+  c->N = c->n_pre + N_own;
+  c->N1 = c->n1_pre + N1_own;
+  // a6: RecGen keeps only the top-level KV (RecGen section)
+  if (mode == PHOTON_MODE_REC) {
+    cudaFreeAsync(c->l1_k, s);
+    cudaFreeAsync(c->l1_v, s);
+    for (auto it = c->allocs.begin(); it != c->allocs.end();) {
+      if (*it == c->l1_k || *it == c->l1_v)
+        it = c->allocs.erase(it);
+      else
+        ++it;
+    }
+    c->kv_bytes -= 2 * c->l1_layer * m->L1;
+    c->l1_k = c->l1_v = nullptr;
+    c->N1 = 0;
+  }
+  m->live_caches++;
+  if (mode == PHOTON_MODE_HIER) m->hier_caches++;
+  if (prefix) prefix->dependents++;
+  if (m->hier_caches == 0) release_encoder(m, s);
+  *out = c;
+  return PHOTON_OK;
+}
+
+int photon_decode_step_ex(photon_model* m, photon_cache* c, int32_t mode, int32_t* d_out_tokens,
+                          float* d_out_logits, const int32_t* d_force_tokens,
+                          const void* d_force_a, void* stream) {
+  g_err.clear();
+  if (!m || !c || c->m != m) return fail(PHOTON_ERR_ARG, "model/cache mismatch");
+  if (!d_out_tokens) return fail(PHOTON_ERR_ARG, "output token buffer is NULL");
+  if (mode != PHOTON_MODE_HIER && mode != PHOTON_MODE_REC) return fail(PHOTON_ERR_ARG, "unknown mode %d", mode);
+  if (mode == PHOTON_MODE_HIER && (c->mode != PHOTON_MODE_HIER || !c->l1_k))
+    return fail(PHOTON_ERR_MODE, "HierGen needs the level-1 KV, discarded by a RecGen prefill");
+  if (c->steps >= c->max_new) return fail(PHOTON_ERR_CAPACITY, "cache is full (%d steps)", c->max_new);
+  if (mode == PHOTON_MODE_HIER && !m->group_ptr[G_ENC1]) RET(ensure_encoder(m, (cudaStream_t)stream));
+  cudaStream_t s = (cudaStream_t)stream;
+  c->stream = s;
+  const int B = c->B, C1 = m->C1, C2 = m->C2, C = m->C, d = m->d, V = m->V, G = B * C2;
+  const float eps = m->cfg.norm_eps;
+  const Bufs b = decode_bufs(c);
+
+  // a7: Converter_2 -- o [B, d] -> C2 conditioning vectors per sequence
+  gemm(m, b, c->o, d, m->ptr(m->i_cv2), d, B, C2 * d, d, epi(EPI_STORE_F32, c->xd, (long long)C2 * d), s);
+  // a8: level-2 decoder over its C2 positions (chunk-local causal) -> A-hat
+  StackRun r2;
+  r2.G = B;
+  r2.q_len = C2;
+  r2.kc = c->d2k;
+  r2.vc = c->d2v;
+  r2.layer_bytes = c->d2_layer;
+  r2.cap = C2;
+  run_stack(m, m->i_dec2, m->Ld2, c->xd, r2, b, s);
+  launch_rmsnorm(m->dt, c->xd, (const float*)m->ptr(m->i_dec2_g), c->a_hat, G, d, 1, 0, eps, s);
+  // a9: Converter_1 -- each A-hat row -> C1 conditioning vectors (rows g*C1 + i)
+  gemm(m, b, c->a_hat, d, m->ptr(m->i_cv1), d, G, C1 * d, d, epi(EPI_STORE_F32, c->xd, (long long)C1 * d), s);
+  // a10/a11: token decoder, prefix pass over the C1 conditioning positions,
+  // then C1-1 single-row steps; head + greedy argmax after each
+  StackRun r1;
+  r1.G = G;
+  r1.q_len = C1;
+  r1.kc = c->d1k;
+  r1.vc = c->d1v;
+  r1.layer_bytes = c->d1_layer;
+  r1.cap = 2 * C1;
+  run_stack(m, m->i_dec1, m->Ld1, c->xd, r1, b, s);
+  auto head = [&](const float* x, int in_step, int in_off, int i) {
+    launch_rmsnorm(m->dt, x, (const float*)m->ptr(m->i_dec1_g), c->hn, G, d, in_step, in_off, eps, s);
+    float* lg = d_out_logits ? d_out_logits + (size_t)i * V : c->logits;
+    const long long ld = d_out_logits ? (long long)C1 * V : V;
+    gemm(m, b, c->hn, d, m->ptr(m->i_head), d, G, V, d, epi(EPI_STORE_F32, lg, ld), s);
+    launch_argmax(lg, ld, G, V, i, C1, d_force_tokens, d_out_tokens, c->used, c->next_ids, c->d_err, s);
+  };
+  head(c->xd, C1, C1 - 1, 0);
+  for (int i = 1; i < C1; ++i) {
+    launch_embed_f32(m->dt, c->next_ids, m->ptr(m->i_embed), c->xs, G, d, V, c->d_err, s);
+    StackRun rs = r1;
+    rs.q_len = 1;
+    rs.p0 = C1 + i - 1;
+    run_stack(m, m->i_dec1, m->Ld1, c->xs, rs, b, s);
+    head(c->xs, 1, 0, i);
+  }
+  // a12: input of the top encoder's next position
+  if (mode == PHOTON_MODE_REC) {
+    // RecGen: Chunker_2(A-hat), no re-encoding
+    const void* src = d_force_a ? d_force_a : c->a_hat;
+    gemm(m, b, src, (long long)C2 * d, m->ptr(m->i_ch2), (long long)C2 * d, B, d, C2 * d,
+         epi(EPI_STORE_F32, c->xt, d), s);
+  } else {
+    // HierGen: embed the written tokens, Chunker_1, level-1 encoder with its cache, Chunker_2
+    launch_embed(m->dt, c->used, m->ptr(m->i_embed), c->embd, B * C, d, V, c->d_err, s);
+    gemm(m, b, c->embd, (long long)C1 * d, m->ptr(m->i_ch1), (long long)C1 * d, G, d, C1 * d,
+         epi(EPI_STORE_F32, c->x1, d), s);
+    StackRun re;
+    re.G = B;
+    re.q_len = C2;
+    re.p0 = c->N1;
+    re.kv_off = c->n1_pre;
+    re.kc = c->l1_k;
+    re.vc = c->l1_v;
+    re.layer_bytes = c->l1_layer;
+    re.cap = c->N1cap;
+    if (c->prefix) {
+      re.kp = c->prefix->l1_k;
+      re.vp = c->prefix->l1_v;
+      re.pre_layer_bytes = c->prefix->l1_layer;
+      re.cap_pre = c->prefix->N1cap;
+      re.n_pre = c->n1_pre;
+    }
+    run_stack(m, m->i_enc1, m->L1, c->x1, re, b, s);
+    launch_rmsnorm(m->dt, c->x1, (const float*)m->ptr(m->i_enc1_g), c->a, G, d, 1, 0, eps, s);
+    gemm(m, b, c->a, (long long)C2 * d, m->ptr(m->i_ch2), (long long)C2 * d, B, d, C2 * d,
+         epi(EPI_STORE_F32, c->xt, d), s);
+  }
+  // a13: one top-encoder step at position N (KV append + decode attention)
+  StackRun rt;
+  rt.G = B;
+  rt.q_len = 1;
+  rt.p0 = c->N;
+  rt.kv_off = c->n_pre;
+  rt.kc = c->top_k;
+  rt.vc = c->top_v;
+  rt.layer_bytes = c->top_layer;
+  rt.cap = c->Ncap;
+  if (c->prefix) {
+    rt.kp = c->prefix->top_k;
+    rt.vp = c->prefix->top_v;
+    rt.pre_layer_bytes = c->prefix->top_layer;
+    rt.cap_pre = c->prefix->Ncap;
+    rt.n_pre = c->n_pre;
+  }
+  run_stack(m, m->i_top, m->Ltop, c->xt, rt, b, s);
+  launch_rmsnorm(m->dt, c->xt, (const float*)m->ptr(m->i_top_g), c->o, B, d, 1, 0, eps, s);
+  CK(cudaGetLastError());
+  c->N += 1;
+  if (mode == PHOTON_MODE_HIER) {
+    c->N1 += C2;
+    c->has_a = true;
+  }
+  c->has_a_hat = true;
+  c->steps += 1;
+  return PHOTON_OK;
+}
+
+int photon_decode_step_hier(photon_model* m, photon_cache* c, int32_t* d_out_tokens,
+                            float* d_out_logits, void* stream) {
+  return photon_decode_step_ex(m, c, PHOTON_MODE_HIER, d_out_tokens, d_out_logits, nullptr, nullptr,
+                               stream);
+}
+
+int photon_decode_step_rec(photon_model* m, photon_cache* c, int32_t* d_out_tokens,
+                           float* d_out_logits, void* stream) {
+  return photon_decode_step_ex(m, c, PHOTON_MODE_REC, d_out_tokens, d_out_logits, nullptr, nullptr,
+                               stream);
+}
+
+int photon_free_cache(photon_cache* c) {
+  g_err.clear();
+  if (!c) return fail(PHOTON_ERR_ARG, "cache is NULL");
+  if (c->dependents) return fail(PHOTON_ERR_ARG, "%d caches still read this prefix", c->dependents);
+  photon_model* m = c->m;
+  CK(cudaStreamSynchronize(c->stream));
+  free_list(c->allocs, c->stream);
+  CK(cudaStreamSynchronize(c->stream));
+  if (c->prefix) c->prefix->dependents--;
+  m->live_caches--;
+  if (c->mode == PHOTON_MODE_HIER) m->hier_caches--;
+  delete c;
+  return PHOTON_OK;
+}
+
+int photon_cache_info(photon_cache* c, photon_cache_stats* out) {
+  g_err.clear();
+  if (!c || !out) return fail(PHOTON_ERR_ARG, "NULL argument");
+  memset(out, 0, sizeof(*out));
+  CK(cudaStreamSynchronize(c->stream));
+  int err = 0;
+  CK(cudaMemcpy(&err, c->d_err, sizeof(int), cudaMemcpyDeviceToHost));
+  out->B = c->B;
+  out->T = c->T;
+  out->mode = c->mode;
+  out->N = c->N;
+  out->N1 = c->N1;
+  out->n_prefix = c->n_pre;
+  out->n1_prefix = c->n1_pre;
+  out->capacity = c->Ncap;
+  out->steps = c->steps;
+  out->max_new_chunks = c->max_new;
+  out->device_error = err;
+  out->l1_resident = c->l1_k != nullptr;
+  out->kv_bytes = c->kv_bytes;
+  out->workspace_bytes = c->ws_bytes;
+  return PHOTON_OK;
+}
+
+int photon_export_state(photon_cache* c, int32_t which, int32_t layer, void* d_dst, size_t dst_bytes,
+                        size_t* out_bytes, void* stream) {
+  g_err.clear();
+  if (!c) return fail(PHOTON_ERR_ARG, "cache is NULL");
+  photon_model* m = c->m;
+  cudaStream_t s = (cudaStream_t)stream;
+  const size_t es = m->es, hd = (size_t)m->H * m->dh;
+  const char* src = nullptr;
+  size_t rows = 0, width = 0, pitch = 0;
+  switch (which) {
+    case PHOTON_STATE_TOP_K:
+    case PHOTON_STATE_TOP_V: {
+      if (layer < 0 || layer >= m->Ltop) return fail(PHOTON_ERR_ARG, "layer out of range");
+      const int n = c->N - c->n_pre;
+      src = (which == PHOTON_STATE_TOP_K ? c->top_k : c->top_v) + layer * c->top_layer;
+      rows = (size_t)c->B * m->H;
+      width = (size_t)n * m->dh * es;
+      pitch = (size_t)c->Ncap * m->dh * es;
+      break;
+    }
+    case PHOTON_STATE_L1_K:
+    case PHOTON_STATE_L1_V: {
+      if (!c->l1_k) return fail(PHOTON_ERR_ARG, "level-1 KV was discarded (RecGen cache)");
+      if (layer < 0 || layer >= m->L1) return fail(PHOTON_ERR_ARG, "layer out of range");
+      const int n = c->N1 - c->n1_pre;
+      src = (which == PHOTON_STATE_L1_K ? c->l1_k : c->l1_v) + layer * c->l1_layer;
+      rows = (size_t)c->B * m->H;
+      width = (size_t)n * m->dh * es;
+      pitch = (size_t)c->N1cap * m->dh * es;
+      break;
+    }
+    case PHOTON_STATE_PENDING_O:
+      src = (const char*)c->o;
+      rows = 1;
+      width = pitch = (size_t)c->B * m->d * es;
+      break;
+    case PHOTON_STATE_A_HAT:
+    case PHOTON_STATE_A:
+      if (which == PHOTON_STATE_A_HAT ? !c->has_a_hat : !c->has_a)
+        return fail(PHOTON_ERR_ARG, "no decode step has produced this state yet");
+      src = (const char*)(which == PHOTON_STATE_A_HAT ? c->a_hat : c->a);
+      rows = 1;
+      width = pitch = (size_t)c->B * m->C2 * m->d * es;
+      break;
+    default:
+      return fail(PHOTON_ERR_ARG, "unknown state %d", which);
+  }
+  (void)hd;
+  const size_t bytes = rows * width;
+  if (out_bytes) *out_bytes = bytes;
+  if (!d_dst || bytes == 0) return PHOTON_OK;
+  if (dst_bytes < bytes) return fail(PHOTON_ERR_ARG, "destination holds %zu bytes, need %zu", dst_bytes, bytes);
+  CK(cudaMemcpy2DAsync(d_dst, width, src, pitch, width, rows, cudaMemcpyDeviceToDevice, s));
+  return PHOTON_OK;
+}
+
+int photon_gemm(int32_t dtype, const void* d_A, int64_t lda, const void* d_W, int64_t ldw, int32_t M,
+                int32_t N, int32_t K, float* d_C, int64_t ldc, int32_t path, int32_t splits,
+                int32_t swap, void* stream) {
+  g_err.clear();
+  if (dtype != 0 && dtype != 1) return fail(PHOTON_ERR_ARG, "dtype must be 0 or 1");
+  if (!d_A || !d_W || !d_C || M <= 0 || N <= 0 || K <= 0) return fail(PHOTON_ERR_ARG, "bad GEMM arguments");
+  cudaStream_t s = (cudaStream_t)stream;
+  GemmArgs g;
+  g.A = d_A;
+  g.lda = lda;
+  g.W = d_W;
+  g.ldw = ldw;
+  g.M = M;
+  g.N = N;
+  g.K = K;
+  g.ep = epi(EPI_STORE_F32, d_C, ldc);
+  if (path == 1) {
+    launch_gemm_simt(dtype, g, s);
+    CK(cudaGetLastError());
+    return PHOTON_OK;
+  }
+  if (dtype != DT_BF16 || !tma_available()) {
+    if (path == 2) return fail(PHOTON_ERR_ARG, "the tcgen05 path needs bf16 and TMA");
+    launch_gemm_simt(dtype, g, s);
+    CK(cudaGetLastError());
+    return PHOTON_OK;
+  }
+  // generous scratch for any split count
+  const int nkb = K / 64 > 0 ? K / 64 : 1;
+  const size_t wsb = (size_t)nkb * M * N * sizeof(float);
+  float* ws = nullptr;
+  CK(cudaMallocAsync((void**)&ws, wsb, s));
+  GemmWorkspace w{ws, wsb};
+  int* err = nullptr;
+  bool ok = launch_gemm_tc(g, w, err, s, splits > 0 ? splits : 0, swap);
+  if (!ok && path == 0) {
+    launch_gemm_simt(dtype, g, s);
+    ok = true;
+  }
+  cudaFreeAsync(ws, s);
+  if (!ok) return fail(PHOTON_ERR_ARG, "shape not supported by the tcgen05 kernel");
+  CK(cudaGetLastError());
+  return PHOTON_OK;
+}
+
+int photon_attn_decode(int32_t dtype, const void* d_q, const void* d_k, const void* d_v, int32_t G,
+                       int32_t H, int32_t head_dim, int32_t cap, int32_t q_len, int32_t p0, void* d_o,
+                       void* stream) {
+  g_err.clear();
+  if (dtype != 0 && dtype != 1) return fail(PHOTON_ERR_ARG, "dtype must be 0 or 1");
+  if (!d_q || !d_k || !d_v || !d_o) return fail(PHOTON_ERR_ARG, "NULL buffer");
+  if (G <= 0 || H <= 0 || (head_dim != 32 && head_dim != 64)) return fail(PHOTON_ERR_ARG, "bad shape");
+  if (q_len < 1 || q_len > 4 || p0 < 0 || p0 + q_len > cap) return fail(PHOTON_ERR_ARG, "bad q_len/p0/cap");
+  cudaStream_t s = (cudaStream_t)stream;
+  AttnArgs a;
+  a.Q = d_q;
+  a.q_ld = (long long)H * head_dim;
+  a.K = d_k;
+  a.V = d_v;
+  a.cap = cap;
+  a.G = G;
+  a.H = H;
+  a.dh = head_dim;
+  a.q_len = q_len;
+  a.p0 = p0;
+  a.O = d_o;
+  a.o_ld = (long long)H * head_dim;
+  a.scale = 1.0f / sqrtf((float)head_dim);
+  const size_t wsb = attn_decode_workspace_bytes(a);
+  float* ws = nullptr;
+  if (wsb) CK(cudaMallocAsync((void**)&ws, wsb, s));
+  const bool ok = launch_attn_decode(dtype, a, ws, wsb, nullptr, s);
+  if (ws) cudaFreeAsync(ws, s);
+  if (!ok) return fail(PHOTON_ERR_ARG, "decode attention rejected the shape");
+  CK(cudaGetLastError());
+  return PHOTON_OK;
+}
+
+}  // extern "C"

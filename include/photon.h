@@ -1,0 +1,245 @@
+/*
+ * photon.h -- C ABI of the B200 PHOTON inference library (libphoton.so).
+ *
+ * PHOTON (ACL 2026, "Hierarchical Autoregressive Modeling for Lightspeed and
+ * Memory-Efficient Language Generation") keeps a hierarchy of latent
+ * streams: a bottom-up Context Chunker + Context Encoder compress tokens into
+ * coarse states, and top-down Context Converter + Context Decoder stacks
+ * write tokens back chunk by chunk.  This library implements, for L = 2
+ * levels, the hierarchical prefill and the two per-chunk decode procedures
+ * described on the "PHOTON vertical scan" explainer page (RecGen section):
+ * HierGen (re-encode the written tokens) and RecGen (feed the decoder's
+ * bottleneck reconstruction A-hat straight to the top encoder).
+ *
+ * Conventions (all entry points):
+ *  - Every call returns PHOTON_OK (0) or a negative PHOTON_ERR_* code and
+ *    never exits or throws.  photon_last_error() returns a message for the
+ *    last failing call on the calling thread.
+ *  - Device pointers ("d_" prefix) are caller-owned CUDA device memory, for
+ *    example torch tensors' data_ptr().  The library owns the model, the
+ *    caches and all their device buffers.
+ *  - `stream` is a cudaStream_t (NULL = legacy default stream).  Work is
+ *    enqueued on it and the calls return before the GPU finishes, except
+ *    where a call is documented as synchronising.
+ *  - Storage: dtype 0 = fp32 everywhere; dtype 1 = bf16 weights, KV caches
+ *    and inter-kernel activations with fp32 residual stream, accumulation,
+ *    norms, softmax and GELU.
+ *  - Token ids are int32.  Sequences in a batch never interact.
+ */
+#ifndef PHOTON_H_
+#define PHOTON_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define PHOTON_API __attribute__((visibility("default")))
+#else
+#define PHOTON_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct photon_model photon_model; /* opaque, library-owned */
+typedef struct photon_cache photon_cache; /* opaque, library-owned */
+
+/* Model shape.  Explainer, architecture section (module table and the
+ * hierarchy setting: L = 2, C1 = C2 = 4, or 2 x 2).  Readings taken where the
+ * pages are silent: pre-RMSNorm blocks (gain 1), full multi-head attention
+ * with rotate-half RoPE per stream, erf-GELU MLP of width mlp_mult*d_model,
+ * no biases, untied head.  Constraints checked by photon_init_weights:
+ * levels == 2; d_model == n_heads * head_dim; head_dim in {32, 64};
+ * d_model % 64 == 0; 1 <= C1, C2 <= 4; conv_kernel == 0 or equal to both C1
+ * and C2 (the converter is a transposed 1-D convolution with kernel = stride
+ * = C); dtype in {0, 1}. */
+typedef struct photon_config {
+  int32_t vocab;
+  int32_t d_model;
+  int32_t n_heads;
+  int32_t head_dim;
+  int32_t levels;        /* must be 2 */
+  int32_t chunk[2];      /* C1 (tokens per level-1 state), C2 (level-1 states per top state) */
+  int32_t enc_layers[2]; /* L1 (level-1 encoder), Ltop (top encoder) */
+  int32_t dec_layers[2]; /* Ld1 (token decoder), Ld2 (level-2 decoder) */
+  int32_t mlp_mult;      /* MLP width multiple (4) */
+  int32_t conv_kernel;   /* 0 = C_l; otherwise must equal C1 and C2 */
+  int32_t dtype;         /* 0 fp32, 1 bf16 */
+  float init_std;        /* 0.02 */
+  float rope_theta;      /* 10000 */
+  float norm_eps;        /* 1e-6 */
+} photon_config;
+
+enum {
+  PHOTON_OK = 0,
+  PHOTON_ERR_ARG = -1,          /* invalid argument or shape */
+  PHOTON_ERR_OOM = -2,          /* device allocation failed */
+  PHOTON_ERR_CUDA = -3,         /* a CUDA runtime call failed */
+  PHOTON_ERR_CAPACITY = -4,     /* decoding past max_new_chunks */
+  PHOTON_ERR_MODE = -5,         /* HierGen on a cache whose level-1 KV was discarded */
+  PHOTON_ERR_DEVICE_CHECK = -6  /* a kernel reported an error word (bad token id, expired wait) */
+};
+
+enum { PHOTON_MODE_HIER = 0, PHOTON_MODE_REC = 1 };
+
+/* Builds a model with weights drawn on the device by the counter-based
+ * generator: tensor t (fixed order: embed, chunker1, level-1 encoder
+ * blocks + final gain, chunker2, top blocks + final gain, converter2,
+ * level-2 decoder blocks + gain, converter1, token decoder blocks + gain,
+ * head; per block g_attn, wq, wk, wv, wo, g_mlp, w1, w2), element e: SplitMix64
+ * key mix(seed + gamma*(t+1)), draw z = mix(key + gamma*(e+1)), S = sum of the
+ * four 16-bit fields of z, w = fp64(S - 131070) * init_std*1.7320508075688772/65536,
+ * rounded to fp32 then to the storage type; RMSNorm gains are 1.  Linear maps
+ * are [out, in].  Synchronising.  Errors: ERR_ARG (bad config or out==NULL),
+ * ERR_OOM, ERR_CUDA. */
+PHOTON_API int photon_init_weights(const photon_config* cfg, uint64_t seed, photon_model** out);
+
+/* Frees a model.  Every cache built on it must have been freed first
+ * (ERR_ARG otherwise).  Synchronising. */
+PHOTON_API int photon_free_model(photon_model* m);
+
+/* Hierarchical prefill (explainer, module table: Chunker -> Encoder per
+ * level; the top encoder's KV is the only global cache).
+ *   d_tokens: device int32 [B, T] row-major prompt ids, 0 <= id < vocab.
+ *   T must be a positive multiple of C1*C2 (partial chunks are undefined).
+ *   mode: PHOTON_MODE_HIER keeps the level-1 encoder KV for HierGen;
+ *         PHOTON_MODE_REC discards it after prefill (RecGen section: only the
+ *         top-level global KV is kept) and, when no HierGen cache is alive,
+ *         releases the level-1 encoder and chunker weights until the next
+ *         prefill needs them.
+ *   max_new_chunks: decode steps this cache can take (each step appends one
+ *         top-level entry and, in HIER mode, C2 level-1 entries).
+ *   prefix: NULL, or a cache prefilled in HIER mode with B = 1 whose context
+ *         precedes every sequence of this batch (shared-prefix serving).  The
+ *         new cache reads the prefix's top and level-1 KV in place; the
+ *         prefix must outlive it.
+ *   out: receives the new cache.  Invalid token ids set the device error
+ *         word (see photon_cache_info).
+ * Errors: ERR_ARG, ERR_OOM, ERR_CUDA. */
+PHOTON_API int photon_prefill(photon_model* m, const photon_cache* prefix, const int32_t* d_tokens,
+                   int32_t B, int32_t T, int32_t mode, int32_t max_new_chunks, void* stream,
+                   photon_cache** out);
+
+/* One HierGen decode step = one top-level chunk of C1*C2 tokens per sequence
+ * (explainer, RecGen section, the three-stage loop): Converter_2 and the
+ * level-2 decoder turn the pending top output into A-hat; Converter_1 and the
+ * token decoder write the tokens greedily (lowest id on ties), the chunk's
+ * sub-chunks in parallel; the tokens are re-encoded (Chunker_1, level-1
+ * encoder with its cache, Chunker_2) and the top encoder advances one step.
+ *   d_out_tokens: device int32 [B, C1*C2]; token t = j*C1 + i is position i
+ *                 of level-1 sub-chunk j.
+ *   d_out_logits: NULL or device fp32 [B, C1*C2, vocab] logits of each token.
+ * Errors: ERR_ARG, ERR_MODE (cache prefilled in REC mode), ERR_CAPACITY. */
+PHOTON_API int photon_decode_step_hier(photon_model* m, photon_cache* c, int32_t* d_out_tokens,
+                            float* d_out_logits, void* stream);
+
+/* One RecGen decode step (explainer, RecGen section): tokens as in HierGen,
+ * then Chunker_2(A-hat) is fed straight to the top encoder; no level-1
+ * encoder work and no level-1 cache.  Same buffers and errors as HierGen
+ * except that it accepts caches of both modes. */
+PHOTON_API int photon_decode_step_rec(photon_model* m, photon_cache* c, int32_t* d_out_tokens,
+                           float* d_out_logits, void* stream);
+
+/* The decode step with its test hooks.
+ *   mode: PHOTON_MODE_HIER or PHOTON_MODE_REC.
+ *   d_force_tokens: NULL or device int32 [B, C1*C2]; entries >= 0 replace the
+ *     token fed back into the decoder (and, in HierGen, re-encoded), entries
+ *     < 0 keep the greedy choice.  d_out_tokens always receives the greedy
+ *     choice.  (Teacher forcing.)
+ *   d_force_a: NULL or device [B*C2, d_model] of the storage type; in RecGen
+ *     it replaces A-hat as the top encoder's input (the condition of
+ *     Theorem A.6, explainer RecGen section).  Ignored in HierGen.
+ * Errors as above. */
+PHOTON_API int photon_decode_step_ex(photon_model* m, photon_cache* c, int32_t mode, int32_t* d_out_tokens,
+                          float* d_out_logits, const int32_t* d_force_tokens,
+                          const void* d_force_a, void* stream);
+
+/* Frees a cache and its device buffers.  A prefix cache can only be freed
+ * after every cache built on it (ERR_ARG otherwise).  Synchronising. */
+PHOTON_API int photon_free_cache(photon_cache* c);
+
+typedef struct photon_cache_stats {
+  int32_t B, T, mode;
+  int32_t N;          /* top-level entries visible (prefix + own) */
+  int32_t N1;         /* level-1 entries visible (0 once discarded) */
+  int32_t n_prefix;   /* top entries read from the shared prefix */
+  int32_t n1_prefix;  /* level-1 entries read from the shared prefix */
+  int32_t capacity;   /* own top-level slots */
+  int32_t steps;      /* decode steps taken */
+  int32_t max_new_chunks;
+  int32_t device_error; /* first error word reported by a kernel, 0 if none */
+  int32_t l1_resident;  /* 1 while the level-1 KV is allocated */
+  uint64_t kv_bytes;    /* top + level-1 KV allocated for this cache */
+  uint64_t workspace_bytes;
+} photon_cache_stats;
+
+/* Cache bookkeeping.  Synchronises the cache's last stream to read the
+ * device error word.  Errors: ERR_ARG. */
+PHOTON_API int photon_cache_info(photon_cache* c, photon_cache_stats* out);
+
+typedef struct photon_model_stats {
+  uint64_t param_count;       /* all parameters */
+  uint64_t resident_bytes;    /* weight bytes currently on the device */
+  uint64_t encoder_bytes;     /* level-1 encoder + chunker-1 weight bytes */
+  int32_t encoder_resident;   /* 1 if those weights are on the device */
+  int32_t n_tensors;
+  int32_t live_caches;
+  int32_t tcgen05_gemm;       /* 1 if the tcgen05/TMA GEMM path is available */
+} photon_model_stats;
+
+PHOTON_API int photon_model_info(const photon_model* m, photon_model_stats* out);
+
+/* Copies parameter tensor `index` (generator order) into d_dst as stored:
+ * the storage type for drawn tensors, fp32 for RMSNorm gains; out_bytes
+ * receives the size.  Call with d_dst = NULL to query the size.  The level-1
+ * encoder tensors are regenerated if they are not resident.
+ * Errors: ERR_ARG (index, buffer too small). */
+PHOTON_API int photon_export_weight(photon_model* m, int32_t index, void* d_dst, size_t dst_bytes,
+                         size_t* out_bytes, void* stream);
+
+enum {
+  PHOTON_STATE_TOP_K = 0,   /* [B][H][N_own][head_dim] own top-level keys (post-RoPE), layer `layer` */
+  PHOTON_STATE_TOP_V = 1,   /* same layout, values */
+  PHOTON_STATE_L1_K = 2,    /* [B][H][N1_own][head_dim] level-1 keys */
+  PHOTON_STATE_L1_V = 3,
+  PHOTON_STATE_PENDING_O = 4, /* [B][d_model] top output after the final norm (conditions the next chunk) */
+  PHOTON_STATE_A_HAT = 5,   /* [B*C2][d_model] last step's level-2 decoder reconstruction */
+  PHOTON_STATE_A = 6        /* [B*C2][d_model] last HierGen step's level-1 encoder states */
+};
+
+/* Copies a piece of cache state (storage type) into d_dst, compacted to
+ * the entries in use.  Call with d_dst = NULL to query the size.
+ * Errors: ERR_ARG (unknown state, layer out of range, discarded level-1 KV,
+ * buffer too small). */
+PHOTON_API int photon_export_state(photon_cache* c, int32_t which, int32_t layer, void* d_dst,
+                        size_t dst_bytes, size_t* out_bytes, void* stream);
+
+/* Kernel-level entry: C[M, N] (fp32, row stride ldc) = A[M, K] * W[N, K]^T
+ * with A, W of the storage type (row strides lda, ldw in elements).
+ * path: 0 = the library's choice, 1 = CUDA-core kernel, 2 = tcgen05 kernel
+ * (bf16 only; K % 64 == 0, N % 64 == 0).  splits / swap (-1 = automatic)
+ * steer the tcgen05 kernel's split-K count and operand swap.  Allocates its
+ * split-K scratch internally.  Errors: ERR_ARG (unsupported shape or path). */
+PHOTON_API int photon_gemm(int32_t dtype, const void* d_A, int64_t lda, const void* d_W, int64_t ldw,
+                int32_t M, int32_t N, int32_t K, float* d_C, int64_t ldc, int32_t path,
+                int32_t splits, int32_t swap, void* stream);
+
+/* Kernel-level entry: split-K decode attention (the top-encoder decode
+ * kernel).  For G groups x H heads, q_len <= 4 new queries at positions
+ * p0..p0+q_len-1 attend causally over keys 0..p0+i of a cache
+ * d_k/d_v [G][H][cap][head_dim] (storage type, post-RoPE keys);
+ * d_q and d_o are [G*q_len][H*head_dim].  Scale 1/sqrt(head_dim).
+ * Allocates its split scratch internally.  Errors: ERR_ARG. */
+PHOTON_API int photon_attn_decode(int32_t dtype, const void* d_q, const void* d_k, const void* d_v, int32_t G,
+                       int32_t H, int32_t head_dim, int32_t cap, int32_t q_len, int32_t p0,
+                       void* d_o, void* stream);
+
+/* Message describing the last error on this thread ("" if none). */
+PHOTON_API const char* photon_last_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PHOTON_H_ */

@@ -1,0 +1,56 @@
+"""CPU checks of the C ABI: the library loads and exports every declared entry point."""
+import os
+import re
+
+import pytest
+
+import hierarchical_autoregressive_lm_b200 as hal
+
+HEADER = os.path.join(os.path.dirname(os.path.dirname(__file__)), "include", "photon.h")
+
+
+def declared():
+    src = open(HEADER).read()
+    return sorted(set(re.findall(r"PHOTON_API\s+[\w\s\*]+?\b(photon_\w+)\s*\(", src)))
+
+
+def test_header_declares_the_boundary():
+    names = declared()
+    for req in ("photon_init_weights", "photon_prefill", "photon_decode_step_hier",
+                "photon_decode_step_rec", "photon_free_cache"):
+        assert req in names
+    assert sorted(hal.EXPORTED) == names
+
+
+def test_library_loads_and_exports_every_symbol():
+    if not os.path.exists(hal.LIB_PATH):
+        from hierarchical_autoregressive_lm_b200.build import build
+        build()
+    lib = hal.load_library()
+    for name in declared():
+        assert hasattr(lib, name), name
+    assert lib.photon_last_error() == b""
+
+
+def test_config_struct_layout():
+    import ctypes
+    # 12 int32 fields (two of them arrays of 2) + 3 floats, no padding
+    assert ctypes.sizeof(hal.photon_config) == 4 * (5 + 6 + 3 + 3)
+    c = hal.config_struct({"vocab": 256, "d_model": 64, "n_heads": 2, "head_dim": 32, "C1": 4,
+                           "C2": 4, "L1": 1, "Ltop": 1, "Ld1": 1, "Ld2": 1, "dtype": "fp32"})
+    assert (c.chunk[0], c.chunk[1], c.levels, c.dtype) == (4, 4, 2, 0)
+
+
+def test_missing_library_fails_loudly(tmp_path):
+    with pytest.raises(ImportError):
+        hal.load_library.__wrapped__(str(tmp_path / "nope.so")) if hasattr(hal.load_library, "__wrapped__") \
+            else _load_missing(str(tmp_path / "nope.so"))
+
+
+def _load_missing(path):
+    saved = hal._lib
+    hal._lib = None
+    try:
+        hal.load_library(path)
+    finally:
+        hal._lib = saved

@@ -1,0 +1,102 @@
+"""Kernel-level GPU parity: GEMM paths and the split-K decode attention.
+
+Each kernel is called through the C ABI and compared element by element
+with the oracle's definition of the same operation (fp64 on the CPU, on the
+same rounded inputs).
+"""
+import numpy as np
+import pytest
+import torch
+
+import hierarchical_autoregressive_lm_b200 as hal
+import oracle
+
+pytestmark = pytest.mark.gpu
+
+
+def _rand(shape, dtype, seed, scale=1.0):
+    g = torch.Generator().manual_seed(seed)
+    return (torch.randn(*shape, generator=g) * scale).to(dtype)
+
+
+def _gemm_ref(A, W):
+    return A.double().numpy() @ W.double().numpy().T
+
+
+@pytest.mark.parametrize("M,N,K", [(64, 128, 64), (100, 192, 320), (7, 64, 128)])
+def test_gemm_simt_fp32(M, N, K):
+    A, W = _rand((M, K), torch.float32, 1), _rand((N, K), torch.float32, 2)
+    C = torch.zeros(M, N, device="cuda")
+    hal.gemm(A.cuda(), W.cuda(), C, path=1)
+    torch.cuda.synchronize()
+    np.testing.assert_allclose(C.cpu().numpy(), _gemm_ref(A, W), rtol=1e-4, atol=1e-4)
+
+
+# (M, N, K, splits, swap): both operand orientations, split-K, ragged M
+TC_CASES = [
+    (128, 128, 64, 1, 0), (256, 512, 1024, 1, 0), (300, 256, 512, 1, 0), (4096, 1024, 1024, 1, 0),
+    (64, 1024, 1024, 1, 1), (64, 1024, 1024, 4, 1), (256, 3072, 1024, 2, 1), (100, 384, 256, 1, 1),
+    (256, 32000, 1024, 1, 1), (1024, 4096, 1024, 1, 0), (512, 1024, 4096, 8, 0),
+]
+
+
+@pytest.mark.parametrize("M,N,K,splits,swap", TC_CASES)
+def test_gemm_tcgen05_bf16(M, N, K, splits, swap):
+    A, W = _rand((M, K), torch.bfloat16, 3), _rand((N, K), torch.bfloat16, 4)
+    C = torch.full((M, N), float("nan"), device="cuda")
+    hal.gemm(A.cuda(), W.cuda(), C, path=2, splits=splits, swap=swap)
+    torch.cuda.synchronize()
+    ref = _gemm_ref(A, W)
+    got = C.cpu().double().numpy()
+    # fp32 accumulation over K bf16 products: |err| <~ K * 2^-24 * sum|a*b|
+    tol = 1e-5 * np.sqrt(K) * 4
+    assert np.isfinite(got).all()
+    np.testing.assert_allclose(got, ref, rtol=0, atol=tol * np.abs(ref).max() + 1e-4)
+
+
+def test_gemm_tcgen05_strided_operands():
+    # leading dimensions larger than K (views into wider buffers)
+    M, N, K = 192, 256, 256
+    Abig = _rand((M, 2 * K), torch.bfloat16, 5)
+    W = _rand((N, K), torch.bfloat16, 6)
+    C = torch.zeros(M, 2 * N, device="cuda")
+    Ad = Abig.cuda()
+    hal.gemm(Ad[:, K:], W.cuda(), C[:, :N], path=2)
+    torch.cuda.synchronize()
+    np.testing.assert_allclose(C[:, :N].cpu().double().numpy(), _gemm_ref(Abig[:, K:], W),
+                               rtol=0, atol=2e-3)
+    assert torch.all(C[:, N:] == 0)
+
+
+def _attn_case(dtype, G, H, dh, cap, q_len, p0, seed):
+    q = _rand((G * q_len, H * dh), dtype, seed)
+    k = _rand((G, H, cap, dh), dtype, seed + 1)
+    v = _rand((G, H, cap, dh), dtype, seed + 2)
+    out = torch.zeros(G * q_len, H * dh, dtype=dtype, device="cuda")
+    hal.attn_decode(q.cuda(), k.cuda(), v.cuda(), q_len, p0, out)
+    torch.cuda.synchronize()
+    got = out.float().cpu().numpy().reshape(G, q_len, H, dh)
+    qd = q.double().numpy().reshape(G, q_len, H, dh)
+    kd, vd = k.double().numpy(), v.double().numpy()
+    ref = np.zeros_like(got, dtype=np.float64)
+    for g in range(G):
+        for h in range(H):
+            ref[g, :, h] = oracle.decode_attention(qd[g, :, h], kd[g, h, :p0 + q_len],
+                                                   vd[g, h, :p0 + q_len], p0)
+    return got, ref
+
+
+@pytest.mark.parametrize("G,H,cap,q_len,p0", [
+    (4, 16, 300, 1, 256), (2, 16, 2200, 1, 2111), (3, 4, 40, 4, 30), (64, 16, 288, 1, 271),
+    (5, 2, 8, 1, 0), (16, 16, 1200, 4, 1100), (7, 3, 513, 1, 512),
+])
+def test_attn_decode_bf16(G, H, cap, q_len, p0):
+    got, ref = _attn_case(torch.bfloat16, G, H, 64, cap, q_len, p0, 10)
+    # output rounded to bf16: 2^-8 relative
+    np.testing.assert_allclose(got, ref, rtol=1e-2, atol=1e-2 * np.abs(ref).max())
+
+
+@pytest.mark.parametrize("G,H,cap,q_len,p0", [(1, 2, 80, 1, 70), (1, 2, 70, 4, 60), (3, 2, 8, 1, 3)])
+def test_attn_decode_fp32(G, H, cap, q_len, p0):
+    got, ref = _attn_case(torch.float32, G, H, 32, cap, q_len, p0, 20)
+    np.testing.assert_allclose(got, ref, rtol=1e-5, atol=1e-5)
