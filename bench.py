@@ -58,8 +58,8 @@ class ClockSampler:
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
-    def __init__(self, gpu_index: int):
-        self.idx = gpu_index
+    def __init__(self, gpu_id: str):
+        self.idx = gpu_id
         self.proc = None
         self.lines: list[str] = []
         self.t = None
@@ -173,7 +173,10 @@ def run_gpu(args) -> None:
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
-    with ClockSampler(dev.index) as clk:
+    n_launch0 = hal.launch_count()
+    props = torch.cuda.get_device_properties(dev)
+    gpu_id = f"GPU-{props.uuid}" if getattr(props, "uuid", None) else str(dev.index)
+    with ClockSampler(gpu_id) as clk:
         t0 = torch.cuda.Event(enable_timing=True)
         t1 = torch.cuda.Event(enable_timing=True)
         t0.record(stream)
@@ -183,6 +186,7 @@ def run_gpu(args) -> None:
                 caches.pop(0).free()
         t1.record(stream)
         torch.cuda.synchronize()
+    launches = hal.launch_count() - n_launch0
     for c in caches:
         c.free()
     if world > 1:
@@ -247,7 +251,7 @@ def run_gpu(args) -> None:
         "e2e": {"value": round(world * B * chunks * C * e2e_steps / (e2e_ms / 1e3), 1), "unit": UNIT,
                 "h2d_bytes_per_step": int(B * T * 4), "d2h_bytes_per_step": int(B * chunks * C * 4),
                 "covers": "H2D prompt + prefill + RecGen decode + per-chunk D2H of tokens"},
-        "gpu_launches": launch_count(model, wl, B) * args.steps,
+        "gpu_launches": launches,
         "roofline": roof,
         "clocks": clk.summary(),
     }
@@ -258,20 +262,6 @@ def run_gpu(args) -> None:
     model.free()
     if world > 1:
         dist.destroy_process_group()
-
-
-def launch_count(model, wl, B) -> int:
-    """Kernels the library launches for one prefill + the decode chunks
-    (counted from the launch sequences in runtime.cu)."""
-    s = model.shape
-    C1, C2, chunks = s["C1"], s["C2"], wl["decode_tokens"] // (s["C1"] * s["C2"])
-    M = B  # rows of the smallest GEMMs; split-K adds one reduction launch per split GEMM
-    per_block = 8            # 2 norms + 4 GEMMs + attention (+ combine) ~ 8 launches
-    prefill = 3 + per_block * (s["L1"] + s["Ltop"]) + 2
-    dec = (1 + per_block * s["Ld2"] + 1 + 1 + per_block * s["Ld1"] + 3
-           + (C1 - 1) * (1 + per_block * s["Ld1"] + 3) + 1 + per_block * s["Ltop"] + 1)
-    del M
-    return prefill + chunks * dec
 
 
 def measure_roofline(model, wl, dev, stream) -> dict:

@@ -16,7 +16,7 @@ import os
 from typing import Optional
 
 __all__ = ["PhotonError", "Model", "Cache", "load_library", "LIB_PATH", "MODE_HIER",
-           "MODE_REC", "STATE", "gemm", "attn_decode", "config_struct", "EXPORTED"]
+           "MODE_REC", "STATE", "launch_count", "gemm", "attn_decode", "config_struct", "EXPORTED"]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libphoton.so")
 
@@ -31,7 +31,7 @@ EXPORTED = ("photon_init_weights", "photon_free_model", "photon_prefill",
             "photon_decode_step_hier", "photon_decode_step_rec", "photon_decode_step_ex",
             "photon_free_cache", "photon_cache_info", "photon_model_info",
             "photon_export_weight", "photon_export_state", "photon_gemm",
-            "photon_attn_decode", "photon_last_error")
+            "photon_attn_decode", "photon_launch_count", "photon_last_error")
 
 
 class PhotonError(RuntimeError):
@@ -96,6 +96,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         fn = getattr(L, name)
         fn.argtypes = args
         fn.restype = ctypes.c_int
+    L.photon_launch_count.argtypes = []
+    L.photon_launch_count.restype = ctypes.c_uint64
     L.photon_last_error.argtypes = []
     L.photon_last_error.restype = ctypes.c_char_p
     _lib = L
@@ -231,6 +233,11 @@ class Cache:
         if self._h:
             _check(load_library().photon_free_cache(self._h))
             self._h = None
+
+
+def launch_count() -> int:
+    """Kernels launched by the library in this process so far."""
+    return int(load_library().photon_launch_count())
 
 
 def gemm(A, W, C, path: int = 0, splits: int = 0, swap: int = -1, stream=None) -> None:

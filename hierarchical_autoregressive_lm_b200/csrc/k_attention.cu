@@ -262,9 +262,11 @@ void run_decode(const AttnArgs& a, const DecPlan& p, float* part, int* err, cuda
   }
   dim3 grid(p.splits, a.H, a.G);
   k_attn_decode<T, DH, QMAX><<<grid, kDecThreads, smem, s>>>(a, p.chunk, p.splits, part, err);
+  note_launch();
   if (p.splits > 1) {
     dim3 cg(a.H, a.G * a.q_len);
     k_attn_combine<T, DH><<<cg, DH, 0, s>>>(a, p.splits, part);
+    note_launch();
   }
 }
 
@@ -369,13 +371,25 @@ void launch_attn_prefill(int dt, const AttnArgs& a, cudaStream_t s) {
   if (a.G <= 0 || a.q_len <= 0) return;
   dim3 grid((a.q_len + 31) / 32, a.H, a.G);
   if (dt == DT_BF16 && a.dh == 64)
-    k_attn_prefill<bf16, 64><<<grid, 128, 0, s>>>(a);
+    {
+      k_attn_prefill<bf16, 64><<<grid, 128, 0, s>>>(a);
+      note_launch();
+    }
   else if (dt == DT_F32 && a.dh == 32)
-    k_attn_prefill<float, 32><<<grid, 128, 0, s>>>(a);
+    {
+      k_attn_prefill<float, 32><<<grid, 128, 0, s>>>(a);
+      note_launch();
+    }
   else if (dt == DT_F32 && a.dh == 64)
-    k_attn_prefill<float, 64><<<grid, 128, 0, s>>>(a);
+    {
+      k_attn_prefill<float, 64><<<grid, 128, 0, s>>>(a);
+      note_launch();
+    }
   else if (dt == DT_BF16 && a.dh == 32)
-    k_attn_prefill<bf16, 32><<<grid, 128, 0, s>>>(a);
+    {
+      k_attn_prefill<bf16, 32><<<grid, 128, 0, s>>>(a);
+      note_launch();
+    }
 }
 
 }  // namespace photon

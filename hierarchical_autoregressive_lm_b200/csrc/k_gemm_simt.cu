@@ -76,11 +76,17 @@ void launch_gemm_simt(int dt, const GemmArgs& a, cudaStream_t s) {
   if (a.M <= 0 || a.N <= 0) return;
   dim3 grid((a.N + 63) / 64, (a.M + 63) / 64);
   if (dt == DT_F32)
-    k_gemm_simt<float><<<grid, 256, 0, s>>>((const float*)a.A, a.lda, (const float*)a.W, a.ldw,
-                                            a.M, a.N, a.K, a.ep);
+    {
+      k_gemm_simt<float><<<grid, 256, 0, s>>>((const float*)a.A, a.lda, (const float*)a.W, a.ldw,
+                                              a.M, a.N, a.K, a.ep);
+      note_launch();
+    }
   else
-    k_gemm_simt<bf16><<<grid, 256, 0, s>>>((const bf16*)a.A, a.lda, (const bf16*)a.W, a.ldw, a.M,
-                                           a.N, a.K, a.ep);
+    {
+      k_gemm_simt<bf16><<<grid, 256, 0, s>>>((const bf16*)a.A, a.lda, (const bf16*)a.W, a.ldw, a.M,
+                                             a.N, a.K, a.ep);
+      note_launch();
+    }
 }
 
 void launch_gemm(int dt, const GemmArgs& a, const GemmWorkspace& ws, int* err, cudaStream_t s) {

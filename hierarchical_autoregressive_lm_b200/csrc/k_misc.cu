@@ -1,10 +1,16 @@
 // Weight generation, embeddings, RMSNorm, greedy argmax and the split-K
 // reduction.  All memory-bound row kernels.
+#include <atomic>
+
 #include "common.cuh"
 #include "epilogue.cuh"
 #include "kernels.h"
 
 namespace photon {
+
+static std::atomic<unsigned long long> g_launches{0};
+void note_launch(int n) { g_launches.fetch_add((unsigned long long)n, std::memory_order_relaxed); }
+unsigned long long launch_total() { return g_launches.load(std::memory_order_relaxed); }
 
 // ------------------------------------------------------------------ weights
 // Counter-based draw, defined independently of any other implementation:
@@ -50,9 +56,15 @@ void launch_init_normal(int dt, void* dst, long long numel, uint64_t seed, int t
   if (blocks > 148 * 64) blocks = 148 * 64;
   if (blocks < 1) blocks = 1;
   if (dt == DT_F32)
-    k_init_normal<float><<<(int)blocks, threads, 0, s>>>((float*)dst, numel, base, K);
+    {
+      k_init_normal<float><<<(int)blocks, threads, 0, s>>>((float*)dst, numel, base, K);
+      note_launch();
+    }
   else
-    k_init_normal<bf16><<<(int)blocks, threads, 0, s>>>((bf16*)dst, numel, base, K);
+    {
+      k_init_normal<bf16><<<(int)blocks, threads, 0, s>>>((bf16*)dst, numel, base, K);
+      note_launch();
+    }
 }
 
 __global__ void k_fill_f32(float* dst, long long n, float v) {
@@ -65,6 +77,7 @@ void launch_fill_f32(float* dst, long long n, float v, cudaStream_t s) {
   if (blocks > 148 * 16) blocks = 148 * 16;
   if (blocks < 1) blocks = 1;
   k_fill_f32<<<(int)blocks, 256, 0, s>>>(dst, n, v);
+  note_launch();
 }
 
 template <typename T>
@@ -78,9 +91,15 @@ void launch_to_f32(int dt, const void* src, float* dst, long long n, cudaStream_
   if (blocks > 148 * 16) blocks = 148 * 16;
   if (blocks < 1) blocks = 1;
   if (dt == DT_F32)
-    k_to_f32<float><<<(int)blocks, 256, 0, s>>>((const float*)src, dst, n);
+    {
+      k_to_f32<float><<<(int)blocks, 256, 0, s>>>((const float*)src, dst, n);
+      note_launch();
+    }
   else
-    k_to_f32<bf16><<<(int)blocks, 256, 0, s>>>((const bf16*)src, dst, n);
+    {
+      k_to_f32<bf16><<<(int)blocks, 256, 0, s>>>((const bf16*)src, dst, n);
+      note_launch();
+    }
 }
 
 // ------------------------------------------------------------------ embedding
@@ -107,9 +126,15 @@ void launch_embed(int dt, const int32_t* ids, const void* E, void* out, int rows
   const int threads = 256;
   const int blocks = (rows * 32 + threads - 1) / threads;
   if (dt == DT_F32)
-    k_embed<float><<<blocks, threads, 0, s>>>(ids, (const float*)E, (float*)out, rows, d, vocab, err);
+    {
+      k_embed<float><<<blocks, threads, 0, s>>>(ids, (const float*)E, (float*)out, rows, d, vocab, err);
+      note_launch();
+    }
   else
-    k_embed<bf16><<<blocks, threads, 0, s>>>(ids, (const bf16*)E, (bf16*)out, rows, d, vocab, err);
+    {
+      k_embed<bf16><<<blocks, threads, 0, s>>>(ids, (const bf16*)E, (bf16*)out, rows, d, vocab, err);
+      note_launch();
+    }
 }
 
 template <typename T>
@@ -133,9 +158,15 @@ void launch_embed_f32(int dt, const int32_t* ids, const void* E, float* x, int r
   const int threads = 256;
   const int blocks = (rows * 32 + threads - 1) / threads;
   if (dt == DT_F32)
-    k_embed_f32<float><<<blocks, threads, 0, s>>>(ids, (const float*)E, x, rows, d, vocab, err);
+    {
+      k_embed_f32<float><<<blocks, threads, 0, s>>>(ids, (const float*)E, x, rows, d, vocab, err);
+      note_launch();
+    }
   else
-    k_embed_f32<bf16><<<blocks, threads, 0, s>>>(ids, (const bf16*)E, x, rows, d, vocab, err);
+    {
+      k_embed_f32<bf16><<<blocks, threads, 0, s>>>(ids, (const bf16*)E, x, rows, d, vocab, err);
+      note_launch();
+    }
 }
 
 // ------------------------------------------------------------------ RMSNorm
@@ -170,9 +201,15 @@ void launch_rmsnorm(int dt, const float* x, const float* g, void* out, int rows,
   const int threads = 256;
   const int blocks = (rows * 32 + threads - 1) / threads;
   if (dt == DT_F32)
-    k_rmsnorm<float><<<blocks, threads, 0, s>>>(x, g, (float*)out, rows, d, in_step, in_off, eps);
+    {
+      k_rmsnorm<float><<<blocks, threads, 0, s>>>(x, g, (float*)out, rows, d, in_step, in_off, eps);
+      note_launch();
+    }
   else
-    k_rmsnorm<bf16><<<blocks, threads, 0, s>>>(x, g, (bf16*)out, rows, d, in_step, in_off, eps);
+    {
+      k_rmsnorm<bf16><<<blocks, threads, 0, s>>>(x, g, (bf16*)out, rows, d, in_step, in_off, eps);
+      note_launch();
+    }
 }
 
 // ------------------------------------------------------------------ argmax
@@ -228,6 +265,7 @@ void launch_argmax(const float* logits, long long ld, int rows, int V, int i, in
                    cudaStream_t s) {
   if (rows <= 0) return;
   k_argmax<<<rows, 256, 0, s>>>(logits, ld, rows, V, i, C1, force, own, used, next_ids, err);
+  note_launch();
 }
 
 // ------------------------------------------------------------------ split-K reduce
@@ -260,9 +298,15 @@ void launch_splitk_reduce(int dt, const float* part, int splits, int M, int N, c
   const int threads = 256;
   const long long blocks = (total + threads - 1) / threads;
   if (dt == DT_F32)
-    k_splitk_reduce<float><<<(int)blocks, threads, 0, s>>>(part, splits, M, N, ep);
+    {
+      k_splitk_reduce<float><<<(int)blocks, threads, 0, s>>>(part, splits, M, N, ep);
+      note_launch();
+    }
   else
-    k_splitk_reduce<bf16><<<(int)blocks, threads, 0, s>>>(part, splits, M, N, ep);
+    {
+      k_splitk_reduce<bf16><<<(int)blocks, threads, 0, s>>>(part, splits, M, N, ep);
+      note_launch();
+    }
 }
 
 }  // namespace photon

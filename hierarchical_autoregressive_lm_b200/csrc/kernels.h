@@ -117,6 +117,11 @@ bool launch_attn_decode(int dt, const AttnArgs& a, float* part, size_t part_byte
 // Causal attention for many new queries per group (prefill).
 void launch_attn_prefill(int dt, const AttnArgs& a, cudaStream_t s);
 
+// ---- launch accounting ------------------------------------------------------
+// Process-wide count of kernels this library has launched.
+void note_launch(int n = 1);
+unsigned long long launch_total();
+
 // ---- TMA descriptors -----------------------------------------------------
 bool tma_available();
 

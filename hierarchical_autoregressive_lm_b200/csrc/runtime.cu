@@ -427,6 +427,8 @@ extern "C" {
 
 const char* photon_last_error(void) { return g_err.c_str(); }
 
+uint64_t photon_launch_count(void) { return (uint64_t)launch_total(); }
+
 int photon_init_weights(const photon_config* cfg, uint64_t seed, photon_model** out) {
   g_err.clear();
   if (!out) return fail(PHOTON_ERR_ARG, "out is NULL");

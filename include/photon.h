@@ -235,6 +235,10 @@ PHOTON_API int photon_attn_decode(int32_t dtype, const void* d_q, const void* d_
                        int32_t H, int32_t head_dim, int32_t cap, int32_t q_len, int32_t p0,
                        void* d_o, void* stream);
 
+/* Number of kernels this library has launched in this process so far
+ * (every launch of every entry point; host-side counter, no GPU access). */
+PHOTON_API uint64_t photon_launch_count(void);
+
 /* Message describing the last error on this thread ("" if none). */
 PHOTON_API const char* photon_last_error(void);
 

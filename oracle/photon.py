@@ -116,13 +116,31 @@ def attention(q: np.ndarray, k: np.ndarray, v: np.ndarray,
     positions <= p.  Returns [nq, H, dh].
     """
     dh = q.shape[-1]
-    s = np.einsum("qhd,khd->hqk", q, k) / math.sqrt(dh)
-    allowed = np.asarray(k_pos)[None, :] <= np.asarray(q_pos)[:, None]
-    s = np.where(allowed[None], s, -np.inf)
-    s = s - s.max(axis=-1, keepdims=True)
-    p = np.exp(s)
-    p = p / p.sum(axis=-1, keepdims=True)
-    return np.einsum("hqk,khd->qhd", p, v)
+    q_pos = np.asarray(q_pos)
+    k_pos = np.asarray(k_pos)
+    out = np.empty(q.shape[:1] + v.shape[1:])
+    kt = k.transpose(1, 2, 0)            # [H, dh, nk]
+    vt = v.transpose(1, 0, 2)            # [H, nk, dh]
+    ascending = bool(np.all(np.diff(k_pos) > 0))
+    # Query rows are independent (one softmax per row); they are processed
+    # in groups only to bound the memory of the score matrix.  With keys in
+    # ascending position order, keys after the group's last visible position
+    # have weight exactly 0 and are left out of the group's products.
+    step = max(1, (1 << 25) // max(1, q.shape[1] * k.shape[0]))
+    for lo in range(0, q.shape[0], step):
+        hi = min(q.shape[0], lo + step)
+        nk = k.shape[0]
+        if ascending:
+            nk = int(np.searchsorted(k_pos, q_pos[lo:hi].max(), side="right"))
+        s = np.matmul(q[lo:hi].transpose(1, 0, 2), kt[:, :, :nk])
+        s *= 1.0 / math.sqrt(dh)
+        allowed = k_pos[None, :nk] <= q_pos[lo:hi, None]
+        np.copyto(s, -np.inf, where=~allowed[None])
+        s -= s.max(axis=-1, keepdims=True)
+        np.exp(s, out=s)
+        s /= s.sum(axis=-1, keepdims=True)
+        out[lo:hi] = np.matmul(s, vt[:, :nk]).transpose(1, 0, 2)
+    return out
 
 
 @dataclass
@@ -260,6 +278,27 @@ class PhotonOracle:
                         N1=(T // cfg.C1 if mode == "hier" else 0),
                         tokens=[int(t) for t in tokens],
                         top_inputs=[r.copy() for r in u])
+
+    def prefill_after(self, prefix: SeqState, tokens: np.ndarray, mode: str) -> SeqState:
+        """Prefill of `tokens` continuing a HierGen-mode state `prefix` (a shared
+        context that precedes them): the same Chunker/Encoder passes as
+        `prefill`, with the prefix's level-1 and top caches as the past.
+        Equal to prefill(prefix tokens + tokens), which the tests pin."""
+        cfg = self.cfg
+        if prefix.l1 is None:
+            raise ValueError("the prefix must keep its level-1 cache (HierGen mode)")
+        tokens = np.asarray(tokens, dtype=np.int64)
+        T = tokens.shape[0]
+        if T <= 0 or T % cfg.C:
+            raise ValueError("prompt length must be a positive multiple of C1*C2")
+        s1, l1 = self.encode_level1(tokens, prefix.N1, prefix.l1)
+        u = chunker(s1, self.w["chunker2"], cfg.C2)
+        o_all, top = self.top_encode(u, prefix.N, prefix.top)
+        return SeqState(mode=mode, top=top, l1=(l1 if mode == "hier" else None),
+                        o=o_all[-1].copy(), N=prefix.N + T // cfg.C,
+                        N1=(prefix.N1 + T // cfg.C1 if mode == "hier" else 0),
+                        tokens=list(prefix.tokens) + [int(t) for t in tokens],
+                        top_inputs=list(prefix.top_inputs) + [r.copy() for r in u])
 
     # -- top-down -------------------------------------------------------------
     def decode_chunk2(self, o: np.ndarray) -> np.ndarray:

@@ -34,6 +34,9 @@ Definition (all integer arithmetic modulo 2^64):
 """
 from __future__ import annotations
 
+import os
+from concurrent.futures import ThreadPoolExecutor
+
 import numpy as np
 
 GAMMA = np.uint64(0x9E3779B97F4A7C15)
@@ -114,14 +117,16 @@ def round_fp32_to_bf16(x32: np.ndarray) -> np.ndarray:
 
 
 def draw_tensor(seed: int, t: int, numel: int, init_std: float, dtype: str,
-                chunk: int = 1 << 22) -> np.ndarray:
+                chunk: int = 1 << 18) -> np.ndarray:
     """Values of tensor t as float32 (already rounded to the storage precision)."""
     K = (float(np.float32(init_std)) * SQRT3) / 65536.0
     with np.errstate(over="ignore"):
         base = mix64(np.uint64(seed) + GAMMA * np.uint64(t + 1))
     out = np.empty(numel, dtype=np.float32)
     mask = np.uint64(0xFFFF)
-    for lo in range(0, numel, chunk):
+
+    def fill(lo: int) -> None:
+        # elements lo..hi-1; independent of every other range
         hi = min(numel, lo + chunk)
         e1 = np.arange(lo + 1, hi + 1, dtype=np.uint64)
         with np.errstate(over="ignore"):
@@ -130,6 +135,15 @@ def draw_tensor(seed: int, t: int, numel: int, init_std: float, dtype: str,
              + ((z >> np.uint64(32)) & mask) + (z >> np.uint64(48)))
         w64 = (s.astype(np.int64) - 131070).astype(np.float64) * K
         out[lo:hi] = w64.astype(np.float32)
+
+    starts = range(0, numel, chunk)
+    if len(starts) > 1:
+        # NumPy releases the GIL inside these array operations
+        with ThreadPoolExecutor(max_workers=min(len(starts), os.cpu_count() or 1)) as ex:
+            list(ex.map(fill, starts))
+    else:
+        for lo in starts:
+            fill(lo)
     if dtype == "bf16":
         out = round_fp32_to_bf16(out)
     return out

@@ -398,3 +398,21 @@ def test_token_decoder_against_library_composition(orc):
     ref = F.linear(torch.tensor(h[-1]), torch.tensor(w["head"])).numpy()
     got = orc.token_decoder_logits(oracle.converter(a, w["converter1"], cfg.C1), toks)
     np.testing.assert_allclose(got, ref, rtol=1e-10, atol=1e-11)
+
+
+def test_prefill_after_prefix_equals_full_prefill(orc):
+    # shared-prefix prefill continues the prefix's caches; it must equal the
+    # from-scratch prefill of the concatenated prompt
+    p = _tiny_prompt(T=48, seed=21)[0]
+    q = _tiny_prompt(T=32, seed=22)[0]
+    pre = orc.prefill(p, "hier")
+    a = orc.prefill_after(pre, q, "hier")
+    b = orc.prefill(np.concatenate([p, q]), "hier")
+    assert (a.N, a.N1) == (b.N, b.N1)
+    np.testing.assert_allclose(a.o, b.o, rtol=1e-12, atol=1e-12)
+    for x, y in zip(a.top + a.l1, b.top + b.l1):
+        np.testing.assert_allclose(x.k, y.k, rtol=1e-12, atol=1e-12)
+        np.testing.assert_allclose(x.v, y.v, rtol=1e-12, atol=1e-12)
+    r = orc.prefill_after(pre, q, "rec")
+    assert r.l1 is None and r.N1 == 0
+    assert pre.N == 3 and pre.top[0].k.shape[0] == 3      # the prefix itself is untouched
