@@ -9,6 +9,7 @@
 #include "common.cuh"
 #include "epilogue.cuh"
 #include "kernels.h"
+#include "launch.cuh"
 
 namespace photon {
 
@@ -16,6 +17,8 @@ template <typename T>
 __global__ void __launch_bounds__(256) k_gemm_simt(const T* __restrict__ A, long long lda,
                                                    const T* __restrict__ W, long long ldw, int M,
                                                    int N, int K, Epilogue ep) {
+  pdl_wait();
+  pdl_trigger();
   __shared__ float As[16][64 + 1];
   __shared__ float Ws[16][64 + 1];
   const int m0 = blockIdx.y * 64, n0 = blockIdx.x * 64;
@@ -77,15 +80,11 @@ void launch_gemm_simt(int dt, const GemmArgs& a, cudaStream_t s) {
   dim3 grid((a.N + 63) / 64, (a.M + 63) / 64);
   if (dt == DT_F32)
     {
-      k_gemm_simt<float><<<grid, 256, 0, s>>>((const float*)a.A, a.lda, (const float*)a.W, a.ldw,
-                                              a.M, a.N, a.K, a.ep);
-      note_launch();
+      launch_kernel(k_gemm_simt<float>, grid, 256, 0, s, (const float*)a.A, a.lda, (const float*)a.W, a.ldw, a.M, a.N, a.K, a.ep);
     }
   else
     {
-      k_gemm_simt<bf16><<<grid, 256, 0, s>>>((const bf16*)a.A, a.lda, (const bf16*)a.W, a.ldw, a.M,
-                                             a.N, a.K, a.ep);
-      note_launch();
+      launch_kernel(k_gemm_simt<bf16>, grid, 256, 0, s, (const bf16*)a.A, a.lda, (const bf16*)a.W, a.ldw, a.M, a.N, a.K, a.ep);
     }
 }
 

@@ -17,11 +17,13 @@
 // fixed order and applies the epilogue, so results are deterministic.
 #include <cuda.h>
 
+#include <cstdlib>
 #include <mutex>
 
 #include "common.cuh"
 #include "epilogue.cuh"
 #include "kernels.h"
+#include "launch.cuh"
 #include "ptx_sm100.cuh"
 
 namespace photon {
@@ -92,10 +94,31 @@ __global__ void __launch_bounds__(128, 1)
   __syncthreads();
   ptx::tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  // Everything above touched only shared/tensor memory and the kernel's
+  // own parameters.  Activations are read and outputs written only after the
+  // previous kernel in the stream has completed (pdl_wait).  The weight
+  // operand is never written by any kernel, so the producer fetches the
+  // weight tiles of the first ring stages before waiting: with programmatic
+  // dependent launch that streaming overlaps the previous kernel's tail.
+  if (threadIdx.x != 0) pdl_wait();
+  pdl_trigger();
 
   if (threadIdx.x == 0) {
     // ---- TMA producer
-    for (int it = 0; it < nk; ++it) {
+    const CUtensorMap* tm_w = SWAP ? &tmA : &tmB;   // weights
+    const CUtensorMap* tm_x = SWAP ? &tmB : &tmA;   // activations
+    const int w_row = SWAP ? a0 : b0, x_row = SWAP ? b0 : a0;
+    auto w_tile = [&](int st) { return SWAP ? a_tile(st) : b_tile(st); };
+    auto x_tile = [&](int st) { return SWAP ? b_tile(st) : a_tile(st); };
+    const int pre = nk < STAGES ? nk : STAGES;
+    for (int it = 0; it < pre; ++it) {  // fresh ring: no slot to wait for
+      ptx::mbar_arrive_expect_tx(full_bar(it), (uint32_t)Cfg::kStageBytes);
+      ptx::tma_load_2d(w_tile(it), tm_w, (kb0 + it) * kBK, w_row, full_bar(it));
+    }
+    pdl_wait();
+    for (int it = 0; it < pre; ++it)
+      ptx::tma_load_2d(x_tile(it), tm_x, (kb0 + it) * kBK, x_row, full_bar(it));
+    for (int it = pre; it < nk; ++it) {
       const int s = it % STAGES;
       const uint32_t ph = (uint32_t)(it / STAGES) & 1u;
       if (!ptx::mbar_wait(empty_bar(s), ph ^ 1u, abort_flag)) {
@@ -130,7 +153,7 @@ __global__ void __launch_bounds__(128, 1)
   }
   __syncwarp();
 
-  // ---- epilogue: TMEM -> shared staging tile (output-row-major)
+  // ---- epilogue
   if (!ptx::mbar_wait(done_bar, 0, abort_flag)) {
     report_error(err, DEV_WAIT_TIMEOUT_EPILOGUE);
     *abort_flag = 1;
@@ -139,53 +162,124 @@ __global__ void __launch_bounds__(128, 1)
   const bool ok = (*abort_flag == 0);  // CTA-uniform: the TMEM loads below need whole warps
   ptx::tc_fence_after();
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-  float* tile = reinterpret_cast<float*>(smem);
-  constexpr int R = SWAP ? BN : kBM;     // output rows in the tile (tokens)
-  constexpr int CC = SWAP ? kBM : BN;    // output columns in the tile (features)
-  constexpr int LD = CC + 1;
-  if (ok) {
-    const int tl = warp * 32 + lane;     // this thread's TMEM lane
+  const int tl = warp * 32 + lane;     // this thread's TMEM lane
+  const uint32_t trow = tmem + ((uint32_t)(warp * 32) << 16);
+  const long long plane = (long long)M * N;
+  const bool staged = SWAP && ep.kind == EPI_QKV && part == nullptr;
+  if (ok && nk > 0 && !staged) {
+    if (!SWAP) {
+      // thread = output row; 64 columns at a time (a whole RoPE head)
+      const long long grow = a0 + tl;
+      unsigned long long best = 0ull;
+#pragma unroll 1
+      for (int j0 = 0; j0 < BN; j0 += 64) {
+        float lo[32], hi[32];
+        ptx::tmem_ld32(trow + (uint32_t)j0, lo);
+        ptx::tmem_ld32(trow + (uint32_t)(j0 + 32), hi);
+        const int gc = b0 + j0;
+        if (grow >= M || gc >= N) continue;
+        if (part) {
+          float4* p = reinterpret_cast<float4*>(part + (long long)z * plane + grow * N + gc);
+#pragma unroll
+          for (int i = 0; i < 8; ++i) p[i] = make_float4(lo[4 * i], lo[4 * i + 1], lo[4 * i + 2], lo[4 * i + 3]);
+#pragma unroll
+          for (int i = 0; i < 8; ++i) p[8 + i] = make_float4(hi[4 * i], hi[4 * i + 1], hi[4 * i + 2], hi[4 * i + 3]);
+        } else if (ep.kind == EPI_ARGMAX) {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            best = max(best, argmax_key(lo[i], gc + i));
+            best = max(best, argmax_key(hi[i], gc + 32 + i));
+          }
+          if (ep.out) {
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+              reinterpret_cast<float*>(ep.out)[grow * ep.ldo + gc + i] = lo[i];
+              reinterpret_cast<float*>(ep.out)[grow * ep.ldo + gc + 32 + i] = hi[i];
+            }
+          }
+        } else {
+          epi_row64(ep, grow, gc, lo, hi);
+        }
+      }
+      if (ep.kind == EPI_ARGMAX && !part && grow < M)
+        ep.argmax_part[grow * ep.argmax_tiles + blockIdx.y] = best;
+    } else {
+      // thread = output column (feature); 32 tokens at a time, stores
+      // coalesced across the warp for each token
+      const int gf = a0 + tl;
+      __shared__ unsigned long long red[4][BN];
+#pragma unroll 1
+      for (int j0 = 0; j0 < BN; j0 += 32) {
+        float v[32];
+        ptx::tmem_ld32(trow + (uint32_t)j0, v);
+        if (ep.kind == EPI_ARGMAX && !part) {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            unsigned long long k = gf < N ? argmax_key(v[i], gf) : 0ull;
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) k = max(k, __shfl_xor_sync(0xffffffffu, k, o));
+            if (lane == 0) red[warp][j0 + i] = k;
+          }
+        }
+        if (gf < N) {
+          if (part) {
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+              const long long t = b0 + j0 + i;
+              if (t < M) part[(long long)z * plane + t * N + gf] = v[i];
+            }
+          } else if (ep.kind == EPI_ARGMAX) {
+            if (ep.out) {
+#pragma unroll
+              for (int i = 0; i < 32; ++i) {
+                const long long t = b0 + j0 + i;
+                if (t < M) reinterpret_cast<float*>(ep.out)[t * ep.ldo + gf] = v[i];
+              }
+            }
+          } else {
+            epi_col32(ep, b0 + j0, M, gf, v);
+          }
+        }
+      }
+      if (ep.kind == EPI_ARGMAX && !part) {
+        __syncthreads();
+        for (int j = threadIdx.x; j < BN; j += 128) {
+          const long long t = b0 + j;
+          if (t < M)
+            ep.argmax_part[t * ep.argmax_tiles + blockIdx.x] =
+                max(max(red[0][j], red[1][j]), max(red[2][j], red[3][j]));
+        }
+      }
+    }
+  }
+  if (ok && nk > 0 && staged) {
+    // swapped QKV: the RoPE partner of feature f (f + 32) sits in another
+    // warp's TMEM lanes, so the tile goes through shared memory first
+    float* tile = reinterpret_cast<float*>(smem);
+    constexpr int LD = kBM + 1;
 #pragma unroll 1
     for (int j0 = 0; j0 < BN; j0 += 32) {
       float v[32];
-      ptx::tmem_ld32(tmem + ((uint32_t)(warp * 32) << 16) + (uint32_t)j0, v);
+      ptx::tmem_ld32(trow + (uint32_t)j0, v);
 #pragma unroll
-      for (int i = 0; i < 32; ++i) {
-        if (SWAP)
-          tile[(j0 + i) * LD + tl] = v[i];
-        else
-          tile[tl * LD + j0 + i] = v[i];
+      for (int i = 0; i < 32; ++i) tile[(j0 + i) * LD + tl] = v[i];
+    }
+    __syncthreads();
+#pragma unroll 4
+    for (int r = warp; r < BN; r += 4) {
+      const long long grow = b0 + r;
+      if (grow >= M) break;
+#pragma unroll
+      for (int seg = 0; seg < kBM / 64; ++seg) {
+        if (a0 + seg * 64 >= N) break;  // N is a multiple of 64
+        const int c0 = seg * 64 + lane;
+        epi_pair<bf16>(ep, grow, a0 + c0, tile[r * LD + c0], a0 + c0 + 32, tile[r * LD + c0 + 32]);
       }
     }
   }
   ptx::tc_fence_before();
   __syncthreads();
   if (warp == 0) ptx::tmem_dealloc(tmem, Cfg::kTmemCols);
-  if (!ok || nk <= 0) return;
-
-  const int row_base = SWAP ? b0 : a0;
-  const int col_base = SWAP ? a0 : b0;
-  const long long plane = (long long)M * N;
-#pragma unroll 1
-  for (int r = warp; r < R; r += 4) {
-    const long long grow = row_base + r;
-    if (grow >= M) break;
-#pragma unroll 1
-    for (int seg = 0; seg < CC / 64; ++seg) {
-      if (col_base + seg * 64 >= N) break;  // N is a multiple of 64
-      const int c0 = seg * 64 + lane;
-      const int gc0 = col_base + c0;
-      const float v0 = tile[r * LD + c0];
-      const float v1 = tile[r * LD + c0 + 32];
-      if (part) {
-        float* p = part + (long long)z * plane + grow * N + gc0;
-        p[0] = v0;
-        p[32] = v1;
-      } else {
-        epi_pair<bf16>(ep, grow, gc0, v0, gc0 + 32, v1);
-      }
-    }
-  }
 }
 
 // ------------------------------------------------------------------ host side
@@ -235,9 +329,7 @@ void run_tc(const CUtensorMap& ma, const CUtensorMap& mb, int grid_a, int grid_b
     configured = true;
   }
   dim3 grid(grid_a, grid_b, splits);
-  k_gemm_tc<BN, STAGES, SWAP><<<grid, 128, Cfg::kSmemBytes, s>>>(ma, mb, M, N, nkb, kbs, ep, part,
-                                                                 err);
-  note_launch();
+  launch_kernel(k_gemm_tc<BN, STAGES, SWAP>, grid, 128, Cfg::kSmemBytes, s, ma, mb, M, N, nkb, kbs, ep, part, err);
 }
 
 struct Plan {
@@ -245,28 +337,36 @@ struct Plan {
   int bn;
   int splits;
   int kbs;
+  int ga, gb;
 };
 
-Plan plan_for(int M, int N, int K, int force_splits, int force_swap) {
+Plan plan_for(int M, int N, int K, int force_splits, int force_swap, bool argmax) {
   Plan p;
   const int nkb = K / kBK;
   p.swap = force_swap >= 0 ? (force_swap != 0) : (M <= 256);
   if (p.swap)
-    p.bn = M <= 64 ? 64 : (M <= 128 ? 128 : 256);
+    p.bn = 64;  // token tiles of 64: M = 256 gives 4 CTAs per 128-feature tile
   else
     p.bn = (N % 256 == 0 && M >= 4096) ? 256 : 128;
   const int ga = p.swap ? (N + kBM - 1) / kBM : (M + kBM - 1) / kBM;
-  const int gb = p.swap ? 1 : (N + p.bn - 1) / p.bn;
+  const int gb = p.swap ? (M + p.bn - 1) / p.bn : (N + p.bn - 1) / p.bn;
   const int tiles = ga * gb;
+  // Split K only to bound the K run of one CTA (1024) when the tile grid
+  // alone leaves SMs idle; the fp32 partial tiles cost M*N*8 bytes per split.
   int splits = 1;
   if (force_splits > 0)
     splits = force_splits;
-  else if (tiles < 148)
-    splits = (148 + tiles - 1) / tiles;
+  else if (tiles < 148 && !argmax) {
+    splits = (nkb + 15) / 16;
+    const int cap = (2 * 148 + tiles - 1) / tiles;
+    if (splits > cap) splits = cap;
+  }
   if (splits > nkb) splits = nkb;
   if (splits < 1) splits = 1;
   p.kbs = (nkb + splits - 1) / splits;
   p.splits = (nkb + p.kbs - 1) / p.kbs;  // no empty split
+  p.ga = ga;
+  p.gb = gb;
   return p;
 }
 
@@ -274,8 +374,14 @@ Plan plan_for(int M, int N, int K, int force_splits, int force_swap) {
 
 bool tma_available() { return encode_fn() != nullptr; }
 
+int gemm_tc_argmax_tiles(int M, int N, int K) {
+  if (M <= 0 || N <= 0 || K <= 0 || K % kBK || N % 64) return 0;
+  const Plan p = plan_for(M, N, K, 1, -1, true);
+  return p.swap ? p.ga : p.gb;
+}
+
 size_t gemm_tc_workspace_bytes(int M, int N, int K) {
-  const Plan p = plan_for(M, N, K, 0, -1);
+  const Plan p = plan_for(M, N, K, 0, -1, false);
   return p.splits > 1 ? (size_t)p.splits * M * N * sizeof(float) : 0;
 }
 
@@ -287,7 +393,9 @@ bool launch_gemm_tc(const GemmArgs& a, const GemmWorkspace& ws, int* err, cudaSt
   if (a.ep.kind == EPI_QKV && a.ep.dh != 64) return false;
   if ((a.lda * 2) % 16 || (a.ldw * 2) % 16) return false;
   if (reinterpret_cast<uintptr_t>(a.A) % 16 || reinterpret_cast<uintptr_t>(a.W) % 16) return false;
-  const Plan p = plan_for(M, N, K, force_splits, force_swap);
+  const bool argmax = a.ep.kind == EPI_ARGMAX;
+  const Plan p = plan_for(M, N, K, argmax ? 1 : force_splits, force_swap, argmax);
+  if (argmax && p.splits != 1) return false;
   float* part = nullptr;
   if (p.splits > 1) {
     const size_t need = (size_t)p.splits * M * N * sizeof(float);
@@ -298,20 +406,18 @@ bool launch_gemm_tc(const GemmArgs& a, const GemmWorkspace& ws, int* err, cudaSt
   const int nkb = K / kBK;
   if (p.swap) {
     if (!make_map(&ma, a.W, N, K, a.ldw, kBM) || !make_map(&mb, a.A, M, K, a.lda, p.bn)) return false;
-    const int ga = (N + kBM - 1) / kBM;
     if (p.bn == 64)
-      run_tc<64, 6, true>(ma, mb, ga, 1, p.splits, M, N, nkb, p.kbs, a.ep, part, err, s);
+      run_tc<64, 4, true>(ma, mb, p.ga, p.gb, p.splits, M, N, nkb, p.kbs, a.ep, part, err, s);
     else if (p.bn == 128)
-      run_tc<128, 4, true>(ma, mb, ga, 1, p.splits, M, N, nkb, p.kbs, a.ep, part, err, s);
+      run_tc<128, 4, true>(ma, mb, p.ga, p.gb, p.splits, M, N, nkb, p.kbs, a.ep, part, err, s);
     else
-      run_tc<256, 4, true>(ma, mb, ga, 1, p.splits, M, N, nkb, p.kbs, a.ep, part, err, s);
+      run_tc<256, 4, true>(ma, mb, p.ga, p.gb, p.splits, M, N, nkb, p.kbs, a.ep, part, err, s);
   } else {
     if (!make_map(&ma, a.A, M, K, a.lda, kBM) || !make_map(&mb, a.W, N, K, a.ldw, p.bn)) return false;
-    const int ga = (M + kBM - 1) / kBM, gb = (N + p.bn - 1) / p.bn;
     if (p.bn == 256)
-      run_tc<256, 4, false>(ma, mb, ga, gb, p.splits, M, N, nkb, p.kbs, a.ep, part, err, s);
+      run_tc<256, 4, false>(ma, mb, p.ga, p.gb, p.splits, M, N, nkb, p.kbs, a.ep, part, err, s);
     else
-      run_tc<128, 4, false>(ma, mb, ga, gb, p.splits, M, N, nkb, p.kbs, a.ep, part, err, s);
+      run_tc<128, 4, false>(ma, mb, p.ga, p.gb, p.splits, M, N, nkb, p.kbs, a.ep, part, err, s);
   }
   if (p.splits > 1) launch_splitk_reduce(DT_BF16, part, p.splits, M, N, a.ep, s);
   return true;

@@ -1,16 +1,27 @@
 // Weight generation, embeddings, RMSNorm, greedy argmax and the split-K
 // reduction.  All memory-bound row kernels.
 #include <atomic>
+#include <cstdlib>
 
 #include "common.cuh"
 #include "epilogue.cuh"
 #include "kernels.h"
+#include "launch.cuh"
 
 namespace photon {
 
 static std::atomic<unsigned long long> g_launches{0};
 void note_launch(int n) { g_launches.fetch_add((unsigned long long)n, std::memory_order_relaxed); }
 unsigned long long launch_total() { return g_launches.load(std::memory_order_relaxed); }
+
+// Programmatic dependent launch is on unless PHOTON_PDL=0.
+bool pdl_enabled() {
+  static const bool on = [] {
+    const char* e = getenv("PHOTON_PDL");
+    return !(e && e[0] == '0');
+  }();
+  return on;
+}
 
 // ------------------------------------------------------------------ weights
 // Counter-based draw, defined independently of any other implementation:
@@ -38,6 +49,8 @@ constexpr uint64_t kGamma = 0x9E3779B97F4A7C15ull;
 
 template <typename T>
 __global__ void k_init_normal(T* __restrict__ dst, long long n, uint64_t base, double K) {
+  pdl_wait();
+  pdl_trigger();
   for (long long e = blockIdx.x * (long long)blockDim.x + threadIdx.x; e < n;
        e += (long long)gridDim.x * blockDim.x) {
     const uint64_t z = splitmix_mix(base + kGamma * (uint64_t)(e + 1));
@@ -57,17 +70,17 @@ void launch_init_normal(int dt, void* dst, long long numel, uint64_t seed, int t
   if (blocks < 1) blocks = 1;
   if (dt == DT_F32)
     {
-      k_init_normal<float><<<(int)blocks, threads, 0, s>>>((float*)dst, numel, base, K);
-      note_launch();
+      launch_kernel(k_init_normal<float>, (int)blocks, threads, 0, s, (float*)dst, numel, base, K);
     }
   else
     {
-      k_init_normal<bf16><<<(int)blocks, threads, 0, s>>>((bf16*)dst, numel, base, K);
-      note_launch();
+      launch_kernel(k_init_normal<bf16>, (int)blocks, threads, 0, s, (bf16*)dst, numel, base, K);
     }
 }
 
 __global__ void k_fill_f32(float* dst, long long n, float v) {
+  pdl_wait();
+  pdl_trigger();
   for (long long e = blockIdx.x * (long long)blockDim.x + threadIdx.x; e < n;
        e += (long long)gridDim.x * blockDim.x)
     dst[e] = v;
@@ -76,12 +89,13 @@ void launch_fill_f32(float* dst, long long n, float v, cudaStream_t s) {
   long long blocks = (n + 255) / 256;
   if (blocks > 148 * 16) blocks = 148 * 16;
   if (blocks < 1) blocks = 1;
-  k_fill_f32<<<(int)blocks, 256, 0, s>>>(dst, n, v);
-  note_launch();
+  launch_kernel(k_fill_f32, (int)blocks, 256, 0, s, dst, n, v);
 }
 
 template <typename T>
 __global__ void k_to_f32(const T* src, float* dst, long long n) {
+  pdl_wait();
+  pdl_trigger();
   for (long long e = blockIdx.x * (long long)blockDim.x + threadIdx.x; e < n;
        e += (long long)gridDim.x * blockDim.x)
     dst[e] = ld_f(src + e);
@@ -92,13 +106,11 @@ void launch_to_f32(int dt, const void* src, float* dst, long long n, cudaStream_
   if (blocks < 1) blocks = 1;
   if (dt == DT_F32)
     {
-      k_to_f32<float><<<(int)blocks, 256, 0, s>>>((const float*)src, dst, n);
-      note_launch();
+      launch_kernel(k_to_f32<float>, (int)blocks, 256, 0, s, (const float*)src, dst, n);
     }
   else
     {
-      k_to_f32<bf16><<<(int)blocks, 256, 0, s>>>((const bf16*)src, dst, n);
-      note_launch();
+      launch_kernel(k_to_f32<bf16>, (int)blocks, 256, 0, s, (const bf16*)src, dst, n);
     }
 }
 
@@ -107,6 +119,8 @@ void launch_to_f32(int dt, const void* src, float* dst, long long n, cudaStream_
 template <typename T>
 __global__ void k_embed(const int32_t* __restrict__ ids, const T* __restrict__ E, T* __restrict__ out,
                         int rows, int d, int vocab, int* err) {
+  pdl_wait();
+  pdl_trigger();
   const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
   if (warp >= rows) return;
@@ -127,19 +141,19 @@ void launch_embed(int dt, const int32_t* ids, const void* E, void* out, int rows
   const int blocks = (rows * 32 + threads - 1) / threads;
   if (dt == DT_F32)
     {
-      k_embed<float><<<blocks, threads, 0, s>>>(ids, (const float*)E, (float*)out, rows, d, vocab, err);
-      note_launch();
+      launch_kernel(k_embed<float>, blocks, threads, 0, s, ids, (const float*)E, (float*)out, rows, d, vocab, err);
     }
   else
     {
-      k_embed<bf16><<<blocks, threads, 0, s>>>(ids, (const bf16*)E, (bf16*)out, rows, d, vocab, err);
-      note_launch();
+      launch_kernel(k_embed<bf16>, blocks, threads, 0, s, ids, (const bf16*)E, (bf16*)out, rows, d, vocab, err);
     }
 }
 
 template <typename T>
 __global__ void k_embed_f32(const int32_t* __restrict__ ids, const T* __restrict__ E,
                             float* __restrict__ x, int rows, int d, int vocab, int* err) {
+  pdl_wait();
+  pdl_trigger();
   const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
   if (warp >= rows) return;
@@ -159,13 +173,11 @@ void launch_embed_f32(int dt, const int32_t* ids, const void* E, float* x, int r
   const int blocks = (rows * 32 + threads - 1) / threads;
   if (dt == DT_F32)
     {
-      k_embed_f32<float><<<blocks, threads, 0, s>>>(ids, (const float*)E, x, rows, d, vocab, err);
-      note_launch();
+      launch_kernel(k_embed_f32<float>, blocks, threads, 0, s, ids, (const float*)E, x, rows, d, vocab, err);
     }
   else
     {
-      k_embed_f32<bf16><<<blocks, threads, 0, s>>>(ids, (const bf16*)E, x, rows, d, vocab, err);
-      note_launch();
+      launch_kernel(k_embed_f32<bf16>, blocks, threads, 0, s, ids, (const bf16*)E, x, rows, d, vocab, err);
     }
 }
 
@@ -174,6 +186,8 @@ void launch_embed_f32(int dt, const int32_t* ids, const void* E, float* x, int r
 template <typename T>
 __global__ void k_rmsnorm(const float* __restrict__ x, const float* __restrict__ g,
                           T* __restrict__ out, int rows, int d, int in_step, int in_off, float eps) {
+  pdl_wait();
+  pdl_trigger();
   const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
   if (warp >= rows) return;
@@ -202,13 +216,11 @@ void launch_rmsnorm(int dt, const float* x, const float* g, void* out, int rows,
   const int blocks = (rows * 32 + threads - 1) / threads;
   if (dt == DT_F32)
     {
-      k_rmsnorm<float><<<blocks, threads, 0, s>>>(x, g, (float*)out, rows, d, in_step, in_off, eps);
-      note_launch();
+      launch_kernel(k_rmsnorm<float>, blocks, threads, 0, s, x, g, (float*)out, rows, d, in_step, in_off, eps);
     }
   else
     {
-      k_rmsnorm<bf16><<<blocks, threads, 0, s>>>(x, g, (bf16*)out, rows, d, in_step, in_off, eps);
-      note_launch();
+      launch_kernel(k_rmsnorm<bf16>, blocks, threads, 0, s, x, g, (bf16*)out, rows, d, in_step, in_off, eps);
     }
 }
 
@@ -222,6 +234,8 @@ __device__ __forceinline__ void better(float& bv, int& bi, float v, int i) {
 __global__ void k_argmax(const float* __restrict__ logits, long long ld, int rows, int V, int step,
                          int C1, const int32_t* __restrict__ force, int32_t* own, int32_t* used,
                          int32_t* next_ids, int* err) {
+  pdl_wait();
+  pdl_trigger();
   const int row = blockIdx.x;
   if (row >= rows) return;
   const float* lr = logits + (long long)row * ld;
@@ -264,8 +278,57 @@ void launch_argmax(const float* logits, long long ld, int rows, int V, int i, in
                    const int32_t* force, int32_t* own, int32_t* used, int32_t* next_ids, int* err,
                    cudaStream_t s) {
   if (rows <= 0) return;
-  k_argmax<<<rows, 256, 0, s>>>(logits, ld, rows, V, i, C1, force, own, used, next_ids, err);
-  note_launch();
+  launch_kernel(k_argmax, rows, 256, 0, s, logits, ld, rows, V, i, C1, force, own, used, next_ids, err);
+}
+
+// One warp per row: max over the row's tile partials, then the same token
+// bookkeeping as k_argmax.
+__global__ void k_argmax_partials(const unsigned long long* __restrict__ part, int tiles, int rows,
+                                  int V, int step, int C1, const int32_t* __restrict__ force,
+                                  int32_t* own, int32_t* used, int32_t* next_ids, int* err) {
+  pdl_wait();
+  pdl_trigger();
+  const int row = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  if (row >= rows) return;
+  unsigned long long k = 0ull;
+  for (int t = lane; t < tiles; t += 32) k = max(k, part[(long long)row * tiles + t]);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) k = max(k, __shfl_xor_sync(0xffffffffu, k, o));
+  if (lane == 0) {
+    int bi = (int)(0xFFFFFFFFu - (uint32_t)(k & 0xFFFFFFFFull));
+    if (k == 0ull || bi < 0 || bi >= V) {
+      report_error(err, DEV_BAD_TOKEN);
+      bi = 0;
+    }
+    const long long slot = (long long)row * C1 + step;
+    int u = bi;
+    if (force) {
+      const int f = force[slot];
+      if (f >= 0) u = (f < V) ? f : 0;
+      if (f >= V) report_error(err, DEV_BAD_TOKEN);
+    }
+    if (own) own[slot] = bi;
+    if (used) used[slot] = u;
+    if (next_ids) next_ids[row] = u;
+  }
+}
+void launch_argmax_partials(const unsigned long long* part, int tiles, int rows, int V, int i,
+                            int C1, const int32_t* force, int32_t* own, int32_t* used,
+                            int32_t* next_ids, int* err, cudaStream_t s) {
+  if (rows <= 0) return;
+  launch_kernel(k_argmax_partials, (rows * 32 + 255) / 256, 256, 0, s, part, tiles, rows, V, i, C1,
+                force, own, used, next_ids, err);
+}
+
+__global__ void k_advance(int* pos, int dN, int dN1) {
+  pdl_wait();
+  pdl_trigger();
+  pos[0] += dN;
+  pos[1] += dN1;
+}
+void launch_advance(int* pos, int dN, int dN1, cudaStream_t s) {
+  launch_kernel(k_advance, 1, 1, 0, s, pos, dN, dN1);
 }
 
 // ------------------------------------------------------------------ split-K reduce
@@ -275,6 +338,8 @@ void launch_argmax(const float* logits, long long ld, int rows, int V, int i, in
 template <typename T>
 __global__ void k_splitk_reduce(const float* __restrict__ part, int splits, int M, int N,
                                 Epilogue ep) {
+  pdl_wait();
+  pdl_trigger();
   const long long t = blockIdx.x * (long long)blockDim.x + threadIdx.x;
   const int segs = N >> 6;
   const long long total = (long long)M * segs * 32;
@@ -299,13 +364,11 @@ void launch_splitk_reduce(int dt, const float* part, int splits, int M, int N, c
   const long long blocks = (total + threads - 1) / threads;
   if (dt == DT_F32)
     {
-      k_splitk_reduce<float><<<(int)blocks, threads, 0, s>>>(part, splits, M, N, ep);
-      note_launch();
+      launch_kernel(k_splitk_reduce<float>, (int)blocks, threads, 0, s, part, splits, M, N, ep);
     }
   else
     {
-      k_splitk_reduce<bf16><<<(int)blocks, threads, 0, s>>>(part, splits, M, N, ep);
-      note_launch();
+      launch_kernel(k_splitk_reduce<bf16>, (int)blocks, threads, 0, s, part, splits, M, N, ep);
     }
 }
 

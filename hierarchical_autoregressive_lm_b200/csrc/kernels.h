@@ -17,6 +17,7 @@ enum EpiKind : int {
   EPI_ADD_F32 = 2,    // out[row, col] += acc (fp32 residual stream)
   EPI_GELU_T = 3,     // out[row, col] = T(gelu(acc))
   EPI_QKV = 4,        // fused q/k/v split + RoPE + KV-cache write (see below)
+  EPI_ARGMAX = 5,     // LM head: per-tile greedy partials (+ optional fp32 logits)
 };
 
 // Epilogue parameters.  For EPI_QKV the GEMM output has 3*d columns
@@ -34,6 +35,14 @@ struct Epilogue {
   void* v_cache = nullptr;
   int d = 0, H = 0, dh = 0, cap = 0, q_len = 1, p0 = 0, kv_off = 0;
   const float2* rope = nullptr;
+  // If set, the position of a group's first row is *p0_dev + p0 (read on the
+  // device, so a captured decode step can be replayed at later positions).
+  const int* p0_dev = nullptr;
+  // EPI_ARGMAX: argmax_part[row * argmax_tiles + tile] receives the packed
+  // (value, lowest index) maximum of the row over the tile's columns; `out`
+  // (if set) receives the fp32 logits.
+  unsigned long long* argmax_part = nullptr;
+  int argmax_tiles = 0;
 };
 
 // C = A[M, K] * W[N, K]^T with A, W of the storage type, fp32 accumulation.
@@ -72,6 +81,12 @@ struct AttnArgs {
   void* O = nullptr;
   long long o_ld = 0;
   float scale = 1.0f;
+  // If set, the first query's position is *p0_dev + p0 (read on the device).
+  const int* p0_dev = nullptr;
+  // Largest key count the launch must cover (0: p0 + q_len).  The key
+  // chunking is planned for this count; chunks past the live keys write
+  // empty partials.
+  int n_plan = 0;
 };
 
 // ---- weights -----------------------------------------------------------
@@ -96,6 +111,13 @@ void launch_rmsnorm(int dt, const float* x, const float* g, void* out, int rows,
 void launch_argmax(const float* logits, long long ld, int rows, int V, int i, int C1,
                    const int32_t* force, int32_t* own, int32_t* used, int32_t* next_ids, int* err,
                    cudaStream_t s);
+// Greedy token per row from the head GEMM's per-tile partials (EPI_ARGMAX);
+// same outputs as launch_argmax.
+void launch_argmax_partials(const unsigned long long* part, int tiles, int rows, int V, int i,
+                            int C1, const int32_t* force, int32_t* own, int32_t* used,
+                            int32_t* next_ids, int* err, cudaStream_t s);
+// pos[0] += dN; pos[1] += dN1 (device-side decode positions).
+void launch_advance(int* pos, int dN, int dN1, cudaStream_t s);
 
 // ---- GEMM ----------------------------------------------------------------
 void launch_gemm(int dt, const GemmArgs& a, const GemmWorkspace& ws, int* err, cudaStream_t s);
@@ -104,18 +126,24 @@ void launch_gemm_simt(int dt, const GemmArgs& a, cudaStream_t s);
 bool launch_gemm_tc(const GemmArgs& a, const GemmWorkspace& ws, int* err, cudaStream_t s,
                     int force_splits = 0, int force_swap = -1);
 size_t gemm_tc_workspace_bytes(int M, int N, int K);
+// Column tiles of the tcgen05 plan for an EPI_ARGMAX GEMM (0: not supported).
+int gemm_tc_argmax_tiles(int M, int N, int K);
 void launch_splitk_reduce(int dt, const float* part, int splits, int M, int N, const Epilogue& ep,
                           cudaStream_t s);
 
 // ---- attention ------------------------------------------------------------
-// Split-K decode attention (q_len <= 8).  `part` is fp32 scratch for the
-// split partials; attn_decode_workspace_bytes gives its size.
-size_t attn_decode_workspace_bytes(const AttnArgs& a);
+// Decode attention (q_len <= 4).  `part` is fp32 scratch for the partials of
+// (group, head) pairs whose keys are split across CTAs;
+// attn_decode_workspace_bytes gives its size (0 when nothing is split).
+size_t attn_decode_workspace_bytes(int dt, const AttnArgs& a);
 // Returns false (nothing launched) for unsupported shapes or too little scratch.
 bool launch_attn_decode(int dt, const AttnArgs& a, float* part, size_t part_bytes, int* err,
                         cudaStream_t s);
 // Causal attention for many new queries per group (prefill).
 void launch_attn_prefill(int dt, const AttnArgs& a, cudaStream_t s);
+
+// ---- error message of the calling thread (read by photon_last_error) ----
+void set_error_message(const char* msg);
 
 // ---- launch accounting ------------------------------------------------------
 // Process-wide count of kernels this library has launched.

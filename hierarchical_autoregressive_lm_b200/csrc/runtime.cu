@@ -9,6 +9,7 @@
 // attention confined to the chunk).
 #include <cmath>
 #include <cstdarg>
+#include <cstdlib>
 #include <cstdio>
 #include <cstring>
 #include <string>
@@ -31,6 +32,10 @@ static int fail(int code, const char* fmt, ...) {
   g_err = buf;
   return code;
 }
+
+namespace photon {
+void set_error_message(const char* msg) { g_err = msg; }
+}  // namespace photon
 
 #define CK(call)                                                                   \
   do {                                                                             \
@@ -242,6 +247,12 @@ struct photon_cache {
   float* attn_ws = nullptr;
   size_t attn_ws_bytes = 0;
   int* d_err = nullptr;
+  int* d_pos = nullptr;          // device copies of {N, N1} read by the decode kernels
+  unsigned long long* amax_part = nullptr;  // [B*C2][amax_cap] head partials
+  int amax_cap = 0;
+  int32_t* tok_out = nullptr;    // [B, C] greedy tokens of the last graph-replayed step
+  cudaGraphExec_t graph[2] = {nullptr, nullptr};  // captured decode step per mode
+  bool graph_failed[2] = {false, false};
   std::vector<void*> allocs;
   size_t kv_bytes = 0, ws_bytes = 0;
   bool has_a_hat = false, has_a = false;
@@ -280,6 +291,8 @@ struct StackRun {
   const char* vp = nullptr;
   size_t pre_layer_bytes = 0;
   int cap_pre = 0, n_pre = 0;
+  const int* p0_dev = nullptr;  // device position of the first row (added to p0)
+  int n_plan = 0;               // key count the decode attention is planned for
 };
 
 static void gemm(photon_model* m, const Bufs& b, const void* A, long long lda, const void* W,
@@ -327,6 +340,7 @@ static void run_block(photon_model* m, const BlockW& w, float* x, const StackRun
   e.p0 = r.p0;
   e.kv_off = r.kv_off;
   e.rope = b.rope;
+  e.p0_dev = r.p0_dev;
   gemm(m, b, b.xn, d, w.wqkv, d, rows, 3 * d, d, e, s);
 
   AttnArgs a;
@@ -349,6 +363,8 @@ static void run_block(photon_model* m, const BlockW& w, float* x, const StackRun
   a.O = b.att;
   a.o_ld = d;
   a.scale = 1.0f / sqrtf((float)m->dh);
+  a.p0_dev = r.p0_dev;
+  a.n_plan = r.n_plan;
   bool done = false;
   if (r.q_len <= 4) done = launch_attn_decode(m->dt, a, b.attn_ws, b.attn_ws_bytes, b.err, s);
   if (!done) launch_attn_prefill(m->dt, a, s);
@@ -376,18 +392,16 @@ static size_t block_ws_need(const photon_model* m, int rows) {
   w = std::max(w, gemm_ws_need(m, rows, m->d, m->f));
   return w;
 }
-static size_t attn_ws_need(int G, int H, int dh, int q_len, int n_max) {
-  size_t w = 0;
+// Scratch of a decode-attention launch planned for n_plan keys per pair.
+static size_t attn_ws_need(int dt, int G, int H, int dh, int q_len, int n_plan) {
   AttnArgs a;
   a.G = G;
   a.H = H;
   a.dh = dh;
   a.q_len = q_len;
-  for (int n = q_len; n <= n_max; ++n) {
-    a.p0 = n - q_len;
-    w = std::max(w, attn_decode_workspace_bytes(a));
-  }
-  return w;
+  a.p0 = n_plan - q_len;
+  a.n_plan = n_plan;
+  return attn_decode_workspace_bytes(dt, a);
 }
 
 // cos/sin table: entry [pos][i] = (cos, sin)(pos * theta^(-2i/dh)), computed in fp64.
@@ -607,6 +621,10 @@ int photon_prefill(photon_model* m, const photon_cache* prefix, const int32_t* d
   c->next_ids = al.get<int32_t>((size_t)rows_g * 4);
   c->used = al.get<int32_t>((size_t)rows_c * 4);
   c->d_err = al.get<int>(16);
+  c->d_pos = al.get<int>(16);
+  c->amax_cap = (m->V + 127) / 128;
+  c->amax_part = al.get<unsigned long long>((size_t)rows_g * c->amax_cap * 8);
+  c->tok_out = al.get<int32_t>((size_t)rows_c * 4);
   size_t gw = 0;
   gw = std::max(gw, block_ws_need(m, B));
   gw = std::max(gw, block_ws_need(m, rows_g));
@@ -618,11 +636,12 @@ int photon_prefill(photon_model* m, const photon_cache* prefix, const int32_t* d
   gw = std::max(gw, gemm_ws_need(m, rows_g, m->V, d));
   c->gemm_ws_bytes = gw;
   c->gemm_ws = al.get<float>(gw);
-  size_t aw = attn_ws_need(B, m->H, m->dh, 1, c->n_pre + c->Ncap);
+  size_t aw = attn_ws_need(m->dt, B, m->H, m->dh, 1, c->n_pre + c->Ncap);
   if (mode == PHOTON_MODE_HIER)
-    aw = std::max(aw, attn_ws_need(B, m->H, m->dh, C2, c->n1_pre + c->N1cap));
-  aw = std::max(aw, attn_ws_need(B, m->H, m->dh, C2, C2));
-  aw = std::max(aw, attn_ws_need(rows_g, m->H, m->dh, C1, 2 * C1));
+    aw = std::max(aw, attn_ws_need(m->dt, B, m->H, m->dh, C2, c->n1_pre + c->N1cap));
+  aw = std::max(aw, attn_ws_need(m->dt, B, m->H, m->dh, C2, C2));
+  for (int i = 0; i < C1; ++i)
+    aw = std::max(aw, attn_ws_need(m->dt, rows_g, m->H, m->dh, i == 0 ? C1 : 1, C1 + i));
   c->attn_ws_bytes = aw;
   c->attn_ws = al.get<float>(aw);
   const int positions =
@@ -722,6 +741,11 @@ int photon_prefill(photon_model* m, const photon_cache* prefix, const int32_t* d
     c->l1_k = c->l1_v = nullptr;
     c->N1 = 0;
   }
+  {
+    const int pos[2] = {c->N, c->N1};  // pageable source: staged before the call returns
+    if (cudaMemcpyAsync(c->d_pos, pos, sizeof(pos), cudaMemcpyHostToDevice, s) != cudaSuccess)
+      return bail(fail(PHOTON_ERR_CUDA, "position upload failed"));
+  }
   m->live_caches++;
   if (mode == PHOTON_MODE_HIER) m->hier_caches++;
   if (prefix) prefix->dependents++;
@@ -730,19 +754,15 @@ int photon_prefill(photon_model* m, const photon_cache* prefix, const int32_t* d
   return PHOTON_OK;
 }
 
-int photon_decode_step_ex(photon_model* m, photon_cache* c, int32_t mode, int32_t* d_out_tokens,
-                          float* d_out_logits, const int32_t* d_force_tokens,
-                          const void* d_force_a, void* stream) {
-  g_err.clear();
-  if (!m || !c || c->m != m) return fail(PHOTON_ERR_ARG, "model/cache mismatch");
-  if (!d_out_tokens) return fail(PHOTON_ERR_ARG, "output token buffer is NULL");
-  if (mode != PHOTON_MODE_HIER && mode != PHOTON_MODE_REC) return fail(PHOTON_ERR_ARG, "unknown mode %d", mode);
-  if (mode == PHOTON_MODE_HIER && (c->mode != PHOTON_MODE_HIER || !c->l1_k))
-    return fail(PHOTON_ERR_MODE, "HierGen needs the level-1 KV, discarded by a RecGen prefill");
-  if (c->steps >= c->max_new) return fail(PHOTON_ERR_CAPACITY, "cache is full (%d steps)", c->max_new);
-  if (mode == PHOTON_MODE_HIER && !m->group_ptr[G_ENC1]) RET(ensure_encoder(m, (cudaStream_t)stream));
-  cudaStream_t s = (cudaStream_t)stream;
-  c->stream = s;
+}  // extern "C"
+
+// Enqueues one decode step (a7..a13) on s.  Every per-step varying value is
+// read on the device (positions from c->d_pos), so the same launches can be
+// captured once into a CUDA graph and replayed for later steps.
+static void enqueue_decode(photon_model* m, photon_cache* c, int mode, int32_t* own_tokens,
+                           float* d_out_logits, const int32_t* d_force_tokens,
+                           const void* d_force_a, cudaStream_t s) {
+  int32_t* d_out_tokens = own_tokens;
   const int B = c->B, C1 = m->C1, C2 = m->C2, C = m->C, d = m->d, V = m->V, G = B * C2;
   const float eps = m->cfg.norm_eps;
   const Bufs b = decode_bufs(c);
@@ -771,12 +791,25 @@ int photon_decode_step_ex(photon_model* m, photon_cache* c, int32_t mode, int32_
   r1.layer_bytes = c->d1_layer;
   r1.cap = 2 * C1;
   run_stack(m, m->i_dec1, m->Ld1, c->xd, r1, b, s);
+  const int amax_tiles = m->use_tc ? gemm_tc_argmax_tiles(G, V, d) : 0;
   auto head = [&](const float* x, int in_step, int in_off, int i) {
     launch_rmsnorm(m->dt, x, (const float*)m->ptr(m->i_dec1_g), c->hn, G, d, in_step, in_off, eps, s);
-    float* lg = d_out_logits ? d_out_logits + (size_t)i * V : c->logits;
     const long long ld = d_out_logits ? (long long)C1 * V : V;
-    gemm(m, b, c->hn, d, m->ptr(m->i_head), d, G, V, d, epi(EPI_STORE_F32, lg, ld), s);
-    launch_argmax(lg, ld, G, V, i, C1, d_force_tokens, d_out_tokens, c->used, c->next_ids, c->d_err, s);
+    if (amax_tiles > 0 && amax_tiles <= c->amax_cap) {
+      // tensor-core head with the greedy choice fused into its epilogue;
+      // logits are written only when the caller asks for them
+      Epilogue e = epi(EPI_ARGMAX, d_out_logits ? d_out_logits + (size_t)i * V : nullptr, ld);
+      e.argmax_part = c->amax_part;
+      e.argmax_tiles = amax_tiles;
+      gemm(m, b, c->hn, d, m->ptr(m->i_head), d, G, V, d, e, s);
+      launch_argmax_partials(c->amax_part, amax_tiles, G, V, i, C1, d_force_tokens, d_out_tokens,
+                             c->used, c->next_ids, c->d_err, s);
+    } else {
+      float* lg = d_out_logits ? d_out_logits + (size_t)i * V : c->logits;
+      gemm(m, b, c->hn, d, m->ptr(m->i_head), d, G, V, d, epi(EPI_STORE_F32, lg, ld), s);
+      launch_argmax(lg, ld, G, V, i, C1, d_force_tokens, d_out_tokens, c->used, c->next_ids,
+                    c->d_err, s);
+    }
   };
   head(c->xd, C1, C1 - 1, 0);
   for (int i = 1; i < C1; ++i) {
@@ -801,7 +834,9 @@ int photon_decode_step_ex(photon_model* m, photon_cache* c, int32_t mode, int32_
     StackRun re;
     re.G = B;
     re.q_len = C2;
-    re.p0 = c->N1;
+    re.p0 = 0;
+    re.p0_dev = c->d_pos + 1;
+    re.n_plan = c->n1_pre + c->N1cap;
     re.kv_off = c->n1_pre;
     re.kc = c->l1_k;
     re.vc = c->l1_v;
@@ -823,7 +858,9 @@ int photon_decode_step_ex(photon_model* m, photon_cache* c, int32_t mode, int32_
   StackRun rt;
   rt.G = B;
   rt.q_len = 1;
-  rt.p0 = c->N;
+  rt.p0 = 0;
+  rt.p0_dev = c->d_pos;
+  rt.n_plan = c->n_pre + c->Ncap;
   rt.kv_off = c->n_pre;
   rt.kc = c->top_k;
   rt.vc = c->top_v;
@@ -838,6 +875,60 @@ int photon_decode_step_ex(photon_model* m, photon_cache* c, int32_t mode, int32_
   }
   run_stack(m, m->i_top, m->Ltop, c->xt, rt, b, s);
   launch_rmsnorm(m->dt, c->xt, (const float*)m->ptr(m->i_top_g), c->o, B, d, 1, 0, eps, s);
+  launch_advance(c->d_pos, 1, mode == PHOTON_MODE_HIER ? C2 : 0, s);
+}
+
+static bool graphs_enabled() {
+  static const bool on = [] {
+    const char* e = getenv("PHOTON_DECODE_GRAPH");
+    return !(e && e[0] == '0');
+  }();
+  return on;
+}
+
+extern "C" {
+
+int photon_decode_step_ex(photon_model* m, photon_cache* c, int32_t mode, int32_t* d_out_tokens,
+                          float* d_out_logits, const int32_t* d_force_tokens,
+                          const void* d_force_a, void* stream) {
+  g_err.clear();
+  if (!m || !c || c->m != m) return fail(PHOTON_ERR_ARG, "model/cache mismatch");
+  if (!d_out_tokens) return fail(PHOTON_ERR_ARG, "output token buffer is NULL");
+  if (mode != PHOTON_MODE_HIER && mode != PHOTON_MODE_REC) return fail(PHOTON_ERR_ARG, "unknown mode %d", mode);
+  if (mode == PHOTON_MODE_HIER && (c->mode != PHOTON_MODE_HIER || !c->l1_k))
+    return fail(PHOTON_ERR_MODE, "HierGen needs the level-1 KV, discarded by a RecGen prefill");
+  if (c->steps >= c->max_new) return fail(PHOTON_ERR_CAPACITY, "cache is full (%d steps)", c->max_new);
+  if (mode == PHOTON_MODE_HIER && !m->group_ptr[G_ENC1]) RET(ensure_encoder(m, (cudaStream_t)stream));
+  cudaStream_t s = (cudaStream_t)stream;
+  c->stream = s;
+  const int C2 = m->C2;
+  // The plain step (no hooks, no logits) is captured once per mode, after
+  // one eager step has configured every kernel, and replayed afterwards.
+  const bool plain = !d_out_logits && !d_force_tokens && !d_force_a;
+  bool replay = plain && s != nullptr && graphs_enabled() && c->steps >= 1 && !c->graph_failed[mode];
+  if (replay && !c->graph[mode]) {
+    cudaGraph_t g = nullptr;
+    bool ok = cudaStreamBeginCapture(s, cudaStreamCaptureModeRelaxed) == cudaSuccess;
+    if (ok) {
+      enqueue_decode(m, c, mode, c->tok_out, nullptr, nullptr, nullptr, s);
+      ok = cudaStreamEndCapture(s, &g) == cudaSuccess && g;
+    }
+    if (ok) ok = cudaGraphInstantiate(&c->graph[mode], g, 0) == cudaSuccess;
+    if (g) cudaGraphDestroy(g);
+    if (!ok) {
+      cudaGetLastError();
+      c->graph[mode] = nullptr;
+      c->graph_failed[mode] = true;
+      replay = false;
+    }
+  }
+  if (replay) {
+    CK(cudaGraphLaunch(c->graph[mode], s));
+    CK(cudaMemcpyAsync(d_out_tokens, c->tok_out, (size_t)c->B * m->C * sizeof(int32_t),
+                       cudaMemcpyDeviceToDevice, s));
+  } else {
+    enqueue_decode(m, c, mode, d_out_tokens, d_out_logits, d_force_tokens, d_force_a, s);
+  }
   CK(cudaGetLastError());
   c->N += 1;
   if (mode == PHOTON_MODE_HIER) {
@@ -867,6 +958,8 @@ int photon_free_cache(photon_cache* c) {
   if (c->dependents) return fail(PHOTON_ERR_ARG, "%d caches still read this prefix", c->dependents);
   photon_model* m = c->m;
   CK(cudaStreamSynchronize(c->stream));
+  for (int k = 0; k < 2; ++k)
+    if (c->graph[k]) cudaGraphExecDestroy(c->graph[k]);
   free_list(c->allocs, c->stream);
   CK(cudaStreamSynchronize(c->stream));
   if (c->prefix) c->prefix->dependents--;
@@ -1024,7 +1117,7 @@ int photon_attn_decode(int32_t dtype, const void* d_q, const void* d_k, const vo
   a.O = d_o;
   a.o_ld = (long long)H * head_dim;
   a.scale = 1.0f / sqrtf((float)head_dim);
-  const size_t wsb = attn_decode_workspace_bytes(a);
+  const size_t wsb = attn_decode_workspace_bytes(dtype, a);
   float* ws = nullptr;
   if (wsb) CK(cudaMallocAsync((void**)&ws, wsb, s));
   const bool ok = launch_attn_decode(dtype, a, ws, wsb, nullptr, s);

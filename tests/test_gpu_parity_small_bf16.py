@@ -1,0 +1,96 @@
+"""bf16 end-to-end parity on a small model with ragged shapes everywhere.
+
+B = 3 sequences of 336 tokens: 84 level-1 positions per sequence (two
+64-query attention tiles, the second ragged), 21 top positions, GEMM row
+counts 1008 / 252 / 63 / 48 / 12 / 3 (tails in both tcgen05 orientations),
+d = 128 (two 64-wide K slices), vocab 512.  Whole batch compared with the
+oracle, both modes, three decode chunks, bf16 tolerance 2e-2.
+"""
+import numpy as np
+import pytest
+import torch
+
+import hierarchical_autoregressive_lm_b200 as hal
+from oracle import Config, PhotonOracle
+
+pytestmark = pytest.mark.gpu
+
+SHAPE = dict(vocab=512, d_model=128, n_heads=2, head_dim=64, C1=4, C2=4, L1=2, Ltop=2, Ld1=2,
+             Ld2=2, mlp_mult=4, dtype="bf16", init_std=0.02, rope_theta=10000.0, norm_eps=1e-6)
+CFG = Config.from_dict(SHAPE)
+B, T, STEPS, TOL = 3, 336, 3, 2e-2
+
+
+def f64(buf):
+    return buf.view(torch.bfloat16).float().cpu().numpy().astype(np.float64)
+
+
+def rel(g, o):
+    return float(np.max(np.abs(g - o)) / np.max(np.abs(o)))
+
+
+@pytest.mark.parametrize("mode", ["rec", "hier"])
+def test_small_bf16_parity(mode):
+    orc = PhotonOracle(CFG, 7)
+    model = hal.Model(SHAPE, 7)
+    toks = np.random.default_rng(3).integers(0, SHAPE["vocab"], size=(B, T)).astype(np.int32)
+    code = hal.MODE_HIER if mode == "hier" else hal.MODE_REC
+    sts = [orc.prefill(toks[b], mode) for b in range(B)]
+    cache = model.prefill(torch.from_numpy(toks).cuda(), code, STEPS)
+    H, dh = CFG.n_heads, CFG.head_dim
+    for l in range(CFG.Ltop):
+        k = f64(cache.export_state("top_k", l)).reshape(B, H, -1, dh)
+        for b in range(B):
+            assert rel(k[b], sts[b].top[l].k.transpose(1, 0, 2)) < TOL
+    if mode == "hier":
+        for l in range(CFG.L1):
+            v = f64(cache.export_state("l1_v", l)).reshape(B, H, -1, dh)
+            for b in range(B):
+                assert rel(v[b], sts[b].l1[l].v.transpose(1, 0, 2)) < TOL
+    o = f64(cache.export_state("pending_o")).reshape(B, -1)
+    for b in range(B):
+        assert rel(o[b], sts[b].o) < TOL
+    out = torch.empty(B, CFG.C, dtype=torch.int32, device="cuda")
+    lg = torch.empty(B, CFG.C, CFG.vocab, device="cuda")
+    for step in range(STEPS):
+        refs = [orc.decode_step(st, mode) for st in sts]
+        force = torch.from_numpy(np.stack([r.tokens for r in refs]).astype(np.int32)).cuda()
+        cache.decode_step(code, out, lg, force_tokens=force)
+        torch.cuda.synchronize()
+        g = lg.double().cpu().numpy()
+        toks_gpu = out.cpu().numpy()
+        for b, r in enumerate(refs):
+            err = np.max(np.abs(g[b] - r.logits), axis=1)
+            assert np.max(err / np.max(np.abs(r.logits), axis=1)) < TOL, (step, b)
+            srt = np.sort(r.logits, axis=1)
+            decisive = (srt[:, -1] - srt[:, -2]) > 2 * err
+            np.testing.assert_array_equal(toks_gpu[b][decisive], r.tokens[decisive])
+        info = cache.info()
+        assert (info["N"], info["N1"], info["device_error"]) == (sts[0].N, sts[0].N1, 0)
+    o = f64(cache.export_state("pending_o")).reshape(B, -1)
+    for b in range(B):
+        assert rel(o[b], sts[b].o) < TOL
+    cache.free()
+    model.free()
+
+
+def test_small_bf16_graph_replay_equals_eager():
+    # tcgen05 path: captured-and-replayed decode steps give exactly the
+    # tokens and caches of the eager path (a force buffer of -1 keeps eager)
+    model = hal.Model(SHAPE, 7)
+    toks = torch.from_numpy(np.random.default_rng(4).integers(0, SHAPE["vocab"], size=(B, T))
+                            .astype(np.int32)).cuda()
+    g = model.prefill(toks, hal.MODE_REC, 4)
+    e = model.prefill(toks, hal.MODE_REC, 4)
+    none = torch.full((B, CFG.C), -1, dtype=torch.int32, device="cuda")
+    og = torch.empty(B, CFG.C, dtype=torch.int32, device="cuda")
+    oe = torch.empty_like(og)
+    for _ in range(4):
+        g.decode_step(hal.MODE_REC, og)
+        e.decode_step(hal.MODE_REC, oe, force_tokens=none)
+        torch.cuda.synchronize()
+        assert torch.equal(og, oe)
+    for l in range(CFG.Ltop):
+        assert torch.equal(g.export_state("top_k", l), e.export_state("top_k", l))
+    assert torch.equal(g.export_state("pending_o"), e.export_state("pending_o"))
+    g.free(); e.free(); model.free()
