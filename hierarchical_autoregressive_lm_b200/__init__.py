@@ -16,7 +16,7 @@ import os
 from typing import Optional
 
 __all__ = ["PhotonError", "Model", "Cache", "load_library", "LIB_PATH", "MODE_HIER",
-           "MODE_REC", "STATE", "launch_count", "gemm", "attn_decode", "config_struct", "EXPORTED"]
+           "MODE_REC", "STATE", "launch_count", "gemm", "attn_decode", "attn_decode_noalloc", "config_struct", "EXPORTED"]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libphoton.so")
 
@@ -31,7 +31,8 @@ EXPORTED = ("photon_init_weights", "photon_free_model", "photon_prefill",
             "photon_decode_step_hier", "photon_decode_step_rec", "photon_decode_step_ex",
             "photon_free_cache", "photon_cache_info", "photon_model_info",
             "photon_export_weight", "photon_export_state", "photon_gemm",
-            "photon_attn_decode", "photon_launch_count", "photon_last_error")
+            "photon_attn_decode", "photon_attn_decode_noalloc", "photon_launch_count",
+            "photon_last_error")
 
 
 class PhotonError(RuntimeError):
@@ -91,6 +92,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "photon_export_state": [P, I32, I32, P, SZ, ctypes.POINTER(SZ), P],
         "photon_gemm": [I32, P, I64, P, I64, I32, I32, I32, P, I64, I32, I32, I32, P],
         "photon_attn_decode": [I32, P, P, P, I32, I32, I32, I32, I32, I32, P, P],
+        "photon_attn_decode_noalloc": [I32, P, P, P, I32, I32, I32, I32, I32, I32, P, P],
     }
     for name, args in sig.items():
         fn = getattr(L, name)
@@ -248,6 +250,16 @@ def gemm(A, W, C, path: int = 0, splits: int = 0, swap: int = -1, stream=None) -
     N = W.shape[0]
     _check(load_library().photon_gemm(dt, _ptr(A), A.stride(0), _ptr(W), W.stride(0), M, N, K,
                                       _ptr(C), C.stride(0), path, splits, swap, _stream(stream)))
+
+
+def attn_decode_noalloc(q, k, v, q_len: int, p0: int, out, stream=None) -> None:
+    """attn_decode through the allocation-free entry point (fixed 1 MiB scratch
+    inside the library; for callers whose memory is owned by someone else)."""
+    import torch
+    dt = 0 if q.dtype == torch.float32 else 1
+    G, H, cap, dh = k.shape
+    _check(load_library().photon_attn_decode_noalloc(dt, _ptr(q), _ptr(k), _ptr(v), G, H, dh,
+                                                     cap, q_len, p0, _ptr(out), _stream(stream)))
 
 
 def attn_decode(q, k, v, q_len: int, p0: int, out, stream=None) -> None:
