@@ -17,8 +17,9 @@ Reported (rank 0, one JSON line):
   e2e          the same metric through the public API with host buffers:
                prompt copied from pinned host memory and every chunk's tokens
                read back each decode step, copies inside the timed region;
-  roofline     the dominant decode kernel's achieved bandwidth against the
-               measured HBM copy peak;
+  roofline     the decode's dominant kernel (the weight-streaming tcgen05
+               GEMM launches of one decode chunk) against the measured HBM
+               copy peak; roofline_attention the same for the decode attention;
   cpu_baseline the CPU oracle timed on a bounded sample on the host cores.
 Between timed steps nothing is flushed: the step's working set (0.66 GB of
 decoder+top weights streamed per chunk, 0.9 GB of top KV) exceeds the 126 MB L2.
@@ -190,10 +191,8 @@ def run_gpu(args) -> None:
         t0 = torch.cuda.Event(enable_timing=True)
         t1 = torch.cuda.Event(enable_timing=True)
         t0.record(stream)
-        for k in range(args.steps):
+        for k in range(args.steps):      # caches are freed after the timed region
             caches.append(one_step(evs[k], mark=(k == 0)))
-            if len(caches) > 1:          # keep at most two caches alive
-                caches.pop(0).free()
         t1.record(stream)
         torch.cuda.synchronize()
     launches = hal.launch_count() - n_launch0
@@ -228,8 +227,10 @@ def run_gpu(args) -> None:
     torch.cuda.synchronize()
     e2e_ms = e0.elapsed_time(e1)
 
-    # ---- dominant decode kernel alone, same shapes and launch configuration
-    roof = measure_roofline(model, wl, dev, stream)
+    # ---- the decode's dominant kernel (its GEMM launches) and its attention,
+    # alone, at the same shapes and launch configuration
+    roof = measure_gemm_roofline(model, wl, dev, stream)
+    roof_attn = measure_attn_roofline(model, wl, dev, stream)
 
     times = torch.tensor([total_ms, prefill_ms, decode_ms, e2e_ms], device=dev, dtype=torch.float64)
     if world > 1:
@@ -263,6 +264,7 @@ def run_gpu(args) -> None:
                 "covers": "H2D prompt + prefill + RecGen decode + per-chunk D2H of tokens"},
         "gpu_launches": launches,
         "roofline": roof,
+        "roofline_attention": roof_attn,
         "clocks": clk.summary(),
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -274,10 +276,71 @@ def run_gpu(args) -> None:
         dist.destroy_process_group()
 
 
-def measure_roofline(model, wl, dev, stream) -> dict:
-    """Times the split-K decode attention of the top encoder alone at the
-    decode's shapes (B sequences, H heads, N top entries averaged over the
-    decode, all Ltop layers in turn so the 0.9 GB working set exceeds L2)."""
+def _peak_gbs():
+    peaks, src = _peaks()
+    return peaks["hbm_gbs"], src
+
+
+def measure_gemm_roofline(model, wl, dev, stream) -> dict:
+    """The decode chunk's swapped-orientation tcgen05 GEMM launches (the
+    step's largest time share), replayed from a captured graph: every
+    projection of the top encoder (M = B), of the level-2 decoder and of the
+    three single-row token-decoder steps (M = B*C2), the two converters and
+    Chunker_2, each layer with its own weights (0.4 GB, more than L2).
+    Algorithmic bytes = weights + bf16 inputs + fp32 outputs of each launch."""
+    import torch
+    import hierarchical_autoregressive_lm_b200 as hal
+    s = model.shape
+    B, d, f = wl["batch"], s["d_model"], s["mlp_mult"] * s["d_model"]
+    C1, C2 = s["C1"], s["C2"]
+    G = B * C2
+    shapes = []
+    for _ in range(s["Ltop"]):
+        shapes += [(B, 3 * d, d), (B, d, d), (B, f, d), (B, d, f)]
+    for _ in range(s["Ld2"] + (C1 - 1) * s["Ld1"]):
+        shapes += [(G, 3 * d, d), (G, d, d), (G, f, d), (G, d, f)]
+    shapes += [(B, C2 * d, d), (G, C1 * d, d), (B, d, C2 * d)]
+    g = torch.Generator(device=dev).manual_seed(11)
+    bufs = []
+    for (M, N, K) in shapes:
+        bufs.append((torch.randn(M, K, device=dev, generator=g).to(torch.bfloat16),
+                     torch.randn(N, K, device=dev, generator=g).to(torch.bfloat16),
+                     torch.empty(M, N, device=dev)))
+    for A, W, C in bufs:                         # warm-up (configures kernels, fills the pool)
+        hal.gemm(A, W, C)
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=torch.cuda.Stream()):
+        for A, W, C in bufs:
+            hal.gemm(A, W, C)
+    graph.replay()
+    torch.cuda.synchronize()
+    reps = 10
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    a.record()
+    for _ in range(reps):
+        graph.replay()
+    b.record()
+    torch.cuda.synchronize()
+    ms = a.elapsed_time(b) / reps
+    algo = sum(N * K * 2 + M * K * 2 + M * N * 4 for (M, N, K) in shapes)
+    peak, src = _peak_gbs()
+    achieved = algo / (ms / 1e3) / 1e9
+    del graph, bufs
+    return {"kernel": "k_gemm_tc<64,4,swapped> (decode weight streaming: top encoder, level-2 "
+                      "decoder, token-decoder steps, converters, Chunker_2 of one decode chunk)",
+            "bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
+            "frac": round(achieved / peak, 4), "peak_source": f"{src} (STREAM-style copy)",
+            "traffic": None, "launches": len(shapes),
+            "bytes_per_launch": int(algo / len(shapes)),
+            "us_per_launch": round(ms * 1e3 / len(shapes), 3)}
+
+
+def measure_attn_roofline(model, wl, dev, stream) -> dict:
+    """The top encoder's decode attention alone at the decode's shapes (B
+    sequences, H heads, the middle step's key count), all Ltop layers' caches
+    in turn so the 0.86 GB working set exceeds L2."""
     import torch
     import hierarchical_autoregressive_lm_b200 as hal
     s = model.shape
@@ -311,12 +374,11 @@ def measure_roofline(model, wl, dev, stream) -> dict:
     ms = a.elapsed_time(b) / (reps * L)
     es = 2 if dt == torch.bfloat16 else 4
     algo = 2 * B * H * n_mid * dh * es + 2 * B * H * dh * es   # K,V rows read + q read + o write
-    peaks, src = _peaks()
+    peak, src = _peak_gbs()
     achieved = algo / (ms / 1e3) / 1e9
-    return {"kernel": "k_attn_decode (top-encoder decode attention; one CTA streams all keys of a "
-                      "(sequence, head) through a 4-stage bulk-copy ring at this shape)",
-            "bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"],
-            "unit": "GB/s", "frac": round(achieved / peaks["hbm_gbs"], 4),
+    return {"kernel": "k_attn_decode (top-encoder decode attention, one CTA per (sequence, head))",
+            "bound": "hbm", "achieved": round(achieved, 1), "peak": peak,
+            "unit": "GB/s", "frac": round(achieved / peak, 4),
             "peak_source": f"{src} (STREAM-style copy)", "traffic": None,
             "bytes_per_launch": algo, "us_per_launch": round(ms * 1e3, 3),
             "shape": f"B={B} H={H} dh={dh} keys={n_mid}"}

@@ -2,17 +2,15 @@
 //
 //  * k_attn_decode: a few new queries (q_len <= 4) per (group, head) over a
 //    long cache -- the top-encoder decode step, the level-1 re-encode of
-//    HierGen, and the chunk-local decoder attention.  Memory bound: the
-//    cache is split along the key axis into chunks; one CTA per (chunk,
-//    head, group) pulls its K and V rows into shared memory with two bulk
-//    async copies (TMA, completion on an mbarrier), computes scores with
-//    16-byte vector reads and shuffle reductions, a warp-level softmax per
-//    query, and the P*V product.  With several chunks, each CTA writes its
-//    unnormalised partial (acc, max, sum) and k_attn_combine merges them in
-//    chunk order.
-//  * k_attn_prefill: causal attention for many new queries (prefill).  Four
-//    threads per query, online softmax over 64-key blocks staged in shared
-//    memory.
+//    HierGen, and the chunk-local decoder attention.  Memory bound: every
+//    lane streams 16-byte slices of key and value rows straight from global
+//    memory with several loads in flight, each key group keeps its own
+//    online softmax, and the CTA merges its 16 key groups at the end.  Long
+//    caches with few (group, head) pairs are cut into chunks whose partials
+//    k_attn_combine merges in chunk order.
+//  * k_attn_prefill_mma: causal flash attention for many new queries
+//    (prefill) on mma.sync tensor-core tiles; k_attn_prefill is the
+//    CUDA-core version used for fp32 and other head sizes.
 //
 // Keys at positions < n_pre come from a shared prefix cache (the same for
 // every group); later keys from the group's own cache at slot pos - n_pre.
@@ -27,9 +25,6 @@ namespace photon {
 
 namespace {
 
-constexpr int kSub = 64;         // keys per ring stage of the decode attention
-constexpr int kRing = 4;         // ring stages
-constexpr int kDecThreads = 128;
 
 template <typename T, int DH>
 __device__ __forceinline__ const T* key_row(const AttnArgs& a, const T* own, const T* pre, int g,
@@ -38,343 +33,287 @@ __device__ __forceinline__ const T* key_row(const AttnArgs& a, const T* own, con
   return own + (((long long)g * a.H + h) * a.cap + (pos - a.n_pre)) * DH;
 }
 
-// Work split of the decode attention.  The key rows of all P = G*H
-// (group, head) pairs form one flattened axis of P*n rows (n live keys per
-// pair); CTA c takes rows [c*per, (c+1)*per).  A pair that falls inside one
-// CTA is finished there; a pair cut by CTA boundaries leaves one partial per
-// CTA, merged by k_attn_combine.
-struct DecSplit {
-  long long per;  // key rows per CTA (flattened mode)
-  int nc;         // CTAs
-  int ppc;        // > 0: whole-pair mode, ppc pairs per CTA (pairs never cut)
-};
-// CTAs whose row ranges hold pair p's keys (n live keys per pair).
-__host__ __device__ inline void dec_seg_range(const DecSplit& sp, long long p, int n, int& first,
-                                              int& last) {
-  if (sp.ppc > 0) {
-    first = last = (int)(p / sp.ppc);
-  } else {
-    first = (int)((p * n) / sp.per);
-    last = (int)(((p + 1) * n - 1) / sp.per);
-  }
+// Decode attention: one CTA (2 warps) per (key chunk, head, group).  Warp w
+// streams half of the chunk's keys: each 16-byte slice of a key row goes to
+// one lane (TPK lanes per row, 32/TPK rows per warp-wide load).  Every lane
+// keeps a private ring of kDecStages stages in shared memory and fills it
+// with cp.async copies of its own slices, kDecStages-1 batches ahead of
+// the batch it is using; since a lane only reads back what it copied itself,
+// no barrier or warp synchronisation is needed until the end.  Each key
+// group keeps its own online-softmax state; the key groups are merged with
+// shuffles inside a warp and through shared memory across the two warps.
+// With several chunks per (group, head), partials (acc, max, sum) are
+// merged in chunk order by k_attn_combine.
+constexpr int kDecWarps = 2;
+constexpr int kDecStages = 3;
+constexpr int kDecU = 2;  // rows per key group per stage
+
+__device__ __forceinline__ void cp_async16_zfill(uint32_t dst, const void* src, bool valid) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src),
+               "r"(valid ? 16 : 0)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_commit_group() {
+  asm volatile("cp.async.commit_group;" ::: "memory");
+}
+template <int N>
+__device__ __forceinline__ void cp_async_wait_group() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
 }
 
 template <typename T, int DH, int QMAX>
-__global__ void __launch_bounds__(kDecThreads)
-    k_attn_decode(AttnArgs a, DecSplit sp, int seg_max, float* __restrict__ part, int* err) {
-  constexpr int VEC = 16 / sizeof(T);          // elements per 16-byte slice
-  constexpr int TPK = DH / VEC;                // threads per key row
-  constexpr int KG = kDecThreads / TPK;        // key groups per pass
-  static_assert(32 % TPK == 0, "a key row must map inside one warp");
-
-  extern __shared__ __align__(128) uint8_t smem_raw[];
-  T* Kr = reinterpret_cast<T*>(smem_raw);                          // [kRing][kSub][DH]
-  T* Vr = Kr + kRing * kSub * DH;                                  // [kRing][kSub][DH]
-  float* sc = reinterpret_cast<float*>(Vr + kRing * kSub * DH);    // [QMAX][kSub]
-  float* red = sc + QMAX * kSub;                                   // [4][QMAX][DH]
-  float* lsum = red + 4 * QMAX * DH;                               // [4][QMAX]
-  __shared__ __align__(8) uint64_t bars[kRing];
+__global__ void __launch_bounds__(32 * kDecWarps, (QMAX == 1 ? 12 : 4))
+    k_attn_decode(AttnArgs a, int chunk, int splits, float* __restrict__ part, int* err) {
+  constexpr int SPL = 2;                       // 16-byte slices per lane per row
+  constexpr int VEC = 16 / sizeof(T);          // elements per slice
+  constexpr int LV = SPL * VEC;                // elements per lane per row
+  constexpr int TPK = DH / LV;                 // lanes per key row
+  constexpr int GPW = 32 / TPK;                // key rows per warp-wide access
+  constexpr int U = kDecU;
+  constexpr int STEP = GPW * U;                // rows per warp per stage
+  static_assert(32 % TPK == 0 && TPK >= 1, "a key row must map inside one warp");
+  __shared__ float sm_m[kDecWarps][QMAX], sm_l[kDecWarps][QMAX];
+  __shared__ float sm_acc[kDecWarps][QMAX][DH];
+  extern __shared__ uint4 ring[];  // [warp][stage][K,V][U][SPL][lane]
 
   pdl_wait();  // before any global access, including the device-side position
   pdl_trigger();
+  const int s = blockIdx.x, h = blockIdx.y, g = blockIdx.z;
   const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
+  const int kgrp = lane / TPK, sl = lane % TPK;
   const int p0 = a.p0_dev ? (*a.p0_dev + a.p0) : a.p0;
-  const int n = p0 + a.q_len;                     // live keys of every pair
-  const long long P = (long long)a.G * a.H;
-  long long r0, r1;
-  if (sp.ppc > 0) {
-    r0 = (long long)blockIdx.x * sp.ppc * n;
-    r1 = min(P, (long long)(blockIdx.x + 1) * sp.ppc) * n;
-  } else {
-    r0 = (long long)blockIdx.x * sp.per;
-    r1 = min(P * n, r0 + sp.per);
-  }
-  if (r0 >= r1) return;
-  const T* Kown = reinterpret_cast<const T*>(a.K);
-  const T* Vown = reinterpret_cast<const T*>(a.V);
-  const T* Kpre = reinterpret_cast<const T*>(a.Kp);
-  const T* Vpre = reinterpret_cast<const T*>(a.Vp);
+  const int n = min(p0 + a.q_len, splits * chunk);
+  const int k0 = s * chunk, k1 = min(n, k0 + chunk);
+  const int nk = max(0, k1 - k0);
+  const int wc = (nk + kDecWarps - 1) / kDecWarps;
+  const int kw0 = k0 + warp * wc, kw1 = min(k1, kw0 + wc);
+  // per-lane row bases: row `key` of this (group, head) starts at base + key*DH
+  const T* kpre = a.Kp ? reinterpret_cast<const T*>(a.Kp) + (long long)h * a.cap_pre * DH + sl * LV : nullptr;
+  const T* vpre = a.Vp ? reinterpret_cast<const T*>(a.Vp) + (long long)h * a.cap_pre * DH + sl * LV : nullptr;
+  const long long own_off = ((long long)g * a.H + h) * a.cap * DH - (long long)a.n_pre * DH + sl * LV;
+  const T* kown = reinterpret_cast<const T*>(a.K) + own_off;
+  const T* vown = reinterpret_cast<const T*>(a.V) + own_off;
 
-  // Units: consecutive runs of <= kSub keys inside one pair, in row order.
-  struct Unit {
-    long long p;
-    int ks, ke;
+  auto slot = [&](int st, int kv, int u, int sp) -> uint4* {
+    return ring + (((((warp * kDecStages + st) * 2 + kv) * U + u) * SPL + sp) * 32 + lane);
   };
-  auto unit_at = [&](long long row) -> Unit {  // unit starting at flattened row
-    const long long p = row / n;
-    const int ks = (int)(row - p * n);
-    const int lim = (int)min((long long)n, r1 - p * n);
-    return {p, ks, min(lim, ks + kSub)};
-  };
-  if (t == 0) {
-    for (int i = 0; i < kRing; ++i) ptx::mbar_init(ptx::smem_u32(&bars[i]), 1);
-    ptx::fence_barrier_init();
-  }
-  __syncthreads();
-  auto issue = [&](const Unit& u, int slot) {
-    const int g = (int)(u.p / a.H), h = (int)(u.p - (long long)g * a.H);
-    const uint32_t bar = ptx::smem_u32(&bars[slot]);
-    ptx::mbar_arrive_expect_tx(bar, (uint32_t)(2 * (u.ke - u.ks) * DH * sizeof(T)));
-    T* kd = Kr + (size_t)slot * kSub * DH;
-    T* vd = Vr + (size_t)slot * kSub * DH;
-    const int pe = min(u.ke, a.n_pre);
-    if (pe > u.ks) {
-      const uint32_t bytes = (uint32_t)((pe - u.ks) * DH * sizeof(T));
-      ptx::bulk_load(ptx::smem_u32(kd), key_row<T, DH>(a, Kown, Kpre, g, h, u.ks), bytes, bar);
-      ptx::bulk_load(ptx::smem_u32(vd), key_row<T, DH>(a, Vown, Vpre, g, h, u.ks), bytes, bar);
-    }
-    const int os = max(u.ks, a.n_pre);
-    if (u.ke > os) {
-      const uint32_t bytes = (uint32_t)((u.ke - os) * DH * sizeof(T));
-      const size_t off = (size_t)(os - u.ks) * DH;
-      ptx::bulk_load(ptx::smem_u32(kd + off), key_row<T, DH>(a, Kown, Kpre, g, h, os), bytes, bar);
-      ptx::bulk_load(ptx::smem_u32(vd + off), key_row<T, DH>(a, Vown, Vpre, g, h, os), bytes, bar);
+  auto issue = [&](int st, int base) {
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int key = base + u * GPW + kgrp;
+      const bool ok = key < kw1;
+      const bool pre = key < a.n_pre;
+      const T* kr = ok ? (pre ? kpre : kown) + (long long)key * DH : reinterpret_cast<const T*>(a.K);
+      const T* vr = ok ? (pre ? vpre : vown) + (long long)key * DH : reinterpret_cast<const T*>(a.V);
+#pragma unroll
+      for (int sp = 0; sp < SPL; ++sp) {
+        cp_async16_zfill(ptx::smem_u32(slot(st, 0, u, sp)), kr + (ok ? sp * VEC : 0), ok);
+        cp_async16_zfill(ptx::smem_u32(slot(st, 1, u, sp)), vr + (ok ? sp * VEC : 0), ok);
+      }
     }
   };
-  // producer cursor (thread 0 only): the first kRing units go out now
-  long long prow = r0;
-  int issued = 0;
-  if (t == 0) {
-    while (issued < kRing && prow < r1) {
-      const Unit u = unit_at(prow);
-      issue(u, issued % kRing);
-      prow = u.p * n + u.ke;
-      ++issued;
+
+  float qv[QMAX][LV], m[QMAX], l[QMAX], acc[QMAX][LV];
+#pragma unroll
+  for (int qi = 0; qi < QMAX; ++qi) {
+    m[qi] = -INFINITY;
+    l[qi] = 0.f;
+#pragma unroll
+    for (int e = 0; e < LV; ++e) acc[qi][e] = 0.f;
+    if (qi < a.q_len) {
+      const T* qrow = reinterpret_cast<const T*>(a.Q) + ((long long)g * a.q_len + qi) * a.q_ld + h * DH + sl * LV;
+#pragma unroll
+      for (int sp = 0; sp < SPL; ++sp) {
+        const uint4 raw = __ldg(reinterpret_cast<const uint4*>(qrow + sp * VEC));
+        const T* qp = reinterpret_cast<const T*>(&raw);
+#pragma unroll
+        for (int e = 0; e < VEC; ++e) qv[qi][sp * VEC + e] = Elem<T>::to_f(qp[e]) * a.scale;
+      }
+    } else {
+#pragma unroll
+      for (int e = 0; e < LV; ++e) qv[qi][e] = 0.f;
     }
   }
 
-  const int kg = t / TPK, sl = t % TPK;
-  float qv[QMAX][VEC], m[QMAX], lp[QMAX], acc[QMAX][VEC];
-  long long row = r0;
-  int ui = 0;
-  long long cur_p = -1;
-  while (row < r1) {
-    const Unit u = unit_at(row);
-    if (u.p != cur_p) {  // a new pair: its query slices, fresh softmax state
-      cur_p = u.p;
-      const int g = (int)(u.p / a.H), h = (int)(u.p - (long long)g * a.H);
+  const int nb = (kw1 - kw0 + STEP - 1) / STEP;  // stages this warp consumes
+#pragma unroll
+  for (int st = 0; st < kDecStages - 1; ++st) {
+    if (st < nb) issue(st, kw0 + st * STEP);
+    cp_async_commit_group();
+  }
+  for (int b = 0; b < nb; ++b) {
+    const int nxt = b + kDecStages - 1;
+    if (nxt < nb) issue(nxt % kDecStages, kw0 + nxt * STEP);
+    cp_async_commit_group();
+    cp_async_wait_group<kDecStages - 1>();  // this lane's copies of stage b have landed
+    const int st = b % kDecStages, base = kw0 + b * STEP;
+    // scores of this stage's U rows, then one online-softmax update per query
+    float sc[QMAX][U];
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      float kf[LV];
+#pragma unroll
+      for (int sp = 0; sp < SPL; ++sp) {
+        const uint4 kraw = *slot(st, 0, u, sp);
+        const T* kp = reinterpret_cast<const T*>(&kraw);
+#pragma unroll
+        for (int e = 0; e < VEC; ++e) kf[sp * VEC + e] = Elem<T>::to_f(kp[e]);
+      }
+      const int key = base + u * GPW + kgrp;
 #pragma unroll
       for (int qi = 0; qi < QMAX; ++qi) {
-        m[qi] = -INFINITY;
-        lp[qi] = 0.f;
+        float d = 0.f;
 #pragma unroll
-        for (int e = 0; e < VEC; ++e) acc[qi][e] = 0.f;
-        if (qi < a.q_len) {
-          const T* qp = reinterpret_cast<const T*>(a.Q) + ((long long)g * a.q_len + qi) * a.q_ld +
-                        h * DH + sl * VEC;
+        for (int e = 0; e < LV; ++e) d = fmaf(qv[qi][e], kf[e], d);
 #pragma unroll
-          for (int e = 0; e < VEC; ++e) qv[qi][e] = ld_f(qp + e) * a.scale;
-        } else {
-#pragma unroll
-          for (int e = 0; e < VEC; ++e) qv[qi][e] = 0.f;
-        }
+        for (int o = TPK / 2; o > 0; o >>= 1) d += __shfl_xor_sync(0xffffffffu, d, o);
+        sc[qi][u] = (qi < a.q_len && key < kw1 && key <= p0 + qi) ? d : -INFINITY;
       }
     }
-    const int slot = ui % kRing;
-    if (!ptx::mbar_wait(ptx::smem_u32(&bars[slot]), (uint32_t)(ui / kRing) & 1u, nullptr)) {
-      if (t == 0) report_error(err, DEV_WAIT_TIMEOUT_BULK);
-      return;  // the copies never landed: nothing in flight is waited for
-    }
-    const T* Ks = Kr + (size_t)slot * kSub * DH;
-    const T* Vs = Vr + (size_t)slot * kSub * DH;
-    const int cnt = u.ke - u.ks;
-    // scores (all lanes run every pass so the shuffles stay converged)
-#pragma unroll
-    for (int jb = 0; jb < kSub; jb += KG) {
-      const int j = jb + kg;
-      const bool in = j < cnt;
-      uint4 raw = make_uint4(0u, 0u, 0u, 0u);
-      if (in) raw = *reinterpret_cast<const uint4*>(Ks + (size_t)j * DH + sl * VEC);
-      const T* kp = reinterpret_cast<const T*>(&raw);
-      float kf[VEC];
-#pragma unroll
-      for (int e = 0; e < VEC; ++e) kf[e] = Elem<T>::to_f(kp[e]);
-#pragma unroll
-      for (int qi = 0; qi < QMAX; ++qi) {
-        float pv = 0.f;
-#pragma unroll
-        for (int e = 0; e < VEC; ++e) pv = fmaf(qv[qi][e], kf[e], pv);
-#pragma unroll
-        for (int o = TPK / 2; o > 0; o >>= 1) pv += __shfl_xor_sync(0xffffffffu, pv, o);
-        if (in && sl == 0 && qi < a.q_len)
-          sc[qi * kSub + j] = (u.ks + j <= p0 + qi) ? pv : -INFINITY;
-      }
-    }
-    __syncthreads();
-    // online softmax: every warp derives the same running max from shared memory
-    float pr[QMAX];
 #pragma unroll
     for (int qi = 0; qi < QMAX; ++qi) {
-      float mx = -INFINITY;
-      if (qi < a.q_len) {
-        if (lane < cnt) mx = sc[qi * kSub + lane];
-        if (lane + 32 < cnt) mx = fmaxf(mx, sc[qi * kSub + lane + 32]);
-      }
-      mx = warp_max(mx);
+      float mx = sc[qi][0];
+#pragma unroll
+      for (int u = 1; u < U; ++u) mx = fmaxf(mx, sc[qi][u]);
+      if (mx == -INFINITY) continue;  // nothing visible in this batch
       const float mn = fmaxf(m[qi], mx);
-      const float corr = (mn == -INFINITY) ? 1.f : __expf(m[qi] - mn);
+      const float c = __expf(m[qi] - mn);  // 0 when m was -inf
+      float pe[U], ps = 0.f;
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        pe[u] = __expf(sc[qi][u] - mn);
+        ps += pe[u];
+      }
+      l[qi] = l[qi] * c + ps;
+#pragma unroll
+      for (int e = 0; e < LV; ++e) acc[qi][e] *= c;
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+#pragma unroll
+        for (int sp = 0; sp < SPL; ++sp) {
+          const uint4 vraw = *slot(st, 1, u, sp);
+          const T* vp = reinterpret_cast<const T*>(&vraw);
+#pragma unroll
+          for (int e = 0; e < VEC; ++e)
+            acc[qi][sp * VEC + e] = fmaf(pe[u], Elem<T>::to_f(vp[e]), acc[qi][sp * VEC + e]);
+        }
+      }
       m[qi] = mn;
-      lp[qi] *= corr;
-#pragma unroll
-      for (int e = 0; e < VEC; ++e) acc[qi][e] *= corr;
-      pr[qi] = mn;
     }
-    for (int j = kg; j < cnt; j += KG) {
-      const uint4 raw = *reinterpret_cast<const uint4*>(Vs + (size_t)j * DH + sl * VEC);
-      const T* vp = reinterpret_cast<const T*>(&raw);
-      float vf[VEC];
+  }
+  cp_async_wait_group<0>();
+
+  // merge the key groups of this warp (lanes sl, sl + TPK, ...)
 #pragma unroll
-      for (int e = 0; e < VEC; ++e) vf[e] = Elem<T>::to_f(vp[e]);
+  for (int qi = 0; qi < QMAX; ++qi) {
+    float M = m[qi];
 #pragma unroll
-      for (int qi = 0; qi < QMAX; ++qi) {
-        if (qi >= a.q_len) continue;
-        const float pv = (pr[qi] == -INFINITY) ? 0.f : __expf(sc[qi * kSub + j] - pr[qi]);
-        if (sl == 0) lp[qi] += pv;
+    for (int o = TPK; o < 32; o <<= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+    const float c = (M == -INFINITY) ? 0.f : __expf(m[qi] - M);
+    float L = l[qi] * c;
 #pragma unroll
-        for (int e = 0; e < VEC; ++e) acc[qi][e] = fmaf(pv, vf[e], acc[qi][e]);
-      }
+    for (int o = TPK; o < 32; o <<= 1) L += __shfl_xor_sync(0xffffffffu, L, o);
+#pragma unroll
+    for (int e = 0; e < LV; ++e) {
+      float v = acc[qi][e] * c;
+#pragma unroll
+      for (int o = TPK; o < 32; o <<= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+      acc[qi][e] = v;
     }
-    __syncthreads();  // slot and scores free again
-    if (t == 0 && prow < r1) {
-      const Unit nu = unit_at(prow);
-      issue(nu, issued % kRing);
-      prow = nu.p * n + nu.ke;
-      ++issued;
+    if (lane < TPK) {
+#pragma unroll
+      for (int e = 0; e < LV; ++e) sm_acc[warp][qi][sl * LV + e] = acc[qi][e];
     }
-    row = u.p * n + u.ke;
-    ++ui;
-    if (row >= r1 || row / n != cur_p) {
-      // the pair's run in this CTA ends: reduce over key groups and warps
-      const int g = (int)(cur_p / a.H), h = (int)(cur_p - (long long)g * a.H);
+    if (lane == 0) {
+      sm_m[warp][qi] = M;
+      sm_l[warp][qi] = L;
+    }
+  }
+  __syncthreads();
+  // merge the warps and write the output (or this chunk's partial)
+  for (int idx = t; idx < a.q_len * DH; idx += 32 * kDecWarps) {
+    const int qi = idx / DH, dd = idx - qi * DH;
+    float M = -INFINITY;
 #pragma unroll
-      for (int qi = 0; qi < QMAX; ++qi) {
-        float l = warp_sum(lp[qi]);
+    for (int w = 0; w < kDecWarps; ++w) M = fmaxf(M, sm_m[w][qi]);
+    float L = 0.f, v = 0.f;
 #pragma unroll
-        for (int e = 0; e < VEC; ++e) {
-          float v = acc[qi][e];
-#pragma unroll
-          for (int o = TPK; o < 32; o <<= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-          acc[qi][e] = v;
-        }
-        if (lane == 0) lsum[warp * QMAX + qi] = l;
+    for (int w = 0; w < kDecWarps; ++w) {
+      const float c = (sm_m[w][qi] == -INFINITY) ? 0.f : __expf(sm_m[w][qi] - M);
+      L += c * sm_l[w][qi];
+      v += c * sm_acc[w][qi][dd];
+    }
+    const long long row = (long long)g * a.q_len + qi;
+    if (splits == 1) {
+      st_f(reinterpret_cast<T*>(a.O) + row * a.o_ld + h * DH + dd, L > 0.f ? v / L : 0.f);
+    } else {
+      float* pp = part + ((row * a.H + h) * splits + s) * (DH + 2);
+      pp[dd] = v;
+      if (dd == 0) {
+        pp[DH] = M;
+        pp[DH + 1] = L;
       }
-      if (lane < TPK) {
-#pragma unroll
-        for (int qi = 0; qi < QMAX; ++qi)
-#pragma unroll
-          for (int e = 0; e < VEC; ++e) red[(warp * QMAX + qi) * DH + sl * VEC + e] = acc[qi][e];
-      }
-      __syncthreads();
-      int sf, sl_;
-      dec_seg_range(sp, cur_p, n, sf, sl_);
-      for (int idx = t; idx < a.q_len * DH; idx += kDecThreads) {
-        const int qi = idx / DH, dd = idx - qi * DH;
-        const float v = red[(0 * QMAX + qi) * DH + dd] + red[(1 * QMAX + qi) * DH + dd] +
-                        red[(2 * QMAX + qi) * DH + dd] + red[(3 * QMAX + qi) * DH + dd];
-        const float l = lsum[qi] + lsum[QMAX + qi] + lsum[2 * QMAX + qi] + lsum[3 * QMAX + qi];
-        const long long orow = (long long)g * a.q_len + qi;
-        if (sf == sl_) {
-          st_f(reinterpret_cast<T*>(a.O) + orow * a.o_ld + h * DH + dd, l > 0.f ? v / l : 0.f);
-        } else {
-          float* pp = part + ((cur_p * a.q_len + qi) * seg_max + ((int)blockIdx.x - sf)) * (DH + 2);
-          pp[dd] = v;
-          if (dd == 0) {
-            pp[DH] = m[qi];
-            pp[DH + 1] = l;
-          }
-        }
-      }
-      __syncthreads();  // red / lsum reused by the next pair
     }
   }
 }
 
-// Merge the partials of the pairs that were cut by CTA boundaries.
+// Merge the chunk partials of one (row, head) in chunk order.
 template <typename T, int DH>
-__global__ void k_attn_combine(AttnArgs a, DecSplit sp, int seg_max, const float* __restrict__ part) {
+__global__ void k_attn_combine(AttnArgs a, int splits, const float* __restrict__ part) {
   pdl_wait();
   pdl_trigger();
-  const long long pq = blockIdx.x;  // pair * q_len + qi
-  const long long p = pq / a.q_len;
-  const int qi = (int)(pq - p * a.q_len);
+  const int h = blockIdx.x;
+  const long long row = blockIdx.y;
   const int dd = threadIdx.x;
-  const int p0 = a.p0_dev ? (*a.p0_dev + a.p0) : a.p0;
-  const int n = p0 + a.q_len;
-  int sf, sl;
-  dec_seg_range(sp, p, n, sf, sl);
-  if (sf == sl) return;  // finished by its only CTA
-  const float* pp = part + pq * seg_max * (DH + 2);
-  const int S = sl - sf + 1;
+  const float* p = part + ((row * a.H + h) * splits) * (DH + 2);
   float M = -INFINITY;
-  for (int s = 0; s < S; ++s) M = fmaxf(M, pp[s * (DH + 2) + DH]);
+  for (int s = 0; s < splits; ++s) M = fmaxf(M, p[s * (DH + 2) + DH]);
   float L = 0.f, acc = 0.f;
-  for (int s = 0; s < S; ++s) {
-    const float mm = pp[s * (DH + 2) + DH];
+  for (int s = 0; s < splits; ++s) {
+    const float mm = p[s * (DH + 2) + DH];
     if (mm == -INFINITY) continue;
     const float w = __expf(mm - M);
-    L += w * pp[s * (DH + 2) + DH + 1];
-    acc += w * pp[s * (DH + 2) + dd];
+    L += w * p[s * (DH + 2) + DH + 1];
+    acc += w * p[s * (DH + 2) + dd];
   }
-  const int g = (int)(p / a.H), h = (int)(p - (long long)g * a.H);
-  st_f(reinterpret_cast<T*>(a.O) + ((long long)g * a.q_len + qi) * a.o_ld + h * DH + dd,
-       L > 0.f ? acc / L : 0.f);
+  st_f(reinterpret_cast<T*>(a.O) + row * a.o_ld + h * DH + dd, L > 0.f ? acc / L : 0.f);
 }
 
-template <typename T, int DH>
-size_t dec_smem(int qmax) {
-  return (size_t)2 * kRing * kSub * DH * sizeof(T) + (size_t)qmax * kSub * 4 +
-         (size_t)4 * qmax * DH * 4 + (size_t)4 * qmax * 4 + 128;
-}
-
-// Resident CTAs of the decode attention on this device (all SMs).
-template <typename T, int DH, int QMAX>
-int dec_resident_ctas() {
-  static int nc = 0;
-  if (nc == 0) {
-    const int smem = (int)dec_smem<T, DH>(QMAX);
-    cudaFuncSetAttribute(k_attn_decode<T, DH, QMAX>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-    int per_sm = 0, dev = 0, sms = 0;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k_attn_decode<T, DH, QMAX>, kDecThreads, smem);
-    nc = (per_sm > 0 ? per_sm : 1) * (sms > 0 ? sms : 148);
-  }
-  return nc;
-}
-
-// Split for a launch covering n_plan keys per pair.  Short caches (<= 256
-// keys) are never cut: each CTA takes whole pairs.
 struct DecPlan {
-  DecSplit sp;
-  int seg_max;
+  int chunk, splits;
 };
-DecPlan dec_plan_for(const AttnArgs& a, int nc) {
+// About 2048 resident warps fill the GPU (registers allow ~14 per SM).  One
+// CTA (2 warps) per (group, head) when the pairs alone come close to that;
+// otherwise the keys are cut into chunks of at least 128.  Planned for
+// n_plan keys when set (graph replays), so the grid never depends on the
+// live key count.
+DecPlan dec_plan(const AttnArgs& a) {
   const int n = a.n_plan > 0 ? a.n_plan : a.p0 + a.q_len;
-  const long long P = (long long)a.G * a.H;
-  DecPlan d;
-  if (n <= 256) {
-    d.sp.ppc = (int)((P + nc - 1) / nc);
-    d.sp.per = (long long)d.sp.ppc * n;
-    d.sp.nc = (int)((P + d.sp.ppc - 1) / d.sp.ppc);
-    d.seg_max = 1;
-  } else {
-    d.sp.ppc = 0;
-    d.sp.per = (P * n + nc - 1) / nc;
-    d.sp.nc = (int)((P * n + d.sp.per - 1) / d.sp.per);
-    d.seg_max = (int)((n + d.sp.per - 1) / d.sp.per) + 1;
-  }
-  return d;
+  const long long warps = (long long)a.G * a.H * kDecWarps;
+  int splits = (int)((2048 + warps / 2) / warps);
+  const int max_splits = (n + 127) / 128;
+  if (splits > max_splits) splits = max_splits;
+  if (splits < 1) splits = 1;
+  const int chunk = (n + splits - 1) / splits;
+  splits = (n + chunk - 1) / chunk;
+  return {chunk, splits};
 }
 
 template <typename T, int DH, int QMAX>
 void run_decode(const AttnArgs& a, const DecPlan& p, float* part, int* err, cudaStream_t s) {
-  const size_t smem = dec_smem<T, DH>(QMAX);
-  (void)dec_resident_ctas<T, DH, QMAX>();  // configures the shared-memory limit
-  launch_kernel(k_attn_decode<T, DH, QMAX>, dim3(p.sp.nc), kDecThreads, smem, s, a, p.sp, p.seg_max,
-                part, err);
-  if (p.seg_max > 1) {
-    const long long pq = (long long)a.G * a.H * a.q_len;
-    launch_kernel(k_attn_combine<T, DH>, dim3((unsigned)pq), DH, 0, s, a, p.sp, p.seg_max, part);
+  constexpr int kRingBytes = kDecWarps * kDecStages * 2 * kDecU * 2 * 32 * 16;
+  static bool configured = false;
+  if (!configured) {
+    cudaFuncSetAttribute(k_attn_decode<T, DH, QMAX>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         kRingBytes);
+    configured = true;
+  }
+  dim3 grid(p.splits, a.H, a.G);
+  launch_kernel(k_attn_decode<T, DH, QMAX>, grid, 32 * kDecWarps, kRingBytes, s, a, p.chunk,
+                p.splits, part, err);
+  if (p.splits > 1) {
+    dim3 cg(a.H, a.G * a.q_len);
+    launch_kernel(k_attn_combine<T, DH>, cg, DH, 0, s, a, p.splits, part);
   }
 }
 
@@ -685,32 +624,20 @@ static bool tc_attn_disabled() {
   return off;
 }
 
-// Resident-CTA count of the kernel instance a launch would use (0: none).
-static int dec_nc(int dt, int dh, int q_len) {
-  const bool q1 = q_len == 1;
-  if (dt == DT_BF16 && dh == 64) return q1 ? dec_resident_ctas<bf16, 64, 1>() : dec_resident_ctas<bf16, 64, 4>();
-  if (dt == DT_F32 && dh == 32) return q1 ? dec_resident_ctas<float, 32, 1>() : dec_resident_ctas<float, 32, 4>();
-  if (dt == DT_F32 && dh == 64) return q1 ? dec_resident_ctas<float, 64, 1>() : dec_resident_ctas<float, 64, 4>();
-  if (dt == DT_BF16 && dh == 32) return q1 ? dec_resident_ctas<bf16, 32, 1>() : dec_resident_ctas<bf16, 32, 4>();
-  return 0;
-}
-
 size_t attn_decode_workspace_bytes(int dt, const AttnArgs& a) {
-  const int nc = dec_nc(dt, a.dh, a.q_len);
-  if (nc <= 0 || a.G <= 0 || a.q_len <= 0) return 0;
-  const DecPlan p = dec_plan_for(a, nc);
-  if (p.seg_max <= 1) return 0;
-  return (size_t)a.G * a.H * a.q_len * p.seg_max * (a.dh + 2) * sizeof(float);
+  (void)dt;
+  if (a.G <= 0 || a.q_len <= 0) return 0;
+  const DecPlan p = dec_plan(a);
+  if (p.splits <= 1) return 0;
+  return (size_t)a.G * a.q_len * a.H * p.splits * (a.dh + 2) * sizeof(float);
 }
 
 bool launch_attn_decode(int dt, const AttnArgs& a, float* part, size_t part_bytes, int* err,
                         cudaStream_t s) {
   if (a.G <= 0 || a.q_len <= 0) return true;
   if (a.q_len > 4) return false;
-  const int nc = dec_nc(dt, a.dh, a.q_len);
-  if (nc <= 0) return false;
-  const DecPlan p = dec_plan_for(a, nc);
-  if (p.seg_max > 1 && (part == nullptr || part_bytes < attn_decode_workspace_bytes(dt, a)))
+  const DecPlan p = dec_plan(a);
+  if (p.splits > 1 && (part == nullptr || part_bytes < attn_decode_workspace_bytes(dt, a)))
     return false;
   if (dt == DT_BF16 && a.dh == 64)
     run_decode_q<bf16, 64>(a, p, part, err, s);
@@ -718,8 +645,10 @@ bool launch_attn_decode(int dt, const AttnArgs& a, float* part, size_t part_byte
     run_decode_q<float, 32>(a, p, part, err, s);
   else if (dt == DT_F32 && a.dh == 64)
     run_decode_q<float, 64>(a, p, part, err, s);
-  else
+  else if (dt == DT_BF16 && a.dh == 32)
     run_decode_q<bf16, 32>(a, p, part, err, s);
+  else
+    return false;
   return true;
 }
 

@@ -51,6 +51,7 @@ template <int BN, int STAGES, bool SWAP>
 __global__ void __launch_bounds__(128, 1)
     k_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
               int M, int N, int nkb, int kb_per_split, Epilogue ep, float* __restrict__ part,
+              int* __restrict__ tile_count, const char* __restrict__ w_ptr, long long w_ld_bytes,
               int* err) {
   using Cfg = TcCfg<BN, STAGES>;
   extern __shared__ uint8_t smem_raw[];
@@ -114,6 +115,15 @@ __global__ void __launch_bounds__(128, 1)
     for (int it = 0; it < pre; ++it) {  // fresh ring: no slot to wait for
       ptx::mbar_arrive_expect_tx(full_bar(it), (uint32_t)Cfg::kStageBytes);
       ptx::tma_load_2d(w_tile(it), tm_w, (kb0 + it) * kBK, w_row, full_bar(it));
+    }
+    if (w_ptr != nullptr && nk > pre) {
+      // the rest of this CTA's weight rows go to L2 while the previous kernel finishes
+      const int w_rows = SWAP ? kBM : BN;
+      const int w_lim = N;  // weight rows are output features in both orientations
+      const uint32_t bytes = (uint32_t)(nk - pre) * kBK * 2;
+      for (int r = 0; r < w_rows && w_row + r < w_lim; ++r)
+        ptx::bulk_prefetch_l2(w_ptr + (long long)(w_row + r) * w_ld_bytes + (long long)(kb0 + pre) * kBK * 2,
+                              bytes);
     }
     pdl_wait();
     for (int it = 0; it < pre; ++it)
@@ -280,6 +290,375 @@ __global__ void __launch_bounds__(128, 1)
   ptx::tc_fence_before();
   __syncthreads();
   if (warp == 0) ptx::tmem_dealloc(tmem, Cfg::kTmemCols);
+
+  // ---- split-K: the last CTA of a tile sums the partials in split order
+  if (part != nullptr && ok) {
+    __shared__ int s_last;
+    __threadfence();
+    __syncthreads();
+    const int tile = blockIdx.x * gridDim.y + blockIdx.y;
+    if (threadIdx.x == 0) s_last = atomicAdd(&tile_count[tile], 1) == (int)gridDim.z - 1;
+    __syncthreads();
+    if (!s_last) return;
+    __threadfence();
+    const int splits = gridDim.z;
+    if (!SWAP) {
+      const long long grow = a0 + tl;
+#pragma unroll 1
+      for (int j0 = 0; j0 < BN; j0 += 64) {
+        const int gc = b0 + j0;
+        if (grow >= M || gc >= N) continue;
+        float lo[32], hi[32];
+#pragma unroll
+        for (int i = 0; i < 32; ++i) lo[i] = hi[i] = 0.f;
+        for (int sp = 0; sp < splits; ++sp) {
+          const float4* p = reinterpret_cast<const float4*>(part + (long long)sp * plane + grow * N + gc);
+#pragma unroll
+          for (int q = 0; q < 8; ++q) {
+            const float4 a4 = __ldcg(p + q), b4 = __ldcg(p + 8 + q);
+            lo[4 * q] += a4.x; lo[4 * q + 1] += a4.y; lo[4 * q + 2] += a4.z; lo[4 * q + 3] += a4.w;
+            hi[4 * q] += b4.x; hi[4 * q + 1] += b4.y; hi[4 * q + 2] += b4.z; hi[4 * q + 3] += b4.w;
+          }
+        }
+        epi_row64(ep, grow, gc, lo, hi);
+      }
+    } else {
+      const int gf = a0 + tl;
+#pragma unroll 1
+      for (int j0 = 0; j0 < BN; j0 += 32) {
+        if (gf >= N) break;
+        float v[32];
+#pragma unroll
+        for (int i = 0; i < 32; ++i) v[i] = 0.f;
+        for (int sp = 0; sp < splits; ++sp) {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            const long long t = b0 + j0 + i;
+            if (t < M) v[i] += __ldcg(part + (long long)sp * plane + t * N + gf);
+          }
+        }
+        epi_col32(ep, b0 + j0, M, gf, v);
+      }
+    }
+    if (threadIdx.x == 0) tile_count[tile] = 0;  // ready for the next launch
+  }
+}
+
+// ------------------------------------------------------------------ persistent variant
+// For large M (prefill) one CTA per SM loops over 128 x BN output tiles
+// (row-major tile order, so the CTAs working at one moment share A tiles in
+// L2).  Warp 0 issues the TMA loads, warp 1 the MMAs, warps 2-5 drain the
+// accumulators; two TMEM accumulators (2 x BN columns) let the epilogue of
+// tile i overlap the main loop of tile i+1.  Epilogue warp w owns TMEM lanes
+// 32*(w%4)..+31, i.e. output rows of that quarter.
+template <int BN, int STAGES>
+__global__ void __launch_bounds__(192, 1)
+    k_gemm_tc_persist(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                      int M, int N, int nkb, int tiles_n, int n_tiles, Epilogue ep, int* err) {
+  using Cfg = TcCfg<BN, STAGES>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Cfg::kRingBytes);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * STAGES + 4);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  auto full_bar = [&](int st) { return ptx::smem_u32(bars + st); };
+  auto empty_bar = [&](int st) { return ptx::smem_u32(bars + STAGES + st); };
+  auto tfull_bar = [&](int b) { return ptx::smem_u32(bars + 2 * STAGES + b); };
+  auto tempty_bar = [&](int b) { return ptx::smem_u32(bars + 2 * STAGES + 2 + b); };
+  auto a_tile = [&](int st) { return ptx::smem_u32(smem + st * Cfg::kStageBytes); };
+  auto b_tile = [&](int st) { return ptx::smem_u32(smem + st * Cfg::kStageBytes + kATileBytes); };
+
+  if (threadIdx.x == 0) {
+    for (int st = 0; st < STAGES; ++st) {
+      ptx::mbar_init(full_bar(st), 1);
+      ptx::mbar_init(empty_bar(st), 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      ptx::mbar_init(tfull_bar(b), 1);
+      ptx::mbar_init(tempty_bar(b), 4);  // one arrival per epilogue warp
+    }
+    *abort_flag = 0;
+    ptx::fence_barrier_init();
+    ptx::prefetch_tmap(&tmA);
+    ptx::prefetch_tmap(&tmB);
+  }
+  __syncwarp();
+  if (warp == 0) {
+    ptx::tmem_alloc(ptx::smem_u32(tmem_slot), 2 * BN);
+    ptx::tmem_relinquish();
+  }
+  ptx::tc_fence_before();
+  __syncthreads();
+  ptx::tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  pdl_wait();  // every role touches global memory only after this point
+  pdl_trigger();
+
+  if (warp == 0) {
+    if (lane == 0) {  // ---- TMA producer
+      int it = 0;
+      for (int tile = blockIdx.x; tile < n_tiles && !*abort_flag; tile += gridDim.x) {
+        const int mt = tile / tiles_n, nt = tile - mt * tiles_n;
+        for (int kb = 0; kb < nkb; ++kb, ++it) {
+          const int st = it % STAGES;
+          const uint32_t ph = (uint32_t)(it / STAGES) & 1u;
+          if (!ptx::mbar_wait(empty_bar(st), ph ^ 1u, abort_flag)) {
+            report_error(err, DEV_WAIT_TIMEOUT_PRODUCER);
+            *abort_flag = 1;
+            break;
+          }
+          ptx::mbar_arrive_expect_tx(full_bar(st), (uint32_t)Cfg::kStageBytes);
+          ptx::tma_load_2d(a_tile(st), &tmA, kb * kBK, mt * kBM, full_bar(st));
+          ptx::tma_load_2d(b_tile(st), &tmB, kb * kBK, nt * BN, full_bar(st));
+        }
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {  // ---- MMA issuer
+      constexpr uint32_t idesc = ptx::idesc_bf16_f32(kBM, BN);
+      int it = 0, local = 0;
+      for (int tile = blockIdx.x; tile < n_tiles && !*abort_flag; tile += gridDim.x, ++local) {
+        const int b = local & 1;
+        const uint32_t use = (uint32_t)(local >> 1);
+        if (!ptx::mbar_wait(tempty_bar(b), (use & 1u) ^ 1u, abort_flag)) {
+          report_error(err, DEV_WAIT_TIMEOUT_MMA);
+          *abort_flag = 1;
+          break;
+        }
+        ptx::tc_fence_after();
+        const uint32_t d = tmem + (uint32_t)(b * BN);
+        for (int kb = 0; kb < nkb; ++kb, ++it) {
+          const int st = it % STAGES;
+          const uint32_t ph = (uint32_t)(it / STAGES) & 1u;
+          if (!ptx::mbar_wait(full_bar(st), ph, abort_flag)) {
+            report_error(err, DEV_WAIT_TIMEOUT_MMA);
+            *abort_flag = 1;
+            break;
+          }
+          ptx::tc_fence_after();
+          const uint64_t ad = ptx::sdesc_kmajor_sw128(a_tile(st));
+          const uint64_t bd = ptx::sdesc_kmajor_sw128(b_tile(st));
+#pragma unroll
+          for (int k = 0; k < kBK / 16; ++k)
+            ptx::mma_bf16(d, ad + 2 * k, bd + 2 * k, idesc, (kb > 0 || k > 0) ? 1u : 0u);
+          ptx::mma_commit(empty_bar(st));
+        }
+        ptx::mma_commit(tfull_bar(b));  // accumulator b complete
+      }
+    }
+  } else {
+    // ---- epilogue warps 2..5
+    const int q = warp & 3;
+    int local = 0;
+    for (int tile = blockIdx.x; tile < n_tiles; tile += gridDim.x, ++local) {
+      const int b = local & 1;
+      const uint32_t use = (uint32_t)(local >> 1);
+      if (!ptx::mbar_wait(tfull_bar(b), use & 1u, abort_flag)) {
+        if (lane == 0) report_error(err, DEV_WAIT_TIMEOUT_EPILOGUE);
+        *abort_flag = 1;
+        break;
+      }
+      ptx::tc_fence_after();
+      const int mt = tile / tiles_n, nt = tile - mt * tiles_n;
+      const long long grow = (long long)mt * kBM + q * 32 + lane;
+      const uint32_t trow = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(b * BN);
+#pragma unroll 1
+      for (int j0 = 0; j0 < BN; j0 += 64) {
+        float lo[32], hi[32];
+        ptx::tmem_ld32(trow + (uint32_t)j0, lo);
+        ptx::tmem_ld32(trow + (uint32_t)(j0 + 32), hi);
+        const int gc = nt * BN + j0;
+        if (grow < M && gc < N) epi_row64(ep, grow, gc, lo, hi);
+      }
+      ptx::tc_fence_before();
+      __syncwarp();
+      if (lane == 0) ptx::mbar_arrive(tempty_bar(b));
+    }
+  }
+  ptx::tc_fence_before();
+  __syncthreads();
+  if (warp == 0) ptx::tmem_dealloc(tmem, 2 * BN);
+}
+
+// ------------------------------------------------------------------ cluster split-K variant
+// Few-token GEMM in the swapped orientation (decode).  A 128 x BN output
+// tile (128 output features x BN tokens) is computed by the S CTAs of one
+// thread-block cluster, CTA r taking the r-th run of K slices, so a weight
+// matrix with only a handful of 128-row tiles is still streamed by many SMs.
+// Each CTA moves its fp32 partial tile from TMEM into its own shared memory;
+// after a cluster barrier CTA r sums, in rank order, the rows it owns from
+// all S partial tiles through distributed shared memory and applies the
+// epilogue to them.  No partial tile goes to global memory and the sum
+// order is fixed, so results are deterministic.
+//
+// CTA r owns the RoPE pairs (f, f + 32) of the tile with pair index
+// u = (f / 64) * 32 + f % 64 in [r * 64 / S, (r + 1) * 64 / S), so the
+// QKV epilogue finds both values of a pair in one CTA.
+template <int BN, int S, int STAGES>
+__global__ void __launch_bounds__(128, 1)
+    k_gemm_dec(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX,
+               int M, int N, int nkb, int kbs, Epilogue ep, int* err) {
+  using Cfg = TcCfg<BN, STAGES>;
+  constexpr int LDP = BN + 4;  // partial-tile row stride in floats (16-byte skew per row)
+  static_assert(128 * LDP * 4 <= Cfg::kRingBytes, "the partial tile reuses the ring");
+  static_assert(64 % S == 0, "pairs must divide evenly over the cluster");
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Cfg::kRingBytes);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * STAGES + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = ptx::cluster_ctarank();
+  const int a0 = (blockIdx.x / S) * kBM;  // weight rows = output features
+  const int b0 = blockIdx.y * BN;         // token rows
+  const int kb0 = (int)rank * kbs;
+  const int kb1 = min(nkb, kb0 + kbs);
+  const int nk = max(0, kb1 - kb0);
+
+  auto full_bar = [&](int st) { return ptx::smem_u32(bars + st); };
+  auto empty_bar = [&](int st) { return ptx::smem_u32(bars + STAGES + st); };
+  const uint32_t done_bar = ptx::smem_u32(bars + 2 * STAGES);
+  auto w_tile = [&](int st) { return ptx::smem_u32(smem + st * Cfg::kStageBytes); };
+  auto x_tile = [&](int st) { return ptx::smem_u32(smem + st * Cfg::kStageBytes + kATileBytes); };
+
+  if (threadIdx.x == 0) {
+    for (int st = 0; st < STAGES; ++st) {
+      ptx::mbar_init(full_bar(st), 1);
+      ptx::mbar_init(empty_bar(st), 1);
+    }
+    ptx::mbar_init(done_bar, 1);
+    *abort_flag = 0;
+    ptx::fence_barrier_init();
+    ptx::prefetch_tmap(&tmW);
+    ptx::prefetch_tmap(&tmX);
+  }
+  __syncwarp();
+  if (warp == 0) {
+    ptx::tmem_alloc(ptx::smem_u32(tmem_slot), Cfg::kTmemCols);
+    ptx::tmem_relinquish();
+  }
+  ptx::tc_fence_before();
+  __syncthreads();
+  ptx::tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  // weights are never written by any kernel: the producer starts on them
+  // before waiting for the previous kernel (see k_gemm_tc)
+  if (threadIdx.x != 0) pdl_wait();
+  pdl_trigger();
+
+  if (threadIdx.x == 0) {
+    const int pre = nk < STAGES ? nk : STAGES;
+    for (int it = 0; it < pre; ++it) {
+      ptx::mbar_arrive_expect_tx(full_bar(it), (uint32_t)Cfg::kStageBytes);
+      ptx::tma_load_2d(w_tile(it), &tmW, (kb0 + it) * kBK, a0, full_bar(it));
+    }
+    pdl_wait();
+    for (int it = 0; it < pre; ++it)
+      ptx::tma_load_2d(x_tile(it), &tmX, (kb0 + it) * kBK, b0, full_bar(it));
+    for (int it = pre; it < nk; ++it) {
+      const int st = it % STAGES;
+      const uint32_t ph = (uint32_t)(it / STAGES) & 1u;
+      if (!ptx::mbar_wait(empty_bar(st), ph ^ 1u, abort_flag)) {
+        report_error(err, DEV_WAIT_TIMEOUT_PRODUCER);
+        *abort_flag = 1;
+        break;
+      }
+      ptx::mbar_arrive_expect_tx(full_bar(st), (uint32_t)Cfg::kStageBytes);
+      ptx::tma_load_2d(w_tile(st), &tmW, (kb0 + it) * kBK, a0, full_bar(st));
+      ptx::tma_load_2d(x_tile(st), &tmX, (kb0 + it) * kBK, b0, full_bar(st));
+    }
+  } else if (threadIdx.x == 32 && nk > 0) {
+    constexpr uint32_t idesc = ptx::idesc_bf16_f32(kBM, BN);
+    for (int it = 0; it < nk; ++it) {
+      const int st = it % STAGES;
+      const uint32_t ph = (uint32_t)(it / STAGES) & 1u;
+      if (!ptx::mbar_wait(full_bar(st), ph, abort_flag)) {
+        report_error(err, DEV_WAIT_TIMEOUT_MMA);
+        *abort_flag = 1;
+        break;
+      }
+      ptx::tc_fence_after();
+      const uint64_t wd = ptx::sdesc_kmajor_sw128(w_tile(st));
+      const uint64_t xd = ptx::sdesc_kmajor_sw128(x_tile(st));
+#pragma unroll
+      for (int k = 0; k < kBK / 16; ++k)
+        ptx::mma_bf16(tmem, wd + 2 * k, xd + 2 * k, idesc, (it > 0 || k > 0) ? 1u : 0u);
+      ptx::mma_commit(empty_bar(st));
+    }
+    ptx::mma_commit(done_bar);
+  }
+  __syncwarp();
+
+  // ---- this CTA's partial tile: TMEM -> shared memory (row = feature)
+  if (nk > 0 && !ptx::mbar_wait(done_bar, 0, abort_flag)) {
+    report_error(err, DEV_WAIT_TIMEOUT_EPILOGUE);
+    *abort_flag = 1;
+  }
+  __syncthreads();
+  const bool ok = (*abort_flag == 0);
+  ptx::tc_fence_after();
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+  float* P = reinterpret_cast<float*>(smem);
+  {
+    const int tl = warp * 32 + lane;
+    const uint32_t trow = tmem + ((uint32_t)(warp * 32) << 16);
+    float4* prow = reinterpret_cast<float4*>(P + tl * LDP);
+#pragma unroll 1
+    for (int j0 = 0; j0 < BN; j0 += 32) {
+      float v[32];
+      if (ok && nk > 0) {
+        ptx::tmem_ld32(trow + (uint32_t)j0, v);
+      } else {
+#pragma unroll
+        for (int i = 0; i < 32; ++i) v[i] = 0.f;
+      }
+#pragma unroll
+      for (int q = 0; q < 8; ++q)
+        prow[j0 / 4 + q] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+    }
+  }
+  ptx::tc_fence_before();
+  __syncthreads();
+  if (warp == 0) ptx::tmem_dealloc(tmem, Cfg::kTmemCols);
+  ptx::cluster_sync();  // every partial tile of the cluster is in place
+
+  // ---- reduce the owned pairs over the cluster, then the epilogue
+  constexpr int PU = 64 / S;          // pairs owned by one CTA
+  constexpr int ITEMS = PU * (BN / 4);
+  const uint32_t pbase = ptx::smem_u32(P);
+  if (ok) {
+#pragma unroll 1
+    for (int i = threadIdx.x; i < ITEMS; i += 128) {
+      const int u = (int)rank * PU + i % PU;
+      const int q = i / PU;  // token quad
+      const int f0 = (u >> 5) * 64 + (u & 31);
+      const uint32_t off0 = (uint32_t)(f0 * LDP + 4 * q) * 4u;
+      const uint32_t off1 = off0 + 32u * LDP * 4u;
+      float4 s0 = make_float4(0.f, 0.f, 0.f, 0.f), s1 = s0;
+#pragma unroll
+      for (int p = 0; p < S; ++p) {
+        const uint32_t peer = ptx::map_shared_rank(pbase, (uint32_t)p);
+        const float4 x0 = ptx::ld_shared_cluster_f4(peer + off0);
+        const float4 x1 = ptx::ld_shared_cluster_f4(peer + off1);
+        s0.x += x0.x; s0.y += x0.y; s0.z += x0.z; s0.w += x0.w;
+        s1.x += x1.x; s1.y += x1.y; s1.z += x1.z; s1.w += x1.w;
+      }
+      const int gf0 = a0 + f0;
+      if (gf0 >= N) continue;  // N is a multiple of 64: gf0 + 32 < N as well
+      const float v0[4] = {s0.x, s0.y, s0.z, s0.w}, v1[4] = {s1.x, s1.y, s1.z, s1.w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const long long t = b0 + 4 * q + e;
+        if (t < M) epi_pair<bf16>(ep, t, gf0, v0[e], gf0 + 32, v1[e]);
+      }
+    }
+  }
+  ptx::cluster_sync();  // peers keep their partial tiles until all reads are done
 }
 
 // ------------------------------------------------------------------ host side
@@ -319,8 +698,8 @@ bool make_map(CUtensorMap* m, const void* ptr, long long rows, int K, long long 
 
 template <int BN, int STAGES, bool SWAP>
 void run_tc(const CUtensorMap& ma, const CUtensorMap& mb, int grid_a, int grid_b, int splits,
-            int M, int N, int nkb, int kbs, const Epilogue& ep, float* part, int* err,
-            cudaStream_t s) {
+            int M, int N, int nkb, int kbs, const Epilogue& ep, float* part, int* counters,
+            const void* w_ptr, long long w_ld_bytes, int* err, cudaStream_t s) {
   using Cfg = TcCfg<BN, STAGES>;
   static bool configured = false;
   if (!configured) {
@@ -329,7 +708,124 @@ void run_tc(const CUtensorMap& ma, const CUtensorMap& mb, int grid_a, int grid_b
     configured = true;
   }
   dim3 grid(grid_a, grid_b, splits);
-  launch_kernel(k_gemm_tc<BN, STAGES, SWAP>, grid, 128, Cfg::kSmemBytes, s, ma, mb, M, N, nkb, kbs, ep, part, err);
+  launch_kernel(k_gemm_tc<BN, STAGES, SWAP>, grid, 128, Cfg::kSmemBytes, s, ma, mb, M, N, nkb, kbs, ep, part,
+                counters, static_cast<const char*>(w_ptr), w_ld_bytes, err);
+}
+
+template <int BN, int STAGES>
+void run_tc_persist(const CUtensorMap& ma, const CUtensorMap& mb, int M, int N, int nkb,
+                    const Epilogue& ep, int* err, cudaStream_t s) {
+  using Cfg = TcCfg<BN, STAGES>;
+  static int sms = 0;
+  if (!sms) {
+    cudaFuncSetAttribute(k_gemm_tc_persist<BN, STAGES>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         Cfg::kSmemBytes);
+    int dev = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (sms <= 0) sms = 148;
+  }
+  const int tiles_n = (N + BN - 1) / BN;
+  const int n_tiles = ((M + kBM - 1) / kBM) * tiles_n;
+  const int grid = n_tiles < sms ? n_tiles : sms;
+  launch_kernel(k_gemm_tc_persist<BN, STAGES>, dim3(grid), dim3(192), Cfg::kSmemBytes, s, ma, mb, M,
+                N, nkb, tiles_n, n_tiles, ep, err);
+}
+
+template <int BN, int S, int STAGES>
+bool cluster_launchable() {
+  static int state = 0;  // 0 unknown, 1 yes, -1 no
+  if (state == 0) {
+    using Cfg = TcCfg<BN, STAGES>;
+    auto k = k_gemm_dec<BN, S, STAGES>;
+    bool okf = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::kSmemBytes) ==
+               cudaSuccess;
+    if (S > 8)
+      okf = okf && cudaFuncSetAttribute(k, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) ==
+                       cudaSuccess;
+    int n = 0;
+    if (okf) {
+      cudaLaunchConfig_t cfg = {};
+      cfg.gridDim = dim3(S, 1, 1);
+      cfg.blockDim = dim3(128);
+      cfg.dynamicSmemBytes = Cfg::kSmemBytes;
+      cudaLaunchAttribute attr[1];
+      attr[0].id = cudaLaunchAttributeClusterDimension;
+      attr[0].val.clusterDim.x = S;
+      attr[0].val.clusterDim.y = 1;
+      attr[0].val.clusterDim.z = 1;
+      cfg.attrs = attr;
+      cfg.numAttrs = 1;
+      if (cudaOccupancyMaxActiveClusters(&n, k, &cfg) != cudaSuccess) n = 0;
+    }
+    cudaGetLastError();
+    state = (okf && n > 0) ? 1 : -1;
+  }
+  return state > 0;
+}
+
+template <int BN, int S, int STAGES>
+void run_dec(const CUtensorMap& mw, const CUtensorMap& mx, int ga, int gb, int M, int N, int nkb,
+             int kbs, const Epilogue& ep, int* err, cudaStream_t s) {
+  using Cfg = TcCfg<BN, STAGES>;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(ga * S, gb, 1);
+  cfg.blockDim = dim3(128);
+  cfg.dynamicSmemBytes = Cfg::kSmemBytes;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = S;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl_enabled() ? 2 : 1;
+  cudaLaunchKernelEx(&cfg, k_gemm_dec<BN, S, STAGES>, mw, mx, M, N, nkb, kbs, ep, err);
+  note_launch();
+}
+
+// Cluster split-K for the swapped orientation: one token tile of BN >= M
+// rows, S CTAs per 128-feature tile with S chosen so the grid covers about
+// one CTA per SM.  Returns false when the shape is left to k_gemm_tc.
+bool cluster_enabled() {
+  static const bool on = [] {
+    const char* e = getenv("PHOTON_GEMM_CLUSTER");
+    return !(e && e[0] == '0');
+  }();
+  return on;
+}
+
+template <int BN, int STAGES>
+bool try_dec(const GemmArgs& a, int* err, cudaStream_t s) {
+  const int M = a.M, N = a.N, nkb = a.K / kBK;
+  const int ga = (N + kBM - 1) / kBM;
+  int S = 1;
+  while (S < 16 && ga * S * 2 <= 148 && S * 2 <= nkb) S *= 2;
+  if (S == 16 && !cluster_launchable<BN, 16, STAGES>()) S = 8;
+  if (S < 2) return false;
+  const int kbs = (nkb + S - 1) / S;
+  CUtensorMap mw, mx;
+  if (!make_map(&mw, a.W, N, a.K, a.ldw, kBM) || !make_map(&mx, a.A, M, a.K, a.lda, BN)) return false;
+  switch (S) {
+    case 2:
+      if (!cluster_launchable<BN, 2, STAGES>()) return false;
+      run_dec<BN, 2, STAGES>(mw, mx, ga, 1, M, N, nkb, kbs, a.ep, err, s);
+      break;
+    case 4:
+      if (!cluster_launchable<BN, 4, STAGES>()) return false;
+      run_dec<BN, 4, STAGES>(mw, mx, ga, 1, M, N, nkb, kbs, a.ep, err, s);
+      break;
+    case 8:
+      if (!cluster_launchable<BN, 8, STAGES>()) return false;
+      run_dec<BN, 8, STAGES>(mw, mx, ga, 1, M, N, nkb, kbs, a.ep, err, s);
+      break;
+    default:
+      run_dec<BN, 16, STAGES>(mw, mx, ga, 1, M, N, nkb, kbs, a.ep, err, s);
+      break;
+  }
+  return true;
 }
 
 struct Plan {
@@ -351,12 +847,14 @@ Plan plan_for(int M, int N, int K, int force_splits, int force_swap, bool argmax
   const int ga = p.swap ? (N + kBM - 1) / kBM : (M + kBM - 1) / kBM;
   const int gb = p.swap ? (M + p.bn - 1) / p.bn : (N + p.bn - 1) / p.bn;
   const int tiles = ga * gb;
-  // Split K only to bound the K run of one CTA (1024) when the tile grid
-  // alone leaves SMs idle; the fp32 partial tiles cost M*N*8 bytes per split.
+  // Split K only to bound one CTA's K run at 1024 when the tile grid alone
+  // leaves SMs idle: each split costs M*N*8 bytes of fp32 partials and a
+  // reduction launch, which measured slower than the longer K run for the
+  // decode's K = 1024 projections.
   int splits = 1;
   if (force_splits > 0)
     splits = force_splits;
-  else if (tiles < 148 && !argmax) {
+  else if (!argmax && tiles < 148) {
     splits = (nkb + 15) / 16;
     const int cap = (2 * 148 + tiles - 1) / tiles;
     if (splits > cap) splits = cap;
@@ -368,6 +866,14 @@ Plan plan_for(int M, int N, int K, int force_splits, int force_swap, bool argmax
   p.ga = ga;
   p.gb = gb;
   return p;
+}
+
+bool persistent_enabled() {
+  static const bool on = [] {
+    const char* e = getenv("PHOTON_GEMM_PERSISTENT");
+    return !(e && e[0] == '0');
+  }();
+  return on;
 }
 
 }  // namespace
@@ -397,29 +903,48 @@ bool launch_gemm_tc(const GemmArgs& a, const GemmWorkspace& ws, int* err, cudaSt
   const Plan p = plan_for(M, N, K, argmax ? 1 : force_splits, force_swap, argmax);
   if (argmax && p.splits != 1) return false;
   float* part = nullptr;
+  int* counters = nullptr;
   if (p.splits > 1) {
     const size_t need = (size_t)p.splits * M * N * sizeof(float);
-    if (!ws.part || ws.bytes < need) return false;
+    if (!ws.part || ws.bytes < need || !ws.counters || ws.n_counters < p.ga * p.gb) return false;
     part = ws.part;
+    counters = ws.counters;
+  }
+  if (p.swap && force_splits <= 0 && !argmax && M <= 256 && cluster_enabled()) {
+    // few tokens: cluster split-K, the whole token range in one tile
+    bool done;
+    if (M <= 64)
+      done = try_dec<64, 4>(a, err, s);
+    else if (M <= 128)
+      done = try_dec<128, 4>(a, err, s);
+    else
+      done = try_dec<256, 3>(a, err, s);
+    if (done) return true;
   }
   CUtensorMap ma, mb;
   const int nkb = K / kBK;
   if (p.swap) {
     if (!make_map(&ma, a.W, N, K, a.ldw, kBM) || !make_map(&mb, a.A, M, K, a.lda, p.bn)) return false;
     if (p.bn == 64)
-      run_tc<64, 4, true>(ma, mb, p.ga, p.gb, p.splits, M, N, nkb, p.kbs, a.ep, part, err, s);
+      run_tc<64, 8, true>(ma, mb, p.ga, p.gb, p.splits, M, N, nkb, p.kbs, a.ep, part, counters, a.W, a.ldw * 2, err, s);
     else if (p.bn == 128)
-      run_tc<128, 4, true>(ma, mb, p.ga, p.gb, p.splits, M, N, nkb, p.kbs, a.ep, part, err, s);
+      run_tc<128, 4, true>(ma, mb, p.ga, p.gb, p.splits, M, N, nkb, p.kbs, a.ep, part, counters, a.W, a.ldw * 2, err, s);
     else
-      run_tc<256, 4, true>(ma, mb, p.ga, p.gb, p.splits, M, N, nkb, p.kbs, a.ep, part, err, s);
+      run_tc<256, 4, true>(ma, mb, p.ga, p.gb, p.splits, M, N, nkb, p.kbs, a.ep, part, counters, a.W, a.ldw * 2, err, s);
   } else {
     if (!make_map(&ma, a.A, M, K, a.lda, kBM) || !make_map(&mb, a.W, N, K, a.ldw, p.bn)) return false;
+    if (p.splits == 1 && !argmax && p.ga * p.gb >= 2 * 148 && persistent_enabled()) {
+      if (p.bn == 256)
+        run_tc_persist<256, 4>(ma, mb, M, N, nkb, a.ep, err, s);
+      else
+        run_tc_persist<128, 6>(ma, mb, M, N, nkb, a.ep, err, s);
+      return true;
+    }
     if (p.bn == 256)
-      run_tc<256, 4, false>(ma, mb, p.ga, p.gb, p.splits, M, N, nkb, p.kbs, a.ep, part, err, s);
+      run_tc<256, 4, false>(ma, mb, p.ga, p.gb, p.splits, M, N, nkb, p.kbs, a.ep, part, counters, a.W, a.ldw * 2, err, s);
     else
-      run_tc<128, 4, false>(ma, mb, p.ga, p.gb, p.splits, M, N, nkb, p.kbs, a.ep, part, err, s);
+      run_tc<128, 4, false>(ma, mb, p.ga, p.gb, p.splits, M, N, nkb, p.kbs, a.ep, part, counters, a.W, a.ldw * 2, err, s);
   }
-  if (p.splits > 1) launch_splitk_reduce(DT_BF16, part, p.splits, M, N, a.ep, s);
   return true;
 }
 

@@ -55,11 +55,16 @@ struct GemmArgs {
   Epilogue ep;
 };
 
-// Scratch the GEMM may use for split-K partial tiles (fp32).
+// Scratch the GEMM may use for split-K: fp32 partial tiles, and one counter
+// per output tile that must be zero before the first split launch (the
+// kernel leaves every counter at zero again).
 struct GemmWorkspace {
   float* part = nullptr;
   size_t bytes = 0;
+  int* counters = nullptr;
+  int n_counters = 0;
 };
+constexpr int kGemmTileCounters = 4096;
 
 // Attention of q_len new queries per group over a key/value cache.
 // Query i of group g sits at absolute position p0 + i and sees keys at

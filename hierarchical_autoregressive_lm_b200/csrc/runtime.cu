@@ -12,6 +12,7 @@
 #include <cstdlib>
 #include <cstdio>
 #include <cstring>
+#include <mutex>
 #include <string>
 #include <vector>
 
@@ -90,6 +91,10 @@ struct photon_model {
   int live_caches = 0;
   int hier_caches = 0;
   bool use_tc = false;
+  // Decode-step graph executables, one per mode, reused across caches: a new
+  // cache's captured step updates the executable instead of instantiating.
+  cudaGraphExec_t graph[2] = {nullptr, nullptr};
+  const void* graph_owner[2] = {nullptr, nullptr};
 
   const void* ptr(int idx) const { return group_ptr[t[idx].group] + t[idx].offset; }
   BlockW block(int first, int l) const {
@@ -174,6 +179,49 @@ static void build_specs(photon_model* m) {
   }
 }
 
+// Stream-ordered pool owned by the library, one per device.  Its release
+// threshold is unbounded: memory that a freed cache returns stays mapped and
+// is handed to the next cache, instead of being unmapped at the next
+// synchronisation and mapped again by the next prefill.  photon_free_model
+// trims it back to nothing.
+static std::mutex g_pool_mu;
+static cudaMemPool_t g_pool[64];
+
+static cudaError_t library_pool(cudaMemPool_t* out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lk(g_pool_mu);
+  if (!g_pool[dev]) {
+    cudaMemPoolProps p;
+    memset(&p, 0, sizeof(p));
+    p.allocType = cudaMemAllocationTypePinned;
+    p.handleTypes = cudaMemHandleTypeNone;
+    p.location.type = cudaMemLocationTypeDevice;
+    p.location.id = dev;
+    cudaMemPool_t pool = nullptr;
+    e = cudaMemPoolCreate(&pool, &p);
+    if (e != cudaSuccess) return e;
+    uint64_t keep = ~0ull;
+    e = cudaMemPoolSetAttribute(pool, cudaMemPoolAttrReleaseThreshold, &keep);
+    if (e != cudaSuccess) {
+      cudaMemPoolDestroy(pool);
+      return e;
+    }
+    g_pool[dev] = pool;
+  }
+  *out = g_pool[dev];
+  return cudaSuccess;
+}
+
+static cudaError_t pool_malloc(void** p, size_t bytes, cudaStream_t s) {
+  cudaMemPool_t pool = nullptr;
+  cudaError_t e = library_pool(&pool);
+  if (e != cudaSuccess) return e;
+  return cudaMallocFromPoolAsync(p, bytes, pool, s);
+}
+
 // Draws (or fills) every tensor of one group into its buffer.
 static void generate_group(photon_model* m, int g, cudaStream_t s) {
   const double K = ((double)m->cfg.init_std * 1.7320508075688772) / 65536.0;
@@ -194,7 +242,7 @@ static void generate_group(photon_model* m, int g, cudaStream_t s) {
 // is alive, and regenerated from the seed when needed again.
 static int ensure_encoder(photon_model* m, cudaStream_t s) {
   if (m->group_ptr[G_ENC1]) return PHOTON_OK;
-  CK(cudaMallocAsync((void**)&m->group_ptr[G_ENC1], m->group_bytes[G_ENC1], s));
+  CK(pool_malloc((void**)&m->group_ptr[G_ENC1], m->group_bytes[G_ENC1], s));
   generate_group(m, G_ENC1, s);
   CK(cudaGetLastError());
   return PHOTON_OK;
@@ -215,6 +263,7 @@ struct Bufs {
   const float2* rope;
   float* gemm_ws;
   size_t gemm_ws_bytes;
+  int* gemm_cnt;  // split-K tile counters (zeroed; one array per concurrent stream)
   float* attn_ws;
   size_t attn_ws_bytes;
   int* err;
@@ -244,6 +293,8 @@ struct photon_cache {
   int32_t *next_ids = nullptr, *used = nullptr;
   float* gemm_ws = nullptr;
   size_t gemm_ws_bytes = 0;
+  int* gemm_cnt = nullptr;
+  int* gemm_cnt_t = nullptr;
   float* attn_ws = nullptr;
   size_t attn_ws_bytes = 0;
   int* d_err = nullptr;
@@ -251,7 +302,12 @@ struct photon_cache {
   unsigned long long* amax_part = nullptr;  // [B*C2][amax_cap] head partials
   int amax_cap = 0;
   int32_t* tok_out = nullptr;    // [B, C] greedy tokens of the last graph-replayed step
-  cudaGraphExec_t graph[2] = {nullptr, nullptr};  // captured decode step per mode
+  // RecGen's top-encoder branch runs on its own stream with its own buffers
+  cudaStream_t side = nullptr;
+  cudaEvent_t ev_fork = nullptr, ev_join = nullptr;
+  void *xn_t = nullptr, *q_t = nullptr, *att_t = nullptr, *hid_t = nullptr;
+  float* gemm_ws_t = nullptr;
+  float* attn_ws_t = nullptr;
   bool graph_failed[2] = {false, false};
   std::vector<void*> allocs;
   size_t kv_bytes = 0, ws_bytes = 0;
@@ -267,7 +323,7 @@ struct Allocator {
   P* get(size_t bytes) {
     if (bytes == 0 || err != cudaSuccess) return nullptr;
     void* p = nullptr;
-    err = cudaMallocAsync(&p, (bytes + 255) & ~size_t(255), s);
+    err = pool_malloc(&p, (bytes + 255) & ~size_t(255), s);
     if (err != cudaSuccess) return nullptr;
     list->push_back(p);
     if (counter) *counter += bytes;
@@ -306,7 +362,7 @@ static void gemm(photon_model* m, const Bufs& b, const void* A, long long lda, c
   g.N = N;
   g.K = K;
   g.ep = ep;
-  GemmWorkspace ws{b.gemm_ws, b.gemm_ws_bytes};
+  GemmWorkspace ws{b.gemm_ws, b.gemm_ws_bytes, b.gemm_cnt, b.gemm_cnt ? kGemmTileCounters : 0};
   if (m->use_tc)
     launch_gemm(m->dt, g, ws, b.err, s);
   else
@@ -430,6 +486,7 @@ static Bufs decode_bufs(photon_cache* c) {
   b.rope = c->rope;
   b.gemm_ws = c->gemm_ws;
   b.gemm_ws_bytes = c->gemm_ws_bytes;
+  b.gemm_cnt = c->gemm_cnt;
   b.attn_ws = c->attn_ws;
   b.attn_ws_bytes = c->attn_ws_bytes;
   b.err = c->d_err;
@@ -497,9 +554,13 @@ int photon_free_model(photon_model* m) {
   if (!m) return fail(PHOTON_ERR_ARG, "model is NULL");
   if (m->live_caches) return fail(PHOTON_ERR_ARG, "%d caches still use this model", m->live_caches);
   CK(cudaDeviceSynchronize());
+  for (int k = 0; k < 2; ++k)
+    if (m->graph[k]) cudaGraphExecDestroy(m->graph[k]);
   for (int g = 0; g < G_COUNT; ++g)
     if (m->group_ptr[g]) cudaFree(m->group_ptr[g]);
   delete m;
+  cudaMemPool_t pool = nullptr;
+  if (library_pool(&pool) == cudaSuccess) cudaMemPoolTrimTo(pool, 0);
   return PHOTON_OK;
 }
 
@@ -577,6 +638,9 @@ int photon_prefill(photon_model* m, const photon_cache* prefix, const int32_t* d
   Allocator al{s, &c->allocs, &c->kv_bytes};
   auto bail = [&](int code) {
     cudaGetLastError();
+    if (c->side) cudaStreamDestroy(c->side);
+    if (c->ev_fork) cudaEventDestroy(c->ev_fork);
+    if (c->ev_join) cudaEventDestroy(c->ev_join);
     free_list(c->allocs, s);
     cudaStreamSynchronize(s);
     delete c;
@@ -644,11 +708,27 @@ int photon_prefill(photon_model* m, const photon_cache* prefix, const int32_t* d
     aw = std::max(aw, attn_ws_need(m->dt, rows_g, m->H, m->dh, i == 0 ? C1 : 1, C1 + i));
   c->attn_ws_bytes = aw;
   c->attn_ws = al.get<float>(aw);
+  // top-encoder branch (B rows) of RecGen, run concurrently with the token decoder
+  c->xn_t = al.get<void>((size_t)B * d * es);
+  c->q_t = al.get<void>((size_t)B * d * es);
+  c->att_t = al.get<void>((size_t)B * d * es);
+  c->hid_t = al.get<void>((size_t)B * m->f * es);
+  c->gemm_ws_t = al.get<float>(gw);
+  c->gemm_cnt = al.get<int>(kGemmTileCounters * sizeof(int));
+  c->gemm_cnt_t = al.get<int>(kGemmTileCounters * sizeof(int));
+  c->attn_ws_t = al.get<float>(aw);
+  if (cudaStreamCreateWithFlags(&c->side, cudaStreamNonBlocking) != cudaSuccess ||
+      cudaEventCreateWithFlags(&c->ev_fork, cudaEventDisableTiming) != cudaSuccess ||
+      cudaEventCreateWithFlags(&c->ev_join, cudaEventDisableTiming) != cudaSuccess)
+    return bail(fail(PHOTON_ERR_CUDA, "stream/event creation failed"));
   const int positions =
       std::max(std::max(c->n_pre + c->Ncap, c->n1_pre + N1_own + C2 * max_new_chunks), 2 * C1 + C2) + 1;
   rc = upload_rope(m, c, al, positions);
   if (al.err != cudaSuccess || rc) return bail(PHOTON_ERR_OOM);
-  if (cudaMemsetAsync(c->d_err, 0, 16, s) != cudaSuccess) return bail(PHOTON_ERR_CUDA);
+  if (cudaMemsetAsync(c->d_err, 0, 16, s) != cudaSuccess ||
+      cudaMemsetAsync(c->gemm_cnt, 0, kGemmTileCounters * sizeof(int), s) != cudaSuccess ||
+      cudaMemsetAsync(c->gemm_cnt_t, 0, kGemmTileCounters * sizeof(int), s) != cudaSuccess)
+    return bail(PHOTON_ERR_CUDA);
 
   // prefill workspace (released at the end of this call)
   std::vector<void*> tmp;
@@ -669,7 +749,7 @@ int photon_prefill(photon_model* m, const photon_cache* prefix, const int32_t* d
     free_list(tmp, s);
     return bail(PHOTON_ERR_OOM);
   }
-  Bufs pb{xn, q, att, hid, c->rope, pws, pgw, nullptr, 0, c->d_err};
+  Bufs pb{xn, q, att, hid, c->rope, pws, pgw, c->gemm_cnt, nullptr, 0, c->d_err};
 
   // a1: embedding; a2: Chunker_1 (concatenate C1 states, linear C1*d -> d)
   launch_embed(m->dt, d_tokens, m->ptr(m->i_embed), emb, (int)rows0, d, m->V, c->d_err, s);
@@ -766,6 +846,29 @@ static void enqueue_decode(photon_model* m, photon_cache* c, int mode, int32_t* 
   const int B = c->B, C1 = m->C1, C2 = m->C2, C = m->C, d = m->d, V = m->V, G = B * C2;
   const float eps = m->cfg.norm_eps;
   const Bufs b = decode_bufs(c);
+  auto top_step = [&](float* x, const Bufs& bb, cudaStream_t st) {
+    StackRun rt;
+    rt.G = B;
+    rt.q_len = 1;
+    rt.p0 = 0;
+    rt.p0_dev = c->d_pos;
+    rt.n_plan = c->n_pre + c->Ncap;
+    rt.kv_off = c->n_pre;
+    rt.kc = c->top_k;
+    rt.vc = c->top_v;
+    rt.layer_bytes = c->top_layer;
+    rt.cap = c->Ncap;
+    if (c->prefix) {
+      rt.kp = c->prefix->top_k;
+      rt.vp = c->prefix->top_v;
+      rt.pre_layer_bytes = c->prefix->top_layer;
+      rt.cap_pre = c->prefix->Ncap;
+      rt.n_pre = c->n_pre;
+    }
+    run_stack(m, m->i_top, m->Ltop, x, rt, bb, st);
+    launch_rmsnorm(m->dt, x, (const float*)m->ptr(m->i_top_g), c->o, B, d, 1, 0, eps, st);
+    launch_advance(c->d_pos, 1, mode == PHOTON_MODE_HIER ? C2 : 0, st);
+  };
 
   // a7: Converter_2 -- o [B, d] -> C2 conditioning vectors per sequence
   gemm(m, b, c->o, d, m->ptr(m->i_cv2), d, B, C2 * d, d, epi(EPI_STORE_F32, c->xd, (long long)C2 * d), s);
@@ -779,6 +882,28 @@ static void enqueue_decode(photon_model* m, photon_cache* c, int mode, int32_t* 
   r2.cap = C2;
   run_stack(m, m->i_dec2, m->Ld2, c->xd, r2, b, s);
   launch_rmsnorm(m->dt, c->xd, (const float*)m->ptr(m->i_dec2_g), c->a_hat, G, d, 1, 0, eps, s);
+  // RecGen: the top encoder's next input is Chunker_2(A-hat) and does not
+  // depend on the tokens, so the top-encoder branch (a12-R, a13) runs on the
+  // side stream, with its own buffers, while the token decoder (a9-a11)
+  // runs here; the two chains join at the end of the step.
+  const bool fork = mode == PHOTON_MODE_REC && c->side != nullptr;
+  if (fork) {
+    cudaEventRecord(c->ev_fork, s);
+    cudaStreamWaitEvent(c->side, c->ev_fork, 0);
+    Bufs bt = b;
+    bt.xn = c->xn_t;
+    bt.q = c->q_t;
+    bt.att = c->att_t;
+    bt.hid = c->hid_t;
+    bt.gemm_ws = c->gemm_ws_t;
+    bt.gemm_cnt = c->gemm_cnt_t;
+    bt.attn_ws = c->attn_ws_t;
+    const void* src = d_force_a ? d_force_a : c->a_hat;
+    gemm(m, bt, src, (long long)C2 * d, m->ptr(m->i_ch2), (long long)C2 * d, B, d, C2 * d,
+         epi(EPI_STORE_F32, c->xt, d), c->side);
+    top_step(c->xt, bt, c->side);
+    cudaEventRecord(c->ev_join, c->side);
+  }
   // a9: Converter_1 -- each A-hat row -> C1 conditioning vectors (rows g*C1 + i)
   gemm(m, b, c->a_hat, d, m->ptr(m->i_cv1), d, G, C1 * d, d, epi(EPI_STORE_F32, c->xd, (long long)C1 * d), s);
   // a10/a11: token decoder, prefix pass over the C1 conditioning positions,
@@ -821,8 +946,12 @@ static void enqueue_decode(photon_model* m, photon_cache* c, int mode, int32_t* 
     head(c->xs, 1, 0, i);
   }
   // a12: input of the top encoder's next position
+  if (fork) {
+    cudaStreamWaitEvent(s, c->ev_join, 0);  // join the top-encoder branch
+    return;
+  }
   if (mode == PHOTON_MODE_REC) {
-    // RecGen: Chunker_2(A-hat), no re-encoding
+    // RecGen without a side stream: Chunker_2(A-hat), no re-encoding
     const void* src = d_force_a ? d_force_a : c->a_hat;
     gemm(m, b, src, (long long)C2 * d, m->ptr(m->i_ch2), (long long)C2 * d, B, d, C2 * d,
          epi(EPI_STORE_F32, c->xt, d), s);
@@ -855,27 +984,7 @@ static void enqueue_decode(photon_model* m, photon_cache* c, int mode, int32_t* 
          epi(EPI_STORE_F32, c->xt, d), s);
   }
   // a13: one top-encoder step at position N (KV append + decode attention)
-  StackRun rt;
-  rt.G = B;
-  rt.q_len = 1;
-  rt.p0 = 0;
-  rt.p0_dev = c->d_pos;
-  rt.n_plan = c->n_pre + c->Ncap;
-  rt.kv_off = c->n_pre;
-  rt.kc = c->top_k;
-  rt.vc = c->top_v;
-  rt.layer_bytes = c->top_layer;
-  rt.cap = c->Ncap;
-  if (c->prefix) {
-    rt.kp = c->prefix->top_k;
-    rt.vp = c->prefix->top_v;
-    rt.pre_layer_bytes = c->prefix->top_layer;
-    rt.cap_pre = c->prefix->Ncap;
-    rt.n_pre = c->n_pre;
-  }
-  run_stack(m, m->i_top, m->Ltop, c->xt, rt, b, s);
-  launch_rmsnorm(m->dt, c->xt, (const float*)m->ptr(m->i_top_g), c->o, B, d, 1, 0, eps, s);
-  launch_advance(c->d_pos, 1, mode == PHOTON_MODE_HIER ? C2 : 0, s);
+  top_step(c->xt, b, s);
 }
 
 static bool graphs_enabled() {
@@ -906,24 +1015,37 @@ int photon_decode_step_ex(photon_model* m, photon_cache* c, int32_t mode, int32_
   // one eager step has configured every kernel, and replayed afterwards.
   const bool plain = !d_out_logits && !d_force_tokens && !d_force_a;
   bool replay = plain && s != nullptr && graphs_enabled() && c->steps >= 1 && !c->graph_failed[mode];
-  if (replay && !c->graph[mode]) {
+  if (replay && m->graph_owner[mode] != c) {
+    // capture this cache's step; update the model's executable in place when
+    // the topology matches, otherwise instantiate a new one
     cudaGraph_t g = nullptr;
     bool ok = cudaStreamBeginCapture(s, cudaStreamCaptureModeRelaxed) == cudaSuccess;
     if (ok) {
       enqueue_decode(m, c, mode, c->tok_out, nullptr, nullptr, nullptr, s);
       ok = cudaStreamEndCapture(s, &g) == cudaSuccess && g;
     }
-    if (ok) ok = cudaGraphInstantiate(&c->graph[mode], g, 0) == cudaSuccess;
+    if (ok && m->graph[mode]) {
+      cudaGraphExecUpdateResultInfo info;
+      if (cudaGraphExecUpdate(m->graph[mode], g, &info) != cudaSuccess) {
+        cudaGetLastError();
+        cudaGraphExecDestroy(m->graph[mode]);
+        m->graph[mode] = nullptr;
+      }
+    }
+    if (ok && !m->graph[mode]) ok = cudaGraphInstantiate(&m->graph[mode], g, 0) == cudaSuccess;
     if (g) cudaGraphDestroy(g);
     if (!ok) {
       cudaGetLastError();
-      c->graph[mode] = nullptr;
+      m->graph[mode] = nullptr;
+      m->graph_owner[mode] = nullptr;
       c->graph_failed[mode] = true;
       replay = false;
+    } else {
+      m->graph_owner[mode] = c;
     }
   }
   if (replay) {
-    CK(cudaGraphLaunch(c->graph[mode], s));
+    CK(cudaGraphLaunch(m->graph[mode], s));
     CK(cudaMemcpyAsync(d_out_tokens, c->tok_out, (size_t)c->B * m->C * sizeof(int32_t),
                        cudaMemcpyDeviceToDevice, s));
   } else {
@@ -959,7 +1081,13 @@ int photon_free_cache(photon_cache* c) {
   photon_model* m = c->m;
   CK(cudaStreamSynchronize(c->stream));
   for (int k = 0; k < 2; ++k)
-    if (c->graph[k]) cudaGraphExecDestroy(c->graph[k]);
+    if (m->graph_owner[k] == c) m->graph_owner[k] = nullptr;  // its buffers are going away
+  if (c->side) {
+    cudaStreamSynchronize(c->side);
+    cudaStreamDestroy(c->side);
+  }
+  if (c->ev_fork) cudaEventDestroy(c->ev_fork);
+  if (c->ev_join) cudaEventDestroy(c->ev_join);
   free_list(c->allocs, c->stream);
   CK(cudaStreamSynchronize(c->stream));
   if (c->prefix) c->prefix->dependents--;
@@ -1080,8 +1208,11 @@ int photon_gemm(int32_t dtype, const void* d_A, int64_t lda, const void* d_W, in
   const int nkb = K / 64 > 0 ? K / 64 : 1;
   const size_t wsb = (size_t)nkb * M * N * sizeof(float);
   float* ws = nullptr;
-  CK(cudaMallocAsync((void**)&ws, wsb, s));
-  GemmWorkspace w{ws, wsb};
+  int* cnt = nullptr;
+  CK(pool_malloc((void**)&ws, wsb, s));
+  CK(pool_malloc((void**)&cnt, kGemmTileCounters * sizeof(int), s));
+  CK(cudaMemsetAsync(cnt, 0, kGemmTileCounters * sizeof(int), s));
+  GemmWorkspace w{ws, wsb, cnt, kGemmTileCounters};
   int* err = nullptr;
   bool ok = launch_gemm_tc(g, w, err, s, splits > 0 ? splits : 0, swap);
   if (!ok && path == 0) {
@@ -1089,6 +1220,7 @@ int photon_gemm(int32_t dtype, const void* d_A, int64_t lda, const void* d_W, in
     ok = true;
   }
   cudaFreeAsync(ws, s);
+  cudaFreeAsync(cnt, s);
   if (!ok) return fail(PHOTON_ERR_ARG, "shape not supported by the tcgen05 kernel");
   CK(cudaGetLastError());
   return PHOTON_OK;
@@ -1119,7 +1251,7 @@ int photon_attn_decode(int32_t dtype, const void* d_q, const void* d_k, const vo
   a.scale = 1.0f / sqrtf((float)head_dim);
   const size_t wsb = attn_decode_workspace_bytes(dtype, a);
   float* ws = nullptr;
-  if (wsb) CK(cudaMallocAsync((void**)&ws, wsb, s));
+  if (wsb) CK(pool_malloc((void**)&ws, wsb, s));
   const bool ok = launch_attn_decode(dtype, a, ws, wsb, nullptr, s);
   if (ws) cudaFreeAsync(ws, s);
   if (!ok) return fail(PHOTON_ERR_ARG, "decode attention rejected the shape");

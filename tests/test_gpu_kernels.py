@@ -37,6 +37,13 @@ TC_CASES = [
     (128, 128, 64, 1, 0), (256, 512, 1024, 1, 0), (300, 256, 512, 1, 0), (4096, 1024, 1024, 1, 0),
     (64, 1024, 1024, 1, 1), (64, 1024, 1024, 4, 1), (256, 3072, 1024, 2, 1), (100, 384, 256, 1, 1),
     (256, 32000, 1024, 1, 1), (1024, 4096, 1024, 1, 0), (512, 1024, 4096, 8, 0),
+    # persistent warp-specialised kernel (>= 2 tiles per SM): BN 256 and 128, ragged M
+    (8192, 2048, 512, 0, 0), (8000, 1152, 256, 0, 0),
+    # automatic plan for few tokens: cluster split-K with the reduction in
+    # distributed shared memory; clusters of 16, 8 and 4, token tiles of
+    # 64 / 128 / 256, CTAs left without K slices (K = 18 and 10 slices)
+    (64, 1024, 1024, 0, 1), (256, 1024, 4096, 0, 1), (64, 3072, 1024, 0, 1), (100, 384, 256, 0, 1),
+    (256, 4096, 1024, 0, 1), (192, 1152, 1152, 0, 1), (1, 640, 640, 0, 1), (130, 2048, 2048, 0, 1),
 ]
 
 
@@ -44,7 +51,7 @@ TC_CASES = [
 def test_gemm_tcgen05_bf16(M, N, K, splits, swap):
     A, W = _rand((M, K), torch.bfloat16, 3), _rand((N, K), torch.bfloat16, 4)
     C = torch.full((M, N), float("nan"), device="cuda")
-    hal.gemm(A.cuda(), W.cuda(), C, path=2, splits=splits, swap=swap)
+    hal.gemm(A.cuda(), W.cuda(), C, path=2, splits=splits, swap=swap if splits else -1)
     torch.cuda.synchronize()
     ref = _gemm_ref(A, W)
     got = C.cpu().double().numpy()
