@@ -253,7 +253,7 @@ def gemm(A, W, C, path: int = 0, splits: int = 0, swap: int = -1, stream=None) -
 
 
 def attn_decode_noalloc(q, k, v, q_len: int, p0: int, out, stream=None) -> None:
-    """attn_decode through the allocation-free entry point (fixed 1 MiB scratch
+    """attn_decode through the allocation-free entry point (fixed 256 KiB scratch
     inside the library; for callers whose memory is owned by someone else)."""
     import torch
     dt = 0 if q.dtype == torch.float32 else 1

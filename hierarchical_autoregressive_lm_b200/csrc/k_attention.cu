@@ -44,9 +44,23 @@ __device__ __forceinline__ const T* key_row(const AttnArgs& a, const T* own, con
 // shuffles inside a warp and through shared memory across the two warps.
 // With several chunks per (group, head), partials (acc, max, sum) are
 // merged in chunk order by k_attn_combine.
-constexpr int kDecWarps = 2;
-constexpr int kDecStages = 3;
-constexpr int kDecU = 2;  // rows per key group per stage
+// Decode-attention tiling (compile-time; -D overrides exist for tuning sweeps).
+#ifndef PHOTON_DEC_WARPS
+#define PHOTON_DEC_WARPS 8
+#endif
+#ifndef PHOTON_DEC_STAGES
+#define PHOTON_DEC_STAGES 4
+#endif
+#ifndef PHOTON_DEC_U
+#define PHOTON_DEC_U 2
+#endif
+#ifndef PHOTON_DEC_SPL
+#define PHOTON_DEC_SPL 1
+#endif
+constexpr int kDecWarps = PHOTON_DEC_WARPS;    // warps per CTA
+constexpr int kDecStages = PHOTON_DEC_STAGES;  // cp.async ring depth per warp
+constexpr int kDecU = PHOTON_DEC_U;            // rows per key group per stage
+constexpr int kDecSPL = PHOTON_DEC_SPL;        // 16-byte slices of a key row per lane
 
 __device__ __forceinline__ void cp_async16_zfill(uint32_t dst, const void* src, bool valid) {
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src),
@@ -61,10 +75,10 @@ __device__ __forceinline__ void cp_async_wait_group() {
   asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
 }
 
-template <typename T, int DH, int QMAX>
-__global__ void __launch_bounds__(32 * kDecWarps, (QMAX == 1 ? 12 : 4))
+template <typename T, int DH, int QMAX, int W>
+__global__ void __launch_bounds__(32 * W, (QMAX == 1 ? 24 : 8) / W)
     k_attn_decode(AttnArgs a, int chunk, int splits, float* __restrict__ part, int* err) {
-  constexpr int SPL = 2;                       // 16-byte slices per lane per row
+  constexpr int SPL = kDecSPL;
   constexpr int VEC = 16 / sizeof(T);          // elements per slice
   constexpr int LV = SPL * VEC;                // elements per lane per row
   constexpr int TPK = DH / LV;                 // lanes per key row
@@ -72,8 +86,8 @@ __global__ void __launch_bounds__(32 * kDecWarps, (QMAX == 1 ? 12 : 4))
   constexpr int U = kDecU;
   constexpr int STEP = GPW * U;                // rows per warp per stage
   static_assert(32 % TPK == 0 && TPK >= 1, "a key row must map inside one warp");
-  __shared__ float sm_m[kDecWarps][QMAX], sm_l[kDecWarps][QMAX];
-  __shared__ float sm_acc[kDecWarps][QMAX][DH];
+  __shared__ float sm_m[W][QMAX], sm_l[W][QMAX];
+  __shared__ float sm_acc[W][QMAX][DH];
   extern __shared__ uint4 ring[];  // [warp][stage][K,V][U][SPL][lane]
 
   pdl_wait();  // before any global access, including the device-side position
@@ -85,12 +99,14 @@ __global__ void __launch_bounds__(32 * kDecWarps, (QMAX == 1 ? 12 : 4))
   const int n = min(p0 + a.q_len, splits * chunk);
   const int k0 = s * chunk, k1 = min(n, k0 + chunk);
   const int nk = max(0, k1 - k0);
-  const int wc = (nk + kDecWarps - 1) / kDecWarps;
+  const int wc = (nk + W - 1) / W;
   const int kw0 = k0 + warp * wc, kw1 = min(k1, kw0 + wc);
-  // per-lane row bases: row `key` of this (group, head) starts at base + key*DH
-  const T* kpre = a.Kp ? reinterpret_cast<const T*>(a.Kp) + (long long)h * a.cap_pre * DH + sl * LV : nullptr;
-  const T* vpre = a.Vp ? reinterpret_cast<const T*>(a.Vp) + (long long)h * a.cap_pre * DH + sl * LV : nullptr;
-  const long long own_off = ((long long)g * a.H + h) * a.cap * DH - (long long)a.n_pre * DH + sl * LV;
+  // per-lane row bases: row `key` of this (group, head) starts at base + key*DH.
+  // Lane sl of a key group holds the 16-byte slices sl, sl + TPK, ... of the
+  // row, so each warp-wide copy reads whole 32-byte sectors.
+  const T* kpre = a.Kp ? reinterpret_cast<const T*>(a.Kp) + (long long)h * a.cap_pre * DH + sl * VEC : nullptr;
+  const T* vpre = a.Vp ? reinterpret_cast<const T*>(a.Vp) + (long long)h * a.cap_pre * DH + sl * VEC : nullptr;
+  const long long own_off = ((long long)g * a.H + h) * a.cap * DH - (long long)a.n_pre * DH + sl * VEC;
   const T* kown = reinterpret_cast<const T*>(a.K) + own_off;
   const T* vown = reinterpret_cast<const T*>(a.V) + own_off;
 
@@ -107,8 +123,8 @@ __global__ void __launch_bounds__(32 * kDecWarps, (QMAX == 1 ? 12 : 4))
       const T* vr = ok ? (pre ? vpre : vown) + (long long)key * DH : reinterpret_cast<const T*>(a.V);
 #pragma unroll
       for (int sp = 0; sp < SPL; ++sp) {
-        cp_async16_zfill(ptx::smem_u32(slot(st, 0, u, sp)), kr + (ok ? sp * VEC : 0), ok);
-        cp_async16_zfill(ptx::smem_u32(slot(st, 1, u, sp)), vr + (ok ? sp * VEC : 0), ok);
+        cp_async16_zfill(ptx::smem_u32(slot(st, 0, u, sp)), kr + (ok ? sp * TPK * VEC : 0), ok);
+        cp_async16_zfill(ptx::smem_u32(slot(st, 1, u, sp)), vr + (ok ? sp * TPK * VEC : 0), ok);
       }
     }
   };
@@ -121,10 +137,10 @@ __global__ void __launch_bounds__(32 * kDecWarps, (QMAX == 1 ? 12 : 4))
 #pragma unroll
     for (int e = 0; e < LV; ++e) acc[qi][e] = 0.f;
     if (qi < a.q_len) {
-      const T* qrow = reinterpret_cast<const T*>(a.Q) + ((long long)g * a.q_len + qi) * a.q_ld + h * DH + sl * LV;
+      const T* qrow = reinterpret_cast<const T*>(a.Q) + ((long long)g * a.q_len + qi) * a.q_ld + h * DH + sl * VEC;
 #pragma unroll
       for (int sp = 0; sp < SPL; ++sp) {
-        const uint4 raw = __ldg(reinterpret_cast<const uint4*>(qrow + sp * VEC));
+        const uint4 raw = __ldg(reinterpret_cast<const uint4*>(qrow + sp * TPK * VEC));
         const T* qp = reinterpret_cast<const T*>(&raw);
 #pragma unroll
         for (int e = 0; e < VEC; ++e) qv[qi][sp * VEC + e] = Elem<T>::to_f(qp[e]) * a.scale;
@@ -222,7 +238,7 @@ __global__ void __launch_bounds__(32 * kDecWarps, (QMAX == 1 ? 12 : 4))
     }
     if (lane < TPK) {
 #pragma unroll
-      for (int e = 0; e < LV; ++e) sm_acc[warp][qi][sl * LV + e] = acc[qi][e];
+      for (int e = 0; e < LV; ++e) sm_acc[warp][qi][(sl + (e / VEC) * TPK) * VEC + e % VEC] = acc[qi][e];
     }
     if (lane == 0) {
       sm_m[warp][qi] = M;
@@ -231,14 +247,14 @@ __global__ void __launch_bounds__(32 * kDecWarps, (QMAX == 1 ? 12 : 4))
   }
   __syncthreads();
   // merge the warps and write the output (or this chunk's partial)
-  for (int idx = t; idx < a.q_len * DH; idx += 32 * kDecWarps) {
+  for (int idx = t; idx < a.q_len * DH; idx += 32 * W) {
     const int qi = idx / DH, dd = idx - qi * DH;
     float M = -INFINITY;
 #pragma unroll
-    for (int w = 0; w < kDecWarps; ++w) M = fmaxf(M, sm_m[w][qi]);
+    for (int w = 0; w < W; ++w) M = fmaxf(M, sm_m[w][qi]);
     float L = 0.f, v = 0.f;
 #pragma unroll
-    for (int w = 0; w < kDecWarps; ++w) {
+    for (int w = 0; w < W; ++w) {
       const float c = (sm_m[w][qi] == -INFINITY) ? 0.f : __expf(sm_m[w][qi] - M);
       L += c * sm_l[w][qi];
       v += c * sm_acc[w][qi][dd];
@@ -280,37 +296,47 @@ __global__ void k_attn_combine(AttnArgs a, int splits, const float* __restrict__
 }
 
 struct DecPlan {
-  int chunk, splits;
+  int chunk, splits, warps;
 };
-// About 2048 resident warps fill the GPU (registers allow ~14 per SM).  One
-// CTA (2 warps) per (group, head) when the pairs alone come close to that;
-// otherwise the keys are cut into chunks of at least 128.  Planned for
-// n_plan keys when set (graph replays), so the grid never depends on the
-// live key count.
+// Warps per CTA: kDecWarps when a (group, head) pair has many keys, two for
+// the short chunk-local decoder caches (where extra warps would idle).
+// About 2048 resident warps fill the GPU; when the pairs alone come short of
+// that the keys are cut into chunks of at least 128.  Planned for n_plan
+// keys when set (graph replays), so the grid never depends on the live key
+// count.
 DecPlan dec_plan(const AttnArgs& a) {
   const int n = a.n_plan > 0 ? a.n_plan : a.p0 + a.q_len;
-  const long long warps = (long long)a.G * a.H * kDecWarps;
+  const int w = n >= 192 ? kDecWarps : 2;
+  const long long warps = (long long)a.G * a.H * w;
   int splits = (int)((2048 + warps / 2) / warps);
   const int max_splits = (n + 127) / 128;
   if (splits > max_splits) splits = max_splits;
   if (splits < 1) splits = 1;
   const int chunk = (n + splits - 1) / splits;
   splits = (n + chunk - 1) / chunk;
-  return {chunk, splits};
+  return {chunk, splits, w};
 }
 
-template <typename T, int DH, int QMAX>
-void run_decode(const AttnArgs& a, const DecPlan& p, float* part, int* err, cudaStream_t s) {
-  constexpr int kRingBytes = kDecWarps * kDecStages * 2 * kDecU * 2 * 32 * 16;
+template <typename T, int DH, int QMAX, int W>
+void run_decode_w(const AttnArgs& a, const DecPlan& p, float* part, int* err, cudaStream_t s) {
+  constexpr int kRingBytes = W * kDecStages * 2 * kDecU * kDecSPL * 32 * 16;
   static bool configured = false;
   if (!configured) {
-    cudaFuncSetAttribute(k_attn_decode<T, DH, QMAX>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    cudaFuncSetAttribute(k_attn_decode<T, DH, QMAX, W>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                          kRingBytes);
     configured = true;
   }
   dim3 grid(p.splits, a.H, a.G);
-  launch_kernel(k_attn_decode<T, DH, QMAX>, grid, 32 * kDecWarps, kRingBytes, s, a, p.chunk,
-                p.splits, part, err);
+  launch_kernel(k_attn_decode<T, DH, QMAX, W>, grid, 32 * W, kRingBytes, s, a, p.chunk, p.splits,
+                part, err);
+}
+
+template <typename T, int DH, int QMAX>
+void run_decode(const AttnArgs& a, const DecPlan& p, float* part, int* err, cudaStream_t s) {
+  if (p.warps == 2)
+    run_decode_w<T, DH, QMAX, 2>(a, p, part, err, s);
+  else
+    run_decode_w<T, DH, QMAX, kDecWarps>(a, p, part, err, s);
   if (p.splits > 1) {
     dim3 cg(a.H, a.G * a.q_len);
     launch_kernel(k_attn_combine<T, DH>, cg, DH, 0, s, a, p.splits, part);

@@ -17,6 +17,7 @@
 // fixed order and applies the epilogue, so results are deterministic.
 #include <cuda.h>
 
+#include <cstdio>
 #include <cstdlib>
 #include <mutex>
 
@@ -345,6 +346,22 @@ __global__ void __launch_bounds__(128, 1)
 }
 
 // ------------------------------------------------------------------ persistent variant
+// Tile order of the persistent kernel: row-major (consecutive tiles share an
+// A row tile) or, with nt_major, column-major (consecutive tiles share a
+// weight tile, so the few row tiles of a small-M GEMM read it while it is
+// still in L2).
+__device__ __forceinline__ void tile_coords(int tile, int tiles_n, int n_tiles, int nt_major, int& mt,
+                                            int& nt) {
+  if (nt_major) {
+    const int tiles_m = n_tiles / tiles_n;
+    nt = tile / tiles_m;
+    mt = tile - nt * tiles_m;
+  } else {
+    mt = tile / tiles_n;
+    nt = tile - mt * tiles_n;
+  }
+}
+
 // For large M (prefill) one CTA per SM loops over 128 x BN output tiles
 // (row-major tile order, so the CTAs working at one moment share A tiles in
 // L2).  Warp 0 issues the TMA loads, warp 1 the MMAs, warps 2-5 drain the
@@ -354,7 +371,8 @@ __global__ void __launch_bounds__(128, 1)
 template <int BN, int STAGES>
 __global__ void __launch_bounds__(192, 1)
     k_gemm_tc_persist(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                      int M, int N, int nkb, int tiles_n, int n_tiles, Epilogue ep, int* err) {
+                      int M, int N, int nkb, int tiles_n, int n_tiles, int nt_major, Epilogue ep,
+                      int* err) {
   using Cfg = TcCfg<BN, STAGES>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -401,7 +419,8 @@ __global__ void __launch_bounds__(192, 1)
     if (lane == 0) {  // ---- TMA producer
       int it = 0;
       for (int tile = blockIdx.x; tile < n_tiles && !*abort_flag; tile += gridDim.x) {
-        const int mt = tile / tiles_n, nt = tile - mt * tiles_n;
+        int mt, nt;
+        tile_coords(tile, tiles_n, n_tiles, nt_major, mt, nt);
         for (int kb = 0; kb < nkb; ++kb, ++it) {
           const int st = it % STAGES;
           const uint32_t ph = (uint32_t)(it / STAGES) & 1u;
@@ -462,17 +481,34 @@ __global__ void __launch_bounds__(192, 1)
         break;
       }
       ptx::tc_fence_after();
-      const int mt = tile / tiles_n, nt = tile - mt * tiles_n;
+      int mt, nt;
+        tile_coords(tile, tiles_n, n_tiles, nt_major, mt, nt);
       const long long grow = (long long)mt * kBM + q * 32 + lane;
       const uint32_t trow = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(b * BN);
+      unsigned long long best = 0ull;
 #pragma unroll 1
       for (int j0 = 0; j0 < BN; j0 += 64) {
         float lo[32], hi[32];
         ptx::tmem_ld32(trow + (uint32_t)j0, lo);
         ptx::tmem_ld32(trow + (uint32_t)(j0 + 32), hi);
         const int gc = nt * BN + j0;
-        if (grow < M && gc < N) epi_row64(ep, grow, gc, lo, hi);
+        if (grow >= M || gc >= N) continue;
+        if (ep.kind == EPI_ARGMAX) {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            best = max(best, argmax_key(lo[i], gc + i));
+            best = max(best, argmax_key(hi[i], gc + 32 + i));
+          }
+          if (ep.out) {
+            float* o = reinterpret_cast<float*>(ep.out) + grow * ep.ldo + gc;
+            store32_f32(o, lo);
+            store32_f32(o + 32, hi);
+          }
+        } else {
+          epi_row64(ep, grow, gc, lo, hi);
+        }
       }
+      if (ep.kind == EPI_ARGMAX && grow < M) ep.argmax_part[grow * ep.argmax_tiles + nt] = best;
       ptx::tc_fence_before();
       __syncwarp();
       if (lane == 0) ptx::mbar_arrive(tempty_bar(b));
@@ -714,7 +750,7 @@ void run_tc(const CUtensorMap& ma, const CUtensorMap& mb, int grid_a, int grid_b
 
 template <int BN, int STAGES>
 void run_tc_persist(const CUtensorMap& ma, const CUtensorMap& mb, int M, int N, int nkb,
-                    const Epilogue& ep, int* err, cudaStream_t s) {
+                    const Epilogue& ep, int nt_major, int* err, cudaStream_t s) {
   using Cfg = TcCfg<BN, STAGES>;
   static int sms = 0;
   if (!sms) {
@@ -729,13 +765,16 @@ void run_tc_persist(const CUtensorMap& ma, const CUtensorMap& mb, int M, int N, 
   const int n_tiles = ((M + kBM - 1) / kBM) * tiles_n;
   const int grid = n_tiles < sms ? n_tiles : sms;
   launch_kernel(k_gemm_tc_persist<BN, STAGES>, dim3(grid), dim3(192), Cfg::kSmemBytes, s, ma, mb, M,
-                N, nkb, tiles_n, n_tiles, ep, err);
+                N, nkb, tiles_n, n_tiles, nt_major, ep, err);
 }
 
+// How many clusters of k_gemm_dec<BN, S, STAGES> can be resident at once
+// (0 if the cluster shape cannot be launched).  Host-side occupancy query,
+// made once per instance.
 template <int BN, int S, int STAGES>
-bool cluster_launchable() {
-  static int state = 0;  // 0 unknown, 1 yes, -1 no
-  if (state == 0) {
+int dec_max_clusters() {
+  static int n = -1;
+  if (n < 0) {
     using Cfg = TcCfg<BN, STAGES>;
     auto k = k_gemm_dec<BN, S, STAGES>;
     bool okf = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::kSmemBytes) ==
@@ -743,7 +782,7 @@ bool cluster_launchable() {
     if (S > 8)
       okf = okf && cudaFuncSetAttribute(k, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) ==
                        cudaSuccess;
-    int n = 0;
+    int c = 0;
     if (okf) {
       cudaLaunchConfig_t cfg = {};
       cfg.gridDim = dim3(S, 1, 1);
@@ -756,12 +795,15 @@ bool cluster_launchable() {
       attr[0].val.clusterDim.z = 1;
       cfg.attrs = attr;
       cfg.numAttrs = 1;
-      if (cudaOccupancyMaxActiveClusters(&n, k, &cfg) != cudaSuccess) n = 0;
+      if (cudaOccupancyMaxActiveClusters(&c, k, &cfg) != cudaSuccess) c = 0;
     }
     cudaGetLastError();
-    state = (okf && n > 0) ? 1 : -1;
+    n = okf ? c : 0;
+#ifdef PHOTON_GEMM_DEBUG
+    fprintf(stderr, "k_gemm_dec<%d,%d,%d>: %d clusters resident\n", BN, S, STAGES, n);
+#endif
   }
-  return state > 0;
+  return n;
 }
 
 template <int BN, int S, int STAGES>
@@ -786,9 +828,6 @@ void run_dec(const CUtensorMap& mw, const CUtensorMap& mx, int ga, int gb, int M
   note_launch();
 }
 
-// Cluster split-K for the swapped orientation: one token tile of BN >= M
-// rows, S CTAs per 128-feature tile with S chosen so the grid covers about
-// one CTA per SM.  Returns false when the shape is left to k_gemm_tc.
 bool cluster_enabled() {
   static const bool on = [] {
     const char* e = getenv("PHOTON_GEMM_CLUSTER");
@@ -797,33 +836,59 @@ bool cluster_enabled() {
   return on;
 }
 
-template <int BN, int STAGES>
+int dec_cluster_max() {
+  static const int v = [] {
+    const char* e = getenv("PHOTON_GEMM_CLUSTER_MAX");
+    const int x = e ? atoi(e) : 16;
+    return x >= 16 ? 16 : x >= 8 ? 8 : x >= 4 ? 4 : 2;
+  }();
+  return v;
+}
+
+// Token tile of the cluster kernel: 64 rows (several tiles when M > 64).
+constexpr int kDecBN = 64;
+constexpr int kDecStages = 4;
+
+// Cluster size for a few-token GEMM: the largest S (<= 16, <= the number of
+// K slices) such that all ga * gb clusters are resident at once and the grid
+// stays within two CTAs per SM.  1 means the shape is left to k_gemm_tc.
+int dec_cluster_size(int M, int N, int K) {
+  const int ga = (N + kBM - 1) / kBM, gb = (M + kDecBN - 1) / kDecBN, nkb = K / kBK;
+  const int tiles = ga * gb;
+  const int smax = dec_cluster_max();
+  const int cand[4] = {16, 8, 4, 2};
+  for (int c : cand) {
+    if (c > smax || c > nkb || tiles * c > 2 * 148) continue;
+    int fit = 0;
+    switch (c) {
+      case 16: fit = dec_max_clusters<kDecBN, 16, kDecStages>(); break;
+      case 8: fit = dec_max_clusters<kDecBN, 8, kDecStages>(); break;
+      case 4: fit = dec_max_clusters<kDecBN, 4, kDecStages>(); break;
+      default: fit = dec_max_clusters<kDecBN, 2, kDecStages>(); break;
+    }
+    if (tiles <= fit) return c;
+  }
+  return 1;
+}
+
+bool dec_path(int M, int N, int K, int force_splits, int force_swap) {
+  const bool swap = force_swap >= 0 ? (force_swap != 0) : (M <= 256);
+  return swap && force_splits <= 0 && M <= 256 && cluster_enabled() && dec_cluster_size(M, N, K) >= 2;
+}
+
 bool try_dec(const GemmArgs& a, int* err, cudaStream_t s) {
   const int M = a.M, N = a.N, nkb = a.K / kBK;
-  const int ga = (N + kBM - 1) / kBM;
-  int S = 1;
-  while (S < 16 && ga * S * 2 <= 148 && S * 2 <= nkb) S *= 2;
-  if (S == 16 && !cluster_launchable<BN, 16, STAGES>()) S = 8;
+  const int ga = (N + kBM - 1) / kBM, gb = (M + kDecBN - 1) / kDecBN;
+  const int S = dec_cluster_size(M, N, a.K);
   if (S < 2) return false;
   const int kbs = (nkb + S - 1) / S;
   CUtensorMap mw, mx;
-  if (!make_map(&mw, a.W, N, a.K, a.ldw, kBM) || !make_map(&mx, a.A, M, a.K, a.lda, BN)) return false;
+  if (!make_map(&mw, a.W, N, a.K, a.ldw, kBM) || !make_map(&mx, a.A, M, a.K, a.lda, kDecBN)) return false;
   switch (S) {
-    case 2:
-      if (!cluster_launchable<BN, 2, STAGES>()) return false;
-      run_dec<BN, 2, STAGES>(mw, mx, ga, 1, M, N, nkb, kbs, a.ep, err, s);
-      break;
-    case 4:
-      if (!cluster_launchable<BN, 4, STAGES>()) return false;
-      run_dec<BN, 4, STAGES>(mw, mx, ga, 1, M, N, nkb, kbs, a.ep, err, s);
-      break;
-    case 8:
-      if (!cluster_launchable<BN, 8, STAGES>()) return false;
-      run_dec<BN, 8, STAGES>(mw, mx, ga, 1, M, N, nkb, kbs, a.ep, err, s);
-      break;
-    default:
-      run_dec<BN, 16, STAGES>(mw, mx, ga, 1, M, N, nkb, kbs, a.ep, err, s);
-      break;
+    case 2: run_dec<kDecBN, 2, kDecStages>(mw, mx, ga, gb, M, N, nkb, kbs, a.ep, err, s); break;
+    case 4: run_dec<kDecBN, 4, kDecStages>(mw, mx, ga, gb, M, N, nkb, kbs, a.ep, err, s); break;
+    case 8: run_dec<kDecBN, 8, kDecStages>(mw, mx, ga, gb, M, N, nkb, kbs, a.ep, err, s); break;
+    default: run_dec<kDecBN, 16, kDecStages>(mw, mx, ga, gb, M, N, nkb, kbs, a.ep, err, s); break;
   }
   return true;
 }
@@ -839,11 +904,13 @@ struct Plan {
 Plan plan_for(int M, int N, int K, int force_splits, int force_swap, bool argmax) {
   Plan p;
   const int nkb = K / kBK;
-  p.swap = force_swap >= 0 ? (force_swap != 0) : (M <= 256);
+  // the vocabulary head (fused argmax) runs in the normal orientation on the
+  // persistent kernel: every 128-token row tile of a weight tile in a row
+  p.swap = force_swap >= 0 ? (force_swap != 0) : (!argmax && M <= 256);
   if (p.swap)
     p.bn = 64;  // token tiles of 64: M = 256 gives 4 CTAs per 128-feature tile
   else
-    p.bn = (N % 256 == 0 && M >= 4096) ? 256 : 128;
+    p.bn = (N % 256 == 0 && (M >= 4096 || argmax)) ? 256 : 128;
   const int ga = p.swap ? (N + kBM - 1) / kBM : (M + kBM - 1) / kBM;
   const int gb = p.swap ? (M + p.bn - 1) / p.bn : (N + p.bn - 1) / p.bn;
   const int tiles = ga * gb;
@@ -886,8 +953,10 @@ int gemm_tc_argmax_tiles(int M, int N, int K) {
   return p.swap ? p.ga : p.gb;
 }
 
-size_t gemm_tc_workspace_bytes(int M, int N, int K) {
-  const Plan p = plan_for(M, N, K, 0, -1, false);
+size_t gemm_tc_workspace_bytes(int M, int N, int K, int force_splits, int force_swap) {
+  if (M <= 0 || N <= 0 || K < kBK) return 0;
+  if (dec_path(M, N, K, force_splits, force_swap)) return 0;  // reduction stays on chip
+  const Plan p = plan_for(M, N, K, force_splits, force_swap, false);
   return p.splits > 1 ? (size_t)p.splits * M * N * sizeof(float) : 0;
 }
 
@@ -902,6 +971,10 @@ bool launch_gemm_tc(const GemmArgs& a, const GemmWorkspace& ws, int* err, cudaSt
   const bool argmax = a.ep.kind == EPI_ARGMAX;
   const Plan p = plan_for(M, N, K, argmax ? 1 : force_splits, force_swap, argmax);
   if (argmax && p.splits != 1) return false;
+  if (!argmax && dec_path(M, N, K, force_splits, force_swap)) {
+    // few tokens: cluster split-K with the reduction on chip
+    if (try_dec(a, err, s)) return true;
+  }
   float* part = nullptr;
   int* counters = nullptr;
   if (p.splits > 1) {
@@ -909,17 +982,6 @@ bool launch_gemm_tc(const GemmArgs& a, const GemmWorkspace& ws, int* err, cudaSt
     if (!ws.part || ws.bytes < need || !ws.counters || ws.n_counters < p.ga * p.gb) return false;
     part = ws.part;
     counters = ws.counters;
-  }
-  if (p.swap && force_splits <= 0 && !argmax && M <= 256 && cluster_enabled()) {
-    // few tokens: cluster split-K, the whole token range in one tile
-    bool done;
-    if (M <= 64)
-      done = try_dec<64, 4>(a, err, s);
-    else if (M <= 128)
-      done = try_dec<128, 4>(a, err, s);
-    else
-      done = try_dec<256, 3>(a, err, s);
-    if (done) return true;
   }
   CUtensorMap ma, mb;
   const int nkb = K / kBK;
@@ -933,11 +995,12 @@ bool launch_gemm_tc(const GemmArgs& a, const GemmWorkspace& ws, int* err, cudaSt
       run_tc<256, 4, true>(ma, mb, p.ga, p.gb, p.splits, M, N, nkb, p.kbs, a.ep, part, counters, a.W, a.ldw * 2, err, s);
   } else {
     if (!make_map(&ma, a.A, M, K, a.lda, kBM) || !make_map(&mb, a.W, N, K, a.ldw, p.bn)) return false;
-    if (p.splits == 1 && !argmax && p.ga * p.gb >= 2 * 148 && persistent_enabled()) {
+    if (p.splits == 1 && (argmax || p.ga * p.gb >= 2 * 148) && persistent_enabled()) {
+      const int nt_major = argmax ? 1 : 0;
       if (p.bn == 256)
-        run_tc_persist<256, 4>(ma, mb, M, N, nkb, a.ep, err, s);
+        run_tc_persist<256, 4>(ma, mb, M, N, nkb, a.ep, nt_major, err, s);
       else
-        run_tc_persist<128, 6>(ma, mb, M, N, nkb, a.ep, err, s);
+        run_tc_persist<128, 6>(ma, mb, M, N, nkb, a.ep, nt_major, err, s);
       return true;
     }
     if (p.bn == 256)

@@ -130,7 +130,7 @@ void launch_gemm_simt(int dt, const GemmArgs& a, cudaStream_t s);
 // tcgen05 path (bf16): returns false if the shape is not supported.
 bool launch_gemm_tc(const GemmArgs& a, const GemmWorkspace& ws, int* err, cudaStream_t s,
                     int force_splits = 0, int force_swap = -1);
-size_t gemm_tc_workspace_bytes(int M, int N, int K);
+size_t gemm_tc_workspace_bytes(int M, int N, int K, int force_splits = 0, int force_swap = -1);
 // Column tiles of the tcgen05 plan for an EPI_ARGMAX GEMM (0: not supported).
 int gemm_tc_argmax_tiles(int M, int N, int K);
 void launch_splitk_reduce(int dt, const float* part, int splits, int M, int N, const Epilogue& ep,

@@ -10,7 +10,7 @@
 // scratch array that lives in the library image itself.
 //
 // The scratch array below is a file-scope __device__ variable of
-// kNoAllocScratchBytes (1 MiB): every GPU that loads the library holds it
+// kNoAllocScratchBytes (256 KiB): every GPU that loads the library holds it
 // until the process exits.  Host code cannot use the array's name as a
 // device address, so the address is looked up once per device with
 // cudaGetSymbolAddress, during the first call made on that device (with
@@ -29,7 +29,7 @@
 
 namespace {
 
-constexpr size_t kNoAllocScratchBytes = 1u << 20;
+constexpr size_t kNoAllocScratchBytes = 256u << 10;
 constexpr int kMaxDevices = 64;
 
 static __device__ __align__(256) float g_noalloc_scratch[kNoAllocScratchBytes / sizeof(float)];

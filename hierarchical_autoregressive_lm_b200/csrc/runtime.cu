@@ -1204,14 +1204,15 @@ int photon_gemm(int32_t dtype, const void* d_A, int64_t lda, const void* d_W, in
     CK(cudaGetLastError());
     return PHOTON_OK;
   }
-  // generous scratch for any split count
-  const int nkb = K / 64 > 0 ? K / 64 : 1;
-  const size_t wsb = (size_t)nkb * M * N * sizeof(float);
+  // split-K scratch only when the plan needs it (partials + zeroed tile counters)
+  const size_t wsb = gemm_tc_workspace_bytes(M, N, K, splits > 0 ? splits : 0, swap);
   float* ws = nullptr;
   int* cnt = nullptr;
-  CK(pool_malloc((void**)&ws, wsb, s));
-  CK(pool_malloc((void**)&cnt, kGemmTileCounters * sizeof(int), s));
-  CK(cudaMemsetAsync(cnt, 0, kGemmTileCounters * sizeof(int), s));
+  if (wsb) {
+    CK(pool_malloc((void**)&ws, wsb, s));
+    CK(pool_malloc((void**)&cnt, kGemmTileCounters * sizeof(int), s));
+    CK(cudaMemsetAsync(cnt, 0, kGemmTileCounters * sizeof(int), s));
+  }
   GemmWorkspace w{ws, wsb, cnt, kGemmTileCounters};
   int* err = nullptr;
   bool ok = launch_gemm_tc(g, w, err, s, splits > 0 ? splits : 0, swap);
@@ -1219,8 +1220,8 @@ int photon_gemm(int32_t dtype, const void* d_A, int64_t lda, const void* d_W, in
     launch_gemm_simt(dtype, g, s);
     ok = true;
   }
-  cudaFreeAsync(ws, s);
-  cudaFreeAsync(cnt, s);
+  if (ws) cudaFreeAsync(ws, s);
+  if (cnt) cudaFreeAsync(cnt, s);
   if (!ok) return fail(PHOTON_ERR_ARG, "shape not supported by the tcgen05 kernel");
   CK(cudaGetLastError());
   return PHOTON_OK;

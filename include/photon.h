@@ -241,13 +241,13 @@ PHOTON_API int photon_attn_decode(int32_t dtype, const void* d_q, const void* d_
  * memory through its own pool, a latency-critical loop where an allocation
  * may synchronise the device, or a process close to its memory limit).
  * Same arguments, layouts and results as photon_attn_decode, but the split
- * scratch is a fixed 1 MiB array compiled into the library (held on every
+ * scratch is a fixed 256 KiB array compiled into the library (held on every
  * GPU that loads the library until the process exits); the call allocates
  * and frees nothing.  The array's device address is looked up during the
  * first call on each device, so make that first call before any stream
  * capture.  All calls share the array: calls whose GPU work may overlap
  * race on it and must be ordered by the caller.  Errors: ERR_ARG (bad
- * arguments), ERR_CAPACITY (the shape needs more than the 1 MiB of scratch;
+ * arguments), ERR_CAPACITY (the shape needs more than the 256 KiB of scratch;
  * the message says how much), ERR_CUDA. */
 PHOTON_API int photon_attn_decode_noalloc(int32_t dtype, const void* d_q, const void* d_k,
                                           const void* d_v, int32_t G, int32_t H, int32_t head_dim,

@@ -29,7 +29,7 @@ def test_noalloc_matches_allocating_entry_point_twice():
     # two calls in a row with few (group, head) pairs and long caches, so the
     # keys are cut into chunks whose partials live in the scratch array; the
     # second call's partials overlap what the first one left behind
-    for G, H, cap, p0, seed in ((8, 16, 900, 899, 1), (16, 16, 2200, 2111, 2)):
+    for G, H, cap, p0, seed in ((8, 16, 900, 899, 1), (4, 16, 2200, 2111, 2)):
         q, k, v = _case(G, H, cap, seed)
         ref = torch.zeros(G, H * 64, dtype=torch.bfloat16, device="cuda")
         got = torch.full_like(ref, float("nan"))
@@ -43,9 +43,10 @@ def test_noalloc_matches_allocating_entry_point_twice():
 
 
 def test_noalloc_rejects_shapes_beyond_its_scratch():
-    # 32 groups x 16 heads x 4 queries over 1104 keys: the chunk partials
-    # need more than the fixed 1 MiB
-    G, H, cap = 32, 16, 1104
+    # 10 groups x 16 heads x 4 queries over 1104 keys: the keys are cut in
+    # two chunks whose partials (4 queries x 160 pairs x 2 chunks x 66
+    # floats) need more than the fixed 256 KiB
+    G, H, cap = 10, 16, 1104
     q = torch.zeros(G * 4, H * 64, dtype=torch.bfloat16, device="cuda")
     k = torch.zeros(G, H, cap, 64, dtype=torch.bfloat16, device="cuda")
     out = torch.zeros_like(q)
