@@ -20,6 +20,9 @@ Reported (rank 0, one JSON line):
   roofline     the decode's dominant kernel (the weight-streaming tcgen05
                GEMM launches of one decode chunk) against the measured HBM
                copy peak; roofline_attention the same for the decode attention;
+               roofline_prefill the prefill's persistent GEMM against the
+               measured bf16 GEMM peak;
+  hiergen      HierGen decode of the same batch (one timed pass);
   cpu_baseline the CPU oracle timed on a bounded sample on the host cores.
 Between timed steps nothing is flushed: the step's working set (0.66 GB of
 decoder+top weights streamed per chunk, 0.9 GB of top KV) exceeds the 126 MB L2.
@@ -114,6 +117,7 @@ def run_gpu(args) -> None:
     import torch.distributed as dist
 
     import hierarchical_autoregressive_lm_b200 as hal
+    from hierarchical_autoregressive_lm_b200.dist import job_throughput, max_over_ranks, rank_rows
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -140,7 +144,8 @@ def run_gpu(args) -> None:
     if toks_all is None:
         from synth_inputs import zipf_tokens
         toks_all = zipf_tokens(B * world, T, wl["vocab"], wl["prompt_seed"])
-    toks_host = torch.from_numpy(np.ascontiguousarray(toks_all[rank * B:(rank + 1) * B]))
+    lo, hi = rank_rows(B, rank, world)
+    toks_host = torch.from_numpy(np.ascontiguousarray(toks_all[lo:hi]))
     toks = toks_host.to(dev)
     out = torch.empty(B, chunks * C, dtype=torch.int32, device=dev)
     stream = torch.cuda.current_stream()
@@ -227,18 +232,40 @@ def run_gpu(args) -> None:
     torch.cuda.synchronize()
     e2e_ms = e0.elapsed_time(e1)
 
+    # ---- HierGen decode of the same batch (one prefill + all chunks, after
+    # one untimed warm-up pass): reported beside the RecGen metric
+    def hier_pass(ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        c = model.prefill(toks, hal.MODE_HIER, chunks)
+        if ev is not None:
+            ev[1].record(stream)
+        for s in range(chunks):
+            c.step_hier(out[:, s * C:(s + 1) * C])
+        if ev is not None:
+            ev[2].record(stream)
+        return c
+    hier_pass().free()
+    hev = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+    torch.cuda.synchronize()
+    hc = hier_pass(hev)
+    torch.cuda.synchronize()
+    hier_kv = hc.info()["kv_bytes"]
+    hier_res = model.info()["resident_bytes"] + hier_kv
+    hc.free()
+    hier_dec_ms = hev[1].elapsed_time(hev[2])
+
     # ---- the decode's dominant kernel (its GEMM launches) and its attention,
     # alone, at the same shapes and launch configuration
     roof = measure_gemm_roofline(model, wl, dev, stream)
     roof_attn = measure_attn_roofline(model, wl, dev, stream)
+    roof_prefill = measure_prefill_roofline(model, wl, dev, stream)
 
-    times = torch.tensor([total_ms, prefill_ms, decode_ms, e2e_ms], device=dev, dtype=torch.float64)
-    if world > 1:
-        dist.all_reduce(times, op=dist.ReduceOp.MAX)
-    total_ms, prefill_ms, decode_ms, e2e_ms = times.tolist()
+    total_ms, prefill_ms, decode_ms, e2e_ms, hier_dec_ms = max_over_ranks(
+        [total_ms, prefill_ms, decode_ms, e2e_ms, hier_dec_ms], device=dev)
 
     dec_tokens = world * B * chunks * C * args.steps
-    value = dec_tokens / (decode_ms / 1e3)
+    value = job_throughput(B * chunks * C * args.steps, world, decode_ms)
     gib = resident / 2 ** 30
     line = {
         "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world,
@@ -262,9 +289,15 @@ def run_gpu(args) -> None:
         "e2e": {"value": round(world * B * chunks * C * e2e_steps / (e2e_ms / 1e3), 1), "unit": UNIT,
                 "h2d_bytes_per_step": int(B * T * 4), "d2h_bytes_per_step": int(B * chunks * C * 4),
                 "covers": "H2D prompt + prefill + RecGen decode + per-chunk D2H of tokens"},
+        "hiergen": {"decode_tok_s": round(job_throughput(B * chunks * C, world, hier_dec_ms), 1),
+                    "decode_ms_per_chunk": round(hier_dec_ms / chunks, 4),
+                    "resident_gib": round(hier_res / 2 ** 30, 4),
+                    "tok_s_per_gib": round(B * chunks * C / (hier_dec_ms / 1e3) / (hier_res / 2 ** 30), 1),
+                    "steps": 1},
         "gpu_launches": launches,
         "roofline": roof,
         "roofline_attention": roof_attn,
+        "roofline_prefill": roof_prefill,
         "clocks": clk.summary(),
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -334,6 +367,53 @@ def measure_gemm_roofline(model, wl, dev, stream) -> dict:
             "frac": round(achieved / peak, 4), "peak_source": f"{src} (STREAM-style copy)",
             "traffic": None, "launches": len(shapes),
             "bytes_per_launch": int(algo / len(shapes)),
+            "us_per_launch": round(ms * 1e3 / len(shapes), 3)}
+
+
+def measure_prefill_roofline(model, wl, dev, stream) -> dict:
+    """The prefill's dominant kernel (the persistent tcgen05 GEMM) alone at
+    the top encoder's prefill shapes: one block's QKV, O, W1 and W2
+    projections over M = B*T/C rows, replayed from a captured graph.
+    Algorithmic flops = 2*M*N*K per launch, against the measured bf16 GEMM
+    peak (burst: the launches are timed on their own)."""
+    import torch
+    import hierarchical_autoregressive_lm_b200 as hal
+    s = model.shape
+    d, f = s["d_model"], s["mlp_mult"] * s["d_model"]
+    M = wl["batch"] * wl["prompt_len"] // (s["C1"] * s["C2"])
+    shapes = [(M, 3 * d, d), (M, d, d), (M, f, d), (M, d, f)]
+    g = torch.Generator(device=dev).manual_seed(13)
+    bufs = [(torch.randn(m, k, device=dev, generator=g).to(torch.bfloat16),
+             torch.randn(n, k, device=dev, generator=g).to(torch.bfloat16),
+             torch.empty(m, n, device=dev)) for (m, n, k) in shapes]
+    for A, W, C in bufs:
+        hal.gemm(A, W, C)
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=torch.cuda.Stream()):
+        for A, W, C in bufs:
+            hal.gemm(A, W, C)
+    graph.replay()
+    torch.cuda.synchronize()
+    reps = 10
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    a.record()
+    for _ in range(reps):
+        graph.replay()
+    b.record()
+    torch.cuda.synchronize()
+    ms = a.elapsed_time(b) / reps
+    flops = sum(2 * m * n * k for (m, n, k) in shapes)
+    peaks, src = _peaks()
+    tf = flops / (ms / 1e3) / 1e12
+    del graph, bufs
+    return {"kernel": "k_gemm_tc_persist (prefill projections of one top-encoder block, "
+                      f"M={M})", "bound": "tensor", "achieved": round(tf, 1),
+            "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+            "frac": round(tf / peaks["bf16_tflops"], 4),
+            "peak_source": f"{src} (cuBLAS bf16 GEMM, burst)", "traffic": None,
+            "launches": len(shapes), "flops_per_launch": int(flops / len(shapes)),
             "us_per_launch": round(ms * 1e3 / len(shapes), 3)}
 
 

@@ -779,6 +779,9 @@ int dec_max_clusters() {
     auto k = k_gemm_dec<BN, S, STAGES>;
     bool okf = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::kSmemBytes) ==
                cudaSuccess;
+    // all of the unified L1/shared storage as shared memory: two CTAs per SM
+    okf = okf && cudaFuncSetAttribute(k, cudaFuncAttributePreferredSharedMemoryCarveout, 100) ==
+                     cudaSuccess;
     if (S > 8)
       okf = okf && cudaFuncSetAttribute(k, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) ==
                        cudaSuccess;
@@ -795,6 +798,13 @@ int dec_max_clusters() {
       attr[0].val.clusterDim.z = 1;
       cfg.attrs = attr;
       cfg.numAttrs = 1;
+#ifdef PHOTON_GEMM_LB
+      cudaLaunchAttribute attr2[2] = {attr[0], {}};
+      attr2[1].id = cudaLaunchAttributeClusterSchedulingPolicyPreference;
+      attr2[1].val.clusterSchedulingPolicyPreference = cudaClusterSchedulingPolicyLoadBalancing;
+      cfg.attrs = attr2;
+      cfg.numAttrs = 2;
+#endif
       if (cudaOccupancyMaxActiveClusters(&c, k, &cfg) != cudaSuccess) c = 0;
     }
     cudaGetLastError();
@@ -847,7 +857,10 @@ int dec_cluster_max() {
 
 // Token tile of the cluster kernel: 64 rows (several tiles when M > 64).
 constexpr int kDecBN = 64;
-constexpr int kDecStages = 4;
+#ifndef PHOTON_GEMM_DEC_STAGES
+#define PHOTON_GEMM_DEC_STAGES 4
+#endif
+constexpr int kDecStages = PHOTON_GEMM_DEC_STAGES;
 
 // Cluster size for a few-token GEMM: the largest S (<= 16, <= the number of
 // K slices) such that all ga * gb clusters are resident at once and the grid
