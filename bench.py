@@ -294,6 +294,8 @@ def run_gpu(args) -> None:
                     "resident_gib": round(hier_res / 2 ** 30, 4),
                     "tok_s_per_gib": round(B * chunks * C / (hier_dec_ms / 1e3) / (hier_res / 2 ** 30), 1),
                     "steps": 1},
+        "decode_graph": {"steps_replayed_per_cache": cinfo["graph_steps"], "steps_per_cache": chunks,
+                         "kernels_per_step": cinfo["graph_kernels"]},
         "gpu_launches": launches,
         "roofline": roof,
         "roofline_attention": roof_attn,

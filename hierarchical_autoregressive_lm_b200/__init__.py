@@ -16,7 +16,7 @@ import os
 from typing import Optional
 
 __all__ = ["PhotonError", "Model", "Cache", "load_library", "LIB_PATH", "MODE_HIER",
-           "MODE_REC", "STATE", "launch_count", "gemm", "attn_decode", "attn_decode_noalloc", "config_struct", "EXPORTED"]
+           "MODE_REC", "STATE", "launch_count", "gemm", "gemm_rmsnorm", "attn_decode", "attn_decode_noalloc", "config_struct", "EXPORTED"]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libphoton.so")
 
@@ -30,7 +30,7 @@ _ERRORS = {-1: "PHOTON_ERR_ARG", -2: "PHOTON_ERR_OOM", -3: "PHOTON_ERR_CUDA",
 EXPORTED = ("photon_init_weights", "photon_free_model", "photon_prefill",
             "photon_decode_step_hier", "photon_decode_step_rec", "photon_decode_step_ex",
             "photon_free_cache", "photon_cache_info", "photon_model_info",
-            "photon_export_weight", "photon_export_state", "photon_gemm",
+            "photon_export_weight", "photon_export_state", "photon_gemm", "photon_gemm_rmsnorm",
             "photon_attn_decode", "photon_attn_decode_noalloc", "photon_launch_count",
             "photon_last_error")
 
@@ -55,7 +55,8 @@ class photon_cache_stats(ctypes.Structure):
     _fields_ = [(n, ctypes.c_int32) for n in
                 ("B", "T", "mode", "N", "N1", "n_prefix", "n1_prefix", "capacity", "steps",
                  "max_new_chunks", "device_error", "l1_resident")] + \
-               [("kv_bytes", ctypes.c_uint64), ("workspace_bytes", ctypes.c_uint64)]
+               [("kv_bytes", ctypes.c_uint64), ("workspace_bytes", ctypes.c_uint64),
+                ("graph_steps", ctypes.c_int32), ("graph_kernels", ctypes.c_int32)]
 
 
 class photon_model_stats(ctypes.Structure):
@@ -91,6 +92,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "photon_export_weight": [P, I32, P, SZ, ctypes.POINTER(SZ), P],
         "photon_export_state": [P, I32, I32, P, SZ, ctypes.POINTER(SZ), P],
         "photon_gemm": [I32, P, I64, P, I64, I32, I32, I32, P, I64, I32, I32, I32, P],
+        "photon_gemm_rmsnorm": [P, I64, P, ctypes.c_float, P, I64, I32, I32, I32, P, I64, P],
         "photon_attn_decode": [I32, P, P, P, I32, I32, I32, I32, I32, I32, P, P],
         "photon_attn_decode_noalloc": [I32, P, P, P, I32, I32, I32, I32, I32, I32, P, P],
     }
@@ -250,6 +252,16 @@ def gemm(A, W, C, path: int = 0, splits: int = 0, swap: int = -1, stream=None) -
     N = W.shape[0]
     _check(load_library().photon_gemm(dt, _ptr(A), A.stride(0), _ptr(W), W.stride(0), M, N, K,
                                       _ptr(C), C.stride(0), path, splits, swap, _stream(stream)))
+
+
+def gemm_rmsnorm(x, g, W, C, eps: float = 1e-6, stream=None) -> None:
+    """C[M, N] (fp32) = bf16(RMSNorm(x; g, eps)) @ W[N, K]^T; x fp32 [M, K], g fp32 [K],
+    W bf16 [N, K] (the normalisation runs inside the GEMM where the kernel allows)."""
+    M, K = x.shape
+    N = W.shape[0]
+    _check(load_library().photon_gemm_rmsnorm(_ptr(x), x.stride(0), _ptr(g), float(eps), _ptr(W),
+                                              W.stride(0), M, N, K, _ptr(C), C.stride(0),
+                                              _stream(stream)))
 
 
 def attn_decode_noalloc(q, k, v, q_len: int, p0: int, out, stream=None) -> None:

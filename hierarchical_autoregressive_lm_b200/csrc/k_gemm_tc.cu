@@ -533,20 +533,50 @@ __global__ void __launch_bounds__(192, 1)
 // CTA r owns the RoPE pairs (f, f + 32) of the tile with pair index
 // u = (f / 64) * 32 + f % 64 in [r * 64 / S, (r + 1) * 64 / S), so the
 // QKV epilogue finds both values of a pair in one CTA.
-template <int BN, int S, int STAGES>
+//
+// NORM: the token operand is RMSNorm(x) of an fp32 residual stream x,
+// computed here instead of by a separate kernel.  Each CTA sums the squares
+// of its own K run of the BN rows, the S partial sums are added in rank
+// order through distributed shared memory (together the cluster covers the
+// whole row), and each CTA writes its normalised bf16 K run straight into
+// shared memory in the 128-byte-swizzled layout the MMA reads (all of it at
+// once: at most kDecMaxXBlocks slices).  The weight slices still stream
+// through the TMA ring meanwhile.
+constexpr int kDecMaxXBlocks = 8;
+
+template <int BN, int STAGES, bool NORM>
+struct DecCfg {
+  static constexpr int kWBytes = kBM * kBK * 2;  // 16 KB weight slice
+  static constexpr int kXBytes = BN * kBK * 2;   // token slice
+  static constexpr int kStageBytes = NORM ? kWBytes : kWBytes + kXBytes;
+  static constexpr int kRingBytes = STAGES * kStageBytes;
+  static constexpr int kXRegion = NORM ? kDecMaxXBlocks * kXBytes : 0;
+  static constexpr int kDataBytes = kRingBytes + kXRegion;
+  static constexpr int kCtrlBytes = 1024;  // barriers, TMEM slot, abort flag, row sums
+  static constexpr int kSmemBytes = kDataBytes + kCtrlBytes + 1024;  // + alignment slack
+  static constexpr uint32_t kTmemCols = BN;
+};
+
+template <int BN, int S, int STAGES, bool NORM>
 __global__ void __launch_bounds__(128, 1)
     k_gemm_dec(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX,
-               int M, int N, int nkb, int kbs, Epilogue ep, int* err) {
-  using Cfg = TcCfg<BN, STAGES>;
+               int M, int N, int nkb, int kbs, Epilogue ep, const float* __restrict__ nx,
+               long long nldx, const float* __restrict__ ng, float eps, int* err) {
+  using Cfg = DecCfg<BN, STAGES, NORM>;
   constexpr int LDP = BN + 4;  // partial-tile row stride in floats (16-byte skew per row)
-  static_assert(128 * LDP * 4 <= Cfg::kRingBytes, "the partial tile reuses the ring");
+  static_assert(128 * LDP * 4 <= Cfg::kDataBytes, "the partial tile reuses the data region");
   static_assert(64 % S == 0, "pairs must divide evenly over the cluster");
+  static_assert(!NORM || BN == 64, "the normalisation pass maps 64 token rows");
+  static_assert((2 * STAGES + 1) * 8 + 8 <= 256, "control block layout");
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Cfg::kRingBytes);
+  uint8_t* ctrl = smem + Cfg::kDataBytes;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(ctrl);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * STAGES + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  float* row_ssq = reinterpret_cast<float*>(ctrl + 256);  // [64] this CTA's partial sums
+  float* row_rstd = row_ssq + 64;                          // [64] 1 / rms of each row
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t rank = ptx::cluster_ctarank();
@@ -560,7 +590,11 @@ __global__ void __launch_bounds__(128, 1)
   auto empty_bar = [&](int st) { return ptx::smem_u32(bars + STAGES + st); };
   const uint32_t done_bar = ptx::smem_u32(bars + 2 * STAGES);
   auto w_tile = [&](int st) { return ptx::smem_u32(smem + st * Cfg::kStageBytes); };
-  auto x_tile = [&](int st) { return ptx::smem_u32(smem + st * Cfg::kStageBytes + kATileBytes); };
+  // token slice of K block `it` (held in stage it % STAGES, or in the NORM region)
+  auto x_tile = [&](int it) {
+    return NORM ? ptx::smem_u32(smem + Cfg::kRingBytes + it * Cfg::kXBytes)
+                : ptx::smem_u32(smem + (it % STAGES) * Cfg::kStageBytes + Cfg::kWBytes);
+  };
 
   if (threadIdx.x == 0) {
     for (int st = 0; st < STAGES; ++st) {
@@ -571,7 +605,7 @@ __global__ void __launch_bounds__(128, 1)
     *abort_flag = 0;
     ptx::fence_barrier_init();
     ptx::prefetch_tmap(&tmW);
-    ptx::prefetch_tmap(&tmX);
+    if (!NORM) ptx::prefetch_tmap(&tmX);
   }
   __syncwarp();
   if (warp == 0) {
@@ -587,15 +621,82 @@ __global__ void __launch_bounds__(128, 1)
   if (threadIdx.x != 0) pdl_wait();
   pdl_trigger();
 
+  const int pre = nk < STAGES ? nk : STAGES;
   if (threadIdx.x == 0) {
-    const int pre = nk < STAGES ? nk : STAGES;
     for (int it = 0; it < pre; ++it) {
       ptx::mbar_arrive_expect_tx(full_bar(it), (uint32_t)Cfg::kStageBytes);
       ptx::tma_load_2d(w_tile(it), &tmW, (kb0 + it) * kBK, a0, full_bar(it));
     }
     pdl_wait();
-    for (int it = 0; it < pre; ++it)
-      ptx::tma_load_2d(x_tile(it), &tmX, (kb0 + it) * kBK, b0, full_bar(it));
+    if (!NORM)
+      for (int it = 0; it < pre; ++it)
+        ptx::tma_load_2d(x_tile(it), &tmX, (kb0 + it) * kBK, b0, full_bar(it));
+  }
+
+  if constexpr (NORM) {
+    // ---- RMSNorm of the BN = 64 token rows, this CTA's K run into shared memory
+    const int t = threadIdx.x;
+    const int ch = t & 7;  // 16-byte chunk of a 64-column slice
+    const int kc0 = kb0 * kBK;
+    float part[4] = {0.f, 0.f, 0.f, 0.f};  // rows t / 8 + 16 j
+#pragma unroll 1
+    for (int it = 0; it < nk; ++it) {
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const long long grow = b0 + (t >> 3) + 16 * j;
+        if (grow < M) {
+          const float4* p = reinterpret_cast<const float4*>(nx + grow * nldx + kc0 + it * kBK + ch * 8);
+          const float4 u = p[0], v = p[1];
+          part[j] += u.x * u.x + u.y * u.y + u.z * u.z + u.w * u.w + v.x * v.x + v.y * v.y +
+                     v.z * v.z + v.w * v.w;
+        }
+      }
+    }
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+#pragma unroll
+      for (int o = 1; o < 8; o <<= 1) part[j] += __shfl_xor_sync(0xffffffffu, part[j], o);
+    }
+    if (ch == 0) {
+#pragma unroll
+      for (int j = 0; j < 4; ++j) row_ssq[(t >> 3) + 16 * j] = part[j];
+    }
+    ptx::cluster_sync();  // every CTA's partial sums are in place
+    if (t < 64) {
+      const uint32_t mine = ptx::smem_u32(row_ssq + t);
+      float tot = 0.f;
+#pragma unroll
+      for (int p = 0; p < S; ++p) tot += ptx::ld_shared_cluster_f32(ptx::map_shared_rank(mine, (uint32_t)p));
+      row_rstd[t] = 1.0f / sqrtf(tot / (float)(nkb * kBK) + eps);
+    }
+    __syncthreads();
+#pragma unroll 1
+    for (int it = 0; it < nk; ++it) {
+      uint8_t* xt = smem + Cfg::kRingBytes + it * Cfg::kXBytes;
+      const int col = kc0 + it * kBK + ch * 8;
+      const float4 g0 = reinterpret_cast<const float4*>(ng + col)[0];
+      const float4 g1 = reinterpret_cast<const float4*>(ng + col)[1];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int row = (t >> 3) + 16 * j;
+        const long long grow = b0 + row;
+        uint4 q = make_uint4(0u, 0u, 0u, 0u);
+        if (grow < M) {
+          const float4* p = reinterpret_cast<const float4*>(nx + grow * nldx + col);
+          const float4 u = p[0], v = p[1];
+          const float r = row_rstd[row];
+          q = make_uint4(pack2_bf16(u.x * r * g0.x, u.y * r * g0.y), pack2_bf16(u.z * r * g0.z, u.w * r * g0.w),
+                         pack2_bf16(v.x * r * g1.x, v.y * r * g1.y), pack2_bf16(v.z * r * g1.z, v.w * r * g1.w));
+        }
+        // 128-byte swizzle: the 16-byte chunk index is XORed with the row mod 8
+        *reinterpret_cast<uint4*>(xt + row * 128 + ((ch ^ (row & 7)) << 4)) = q;
+      }
+    }
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");  // visible to tcgen05.mma
+    __syncthreads();
+  }
+
+  if (threadIdx.x == 0) {
     for (int it = pre; it < nk; ++it) {
       const int st = it % STAGES;
       const uint32_t ph = (uint32_t)(it / STAGES) & 1u;
@@ -606,7 +707,7 @@ __global__ void __launch_bounds__(128, 1)
       }
       ptx::mbar_arrive_expect_tx(full_bar(st), (uint32_t)Cfg::kStageBytes);
       ptx::tma_load_2d(w_tile(st), &tmW, (kb0 + it) * kBK, a0, full_bar(st));
-      ptx::tma_load_2d(x_tile(st), &tmX, (kb0 + it) * kBK, b0, full_bar(st));
+      if (!NORM) ptx::tma_load_2d(x_tile(it), &tmX, (kb0 + it) * kBK, b0, full_bar(st));
     }
   } else if (threadIdx.x == 32 && nk > 0) {
     constexpr uint32_t idesc = ptx::idesc_bf16_f32(kBM, BN);
@@ -620,7 +721,7 @@ __global__ void __launch_bounds__(128, 1)
       }
       ptx::tc_fence_after();
       const uint64_t wd = ptx::sdesc_kmajor_sw128(w_tile(st));
-      const uint64_t xd = ptx::sdesc_kmajor_sw128(x_tile(st));
+      const uint64_t xd = ptx::sdesc_kmajor_sw128(x_tile(it));
 #pragma unroll
       for (int k = 0; k < kBK / 16; ++k)
         ptx::mma_bf16(tmem, wd + 2 * k, xd + 2 * k, idesc, (it > 0 || k > 0) ? 1u : 0u);
@@ -771,15 +872,17 @@ void run_tc_persist(const CUtensorMap& ma, const CUtensorMap& mb, int M, int N, 
 // How many clusters of k_gemm_dec<BN, S, STAGES> can be resident at once
 // (0 if the cluster shape cannot be launched).  Host-side occupancy query,
 // made once per instance.
-template <int BN, int S, int STAGES>
+// How many clusters of k_gemm_dec<BN, S, STAGES, NORM> can be resident at
+// once (0 if the cluster shape cannot be launched).  Host-side occupancy
+// query, made once per instance; it also sets the instance's attributes.
+template <int BN, int S, int STAGES, bool NORM>
 int dec_max_clusters() {
   static int n = -1;
   if (n < 0) {
-    using Cfg = TcCfg<BN, STAGES>;
-    auto k = k_gemm_dec<BN, S, STAGES>;
+    using Cfg = DecCfg<BN, STAGES, NORM>;
+    auto k = k_gemm_dec<BN, S, STAGES, NORM>;
     bool okf = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::kSmemBytes) ==
                cudaSuccess;
-    // all of the unified L1/shared storage as shared memory: two CTAs per SM
     okf = okf && cudaFuncSetAttribute(k, cudaFuncAttributePreferredSharedMemoryCarveout, 100) ==
                      cudaSuccess;
     if (S > 8)
@@ -798,28 +901,21 @@ int dec_max_clusters() {
       attr[0].val.clusterDim.z = 1;
       cfg.attrs = attr;
       cfg.numAttrs = 1;
-#ifdef PHOTON_GEMM_LB
-      cudaLaunchAttribute attr2[2] = {attr[0], {}};
-      attr2[1].id = cudaLaunchAttributeClusterSchedulingPolicyPreference;
-      attr2[1].val.clusterSchedulingPolicyPreference = cudaClusterSchedulingPolicyLoadBalancing;
-      cfg.attrs = attr2;
-      cfg.numAttrs = 2;
-#endif
       if (cudaOccupancyMaxActiveClusters(&c, k, &cfg) != cudaSuccess) c = 0;
     }
     cudaGetLastError();
     n = okf ? c : 0;
 #ifdef PHOTON_GEMM_DEBUG
-    fprintf(stderr, "k_gemm_dec<%d,%d,%d>: %d clusters resident\n", BN, S, STAGES, n);
+    fprintf(stderr, "k_gemm_dec<%d,%d,%d,%d>: %d clusters resident\n", BN, S, STAGES, (int)NORM, n);
 #endif
   }
   return n;
 }
 
-template <int BN, int S, int STAGES>
-void run_dec(const CUtensorMap& mw, const CUtensorMap& mx, int ga, int gb, int M, int N, int nkb,
-             int kbs, const Epilogue& ep, int* err, cudaStream_t s) {
-  using Cfg = TcCfg<BN, STAGES>;
+template <int BN, int S, int STAGES, bool NORM>
+void run_dec(const CUtensorMap& mw, const CUtensorMap& mx, int ga, int gb, const GemmArgs& a,
+             int kbs, int* err, cudaStream_t s) {
+  using Cfg = DecCfg<BN, STAGES, NORM>;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(ga * S, gb, 1);
   cfg.blockDim = dim3(128);
@@ -834,7 +930,8 @@ void run_dec(const CUtensorMap& mw, const CUtensorMap& mx, int ga, int gb, int M
   attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = pdl_enabled() ? 2 : 1;
-  cudaLaunchKernelEx(&cfg, k_gemm_dec<BN, S, STAGES>, mw, mx, M, N, nkb, kbs, ep, err);
+  cudaLaunchKernelEx(&cfg, k_gemm_dec<BN, S, STAGES, NORM>, mw, mx, a.M, a.N, a.K / kBK, kbs, a.ep,
+                     a.norm_x, a.norm_ld, a.norm_g, a.norm_eps, err);
   note_launch();
 }
 
@@ -862,47 +959,73 @@ constexpr int kDecBN = 64;
 #endif
 constexpr int kDecStages = PHOTON_GEMM_DEC_STAGES;
 
+template <int S>
+int dec_fit(bool norm) {
+  return norm ? dec_max_clusters<kDecBN, S, kDecStages, true>()
+              : dec_max_clusters<kDecBN, S, kDecStages, false>();
+}
+
 // Cluster size for a few-token GEMM: the largest S (<= 16, <= the number of
-// K slices) such that all ga * gb clusters are resident at once and the grid
-// stays within two CTAs per SM.  1 means the shape is left to k_gemm_tc.
-int dec_cluster_size(int M, int N, int K) {
+// K slices) whose ga * gb clusters are all resident at once, within two
+// CTAs per SM; if none fits, pairs (S = 2) in at most two waves, which
+// measured faster than k_gemm_tc for the 256-token projections.  With a
+// fused RMSNorm one CTA's K run must fit the token region (at most
+// kDecMaxXBlocks slices).  1 means the shape is left to k_gemm_tc.
+int dec_cluster_size(int M, int N, int K, bool norm) {
   const int ga = (N + kBM - 1) / kBM, gb = (M + kDecBN - 1) / kDecBN, nkb = K / kBK;
   const int tiles = ga * gb;
   const int smax = dec_cluster_max();
   const int cand[4] = {16, 8, 4, 2};
+  auto run_fits = [&](int c) { return !norm || (nkb + c - 1) / c <= kDecMaxXBlocks; };
   for (int c : cand) {
-    if (c > smax || c > nkb || tiles * c > 2 * 148) continue;
+    if (c > smax || c > nkb || tiles * c > 2 * 148 || !run_fits(c)) continue;
     int fit = 0;
     switch (c) {
-      case 16: fit = dec_max_clusters<kDecBN, 16, kDecStages>(); break;
-      case 8: fit = dec_max_clusters<kDecBN, 8, kDecStages>(); break;
-      case 4: fit = dec_max_clusters<kDecBN, 4, kDecStages>(); break;
-      default: fit = dec_max_clusters<kDecBN, 2, kDecStages>(); break;
+      case 16: fit = dec_fit<16>(norm); break;
+      case 8: fit = dec_fit<8>(norm); break;
+      case 4: fit = dec_fit<4>(norm); break;
+      default: fit = dec_fit<2>(norm); break;
     }
     if (tiles <= fit) return c;
   }
+  if (nkb >= 2 && run_fits(2) && tiles <= 2 * dec_fit<2>(norm)) return 2;
   return 1;
 }
 
-bool dec_path(int M, int N, int K, int force_splits, int force_swap) {
+bool dec_path(int M, int N, int K, int force_splits, int force_swap, bool norm = false) {
   const bool swap = force_swap >= 0 ? (force_swap != 0) : (M <= 256);
-  return swap && force_splits <= 0 && M <= 256 && cluster_enabled() && dec_cluster_size(M, N, K) >= 2;
+  return swap && force_splits <= 0 && M <= 256 && K % kBK == 0 && N % 64 == 0 && cluster_enabled() &&
+         dec_cluster_size(M, N, K, norm) >= 2;
 }
 
 bool try_dec(const GemmArgs& a, int* err, cudaStream_t s) {
   const int M = a.M, N = a.N, nkb = a.K / kBK;
+  const bool norm = a.norm_x != nullptr;
   const int ga = (N + kBM - 1) / kBM, gb = (M + kDecBN - 1) / kDecBN;
-  const int S = dec_cluster_size(M, N, a.K);
+  const int S = dec_cluster_size(M, N, a.K, norm);
   if (S < 2) return false;
   const int kbs = (nkb + S - 1) / S;
+  if (norm && (kbs > kDecMaxXBlocks || !a.norm_g || a.norm_ld % 4 ||
+               reinterpret_cast<uintptr_t>(a.norm_x) % 16 || reinterpret_cast<uintptr_t>(a.norm_g) % 16))
+    return false;
   CUtensorMap mw, mx;
-  if (!make_map(&mw, a.W, N, a.K, a.ldw, kBM) || !make_map(&mx, a.A, M, a.K, a.lda, kDecBN)) return false;
+  if (!make_map(&mw, a.W, N, a.K, a.ldw, kBM)) return false;
+  if (norm)
+    mx = mw;  // the token operand is built in shared memory
+  else if (!make_map(&mx, a.A, M, a.K, a.lda, kDecBN))
+    return false;
+#define PHOTON_RUN_DEC(SS)                                                       \
+  if (norm)                                                                      \
+    run_dec<kDecBN, SS, kDecStages, true>(mw, mx, ga, gb, a, kbs, err, s);       \
+  else                                                                           \
+    run_dec<kDecBN, SS, kDecStages, false>(mw, mx, ga, gb, a, kbs, err, s);
   switch (S) {
-    case 2: run_dec<kDecBN, 2, kDecStages>(mw, mx, ga, gb, M, N, nkb, kbs, a.ep, err, s); break;
-    case 4: run_dec<kDecBN, 4, kDecStages>(mw, mx, ga, gb, M, N, nkb, kbs, a.ep, err, s); break;
-    case 8: run_dec<kDecBN, 8, kDecStages>(mw, mx, ga, gb, M, N, nkb, kbs, a.ep, err, s); break;
-    default: run_dec<kDecBN, 16, kDecStages>(mw, mx, ga, gb, M, N, nkb, kbs, a.ep, err, s); break;
+    case 2: PHOTON_RUN_DEC(2) break;
+    case 4: PHOTON_RUN_DEC(4) break;
+    case 8: PHOTON_RUN_DEC(8) break;
+    default: PHOTON_RUN_DEC(16) break;
   }
+#undef PHOTON_RUN_DEC
   return true;
 }
 
@@ -966,6 +1089,11 @@ int gemm_tc_argmax_tiles(int M, int N, int K) {
   return p.swap ? p.ga : p.gb;
 }
 
+bool gemm_tc_fuses_norm(int M, int N, int K) {
+  if (M <= 0 || N <= 0 || K < kBK || !tma_available()) return false;
+  return dec_path(M, N, K, 0, -1, true);
+}
+
 size_t gemm_tc_workspace_bytes(int M, int N, int K, int force_splits, int force_swap) {
   if (M <= 0 || N <= 0 || K < kBK) return 0;
   if (dec_path(M, N, K, force_splits, force_swap)) return 0;  // reduction stays on chip
@@ -982,6 +1110,11 @@ bool launch_gemm_tc(const GemmArgs& a, const GemmWorkspace& ws, int* err, cudaSt
   if ((a.lda * 2) % 16 || (a.ldw * 2) % 16) return false;
   if (reinterpret_cast<uintptr_t>(a.A) % 16 || reinterpret_cast<uintptr_t>(a.W) % 16) return false;
   const bool argmax = a.ep.kind == EPI_ARGMAX;
+  if (a.norm_x) {
+    // fused RMSNorm: only the cluster kernel builds its own token operand
+    if (argmax || !dec_path(M, N, K, force_splits, force_swap, true)) return false;
+    return try_dec(a, err, s);
+  }
   const Plan p = plan_for(M, N, K, argmax ? 1 : force_splits, force_swap, argmax);
   if (argmax && p.splits != 1) return false;
   if (!argmax && dec_path(M, N, K, force_splits, force_swap)) {

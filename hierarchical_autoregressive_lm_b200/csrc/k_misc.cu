@@ -11,7 +11,7 @@
 namespace photon {
 
 static std::atomic<unsigned long long> g_launches{0};
-void note_launch(int n) { g_launches.fetch_add((unsigned long long)n, std::memory_order_relaxed); }
+void note_launch(long long n) { g_launches.fetch_add((unsigned long long)n, std::memory_order_relaxed); }
 unsigned long long launch_total() { return g_launches.load(std::memory_order_relaxed); }
 
 // Programmatic dependent launch is on unless PHOTON_PDL=0.

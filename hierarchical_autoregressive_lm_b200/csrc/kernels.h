@@ -53,6 +53,14 @@ struct GemmArgs {
   long long ldw = 0;
   int M = 0, N = 0, K = 0;
   Epilogue ep;
+  // Fused RMSNorm of the activation operand: when norm_x is set, A is not
+  // read; the kernel uses bf16(norm_x[row] / sqrt(mean(norm_x[row]^2) +
+  // norm_eps) * norm_g) instead (norm_x fp32 [M, K], row stride norm_ld).
+  // Only the tcgen05 few-token path accepts it (gemm_tc_fuses_norm).
+  const float* norm_x = nullptr;
+  long long norm_ld = 0;
+  const float* norm_g = nullptr;
+  float norm_eps = 0.f;
 };
 
 // Scratch the GEMM may use for split-K: fp32 partial tiles, and one counter
@@ -131,6 +139,8 @@ void launch_gemm_simt(int dt, const GemmArgs& a, cudaStream_t s);
 bool launch_gemm_tc(const GemmArgs& a, const GemmWorkspace& ws, int* err, cudaStream_t s,
                     int force_splits = 0, int force_swap = -1);
 size_t gemm_tc_workspace_bytes(int M, int N, int K, int force_splits = 0, int force_swap = -1);
+// True when launch_gemm_tc takes GemmArgs with norm_x set for this shape.
+bool gemm_tc_fuses_norm(int M, int N, int K);
 // Column tiles of the tcgen05 plan for an EPI_ARGMAX GEMM (0: not supported).
 int gemm_tc_argmax_tiles(int M, int N, int K);
 void launch_splitk_reduce(int dt, const float* part, int splits, int M, int N, const Epilogue& ep,
@@ -152,7 +162,7 @@ void set_error_message(const char* msg);
 
 // ---- launch accounting ------------------------------------------------------
 // Process-wide count of kernels this library has launched.
-void note_launch(int n = 1);
+void note_launch(long long n = 1);
 unsigned long long launch_total();
 
 // ---- TMA descriptors -----------------------------------------------------

@@ -95,6 +95,7 @@ struct photon_model {
   // cache's captured step updates the executable instead of instantiating.
   cudaGraphExec_t graph[2] = {nullptr, nullptr};
   const void* graph_owner[2] = {nullptr, nullptr};
+  long long graph_kernels[2] = {0, 0};  // kernel launches captured in graph[mode]
 
   const void* ptr(int idx) const { return group_ptr[t[idx].group] + t[idx].offset; }
   BlockW block(int first, int l) const {
@@ -304,11 +305,13 @@ struct photon_cache {
   int32_t* tok_out = nullptr;    // [B, C] greedy tokens of the last graph-replayed step
   // RecGen's top-encoder branch runs on its own stream with its own buffers
   cudaStream_t side = nullptr;
+  cudaStream_t cap = nullptr;  // the decode step is captured here (any caller stream can replay it)
   cudaEvent_t ev_fork = nullptr, ev_join = nullptr;
   void *xn_t = nullptr, *q_t = nullptr, *att_t = nullptr, *hid_t = nullptr;
   float* gemm_ws_t = nullptr;
   float* attn_ws_t = nullptr;
   bool graph_failed[2] = {false, false};
+  int graph_steps = 0;
   std::vector<void*> allocs;
   size_t kv_bytes = 0, ws_bytes = 0;
   bool has_a_hat = false, has_a = false;
@@ -369,6 +372,42 @@ static void gemm(photon_model* m, const Bufs& b, const void* A, long long lda, c
     launch_gemm_simt(m->dt, g, s);
 }
 
+// GEMM of a pre-norm projection: RMSNorm(x; g) * W^T.  The norm runs first
+// into b.xn; with PHOTON_FUSE_NORM=1 the few-token tcgen05 kernel
+// normalises its own operand instead.
+// Off by default: every weight-tile cluster of a wide projection would
+// normalise the same rows again (fp32 reads, twice), which measured slower
+// than one norm kernel writing a bf16 copy that the GEMM reads with TMA.
+static bool fuse_norm_enabled() {
+  static const bool on = [] {
+    const char* e = getenv("PHOTON_FUSE_NORM");
+    return e && e[0] == '1';
+  }();
+  return on;
+}
+
+static void gemm_normed(photon_model* m, const Bufs& b, const float* x, const float* g,
+                        const void* W, long long ldw, int M, int N, int K, const Epilogue& ep,
+                        cudaStream_t s) {
+  if (m->use_tc && fuse_norm_enabled() && gemm_tc_fuses_norm(M, N, K)) {
+    GemmArgs a;
+    a.W = W;
+    a.ldw = ldw;
+    a.M = M;
+    a.N = N;
+    a.K = K;
+    a.ep = ep;
+    a.norm_x = x;
+    a.norm_ld = K;
+    a.norm_g = g;
+    a.norm_eps = m->cfg.norm_eps;
+    GemmWorkspace ws{b.gemm_ws, b.gemm_ws_bytes, b.gemm_cnt, b.gemm_cnt ? kGemmTileCounters : 0};
+    if (launch_gemm_tc(a, ws, b.err, s)) return;
+  }
+  launch_rmsnorm(m->dt, x, g, b.xn, M, K, 1, 0, m->cfg.norm_eps, s);
+  gemm(m, b, b.xn, K, W, ldw, M, N, K, ep, s);
+}
+
 static Epilogue epi(int kind, void* out, long long ldo) {
   Epilogue e;
   e.kind = kind;
@@ -381,8 +420,6 @@ static Epilogue epi(int kind, void* out, long long ldo) {
 static void run_block(photon_model* m, const BlockW& w, float* x, const StackRun& r, int layer,
                       const Bufs& b, cudaStream_t s) {
   const int d = m->d, rows = r.G * r.q_len;
-  const float eps = m->cfg.norm_eps;
-  launch_rmsnorm(m->dt, x, w.g_attn, b.xn, rows, d, 1, 0, eps, s);
   Epilogue e;
   e.kind = EPI_QKV;
   e.q_out = b.q;
@@ -397,7 +434,7 @@ static void run_block(photon_model* m, const BlockW& w, float* x, const StackRun
   e.kv_off = r.kv_off;
   e.rope = b.rope;
   e.p0_dev = r.p0_dev;
-  gemm(m, b, b.xn, d, w.wqkv, d, rows, 3 * d, d, e, s);
+  gemm_normed(m, b, x, w.g_attn, w.wqkv, d, rows, 3 * d, d, e, s);
 
   AttnArgs a;
   a.Q = b.q;
@@ -426,8 +463,7 @@ static void run_block(photon_model* m, const BlockW& w, float* x, const StackRun
   if (!done) launch_attn_prefill(m->dt, a, s);
 
   gemm(m, b, b.att, d, w.wo, d, rows, d, d, epi(EPI_ADD_F32, x, d), s);
-  launch_rmsnorm(m->dt, x, w.g_mlp, b.xn, rows, d, 1, 0, eps, s);
-  gemm(m, b, b.xn, d, w.w1, d, rows, m->f, d, epi(EPI_GELU_T, b.hid, m->f), s);
+  gemm_normed(m, b, x, w.g_mlp, w.w1, d, rows, m->f, d, epi(EPI_GELU_T, b.hid, m->f), s);
   gemm(m, b, b.hid, m->f, w.w2, m->f, rows, d, m->f, epi(EPI_ADD_F32, x, d), s);
 }
 
@@ -639,6 +675,7 @@ int photon_prefill(photon_model* m, const photon_cache* prefix, const int32_t* d
   auto bail = [&](int code) {
     cudaGetLastError();
     if (c->side) cudaStreamDestroy(c->side);
+    if (c->cap) cudaStreamDestroy(c->cap);
     if (c->ev_fork) cudaEventDestroy(c->ev_fork);
     if (c->ev_join) cudaEventDestroy(c->ev_join);
     free_list(c->allocs, s);
@@ -718,6 +755,7 @@ int photon_prefill(photon_model* m, const photon_cache* prefix, const int32_t* d
   c->gemm_cnt_t = al.get<int>(kGemmTileCounters * sizeof(int));
   c->attn_ws_t = al.get<float>(aw);
   if (cudaStreamCreateWithFlags(&c->side, cudaStreamNonBlocking) != cudaSuccess ||
+      cudaStreamCreateWithFlags(&c->cap, cudaStreamNonBlocking) != cudaSuccess ||
       cudaEventCreateWithFlags(&c->ev_fork, cudaEventDisableTiming) != cudaSuccess ||
       cudaEventCreateWithFlags(&c->ev_join, cudaEventDisableTiming) != cudaSuccess)
     return bail(fail(PHOTON_ERR_CUDA, "stream/event creation failed"));
@@ -1013,17 +1051,26 @@ int photon_decode_step_ex(photon_model* m, photon_cache* c, int32_t mode, int32_
   const int C2 = m->C2;
   // The plain step (no hooks, no logits) is captured once per mode, after
   // one eager step has configured every kernel, and replayed afterwards.
+  // Capture runs on the cache's own stream (capturing executes nothing), so
+  // the caller's stream may be any stream, the legacy default one included;
+  // the graph is launched on the caller's stream.
   const bool plain = !d_out_logits && !d_force_tokens && !d_force_a;
-  bool replay = plain && s != nullptr && graphs_enabled() && c->steps >= 1 && !c->graph_failed[mode];
+  bool replay = plain && c->cap != nullptr && graphs_enabled() && c->steps >= 1 && !c->graph_failed[mode];
   if (replay && m->graph_owner[mode] != c) {
     // capture this cache's step; update the model's executable in place when
     // the topology matches, otherwise instantiate a new one
     cudaGraph_t g = nullptr;
-    bool ok = cudaStreamBeginCapture(s, cudaStreamCaptureModeRelaxed) == cudaSuccess;
+    // the launch counter counts kernels that run: captured launches are
+    // taken back here and added again at every replay
+    const unsigned long long n0 = launch_total();
+    bool ok = cudaStreamBeginCapture(c->cap, cudaStreamCaptureModeRelaxed) == cudaSuccess;
     if (ok) {
-      enqueue_decode(m, c, mode, c->tok_out, nullptr, nullptr, nullptr, s);
-      ok = cudaStreamEndCapture(s, &g) == cudaSuccess && g;
+      enqueue_decode(m, c, mode, c->tok_out, nullptr, nullptr, nullptr, c->cap);
+      ok = cudaStreamEndCapture(c->cap, &g) == cudaSuccess && g;
     }
+    const long long captured = (long long)(launch_total() - n0);
+    note_launch(-captured);
+    m->graph_kernels[mode] = ok ? captured : 0;
     if (ok && m->graph[mode]) {
       cudaGraphExecUpdateResultInfo info;
       if (cudaGraphExecUpdate(m->graph[mode], g, &info) != cudaSuccess) {
@@ -1046,6 +1093,8 @@ int photon_decode_step_ex(photon_model* m, photon_cache* c, int32_t mode, int32_
   }
   if (replay) {
     CK(cudaGraphLaunch(m->graph[mode], s));
+    note_launch(m->graph_kernels[mode]);
+    c->graph_steps += 1;
     CK(cudaMemcpyAsync(d_out_tokens, c->tok_out, (size_t)c->B * m->C * sizeof(int32_t),
                        cudaMemcpyDeviceToDevice, s));
   } else {
@@ -1086,6 +1135,7 @@ int photon_free_cache(photon_cache* c) {
     cudaStreamSynchronize(c->side);
     cudaStreamDestroy(c->side);
   }
+  if (c->cap) cudaStreamDestroy(c->cap);  // only ever captured into, never run
   if (c->ev_fork) cudaEventDestroy(c->ev_fork);
   if (c->ev_join) cudaEventDestroy(c->ev_join);
   free_list(c->allocs, c->stream);
@@ -1118,6 +1168,10 @@ int photon_cache_info(photon_cache* c, photon_cache_stats* out) {
   out->l1_resident = c->l1_k != nullptr;
   out->kv_bytes = c->kv_bytes;
   out->workspace_bytes = c->ws_bytes;
+  out->graph_steps = c->graph_steps;
+  out->graph_kernels = (c->mode >= 0 && c->mode < 2 && c->m->graph_owner[c->mode] == c)
+                           ? (int32_t)c->m->graph_kernels[c->mode]
+                           : 0;
   return PHOTON_OK;
 }
 
@@ -1223,6 +1277,58 @@ int photon_gemm(int32_t dtype, const void* d_A, int64_t lda, const void* d_W, in
   if (ws) cudaFreeAsync(ws, s);
   if (cnt) cudaFreeAsync(cnt, s);
   if (!ok) return fail(PHOTON_ERR_ARG, "shape not supported by the tcgen05 kernel");
+  CK(cudaGetLastError());
+  return PHOTON_OK;
+}
+
+int photon_gemm_rmsnorm(const float* d_x, int64_t ldx, const float* d_g, float eps, const void* d_W,
+                        int64_t ldw, int32_t M, int32_t N, int32_t K, float* d_C, int64_t ldc,
+                        void* stream) {
+  g_err.clear();
+  if (!d_x || !d_g || !d_W || !d_C || M <= 0 || N <= 0 || K <= 0 || ldx < K || ldw < K || ldc < N ||
+      !(eps >= 0.f))
+    return fail(PHOTON_ERR_ARG, "bad GEMM arguments");
+  if (ldx % 4 || reinterpret_cast<uintptr_t>(d_x) % 16 || reinterpret_cast<uintptr_t>(d_g) % 16)
+    return fail(PHOTON_ERR_ARG, "x rows and g must be 16-byte aligned");
+  cudaStream_t s = (cudaStream_t)stream;
+  GemmArgs g;
+  g.W = d_W;
+  g.ldw = ldw;
+  g.M = M;
+  g.N = N;
+  g.K = K;
+  g.ep = epi(EPI_STORE_F32, d_C, ldc);
+  if (tma_available() && gemm_tc_fuses_norm(M, N, K)) {
+    g.norm_x = d_x;
+    g.norm_ld = ldx;
+    g.norm_g = d_g;
+    g.norm_eps = eps;
+    GemmWorkspace w{nullptr, 0, nullptr, 0};
+    if (!launch_gemm_tc(g, w, nullptr, s)) return fail(PHOTON_ERR_ARG, "fused RMSNorm GEMM rejected the shape");
+    CK(cudaGetLastError());
+    return PHOTON_OK;
+  }
+  // separate norm into a bf16 copy, then the library's GEMM (the norm
+  // kernel reads rows with stride K)
+  if (ldx != K) return fail(PHOTON_ERR_ARG, "this shape takes the unfused path, which needs ldx == K");
+  void* xn = nullptr;
+  CK(pool_malloc(&xn, (size_t)M * K * 2, s));
+  launch_rmsnorm(DT_BF16, d_x, d_g, xn, M, K, 1, 0, eps, s);
+  g.A = xn;
+  g.lda = K;
+  const size_t wsb = gemm_tc_workspace_bytes(M, N, K);
+  float* ws = nullptr;
+  int* cnt = nullptr;
+  if (wsb) {
+    CK(pool_malloc((void**)&ws, wsb, s));
+    CK(pool_malloc((void**)&cnt, kGemmTileCounters * sizeof(int), s));
+    CK(cudaMemsetAsync(cnt, 0, kGemmTileCounters * sizeof(int), s));
+  }
+  GemmWorkspace w{ws, wsb, cnt, kGemmTileCounters};
+  launch_gemm(DT_BF16, g, w, nullptr, s);
+  if (ws) cudaFreeAsync(ws, s);
+  if (cnt) cudaFreeAsync(cnt, s);
+  cudaFreeAsync(xn, s);
   CK(cudaGetLastError());
   return PHOTON_OK;
 }

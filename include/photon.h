@@ -172,6 +172,8 @@ typedef struct photon_cache_stats {
   int32_t l1_resident;  /* 1 while the level-1 KV is allocated */
   uint64_t kv_bytes;    /* top + level-1 KV allocated for this cache */
   uint64_t workspace_bytes;
+  int32_t graph_steps;  /* decode steps replayed from a captured CUDA graph */
+  int32_t graph_kernels; /* kernels in that graph (0 before the first capture) */
 } photon_cache_stats;
 
 /* Cache bookkeeping.  Synchronises the cache's last stream to read the
@@ -224,6 +226,22 @@ PHOTON_API int photon_export_state(photon_cache* c, int32_t which, int32_t layer
 PHOTON_API int photon_gemm(int32_t dtype, const void* d_A, int64_t lda, const void* d_W, int64_t ldw,
                 int32_t M, int32_t N, int32_t K, float* d_C, int64_t ldc, int32_t path,
                 int32_t splits, int32_t swap, void* stream);
+
+/* Kernel-level entry for the pre-norm projection of every encoder and
+ * decoder block (each block normalises its residual stream before the
+ * attention and MLP projections; RMSNorm is this library's reading of the
+ * norm): C[M, N] (fp32, row stride ldc) = bf16(RMSNorm(x)) * W[N, K]^T with
+ * RMSNorm(x)[r, k] = x[r, k] / sqrt(mean_k x[r, k]^2 + eps) * g[k].
+ * x: fp32 [M, K] (row stride ldx elements, 16-byte aligned rows), g: fp32
+ * [K], W: bf16 [N, K] (row stride ldw).  bf16 only.  Runs the few-token
+ * tcgen05 kernel that normalises its own operand; where that kernel does not
+ * take the shape (see gemm_tc_fuses_norm: M <= 256, K % 64 == 0, N % 64 == 0,
+ * a cluster plan exists) the norm runs as a separate kernel before the
+ * GEMM, with the same result up to the order of the sum of squares.
+ * Allocates its scratch internally.  Errors: ERR_ARG (bad arguments). */
+PHOTON_API int photon_gemm_rmsnorm(const float* d_x, int64_t ldx, const float* d_g, float eps,
+                                   const void* d_W, int64_t ldw, int32_t M, int32_t N, int32_t K,
+                                   float* d_C, int64_t ldc, void* stream);
 
 /* Kernel-level entry: split-K decode attention (the top-encoder decode
  * kernel).  For G groups x H heads, q_len <= 4 new queries at positions

@@ -107,3 +107,27 @@ def test_attn_decode_bf16(G, H, cap, q_len, p0):
 def test_attn_decode_fp32(G, H, cap, q_len, p0):
     got, ref = _attn_case(torch.float32, G, H, 32, cap, q_len, p0, 20)
     np.testing.assert_allclose(got, ref, rtol=1e-5, atol=1e-5)
+
+
+# (M, N, K): fused RMSNorm in the cluster kernel (clusters of 2..8, ragged M,
+# CTAs without K slices, the 8-slice maximum run) and, for M > 256, the
+# separate norm kernel followed by the GEMM
+@pytest.mark.parametrize("M,N,K", [(64, 3072, 1024), (256, 4096, 1024), (3, 384, 128),
+                                   (100, 1024, 1024), (64, 1024, 640), (300, 512, 256)])
+def test_gemm_rmsnorm_bf16(M, N, K):
+    x = _rand((M, K), torch.float32, 30, scale=3.0)
+    g = 1.0 + 0.1 * _rand((K,), torch.float32, 31)
+    W = _rand((N, K), torch.bfloat16, 32)
+    C = torch.full((M, N), float("nan"), device="cuda")
+    hal.gemm_rmsnorm(x.cuda(), g.cuda(), W.cuda(), C, eps=1e-6)
+    torch.cuda.synchronize()
+    # the kernel feeds bf16(RMSNorm(x)) to the tensor cores: round the fp64
+    # oracle norm the same way, then multiply in fp64
+    xn = oracle.rmsnorm(x.double().numpy(), g.double().numpy(), 1e-6)
+    xn = torch.from_numpy(xn).to(torch.bfloat16).double().numpy()
+    ref = xn @ W.double().numpy().T
+    got = C.cpu().double().numpy()
+    assert np.isfinite(got).all()
+    # fp32 accumulation, plus the odd operand rounded the other way (1 bf16
+    # ulp of one normalised element)
+    np.testing.assert_allclose(got, ref, rtol=0, atol=2e-3 * np.abs(ref).max())

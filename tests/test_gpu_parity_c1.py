@@ -157,8 +157,11 @@ def test_c1_graph_replay_equals_eager(model, mode):
     none = torch.full((1, CFG.C), -1, dtype=torch.int32, device="cuda")
     og = torch.empty(1, CFG.C, dtype=torch.int32, device="cuda")
     oe = torch.empty_like(og)
-    for _ in range(STEPS):
+    for k in range(STEPS):
         g.decode_step(mode, og)
+        # steps after the first replay the captured graph, although the
+        # caller uses the default stream
+        assert g.info()["graph_steps"] == k
         e.decode_step(mode, oe, force_tokens=none)
         torch.cuda.synchronize()
         assert torch.equal(og, oe)
@@ -166,6 +169,7 @@ def test_c1_graph_replay_equals_eager(model, mode):
         assert torch.equal(g.export_state("top_k", l), e.export_state("top_k", l))
     assert torch.equal(g.export_state("pending_o"), e.export_state("pending_o"))
     assert g.info()["N"] == e.info()["N"]
+    assert e.info()["graph_steps"] == 0 and g.info()["graph_kernels"] > 0
     g.free(); e.free()
 
 

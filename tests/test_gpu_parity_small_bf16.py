@@ -85,8 +85,16 @@ def test_small_bf16_graph_replay_equals_eager():
     none = torch.full((B, CFG.C), -1, dtype=torch.int32, device="cuda")
     og = torch.empty(B, CFG.C, dtype=torch.int32, device="cuda")
     oe = torch.empty_like(og)
-    for _ in range(4):
-        g.decode_step(hal.MODE_REC, og)
+    side = torch.cuda.Stream()
+    for k in range(4):
+        if k == 3:
+            # the captured step replays on any stream the caller uses
+            with torch.cuda.stream(side):
+                g.decode_step(hal.MODE_REC, og)
+            torch.cuda.current_stream().wait_stream(side)
+        else:
+            g.decode_step(hal.MODE_REC, og)
+        assert g.info()["graph_steps"] == k  # replayed from the graph after the first step
         e.decode_step(hal.MODE_REC, oe, force_tokens=none)
         torch.cuda.synchronize()
         assert torch.equal(og, oe)
