@@ -135,6 +135,19 @@ def run_gpu(args) -> None:
     shape = model_shape(args.workload)
     B, T = wl["batch"], wl["prompt_len"]
     model = hal.Model(shape, WEIGHT_SEED)
+    if args.only_roofline:
+        # the three roofline measurements alone (a few GB on the device): the
+        # small case the kernel-level profiles are captured on
+        stream = torch.cuda.current_stream()
+        if rank == 0:
+            print(json.dumps({"roofline": measure_gemm_roofline(model, wl, dev, stream),
+                              "roofline_attention": measure_attn_roofline(model, wl, dev, stream),
+                              "roofline_prefill": measure_prefill_roofline(model, wl, dev, stream)}),
+                  flush=True)
+        model.free()
+        if world > 1:
+            dist.destroy_process_group()
+        return
     C = model.C
     chunks = wl["decode_tokens"] // C
     # data parallel over sequences: every rank decodes its own batch of B
@@ -297,9 +310,9 @@ def run_gpu(args) -> None:
         "decode_graph": {"steps_replayed_per_cache": cinfo["graph_steps"], "steps_per_cache": chunks,
                          "kernels_per_step": cinfo["graph_kernels"]},
         "gpu_launches": launches,
-        "roofline": roof,
-        "roofline_attention": roof_attn,
-        "roofline_prefill": roof_prefill,
+        "roofline": _with_traffic(roof, "roofline"),
+        "roofline_attention": _with_traffic(roof_attn, "roofline_attention"),
+        "roofline_prefill": _with_traffic(roof_prefill, "roofline_prefill"),
         "clocks": clk.summary(),
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -309,6 +322,46 @@ def run_gpu(args) -> None:
     model.free()
     if world > 1:
         dist.destroy_process_group()
+
+
+def kernel_sources_sha256() -> str:
+    """sha256 over the relative path and bytes of every kernel source and
+    public header, sorted by path (the key under which profiled DRAM
+    traffic stays valid)."""
+    import glob
+    import hashlib
+    files = sorted(glob.glob(os.path.join(ROOT, "hierarchical_autoregressive_lm_b200", "csrc", "*.cu"))
+                   + glob.glob(os.path.join(ROOT, "hierarchical_autoregressive_lm_b200", "csrc", "*.cuh"))
+                   + glob.glob(os.path.join(ROOT, "hierarchical_autoregressive_lm_b200", "csrc", "*.h"))
+                   + glob.glob(os.path.join(ROOT, "include", "*.h")))
+    h = hashlib.sha256()
+    for f in files:
+        h.update(os.path.relpath(f, ROOT).encode())
+        with open(f, "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()
+
+
+def profiled_traffic() -> dict:
+    """Per-launch DRAM bytes of the roofline kernels from the committed ncu
+    summary, or {} when the kernels changed since it was taken."""
+    path = os.path.join(ROOT, "profiles", "roofline_traffic.txt")
+    if not os.path.exists(path):
+        return {}
+    vals = {}
+    for line in open(path):
+        line = line.strip()
+        if line and not line.startswith("#"):
+            k, v = line.split()[:2]
+            vals[k] = v
+    if vals.get("kernel_sources_sha256") != kernel_sources_sha256():
+        return {}
+    return {k: int(v) for k, v in vals.items() if k != "kernel_sources_sha256"}
+
+
+def _with_traffic(roof: dict, key: str) -> dict:
+    roof["traffic"] = profiled_traffic().get(key)
+    return roof
 
 
 def _peak_gbs():
@@ -353,18 +406,21 @@ def measure_gemm_roofline(model, wl, dev, stream) -> dict:
     reps = 10
     a = torch.cuda.Event(enable_timing=True)
     b = torch.cuda.Event(enable_timing=True)
+    torch.cuda.nvtx.range_push("roofline_gemm")
     a.record()
     for _ in range(reps):
         graph.replay()
     b.record()
+    torch.cuda.nvtx.range_pop()
     torch.cuda.synchronize()
     ms = a.elapsed_time(b) / reps
     algo = sum(N * K * 2 + M * K * 2 + M * N * 4 for (M, N, K) in shapes)
     peak, src = _peak_gbs()
     achieved = algo / (ms / 1e3) / 1e9
     del graph, bufs
-    return {"kernel": "k_gemm_tc<64,4,swapped> (decode weight streaming: top encoder, level-2 "
-                      "decoder, token-decoder steps, converters, Chunker_2 of one decode chunk)",
+    return {"kernel": "decode weight-streaming GEMMs (k_gemm_dec cluster split-K; k_gemm_tc where "
+                      "no cluster plan fits): top encoder, level-2 decoder, token-decoder steps, "
+                      "converters, Chunker_2 of one decode chunk",
             "bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
             "frac": round(achieved / peak, 4), "peak_source": f"{src} (STREAM-style copy)",
             "traffic": None, "launches": len(shapes),
@@ -400,10 +456,12 @@ def measure_prefill_roofline(model, wl, dev, stream) -> dict:
     reps = 10
     a = torch.cuda.Event(enable_timing=True)
     b = torch.cuda.Event(enable_timing=True)
+    torch.cuda.nvtx.range_push("roofline_prefill")
     a.record()
     for _ in range(reps):
         graph.replay()
     b.record()
+    torch.cuda.nvtx.range_pop()
     torch.cuda.synchronize()
     ms = a.elapsed_time(b) / reps
     flops = sum(2 * m * n * k for (m, n, k) in shapes)
@@ -446,7 +504,7 @@ def measure_attn_roofline(model, wl, dev, stream) -> dict:
     a = torch.cuda.Event(enable_timing=True)
     b = torch.cuda.Event(enable_timing=True)
     a.record(stream)
-    torch.cuda.nvtx.range_push("roofline")
+    torch.cuda.nvtx.range_push("roofline_attn")
     for r in range(reps):
         for l in range(L):
             hal.attn_decode(q, K[l], V[l], 1, n_mid - 1, o)
@@ -543,6 +601,8 @@ def main() -> None:
     ap.add_argument("--impl", default="photon", choices=["photon", "reference"])
     ap.add_argument("--cpu-budget", type=float, default=20.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--only-roofline", action="store_true",
+                    help="run only the kernel roofline measurements (profiling case)")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl != "reference":
         args.warmup = 3
