@@ -293,6 +293,7 @@ def run_gpu(args) -> None:
         "decode_ms_per_step": round(decode_ms / args.steps, 3),
         "decode_ms_per_chunk": round(decode_ms / args.steps / chunks, 4),
         "prefill_tok_s": round(world * B * T * args.steps / (prefill_ms / 1e3), 1),
+        "prefill_ms_steps": [round(e[0].elapsed_time(e[1]), 3) for e in evs],
         "job_tok_s": round(dec_tokens / (total_ms / 1e3), 1),
         "tpm": {"tok_s_per_gib": round(value / world / gib, 1), "resident_gib": round(gib, 4),
                 "weights_gib": round(minfo["resident_bytes"] / 2 ** 30, 4),

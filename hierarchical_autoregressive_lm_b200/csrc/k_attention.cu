@@ -650,18 +650,118 @@ static bool tc_attn_disabled() {
   return off;
 }
 
+bool local_attn_ok(const AttnArgs& a);  // short local caches take k_attn_local (no scratch)
+
 size_t attn_decode_workspace_bytes(int dt, const AttnArgs& a) {
   (void)dt;
-  if (a.G <= 0 || a.q_len <= 0) return 0;
+  if (a.G <= 0 || a.q_len <= 0 || local_attn_ok(a)) return 0;
   const DecPlan p = dec_plan(a);
   if (p.splits <= 1) return 0;
   return (size_t)a.G * a.q_len * a.H * p.splits * (a.dh + 2) * sizeof(float);
+}
+
+// ------------------------------------------------------------------ short local caches
+// The chunk-local decoders attend over at most 2*C1 - 1 (token decoder) or
+// C2 (level-2 decoder) keys.  One warp per (group, head): every lane holds
+// DH/32 dimensions of all keys, values and queries in registers, the q.k
+// partial sums are reduced across the warp (each lane ends with every
+// score), and the causal softmax and P.V run in registers.  Eight pairs per
+// CTA, so the grid is a few hundred CTAs instead of one CTA per pair.
+constexpr int kLocalMaxKeys = 16;
+constexpr int kLocalWarps = 4;
+
+template <typename T, int DH, int QMAX, int KEYS>
+__global__ void __launch_bounds__(32 * kLocalWarps) k_attn_local(AttnArgs a) {
+  constexpr int E = DH / 32;  // dimensions per lane
+  pdl_wait();
+  pdl_trigger();
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const long long pair = (long long)blockIdx.x * kLocalWarps + warp;
+  if (pair >= (long long)a.G * a.H) return;
+  const int g = (int)(pair / a.H), h = (int)(pair - (long long)g * a.H);
+  const int p0 = a.p0;
+  const int n = p0 + a.q_len;  // keys visible to the last query (<= KEYS)
+  const T* kb = reinterpret_cast<const T*>(a.K) + ((long long)g * a.H + h) * a.cap * DH + lane * E;
+  const T* vb = reinterpret_cast<const T*>(a.V) + ((long long)g * a.H + h) * a.cap * DH + lane * E;
+  float kf[KEYS][E], vf[KEYS][E];
+#pragma unroll
+  for (int j = 0; j < KEYS; ++j) {
+#pragma unroll
+    for (int e = 0; e < E; ++e) {
+      kf[j][e] = j < n ? Elem<T>::to_f(kb[(long long)j * DH + e]) : 0.f;
+      vf[j][e] = j < n ? Elem<T>::to_f(vb[(long long)j * DH + e]) : 0.f;
+    }
+  }
+#pragma unroll
+  for (int qi = 0; qi < QMAX; ++qi) {
+    if (qi >= a.q_len) break;
+    const long long row = (long long)g * a.q_len + qi;
+    const T* qr = reinterpret_cast<const T*>(a.Q) + row * a.q_ld + h * DH + lane * E;
+    float qf[E];
+#pragma unroll
+    for (int e = 0; e < E; ++e) qf[e] = Elem<T>::to_f(qr[e]) * a.scale;
+    const int vis = p0 + qi + 1;  // causal: keys 0 .. p0 + qi
+    float sc[KEYS];
+    float mx = -INFINITY;
+#pragma unroll
+    for (int j = 0; j < KEYS; ++j) {
+      float d = 0.f;
+#pragma unroll
+      for (int e = 0; e < E; ++e) d = fmaf(qf[e], kf[j][e], d);
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) d += __shfl_xor_sync(0xffffffffu, d, o);
+      sc[j] = j < vis ? d : -INFINITY;
+      mx = fmaxf(mx, sc[j]);
+    }
+    float l = 0.f, acc[E];
+#pragma unroll
+    for (int e = 0; e < E; ++e) acc[e] = 0.f;
+#pragma unroll
+    for (int j = 0; j < KEYS; ++j) {
+      const float p = j < vis ? __expf(sc[j] - mx) : 0.f;
+      l += p;
+#pragma unroll
+      for (int e = 0; e < E; ++e) acc[e] = fmaf(p, vf[j][e], acc[e]);
+    }
+    T* o = reinterpret_cast<T*>(a.O) + row * a.o_ld + h * DH + lane * E;
+#pragma unroll
+    for (int e = 0; e < E; ++e) st_f(o + e, acc[e] / l);
+  }
+}
+
+bool local_attn_ok(const AttnArgs& a) {
+  return a.Kp == nullptr && a.p0_dev == nullptr && a.p0 + a.q_len <= kLocalMaxKeys && a.q_len <= 4 &&
+         (a.dh == 32 || a.dh == 64);
+}
+
+template <typename T, int DH>
+void run_local(const AttnArgs& a, cudaStream_t s) {
+  const long long pairs = (long long)a.G * a.H;
+  const dim3 grid((unsigned)((pairs + kLocalWarps - 1) / kLocalWarps));
+  const bool few = a.p0 + a.q_len <= 8;
+  if (a.q_len == 1)
+    few ? launch_kernel(k_attn_local<T, DH, 1, 8>, grid, 32 * kLocalWarps, 0, s, a)
+        : launch_kernel(k_attn_local<T, DH, 1, 16>, grid, 32 * kLocalWarps, 0, s, a);
+  else
+    few ? launch_kernel(k_attn_local<T, DH, 4, 8>, grid, 32 * kLocalWarps, 0, s, a)
+        : launch_kernel(k_attn_local<T, DH, 4, 16>, grid, 32 * kLocalWarps, 0, s, a);
 }
 
 bool launch_attn_decode(int dt, const AttnArgs& a, float* part, size_t part_bytes, int* err,
                         cudaStream_t s) {
   if (a.G <= 0 || a.q_len <= 0) return true;
   if (a.q_len > 4) return false;
+  if (local_attn_ok(a)) {
+    if (dt == DT_BF16 && a.dh == 64)
+      run_local<bf16, 64>(a, s);
+    else if (dt == DT_F32 && a.dh == 32)
+      run_local<float, 32>(a, s);
+    else if (dt == DT_F32 && a.dh == 64)
+      run_local<float, 64>(a, s);
+    else
+      run_local<bf16, 32>(a, s);
+    return true;
+  }
   const DecPlan p = dec_plan(a);
   if (p.splits > 1 && (part == nullptr || part_bytes < attn_decode_workspace_bytes(dt, a)))
     return false;

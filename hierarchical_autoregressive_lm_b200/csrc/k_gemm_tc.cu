@@ -921,15 +921,25 @@ void run_dec(const CUtensorMap& mw, const CUtensorMap& mx, int ga, int gb, const
   cfg.blockDim = dim3(128);
   cfg.dynamicSmemBytes = Cfg::kSmemBytes;
   cfg.stream = s;
-  cudaLaunchAttribute attr[2];
+  cudaLaunchAttribute attr[3];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = S;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
-  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[1].val.programmaticStreamSerializationAllowed = 1;
+  int n = 1;
+  if (pdl_enabled()) {
+    attr[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[n].val.programmaticStreamSerializationAllowed = 1;
+    ++n;
+  }
+  int prio = 0;
+  if (s != nullptr && cudaStreamGetPriority(s, &prio) == cudaSuccess && prio != 0) {
+    attr[n].id = cudaLaunchAttributePriority;
+    attr[n].val.priority = prio;
+    ++n;
+  }
   cfg.attrs = attr;
-  cfg.numAttrs = pdl_enabled() ? 2 : 1;
+  cfg.numAttrs = n;
   cudaLaunchKernelEx(&cfg, k_gemm_dec<BN, S, STAGES, NORM>, mw, mx, a.M, a.N, a.K / kBK, kbs, a.ep,
                      a.norm_x, a.norm_ld, a.norm_g, a.norm_eps, err);
   note_launch();
@@ -953,16 +963,27 @@ int dec_cluster_max() {
 }
 
 // Token tile of the cluster kernel: 64 rows (several tiles when M > 64).
-constexpr int kDecBN = 64;
+// PHOTON_GEMM_DEC_BN=128 selects 128-row tiles for M > 64 (fewer clusters
+// per projection; measured slower in the decode chain).
 #ifndef PHOTON_GEMM_DEC_STAGES
 #define PHOTON_GEMM_DEC_STAGES 4
 #endif
 constexpr int kDecStages = PHOTON_GEMM_DEC_STAGES;
 
+int dec_bn(int M, bool norm) {
+  static const int forced = [] {
+    const char* e = getenv("PHOTON_GEMM_DEC_BN");
+    return e ? atoi(e) : 0;
+  }();
+  if (norm || M <= 64 || forced != 128) return 64;
+  return 128;
+}
+
 template <int S>
-int dec_fit(bool norm) {
-  return norm ? dec_max_clusters<kDecBN, S, kDecStages, true>()
-              : dec_max_clusters<kDecBN, S, kDecStages, false>();
+int dec_fit(int bn, bool norm) {
+  if (norm) return dec_max_clusters<64, S, kDecStages, true>();
+  return bn == 64 ? dec_max_clusters<64, S, kDecStages, false>()
+                  : dec_max_clusters<128, S, kDecStages, false>();
 }
 
 // Cluster size for a few-token GEMM: the largest S (<= 16, <= the number of
@@ -972,7 +993,8 @@ int dec_fit(bool norm) {
 // fused RMSNorm one CTA's K run must fit the token region (at most
 // kDecMaxXBlocks slices).  1 means the shape is left to k_gemm_tc.
 int dec_cluster_size(int M, int N, int K, bool norm) {
-  const int ga = (N + kBM - 1) / kBM, gb = (M + kDecBN - 1) / kDecBN, nkb = K / kBK;
+  const int bn = dec_bn(M, norm);
+  const int ga = (N + kBM - 1) / kBM, gb = (M + bn - 1) / bn, nkb = K / kBK;
   const int tiles = ga * gb;
   const int smax = dec_cluster_max();
   const int cand[4] = {16, 8, 4, 2};
@@ -981,27 +1003,49 @@ int dec_cluster_size(int M, int N, int K, bool norm) {
     if (c > smax || c > nkb || tiles * c > 2 * 148 || !run_fits(c)) continue;
     int fit = 0;
     switch (c) {
-      case 16: fit = dec_fit<16>(norm); break;
-      case 8: fit = dec_fit<8>(norm); break;
-      case 4: fit = dec_fit<4>(norm); break;
-      default: fit = dec_fit<2>(norm); break;
+      case 16: fit = dec_fit<16>(bn, norm); break;
+      case 8: fit = dec_fit<8>(bn, norm); break;
+      case 4: fit = dec_fit<4>(bn, norm); break;
+      default: fit = dec_fit<2>(bn, norm); break;
     }
     if (tiles <= fit) return c;
   }
-  if (nkb >= 2 && run_fits(2) && tiles <= 2 * dec_fit<2>(norm)) return 2;
+  if (nkb >= 2 && run_fits(2) && tiles <= 2 * dec_fit<2>(bn, norm)) return 2;
   return 1;
 }
 
+int dec_max_m() {
+  static const int v = [] {
+    const char* e = getenv("PHOTON_GEMM_DEC_MMAX");
+    const int x = e ? atoi(e) : 1024;
+    return x < 64 ? 64 : x;
+  }();
+  return v;
+}
+
 bool dec_path(int M, int N, int K, int force_splits, int force_swap, bool norm = false) {
-  const bool swap = force_swap >= 0 ? (force_swap != 0) : (M <= 256);
-  return swap && force_splits <= 0 && M <= 256 && K % kBK == 0 && N % 64 == 0 && cluster_enabled() &&
+  const int mmax = dec_max_m();
+  const bool swap = force_swap >= 0 ? (force_swap != 0) : (M <= mmax);
+  return swap && force_splits <= 0 && M <= mmax && K % kBK == 0 && N % 64 == 0 && cluster_enabled() &&
          dec_cluster_size(M, N, K, norm) >= 2;
+}
+
+template <int BN, bool NORM>
+void run_dec_s(int S, const CUtensorMap& mw, const CUtensorMap& mx, int ga, int gb, const GemmArgs& a,
+               int kbs, int* err, cudaStream_t s) {
+  switch (S) {
+    case 2: run_dec<BN, 2, kDecStages, NORM>(mw, mx, ga, gb, a, kbs, err, s); break;
+    case 4: run_dec<BN, 4, kDecStages, NORM>(mw, mx, ga, gb, a, kbs, err, s); break;
+    case 8: run_dec<BN, 8, kDecStages, NORM>(mw, mx, ga, gb, a, kbs, err, s); break;
+    default: run_dec<BN, 16, kDecStages, NORM>(mw, mx, ga, gb, a, kbs, err, s); break;
+  }
 }
 
 bool try_dec(const GemmArgs& a, int* err, cudaStream_t s) {
   const int M = a.M, N = a.N, nkb = a.K / kBK;
   const bool norm = a.norm_x != nullptr;
-  const int ga = (N + kBM - 1) / kBM, gb = (M + kDecBN - 1) / kDecBN;
+  const int bn = dec_bn(M, norm);
+  const int ga = (N + kBM - 1) / kBM, gb = (M + bn - 1) / bn;
   const int S = dec_cluster_size(M, N, a.K, norm);
   if (S < 2) return false;
   const int kbs = (nkb + S - 1) / S;
@@ -1012,20 +1056,14 @@ bool try_dec(const GemmArgs& a, int* err, cudaStream_t s) {
   if (!make_map(&mw, a.W, N, a.K, a.ldw, kBM)) return false;
   if (norm)
     mx = mw;  // the token operand is built in shared memory
-  else if (!make_map(&mx, a.A, M, a.K, a.lda, kDecBN))
+  else if (!make_map(&mx, a.A, M, a.K, a.lda, bn))
     return false;
-#define PHOTON_RUN_DEC(SS)                                                       \
-  if (norm)                                                                      \
-    run_dec<kDecBN, SS, kDecStages, true>(mw, mx, ga, gb, a, kbs, err, s);       \
-  else                                                                           \
-    run_dec<kDecBN, SS, kDecStages, false>(mw, mx, ga, gb, a, kbs, err, s);
-  switch (S) {
-    case 2: PHOTON_RUN_DEC(2) break;
-    case 4: PHOTON_RUN_DEC(4) break;
-    case 8: PHOTON_RUN_DEC(8) break;
-    default: PHOTON_RUN_DEC(16) break;
-  }
-#undef PHOTON_RUN_DEC
+  if (norm)
+    run_dec_s<64, true>(S, mw, mx, ga, gb, a, kbs, err, s);
+  else if (bn == 64)
+    run_dec_s<64, false>(S, mw, mx, ga, gb, a, kbs, err, s);
+  else
+    run_dec_s<128, false>(S, mw, mx, ga, gb, a, kbs, err, s);
   return true;
 }
 

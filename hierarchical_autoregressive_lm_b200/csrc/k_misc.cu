@@ -321,6 +321,76 @@ void launch_argmax_partials(const unsigned long long* part, int tiles, int rows,
                 force, own, used, next_ids, err);
 }
 
+// Greedy choice from the head's tile partials (as k_argmax_partials), then,
+// for the next single-row step of the token decoder, the chosen token's
+// embedding row written as the step's fp32 residual input x and its RMSNorm
+// (the first block's attention norm) written as the bf16 operand xn: three
+// row-local operations in one launch.  The norm sums squares in the same
+// order as k_rmsnorm, so x and xn are bitwise those of the separate kernels.
+template <typename T>
+__global__ void k_argmax_embed_norm(const unsigned long long* __restrict__ part, int tiles, int rows,
+                                    int V, int step, int C1, const int32_t* __restrict__ force,
+                                    int32_t* own, int32_t* used, int32_t* next_ids, int* err,
+                                    const T* __restrict__ E, float* __restrict__ x,
+                                    const float* __restrict__ g, T* __restrict__ xn, int d, float eps) {
+  pdl_wait();
+  pdl_trigger();
+  const int row = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  if (row >= rows) return;
+  unsigned long long k = 0ull;
+  for (int t = lane; t < tiles; t += 32) k = max(k, part[(long long)row * tiles + t]);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) k = max(k, __shfl_xor_sync(0xffffffffu, k, o));
+  int bi = (int)(0xFFFFFFFFu - (uint32_t)(k & 0xFFFFFFFFull));
+  bool bad = (k == 0ull || bi < 0 || bi >= V);
+  if (bad) bi = 0;
+  const long long slot = (long long)row * C1 + step;
+  int u = bi;
+  if (force) {
+    const int f = force[slot];
+    if (f >= 0) u = (f < V) ? f : 0;
+    if (f >= V) bad = true;
+  }
+  if (lane == 0) {
+    if (bad) report_error(err, DEV_BAD_TOKEN);
+    if (own) own[slot] = bi;
+    if (used) used[slot] = u;
+    if (next_ids) next_ids[row] = u;
+  }
+  const T* src = E + (long long)u * d;
+  float* xr = x + (long long)row * d;
+  float ss = 0.f;
+  for (int c = lane * 4; c < d; c += 128) {
+    const float4 v = make_float4(ld_f(src + c), ld_f(src + c + 1), ld_f(src + c + 2), ld_f(src + c + 3));
+    *reinterpret_cast<float4*>(xr + c) = v;
+    ss += v.x * v.x + v.y * v.y + v.z * v.z + v.w * v.w;
+  }
+  ss = warp_sum(ss);
+  const float r = 1.0f / sqrtf(ss / (float)d + eps);
+  T* o = xn + (long long)row * d;
+  for (int c = lane * 4; c < d; c += 128) {
+    const float4 gg = *reinterpret_cast<const float4*>(g + c);
+    st_f(o + c + 0, ld_f(src + c) * r * gg.x);
+    st_f(o + c + 1, ld_f(src + c + 1) * r * gg.y);
+    st_f(o + c + 2, ld_f(src + c + 2) * r * gg.z);
+    st_f(o + c + 3, ld_f(src + c + 3) * r * gg.w);
+  }
+}
+void launch_argmax_embed_norm(int dt, const unsigned long long* part, int tiles, int rows, int V, int i,
+                              int C1, const int32_t* force, int32_t* own, int32_t* used,
+                              int32_t* next_ids, int* err, const void* E, float* x, const float* g,
+                              void* xn, int d, float eps, cudaStream_t s) {
+  if (rows <= 0) return;
+  const int blocks = (rows * 32 + 255) / 256;
+  if (dt == DT_F32)
+    launch_kernel(k_argmax_embed_norm<float>, blocks, 256, 0, s, part, tiles, rows, V, i, C1, force, own,
+                  used, next_ids, err, (const float*)E, x, g, (float*)xn, d, eps);
+  else
+    launch_kernel(k_argmax_embed_norm<bf16>, blocks, 256, 0, s, part, tiles, rows, V, i, C1, force, own,
+                  used, next_ids, err, (const bf16*)E, x, g, (bf16*)xn, d, eps);
+}
+
 __global__ void k_advance(int* pos, int dN, int dN1) {
   pdl_wait();
   pdl_trigger();

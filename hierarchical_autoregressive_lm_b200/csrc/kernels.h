@@ -126,6 +126,12 @@ void launch_argmax(const float* logits, long long ld, int rows, int V, int i, in
                    cudaStream_t s);
 // Greedy token per row from the head GEMM's per-tile partials (EPI_ARGMAX);
 // same outputs as launch_argmax.
+// argmax from tile partials + embedding of the chosen token into x + its
+// RMSNorm into xn (d % 4 == 0)
+void launch_argmax_embed_norm(int dt, const unsigned long long* part, int tiles, int rows, int V, int i,
+                              int C1, const int32_t* force, int32_t* own, int32_t* used,
+                              int32_t* next_ids, int* err, const void* E, float* x, const float* g,
+                              void* xn, int d, float eps, cudaStream_t s);
 void launch_argmax_partials(const unsigned long long* part, int tiles, int rows, int V, int i,
                             int C1, const int32_t* force, int32_t* own, int32_t* used,
                             int32_t* next_ids, int* err, cudaStream_t s);

@@ -256,6 +256,11 @@ static int release_encoder(photon_model* m, cudaStream_t s) {
 }
 
 // ============================================================== cache
+static int stream_priority_high() {
+  int least = 0, greatest = 0;
+  if (cudaDeviceGetStreamPriorityRange(&least, &greatest) != cudaSuccess) return 0;
+  return greatest;
+}
 struct Bufs {
   void* xn;
   void* q;
@@ -306,7 +311,8 @@ struct photon_cache {
   // RecGen's top-encoder branch runs on its own stream with its own buffers
   cudaStream_t side = nullptr;
   cudaStream_t cap = nullptr;  // the decode step is captured here (any caller stream can replay it)
-  cudaEvent_t ev_fork = nullptr, ev_join = nullptr;
+  cudaStream_t hi = nullptr;   // high-priority stream for the RecGen token branch
+  cudaEvent_t ev_fork = nullptr, ev_join = nullptr, ev_join_hi = nullptr;
   void *xn_t = nullptr, *q_t = nullptr, *att_t = nullptr, *hid_t = nullptr;
   float* gemm_ws_t = nullptr;
   float* attn_ws_t = nullptr;
@@ -352,6 +358,7 @@ struct StackRun {
   int cap_pre = 0, n_pre = 0;
   const int* p0_dev = nullptr;  // device position of the first row (added to p0)
   int n_plan = 0;               // key count the decode attention is planned for
+  bool xn_ready = false;        // the first block's attention norm is already in b.xn
 };
 
 static void gemm(photon_model* m, const Bufs& b, const void* A, long long lda, const void* W,
@@ -388,7 +395,11 @@ static bool fuse_norm_enabled() {
 
 static void gemm_normed(photon_model* m, const Bufs& b, const float* x, const float* g,
                         const void* W, long long ldw, int M, int N, int K, const Epilogue& ep,
-                        cudaStream_t s) {
+                        cudaStream_t s, bool xn_ready = false) {
+  if (xn_ready) {  // a fused row kernel already wrote RMSNorm(x) into b.xn
+    gemm(m, b, b.xn, K, W, ldw, M, N, K, ep, s);
+    return;
+  }
   if (m->use_tc && fuse_norm_enabled() && gemm_tc_fuses_norm(M, N, K)) {
     GemmArgs a;
     a.W = W;
@@ -434,7 +445,7 @@ static void run_block(photon_model* m, const BlockW& w, float* x, const StackRun
   e.kv_off = r.kv_off;
   e.rope = b.rope;
   e.p0_dev = r.p0_dev;
-  gemm_normed(m, b, x, w.g_attn, w.wqkv, d, rows, 3 * d, d, e, s);
+  gemm_normed(m, b, x, w.g_attn, w.wqkv, d, rows, 3 * d, d, e, s, r.xn_ready && layer == 0);
 
   AttnArgs a;
   a.Q = b.q;
@@ -676,7 +687,9 @@ int photon_prefill(photon_model* m, const photon_cache* prefix, const int32_t* d
     cudaGetLastError();
     if (c->side) cudaStreamDestroy(c->side);
     if (c->cap) cudaStreamDestroy(c->cap);
+    if (c->hi) cudaStreamDestroy(c->hi);
     if (c->ev_fork) cudaEventDestroy(c->ev_fork);
+    if (c->ev_join_hi) cudaEventDestroy(c->ev_join_hi);
     if (c->ev_join) cudaEventDestroy(c->ev_join);
     free_list(c->allocs, s);
     cudaStreamSynchronize(s);
@@ -756,7 +769,9 @@ int photon_prefill(photon_model* m, const photon_cache* prefix, const int32_t* d
   c->attn_ws_t = al.get<float>(aw);
   if (cudaStreamCreateWithFlags(&c->side, cudaStreamNonBlocking) != cudaSuccess ||
       cudaStreamCreateWithFlags(&c->cap, cudaStreamNonBlocking) != cudaSuccess ||
+      cudaStreamCreateWithPriority(&c->hi, cudaStreamNonBlocking, stream_priority_high()) != cudaSuccess ||
       cudaEventCreateWithFlags(&c->ev_fork, cudaEventDisableTiming) != cudaSuccess ||
+      cudaEventCreateWithFlags(&c->ev_join_hi, cudaEventDisableTiming) != cudaSuccess ||
       cudaEventCreateWithFlags(&c->ev_join, cudaEventDisableTiming) != cudaSuccess)
     return bail(fail(PHOTON_ERR_CUDA, "stream/event creation failed"));
   const int positions =
@@ -877,6 +892,21 @@ int photon_prefill(photon_model* m, const photon_cache* prefix, const int32_t* d
 // Enqueues one decode step (a7..a13) on s.  Every per-step varying value is
 // read on the device (positions from c->d_pos), so the same launches can be
 // captured once into a CUDA graph and replayed for later steps.
+static bool recgen_fork_enabled() {
+  static const bool on = [] {
+    const char* e = getenv("PHOTON_RECGEN_FORK");
+    return !(e && e[0] == '0');
+  }();
+  return on;
+}
+static bool token_priority_enabled() {
+  static const bool on = [] {
+    const char* e = getenv("PHOTON_TOKEN_PRIORITY");
+    return e && e[0] == '1';
+  }();
+  return on;
+}
+
 static void enqueue_decode(photon_model* m, photon_cache* c, int mode, int32_t* own_tokens,
                            float* d_out_logits, const int32_t* d_force_tokens,
                            const void* d_force_a, cudaStream_t s) {
@@ -924,7 +954,7 @@ static void enqueue_decode(photon_model* m, photon_cache* c, int mode, int32_t* 
   // depend on the tokens, so the top-encoder branch (a12-R, a13) runs on the
   // side stream, with its own buffers, while the token decoder (a9-a11)
   // runs here; the two chains join at the end of the step.
-  const bool fork = mode == PHOTON_MODE_REC && c->side != nullptr;
+  const bool fork = mode == PHOTON_MODE_REC && c->side != nullptr && recgen_fork_enabled();
   if (fork) {
     cudaEventRecord(c->ev_fork, s);
     cudaStreamWaitEvent(c->side, c->ev_fork, 0);
@@ -942,8 +972,15 @@ static void enqueue_decode(photon_model* m, photon_cache* c, int mode, int32_t* 
     top_step(c->xt, bt, c->side);
     cudaEventRecord(c->ev_join, c->side);
   }
+  // the token branch: the caller's stream, or (optionally) a high-priority
+  // internal stream so its kernels win the scheduler against the top branch
+  cudaStream_t ts = s;
+  if (fork && token_priority_enabled() && c->hi) {
+    cudaStreamWaitEvent(c->hi, c->ev_fork, 0);
+    ts = c->hi;
+  }
   // a9: Converter_1 -- each A-hat row -> C1 conditioning vectors (rows g*C1 + i)
-  gemm(m, b, c->a_hat, d, m->ptr(m->i_cv1), d, G, C1 * d, d, epi(EPI_STORE_F32, c->xd, (long long)C1 * d), s);
+  gemm(m, b, c->a_hat, d, m->ptr(m->i_cv1), d, G, C1 * d, d, epi(EPI_STORE_F32, c->xd, (long long)C1 * d), ts);
   // a10/a11: token decoder, prefix pass over the C1 conditioning positions,
   // then C1-1 single-row steps; head + greedy argmax after each
   StackRun r1;
@@ -953,10 +990,11 @@ static void enqueue_decode(photon_model* m, photon_cache* c, int mode, int32_t* 
   r1.vc = c->d1v;
   r1.layer_bytes = c->d1_layer;
   r1.cap = 2 * C1;
-  run_stack(m, m->i_dec1, m->Ld1, c->xd, r1, b, s);
+  run_stack(m, m->i_dec1, m->Ld1, c->xd, r1, b, ts);
   const int amax_tiles = m->use_tc ? gemm_tc_argmax_tiles(G, V, d) : 0;
+  bool fused_embed = false;  // the last head also embedded and normalised the next step's input
   auto head = [&](const float* x, int in_step, int in_off, int i) {
-    launch_rmsnorm(m->dt, x, (const float*)m->ptr(m->i_dec1_g), c->hn, G, d, in_step, in_off, eps, s);
+    launch_rmsnorm(m->dt, x, (const float*)m->ptr(m->i_dec1_g), c->hn, G, d, in_step, in_off, eps, ts);
     const long long ld = d_out_logits ? (long long)C1 * V : V;
     if (amax_tiles > 0 && amax_tiles <= c->amax_cap) {
       // tensor-core head with the greedy choice fused into its epilogue;
@@ -964,27 +1002,42 @@ static void enqueue_decode(photon_model* m, photon_cache* c, int mode, int32_t* 
       Epilogue e = epi(EPI_ARGMAX, d_out_logits ? d_out_logits + (size_t)i * V : nullptr, ld);
       e.argmax_part = c->amax_part;
       e.argmax_tiles = amax_tiles;
-      gemm(m, b, c->hn, d, m->ptr(m->i_head), d, G, V, d, e, s);
-      launch_argmax_partials(c->amax_part, amax_tiles, G, V, i, C1, d_force_tokens, d_out_tokens,
-                             c->used, c->next_ids, c->d_err, s);
+      gemm(m, b, c->hn, d, m->ptr(m->i_head), d, G, V, d, e, ts);
+      if (i + 1 < C1) {
+        // greedy choice + the next step's embedding and first attention norm
+        launch_argmax_embed_norm(m->dt, c->amax_part, amax_tiles, G, V, i, C1, d_force_tokens,
+                                 d_out_tokens, c->used, c->next_ids, c->d_err, m->ptr(m->i_embed),
+                                 c->xs, m->block(m->i_dec1, 0).g_attn, b.xn, d, eps, ts);
+        fused_embed = true;
+      } else {
+        launch_argmax_partials(c->amax_part, amax_tiles, G, V, i, C1, d_force_tokens, d_out_tokens,
+                               c->used, c->next_ids, c->d_err, ts);
+      }
     } else {
       float* lg = d_out_logits ? d_out_logits + (size_t)i * V : c->logits;
-      gemm(m, b, c->hn, d, m->ptr(m->i_head), d, G, V, d, epi(EPI_STORE_F32, lg, ld), s);
+      gemm(m, b, c->hn, d, m->ptr(m->i_head), d, G, V, d, epi(EPI_STORE_F32, lg, ld), ts);
       launch_argmax(lg, ld, G, V, i, C1, d_force_tokens, d_out_tokens, c->used, c->next_ids,
-                    c->d_err, s);
+                    c->d_err, ts);
     }
   };
   head(c->xd, C1, C1 - 1, 0);
   for (int i = 1; i < C1; ++i) {
-    launch_embed_f32(m->dt, c->next_ids, m->ptr(m->i_embed), c->xs, G, d, V, c->d_err, s);
+    if (!fused_embed)
+      launch_embed_f32(m->dt, c->next_ids, m->ptr(m->i_embed), c->xs, G, d, V, c->d_err, ts);
     StackRun rs = r1;
     rs.q_len = 1;
     rs.p0 = C1 + i - 1;
-    run_stack(m, m->i_dec1, m->Ld1, c->xs, rs, b, s);
+    rs.xn_ready = fused_embed;
+    fused_embed = false;
+    run_stack(m, m->i_dec1, m->Ld1, c->xs, rs, b, ts);
     head(c->xs, 1, 0, i);
   }
   // a12: input of the top encoder's next position
   if (fork) {
+    if (ts != s) {
+      cudaEventRecord(c->ev_join_hi, ts);
+      cudaStreamWaitEvent(s, c->ev_join_hi, 0);
+    }
     cudaStreamWaitEvent(s, c->ev_join, 0);  // join the top-encoder branch
     return;
   }
@@ -1136,7 +1189,12 @@ int photon_free_cache(photon_cache* c) {
     cudaStreamDestroy(c->side);
   }
   if (c->cap) cudaStreamDestroy(c->cap);  // only ever captured into, never run
+  if (c->hi) {
+    cudaStreamSynchronize(c->hi);
+    cudaStreamDestroy(c->hi);
+  }
   if (c->ev_fork) cudaEventDestroy(c->ev_fork);
+  if (c->ev_join_hi) cudaEventDestroy(c->ev_join_hi);
   if (c->ev_join) cudaEventDestroy(c->ev_join);
   free_list(c->allocs, c->stream);
   CK(cudaStreamSynchronize(c->stream));

@@ -131,3 +131,18 @@ def test_gemm_rmsnorm_bf16(M, N, K):
     # fp32 accumulation, plus the odd operand rounded the other way (1 bf16
     # ulp of one normalised element)
     np.testing.assert_allclose(got, ref, rtol=0, atol=2e-3 * np.abs(ref).max())
+
+
+# warp-per-(group, head) kernel for the decoders' short local caches:
+# (G, H, cap, q_len, p0) with the causal prefix pass and single-row steps
+@pytest.mark.parametrize("G,H,cap,q_len,p0", [(256, 16, 8, 4, 0), (256, 16, 8, 1, 6), (64, 16, 4, 4, 0),
+                                               (7, 3, 16, 1, 15), (9, 2, 16, 4, 12)])
+def test_attn_local_bf16(G, H, cap, q_len, p0):
+    got, ref = _attn_case(torch.bfloat16, G, H, 64, cap, q_len, p0, 40)
+    np.testing.assert_allclose(got, ref, rtol=1e-2, atol=1e-2 * np.abs(ref).max())
+
+
+@pytest.mark.parametrize("G,H,cap,q_len,p0", [(5, 2, 8, 4, 0), (3, 2, 8, 1, 7)])
+def test_attn_local_fp32(G, H, cap, q_len, p0):
+    got, ref = _attn_case(torch.float32, G, H, 32, cap, q_len, p0, 41)
+    np.testing.assert_allclose(got, ref, rtol=1e-5, atol=1e-5)
