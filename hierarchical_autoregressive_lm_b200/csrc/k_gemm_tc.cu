@@ -544,6 +544,26 @@ __global__ void __launch_bounds__(192, 1)
 // through the TMA ring meanwhile.
 constexpr int kDecMaxXBlocks = 8;
 
+#ifdef PHOTON_DEC_TRACE
+// Diagnostic builds only: phase timestamps (globaltimer, ns) of the first
+// CTA of every k_gemm_dec launch, 8 slots per launch.
+__device__ unsigned long long g_dec_trace[8 * 4096];
+__device__ unsigned int g_dec_trace_n;
+__device__ __forceinline__ unsigned long long gtimer() {
+  unsigned long long t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+#define DEC_TRACE(slot)                                                                  \
+  do {                                                                                   \
+    if (trace_me && threadIdx.x == 0) g_dec_trace[(size_t)trace_id * 8 + (slot)] = gtimer(); \
+  } while (0)
+#else
+#define DEC_TRACE(slot) \
+  do {                  \
+  } while (0)
+#endif
+
 template <int BN, int STAGES, bool NORM>
 struct DecCfg {
   static constexpr int kWBytes = kBM * kBK * 2;  // 16 KB weight slice
@@ -557,8 +577,11 @@ struct DecCfg {
   static constexpr uint32_t kTmemCols = BN;
 };
 
+constexpr int kDecThreads = 256;  // 8 warps: roles in warps 0-1, epilogue items in warps 2-7
+constexpr int kDecWorkers = kDecThreads - 64;
+
 template <int BN, int S, int STAGES, bool NORM>
-__global__ void __launch_bounds__(128, 1)
+__global__ void __launch_bounds__(kDecThreads, 1)
     k_gemm_dec(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX,
                int M, int N, int nkb, int kbs, Epilogue ep, const float* __restrict__ nx,
                long long nldx, const float* __restrict__ ng, float eps, int* err) {
@@ -567,6 +590,7 @@ __global__ void __launch_bounds__(128, 1)
   static_assert(128 * LDP * 4 <= Cfg::kDataBytes, "the partial tile reuses the data region");
   static_assert(64 % S == 0, "pairs must divide evenly over the cluster");
   static_assert(!NORM || BN == 64, "the normalisation pass maps 64 token rows");
+  static_assert(BN % 64 == 0, "the TMEM drain splits the tile into two 32-column-aligned halves");
   static_assert((2 * STAGES + 1) * 8 + 8 <= 256, "control block layout");
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -582,6 +606,14 @@ __global__ void __launch_bounds__(128, 1)
   const uint32_t rank = ptx::cluster_ctarank();
   const int a0 = (blockIdx.x / S) * kBM;  // weight rows = output features
   const int b0 = blockIdx.y * BN;         // token rows
+#ifdef PHOTON_DEC_TRACE
+  const bool trace_me = blockIdx.x == 0 && blockIdx.y == 0;
+  __shared__ unsigned int s_trace_id;
+  if (trace_me && threadIdx.x == 0) s_trace_id = atomicAdd(&g_dec_trace_n, 1u) & 4095u;
+  __syncthreads();
+  const unsigned int trace_id = s_trace_id;
+  DEC_TRACE(0);
+#endif
   const int kb0 = (int)rank * kbs;
   const int kb1 = min(nkb, kb0 + kbs);
   const int nk = max(0, kb1 - kb0);
@@ -616,10 +648,58 @@ __global__ void __launch_bounds__(128, 1)
   __syncthreads();
   ptx::tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  DEC_TRACE(1);
   // weights are never written by any kernel: the producer starts on them
   // before waiting for the previous kernel (see k_gemm_tc)
   if (threadIdx.x != 0) pdl_wait();
   pdl_trigger();
+
+  // ---- epilogue items of this thread (warps 2-7): (RoPE pair, token quad)
+  // units owned by this CTA, and the operands that do not depend on the
+  // GEMM (current residual values, RoPE factors), loaded now so the loads
+  // overlap the main loop
+  constexpr int PU = 64 / S;                                  // pairs owned by one CTA
+  constexpr int ITEMS = PU * (BN / 4);                        // (pair, token quad) items
+  constexpr int IPT = (ITEMS + kDecWorkers - 1) / kDecWorkers;  // items per worker thread
+  const int wid = (int)threadIdx.x - 64;
+  const int kind = ep.kind;
+  bool live[IPT];
+  int gfs[IPT], qs[IPT];
+  uint32_t offs[IPT];
+  float pre0[IPT][4], pre1[IPT][4];
+  if (wid >= 0) {
+    const int qp0 = kind == EPI_QKV ? (ep.p0_dev ? *ep.p0_dev + ep.p0 : ep.p0) : 0;
+#pragma unroll
+    for (int j = 0; j < IPT; ++j) {
+      const int i = wid + kDecWorkers * j;
+      const int u = (int)rank * PU + i % PU;
+      const int q = i / PU;  // token quad
+      const int f0 = (u >> 5) * 64 + (u & 31);
+      gfs[j] = a0 + f0;
+      qs[j] = q;
+      offs[j] = (uint32_t)(f0 * LDP + 4 * q) * 4u;
+      live[j] = i < ITEMS && a0 + f0 < N;  // N % 64 == 0: the partner f0 + 32 is in range too
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        pre0[j][e] = 0.f;
+        pre1[j][e] = 0.f;
+        const long long t = b0 + 4 * q + e;
+        if (!live[j] || t >= M) continue;
+        if (kind == EPI_ADD_F32) {
+          const float* o = reinterpret_cast<const float*>(ep.out) + t * ep.ldo + gfs[j];
+          pre0[j][e] = o[0];
+          pre1[j][e] = o[32];
+        } else if (kind == EPI_QKV && gfs[j] < 2 * ep.d) {
+          const int within = gfs[j] >= ep.d ? gfs[j] - ep.d : gfs[j];
+          const int g = (int)(t / ep.q_len);
+          const int pos = qp0 + (int)(t - (long long)g * ep.q_len);
+          const float2 cs = ep.rope[(long long)pos * 32 + (within & 63)];
+          pre0[j][e] = cs.x;
+          pre1[j][e] = cs.y;
+        }
+      }
+    }
+  }
 
   const int pre = nk < STAGES ? nk : STAGES;
   if (threadIdx.x == 0) {
@@ -628,6 +708,7 @@ __global__ void __launch_bounds__(128, 1)
       ptx::tma_load_2d(w_tile(it), &tmW, (kb0 + it) * kBK, a0, full_bar(it));
     }
     pdl_wait();
+    DEC_TRACE(2);
     if (!NORM)
       for (int it = 0; it < pre; ++it)
         ptx::tma_load_2d(x_tile(it), &tmX, (kb0 + it) * kBK, b0, full_bar(it));
@@ -635,15 +716,19 @@ __global__ void __launch_bounds__(128, 1)
 
   if constexpr (NORM) {
     // ---- RMSNorm of the BN = 64 token rows, this CTA's K run into shared memory
+    constexpr int RPP = kDecThreads / 8;  // rows per pass (8 threads per 64-column slice row)
+    constexpr int PASSES = 64 / RPP;
     const int t = threadIdx.x;
     const int ch = t & 7;  // 16-byte chunk of a 64-column slice
     const int kc0 = kb0 * kBK;
-    float part[4] = {0.f, 0.f, 0.f, 0.f};  // rows t / 8 + 16 j
+    float part[PASSES];
+#pragma unroll
+    for (int j = 0; j < PASSES; ++j) part[j] = 0.f;
 #pragma unroll 1
     for (int it = 0; it < nk; ++it) {
 #pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const long long grow = b0 + (t >> 3) + 16 * j;
+      for (int j = 0; j < PASSES; ++j) {
+        const long long grow = b0 + (t >> 3) + RPP * j;
         if (grow < M) {
           const float4* p = reinterpret_cast<const float4*>(nx + grow * nldx + kc0 + it * kBK + ch * 8);
           const float4 u = p[0], v = p[1];
@@ -653,13 +738,13 @@ __global__ void __launch_bounds__(128, 1)
       }
     }
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
+    for (int j = 0; j < PASSES; ++j) {
 #pragma unroll
       for (int o = 1; o < 8; o <<= 1) part[j] += __shfl_xor_sync(0xffffffffu, part[j], o);
     }
     if (ch == 0) {
 #pragma unroll
-      for (int j = 0; j < 4; ++j) row_ssq[(t >> 3) + 16 * j] = part[j];
+      for (int j = 0; j < PASSES; ++j) row_ssq[(t >> 3) + RPP * j] = part[j];
     }
     ptx::cluster_sync();  // every CTA's partial sums are in place
     if (t < 64) {
@@ -677,8 +762,8 @@ __global__ void __launch_bounds__(128, 1)
       const float4 g0 = reinterpret_cast<const float4*>(ng + col)[0];
       const float4 g1 = reinterpret_cast<const float4*>(ng + col)[1];
 #pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const int row = (t >> 3) + 16 * j;
+      for (int j = 0; j < PASSES; ++j) {
+        const int row = (t >> 3) + RPP * j;
         const long long grow = b0 + row;
         uint4 q = make_uint4(0u, 0u, 0u, 0u);
         if (grow < M) {
@@ -731,22 +816,25 @@ __global__ void __launch_bounds__(128, 1)
   }
   __syncwarp();
 
-  // ---- this CTA's partial tile: TMEM -> shared memory (row = feature)
+  // ---- this CTA's partial tile: TMEM -> shared memory (row = feature); warp w
+  // reads TMEM lanes 32 (w % 4) .. + 31, columns of half w / 4 of the tile
   if (nk > 0 && !ptx::mbar_wait(done_bar, 0, abort_flag)) {
     report_error(err, DEV_WAIT_TIMEOUT_EPILOGUE);
     *abort_flag = 1;
   }
+  DEC_TRACE(3);
   __syncthreads();
   const bool ok = (*abort_flag == 0);
   ptx::tc_fence_after();
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
   float* P = reinterpret_cast<float*>(smem);
   {
-    const int tl = warp * 32 + lane;
-    const uint32_t trow = tmem + ((uint32_t)(warp * 32) << 16);
+    const int q4 = warp & 3, half = warp >> 2;
+    const int tl = q4 * 32 + lane;
+    const uint32_t trow = tmem + ((uint32_t)(q4 * 32) << 16);
     float4* prow = reinterpret_cast<float4*>(P + tl * LDP);
 #pragma unroll 1
-    for (int j0 = 0; j0 < BN; j0 += 32) {
+    for (int j0 = half * (BN / 2); j0 < (half + 1) * (BN / 2); j0 += 32) {
       float v[32];
       if (ok && nk > 0) {
         ptx::tmem_ld32(trow + (uint32_t)j0, v);
@@ -762,40 +850,101 @@ __global__ void __launch_bounds__(128, 1)
   ptx::tc_fence_before();
   __syncthreads();
   if (warp == 0) ptx::tmem_dealloc(tmem, Cfg::kTmemCols);
-  ptx::cluster_sync();  // every partial tile of the cluster is in place
+  ptx::cluster_arrive();  // this CTA's partial tile is in place
+  ptx::cluster_wait();    // every partial tile of the cluster is in place
+  DEC_TRACE(4);
 
-  // ---- reduce the owned pairs over the cluster, then the epilogue
-  constexpr int PU = 64 / S;          // pairs owned by one CTA
-  constexpr int ITEMS = PU * (BN / 4);
+  // ---- sum the owned pairs over the cluster, in rank order
   const uint32_t pbase = ptx::smem_u32(P);
-  if (ok) {
-#pragma unroll 1
-    for (int i = threadIdx.x; i < ITEMS; i += 128) {
-      const int u = (int)rank * PU + i % PU;
-      const int q = i / PU;  // token quad
-      const int f0 = (u >> 5) * 64 + (u & 31);
-      const uint32_t off0 = (uint32_t)(f0 * LDP + 4 * q) * 4u;
-      const uint32_t off1 = off0 + 32u * LDP * 4u;
-      float4 s0 = make_float4(0.f, 0.f, 0.f, 0.f), s1 = s0;
+  float4 s0[IPT], s1[IPT];
+  if (wid >= 0) {
+#pragma unroll
+    for (int j = 0; j < IPT; ++j) {
+      s0[j] = make_float4(0.f, 0.f, 0.f, 0.f);
+      s1[j] = s0[j];
+      if (!live[j] || !ok) continue;
 #pragma unroll
       for (int p = 0; p < S; ++p) {
         const uint32_t peer = ptx::map_shared_rank(pbase, (uint32_t)p);
-        const float4 x0 = ptx::ld_shared_cluster_f4(peer + off0);
-        const float4 x1 = ptx::ld_shared_cluster_f4(peer + off1);
-        s0.x += x0.x; s0.y += x0.y; s0.z += x0.z; s0.w += x0.w;
-        s1.x += x1.x; s1.y += x1.y; s1.z += x1.z; s1.w += x1.w;
-      }
-      const int gf0 = a0 + f0;
-      if (gf0 >= N) continue;  // N is a multiple of 64: gf0 + 32 < N as well
-      const float v0[4] = {s0.x, s0.y, s0.z, s0.w}, v1[4] = {s1.x, s1.y, s1.z, s1.w};
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const long long t = b0 + 4 * q + e;
-        if (t < M) epi_pair<bf16>(ep, t, gf0, v0[e], gf0 + 32, v1[e]);
+        const float4 x0 = ptx::ld_shared_cluster_f4(peer + offs[j]);
+        const float4 x1 = ptx::ld_shared_cluster_f4(peer + offs[j] + 32u * LDP * 4u);
+        s0[j].x += x0.x; s0[j].y += x0.y; s0[j].z += x0.z; s0[j].w += x0.w;
+        s1[j].x += x1.x; s1[j].y += x1.y; s1[j].z += x1.z; s1[j].w += x1.w;
       }
     }
   }
-  ptx::cluster_sync();  // peers keep their partial tiles until all reads are done
+  DEC_TRACE(7);
+  ptx::cluster_arrive();  // done reading the other CTAs' tiles
+
+  // ---- epilogue
+  if (wid >= 0 && ok) {
+    const int qp0 = kind == EPI_QKV ? (ep.p0_dev ? *ep.p0_dev + ep.p0 : ep.p0) : 0;
+#pragma unroll
+    for (int j = 0; j < IPT; ++j) {
+      if (!live[j]) continue;
+      const int gf = gfs[j];
+      const float v0[4] = {s0[j].x, s0[j].y, s0[j].z, s0[j].w};
+      const float v1[4] = {s1[j].x, s1[j].y, s1[j].z, s1[j].w};
+      if (kind == EPI_QKV) {
+        const int d = ep.d;
+        const int which = (gf >= d) + (gf >= 2 * d);
+        const int within = gf - which * d, h = within >> 6, i = within & 63;
+        bf16* base;
+        long long step;  // elements between consecutive token rows' outputs (q only)
+        if (which == 0) {
+          base = reinterpret_cast<bf16*>(ep.q_out) + within;
+          step = d;
+        } else {
+          base = reinterpret_cast<bf16*>(which == 1 ? ep.k_cache : ep.v_cache) + i;
+          step = 0;
+        }
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const long long t = b0 + 4 * qs[j] + e;
+          if (t >= M) continue;
+          float o0 = v0[e], o1 = v1[e];
+          if (which < 2) {
+            const float c = pre0[j][e], sn = pre1[j][e];
+            o0 = v0[e] * c - v1[e] * sn;
+            o1 = v0[e] * sn + v1[e] * c;
+          }
+          bf16* o;
+          if (which == 0) {
+            o = base + t * step;
+          } else {
+            const int g = (int)(t / ep.q_len);
+            const int pos = qp0 + (int)(t - (long long)g * ep.q_len);
+            o = base + (((long long)g * ep.H + h) * ep.cap + (pos - ep.kv_off)) * 64;
+          }
+          st_f(o, o0);
+          st_f(o + 32, o1);
+        }
+        continue;
+      }
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const long long t = b0 + 4 * qs[j] + e;
+        if (t >= M) continue;
+        if (kind == EPI_ADD_F32) {
+          float* o = reinterpret_cast<float*>(ep.out) + t * ep.ldo + gf;
+          o[0] = pre0[j][e] + v0[e];
+          o[32] = pre1[j][e] + v1[e];
+        } else if (kind == EPI_STORE_F32) {
+          float* o = reinterpret_cast<float*>(ep.out) + t * ep.ldo + gf;
+          o[0] = v0[e];
+          o[32] = v1[e];
+        } else if (kind == EPI_STORE_T || kind == EPI_GELU_T) {
+          const bool g = kind == EPI_GELU_T;
+          bf16* o = reinterpret_cast<bf16*>(ep.out) + t * ep.ldo + gf;
+          st_f(o, g ? gelu_erf(v0[e]) : v0[e]);
+          st_f(o + 32, g ? gelu_erf(v1[e]) : v1[e]);
+        }
+      }
+    }
+  }
+  DEC_TRACE(5);
+  ptx::cluster_wait();  // the other CTAs are done reading this CTA's tile
+  DEC_TRACE(6);
 }
 
 // ------------------------------------------------------------------ host side
@@ -892,7 +1041,7 @@ int dec_max_clusters() {
     if (okf) {
       cudaLaunchConfig_t cfg = {};
       cfg.gridDim = dim3(S, 1, 1);
-      cfg.blockDim = dim3(128);
+      cfg.blockDim = dim3(kDecThreads);
       cfg.dynamicSmemBytes = Cfg::kSmemBytes;
       cudaLaunchAttribute attr[1];
       attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -918,7 +1067,7 @@ void run_dec(const CUtensorMap& mw, const CUtensorMap& mx, int ga, int gb, const
   using Cfg = DecCfg<BN, STAGES, NORM>;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(ga * S, gb, 1);
-  cfg.blockDim = dim3(128);
+  cfg.blockDim = dim3(kDecThreads);
   cfg.dynamicSmemBytes = Cfg::kSmemBytes;
   cfg.stream = s;
   cudaLaunchAttribute attr[3];
@@ -979,6 +1128,14 @@ int dec_bn(int M, bool norm) {
   return 128;
 }
 
+bool dec_two_waves() {
+  static const bool on = [] {
+    const char* e = getenv("PHOTON_GEMM_2WAVE");
+    return !(e && e[0] == '0');
+  }();
+  return on;
+}
+
 template <int S>
 int dec_fit(int bn, bool norm) {
   if (norm) return dec_max_clusters<64, S, kDecStages, true>();
@@ -1010,7 +1167,7 @@ int dec_cluster_size(int M, int N, int K, bool norm) {
     }
     if (tiles <= fit) return c;
   }
-  if (nkb >= 2 && run_fits(2) && tiles <= 2 * dec_fit<2>(bn, norm)) return 2;
+  if (dec_two_waves() && nkb >= 2 && run_fits(2) && tiles <= 2 * dec_fit<2>(bn, norm)) return 2;
   return 1;
 }
 
@@ -1075,6 +1232,15 @@ struct Plan {
   int ga, gb;
 };
 
+// Smallest M for 256-wide tiles in the normal orientation (N % 256 == 0).
+int bn256_min_m() {
+  static const int v = [] {
+    const char* e = getenv("PHOTON_GEMM_BN256_MIN_M");
+    return e ? atoi(e) : 4096;
+  }();
+  return v;
+}
+
 Plan plan_for(int M, int N, int K, int force_splits, int force_swap, bool argmax) {
   Plan p;
   const int nkb = K / kBK;
@@ -1084,7 +1250,7 @@ Plan plan_for(int M, int N, int K, int force_splits, int force_swap, bool argmax
   if (p.swap)
     p.bn = 64;  // token tiles of 64: M = 256 gives 4 CTAs per 128-feature tile
   else
-    p.bn = (N % 256 == 0 && (M >= 4096 || argmax)) ? 256 : 128;
+    p.bn = (N % 256 == 0 && (M >= bn256_min_m() || argmax)) ? 256 : 128;
   const int ga = p.swap ? (N + kBM - 1) / kBM : (M + kBM - 1) / kBM;
   const int gb = p.swap ? (M + p.bn - 1) / p.bn : (N + p.bn - 1) / p.bn;
   const int tiles = ga * gb;
@@ -1196,3 +1362,18 @@ bool launch_gemm_tc(const GemmArgs& a, const GemmWorkspace& ws, int* err, cudaSt
 }
 
 }  // namespace photon
+
+#ifdef PHOTON_DEC_TRACE
+// Diagnostic builds only: copy out / reset the k_gemm_dec phase trace.
+extern "C" __attribute__((visibility("default"))) int photon_debug_dec_trace(unsigned long long* host,
+                                                                            int n, unsigned int* count) {
+  if (cudaMemcpyFromSymbol(count, photon::g_dec_trace_n, sizeof(unsigned int)) != cudaSuccess) return -3;
+  if (cudaMemcpyFromSymbol(host, photon::g_dec_trace, (size_t)n * 8 * sizeof(unsigned long long)) != cudaSuccess)
+    return -3;
+  return 0;
+}
+extern "C" __attribute__((visibility("default"))) int photon_debug_dec_trace_reset() {
+  const unsigned int z = 0;
+  return cudaMemcpyToSymbol(photon::g_dec_trace_n, &z, sizeof(z)) == cudaSuccess ? 0 : -3;
+}
+#endif
