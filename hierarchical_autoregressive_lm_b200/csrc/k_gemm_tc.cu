@@ -1232,11 +1232,12 @@ struct Plan {
   int ga, gb;
 };
 
-// Smallest M for 256-wide tiles in the normal orientation (N % 256 == 0).
+// Smallest M for 256-wide tiles in the normal orientation (N % 256 == 0);
+// fewer, larger tiles for the 1024-row prefix pass.
 int bn256_min_m() {
   static const int v = [] {
     const char* e = getenv("PHOTON_GEMM_BN256_MIN_M");
-    return e ? atoi(e) : 4096;
+    return e ? atoi(e) : 512;
   }();
   return v;
 }
@@ -1273,6 +1274,17 @@ Plan plan_for(int M, int N, int K, int force_splits, int force_swap, bool argmax
   p.ga = ga;
   p.gb = gb;
   return p;
+}
+
+// Tile count from which the normal orientation runs the persistent kernel
+// (64: the token decoder's 1024-row prefix pass measured faster there than
+// on k_gemm_tc, with 256-wide tiles).
+int persist_min_tiles() {
+  static const int v = [] {
+    const char* e = getenv("PHOTON_GEMM_PERSIST_MIN_TILES");
+    return e ? atoi(e) : 64;
+  }();
+  return v;
 }
 
 bool persistent_enabled() {
@@ -1345,7 +1357,7 @@ bool launch_gemm_tc(const GemmArgs& a, const GemmWorkspace& ws, int* err, cudaSt
       run_tc<256, 4, true>(ma, mb, p.ga, p.gb, p.splits, M, N, nkb, p.kbs, a.ep, part, counters, a.W, a.ldw * 2, err, s);
   } else {
     if (!make_map(&ma, a.A, M, K, a.lda, kBM) || !make_map(&mb, a.W, N, K, a.ldw, p.bn)) return false;
-    if (p.splits == 1 && (argmax || p.ga * p.gb >= 2 * 148) && persistent_enabled()) {
+    if (p.splits == 1 && (argmax || p.ga * p.gb >= persist_min_tiles()) && persistent_enabled()) {
       const int nt_major = argmax ? 1 : 0;
       if (p.bn == 256)
         run_tc_persist<256, 4>(ma, mb, M, N, nkb, a.ep, nt_major, err, s);

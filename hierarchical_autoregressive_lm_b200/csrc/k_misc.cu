@@ -192,6 +192,28 @@ __global__ void k_rmsnorm(const float* __restrict__ x, const float* __restrict__
   const int lane = threadIdx.x & 31;
   if (warp >= rows) return;
   const float* xr = x + ((long long)warp * in_step + in_off) * d;
+  T* o = out + (long long)warp * d;
+  if (d == 1024) {
+    // the row stays in registers: one read, and every load in flight at once
+    float4 v[8];
+#pragma unroll
+    for (int k = 0; k < 8; ++k) v[k] = *reinterpret_cast<const float4*>(xr + lane * 4 + 128 * k);
+    float ss = 0.f;
+#pragma unroll
+    for (int k = 0; k < 8; ++k) ss += v[k].x * v[k].x + v[k].y * v[k].y + v[k].z * v[k].z + v[k].w * v[k].w;
+    ss = warp_sum(ss);
+    const float r = 1.0f / sqrtf(ss / (float)d + eps);
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      const int c = lane * 4 + 128 * k;
+      const float4 gg = *reinterpret_cast<const float4*>(g + c);
+      st_f(o + c + 0, v[k].x * r * gg.x);
+      st_f(o + c + 1, v[k].y * r * gg.y);
+      st_f(o + c + 2, v[k].z * r * gg.z);
+      st_f(o + c + 3, v[k].w * r * gg.w);
+    }
+    return;
+  }
   float ss = 0.f;
   for (int c = lane * 4; c < d; c += 128) {
     const float4 v = *reinterpret_cast<const float4*>(xr + c);
@@ -199,7 +221,6 @@ __global__ void k_rmsnorm(const float* __restrict__ x, const float* __restrict__
   }
   ss = warp_sum(ss);
   const float r = 1.0f / sqrtf(ss / (float)d + eps);
-  T* o = out + (long long)warp * d;
   for (int c = lane * 4; c < d; c += 128) {
     const float4 v = *reinterpret_cast<const float4*>(xr + c);
     const float4 gg = *reinterpret_cast<const float4*>(g + c);
