@@ -138,6 +138,41 @@ void launch_argmax_partials(const unsigned long long* part, int tiles, int rows,
 // pos[0] += dN; pos[1] += dN1 (device-side decode positions).
 void launch_advance(int* pos, int dN, int dN1, cudaStream_t s);
 
+// ---- persistent single-row step of a chunk-local decoder stack ------------
+// All L pre-norm blocks of one token-decoder step in one cooperative launch
+// (see k_stack.cu).  rows = groups (one new row each), local caches
+// [G][H][cap][64] per layer, the new row at position p0 (< 16).  part /
+// tile_cnt: split scratch (stack_local_scratch_bytes; counters zero, left
+// zero); bar: one zero-initialised word the launch resets itself.
+struct StackLocalLaunch {
+  const void* wqkv[8];
+  const void* wo[8];
+  const void* w1[8];
+  const void* w2[8];
+  const float* g_attn[8];
+  const float* g_mlp[8];
+  float* x;
+  void* xn;
+  void* q;
+  void* att;
+  void* hid;
+  void* kc;
+  void* vc;
+  long long layer_elems;
+  const float2* rope;
+  float* part;
+  int* tile_cnt;
+  int cnt_len;
+  unsigned int* bar;
+  int* err;
+  int rows, d, H, f, L, cap, p0;
+  float eps, scale;
+  int skip_first_norm;
+};
+size_t stack_local_scratch_bytes(int rows, int d);
+bool stack_local_supported(int rows, int d, int H, int dh, int f, int L, int p0, int cap);
+bool launch_stack_local(const StackLocalLaunch& s, cudaStream_t stream);
+
 // ---- GEMM ----------------------------------------------------------------
 void launch_gemm(int dt, const GemmArgs& a, const GemmWorkspace& ws, int* err, cudaStream_t s);
 void launch_gemm_simt(int dt, const GemmArgs& a, cudaStream_t s);

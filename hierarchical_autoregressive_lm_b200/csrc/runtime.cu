@@ -301,6 +301,10 @@ struct photon_cache {
   size_t gemm_ws_bytes = 0;
   int* gemm_cnt = nullptr;
   int* gemm_cnt_t = nullptr;
+  float* stk_part = nullptr;         // persistent token-step kernel: split partials
+  int* stk_cnt = nullptr;            // ... its tile counters (zeroed)
+  unsigned int* stk_bar = nullptr;   // ... its grid-barrier word
+  int stk_cnt_len = 0;
   float* attn_ws = nullptr;
   size_t attn_ws_bytes = 0;
   int* d_err = nullptr;
@@ -766,6 +770,12 @@ int photon_prefill(photon_model* m, const photon_cache* prefix, const int32_t* d
   c->gemm_ws_t = al.get<float>(gw);
   c->gemm_cnt = al.get<int>(kGemmTileCounters * sizeof(int));
   c->gemm_cnt_t = al.get<int>(kGemmTileCounters * sizeof(int));
+  if (m->use_tc) {
+    c->stk_cnt_len = (d / 128) * ((B * C2 + 63) / 64);
+    c->stk_part = al.get<float>(stack_local_scratch_bytes(B * C2, d));
+    c->stk_cnt = al.get<int>((size_t)c->stk_cnt_len * sizeof(int));
+    c->stk_bar = al.get<unsigned int>(256);
+  }
   c->attn_ws_t = al.get<float>(aw);
   if (cudaStreamCreateWithFlags(&c->side, cudaStreamNonBlocking) != cudaSuccess ||
       cudaStreamCreateWithFlags(&c->cap, cudaStreamNonBlocking) != cudaSuccess ||
@@ -780,7 +790,8 @@ int photon_prefill(photon_model* m, const photon_cache* prefix, const int32_t* d
   if (al.err != cudaSuccess || rc) return bail(PHOTON_ERR_OOM);
   if (cudaMemsetAsync(c->d_err, 0, 16, s) != cudaSuccess ||
       cudaMemsetAsync(c->gemm_cnt, 0, kGemmTileCounters * sizeof(int), s) != cudaSuccess ||
-      cudaMemsetAsync(c->gemm_cnt_t, 0, kGemmTileCounters * sizeof(int), s) != cudaSuccess)
+      cudaMemsetAsync(c->gemm_cnt_t, 0, kGemmTileCounters * sizeof(int), s) != cudaSuccess ||
+      (c->stk_cnt && cudaMemsetAsync(c->stk_cnt, 0, (size_t)c->stk_cnt_len * sizeof(int), s) != cudaSuccess))
     return bail(PHOTON_ERR_CUDA);
 
   // prefill workspace (released at the end of this call)
@@ -907,6 +918,58 @@ static bool token_priority_enabled() {
   return on;
 }
 
+static bool stack_mega_enabled() {
+  static const bool on = [] {
+    const char* e = getenv("PHOTON_STACK_MEGA");
+    return e && e[0] == '1';
+  }();
+  return on;
+}
+
+// One single-row token-decoder step (all Ld1 blocks) as one persistent
+// cooperative kernel; false when it does not apply (then run_stack does it).
+static bool token_step_persistent(photon_model* m, photon_cache* c, const Bufs& b, float* x,
+                                  const StackRun& r, cudaStream_t s) {
+  if (!m->use_tc || !stack_mega_enabled() || !c->stk_part || r.q_len != 1 || m->Ld1 > 8) return false;
+  if (!stack_local_supported(r.G, m->d, m->H, m->dh, m->f, m->Ld1, r.p0, r.cap)) return false;
+  StackLocalLaunch k;
+  memset(&k, 0, sizeof(k));
+  for (int l = 0; l < m->Ld1; ++l) {
+    const BlockW w = m->block(m->i_dec1, l);
+    k.wqkv[l] = w.wqkv;
+    k.wo[l] = w.wo;
+    k.w1[l] = w.w1;
+    k.w2[l] = w.w2;
+    k.g_attn[l] = w.g_attn;
+    k.g_mlp[l] = w.g_mlp;
+  }
+  k.x = x;
+  k.xn = b.xn;
+  k.q = b.q;
+  k.att = b.att;
+  k.hid = b.hid;
+  k.kc = r.kc;
+  k.vc = r.vc;
+  k.layer_elems = (long long)(r.layer_bytes / 2);
+  k.rope = b.rope;
+  k.part = c->stk_part;
+  k.tile_cnt = c->stk_cnt;
+  k.cnt_len = c->stk_cnt_len;
+  k.bar = c->stk_bar;
+  k.err = b.err;
+  k.rows = r.G;
+  k.d = m->d;
+  k.H = m->H;
+  k.f = m->f;
+  k.L = m->Ld1;
+  k.cap = r.cap;
+  k.p0 = r.p0;
+  k.eps = m->cfg.norm_eps;
+  k.scale = 1.0f / sqrtf((float)m->dh);
+  k.skip_first_norm = r.xn_ready ? 1 : 0;
+  return launch_stack_local(k, s);
+}
+
 static void enqueue_decode(photon_model* m, photon_cache* c, int mode, int32_t* own_tokens,
                            float* d_out_logits, const int32_t* d_force_tokens,
                            const void* d_force_a, cudaStream_t s) {
@@ -1029,7 +1092,7 @@ static void enqueue_decode(photon_model* m, photon_cache* c, int mode, int32_t* 
     rs.p0 = C1 + i - 1;
     rs.xn_ready = fused_embed;
     fused_embed = false;
-    run_stack(m, m->i_dec1, m->Ld1, c->xs, rs, b, ts);
+    if (!token_step_persistent(m, c, b, c->xs, rs, ts)) run_stack(m, m->i_dec1, m->Ld1, c->xs, rs, b, ts);
     head(c->xs, 1, 0, i);
   }
   // a12: input of the top encoder's next position
