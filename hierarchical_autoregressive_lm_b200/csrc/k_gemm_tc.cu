@@ -486,11 +486,25 @@ __global__ void __launch_bounds__(192, 1)
       const long long grow = (long long)mt * kBM + q * 32 + lane;
       const uint32_t trow = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(b * BN);
       unsigned long long best = 0ull;
+      // split RMSNorm consumer: this row's 1 / rms from the producer's slots
+      float rs = 1.f;
+      if (ep.ssq_in != nullptr && grow < M) {
+        float tot = 0.f;
+        for (int sl = 0; sl < ep.ssq_slots; ++sl) tot += ep.ssq_in[grow * ep.ssq_slots + sl];
+        rs = 1.0f / sqrtf(tot / (float)ep.norm_d + ep.norm_eps);
+      }
 #pragma unroll 1
       for (int j0 = 0; j0 < BN; j0 += 64) {
         float lo[32], hi[32];
         ptx::tmem_ld32(trow + (uint32_t)j0, lo);
         ptx::tmem_ld32(trow + (uint32_t)(j0 + 32), hi);
+        if (ep.ssq_in != nullptr) {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            lo[i] *= rs;
+            hi[i] *= rs;
+          }
+        }
         const int gc = nt * BN + j0;
         if (grow >= M || gc >= N) continue;
         if (ep.kind == EPI_ARGMAX) {
@@ -667,6 +681,7 @@ __global__ void __launch_bounds__(kDecThreads, 1)
   int gfs[IPT], qs[IPT];
   uint32_t offs[IPT];
   float pre0[IPT][4], pre1[IPT][4];
+  float gn0[IPT], gn1[IPT];  // split-RMSNorm producer: gains of the next norm
   if (wid >= 0) {
     const int qp0 = kind == EPI_QKV ? (ep.p0_dev ? *ep.p0_dev + ep.p0 : ep.p0) : 0;
 #pragma unroll
@@ -679,6 +694,8 @@ __global__ void __launch_bounds__(kDecThreads, 1)
       qs[j] = q;
       offs[j] = (uint32_t)(f0 * LDP + 4 * q) * 4u;
       live[j] = i < ITEMS && a0 + f0 < N;  // N % 64 == 0: the partner f0 + 32 is in range too
+      gn0[j] = (ep.xs_out != nullptr && live[j]) ? ep.g_next[a0 + f0] : 0.f;
+      gn1[j] = (ep.xs_out != nullptr && live[j]) ? ep.g_next[a0 + f0 + 32] : 0.f;
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
         pre0[j][e] = 0.f;
@@ -699,6 +716,16 @@ __global__ void __launch_bounds__(kDecThreads, 1)
         }
       }
     }
+  }
+
+  // split RMSNorm consumer: 1 / rms of each token row of the tile, from the
+  // producer's per-CTA partial sums in slot order
+  if (ep.ssq_in != nullptr && wid >= 0 && wid < BN) {
+    const long long row = b0 + wid;
+    float tot = 0.f;
+    if (row < M)
+      for (int sl = 0; sl < ep.ssq_slots; ++sl) tot += ep.ssq_in[row * ep.ssq_slots + sl];
+    row_rstd[wid] = 1.0f / sqrtf(tot / (float)ep.norm_d + ep.norm_eps);
   }
 
   const int pre = nk < STAGES ? nk : STAGES;
@@ -877,14 +904,61 @@ __global__ void __launch_bounds__(kDecThreads, 1)
   ptx::cluster_arrive();  // done reading the other CTAs' tiles
 
   // ---- epilogue
+  // split RMSNorm producer: per token, the sum of squares of the new
+  // residual over this CTA's pairs.  Consecutive lanes hold consecutive pairs
+  // of the same token quad (PU divides 32), so a fixed butterfly over the
+  // PU lanes of a group gives the sum; its first lane writes the slot.
+  static_assert(PU <= 32 && 32 % PU == 0 && kDecWorkers % 32 == 0 && ITEMS % 32 == 0,
+                "pair groups within a warp, warps wholly inside or outside the items");
+  const bool produce = ep.xs_out != nullptr && kind == EPI_ADD_F32;
+  if (produce && wid >= 0) {
+#pragma unroll
+    for (int j = 0; j < IPT; ++j) {
+      const int i = wid + kDecWorkers * j;
+      // ITEMS and kDecWorkers are multiples of 32: a warp is wholly in or out
+      if (i >= ITEMS) continue;
+      float ss[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const bool in = ok && live[j] && b0 + 4 * qs[j] + e < M;
+        ss[e] = 0.f;
+        if (in) {
+          const float v0 = (e == 0 ? s0[j].x : e == 1 ? s0[j].y : e == 2 ? s0[j].z : s0[j].w);
+          const float v1 = (e == 0 ? s1[j].x : e == 1 ? s1[j].y : e == 2 ? s1[j].z : s1[j].w);
+          const float a = pre0[j][e] + v0, b = pre1[j][e] + v1;
+          ss[e] = a * a + b * b;
+        }
+      }
+#pragma unroll
+      for (int o = 1; o < PU; o <<= 1) {
+#pragma unroll
+        for (int e = 0; e < 4; ++e) ss[e] += __shfl_xor_sync(0xffffffffu, ss[e], o);
+      }
+      if (ok && live[j] && i % PU == 0) {
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const long long t = b0 + 4 * qs[j] + e;
+          if (t < M) ep.ssq_out[t * ep.ssq_slots + blockIdx.x] = ss[e];
+        }
+      }
+    }
+  }
   if (wid >= 0 && ok) {
     const int qp0 = kind == EPI_QKV ? (ep.p0_dev ? *ep.p0_dev + ep.p0 : ep.p0) : 0;
 #pragma unroll
     for (int j = 0; j < IPT; ++j) {
       if (!live[j]) continue;
       const int gf = gfs[j];
-      const float v0[4] = {s0[j].x, s0[j].y, s0[j].z, s0[j].w};
-      const float v1[4] = {s1[j].x, s1[j].y, s1[j].z, s1[j].w};
+      float v0[4] = {s0[j].x, s0[j].y, s0[j].z, s0[j].w};
+      float v1[4] = {s1[j].x, s1[j].y, s1[j].z, s1[j].w};
+      if (ep.ssq_in != nullptr) {
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float r = row_rstd[4 * qs[j] + e];
+          v0[e] *= r;
+          v1[e] *= r;
+        }
+      }
       if (kind == EPI_QKV) {
         const int d = ep.d;
         const int which = (gf >= d) + (gf >= 2 * d);
@@ -927,8 +1001,14 @@ __global__ void __launch_bounds__(kDecThreads, 1)
         if (t >= M) continue;
         if (kind == EPI_ADD_F32) {
           float* o = reinterpret_cast<float*>(ep.out) + t * ep.ldo + gf;
-          o[0] = pre0[j][e] + v0[e];
-          o[32] = pre1[j][e] + v1[e];
+          const float n0 = pre0[j][e] + v0[e], n1 = pre1[j][e] + v1[e];
+          o[0] = n0;
+          o[32] = n1;
+          if (produce) {
+            bf16* xs = reinterpret_cast<bf16*>(ep.xs_out) + t * ep.ldo + gf;
+            st_f(xs, n0 * gn0[j]);
+            st_f(xs + 32, n1 * gn1[j]);
+          }
         } else if (kind == EPI_STORE_F32) {
           float* o = reinterpret_cast<float*>(ep.out) + t * ep.ldo + gf;
           o[0] = v0[e];
@@ -1305,6 +1385,18 @@ int gemm_tc_argmax_tiles(int M, int N, int K) {
   return p.swap ? p.ga : p.gb;
 }
 
+int gemm_tc_ssq_slots(int M, int N, int K) {
+  if (M <= 0 || N <= 0 || K < kBK || !tma_available() || !dec_path(M, N, K, 0, -1)) return 0;
+  return ((N + kBM - 1) / kBM) * dec_cluster_size(M, N, K, false);
+}
+
+bool gemm_tc_takes_ssq(int M, int N, int K) {
+  if (M <= 0 || N <= 0 || K < kBK || K % kBK || N % 64 || !tma_available()) return false;
+  if (dec_path(M, N, K, 0, -1)) return true;
+  const Plan p = plan_for(M, N, K, 0, -1, false);
+  return !p.swap && p.splits == 1 && p.ga * p.gb >= persist_min_tiles() && persistent_enabled();
+}
+
 bool gemm_tc_fuses_norm(int M, int N, int K) {
   if (M <= 0 || N <= 0 || K < kBK || !tma_available()) return false;
   return dec_path(M, N, K, 0, -1, true);
@@ -1337,6 +1429,9 @@ bool launch_gemm_tc(const GemmArgs& a, const GemmWorkspace& ws, int* err, cudaSt
     // few tokens: cluster split-K with the reduction on chip
     if (try_dec(a, err, s)) return true;
   }
+  // the split-RMSNorm producer exists only in k_gemm_dec; its consumer also
+  // in the persistent kernel (checked below)
+  if (a.ep.xs_out != nullptr || (a.ep.ssq_in != nullptr && p.swap)) return false;
   float* part = nullptr;
   int* counters = nullptr;
   if (p.splits > 1) {
@@ -1357,6 +1452,8 @@ bool launch_gemm_tc(const GemmArgs& a, const GemmWorkspace& ws, int* err, cudaSt
       run_tc<256, 4, true>(ma, mb, p.ga, p.gb, p.splits, M, N, nkb, p.kbs, a.ep, part, counters, a.W, a.ldw * 2, err, s);
   } else {
     if (!make_map(&ma, a.A, M, K, a.lda, kBM) || !make_map(&mb, a.W, N, K, a.ldw, p.bn)) return false;
+    if (a.ep.ssq_in != nullptr && !(p.splits == 1 && p.ga * p.gb >= persist_min_tiles() && persistent_enabled()))
+      return false;
     if (p.splits == 1 && (argmax || p.ga * p.gb >= persist_min_tiles()) && persistent_enabled()) {
       const int nt_major = argmax ? 1 : 0;
       if (p.bn == 256)

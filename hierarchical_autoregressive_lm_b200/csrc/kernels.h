@@ -43,6 +43,23 @@ struct Epilogue {
   // (if set) receives the fp32 logits.
   unsigned long long* argmax_part = nullptr;
   int argmax_tiles = 0;
+  // RMSNorm split across a producer / consumer pair of GEMMs (a pre-norm
+  // block's residual update and the next projection).  RMSNorm(x)[r] =
+  // rstd[r] * x[r] * g with a scalar rstd per row, so the next projection can
+  // run on bf16(x * g) and scale its accumulator by rstd[r]:
+  //  - producer (EPI_ADD_F32 of k_gemm_dec): also writes xs_out[r, c] =
+  //    bf16(x_new[r, c] * g_next[c]) (row stride ldo) and this CTA's partial
+  //    sum of x_new^2 over its columns into ssq_out[r * ssq_slots + slot];
+  //  - consumer: rstd[r] = 1 / sqrt(sum of ssq_in[r * ssq_slots + 0..ssq_slots)
+  //    in slot order / norm_d + norm_eps) multiplies the accumulator before
+  //    the rest of the epilogue.
+  void* xs_out = nullptr;  // bf16
+  const float* g_next = nullptr;
+  float* ssq_out = nullptr;
+  const float* ssq_in = nullptr;
+  int ssq_slots = 0;
+  int norm_d = 0;
+  float norm_eps = 0.f;
 };
 
 // C = A[M, K] * W[N, K]^T with A, W of the storage type, fp32 accumulation.
@@ -182,6 +199,12 @@ bool launch_gemm_tc(const GemmArgs& a, const GemmWorkspace& ws, int* err, cudaSt
 size_t gemm_tc_workspace_bytes(int M, int N, int K, int force_splits = 0, int force_swap = -1);
 // True when launch_gemm_tc takes GemmArgs with norm_x set for this shape.
 bool gemm_tc_fuses_norm(int M, int N, int K);
+// Split RMSNorm (Epilogue::xs_out / ssq_in): the number of ssq slots the
+// producer GEMM of this shape writes (its CTAs per token tile), or 0 if the
+// shape does not run on a kernel that produces them; and whether the
+// consumer of this shape applies ssq_in.
+int gemm_tc_ssq_slots(int M, int N, int K);
+bool gemm_tc_takes_ssq(int M, int N, int K);
 // Column tiles of the tcgen05 plan for an EPI_ARGMAX GEMM (0: not supported).
 int gemm_tc_argmax_tiles(int M, int N, int K);
 void launch_splitk_reduce(int dt, const float* part, int splits, int M, int N, const Epilogue& ep,

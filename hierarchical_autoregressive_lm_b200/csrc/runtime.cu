@@ -256,6 +256,7 @@ static int release_encoder(photon_model* m, cudaStream_t s) {
 }
 
 // ============================================================== cache
+constexpr int kSsqCap = 256;  // split-RMSNorm partial-sum slots per row (>= CTAs per token tile)
 static int stream_priority_high() {
   int least = 0, greatest = 0;
   if (cudaDeviceGetStreamPriorityRange(&least, &greatest) != cudaSuccess) return 0;
@@ -273,6 +274,9 @@ struct Bufs {
   float* attn_ws;
   size_t attn_ws_bytes;
   int* err;
+  void* sn_x = nullptr;    // split RMSNorm: bf16(x * g) for the next projection
+  float* sn_ss = nullptr;  // ... and its per-row partial sums of squares
+  int sn_cap = 0;          // floats per row in sn_ss
 };
 
 struct photon_cache {
@@ -301,6 +305,11 @@ struct photon_cache {
   size_t gemm_ws_bytes = 0;
   int* gemm_cnt = nullptr;
   int* gemm_cnt_t = nullptr;
+  void* sn_x = nullptr;              // split RMSNorm buffers (main chain / top branch)
+  float* sn_ss = nullptr;
+  void* sn_x_t = nullptr;
+  float* sn_ss_t = nullptr;
+  int sn_rows = 0;                   // rows sn_x / sn_ss hold (sn_x_t / sn_ss_t hold B)
   float* stk_part = nullptr;         // persistent token-step kernel: split partials
   int* stk_cnt = nullptr;            // ... its tile counters (zeroed)
   unsigned int* stk_bar = nullptr;   // ... its grid-barrier word
@@ -363,7 +372,30 @@ struct StackRun {
   const int* p0_dev = nullptr;  // device position of the first row (added to p0)
   int n_plan = 0;               // key count the decode attention is planned for
   bool xn_ready = false;        // the first block's attention norm is already in b.xn
+  int sn_rows = 0;              // rows the split-RMSNorm buffers of the Bufs hold (0: none)
 };
+
+static void gemm(photon_model* m, const Bufs& b, const void* A, long long lda, const void* W,
+                 long long ldw, int M, int N, int K, const Epilogue& ep, cudaStream_t s);
+
+static bool split_norm_enabled() {
+  static const bool on = [] {
+    const char* e = getenv("PHOTON_SPLIT_NORM");
+    return !(e && e[0] == '0');
+  }();
+  return on;
+}
+
+// Whether a block over `rows` rows can split its two RMSNorms across the
+// neighbouring GEMMs (O and W2 produce, QKV and W1 consume); false keeps the
+// norm kernels.
+static bool split_norm_ok(const photon_model* m, const Bufs& b, int rows, int cap_rows) {
+  if (!m->use_tc || !b.sn_x || !b.sn_ss || !split_norm_enabled() || rows > cap_rows) return false;
+  const int d = m->d, f = m->f;
+  const int so = gemm_tc_ssq_slots(rows, d, d), s2 = gemm_tc_ssq_slots(rows, d, f);
+  return so > 0 && so <= b.sn_cap && s2 > 0 && s2 <= b.sn_cap && gemm_tc_takes_ssq(rows, 3 * d, d) &&
+         gemm_tc_takes_ssq(rows, f, d);
+}
 
 static void gemm(photon_model* m, const Bufs& b, const void* A, long long lda, const void* W,
                  long long ldw, int M, int N, int K, const Epilogue& ep, cudaStream_t s) {
@@ -377,6 +409,12 @@ static void gemm(photon_model* m, const Bufs& b, const void* A, long long lda, c
   g.K = K;
   g.ep = ep;
   GemmWorkspace ws{b.gemm_ws, b.gemm_ws_bytes, b.gemm_cnt, b.gemm_cnt ? kGemmTileCounters : 0};
+  if (ep.ssq_in != nullptr || ep.xs_out != nullptr) {
+    // split-RMSNorm roles exist only on the tcgen05 paths the planner chose;
+    // a refusal here is a planning bug: flag it on the device error word
+    if (!launch_gemm_tc(g, ws, b.err, s)) cudaMemsetAsync(b.err, 0x7f, sizeof(int), s);
+    return;
+  }
   if (m->use_tc)
     launch_gemm(m->dt, g, ws, b.err, s);
   else
@@ -432,9 +470,15 @@ static Epilogue epi(int kind, void* out, long long ldo) {
 }
 
 // Pre-norm block (reading R8-R11): x += Attn(RMSNorm(x)); x += MLP(RMSNorm(x)).
+// One pre-norm block.  sn_slots: on entry, > 0 when the previous block's W2
+// already produced bf16(x * g_attn) and its row sums of squares (split
+// RMSNorm, slots of that GEMM); on return, the same for the next block
+// (g_next = its attention gain, null for the last block of the stack).
 static void run_block(photon_model* m, const BlockW& w, float* x, const StackRun& r, int layer,
-                      const Bufs& b, cudaStream_t s) {
+                      const Bufs& b, cudaStream_t s, int& sn_slots, const float* g_next) {
   const int d = m->d, rows = r.G * r.q_len;
+  const float eps = m->cfg.norm_eps;
+  const bool sn = split_norm_ok(m, b, rows, r.sn_rows);
   Epilogue e;
   e.kind = EPI_QKV;
   e.q_out = b.q;
@@ -449,7 +493,15 @@ static void run_block(photon_model* m, const BlockW& w, float* x, const StackRun
   e.kv_off = r.kv_off;
   e.rope = b.rope;
   e.p0_dev = r.p0_dev;
-  gemm_normed(m, b, x, w.g_attn, w.wqkv, d, rows, 3 * d, d, e, s, r.xn_ready && layer == 0);
+  if (sn && sn_slots > 0) {
+    e.ssq_in = b.sn_ss;
+    e.ssq_slots = sn_slots;
+    e.norm_d = d;
+    e.norm_eps = eps;
+    gemm(m, b, b.sn_x, d, w.wqkv, d, rows, 3 * d, d, e, s);
+  } else {
+    gemm_normed(m, b, x, w.g_attn, w.wqkv, d, rows, 3 * d, d, e, s, r.xn_ready && layer == 0);
+  }
 
   AttnArgs a;
   a.Q = b.q;
@@ -477,14 +529,45 @@ static void run_block(photon_model* m, const BlockW& w, float* x, const StackRun
   if (r.q_len <= 4) done = launch_attn_decode(m->dt, a, b.attn_ws, b.attn_ws_bytes, b.err, s);
   if (!done) launch_attn_prefill(m->dt, a, s);
 
-  gemm(m, b, b.att, d, w.wo, d, rows, d, d, epi(EPI_ADD_F32, x, d), s);
-  gemm_normed(m, b, x, w.g_mlp, w.w1, d, rows, m->f, d, epi(EPI_GELU_T, b.hid, m->f), s);
-  gemm(m, b, b.hid, m->f, w.w2, m->f, rows, d, m->f, epi(EPI_ADD_F32, x, d), s);
+  Epilogue eo = epi(EPI_ADD_F32, x, d);
+  int slots_o = 0;
+  if (sn) {  // O projection also produces the MLP norm's operand
+    slots_o = gemm_tc_ssq_slots(rows, d, d);
+    eo.xs_out = b.sn_x;
+    eo.g_next = w.g_mlp;
+    eo.ssq_out = b.sn_ss;
+    eo.ssq_slots = slots_o;
+  }
+  gemm(m, b, b.att, d, w.wo, d, rows, d, d, eo, s);
+  if (sn) {
+    Epilogue e1 = epi(EPI_GELU_T, b.hid, m->f);
+    e1.ssq_in = b.sn_ss;
+    e1.ssq_slots = slots_o;
+    e1.norm_d = d;
+    e1.norm_eps = eps;
+    gemm(m, b, b.sn_x, d, w.w1, d, rows, m->f, d, e1, s);
+  } else {
+    gemm_normed(m, b, x, w.g_mlp, w.w1, d, rows, m->f, d, epi(EPI_GELU_T, b.hid, m->f), s);
+  }
+  Epilogue e2 = epi(EPI_ADD_F32, x, d);
+  sn_slots = 0;
+  if (sn && g_next) {  // W2 also produces the next block's attention-norm operand
+    const int sl = gemm_tc_ssq_slots(rows, d, m->f);
+    e2.xs_out = b.sn_x;
+    e2.g_next = g_next;
+    e2.ssq_out = b.sn_ss;
+    e2.ssq_slots = sl;
+    sn_slots = sl;
+  }
+  gemm(m, b, b.hid, m->f, w.w2, m->f, rows, d, m->f, e2, s);
 }
 
 static void run_stack(photon_model* m, int first, int n_layers, float* x, const StackRun& r,
                       const Bufs& b, cudaStream_t s) {
-  for (int l = 0; l < n_layers; ++l) run_block(m, m->block(first, l), x, r, l, b, s);
+  int sn_slots = 0;
+  for (int l = 0; l < n_layers; ++l)
+    run_block(m, m->block(first, l), x, r, l, b, s, sn_slots,
+              l + 1 < n_layers ? m->block(first, l + 1).g_attn : nullptr);
 }
 
 static size_t gemm_ws_need(const photon_model* m, int M, int N, int K) {
@@ -541,6 +624,9 @@ static Bufs decode_bufs(photon_cache* c) {
   b.attn_ws = c->attn_ws;
   b.attn_ws_bytes = c->attn_ws_bytes;
   b.err = c->d_err;
+  b.sn_x = c->sn_x;
+  b.sn_ss = c->sn_ss;
+  b.sn_cap = c->sn_x ? kSsqCap : 0;
   return b;
 }
 
@@ -771,6 +857,12 @@ int photon_prefill(photon_model* m, const photon_cache* prefix, const int32_t* d
   c->gemm_cnt = al.get<int>(kGemmTileCounters * sizeof(int));
   c->gemm_cnt_t = al.get<int>(kGemmTileCounters * sizeof(int));
   if (m->use_tc) {
+    const size_t srows = (size_t)std::max(rows_g * C1, std::max(rows_g, B));
+    c->sn_rows = (int)srows;
+    c->sn_x = al.get<void>(srows * d * es);
+    c->sn_ss = al.get<float>(srows * kSsqCap * sizeof(float));
+    c->sn_x_t = al.get<void>((size_t)B * d * es);
+    c->sn_ss_t = al.get<float>((size_t)B * kSsqCap * sizeof(float));
     c->stk_cnt_len = (d / 128) * ((B * C2 + 63) / 64);
     c->stk_part = al.get<float>(stack_local_scratch_bytes(B * C2, d));
     c->stk_cnt = al.get<int>((size_t)c->stk_cnt_len * sizeof(int));
@@ -984,6 +1076,7 @@ static void enqueue_decode(photon_model* m, photon_cache* c, int mode, int32_t* 
     rt.p0 = 0;
     rt.p0_dev = c->d_pos;
     rt.n_plan = c->n_pre + c->Ncap;
+    rt.sn_rows = c->sn_x_t ? B : 0;
     rt.kv_off = c->n_pre;
     rt.kc = c->top_k;
     rt.vc = c->top_v;
@@ -1011,6 +1104,7 @@ static void enqueue_decode(photon_model* m, photon_cache* c, int mode, int32_t* 
   r2.vc = c->d2v;
   r2.layer_bytes = c->d2_layer;
   r2.cap = C2;
+  r2.sn_rows = c->sn_rows;
   run_stack(m, m->i_dec2, m->Ld2, c->xd, r2, b, s);
   launch_rmsnorm(m->dt, c->xd, (const float*)m->ptr(m->i_dec2_g), c->a_hat, G, d, 1, 0, eps, s);
   // RecGen: the top encoder's next input is Chunker_2(A-hat) and does not
@@ -1029,6 +1123,8 @@ static void enqueue_decode(photon_model* m, photon_cache* c, int mode, int32_t* 
     bt.gemm_ws = c->gemm_ws_t;
     bt.gemm_cnt = c->gemm_cnt_t;
     bt.attn_ws = c->attn_ws_t;
+    bt.sn_x = c->sn_x_t;
+    bt.sn_ss = c->sn_ss_t;
     const void* src = d_force_a ? d_force_a : c->a_hat;
     gemm(m, bt, src, (long long)C2 * d, m->ptr(m->i_ch2), (long long)C2 * d, B, d, C2 * d,
          epi(EPI_STORE_F32, c->xt, d), c->side);
@@ -1053,6 +1149,7 @@ static void enqueue_decode(photon_model* m, photon_cache* c, int mode, int32_t* 
   r1.vc = c->d1v;
   r1.layer_bytes = c->d1_layer;
   r1.cap = 2 * C1;
+  r1.sn_rows = c->sn_rows;
   run_stack(m, m->i_dec1, m->Ld1, c->xd, r1, b, ts);
   const int amax_tiles = m->use_tc ? gemm_tc_argmax_tiles(G, V, d) : 0;
   bool fused_embed = false;  // the last head also embedded and normalised the next step's input
@@ -1125,6 +1222,7 @@ static void enqueue_decode(photon_model* m, photon_cache* c, int mode, int32_t* 
     re.vc = c->l1_v;
     re.layer_bytes = c->l1_layer;
     re.cap = c->N1cap;
+    re.sn_rows = c->sn_rows;
     if (c->prefix) {
       re.kp = c->prefix->l1_k;
       re.vp = c->prefix->l1_v;
