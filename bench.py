@@ -161,6 +161,7 @@ def run_gpu(args) -> None:
     toks_host = torch.from_numpy(np.ascontiguousarray(toks_all[lo:hi]))
     toks = toks_host.to(dev)
     out = torch.empty(B, chunks * C, dtype=torch.int32, device=dev)
+    step_out = torch.empty(B, C, dtype=torch.int32, device=dev)
     stream = torch.cuda.current_stream()
 
     def one_step(ev=None, mark=False):
@@ -175,12 +176,22 @@ def run_gpu(args) -> None:
             torch.cuda.nvtx.range_pop()
         if ev is not None:
             ev[1].record(stream)
-        for s in range(chunks):
-            if mark and s == chunks // 2:
-                torch.cuda.nvtx.range_push("decode_chunk")
-            cache.step_rec(out[:, s * C:(s + 1) * C])
-            if mark and s == chunks // 2:
+        if args.decode_api == "chunks":
+            # all chunks in one call: each chunk's token decoder overlaps the
+            # next chunk's main chain
+            if mark:
+                torch.cuda.nvtx.range_push("decode")
+            cache.decode_rec_chunks(chunks, out)
+            if mark:
                 torch.cuda.nvtx.range_pop()
+        else:
+            for s in range(chunks):
+                if mark and s == chunks // 2:
+                    torch.cuda.nvtx.range_push("decode_chunk")
+                cache.step_rec(step_out)  # the per-step API writes a contiguous [B, C]
+                out[:, s * C:(s + 1) * C].copy_(step_out)
+                if mark and s == chunks // 2:
+                    torch.cuda.nvtx.range_pop()
         if ev is not None:
             ev[2].record(stream)
         return cache
@@ -198,7 +209,6 @@ def run_gpu(args) -> None:
     resident = minfo["resident_bytes"] + cinfo["kv_bytes"]
 
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
-    caches = []
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
@@ -209,13 +219,13 @@ def run_gpu(args) -> None:
         t0 = torch.cuda.Event(enable_timing=True)
         t1 = torch.cuda.Event(enable_timing=True)
         t0.record(stream)
-        for k in range(args.steps):      # caches are freed after the timed region
-            caches.append(one_step(evs[k], mark=(k == 0)))
+        for k in range(args.steps):
+            # a served batch: prefill, decode, release (stream-ordered, so the
+            # next prefill reuses the memory without a host wait)
+            one_step(evs[k], mark=(k == 0)).free()
         t1.record(stream)
         torch.cuda.synchronize()
     launches = hal.launch_count() - n_launch0
-    for c in caches:
-        c.free()
     if world > 1:
         dist.barrier()
     total_ms = t0.elapsed_time(t1)
@@ -236,11 +246,14 @@ def run_gpu(args) -> None:
     for _ in range(e2e_steps):
         dev_in.copy_(pin_in, non_blocking=True)
         cache = model.prefill(dev_in, hal.MODE_REC, chunks)
-        for s in range(chunks):
-            sl = out[:, s * C:(s + 1) * C]
-            cache.step_rec(sl)
-            pin_out[:, s * C:(s + 1) * C].copy_(sl, non_blocking=True)
-        cache.free()     # synchronises
+        if args.decode_api == "chunks":
+            cache.decode_rec_chunks(chunks, out)
+            pin_out.copy_(out, non_blocking=True)
+        else:
+            for s in range(chunks):
+                cache.step_rec(step_out)
+                pin_out[:, s * C:(s + 1) * C].copy_(step_out, non_blocking=True)
+        cache.free()
     e1.record(stream)
     torch.cuda.synchronize()
     e2e_ms = e0.elapsed_time(e1)
@@ -254,7 +267,7 @@ def run_gpu(args) -> None:
         if ev is not None:
             ev[1].record(stream)
         for s in range(chunks):
-            c.step_hier(out[:, s * C:(s + 1) * C])
+            c.step_hier(step_out)
         if ev is not None:
             ev[2].record(stream)
         return c
@@ -289,7 +302,8 @@ def run_gpu(args) -> None:
         "config": {"workload": f"{args.workload}: PHOTON 600M-class L=2 C1=C2={shape['C1']}, "
                                f"B={B} per GPU, prompt {T}, RecGen decode {chunks * C} tokens",
                    "batch_per_gpu": B, "prompt_len": T, "decode_tokens": chunks * C,
-                   "parallelism": f"dp{world}", "l2": "working set > L2 (no flush)"},
+                   "parallelism": f"dp{world}", "l2": "working set > L2 (no flush)",
+                   "decode_api": args.decode_api},
         "decode_ms_per_step": round(decode_ms / args.steps, 3),
         "decode_ms_per_chunk": round(decode_ms / args.steps / chunks, 4),
         "prefill_tok_s": round(world * B * T * args.steps / (prefill_ms / 1e3), 1),
@@ -302,7 +316,9 @@ def run_gpu(args) -> None:
                 "per_gpu": True},
         "e2e": {"value": round(world * B * chunks * C * e2e_steps / (e2e_ms / 1e3), 1), "unit": UNIT,
                 "h2d_bytes_per_step": int(B * T * 4), "d2h_bytes_per_step": int(B * chunks * C * 4),
-                "covers": "H2D prompt + prefill + RecGen decode + per-chunk D2H of tokens"},
+                "covers": "H2D prompt + prefill + RecGen decode + D2H of the tokens"
+                          + (" (one multi-chunk decode call)" if args.decode_api == "chunks"
+                             else " (per-chunk calls and copies)")},
         "hiergen": {"decode_tok_s": round(job_throughput(B * chunks * C, world, hier_dec_ms), 1),
                     "decode_ms_per_chunk": round(hier_dec_ms / chunks, 4),
                     "resident_gib": round(hier_res / 2 ** 30, 4),
@@ -602,6 +618,8 @@ def main() -> None:
     ap.add_argument("--impl", default="photon", choices=["photon", "reference"])
     ap.add_argument("--cpu-budget", type=float, default=20.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--decode-api", default="chunks", choices=["chunks", "steps"],
+                    help="RecGen decode through one multi-chunk call (default) or per-chunk calls")
     ap.add_argument("--only-roofline", action="store_true",
                     help="run only the kernel roofline measurements (profiling case)")
     args = ap.parse_args()

@@ -29,6 +29,7 @@ _ERRORS = {-1: "PHOTON_ERR_ARG", -2: "PHOTON_ERR_OOM", -3: "PHOTON_ERR_CUDA",
 # Every entry point of include/photon.h (checked against the header by the tests).
 EXPORTED = ("photon_init_weights", "photon_free_model", "photon_prefill",
             "photon_decode_step_hier", "photon_decode_step_rec", "photon_decode_step_ex",
+            "photon_decode_rec_chunks",
             "photon_free_cache", "photon_cache_info", "photon_model_info",
             "photon_export_weight", "photon_export_state", "photon_gemm", "photon_gemm_rmsnorm",
             "photon_attn_decode", "photon_attn_decode_noalloc", "photon_launch_count",
@@ -86,6 +87,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "photon_decode_step_hier": [P, P, P, P, P],
         "photon_decode_step_rec": [P, P, P, P, P],
         "photon_decode_step_ex": [P, P, I32, P, P, P, P, P],
+        "photon_decode_rec_chunks": [P, P, I32, P, P],
         "photon_free_cache": [P],
         "photon_cache_info": [P, ctypes.POINTER(photon_cache_stats)],
         "photon_model_info": [P, ctypes.POINTER(photon_model_stats)],
@@ -215,6 +217,12 @@ class Cache:
     def step_hier(self, out_tokens, out_logits=None, stream=None) -> None:
         _check(load_library().photon_decode_step_hier(self.model._h, self._h, _ptr(out_tokens),
                                                       _ptr(out_logits), _stream(stream)))
+
+    def decode_rec_chunks(self, n_chunks: int, out_tokens, stream=None) -> None:
+        """n RecGen chunks in one call; out_tokens int32 [B, n_chunks * C] on the device
+        (each chunk's token decoder overlapped with the next chunk's main chain)."""
+        _check(load_library().photon_decode_rec_chunks(self.model._h, self._h, n_chunks,
+                                                       _ptr(out_tokens), _stream(stream)))
 
     def info(self) -> dict:
         st = photon_cache_stats()

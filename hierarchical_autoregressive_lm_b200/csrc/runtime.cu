@@ -96,6 +96,14 @@ struct photon_model {
   cudaGraphExec_t graph[2] = {nullptr, nullptr};
   const void* graph_owner[2] = {nullptr, nullptr};
   long long graph_kernels[2] = {0, 0};  // kernel launches captured in graph[mode]
+  // pipelined RecGen graphs [main/token part][A-hat parity], reused across
+  // caches through executable updates; pg_owner = the cache captured last
+  cudaGraphExec_t pg[2][2] = {{nullptr, nullptr}, {nullptr, nullptr}};
+  const void* pg_owner = nullptr;
+  long long pg_kernels[2] = {0, 0};
+  // one event per stream that has enqueued work reading the level-1 encoder
+  // weights since they were generated; their release waits on all of them
+  std::vector<std::pair<cudaStream_t, cudaEvent_t>> enc_users;
 
   const void* ptr(int idx) const { return group_ptr[t[idx].group] + t[idx].offset; }
   BlockW block(int first, int l) const {
@@ -248,8 +256,27 @@ static int ensure_encoder(photon_model* m, cudaStream_t s) {
   CK(cudaGetLastError());
   return PHOTON_OK;
 }
+// Marks the end of the work just enqueued on `s` that reads the encoder.
+static int note_encoder_use(photon_model* m, cudaStream_t s) {
+  for (auto& u : m->enc_users)
+    if (u.first == s) {
+      CK(cudaEventRecord(u.second, s));
+      return PHOTON_OK;
+    }
+  cudaEvent_t e = nullptr;
+  CK(cudaEventCreateWithFlags(&e, cudaEventDisableTiming));
+  m->enc_users.emplace_back(s, e);
+  CK(cudaEventRecord(e, s));
+  return PHOTON_OK;
+}
+// Stream-ordered release on `s`, after every user stream's last recorded use.
 static int release_encoder(photon_model* m, cudaStream_t s) {
   if (!m->group_ptr[G_ENC1]) return PHOTON_OK;
+  for (auto& u : m->enc_users) {
+    CK(cudaStreamWaitEvent(s, u.second, 0));
+    cudaEventDestroy(u.second);
+  }
+  m->enc_users.clear();
   CK(cudaFreeAsync(m->group_ptr[G_ENC1], s));
   m->group_ptr[G_ENC1] = nullptr;
   return PHOTON_OK;
@@ -310,6 +337,18 @@ struct photon_cache {
   void* sn_x_t = nullptr;
   float* sn_ss_t = nullptr;
   int sn_rows = 0;                   // rows sn_x / sn_ss hold (sn_x_t / sn_ss_t hold B)
+  // pipelined RecGen (photon_decode_rec_chunks): the token branch of a chunk
+  // overlaps the next chunk's main chain, so it gets its own buffers, A-hat
+  // is double-buffered, and both halves are captured as separate graphs
+  bool pipe_ready = false;
+  void* ahat_p[2] = {nullptr, nullptr};
+  const void* ahat_latest = nullptr;  // the A-hat of the last decode step
+  float* xd_k = nullptr;
+  void *xn_k = nullptr, *q_k = nullptr, *att_k = nullptr, *hid_k = nullptr, *sn_x_k = nullptr;
+  float *gemm_ws_k = nullptr, *attn_ws_k = nullptr, *sn_ss_k = nullptr;
+  int* gemm_cnt_k = nullptr;
+  cudaStream_t tstream = nullptr;
+  cudaEvent_t ev_main[2] = {nullptr, nullptr}, ev_tok[2] = {nullptr, nullptr};
   float* stk_part = nullptr;         // persistent token-step kernel: split partials
   int* stk_cnt = nullptr;            // ... its tile counters (zeroed)
   unsigned int* stk_bar = nullptr;   // ... its grid-barrier word
@@ -691,8 +730,13 @@ int photon_free_model(photon_model* m) {
   if (!m) return fail(PHOTON_ERR_ARG, "model is NULL");
   if (m->live_caches) return fail(PHOTON_ERR_ARG, "%d caches still use this model", m->live_caches);
   CK(cudaDeviceSynchronize());
-  for (int k = 0; k < 2; ++k)
+  for (auto& u : m->enc_users) cudaEventDestroy(u.second);
+  m->enc_users.clear();
+  for (int k = 0; k < 2; ++k) {
     if (m->graph[k]) cudaGraphExecDestroy(m->graph[k]);
+    for (int p = 0; p < 2; ++p)
+      if (m->pg[k][p]) cudaGraphExecDestroy(m->pg[k][p]);
+  }
   for (int g = 0; g < G_COUNT; ++g)
     if (m->group_ptr[g]) cudaFree(m->group_ptr[g]);
   delete m;
@@ -733,6 +777,7 @@ int photon_export_weight(photon_model* m, int32_t index, void* d_dst, size_t dst
   cudaStream_t s = (cudaStream_t)stream;
   if (r.group == G_ENC1) RET(ensure_encoder(m, s));
   CK(cudaMemcpyAsync(d_dst, m->ptr(index), bytes, cudaMemcpyDeviceToDevice, s));
+  if (r.group == G_ENC1) RET(note_encoder_use(m, s));
   return PHOTON_OK;
 }
 
@@ -982,10 +1027,13 @@ int photon_prefill(photon_model* m, const photon_cache* prefix, const int32_t* d
     if (cudaMemcpyAsync(c->d_pos, pos, sizeof(pos), cudaMemcpyHostToDevice, s) != cudaSuccess)
       return bail(fail(PHOTON_ERR_CUDA, "position upload failed"));
   }
+  // RecGen never reads the encoder again: drop it unless a HierGen cache does
+  if (note_encoder_use(m, s) != PHOTON_OK ||
+      (mode != PHOTON_MODE_HIER && m->hier_caches == 0 && release_encoder(m, s) != PHOTON_OK))
+    return bail(PHOTON_ERR_CUDA);
   m->live_caches++;
   if (mode == PHOTON_MODE_HIER) m->hier_caches++;
   if (prefix) prefix->dependents++;
-  if (m->hier_caches == 0) release_encoder(m, s);
   *out = c;
   return PHOTON_OK;
 }
@@ -1062,13 +1110,38 @@ static bool token_step_persistent(photon_model* m, photon_cache* c, const Bufs& 
   return launch_stack_local(k, s);
 }
 
+// Which part of a decode step to enqueue: the whole step, or (pipelined
+// RecGen) only the main chain (Converter_2, Decoder_2, Chunker_2, top step)
+// or only the token branch (Converter_1, token decoder, heads) of A-hat
+// buffer `parity`.
+enum DecodePart { DEC_ALL = 0, DEC_MAIN = 1, DEC_TOK = 2 };
+
+static Bufs tok_bufs(photon_cache* c) {
+  Bufs b = decode_bufs(c);
+  b.xn = c->xn_k;
+  b.q = c->q_k;
+  b.att = c->att_k;
+  b.hid = c->hid_k;
+  b.gemm_ws = c->gemm_ws_k;
+  b.gemm_cnt = c->gemm_cnt_k;
+  b.attn_ws = c->attn_ws_k;
+  b.sn_x = c->sn_x_k;
+  b.sn_ss = c->sn_ss_k;
+  return b;
+}
+
 static void enqueue_decode(photon_model* m, photon_cache* c, int mode, int32_t* own_tokens,
                            float* d_out_logits, const int32_t* d_force_tokens,
-                           const void* d_force_a, cudaStream_t s) {
+                           const void* d_force_a, cudaStream_t s, int part = DEC_ALL,
+                           int parity = 0) {
   int32_t* d_out_tokens = own_tokens;
   const int B = c->B, C1 = m->C1, C2 = m->C2, C = m->C, d = m->d, V = m->V, G = B * C2;
   const float eps = m->cfg.norm_eps;
   const Bufs b = decode_bufs(c);
+  // A-hat of this step; the token branch's buffers and residual stream
+  void* const ahat = part == DEC_ALL ? c->a_hat : c->ahat_p[parity];
+  const Bufs bk = part == DEC_TOK ? tok_bufs(c) : b;
+  float* const xdk = part == DEC_TOK ? c->xd_k : c->xd;
   auto top_step = [&](float* x, const Bufs& bb, cudaStream_t st) {
     StackRun rt;
     rt.G = B;
@@ -1094,6 +1167,7 @@ static void enqueue_decode(photon_model* m, photon_cache* c, int mode, int32_t* 
     launch_advance(c->d_pos, 1, mode == PHOTON_MODE_HIER ? C2 : 0, st);
   };
 
+  if (part != DEC_TOK) {
   // a7: Converter_2 -- o [B, d] -> C2 conditioning vectors per sequence
   gemm(m, b, c->o, d, m->ptr(m->i_cv2), d, B, C2 * d, d, epi(EPI_STORE_F32, c->xd, (long long)C2 * d), s);
   // a8: level-2 decoder over its C2 positions (chunk-local causal) -> A-hat
@@ -1106,12 +1180,21 @@ static void enqueue_decode(photon_model* m, photon_cache* c, int mode, int32_t* 
   r2.cap = C2;
   r2.sn_rows = c->sn_rows;
   run_stack(m, m->i_dec2, m->Ld2, c->xd, r2, b, s);
-  launch_rmsnorm(m->dt, c->xd, (const float*)m->ptr(m->i_dec2_g), c->a_hat, G, d, 1, 0, eps, s);
+  launch_rmsnorm(m->dt, c->xd, (const float*)m->ptr(m->i_dec2_g), ahat, G, d, 1, 0, eps, s);
+  if (part == DEC_MAIN) {
+    // pipelined RecGen: the top encoder's next input follows at once; the
+    // token branch of this A-hat runs as its own graph
+    gemm(m, b, ahat, (long long)C2 * d, m->ptr(m->i_ch2), (long long)C2 * d, B, d, C2 * d,
+         epi(EPI_STORE_F32, c->xt, d), s);
+    top_step(c->xt, b, s);
+    return;
+  }
+  }
   // RecGen: the top encoder's next input is Chunker_2(A-hat) and does not
   // depend on the tokens, so the top-encoder branch (a12-R, a13) runs on the
   // side stream, with its own buffers, while the token decoder (a9-a11)
   // runs here; the two chains join at the end of the step.
-  const bool fork = mode == PHOTON_MODE_REC && c->side != nullptr && recgen_fork_enabled();
+  const bool fork = part == DEC_ALL && mode == PHOTON_MODE_REC && c->side != nullptr && recgen_fork_enabled();
   if (fork) {
     cudaEventRecord(c->ev_fork, s);
     cudaStreamWaitEvent(c->side, c->ev_fork, 0);
@@ -1125,7 +1208,7 @@ static void enqueue_decode(photon_model* m, photon_cache* c, int mode, int32_t* 
     bt.attn_ws = c->attn_ws_t;
     bt.sn_x = c->sn_x_t;
     bt.sn_ss = c->sn_ss_t;
-    const void* src = d_force_a ? d_force_a : c->a_hat;
+    const void* src = d_force_a ? d_force_a : ahat;
     gemm(m, bt, src, (long long)C2 * d, m->ptr(m->i_ch2), (long long)C2 * d, B, d, C2 * d,
          epi(EPI_STORE_F32, c->xt, d), c->side);
     top_step(c->xt, bt, c->side);
@@ -1139,7 +1222,7 @@ static void enqueue_decode(photon_model* m, photon_cache* c, int mode, int32_t* 
     ts = c->hi;
   }
   // a9: Converter_1 -- each A-hat row -> C1 conditioning vectors (rows g*C1 + i)
-  gemm(m, b, c->a_hat, d, m->ptr(m->i_cv1), d, G, C1 * d, d, epi(EPI_STORE_F32, c->xd, (long long)C1 * d), ts);
+  gemm(m, bk, ahat, d, m->ptr(m->i_cv1), d, G, C1 * d, d, epi(EPI_STORE_F32, xdk, (long long)C1 * d), ts);
   // a10/a11: token decoder, prefix pass over the C1 conditioning positions,
   // then C1-1 single-row steps; head + greedy argmax after each
   StackRun r1;
@@ -1150,7 +1233,7 @@ static void enqueue_decode(photon_model* m, photon_cache* c, int mode, int32_t* 
   r1.layer_bytes = c->d1_layer;
   r1.cap = 2 * C1;
   r1.sn_rows = c->sn_rows;
-  run_stack(m, m->i_dec1, m->Ld1, c->xd, r1, b, ts);
+  run_stack(m, m->i_dec1, m->Ld1, xdk, r1, bk, ts);
   const int amax_tiles = m->use_tc ? gemm_tc_argmax_tiles(G, V, d) : 0;
   bool fused_embed = false;  // the last head also embedded and normalised the next step's input
   auto head = [&](const float* x, int in_step, int in_off, int i) {
@@ -1162,12 +1245,12 @@ static void enqueue_decode(photon_model* m, photon_cache* c, int mode, int32_t* 
       Epilogue e = epi(EPI_ARGMAX, d_out_logits ? d_out_logits + (size_t)i * V : nullptr, ld);
       e.argmax_part = c->amax_part;
       e.argmax_tiles = amax_tiles;
-      gemm(m, b, c->hn, d, m->ptr(m->i_head), d, G, V, d, e, ts);
+      gemm(m, bk, c->hn, d, m->ptr(m->i_head), d, G, V, d, e, ts);
       if (i + 1 < C1) {
         // greedy choice + the next step's embedding and first attention norm
         launch_argmax_embed_norm(m->dt, c->amax_part, amax_tiles, G, V, i, C1, d_force_tokens,
                                  d_out_tokens, c->used, c->next_ids, c->d_err, m->ptr(m->i_embed),
-                                 c->xs, m->block(m->i_dec1, 0).g_attn, b.xn, d, eps, ts);
+                                 c->xs, m->block(m->i_dec1, 0).g_attn, bk.xn, d, eps, ts);
         fused_embed = true;
       } else {
         launch_argmax_partials(c->amax_part, amax_tiles, G, V, i, C1, d_force_tokens, d_out_tokens,
@@ -1175,12 +1258,12 @@ static void enqueue_decode(photon_model* m, photon_cache* c, int mode, int32_t* 
       }
     } else {
       float* lg = d_out_logits ? d_out_logits + (size_t)i * V : c->logits;
-      gemm(m, b, c->hn, d, m->ptr(m->i_head), d, G, V, d, epi(EPI_STORE_F32, lg, ld), ts);
+      gemm(m, bk, c->hn, d, m->ptr(m->i_head), d, G, V, d, epi(EPI_STORE_F32, lg, ld), ts);
       launch_argmax(lg, ld, G, V, i, C1, d_force_tokens, d_out_tokens, c->used, c->next_ids,
                     c->d_err, ts);
     }
   };
-  head(c->xd, C1, C1 - 1, 0);
+  head(xdk, C1, C1 - 1, 0);
   for (int i = 1; i < C1; ++i) {
     if (!fused_embed)
       launch_embed_f32(m->dt, c->next_ids, m->ptr(m->i_embed), c->xs, G, d, V, c->d_err, ts);
@@ -1189,9 +1272,10 @@ static void enqueue_decode(photon_model* m, photon_cache* c, int mode, int32_t* 
     rs.p0 = C1 + i - 1;
     rs.xn_ready = fused_embed;
     fused_embed = false;
-    if (!token_step_persistent(m, c, b, c->xs, rs, ts)) run_stack(m, m->i_dec1, m->Ld1, c->xs, rs, b, ts);
+    if (!token_step_persistent(m, c, bk, c->xs, rs, ts)) run_stack(m, m->i_dec1, m->Ld1, c->xs, rs, bk, ts);
     head(c->xs, 1, 0, i);
   }
+  if (part == DEC_TOK) return;
   // a12: input of the top encoder's next position
   if (fork) {
     if (ts != s) {
@@ -1309,19 +1393,160 @@ int photon_decode_step_ex(photon_model* m, photon_cache* c, int32_t mode, int32_
     CK(cudaGraphLaunch(m->graph[mode], s));
     note_launch(m->graph_kernels[mode]);
     c->graph_steps += 1;
-    CK(cudaMemcpyAsync(d_out_tokens, c->tok_out, (size_t)c->B * m->C * sizeof(int32_t),
-                       cudaMemcpyDeviceToDevice, s));
+    if (d_out_tokens != c->tok_out)
+      CK(cudaMemcpyAsync(d_out_tokens, c->tok_out, (size_t)c->B * m->C * sizeof(int32_t),
+                         cudaMemcpyDeviceToDevice, s));
   } else {
     enqueue_decode(m, c, mode, d_out_tokens, d_out_logits, d_force_tokens, d_force_a, s);
   }
   CK(cudaGetLastError());
+  if (mode == PHOTON_MODE_HIER) RET(note_encoder_use(m, s));
   c->N += 1;
   if (mode == PHOTON_MODE_HIER) {
     c->N1 += C2;
     c->has_a = true;
   }
   c->has_a_hat = true;
+  c->ahat_latest = c->a_hat;
   c->steps += 1;
+  return PHOTON_OK;
+}
+
+// ------------------------------------------------------------------ pipelined RecGen
+static bool pipeline_enabled() {
+  static const bool on = [] {
+    const char* e = getenv("PHOTON_RECGEN_PIPELINE");
+    return !(e && e[0] == '0');
+  }();
+  return on;
+}
+
+// Token-branch buffers, double-buffered A-hat, stream and events of the
+// pipelined RecGen path (allocated on the first call, counted as cache memory).
+static int prepare_pipeline(photon_model* m, photon_cache* c, cudaStream_t s) {
+  if (c->pipe_ready) return PHOTON_OK;
+  const int B = c->B, d = m->d, C = m->C, rows_c = B * C, rows_g = B * m->C2;
+  const size_t es = m->es;
+  Allocator al{s, &c->allocs, &c->kv_bytes};
+  c->ahat_p[0] = al.get<void>((size_t)rows_g * d * es);
+  c->ahat_p[1] = al.get<void>((size_t)rows_g * d * es);
+  c->xd_k = al.get<float>((size_t)rows_c * d * 4);
+  c->xn_k = al.get<void>((size_t)rows_c * d * es);
+  c->q_k = al.get<void>((size_t)rows_c * d * es);
+  c->att_k = al.get<void>((size_t)rows_c * d * es);
+  c->hid_k = al.get<void>((size_t)rows_c * m->f * es);
+  c->gemm_ws_k = al.get<float>(c->gemm_ws_bytes);
+  c->attn_ws_k = al.get<float>(c->attn_ws_bytes);
+  c->gemm_cnt_k = al.get<int>(kGemmTileCounters * sizeof(int));
+  if (c->sn_x) {
+    c->sn_x_k = al.get<void>((size_t)c->sn_rows * d * es);
+    c->sn_ss_k = al.get<float>((size_t)c->sn_rows * kSsqCap * sizeof(float));
+  }
+  if (al.err != cudaSuccess) return fail(PHOTON_ERR_OOM, "device allocation failed (pipelined decode buffers)");
+  CK(cudaMemsetAsync(c->gemm_cnt_k, 0, kGemmTileCounters * sizeof(int), s));
+  if (!c->tstream) {
+    CK(cudaStreamCreateWithFlags(&c->tstream, cudaStreamNonBlocking));
+    for (int p = 0; p < 2; ++p) {
+      CK(cudaEventCreateWithFlags(&c->ev_main[p], cudaEventDisableTiming));
+      CK(cudaEventCreateWithFlags(&c->ev_tok[p], cudaEventDisableTiming));
+    }
+  }
+  c->pipe_ready = true;
+  return PHOTON_OK;
+}
+
+// Captures one half of a pipelined step (part DEC_MAIN or DEC_TOK, A-hat
+// buffer `parity`) on the cache's capture stream; the launch counter keeps
+// counting kernels that run (taken back here, added at every launch).
+static bool capture_part(photon_model* m, photon_cache* c, int part, int parity, cudaGraphExec_t* exec,
+                         long long* kernels) {
+  cudaGraph_t g = nullptr;
+  const unsigned long long n0 = launch_total();
+  bool ok = cudaStreamBeginCapture(c->cap, cudaStreamCaptureModeRelaxed) == cudaSuccess;
+  if (ok) {
+    enqueue_decode(m, c, PHOTON_MODE_REC, c->tok_out, nullptr, nullptr, nullptr, c->cap, part, parity);
+    ok = cudaStreamEndCapture(c->cap, &g) == cudaSuccess && g;
+  }
+  const long long captured = (long long)(launch_total() - n0);
+  note_launch(-captured);
+  if (ok && *exec) {  // same topology for every cache of this model: update in place
+    cudaGraphExecUpdateResultInfo info;
+    if (cudaGraphExecUpdate(*exec, g, &info) != cudaSuccess) {
+      cudaGetLastError();
+      cudaGraphExecDestroy(*exec);
+      *exec = nullptr;
+    }
+  }
+  if (ok && !*exec) ok = cudaGraphInstantiate(exec, g, 0) == cudaSuccess;
+  if (g) cudaGraphDestroy(g);
+  if (!ok) {
+    cudaGetLastError();
+    if (*exec) cudaGraphExecDestroy(*exec);
+    *exec = nullptr;
+    return false;
+  }
+  *kernels = captured;
+  return true;
+}
+
+int photon_decode_rec_chunks(photon_model* m, photon_cache* c, int32_t n, int32_t* d_out_tokens,
+                             void* stream) {
+  g_err.clear();
+  if (!m || !c || c->m != m) return fail(PHOTON_ERR_ARG, "model/cache mismatch");
+  if (n < 0 || (n > 0 && !d_out_tokens)) return fail(PHOTON_ERR_ARG, "bad chunk count or output");
+  if (n == 0) return PHOTON_OK;
+  if (c->steps + n > c->max_new) return fail(PHOTON_ERR_CAPACITY, "cache is full (%d steps)", c->max_new);
+  cudaStream_t s = (cudaStream_t)stream;
+  c->stream = s;
+  const int B = c->B, C = m->C;
+  const size_t pitch = (size_t)n * C * sizeof(int32_t), w = (size_t)C * sizeof(int32_t);
+  int t = 0;
+  // the first step of a cache runs eagerly (it configures every kernel)
+  auto one_step = [&](int k) -> int {
+    RET(photon_decode_step_ex(m, c, PHOTON_MODE_REC, c->tok_out, nullptr, nullptr, nullptr, stream));
+    CK(cudaMemcpy2DAsync(d_out_tokens + (size_t)k * C, pitch, c->tok_out, w, w, B,
+                         cudaMemcpyDeviceToDevice, s));
+    return PHOTON_OK;
+  };
+  if (c->steps == 0) {
+    RET(one_step(0));
+    t = 1;
+  }
+  bool pipe = pipeline_enabled() && graphs_enabled() && c->cap != nullptr && t < n;
+  if (pipe) RET(prepare_pipeline(m, c, s));
+  if (pipe && m->pg_owner != c) {
+    for (int p = 0; p < 2 && pipe; ++p)
+      pipe = capture_part(m, c, DEC_MAIN, p, &m->pg[0][p], &m->pg_kernels[0]) &&
+             capture_part(m, c, DEC_TOK, p, &m->pg[1][p], &m->pg_kernels[1]);
+    m->pg_owner = pipe ? c : nullptr;
+  }
+  if (!pipe) {
+    for (; t < n; ++t) RET(one_step(t));
+    return PHOTON_OK;
+  }
+  // main chain of chunk k on the caller's stream; token branch of chunk k on
+  // the token stream, overlapping the main chain of chunk k + 1
+  int last = 0;
+  for (; t < n; ++t) {
+    const int p = c->steps & 1;
+    CK(cudaStreamWaitEvent(s, c->ev_tok[p], 0));  // token branch of two chunks ago released A-hat[p]
+    CK(cudaGraphLaunch(m->pg[0][p], s));
+    note_launch(m->pg_kernels[0]);
+    CK(cudaEventRecord(c->ev_main[p], s));
+    CK(cudaStreamWaitEvent(c->tstream, c->ev_main[p], 0));
+    CK(cudaGraphLaunch(m->pg[1][p], c->tstream));
+    note_launch(m->pg_kernels[1]);
+    CK(cudaMemcpy2DAsync(d_out_tokens + (size_t)t * C, pitch, c->tok_out, w, w, B,
+                         cudaMemcpyDeviceToDevice, c->tstream));
+    CK(cudaEventRecord(c->ev_tok[p], c->tstream));
+    c->N += 1;
+    c->steps += 1;
+    c->graph_steps += 1;
+    c->has_a_hat = true;
+    c->ahat_latest = c->ahat_p[p];
+    last = p;
+  }
+  CK(cudaStreamWaitEvent(s, c->ev_tok[last], 0));  // everything joins the caller's stream
   return PHOTON_OK;
 }
 
@@ -1342,24 +1567,41 @@ int photon_free_cache(photon_cache* c) {
   if (!c) return fail(PHOTON_ERR_ARG, "cache is NULL");
   if (c->dependents) return fail(PHOTON_ERR_ARG, "%d caches still read this prefix", c->dependents);
   photon_model* m = c->m;
-  CK(cudaStreamSynchronize(c->stream));
   for (int k = 0; k < 2; ++k)
     if (m->graph_owner[k] == c) m->graph_owner[k] = nullptr;  // its buffers are going away
-  if (c->side) {
-    cudaStreamSynchronize(c->side);
-    cudaStreamDestroy(c->side);
+  if (m->pg_owner == c) m->pg_owner = nullptr;
+  // Stream-ordered release: the helper streams' pending work is joined into
+  // the cache's stream, the buffers go back to the pool on that stream, and
+  // streams and events are destroyed at once (the driver releases them when
+  // their work completes).  The next allocation on the same stream reuses the
+  // memory without waiting on the host.
+  cudaStream_t helpers[3] = {c->side, c->tstream, c->hi};
+  for (cudaStream_t h : helpers) {
+    if (!h) continue;
+    cudaEvent_t e = nullptr;
+    CK(cudaEventCreateWithFlags(&e, cudaEventDisableTiming));
+    CK(cudaEventRecord(e, h));
+    CK(cudaStreamWaitEvent(c->stream, e, 0));
+    cudaEventDestroy(e);
   }
+  for (cudaStream_t h : helpers)
+    if (h) cudaStreamDestroy(h);
   if (c->cap) cudaStreamDestroy(c->cap);  // only ever captured into, never run
-  if (c->hi) {
-    cudaStreamSynchronize(c->hi);
-    cudaStreamDestroy(c->hi);
+  for (int p = 0; p < 2; ++p) {
+    if (c->ev_main[p]) cudaEventDestroy(c->ev_main[p]);
+    if (c->ev_tok[p]) cudaEventDestroy(c->ev_tok[p]);
   }
   if (c->ev_fork) cudaEventDestroy(c->ev_fork);
   if (c->ev_join_hi) cudaEventDestroy(c->ev_join_hi);
   if (c->ev_join) cudaEventDestroy(c->ev_join);
   free_list(c->allocs, c->stream);
-  CK(cudaStreamSynchronize(c->stream));
-  if (c->prefix) c->prefix->dependents--;
+  // a cache built on a prefix may run on another stream than the prefix's
+  // eventual free: finish its work before the prefix can be released
+  if (c->prefix) {
+    CK(cudaStreamSynchronize(c->stream));
+    c->prefix->dependents--;
+  }
+  CK(cudaGetLastError());
   m->live_caches--;
   if (c->mode == PHOTON_MODE_HIER) m->hier_caches--;
   delete c;
@@ -1390,7 +1632,7 @@ int photon_cache_info(photon_cache* c, photon_cache_stats* out) {
   out->graph_steps = c->graph_steps;
   out->graph_kernels = (c->mode >= 0 && c->mode < 2 && c->m->graph_owner[c->mode] == c)
                            ? (int32_t)c->m->graph_kernels[c->mode]
-                           : 0;
+                           : c->m->pg_owner == c ? (int32_t)(c->m->pg_kernels[0] + c->m->pg_kernels[1]) : 0;
   return PHOTON_OK;
 }
 
@@ -1434,7 +1676,7 @@ int photon_export_state(photon_cache* c, int32_t which, int32_t layer, void* d_d
     case PHOTON_STATE_A:
       if (which == PHOTON_STATE_A_HAT ? !c->has_a_hat : !c->has_a)
         return fail(PHOTON_ERR_ARG, "no decode step has produced this state yet");
-      src = (const char*)(which == PHOTON_STATE_A_HAT ? c->a_hat : c->a);
+      src = (const char*)(which == PHOTON_STATE_A_HAT ? (c->ahat_latest ? c->ahat_latest : c->a_hat) : c->a);
       rows = 1;
       width = pitch = (size_t)c->B * m->C2 * m->d * es;
       break;

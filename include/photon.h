@@ -155,8 +155,26 @@ PHOTON_API int photon_decode_step_ex(photon_model* m, photon_cache* c, int32_t m
                           float* d_out_logits, const int32_t* d_force_tokens,
                           const void* d_force_a, void* stream);
 
+/* RecGen decode of n consecutive top-level chunks in one call (explainer,
+ * RecGen section): the same tokens as n calls of photon_decode_step_rec,
+ * written to d_out_tokens [B, n * C1 * C2] (device, row-major; chunk k in
+ * columns k*C .. k*C + C - 1).  Because a RecGen chunk's top-encoder input
+ * (Chunker_2 of A-hat) does not depend on its tokens, the token decoder of
+ * chunk k runs on an internal stream while the main chain (Converter_2,
+ * Decoder_2, Chunker_2, top-encoder step) of chunk k + 1 runs on `stream`;
+ * all work is joined into `stream` before the call returns (asynchronous, as
+ * the other decode calls).  Allocates its token-branch buffers on the first
+ * call (counted in the cache's bytes).  Errors: ERR_ARG, ERR_CAPACITY (more
+ * chunks than the cache has room for), ERR_OOM, ERR_CUDA. */
+PHOTON_API int photon_decode_rec_chunks(photon_model* m, photon_cache* c, int32_t n_chunks,
+                                        int32_t* d_out_tokens, void* stream);
+
 /* Frees a cache and its device buffers.  A prefix cache can only be freed
- * after every cache built on it (ERR_ARG otherwise).  Synchronising. */
+ * after every cache built on it (ERR_ARG otherwise).  Stream-ordered: the
+ * buffers return to the library's pool on the stream of the cache's last
+ * call, after all of its pending work, and the call returns without waiting
+ * (a cache built on a shared prefix waits for its own work).  The handle is
+ * invalid afterwards. */
 PHOTON_API int photon_free_cache(photon_cache* c);
 
 typedef struct photon_cache_stats {

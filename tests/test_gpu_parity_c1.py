@@ -191,3 +191,25 @@ def test_sequences_do_not_interact(model):
         c.free()
     assert torch.equal(outs[0][:, 0], outs[1][:, 0]) and torch.equal(outs[0][:, 2], outs[1][:, 2])
     assert not torch.equal(outs[0][:, 1], outs[1][:, 1])
+
+
+def test_c1_rec_chunks_equal_steps_and_oracle(model):
+    # the multi-chunk RecGen call reproduces the per-step tokens bit for bit
+    # (and so the oracle's free-running RecGen tokens)
+    toks = torch.from_numpy(prompt_tokens("c1")).cuda()
+    a = model.prefill(toks, hal.MODE_REC, max_new_chunks=STEPS)
+    c = model.prefill(toks, hal.MODE_REC, max_new_chunks=STEPS)
+    ref = torch.empty(1, STEPS * CFG.C, dtype=torch.int32, device="cuda")
+    step = torch.empty(1, CFG.C, dtype=torch.int32, device="cuda")  # the per-step API writes [B, C]
+    for k in range(STEPS):
+        a.decode_step(hal.MODE_REC, step)
+        ref[:, k * CFG.C:(k + 1) * CFG.C] = step
+    got = torch.empty_like(ref)
+    c.decode_rec_chunks(STEPS, got)
+    torch.cuda.synchronize()
+    assert torch.equal(got, ref)
+    orc = PhotonOracle(CFG, WEIGHT_SEED)
+    st = orc.prefill(prompt_tokens("c1")[0], "rec")
+    want = np.concatenate([orc.decode_step(st, "rec").tokens for _ in range(STEPS)])
+    np.testing.assert_array_equal(got.cpu().numpy()[0], want)
+    a.free(); c.free()

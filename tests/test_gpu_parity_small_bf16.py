@@ -102,3 +102,75 @@ def test_small_bf16_graph_replay_equals_eager():
         assert torch.equal(g.export_state("top_k", l), e.export_state("top_k", l))
     assert torch.equal(g.export_state("pending_o"), e.export_state("pending_o"))
     g.free(); e.free(); model.free()
+
+
+def test_small_bf16_rec_chunks_equal_steps():
+    # photon_decode_rec_chunks (token decoder of chunk k overlapped with the
+    # main chain of chunk k + 1) gives exactly the tokens and caches of
+    # per-step RecGen decoding, across two consecutive calls
+    model = hal.Model(SHAPE, 7)
+    toks = torch.from_numpy(np.random.default_rng(6).integers(0, SHAPE["vocab"], size=(B, T))
+                            .astype(np.int32)).cuda()
+    n = 5
+    a = model.prefill(toks, hal.MODE_REC, n)
+    ref = torch.empty(B, n * CFG.C, dtype=torch.int32, device="cuda")
+    step = torch.empty(B, CFG.C, dtype=torch.int32, device="cuda")  # the per-step API writes [B, C]
+    for k in range(n):
+        a.decode_step(hal.MODE_REC, step)
+        ref[:, k * CFG.C:(k + 1) * CFG.C] = step
+    first = torch.empty(B, 2 * CFG.C, dtype=torch.int32, device="cuda")
+    c2 = model.prefill(toks, hal.MODE_REC, n)
+    c2.decode_rec_chunks(2, first)
+    rest = torch.empty(B, 3 * CFG.C, dtype=torch.int32, device="cuda")
+    c2.decode_rec_chunks(3, rest)
+    torch.cuda.synchronize()
+    assert torch.equal(torch.cat([first, rest], dim=1), ref)
+    for l in range(CFG.Ltop):
+        assert torch.equal(c2.export_state("top_k", l), a.export_state("top_k", l))
+    assert torch.equal(c2.export_state("pending_o"), a.export_state("pending_o"))
+    assert torch.equal(c2.export_state("a_hat"), a.export_state("a_hat"))
+    info = c2.info()
+    assert (info["N"], info["steps"], info["device_error"]) == (a.info()["N"], n, 0)
+    assert info["graph_steps"] >= n - 1  # everything after the first step replayed graphs
+    a.free(); c2.free(); model.free()
+
+
+def test_small_bf16_stream_ordered_free():
+    # a cache is released without a host wait: a HierGen cache decoded and
+    # freed on one stream, then RecGen prefills on another stream (which drop
+    # the level-1 encoder weights the HierGen steps read and reuse the freed
+    # memory), give the tokens of the same work run with full synchronisation
+    model = hal.Model(SHAPE, 7)
+    toks = torch.from_numpy(np.random.default_rng(8).integers(0, SHAPE["vocab"], size=(B, T))
+                            .astype(np.int32)).cuda()
+    n = 4
+    ref = torch.empty(B, n * CFG.C, dtype=torch.int32, device="cuda")
+    step = torch.empty(B, CFG.C, dtype=torch.int32, device="cuda")
+    h = model.prefill(toks, hal.MODE_HIER, n)
+    for k in range(n):
+        h.step_hier(step)
+        ref[:, k * CFG.C:(k + 1) * CFG.C] = step
+    torch.cuda.synchronize()
+    h.free()
+    s1, s2 = torch.cuda.Stream(), torch.cuda.Stream()
+    got = torch.empty_like(ref)
+    steps = [torch.empty(B, CFG.C, dtype=torch.int32, device="cuda") for _ in range(n)]
+    for rep in range(3):
+        got.fill_(-1)
+        with torch.cuda.stream(s1):
+            h = model.prefill(toks, hal.MODE_HIER, n)
+            for k in range(n):
+                h.step_hier(steps[k])
+            h.free()  # returns at once; buffers go back on s1
+        with torch.cuda.stream(s2):
+            for _ in range(2):
+                r = model.prefill(toks, hal.MODE_REC, n)
+                r.decode_rec_chunks(n, torch.empty(B, n * CFG.C, dtype=torch.int32, device="cuda"))
+                r.free()
+        torch.cuda.synchronize()
+        for k in range(n):
+            got[:, k * CFG.C:(k + 1) * CFG.C] = steps[k]
+        assert torch.equal(got, ref), rep
+    info = model.info()
+    assert info["live_caches"] == 0 and info["encoder_resident"] == 0
+    model.free()
