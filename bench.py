@@ -517,17 +517,25 @@ def measure_attn_roofline(model, wl, dev, stream) -> dict:
     for l in range(L):                                    # warm-up
         hal.attn_decode(q, K[l], V[l], 1, n_mid - 1, o)
     torch.cuda.synchronize()
+    # replayed from a captured graph, as inside the decode step: back-to-back
+    # launches with no host gaps between them
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=torch.cuda.Stream()):
+        for l in range(L):
+            hal.attn_decode(q, K[l], V[l], 1, n_mid - 1, o)
+    graph.replay()
+    torch.cuda.synchronize()
     reps = 20
     a = torch.cuda.Event(enable_timing=True)
     b = torch.cuda.Event(enable_timing=True)
     a.record(stream)
     torch.cuda.nvtx.range_push("roofline_attn")
     for r in range(reps):
-        for l in range(L):
-            hal.attn_decode(q, K[l], V[l], 1, n_mid - 1, o)
+        graph.replay()
     torch.cuda.nvtx.range_pop()
     b.record(stream)
     torch.cuda.synchronize()
+    del graph
     ms = a.elapsed_time(b) / (reps * L)
     es = 2 if dt == torch.bfloat16 else 4
     algo = 2 * B * H * n_mid * dh * es + 2 * B * H * dh * es   # K,V rows read + q read + o write

@@ -295,6 +295,244 @@ __global__ void k_attn_combine(AttnArgs a, int splits, const float* __restrict__
   st_f(reinterpret_cast<T*>(a.O) + row * a.o_ld + h * DH + dd, L > 0.f ? acc / L : 0.f);
 }
 
+// Streaming decode attention for long caches: one new query per (group,
+// head), bf16, many pairs (the top-encoder decode step of a long context).
+// A pair's key rows [key, DH] are one contiguous run of its cache, so a
+// single producer thread streams each pair as tiles of kStreamTK rows with
+// bulk copies (K tile, V tile, and the query row with the pair's first
+// tile) into a kStreamStages-deep ring guarded by mbarriers, while
+// kStreamWarps consumer warps reduce the tiles: lanes are grouped 8 per key
+// row (16 bytes each), every key group keeps an online softmax, and the
+// warps merge through shared memory at the pair's end.  A CTA owns an equal
+// run of consecutive pairs and the copies never pause between pairs.  On
+// B200 this beats the chunked kernel only from several hundred keys on (at
+// 272 keys its per-tile barrier round trips cost more than the chunked
+// kernel's per-lane cp.async rings), so it takes caches of at least
+// kStreamMinKeys keys.
+#ifndef PHOTON_STREAM_WARPS
+#define PHOTON_STREAM_WARPS 8
+#endif
+#ifndef PHOTON_STREAM_STAGES
+#define PHOTON_STREAM_STAGES 3
+#endif
+#ifndef PHOTON_STREAM_TK
+#define PHOTON_STREAM_TK 128
+#endif
+constexpr int kStreamWarps = PHOTON_STREAM_WARPS;    // consumer warps (one more warp produces)
+constexpr int kStreamStages = PHOTON_STREAM_STAGES;  // ring depth
+constexpr int kStreamTK = PHOTON_STREAM_TK;          // key rows per tile
+
+template <int DH>
+struct StreamCfg {
+  static constexpr uint32_t kRow = DH * 2;                  // bytes per bf16 row
+  static constexpr uint32_t kTile = kStreamTK * kRow;       // one K (or V) tile
+  static constexpr uint32_t kStage = 2 * kTile + kRow;      // K, V, query row
+  static constexpr uint32_t kRing = kStreamStages * kStage;
+};
+
+template <int DH>
+__global__ void __launch_bounds__(32 * (kStreamWarps + 1))
+    k_attn_decode_stream(AttnArgs a, int pairs_per_cta, int* err) {
+  using Cfg = StreamCfg<DH>;
+  constexpr int W = kStreamWarps, S = kStreamStages, TK = kStreamTK;
+  constexpr int VEC = 8;            // bf16 per 16-byte slice
+  constexpr int TPK = DH / VEC;     // lanes per key row
+  constexpr int GPW = 32 / TPK;     // key rows per warp-wide access
+  constexpr int KPW = TK / W;       // rows of a tile per warp
+  constexpr int U = KPW / GPW;      // rows per key group per tile
+  static_assert(32 % TPK == 0 && KPW % GPW == 0 && U >= 1, "tile must split evenly");
+  extern __shared__ __align__(128) uint8_t stream_ring[];
+  __shared__ __align__(8) uint64_t bars[2 * S];
+  __shared__ float sm_m[2][W], sm_l[2][W];
+  __shared__ float sm_acc[2][W][DH];
+  __shared__ int abort_flag;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  auto full_bar = [&](int st) { return ptx::smem_u32(bars + st); };
+  auto empty_bar = [&](int st) { return ptx::smem_u32(bars + S + st); };
+  auto kt = [&](int st) { return stream_ring + st * Cfg::kStage; };
+  auto vt = [&](int st) { return stream_ring + st * Cfg::kStage + Cfg::kTile; };
+  auto qt = [&](int st) { return stream_ring + st * Cfg::kStage + 2 * Cfg::kTile; };
+  if (threadIdx.x == 0) {
+    for (int st = 0; st < S; ++st) {
+      ptx::mbar_init(full_bar(st), 1);
+      ptx::mbar_init(empty_bar(st), W);  // one arrival per consumer warp
+    }
+    abort_flag = 0;
+    ptx::fence_barrier_init();
+  }
+  __syncthreads();
+  pdl_wait();  // every role touches global memory only after this point
+  pdl_trigger();
+
+  const long long pairs = (long long)a.G * a.H;
+  const long long pair0 = (long long)blockIdx.x * pairs_per_cta;
+  const int npairs = (int)max(0LL, min((long long)pairs_per_cta, pairs - pair0));
+  // visible keys (one query at position p0): [0, p0], prefix rows first
+  const int p0 = a.p0_dev ? (*a.p0_dev + a.p0) : a.p0;
+  const int n = min(p0 + 1, a.n_pre + a.cap);
+  const int npre = min(a.n_pre, n);
+  const int tpre = (npre + TK - 1) / TK, tpp = tpre + (n - npre + TK - 1) / TK;  // tiles per pair
+  const int total = npairs * tpp;
+  // tile j of a pair: first key and row count
+  auto tile_rows = [&](int j, int& k0) {
+    if (j < tpre) {
+      k0 = j * TK;
+      return min(TK, npre - k0);
+    }
+    k0 = npre + (j - tpre) * TK;
+    return min(TK, n - k0);
+  };
+
+  if (warp == W) {  // ---- producer
+    if (lane == 0) {
+      int t = 0;
+      for (; t < total; ++t) {
+        const int st = t % S;
+        const uint32_t ph = (uint32_t)(t / S) & 1u;
+        if (t >= S && !ptx::mbar_wait(empty_bar(st), ph ^ 1u, &abort_flag)) {
+          report_error(err, DEV_WAIT_TIMEOUT_PRODUCER);
+          abort_flag = 1;
+          break;
+        }
+        const long long pair = pair0 + t / tpp;
+        const int j = t % tpp;
+        const int g = (int)(pair / a.H), h = (int)(pair % a.H);
+        int k0;
+        const int rows = tile_rows(j, k0);
+        const uint32_t bytes = (uint32_t)rows * Cfg::kRow;
+        const bool pre = k0 < npre;
+        const long long row0 = pre ? ((long long)h * a.cap_pre + k0)
+                                   : (((long long)g * a.H + h) * a.cap + (k0 - a.n_pre));
+        const bf16* ks = reinterpret_cast<const bf16*>(pre ? a.Kp : a.K) + row0 * DH;
+        const bf16* vs = reinterpret_cast<const bf16*>(pre ? a.Vp : a.V) + row0 * DH;
+        ptx::mbar_arrive_expect_tx(full_bar(st), 2 * bytes + (j == 0 ? Cfg::kRow : 0u));
+        ptx::bulk_load(ptx::smem_u32(kt(st)), ks, bytes, full_bar(st));
+        ptx::bulk_load(ptx::smem_u32(vt(st)), vs, bytes, full_bar(st));
+        if (j == 0)
+          ptx::bulk_load(ptx::smem_u32(qt(st)),
+                         reinterpret_cast<const bf16*>(a.Q) + (long long)g * a.q_ld + h * DH,
+                         Cfg::kRow, full_bar(st));
+      }
+      if (t < total) {
+        // gave up: let the copies already issued land before the CTA exits
+        for (int u = max(0, t - S); u < t; ++u)
+          ptx::mbar_wait(full_bar(u % S), (uint32_t)(u / S) & 1u, nullptr);
+      }
+    }
+    return;
+  }
+
+  // ---- consumers
+  const int kg = lane / TPK, sl = lane % TPK;
+  float qv[VEC], acc[VEC], m = -INFINITY, l = 0.f;
+  for (int t = 0; t < total; ++t) {
+    const int st = t % S;
+    const uint32_t ph = (uint32_t)(t / S) & 1u;
+    const int j = t % tpp;
+    if (!ptx::mbar_wait(full_bar(st), ph, &abort_flag)) {
+      if (lane == 0) report_error(err, DEV_WAIT_TIMEOUT_EPILOGUE);
+      abort_flag = 1;
+      return;
+    }
+    if (j == 0) {
+      const uint4 raw = *reinterpret_cast<const uint4*>(qt(st) + sl * 16);
+      const bf16* qp = reinterpret_cast<const bf16*>(&raw);
+#pragma unroll
+      for (int e = 0; e < VEC; ++e) {
+        qv[e] = __bfloat162float(qp[e]) * a.scale;
+        acc[e] = 0.f;
+      }
+      m = -INFINITY;
+      l = 0.f;
+    }
+    int k0;
+    const int rows = tile_rows(j, k0);
+    float sc[U];
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int r = warp * KPW + u * GPW + kg;  // row within the tile
+      const uint4 kraw = *reinterpret_cast<const uint4*>(kt(st) + r * Cfg::kRow + sl * 16);
+      const bf16* kp = reinterpret_cast<const bf16*>(&kraw);
+      float d = 0.f;
+#pragma unroll
+      for (int e = 0; e < VEC; ++e) d = fmaf(qv[e], __bfloat162float(kp[e]), d);
+#pragma unroll
+      for (int o = TPK / 2; o > 0; o >>= 1) d += __shfl_xor_sync(0xffffffffu, d, o);
+      sc[u] = r < rows ? d : -INFINITY;
+    }
+    float mx = sc[0];
+#pragma unroll
+    for (int u = 1; u < U; ++u) mx = fmaxf(mx, sc[u]);
+    if (mx != -INFINITY) {
+      const float mn = fmaxf(m, mx);
+      const float c = __expf(m - mn);  // 0 while m is -inf
+      float pe[U], ps = 0.f;
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        pe[u] = __expf(sc[u] - mn);
+        ps += pe[u];
+      }
+      l = l * c + ps;
+#pragma unroll
+      for (int e = 0; e < VEC; ++e) acc[e] *= c;
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        if (sc[u] == -INFINITY) continue;
+        const int r = warp * KPW + u * GPW + kg;
+        const uint4 vraw = *reinterpret_cast<const uint4*>(vt(st) + r * Cfg::kRow + sl * 16);
+        const bf16* vp = reinterpret_cast<const bf16*>(&vraw);
+#pragma unroll
+        for (int e = 0; e < VEC; ++e) acc[e] = fmaf(pe[u], __bfloat162float(vp[e]), acc[e]);
+      }
+      m = mn;
+    }
+    __syncwarp();
+    if (lane == 0) ptx::mbar_arrive(empty_bar(st));  // this warp is done with stage st
+
+    if (j == tpp - 1) {
+      // pair complete: merge the key groups of this warp, then the warps
+      const int buf = (t / tpp) & 1;
+      float M = m;
+#pragma unroll
+      for (int o = TPK; o < 32; o <<= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+      const float c = (M == -INFINITY) ? 0.f : __expf(m - M);
+      float L = l * c;
+#pragma unroll
+      for (int o = TPK; o < 32; o <<= 1) L += __shfl_xor_sync(0xffffffffu, L, o);
+#pragma unroll
+      for (int e = 0; e < VEC; ++e) {
+        float v = acc[e] * c;
+#pragma unroll
+        for (int o = TPK; o < 32; o <<= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+        if (lane < TPK) sm_acc[buf][warp][sl * VEC + e] = v;
+      }
+      if (lane == 0) {
+        sm_m[buf][warp] = M;
+        sm_l[buf][warp] = L;
+      }
+      asm volatile("bar.sync 1, %0;" ::"n"(32 * W) : "memory");  // consumer warps only
+      const int dd = threadIdx.x;
+      if (dd < DH) {
+        float Mx = -INFINITY;
+#pragma unroll
+        for (int w = 0; w < W; ++w) Mx = fmaxf(Mx, sm_m[buf][w]);
+        float Ls = 0.f, v = 0.f;
+#pragma unroll
+        for (int w = 0; w < W; ++w) {
+          const float cw = (sm_m[buf][w] == -INFINITY) ? 0.f : __expf(sm_m[buf][w] - Mx);
+          Ls += cw * sm_l[buf][w];
+          v += cw * sm_acc[buf][w][dd];
+        }
+        const long long pair = pair0 + t / tpp;
+        const int g = (int)(pair / a.H), h = (int)(pair % a.H);
+        st_f(reinterpret_cast<bf16*>(a.O) + (long long)g * a.o_ld + h * DH + dd,
+             Ls > 0.f ? v / Ls : 0.f);
+      }
+    }
+  }
+}
+
 struct DecPlan {
   int chunk, splits, warps;
 };
@@ -315,6 +553,55 @@ DecPlan dec_plan(const AttnArgs& a) {
   const int chunk = (n + splits - 1) / splits;
   splits = (n + chunk - 1) / chunk;
   return {chunk, splits, w};
+}
+
+// Streamed path: one bf16 query per pair, at least one pair per SM (fewer
+// pairs leave SMs idle; the chunked path splits their keys instead), a long
+// cache (planned key count >= PHOTON_ATTN_STREAM_MIN_KEYS, default 768; 0
+// turns the path off), and 16-byte aligned rows for the bulk copies.
+static int sm_count() {
+  static int sms = 0;
+  if (!sms) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (sms <= 0) sms = 1;
+  }
+  return sms;
+}
+static int stream_min_keys() {
+  static const int v = [] {
+    const char* e = getenv("PHOTON_ATTN_STREAM_MIN_KEYS");
+    return e ? atoi(e) : 768;
+  }();
+  return v;
+}
+bool stream_attn_ok(int dt, const AttnArgs& a) {
+  auto al16 = [](const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; };
+  const int n = a.n_plan > 0 ? a.n_plan : a.p0 + a.q_len;
+  return stream_min_keys() > 0 && n >= stream_min_keys() && dt == DT_BF16 && (a.dh == 64 || a.dh == 32) &&
+         a.q_len == 1 &&
+         (long long)a.G * a.H >= sm_count() && a.q_ld % 8 == 0 && al16(a.Q) && al16(a.K) &&
+         al16(a.V) && (a.n_pre == 0 || (al16(a.Kp) && al16(a.Vp)));
+}
+
+template <int DH>
+void run_stream(const AttnArgs& a, int* err, cudaStream_t s) {
+  constexpr int kSmem = (int)StreamCfg<DH>::kRing;
+  static int per_sm = 0;
+  if (!per_sm) {
+    cudaFuncSetAttribute(k_attn_decode_stream<DH>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
+    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k_attn_decode_stream<DH>,
+                                                  32 * (kStreamWarps + 1), kSmem);
+    if (per_sm < 1) per_sm = 1;
+  }
+  // every CTA gets the same number of pairs (the last one possibly fewer)
+  const long long pairs = (long long)a.G * a.H;
+  const long long resident = (long long)sm_count() * per_sm;
+  const long long per = (pairs + resident - 1) / resident;
+  const long long ctas = (pairs + per - 1) / per;
+  launch_kernel(k_attn_decode_stream<DH>, dim3((unsigned)ctas), dim3(32 * (kStreamWarps + 1)),
+                (size_t)kSmem, s, a, (int)per, err);
 }
 
 template <typename T, int DH, int QMAX, int W>
@@ -652,9 +939,9 @@ static bool tc_attn_disabled() {
 
 bool local_attn_ok(const AttnArgs& a);  // short local caches take k_attn_local (no scratch)
 
+
 size_t attn_decode_workspace_bytes(int dt, const AttnArgs& a) {
-  (void)dt;
-  if (a.G <= 0 || a.q_len <= 0 || local_attn_ok(a)) return 0;
+  if (a.G <= 0 || a.q_len <= 0 || local_attn_ok(a) || stream_attn_ok(dt, a)) return 0;
   const DecPlan p = dec_plan(a);
   if (p.splits <= 1) return 0;
   return (size_t)a.G * a.q_len * a.H * p.splits * (a.dh + 2) * sizeof(float);
@@ -760,6 +1047,13 @@ bool launch_attn_decode(int dt, const AttnArgs& a, float* part, size_t part_byte
       run_local<float, 64>(a, s);
     else
       run_local<bf16, 32>(a, s);
+    return true;
+  }
+  if (stream_attn_ok(dt, a)) {
+    if (a.dh == 64)
+      run_stream<64>(a, err, s);
+    else
+      run_stream<32>(a, err, s);
     return true;
   }
   const DecPlan p = dec_plan(a);

@@ -103,6 +103,18 @@ def test_attn_decode_bf16(G, H, cap, q_len, p0):
     np.testing.assert_allclose(got, ref, rtol=1e-2, atol=1e-2 * np.abs(ref).max())
 
 
+# one query over a long cache (>= 768 keys) with at least one (group, head)
+# pair per SM takes the streamed kernel (bulk copies of 128-row tiles):
+# exact tiles, a tile plus one row, ragged tails, both head sizes
+@pytest.mark.parametrize("G,H,dh,cap,p0", [
+    (10, 16, 64, 1024, 767), (10, 16, 64, 769, 768), (12, 16, 64, 800, 799),
+    (3, 64, 64, 1100, 1029), (10, 16, 32, 900, 899), (160, 1, 32, 800, 790),
+])
+def test_attn_decode_streamed_bf16(G, H, dh, cap, p0):
+    got, ref = _attn_case(torch.bfloat16, G, H, dh, cap, 1, p0, 30)
+    np.testing.assert_allclose(got, ref, rtol=1e-2, atol=1e-2 * np.abs(ref).max())
+
+
 @pytest.mark.parametrize("G,H,cap,q_len,p0", [(1, 2, 80, 1, 70), (1, 2, 70, 4, 60), (3, 2, 8, 1, 3)])
 def test_attn_decode_fp32(G, H, cap, q_len, p0):
     got, ref = _attn_case(torch.float32, G, H, 32, cap, q_len, p0, 20)
