@@ -541,7 +541,8 @@ def measure_attn_roofline(model, wl, dev, stream) -> dict:
     algo = 2 * B * H * n_mid * dh * es + 2 * B * H * dh * es   # K,V rows read + q read + o write
     peak, src = _peak_gbs()
     achieved = algo / (ms / 1e3) / 1e9
-    return {"kernel": "k_attn_decode (top-encoder decode attention, one CTA per (sequence, head))",
+    return {"kernel": "top-encoder decode attention (k_attn_decode below 768 keys; "
+                      "k_attn_decode_stream from 768 keys with at least one (sequence, head) per SM)",
             "bound": "hbm", "achieved": round(achieved, 1), "peak": peak,
             "unit": "GB/s", "frac": round(achieved / peak, 4),
             "peak_source": f"{src} (STREAM-style copy)", "traffic": None,
