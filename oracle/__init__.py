@@ -13,6 +13,8 @@ Contents:
                 from its definition (SplitMix64 + Irwin-Hall), fp64.
   photon.py  -- the model in plain fp64 NumPy, one sequence at a time,
                 following the PHOTON pages step by step.
+  sampling.py -- temperature sampling by the Gumbel-max rule with a
+                counter-based generator (SplitMix64 + MurmurHash3 fmix32).
 
 Every oracle function is pinned by CPU tests (tests/test_oracle_*.py) to
 facts that do not come from the oracle itself: published SplitMix64 test

@@ -47,6 +47,7 @@ from dataclasses import dataclass, field
 import numpy as np
 from scipy.special import erf
 
+from .sampling import sample as draw
 from .weights import make_weights
 
 
@@ -221,16 +222,17 @@ class SeqState:
     N1: int                            # level-1 entries (0 once discarded)
     tokens: list[int] = field(default_factory=list)   # prompt + generated ids
     top_inputs: list[np.ndarray] = field(default_factory=list)  # chunker-2 outputs fed to the top
+    steps: int = 0                     # decode calls since the prefill (chunks generated)
 
 
 @dataclass
 class StepResult:
-    tokens: np.ndarray      # [C] int: the oracle's own greedy choices (j*C1 + i order)
+    tokens: np.ndarray      # [C] int: the oracle's own choices (j*C1 + i order)
     used: np.ndarray        # [C] int: tokens fed back (forced or own)
     logits: np.ndarray      # [C, V] fp64
     a_hat: np.ndarray       # [C2, d] Decoder_2 reconstruction
     a: np.ndarray | None    # [C2, d] level-1 encoder states of the chunk (HierGen only)
-    near_tie: np.ndarray    # [C] bool: top-2 gap < 1e-5 * logit range (R12)
+    near_tie: np.ndarray    # [C] bool: top-2 gap < 1e-5 * range of the compared values (R12)
 
 
 class PhotonOracle:
@@ -322,13 +324,15 @@ class PhotonOracle:
         h, _ = stack(cfg, w, "dec1", cfg.Ld1, x, np.arange(x.shape[0]), None)
         return h[-1] @ w["head"].T
 
-    def emit_tokens(self, a_hat: np.ndarray, force: np.ndarray | None):
+    def emit_tokens(self, a_hat: np.ndarray, force: np.ndarray | None, sample=None, first_t: int = 0):
         """Write the C tokens of the next top-level chunk from A-hat.
 
         Sub-chunk j uses Converter_1(A-hat_j) as its conditioning; its tokens
-        depend on nothing else (R4).  Greedy argmax, lowest index on ties (R12).
-        `force` (teacher forcing, entries < 0 = not forced) replaces the token
-        fed back, not the recorded argmax."""
+        depend on nothing else (R4).  Greedy argmax, lowest index on ties (R12);
+        with `sample` = (temperature, seed, b) the token is drawn from
+        softmax(logits / temperature) instead (oracle/sampling.py), token
+        index first_t + j*C1 + i.  `force` (teacher forcing, entries < 0 = not
+        forced) replaces the token fed back, not the recorded choice."""
         cfg = self.cfg
         C1, C2, V = cfg.C1, cfg.C2, cfg.vocab
         own = np.zeros(C1 * C2, dtype=np.int64)
@@ -342,8 +346,12 @@ class PhotonOracle:
                 t = j * C1 + i
                 lg = self.token_decoder_logits(cond, prev)
                 logits[t] = lg
-                own[t] = int(np.argmax(lg))
-                srt = np.sort(lg)
+                if sample is None:
+                    own[t], z = int(np.argmax(lg)), lg
+                else:
+                    temperature, seed, b = sample
+                    own[t], z = draw(lg, temperature, seed, b, first_t + t)
+                srt = np.sort(z)
                 tie[t] = (srt[-1] - srt[-2]) < 1e-5 * (srt[-1] - srt[0])
                 used[t] = own[t] if force is None or force[t] < 0 else int(force[t])
                 prev.append(int(used[t]))
@@ -358,7 +366,7 @@ class PhotonOracle:
         st.top_inputs.append(u.copy())
 
     def decode_step(self, st: SeqState, mode: str, force_tokens=None,
-                    force_a=None) -> StepResult:
+                    force_a=None, sample=None) -> StepResult:
         """One top-level chunk of decoding (R7).
 
         HierGen ([hiergen]): write the chunk's tokens, re-encode them
@@ -366,12 +374,13 @@ class PhotonOracle:
         top step.  RecGen ([recgen]): write the tokens, then feed
         Chunker_2(A-hat) to the top encoder; no level-1 work at all.
         `force_a` (test hook for [thm-a6]) replaces A-hat as the RecGen top
-        input."""
+        input.  `sample` = (temperature, seed, b): temperature sampling for
+        the sequence in batch row b (oracle/sampling.py); None = greedy."""
         cfg = self.cfg
         if mode == "hier" and st.l1 is None:
             raise ValueError("HierGen needs the level-1 cache (discarded by a RecGen prefill)")
         a_hat = self.decode_chunk2(st.o)
-        own, used, logits, tie = self.emit_tokens(a_hat, force_tokens)
+        own, used, logits, tie = self.emit_tokens(a_hat, force_tokens, sample, st.steps * cfg.C)
         a = None
         if mode == "hier":
             a, st.l1 = self.encode_level1(used, st.N1, st.l1)
@@ -382,6 +391,7 @@ class PhotonOracle:
         u = chunker(top_in, self.w["chunker2"], cfg.C2)[0]
         self.top_step(st, u)
         st.tokens.extend(int(t) for t in used)
+        st.steps += 1
         return StepResult(tokens=own, used=used, logits=logits, a_hat=a_hat, a=a, near_tie=tie)
 
     # -- full recomputation (used to pin the incremental paths) ---------------

@@ -1,0 +1,87 @@
+"""Temperature sampling of the token decoder's output, fp64 reference.
+
+TEST INFRASTRUCTURE ONLY -- see oracle/__init__.py for who may use it.
+
+The PHOTON explainer's quality section describes closing the single-query
+quality gap by running several slightly varied queries and combining them
+(majority vote or best-of-N).  That needs a stochastic decoder; the pages do
+not say which.  Reading taken here: the next token is drawn from
+softmax(logits / T) with temperature T > 0 (T = 0 keeps the greedy rule).
+
+The draw uses the Gumbel-max rule: with G_v independent standard Gumbel
+variables, argmax_v (l_v / T + G_v) is distributed as softmax(l / T).  The
+Gumbel variables come from a counter-based generator so that a draw depends
+only on (seed, sequence, token position, vocabulary id):
+
+  row key   K   = mix64(mix64(seed + gamma * (b + 1)) + gamma * (t + 1))
+                  (mix64 = the SplitMix64 output function, gamma its
+                  Weyl increment 0x9E3779B97F4A7C15), folded to 32 bits as
+                  k32 = high 32 bits XOR low 32 bits;
+  element   h   = fmix32(k32 + 0x9E3779B9 * (v + 1))   (mod 2^32), fmix32 =
+                  the 32-bit finaliser of MurmurHash3 (xor-shift 16,
+                  multiply 0x85EBCA6B, xor-shift 13, multiply 0xC2B2AE35,
+                  xor-shift 16);
+  uniform   u   = (floor(h / 256) + 1/2) / 2^24, in (0, 1);
+  Gumbel    G   = -ln(-ln u), with -ln u evaluated as -log1p(-(1 - u)) so
+                  that u near 1 keeps its precision.
+
+b is the sequence's row in the batch, t the token's index among the tokens
+the cache has generated (chunk * C1*C2 + sub-chunk * C1 + position), v the
+vocabulary id.  Ties of the perturbed values go to the lowest id, as for
+greedy decoding.
+"""
+from __future__ import annotations
+
+import numpy as np
+
+from .weights import GAMMA, mix64
+
+_F1 = np.uint32(0x85EBCA6B)
+_F2 = np.uint32(0xC2B2AE35)
+_WEYL32 = np.uint32(0x9E3779B9)
+
+
+def fmix32(h: np.ndarray) -> np.ndarray:
+    """MurmurHash3's 32-bit finaliser, elementwise on uint32."""
+    h = np.asarray(h, dtype=np.uint32)
+    with np.errstate(over="ignore"):
+        h = h ^ (h >> np.uint32(16))
+        h = h * _F1
+        h = h ^ (h >> np.uint32(13))
+        h = h * _F2
+        h = h ^ (h >> np.uint32(16))
+    return h
+
+
+def row_key(seed: int, b: int, t: int) -> np.uint32:
+    """32-bit key of one (sequence, token position) draw."""
+    with np.errstate(over="ignore"):
+        k = mix64(np.uint64(seed) + GAMMA * np.uint64(b + 1))
+        k = mix64(k + GAMMA * np.uint64(t + 1))
+    k = int(k)
+    return np.uint32((k >> 32) ^ (k & 0xFFFFFFFF))
+
+
+def uniforms(key: np.uint32, V: int) -> np.ndarray:
+    """u_v for v = 0..V-1, exact binary fractions in (0, 1) (fp64)."""
+    v = np.arange(1, V + 1, dtype=np.uint32)
+    with np.errstate(over="ignore"):
+        h = fmix32(np.uint32(key) + _WEYL32 * v)
+    return ((h >> np.uint32(8)).astype(np.float64) + 0.5) / float(1 << 24)
+
+
+def gumbel(key: np.uint32, V: int) -> np.ndarray:
+    """Standard Gumbel variables G_v = -ln(-ln u_v), v = 0..V-1 (fp64)."""
+    u = uniforms(key, V)
+    e = -np.log1p(-(1.0 - u))   # -ln u, exact 1 - u
+    return -np.log(e)
+
+
+def sample(logits: np.ndarray, temperature: float, seed: int, b: int, t: int):
+    """Token drawn from softmax(logits / T) by the Gumbel-max rule.
+
+    Returns (token, perturbed values); T must be > 0."""
+    if not temperature > 0:
+        raise ValueError("temperature must be positive")
+    z = np.asarray(logits, dtype=np.float64) / temperature + gumbel(row_key(seed, b, t), logits.shape[-1])
+    return int(np.argmax(z)), z

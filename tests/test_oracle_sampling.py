@@ -1,0 +1,93 @@
+"""Pins of the oracle's temperature sampler (oracle/sampling.py).
+
+The sampler's claim is distributional: the Gumbel-max rule over its
+counter-based noise draws token v with probability softmax(l / T)_v.  These
+tests check that claim and the pieces it rests on against facts that do not
+come from the sampler itself: the standard Gumbel law's mean (the
+Euler-Mascheroni constant) and variance (pi^2 / 6), a multinomial
+goodness-of-fit against softmax probabilities computed independently, the
+greedy limit T -> 0, and exact properties of the hash (a bijection of 32-bit
+words, fixed point 0, uniforms on the 2^-24 grid's odd midpoints).
+"""
+import math
+
+import numpy as np
+import pytest
+
+from oracle import Config, PhotonOracle
+from oracle import sampling as S
+
+
+def test_fmix32_is_a_bijection_with_fixed_point_zero():
+    # every step (xor-shift, odd multiply) is invertible on 32-bit words
+    x = np.arange(1 << 16, dtype=np.uint32) * np.uint32(65537)
+    assert np.unique(S.fmix32(x)).size == x.size
+    assert int(S.fmix32(np.uint32(0))) == 0
+
+
+def test_uniforms_are_odd_midpoints_of_the_2p24_grid():
+    u = S.uniforms(S.row_key(5, 1, 2), 50000)
+    assert np.all((u > 0) & (u < 1))
+    k = u * float(1 << 25)
+    assert np.all(k == np.round(k)) and np.all(k.astype(np.int64) % 2 == 1)
+    assert abs(u.mean() - 0.5) < 4 * math.sqrt(1 / 12 / u.size)
+
+
+def test_gumbel_moments():
+    g = np.concatenate([S.gumbel(S.row_key(11, b, t), 4096) for b in range(4) for t in range(16)])
+    n = g.size
+    euler_gamma = 0.5772156649015329
+    assert abs(g.mean() - euler_gamma) < 5 * math.sqrt(math.pi ** 2 / 6 / n)
+    assert abs(g.var() - math.pi ** 2 / 6) < 0.03
+
+
+def test_different_draws_are_uncorrelated():
+    a = S.gumbel(S.row_key(1, 0, 0), 20000)
+    b = S.gumbel(S.row_key(1, 0, 1), 20000)
+    c = S.gumbel(S.row_key(2, 0, 0), 20000)
+    d = S.gumbel(S.row_key(1, 1, 0), 20000)
+    for x in (b, c, d):
+        assert abs(np.corrcoef(a, x)[0, 1]) < 0.03
+    assert np.array_equal(a, S.gumbel(S.row_key(1, 0, 0), 20000))  # a draw is a pure function of its key
+
+
+@pytest.mark.parametrize("T", [0.5, 1.0, 2.0])
+def test_gumbel_max_draws_follow_softmax(T):
+    logits = np.array([1.3, -0.2, 0.7, 2.1, 0.0, -1.5])
+    n = 30000
+    counts = np.zeros(logits.size)
+    for t in range(n):
+        tok, _ = S.sample(logits, T, 42, 3, t)
+        counts[tok] += 1
+    z = logits / T
+    p = np.exp(z - z.max())
+    p /= p.sum()
+    chi2 = float(((counts - n * p) ** 2 / (n * p)).sum())
+    # 5 degrees of freedom: P(chi2 > 25.7) ~ 1e-4
+    assert chi2 < 25.7, (chi2, counts / n, p)
+
+
+def test_small_temperature_is_greedy():
+    rng = np.random.default_rng(0)
+    for t in range(200):
+        lg = rng.normal(size=300)
+        assert S.sample(lg, 1e-6, 9, 0, t)[0] == int(np.argmax(lg))
+
+
+def test_sampled_decode_step_reduces_to_greedy_and_is_reproducible():
+    cfg = Config.from_dict(dict(vocab=256, d_model=64, n_heads=2, head_dim=32, C1=4, C2=4, L1=1, Ltop=1,
+                                Ld1=1, Ld2=1, mlp_mult=4, dtype="fp32", init_std=0.02,
+                                rope_theta=10000.0, norm_eps=1e-6))
+    orc = PhotonOracle(cfg, 1)
+    toks = np.random.default_rng(1).integers(0, 256, size=32)
+    greedy, cold, hot1, hot2 = (orc.prefill(toks, "rec") for _ in range(4))
+    for _ in range(2):
+        g = orc.decode_step(greedy, "rec")
+        c = orc.decode_step(cold, "rec", sample=(1e-7, 5, 0))
+        h1 = orc.decode_step(hot1, "rec", sample=(1.0, 5, 0))
+        h2 = orc.decode_step(hot2, "rec", sample=(1.0, 5, 0))
+        keep = ~g.near_tie
+        assert np.array_equal(c.tokens[keep], g.tokens[keep])
+        assert np.array_equal(h1.tokens, h2.tokens)
+    # at T = 1 over a 256-way, nearly flat distribution the draws leave the greedy path
+    assert hot1.tokens != greedy.tokens
