@@ -30,7 +30,7 @@ _ERRORS = {-1: "PHOTON_ERR_ARG", -2: "PHOTON_ERR_OOM", -3: "PHOTON_ERR_CUDA",
 EXPORTED = ("photon_init_weights", "photon_free_model", "photon_prefill",
             "photon_decode_step_hier", "photon_decode_step_rec", "photon_decode_step_ex",
             "photon_decode_rec_chunks",
-            "photon_free_cache", "photon_cache_info", "photon_model_info",
+            "photon_free_cache", "photon_cache_set_sampling", "photon_cache_info", "photon_model_info",
             "photon_export_weight", "photon_export_state", "photon_gemm", "photon_gemm_rmsnorm",
             "photon_attn_decode", "photon_attn_decode_noalloc", "photon_launch_count",
             "photon_last_error")
@@ -89,6 +89,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "photon_decode_step_ex": [P, P, I32, P, P, P, P, P],
         "photon_decode_rec_chunks": [P, P, I32, P, P],
         "photon_free_cache": [P],
+        "photon_cache_set_sampling": [P, ctypes.c_float, U64],
         "photon_cache_info": [P, ctypes.POINTER(photon_cache_stats)],
         "photon_model_info": [P, ctypes.POINTER(photon_model_stats)],
         "photon_export_weight": [P, I32, P, SZ, ctypes.POINTER(SZ), P],
@@ -223,6 +224,11 @@ class Cache:
         (each chunk's token decoder overlapped with the next chunk's main chain)."""
         _check(load_library().photon_decode_rec_chunks(self.model._h, self._h, n_chunks,
                                                        _ptr(out_tokens), _stream(stream)))
+
+    def set_sampling(self, temperature: float, seed: int = 0) -> None:
+        """Later tokens drawn from softmax(logits / temperature) (Gumbel-max with
+        counter-based noise, see photon.h); temperature 0 = greedy."""
+        _check(load_library().photon_cache_set_sampling(self._h, float(temperature), int(seed)))
 
     def info(self) -> dict:
         st = photon_cache_stats()

@@ -26,6 +26,7 @@
 #include "kernels.h"
 #include "launch.cuh"
 #include "ptx_sm100.cuh"
+#include "sampling.cuh"
 
 namespace photon {
 
@@ -48,7 +49,10 @@ struct TcCfg {
   static constexpr uint32_t kTmemCols = BN < 32 ? 32 : BN;
 };
 
-template <int BN, int STAGES, bool SWAP>
+// SAMPLE: an EPI_ARGMAX head whose rows draw tokens (temperature sampling,
+// sampling.cuh) instead of taking the greedy maximum; only the normal
+// orientation has it, and greedy launches run the SAMPLE = false instances.
+template <int BN, int STAGES, bool SWAP, bool SAMPLE = false>
 __global__ void __launch_bounds__(128, 1)
     k_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
               int M, int N, int nkb, int kb_per_split, Epilogue ep, float* __restrict__ part,
@@ -182,6 +186,8 @@ __global__ void __launch_bounds__(128, 1)
       // thread = output row; 64 columns at a time (a whole RoPE head)
       const long long grow = a0 + tl;
       unsigned long long best = 0ull;
+      const bool skey_on = SAMPLE && ep.kind == EPI_ARGMAX && grow < M && !part;
+      const uint32_t skey = skey_on ? sample_row_key(ep.samp, grow) : 0u;
 #pragma unroll 1
       for (int j0 = 0; j0 < BN; j0 += 64) {
         float lo[32], hi[32];
@@ -196,10 +202,20 @@ __global__ void __launch_bounds__(128, 1)
 #pragma unroll
           for (int i = 0; i < 8; ++i) p[8 + i] = make_float4(hi[4 * i], hi[4 * i + 1], hi[4 * i + 2], hi[4 * i + 3]);
         } else if (ep.kind == EPI_ARGMAX) {
+          if constexpr (SAMPLE) {
+            const float it = ep.samp.inv_t;
 #pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            best = max(best, argmax_key(lo[i], gc + i));
-            best = max(best, argmax_key(hi[i], gc + 32 + i));
+            for (int i = 0; i < 32; ++i) {
+              best = max(best, argmax_key(sample_value(it, skey, lo[i], gc + i), gc + i));
+              best = max(best, argmax_key(sample_value(it, skey, hi[i], gc + 32 + i), gc + 32 + i));
+            }
+            (void)skey_on;
+          } else {
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+              best = max(best, argmax_key(lo[i], gc + i));
+              best = max(best, argmax_key(hi[i], gc + 32 + i));
+            }
           }
           if (ep.out) {
 #pragma unroll
@@ -368,7 +384,7 @@ __device__ __forceinline__ void tile_coords(int tile, int tiles_n, int n_tiles, 
 // accumulators; two TMEM accumulators (2 x BN columns) let the epilogue of
 // tile i overlap the main loop of tile i+1.  Epilogue warp w owns TMEM lanes
 // 32*(w%4)..+31, i.e. output rows of that quarter.
-template <int BN, int STAGES>
+template <int BN, int STAGES, bool SAMPLE = false>
 __global__ void __launch_bounds__(192, 1)
     k_gemm_tc_persist(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                       int M, int N, int nkb, int tiles_n, int n_tiles, int nt_major, Epilogue ep,
@@ -486,6 +502,8 @@ __global__ void __launch_bounds__(192, 1)
       const long long grow = (long long)mt * kBM + q * 32 + lane;
       const uint32_t trow = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(b * BN);
       unsigned long long best = 0ull;
+      const bool skey_on = SAMPLE && ep.kind == EPI_ARGMAX && grow < M;
+      const uint32_t skey = skey_on ? sample_row_key(ep.samp, grow) : 0u;
       // split RMSNorm consumer: this row's 1 / rms from the producer's slots
       float rs = 1.f;
       if (ep.ssq_in != nullptr && grow < M) {
@@ -508,10 +526,20 @@ __global__ void __launch_bounds__(192, 1)
         const int gc = nt * BN + j0;
         if (grow >= M || gc >= N) continue;
         if (ep.kind == EPI_ARGMAX) {
+          if constexpr (SAMPLE) {
+            const float it = ep.samp.inv_t;
 #pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            best = max(best, argmax_key(lo[i], gc + i));
-            best = max(best, argmax_key(hi[i], gc + 32 + i));
+            for (int i = 0; i < 32; ++i) {
+              best = max(best, argmax_key(sample_value(it, skey, lo[i], gc + i), gc + i));
+              best = max(best, argmax_key(sample_value(it, skey, hi[i], gc + 32 + i), gc + 32 + i));
+            }
+            (void)skey_on;
+          } else {
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+              best = max(best, argmax_key(lo[i], gc + i));
+              best = max(best, argmax_key(hi[i], gc + 32 + i));
+            }
           }
           if (ep.out) {
             float* o = reinterpret_cast<float*>(ep.out) + grow * ep.ldo + gc;
@@ -1062,29 +1090,29 @@ bool make_map(CUtensorMap* m, const void* ptr, long long rows, int K, long long 
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int BN, int STAGES, bool SWAP>
+template <int BN, int STAGES, bool SWAP, bool SAMPLE = false>
 void run_tc(const CUtensorMap& ma, const CUtensorMap& mb, int grid_a, int grid_b, int splits,
             int M, int N, int nkb, int kbs, const Epilogue& ep, float* part, int* counters,
             const void* w_ptr, long long w_ld_bytes, int* err, cudaStream_t s) {
   using Cfg = TcCfg<BN, STAGES>;
   static bool configured = false;
   if (!configured) {
-    cudaFuncSetAttribute(k_gemm_tc<BN, STAGES, SWAP>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    cudaFuncSetAttribute(k_gemm_tc<BN, STAGES, SWAP, SAMPLE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                          Cfg::kSmemBytes);
     configured = true;
   }
   dim3 grid(grid_a, grid_b, splits);
-  launch_kernel(k_gemm_tc<BN, STAGES, SWAP>, grid, 128, Cfg::kSmemBytes, s, ma, mb, M, N, nkb, kbs, ep, part,
-                counters, static_cast<const char*>(w_ptr), w_ld_bytes, err);
+  launch_kernel(k_gemm_tc<BN, STAGES, SWAP, SAMPLE>, grid, 128, Cfg::kSmemBytes, s, ma, mb, M, N, nkb, kbs,
+                ep, part, counters, static_cast<const char*>(w_ptr), w_ld_bytes, err);
 }
 
-template <int BN, int STAGES>
+template <int BN, int STAGES, bool SAMPLE = false>
 void run_tc_persist(const CUtensorMap& ma, const CUtensorMap& mb, int M, int N, int nkb,
                     const Epilogue& ep, int nt_major, int* err, cudaStream_t s) {
   using Cfg = TcCfg<BN, STAGES>;
   static int sms = 0;
   if (!sms) {
-    cudaFuncSetAttribute(k_gemm_tc_persist<BN, STAGES>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    cudaFuncSetAttribute(k_gemm_tc_persist<BN, STAGES, SAMPLE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                          Cfg::kSmemBytes);
     int dev = 0;
     cudaGetDevice(&dev);
@@ -1094,8 +1122,8 @@ void run_tc_persist(const CUtensorMap& ma, const CUtensorMap& mb, int M, int N, 
   const int tiles_n = (N + BN - 1) / BN;
   const int n_tiles = ((M + kBM - 1) / kBM) * tiles_n;
   const int grid = n_tiles < sms ? n_tiles : sms;
-  launch_kernel(k_gemm_tc_persist<BN, STAGES>, dim3(grid), dim3(192), Cfg::kSmemBytes, s, ma, mb, M,
-                N, nkb, tiles_n, n_tiles, nt_major, ep, err);
+  launch_kernel(k_gemm_tc_persist<BN, STAGES, SAMPLE>, dim3(grid), dim3(192), Cfg::kSmemBytes, s, ma, mb,
+                M, N, nkb, tiles_n, n_tiles, nt_major, ep, err);
 }
 
 // How many clusters of k_gemm_dec<BN, S, STAGES> can be resident at once
@@ -1442,6 +1470,10 @@ bool launch_gemm_tc(const GemmArgs& a, const GemmWorkspace& ws, int* err, cudaSt
   }
   CUtensorMap ma, mb;
   const int nkb = K / kBK;
+  // a sampling head runs the SAMPLE instances, which exist for the normal
+  // orientation without split-K (the only plan a head gets)
+  const bool sample = argmax && a.ep.samp.inv_t > 0.f;
+  if (sample && (p.swap || p.splits != 1)) return false;
   if (p.swap) {
     if (!make_map(&ma, a.W, N, K, a.ldw, kBM) || !make_map(&mb, a.A, M, K, a.lda, p.bn)) return false;
     if (p.bn == 64)
@@ -1457,15 +1489,23 @@ bool launch_gemm_tc(const GemmArgs& a, const GemmWorkspace& ws, int* err, cudaSt
     if (p.splits == 1 && (argmax || p.ga * p.gb >= persist_min_tiles()) && persistent_enabled()) {
       const int nt_major = argmax ? 1 : 0;
       if (p.bn == 256)
-        run_tc_persist<256, 4>(ma, mb, M, N, nkb, a.ep, nt_major, err, s);
+        sample ? run_tc_persist<256, 4, true>(ma, mb, M, N, nkb, a.ep, nt_major, err, s)
+               : run_tc_persist<256, 4>(ma, mb, M, N, nkb, a.ep, nt_major, err, s);
       else
-        run_tc_persist<128, 6>(ma, mb, M, N, nkb, a.ep, nt_major, err, s);
+        sample ? run_tc_persist<128, 6, true>(ma, mb, M, N, nkb, a.ep, nt_major, err, s)
+               : run_tc_persist<128, 6>(ma, mb, M, N, nkb, a.ep, nt_major, err, s);
       return true;
     }
     if (p.bn == 256)
-      run_tc<256, 4, false>(ma, mb, p.ga, p.gb, p.splits, M, N, nkb, p.kbs, a.ep, part, counters, a.W, a.ldw * 2, err, s);
+      sample ? run_tc<256, 4, false, true>(ma, mb, p.ga, p.gb, p.splits, M, N, nkb, p.kbs, a.ep, part, counters,
+                                           a.W, a.ldw * 2, err, s)
+             : run_tc<256, 4, false>(ma, mb, p.ga, p.gb, p.splits, M, N, nkb, p.kbs, a.ep, part, counters, a.W,
+                                     a.ldw * 2, err, s);
     else
-      run_tc<128, 4, false>(ma, mb, p.ga, p.gb, p.splits, M, N, nkb, p.kbs, a.ep, part, counters, a.W, a.ldw * 2, err, s);
+      sample ? run_tc<128, 4, false, true>(ma, mb, p.ga, p.gb, p.splits, M, N, nkb, p.kbs, a.ep, part, counters,
+                                           a.W, a.ldw * 2, err, s)
+             : run_tc<128, 4, false>(ma, mb, p.ga, p.gb, p.splits, M, N, nkb, p.kbs, a.ep, part, counters, a.W,
+                                     a.ldw * 2, err, s);
   }
   return true;
 }

@@ -7,6 +7,7 @@
 #include "epilogue.cuh"
 #include "kernels.h"
 #include "launch.cuh"
+#include "sampling.cuh"
 
 namespace photon {
 
@@ -254,7 +255,7 @@ __device__ __forceinline__ void better(float& bv, int& bi, float v, int i) {
 }
 __global__ void k_argmax(const float* __restrict__ logits, long long ld, int rows, int V, int step,
                          int C1, const int32_t* __restrict__ force, int32_t* own, int32_t* used,
-                         int32_t* next_ids, int* err) {
+                         int32_t* next_ids, int* err, SampleArgs samp) {
   pdl_wait();
   pdl_trigger();
   const int row = blockIdx.x;
@@ -262,7 +263,12 @@ __global__ void k_argmax(const float* __restrict__ logits, long long ld, int row
   const float* lr = logits + (long long)row * ld;
   float bv = -INFINITY;
   int bi = 0x7fffffff;
-  for (int c = threadIdx.x; c < V; c += blockDim.x) better(bv, bi, lr[c], c);
+  if (samp.inv_t > 0.f) {
+    const uint32_t key = sample_row_key(samp, row);
+    for (int c = threadIdx.x; c < V; c += blockDim.x) better(bv, bi, sample_value(samp.inv_t, key, lr[c], c), c);
+  } else {
+    for (int c = threadIdx.x; c < V; c += blockDim.x) better(bv, bi, lr[c], c);
+  }
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) {
     const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
@@ -297,18 +303,23 @@ __global__ void k_argmax(const float* __restrict__ logits, long long ld, int row
 }
 void launch_argmax(const float* logits, long long ld, int rows, int V, int i, int C1,
                    const int32_t* force, int32_t* own, int32_t* used, int32_t* next_ids, int* err,
-                   cudaStream_t s) {
+                   const SampleArgs& samp, cudaStream_t s) {
   if (rows <= 0) return;
-  launch_kernel(k_argmax, rows, 256, 0, s, logits, ld, rows, V, i, C1, force, own, used, next_ids, err);
+  launch_kernel(k_argmax, rows, 256, 0, s, logits, ld, rows, V, i, C1, force, own, used, next_ids, err,
+                samp);
 }
 
 // One warp per row: max over the row's tile partials, then the same token
 // bookkeeping as k_argmax.
 __global__ void k_argmax_partials(const unsigned long long* __restrict__ part, int tiles, int rows,
                                   int V, int step, int C1, const int32_t* __restrict__ force,
-                                  int32_t* own, int32_t* used, int32_t* next_ids, int* err) {
+                                  int32_t* own, int32_t* used, int32_t* next_ids, int* err,
+                                  int* chunk_ctr) {
   pdl_wait();
   pdl_trigger();
+  // the chunk's last head has been reduced: count the chunk (nothing in this
+  // launch reads the counter; the sampling heads of later chunks do)
+  if (chunk_ctr && blockIdx.x == 0 && threadIdx.x == 0) *chunk_ctr += 1;
   const int row = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
   if (row >= rows) return;
@@ -336,10 +347,10 @@ __global__ void k_argmax_partials(const unsigned long long* __restrict__ part, i
 }
 void launch_argmax_partials(const unsigned long long* part, int tiles, int rows, int V, int i,
                             int C1, const int32_t* force, int32_t* own, int32_t* used,
-                            int32_t* next_ids, int* err, cudaStream_t s) {
+                            int32_t* next_ids, int* err, int* chunk_ctr, cudaStream_t s) {
   if (rows <= 0) return;
   launch_kernel(k_argmax_partials, (rows * 32 + 255) / 256, 256, 0, s, part, tiles, rows, V, i, C1,
-                force, own, used, next_ids, err);
+                force, own, used, next_ids, err, chunk_ctr);
 }
 
 // Greedy choice from the head's tile partials (as k_argmax_partials), then,

@@ -23,6 +23,15 @@ enum EpiKind : int {
 // Epilogue parameters.  For EPI_QKV the GEMM output has 3*d columns
 // (q | k | v).  Row r belongs to group g = r / q_len (a sequence, or a
 // decoder sub-chunk) and sits at stream position pos = p0 + r % q_len.
+// Temperature sampling of the token decoder's head (csrc/sampling.cuh):
+// with inv_t > 0 the row's maximum runs over logit * inv_t + Gumbel noise.
+struct SampleArgs {
+  float inv_t = 0.f;             // 1 / temperature; 0 = greedy
+  unsigned long long seed = 0;
+  const int* chunk = nullptr;    // device: chunks the cache has generated so far
+  int C1 = 0, C2 = 0, i = 0;     // head row = b*C2 + j emits token j*C1 + i of the chunk
+};
+
 // q and k are rotated (rotate-half RoPE with the table `rope`, float2
 // (cos, sin) per [pos][i], i < dh/2); q goes to q_out[r, :d]; k and v go to
 // the caches laid out [G][H][cap][dh] at slot pos - kv_off.
@@ -43,6 +52,7 @@ struct Epilogue {
   // (if set) receives the fp32 logits.
   unsigned long long* argmax_part = nullptr;
   int argmax_tiles = 0;
+  SampleArgs samp;  // EPI_ARGMAX: temperature sampling instead of greedy when samp.inv_t > 0
   // RMSNorm split across a producer / consumer pair of GEMMs (a pre-norm
   // block's residual update and the next projection).  RMSNorm(x)[r] =
   // rstd[r] * x[r] * g with a scalar rstd per row, so the next projection can
@@ -135,12 +145,14 @@ void launch_embed_f32(int dt, const int32_t* ids, const void* E, float* x, int r
 // out[r, :] = T(rmsnorm(x[r*in_step + in_off, :]) * g).
 void launch_rmsnorm(int dt, const float* x, const float* g, void* out, int rows, int d,
                     int in_step, int in_off, float eps, cudaStream_t s);
-// Greedy token for row g of logits (lowest index among maxima).  Writes the
-// own choice to own[g*C1 + i]; the token fed back (force[g*C1+i] if >= 0,
-// else the own choice) to used[g*C1 + i] and next_ids[g].
+// Greedy token for row g of logits (lowest index among maxima), or with
+// samp.inv_t > 0 the token drawn from softmax(logits * inv_t) (Gumbel-max,
+// sampling.cuh).  Writes the own choice to own[g*C1 + i]; the token fed back
+// (force[g*C1+i] if >= 0, else the own choice) to used[g*C1 + i] and
+// next_ids[g].
 void launch_argmax(const float* logits, long long ld, int rows, int V, int i, int C1,
                    const int32_t* force, int32_t* own, int32_t* used, int32_t* next_ids, int* err,
-                   cudaStream_t s);
+                   const SampleArgs& samp, cudaStream_t s);
 // Greedy token per row from the head GEMM's per-tile partials (EPI_ARGMAX);
 // same outputs as launch_argmax.
 // argmax from tile partials + embedding of the chosen token into x + its
@@ -149,9 +161,11 @@ void launch_argmax_embed_norm(int dt, const unsigned long long* part, int tiles,
                               int C1, const int32_t* force, int32_t* own, int32_t* used,
                               int32_t* next_ids, int* err, const void* E, float* x, const float* g,
                               void* xn, int d, float eps, cudaStream_t s);
+// chunk_ctr (nullable): incremented once, after the reduction (the chunk count
+// the sampling heads read).
 void launch_argmax_partials(const unsigned long long* part, int tiles, int rows, int V, int i,
                             int C1, const int32_t* force, int32_t* own, int32_t* used,
-                            int32_t* next_ids, int* err, cudaStream_t s);
+                            int32_t* next_ids, int* err, int* chunk_ctr, cudaStream_t s);
 // pos[0] += dN; pos[1] += dN1 (device-side decode positions).
 void launch_advance(int* pos, int dN, int dN1, cudaStream_t s);
 

@@ -356,7 +356,9 @@ struct photon_cache {
   float* attn_ws = nullptr;
   size_t attn_ws_bytes = 0;
   int* d_err = nullptr;
-  int* d_pos = nullptr;          // device copies of {N, N1} read by the decode kernels
+  int* d_pos = nullptr;          // device {N, N1, chunks generated, 0} read by the decode kernels
+  float samp_inv_t = 0.f;        // token sampling: 1 / temperature (0: greedy)
+  unsigned long long samp_seed = 0;
   unsigned long long* amax_part = nullptr;  // [B*C2][amax_cap] head partials
   int amax_cap = 0;
   int32_t* tok_out = nullptr;    // [B, C] greedy tokens of the last graph-replayed step
@@ -1023,7 +1025,7 @@ int photon_prefill(photon_model* m, const photon_cache* prefix, const int32_t* d
     c->N1 = 0;
   }
   {
-    const int pos[2] = {c->N, c->N1};  // pageable source: staged before the call returns
+    const int pos[4] = {c->N, c->N1, 0, 0};  // pageable source: staged before the call returns
     if (cudaMemcpyAsync(c->d_pos, pos, sizeof(pos), cudaMemcpyHostToDevice, s) != cudaSuccess)
       return bail(fail(PHOTON_ERR_CUDA, "position upload failed"));
   }
@@ -1236,15 +1238,24 @@ static void enqueue_decode(photon_model* m, photon_cache* c, int mode, int32_t* 
   run_stack(m, m->i_dec1, m->Ld1, xdk, r1, bk, ts);
   const int amax_tiles = m->use_tc ? gemm_tc_argmax_tiles(G, V, d) : 0;
   bool fused_embed = false;  // the last head also embedded and normalised the next step's input
+  int* chunk_ctr = c->d_pos + 2;  // chunks this cache has generated (sampling keys)
   auto head = [&](const float* x, int in_step, int in_off, int i) {
     launch_rmsnorm(m->dt, x, (const float*)m->ptr(m->i_dec1_g), c->hn, G, d, in_step, in_off, eps, ts);
     const long long ld = d_out_logits ? (long long)C1 * V : V;
+    SampleArgs sa;
+    sa.inv_t = c->samp_inv_t;
+    sa.seed = c->samp_seed;
+    sa.chunk = chunk_ctr;
+    sa.C1 = C1;
+    sa.C2 = C2;
+    sa.i = i;
     if (amax_tiles > 0 && amax_tiles <= c->amax_cap) {
       // tensor-core head with the greedy choice fused into its epilogue;
       // logits are written only when the caller asks for them
       Epilogue e = epi(EPI_ARGMAX, d_out_logits ? d_out_logits + (size_t)i * V : nullptr, ld);
       e.argmax_part = c->amax_part;
       e.argmax_tiles = amax_tiles;
+      e.samp = sa;
       gemm(m, bk, c->hn, d, m->ptr(m->i_head), d, G, V, d, e, ts);
       if (i + 1 < C1) {
         // greedy choice + the next step's embedding and first attention norm
@@ -1254,13 +1265,14 @@ static void enqueue_decode(photon_model* m, photon_cache* c, int mode, int32_t* 
         fused_embed = true;
       } else {
         launch_argmax_partials(c->amax_part, amax_tiles, G, V, i, C1, d_force_tokens, d_out_tokens,
-                               c->used, c->next_ids, c->d_err, ts);
+                               c->used, c->next_ids, c->d_err, chunk_ctr, ts);
       }
     } else {
       float* lg = d_out_logits ? d_out_logits + (size_t)i * V : c->logits;
       gemm(m, bk, c->hn, d, m->ptr(m->i_head), d, G, V, d, epi(EPI_STORE_F32, lg, ld), ts);
       launch_argmax(lg, ld, G, V, i, C1, d_force_tokens, d_out_tokens, c->used, c->next_ids,
-                    c->d_err, ts);
+                    c->d_err, sa, ts);
+      if (i + 1 == C1) launch_advance(chunk_ctr, 1, 0, ts);  // count the chunk
     }
   };
   head(xdk, C1, C1 - 1, 0);
@@ -1605,6 +1617,23 @@ int photon_free_cache(photon_cache* c) {
   m->live_caches--;
   if (c->mode == PHOTON_MODE_HIER) m->hier_caches--;
   delete c;
+  return PHOTON_OK;
+}
+
+int photon_cache_set_sampling(photon_cache* c, float temperature, uint64_t seed) {
+  g_err.clear();
+  if (!c) return fail(PHOTON_ERR_ARG, "cache is NULL");
+  if (!(temperature >= 0.f) || !std::isfinite(temperature))
+    return fail(PHOTON_ERR_ARG, "temperature must be finite and >= 0");
+  if (temperature > 0.f && !std::isfinite(1.0f / temperature))
+    return fail(PHOTON_ERR_ARG, "temperature %g is too small", (double)temperature);
+  c->samp_inv_t = temperature > 0.f ? 1.0f / temperature : 0.f;
+  c->samp_seed = seed;
+  // captured steps carry the old parameters: capture again on the next step
+  photon_model* m = c->m;
+  for (int k = 0; k < 2; ++k)
+    if (m->graph_owner[k] == c) m->graph_owner[k] = nullptr;
+  if (m->pg_owner == c) m->pg_owner = nullptr;
   return PHOTON_OK;
 }
 

@@ -177,6 +177,25 @@ PHOTON_API int photon_decode_rec_chunks(photon_model* m, photon_cache* c, int32_
  * invalid afterwards. */
 PHOTON_API int photon_free_cache(photon_cache* c);
 
+/* Token choice of the cache's later decode steps (both modes).
+ * temperature == 0: greedy (lowest id among the maxima), the default.
+ * temperature > 0: each token is drawn from softmax(logits / temperature) by
+ * the Gumbel-max rule: argmax_v(logit_v / T + G_v), ties to the lowest id,
+ * with standard Gumbel noise G_v = -ln(-ln u_v) from a counter-based
+ * generator (a pure function of seed, the sequence's batch row b, the
+ * token's index t among the tokens this cache has generated, and v):
+ *   K   = mix64(mix64(seed + g*(b+1)) + g*(t+1)), k32 = (K >> 32) ^ (K & 0xFFFFFFFF)
+ *         (mix64: the SplitMix64 output function, g = 0x9E3779B97F4A7C15),
+ *   h   = fmix32(k32 + 0x9E3779B9*(v+1) mod 2^32)  (MurmurHash3's finaliser),
+ *   u_v = (floor(h / 256) + 1/2) / 2^24.
+ * The explainer's quality section (several varied queries per prompt)
+ * motivates sampling; the pages do not fix the sampler.  Tokens written by
+ * photon_decode_step_ex's teacher forcing are unaffected; the own choices
+ * are sampled.  Host-only (no device work); the next decode call re-captures
+ * its graphs.  Errors: ERR_ARG (NULL cache, negative, NaN, infinite or
+ * subnormal-reciprocal temperature). */
+PHOTON_API int photon_cache_set_sampling(photon_cache* c, float temperature, uint64_t seed);
+
 typedef struct photon_cache_stats {
   int32_t B, T, mode;
   int32_t N;          /* top-level entries visible (prefix + own) */
