@@ -281,14 +281,32 @@ def run_gpu(args) -> None:
     hc.free()
     hier_dec_ms = hev[1].elapsed_time(hev[2])
 
+    # ---- RecGen with temperature sampling (T = 1, the draw fused into the
+    # head's epilogue), one timed multi-chunk call after an untimed one
+    def sampled_pass(ev=None):
+        c = model.prefill(toks, hal.MODE_REC, chunks)
+        c.set_sampling(1.0, 2024)
+        if ev is not None:
+            ev[0].record(stream)
+        c.decode_rec_chunks(chunks, out)
+        if ev is not None:
+            ev[1].record(stream)
+        return c
+    sampled_pass().free()
+    sev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+    torch.cuda.synchronize()
+    sampled_pass(sev).free()
+    torch.cuda.synchronize()
+    samp_dec_ms = sev[0].elapsed_time(sev[1])
+
     # ---- the decode's dominant kernel (its GEMM launches) and its attention,
     # alone, at the same shapes and launch configuration
     roof = measure_gemm_roofline(model, wl, dev, stream)
     roof_attn = measure_attn_roofline(model, wl, dev, stream)
     roof_prefill = measure_prefill_roofline(model, wl, dev, stream)
 
-    total_ms, prefill_ms, decode_ms, e2e_ms, hier_dec_ms = max_over_ranks(
-        [total_ms, prefill_ms, decode_ms, e2e_ms, hier_dec_ms], device=dev)
+    total_ms, prefill_ms, decode_ms, e2e_ms, hier_dec_ms, samp_dec_ms = max_over_ranks(
+        [total_ms, prefill_ms, decode_ms, e2e_ms, hier_dec_ms, samp_dec_ms], device=dev)
 
     dec_tokens = world * B * chunks * C * args.steps
     value = job_throughput(B * chunks * C * args.steps, world, decode_ms)
@@ -324,6 +342,9 @@ def run_gpu(args) -> None:
                     "resident_gib": round(hier_res / 2 ** 30, 4),
                     "tok_s_per_gib": round(B * chunks * C / (hier_dec_ms / 1e3) / (hier_res / 2 ** 30), 1),
                     "steps": 1},
+        "recgen_sampled": {"temperature": 1.0,
+                           "decode_tok_s": round(job_throughput(B * chunks * C, world, samp_dec_ms), 1),
+                           "decode_ms_per_chunk": round(samp_dec_ms / chunks, 4), "steps": 1},
         "decode_graph": {"steps_replayed_per_cache": cinfo["graph_steps"], "steps_per_cache": chunks,
                          "kernels_per_step": cinfo["graph_kernels"]},
         "gpu_launches": launches,
