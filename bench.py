@@ -41,7 +41,7 @@ import time
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
-from synth_inputs import WEIGHT_SEED, WORKLOADS, model_shape, prompt_tokens  # noqa: E402
+from synth_inputs import WEIGHT_SEED, WORKLOADS, model_shape, prefix_tokens, prompt_tokens  # noqa: E402
 
 METRIC = "RecGen decode tok/s and tok/s/GiB (TPM) on 1 B200; % of HBM roofline"
 UNIT = "tok/s"
@@ -164,6 +164,22 @@ def run_gpu(args) -> None:
     step_out = torch.empty(B, C, dtype=torch.int32, device=dev)
     stream = torch.cuda.current_stream()
 
+    # multi-query serving (c5): every rank prefills the shared context once
+    # (HierGen mode keeps its level-1 cache for the queries' prefill); each
+    # step's queries are prefilled after it and read its top cache in place
+    prefix_len = wl.get("prefix_len", 0)
+    pre_cache, prefix_ms = None, 0.0
+    if prefix_len:
+        pre_dev = torch.from_numpy(np.ascontiguousarray(prefix_tokens(args.workload))).to(dev)
+        pe = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+        model.prefill(pre_dev, hal.MODE_HIER, 0).free()          # untimed warm-up
+        torch.cuda.synchronize()
+        pe[0].record(stream)
+        pre_cache = model.prefill(pre_dev, hal.MODE_HIER, 0)
+        pe[1].record(stream)
+        torch.cuda.synchronize()
+        prefix_ms = pe[0].elapsed_time(pe[1])
+
     def one_step(ev=None, mark=False):
         # mark: NVTX ranges around the prefill and one middle decode chunk,
         # the windows the ncu launch-list summaries capture
@@ -171,7 +187,7 @@ def run_gpu(args) -> None:
             ev[0].record(stream)
         if mark:
             torch.cuda.nvtx.range_push("prefill")
-        cache = model.prefill(toks, hal.MODE_REC, chunks)
+        cache = model.prefill(toks, hal.MODE_REC, chunks, prefix=pre_cache)
         if mark:
             torch.cuda.nvtx.range_pop()
         if ev is not None:
@@ -206,7 +222,8 @@ def run_gpu(args) -> None:
     torch.cuda.synchronize()
     cinfo, minfo = probe.info(), model.info()
     probe.free()
-    resident = minfo["resident_bytes"] + cinfo["kv_bytes"]
+    pre_kv = pre_cache.info()["kv_bytes"] if pre_cache is not None else 0
+    resident = minfo["resident_bytes"] + cinfo["kv_bytes"] + pre_kv  # a shared prefix counts once
 
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
     if world > 1:
@@ -245,7 +262,7 @@ def run_gpu(args) -> None:
     e0.record(stream)
     for _ in range(e2e_steps):
         dev_in.copy_(pin_in, non_blocking=True)
-        cache = model.prefill(dev_in, hal.MODE_REC, chunks)
+        cache = model.prefill(dev_in, hal.MODE_REC, chunks, prefix=pre_cache)
         if args.decode_api == "chunks":
             cache.decode_rec_chunks(chunks, out)
             pin_out.copy_(out, non_blocking=True)
@@ -263,7 +280,7 @@ def run_gpu(args) -> None:
     def hier_pass(ev=None):
         if ev is not None:
             ev[0].record(stream)
-        c = model.prefill(toks, hal.MODE_HIER, chunks)
+        c = model.prefill(toks, hal.MODE_HIER, chunks, prefix=pre_cache)
         if ev is not None:
             ev[1].record(stream)
         for s in range(chunks):
@@ -284,7 +301,7 @@ def run_gpu(args) -> None:
     # ---- RecGen with temperature sampling (T = 1, the draw fused into the
     # head's epilogue), one timed multi-chunk call after an untimed one
     def sampled_pass(ev=None):
-        c = model.prefill(toks, hal.MODE_REC, chunks)
+        c = model.prefill(toks, hal.MODE_REC, chunks, prefix=pre_cache)
         c.set_sampling(1.0, 2024)
         if ev is not None:
             ev[0].record(stream)
@@ -302,8 +319,14 @@ def run_gpu(args) -> None:
     # ---- the decode's dominant kernel (its GEMM launches) and its attention,
     # alone, at the same shapes and launch configuration
     roof = measure_gemm_roofline(model, wl, dev, stream)
-    roof_attn = measure_attn_roofline(model, wl, dev, stream)
+    if prefix_len:
+        roof_attn = {"unavailable": "the shared-prefix attention reads one 4 MiB prefix per layer for "
+                                    "all queries (L2-resident); the standalone measurement has no prefix"}
+    else:
+        roof_attn = measure_attn_roofline(model, wl, dev, stream)
     roof_prefill = measure_prefill_roofline(model, wl, dev, stream)
+    if pre_cache is not None:
+        pre_cache.free()
 
     total_ms, prefill_ms, decode_ms, e2e_ms, hier_dec_ms, samp_dec_ms = max_over_ranks(
         [total_ms, prefill_ms, decode_ms, e2e_ms, hier_dec_ms, samp_dec_ms], device=dev)
@@ -318,7 +341,10 @@ def run_gpu(args) -> None:
         "scaling": "weak", "vs_baseline": None, "dtype": shape["dtype"],
         "data": "synthetic: seeded N(0,0.02)-like weights (SplitMix64 + Irwin-Hall), Zipf(1.1) prompt ids",
         "config": {"workload": f"{args.workload}: PHOTON 600M-class L=2 C1=C2={shape['C1']}, "
-                               f"B={B} per GPU, prompt {T}, RecGen decode {chunks * C} tokens",
+                               f"B={B} per GPU, prompt {T}"
+                               + (f" after a shared {prefix_len}-token prefix (prefilled once)"
+                                  if prefix_len else "")
+                               + f", RecGen decode {chunks * C} tokens",
                    "batch_per_gpu": B, "prompt_len": T, "decode_tokens": chunks * C,
                    "parallelism": f"dp{world}", "l2": "working set > L2 (no flush)",
                    "decode_api": args.decode_api},
@@ -326,11 +352,12 @@ def run_gpu(args) -> None:
         "decode_ms_per_chunk": round(decode_ms / args.steps / chunks, 4),
         "prefill_tok_s": round(world * B * T * args.steps / (prefill_ms / 1e3), 1),
         "prefill_ms_steps": [round(e[0].elapsed_time(e[1]), 3) for e in evs],
+        "prefix_prefill_ms": round(prefix_ms, 3) if prefix_len else None,
         "job_tok_s": round(dec_tokens / (total_ms / 1e3), 1),
         "tpm": {"tok_s_per_gib": round(value / world / gib, 1), "resident_gib": round(gib, 4),
                 "weights_gib": round(minfo["resident_bytes"] / 2 ** 30, 4),
-                "kv_gib": round(cinfo["kv_bytes"] / 2 ** 30, 4),
-                "tok_s_per_gib_kv_only": round(value / world / (cinfo["kv_bytes"] / 2 ** 30), 1),
+                "kv_gib": round((cinfo["kv_bytes"] + pre_kv) / 2 ** 30, 4),
+                "tok_s_per_gib_kv_only": round(value / world / ((cinfo["kv_bytes"] + pre_kv) / 2 ** 30), 1),
                 "per_gpu": True},
         "e2e": {"value": round(world * B * chunks * C * e2e_steps / (e2e_ms / 1e3), 1), "unit": UNIT,
                 "h2d_bytes_per_step": int(B * T * 4), "d2h_bytes_per_step": int(B * chunks * C * 4),
@@ -571,6 +598,17 @@ def measure_attn_roofline(model, wl, dev, stream) -> dict:
             "shape": f"B={B} H={H} dh={dh} keys={n_mid}"}
 
 
+def oracle_prompt(workload: str):
+    """Sequence 0's whole context: the shared prefix (if the workload has one)
+    followed by its own prompt; the oracle's prefill of it equals prefilling
+    the prompt after the prefix (a pinned identity)."""
+    import numpy as np
+    toks = prompt_tokens(workload, batch=1)[0]
+    if WORKLOADS[workload].get("prefix_len"):
+        toks = np.concatenate([prefix_tokens(workload)[0], toks])
+    return toks
+
+
 def cpu_baseline(workload: str, budget_s: float = 20.0) -> dict:
     """The fp64 oracle, as it stands, on the host cores: RecGen decode of one
     sequence of the workload after its prefill; decode steps are timed until
@@ -580,8 +618,7 @@ def cpu_baseline(workload: str, budget_s: float = 20.0) -> dict:
     shape = model_shape(workload)
     cfg = Config.from_dict(shape)
     orc = PhotonOracle(cfg, WEIGHT_SEED)
-    toks = prompt_tokens(workload, batch=1)[0]
-    st = orc.prefill(toks, "rec")
+    st = orc.prefill(oracle_prompt(workload), "rec")
     n, t0 = 0, time.perf_counter()
     chunks = WORKLOADS[workload]["decode_tokens"] // cfg.C
     while n < chunks:
@@ -608,8 +645,7 @@ def run_reference(args) -> None:
     shape = model_shape(args.workload)
     cfg = Config.from_dict(shape)
     orc = PhotonOracle(cfg, WEIGHT_SEED)
-    toks = prompt_tokens(args.workload, batch=1)[0]
-    st = orc.prefill(toks, "rec")
+    st = orc.prefill(oracle_prompt(args.workload), "rec")
     for _ in range(min(args.warmup, 1)):
         orc.decode_step(st, "rec")
     per = []
@@ -644,7 +680,7 @@ def main() -> None:
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=5)
     ap.add_argument("--warmup", type=int, default=3)
-    ap.add_argument("--workload", default="c2", choices=["c2", "c3", "c4"])
+    ap.add_argument("--workload", default="c2", choices=["c2", "c3", "c4", "c5"])
     ap.add_argument("--impl", default="photon", choices=["photon", "reference"])
     ap.add_argument("--cpu-budget", type=float, default=20.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")

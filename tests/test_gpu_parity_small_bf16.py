@@ -174,3 +174,46 @@ def test_small_bf16_stream_ordered_free():
     info = model.info()
     assert info["live_caches"] == 0 and info["encoder_resident"] == 0
     model.free()
+
+
+@pytest.mark.parametrize("mode", ["rec", "hier"])
+def test_small_bf16_shared_prefix_parity(mode):
+    # queries prefilled after a shared context (prefilled once in HierGen
+    # mode) decode like the oracle's prefill_after state, in both modes:
+    # the top (and, for HierGen, level-1) attention reads the prefix rows
+    # from the shared cache and the rest from the query's own
+    orc = PhotonOracle(CFG, 7)
+    model = hal.Model(SHAPE, 7)
+    code = hal.MODE_HIER if mode == "hier" else hal.MODE_REC
+    rng = np.random.default_rng(21)
+    pre = rng.integers(0, SHAPE["vocab"], size=(1, T)).astype(np.int32)
+    qs = rng.integers(0, SHAPE["vocab"], size=(B, 64)).astype(np.int32)
+    pre_st = orc.prefill(pre[0], "hier")
+    sts = [orc.prefill_after(pre_st, qs[b], mode) for b in range(B)]
+    pre_cache = model.prefill(torch.from_numpy(pre).cuda(), hal.MODE_HIER, 0)
+    cache = model.prefill(torch.from_numpy(qs).cuda(), code, STEPS, prefix=pre_cache)
+    info = cache.info()
+    assert (info["N"], info["N1"], info["n_prefix"]) == (sts[0].N, sts[0].N1, pre_st.N)
+    out = torch.empty(B, CFG.C, dtype=torch.int32, device="cuda")
+    lg = torch.empty(B, CFG.C, CFG.vocab, device="cuda")
+    for step in range(STEPS):
+        refs = [orc.decode_step(st, mode) for st in sts]
+        force = torch.from_numpy(np.stack([r.tokens for r in refs]).astype(np.int32)).cuda()
+        cache.decode_step(code, out, lg, force_tokens=force)
+        torch.cuda.synchronize()
+        g = lg.double().cpu().numpy()
+        toks_gpu = out.cpu().numpy()
+        for b, r in enumerate(refs):
+            err = np.max(np.abs(g[b] - r.logits), axis=1)
+            assert np.max(err / np.max(np.abs(r.logits), axis=1)) < TOL, (step, b)
+            srt = np.sort(r.logits, axis=1)
+            decisive = (srt[:, -1] - srt[:, -2]) > 2 * err
+            np.testing.assert_array_equal(toks_gpu[b][decisive], r.tokens[decisive])
+        info = cache.info()
+        assert (info["N"], info["N1"], info["device_error"]) == (sts[0].N, sts[0].N1, 0)
+    o = f64(cache.export_state("pending_o")).reshape(B, -1)
+    for b in range(B):
+        assert rel(o[b], sts[b].o) < TOL
+    cache.free()
+    pre_cache.free()
+    model.free()
