@@ -747,19 +747,38 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
 
 }  // namespace fa
 
-__global__ void __launch_bounds__(128) k_attn_prefill_mma(AttnArgs a) {
+// Key segments of the tensor-core attention.  With a shared prefix the
+// attention splits in two passes whose partial softmaxes merge exactly:
+//   SEG_PREFIX: every query row of the batch (all groups stacked, one head
+//     per CTA column) against the prefix rows, no mask (the queries follow
+//     the prefix); writes fp32 partials (unnormalised accumulator, row max in
+//     log2 units, row sum) to part[(row * H + h) * (DH + 2)];
+//   SEG_OWN: one group's queries against its own keys (causal), merged with
+//     the prefix partial of each row before the bf16 store.
+// The prefix tile is then read once per 64 stacked queries instead of once
+// per (group, head), and no tile row is spent on padding.  SEG_ALL is the
+// single pass over prefix and own keys together.
+enum { SEG_ALL = 0, SEG_PREFIX = 1, SEG_OWN = 2 };
+
+template <int SEG>
+__global__ void __launch_bounds__(128) k_attn_prefill_mma(AttnArgs a, float* __restrict__ part) {
   using namespace fa;
   pdl_wait();
   pdl_trigger();
   __shared__ __align__(128) bf16 Qs[BM * LDS];
   __shared__ __align__(128) bf16 Ks[2][BN * LDS];
   __shared__ __align__(128) bf16 Vs[2][BN * LDS];
-  const int h = blockIdx.y, g = blockIdx.z;
+  const int h = blockIdx.y, g = SEG == SEG_PREFIX ? 0 : (int)blockIdx.z;
   const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
-  const int q0 = blockIdx.x * BM;                       // first query (index within the group)
-  const int nq = min(BM, a.q_len - q0);
-  const int last_pos = a.p0 + q0 + nq - 1;              // last query's position
-  const int n_keys = last_pos + 1;
+  const int p0 = a.p0_dev ? (*a.p0_dev + a.p0) : a.p0;  // first query's position
+  const int qrows = SEG == SEG_PREFIX ? a.G * a.q_len : a.q_len;  // this launch's query space
+  const long long qbase = SEG == SEG_PREFIX ? 0 : (long long)g * a.q_len;  // its first Q row
+  const int q0 = blockIdx.x * BM;                       // first query of this CTA
+  const int nq = min(BM, qrows - q0);
+  const int last_pos = p0 + q0 + nq - 1;                // last query's position (ALL, OWN)
+  const int key0 = SEG == SEG_OWN ? a.n_pre : 0;        // first key position of the segment
+  const int key_end = SEG == SEG_PREFIX ? a.n_pre : last_pos + 1;
+  const int n_keys = key_end - key0;
   const int nblocks = (n_keys + BN - 1) / BN;
   const bf16* Kown = reinterpret_cast<const bf16*>(a.K);
   const bf16* Vown = reinterpret_cast<const bf16*>(a.V);
@@ -772,18 +791,18 @@ __global__ void __launch_bounds__(128) k_attn_prefill_mma(AttnArgs a) {
     const int r = c >> 3, col = (c & 7) * 8;
     bf16* dst = Qs + r * LDS + col;
     if (r < nq)
-      cp_async16(dst, Qg + ((long long)g * a.q_len + q0 + r) * a.q_ld + h * D + col);
+      cp_async16(dst, Qg + (qbase + q0 + r) * a.q_ld + h * D + col);
     else
       *reinterpret_cast<uint4*>(dst) = make_uint4(0, 0, 0, 0);
   }
   auto load_kv = [&](int blk, int buf) {
-    const int k0 = blk * BN;
+    const int k0 = key0 + blk * BN;
     for (int c = t; c < BN * (D / 8); c += 128) {
       const int r = c >> 3, col = (c & 7) * 8;
       const int pos = k0 + r;
       bf16* kd = Ks[buf] + r * LDS + col;
       bf16* vd = Vs[buf] + r * LDS + col;
-      if (pos < n_keys) {
+      if (pos < key_end) {
         cp_async16(kd, key_row<bf16, D>(a, Kown, Kpre, g, h, pos) + col);
         cp_async16(vd, key_row<bf16, D>(a, Vown, Vpre, g, h, pos) + col);
       } else {
@@ -797,7 +816,7 @@ __global__ void __launch_bounds__(128) k_attn_prefill_mma(AttnArgs a) {
 
   const int gq = lane >> 2, tg = lane & 3;
   const int row0 = warp * 16 + gq;                      // this thread's rows: row0, row0 + 8
-  const int qpos0 = a.p0 + q0 + row0, qpos1 = qpos0 + 8;
+  const int qpos0 = p0 + q0 + row0, qpos1 = qpos0 + 8;
   const float sl2 = a.scale * 1.4426950408889634f;      // scores in log2 units
   float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
   float o[8][4];
@@ -837,7 +856,7 @@ __global__ void __launch_bounds__(128) k_attn_prefill_mma(AttnArgs a) {
       }
     }
     // causal mask + online softmax (rows row0 and row0 + 8)
-    const int kbase = blk * BN;
+    const int kbase = key0 + blk * BN;
     float mx0 = m0, mx1 = m1;
 #pragma unroll
     for (int nt = 0; nt < 8; ++nt) {
@@ -845,8 +864,12 @@ __global__ void __launch_bounds__(128) k_attn_prefill_mma(AttnArgs a) {
       for (int e = 0; e < 2; ++e) {
         const int kp = kbase + nt * 8 + tg * 2 + e;
         float v0 = sc[nt][e] * sl2, v1 = sc[nt][2 + e] * sl2;
-        if (kp > qpos0) v0 = -INFINITY;
-        if (kp > qpos1) v1 = -INFINITY;
+        if (SEG == SEG_PREFIX) {  // every prefix key is visible; the tail of the last block is not a key
+          if (kp >= key_end) v0 = v1 = -INFINITY;
+        } else {
+          if (kp > qpos0) v0 = -INFINITY;
+          if (kp > qpos1) v1 = -INFINITY;
+        }
         sc[nt][e] = v0;
         sc[nt][2 + e] = v1;
         mx0 = fmaxf(mx0, v0);
@@ -906,23 +929,81 @@ __global__ void __launch_bounds__(128) k_attn_prefill_mma(AttnArgs a) {
     }
     __syncthreads();
   }
-  // finish: row sums across the 4 threads of a row, normalise, store bf16
+  // finish: row sums across the 4 threads of a row
   l0 += __shfl_xor_sync(0xffffffffu, l0, 1);
   l0 += __shfl_xor_sync(0xffffffffu, l0, 2);
   l1 += __shfl_xor_sync(0xffffffffu, l1, 1);
   l1 += __shfl_xor_sync(0xffffffffu, l1, 2);
+  const long long fr0 = qbase + q0 + row0, fr1 = fr0 + 8;  // flattened query rows
+  if constexpr (SEG == SEG_PREFIX) {
+    // partial: unnormalised accumulator, row max (log2 units), row sum
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int col = i * 8 + tg * 2;
+      if (row0 < nq)
+        *reinterpret_cast<float2*>(part + (fr0 * a.H + h) * (D + 2) + col) = make_float2(o[i][0], o[i][1]);
+      if (row0 + 8 < nq)
+        *reinterpret_cast<float2*>(part + (fr1 * a.H + h) * (D + 2) + col) = make_float2(o[i][2], o[i][3]);
+    }
+    if (tg == 0) {
+      if (row0 < nq) *reinterpret_cast<float2*>(part + (fr0 * a.H + h) * (D + 2) + D) = make_float2(m0, l0);
+      if (row0 + 8 < nq) *reinterpret_cast<float2*>(part + (fr1 * a.H + h) * (D + 2) + D) = make_float2(m1, l1);
+    }
+    return;
+  }
+  // own keys (OWN): rescale both segments to their common maximum
+  float cp0 = 0.f, cp1 = 0.f;
+  const float* pp0 = part + (fr0 * a.H + h) * (D + 2);
+  const float* pp1 = part + (fr1 * a.H + h) * (D + 2);
+  if constexpr (SEG == SEG_OWN) {
+    if (row0 < nq) {
+      const float2 ml = *reinterpret_cast<const float2*>(pp0 + D);
+      const float M = fmaxf(m0, ml.x);
+      const float co = exp2f(m0 - M);
+      cp0 = exp2f(ml.x - M);
+      l0 = l0 * co + ml.y * cp0;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        o[i][0] *= co;
+        o[i][1] *= co;
+      }
+    }
+    if (row0 + 8 < nq) {
+      const float2 ml = *reinterpret_cast<const float2*>(pp1 + D);
+      const float M = fmaxf(m1, ml.x);
+      const float co = exp2f(m1 - M);
+      cp1 = exp2f(ml.x - M);
+      l1 = l1 * co + ml.y * cp1;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        o[i][2] *= co;
+        o[i][3] *= co;
+      }
+    }
+  }
+  // normalise, store bf16
   const float i0 = l0 > 0.f ? 1.f / l0 : 0.f, i1 = l1 > 0.f ? 1.f / l1 : 0.f;
   bf16* O = reinterpret_cast<bf16*>(a.O);
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
     const int col = h * D + i * 8 + tg * 2;
     if (row0 < nq) {
-      const long long r = (long long)g * a.q_len + q0 + row0;
-      *reinterpret_cast<uint32_t*>(O + r * a.o_ld + col) = pack_bf16(o[i][0] * i0, o[i][1] * i0);
+      float x = o[i][0], y = o[i][1];
+      if constexpr (SEG == SEG_OWN) {
+        const float2 pa = *reinterpret_cast<const float2*>(pp0 + i * 8 + tg * 2);
+        x += pa.x * cp0;
+        y += pa.y * cp0;
+      }
+      *reinterpret_cast<uint32_t*>(O + fr0 * a.o_ld + col) = pack_bf16(x * i0, y * i0);
     }
     if (row0 + 8 < nq) {
-      const long long r = (long long)g * a.q_len + q0 + row0 + 8;
-      *reinterpret_cast<uint32_t*>(O + r * a.o_ld + col) = pack_bf16(o[i][2] * i1, o[i][3] * i1);
+      float x = o[i][2], y = o[i][3];
+      if constexpr (SEG == SEG_OWN) {
+        const float2 pa = *reinterpret_cast<const float2*>(pp1 + i * 8 + tg * 2);
+        x += pa.x * cp1;
+        y += pa.y * cp1;
+      }
+      *reinterpret_cast<uint32_t*>(O + fr1 * a.o_ld + col) = pack_bf16(x * i1, y * i1);
     }
   }
 }
@@ -1072,11 +1153,26 @@ bool launch_attn_decode(int dt, const AttnArgs& a, float* part, size_t part_byte
   return true;
 }
 
+size_t attn_prefix_split_bytes(const AttnArgs& a) {
+  return (size_t)a.G * a.q_len * a.H * (a.dh + 2) * sizeof(float);
+}
+
+bool launch_attn_prefix_split(int dt, const AttnArgs& a, float* part, size_t part_bytes, cudaStream_t s) {
+  if (a.G <= 0 || a.q_len <= 0) return true;
+  if (!(dt == DT_BF16 && a.dh == 64 && a.Kp != nullptr && a.n_pre > 0 && a.q_ld % 8 == 0 &&
+        a.o_ld % 2 == 0 && !tc_attn_disabled() && part != nullptr && part_bytes >= attn_prefix_split_bytes(a)))
+    return false;
+  const long long rows = (long long)a.G * a.q_len;
+  launch_kernel(k_attn_prefill_mma<SEG_PREFIX>, dim3((unsigned)((rows + 63) / 64), a.H, 1), 128, 0, s, a, part);
+  launch_kernel(k_attn_prefill_mma<SEG_OWN>, dim3((a.q_len + 63) / 64, a.H, a.G), 128, 0, s, a, part);
+  return true;
+}
+
 void launch_attn_prefill(int dt, const AttnArgs& a, cudaStream_t s) {
   if (a.G <= 0 || a.q_len <= 0) return;
   if (dt == DT_BF16 && a.dh == 64 && a.q_ld % 8 == 0 && a.o_ld % 2 == 0 && !tc_attn_disabled()) {
     dim3 g64((a.q_len + 63) / 64, a.H, a.G);
-    launch_kernel(k_attn_prefill_mma, g64, 128, 0, s, a);
+    launch_kernel(k_attn_prefill_mma<SEG_ALL>, g64, 128, 0, s, a, (float*)nullptr);
     return;
   }
   dim3 grid((a.q_len + 31) / 32, a.H, a.G);

@@ -234,6 +234,12 @@ bool launch_attn_decode(int dt, const AttnArgs& a, float* part, size_t part_byte
                         cudaStream_t s);
 // Causal attention for many new queries per group (prefill).
 void launch_attn_prefill(int dt, const AttnArgs& a, cudaStream_t s);
+// Attention with a shared prefix as two passes (bf16, dh = 64): all query
+// rows against the prefix rows, then each group's own causal keys merged
+// with that partial.  part holds attn_prefix_split_bytes(a).  Returns false
+// (nothing launched) when the shape or the scratch does not fit.
+size_t attn_prefix_split_bytes(const AttnArgs& a);
+bool launch_attn_prefix_split(int dt, const AttnArgs& a, float* part, size_t part_bytes, cudaStream_t s);
 
 // ---- error message of the calling thread (read by photon_last_error) ----
 void set_error_message(const char* msg);

@@ -304,6 +304,8 @@ struct Bufs {
   void* sn_x = nullptr;    // split RMSNorm: bf16(x * g) for the next projection
   float* sn_ss = nullptr;  // ... and its per-row partial sums of squares
   int sn_cap = 0;          // floats per row in sn_ss
+  float* pre_ws = nullptr;  // shared-prefix attention: the prefix pass's partials
+  size_t pre_ws_bytes = 0;
 };
 
 struct photon_cache {
@@ -355,6 +357,8 @@ struct photon_cache {
   int stk_cnt_len = 0;
   float* attn_ws = nullptr;
   size_t attn_ws_bytes = 0;
+  float* pre_ws = nullptr;       // shared-prefix attention partials (caches built on a prefix)
+  size_t pre_ws_bytes = 0;
   int* d_err = nullptr;
   int* d_pos = nullptr;          // device {N, N1, chunks generated, 0} read by the decode kernels
   float samp_inv_t = 0.f;        // token sampling: 1 / temperature (0: greedy)
@@ -418,6 +422,16 @@ struct StackRun {
 
 static void gemm(photon_model* m, const Bufs& b, const void* A, long long lda, const void* W,
                  long long ldw, int M, int N, int K, const Epilogue& ep, cudaStream_t s);
+
+// Shared-prefix attention in two passes (PHOTON_PREFIX_SPLIT=0: one pass per
+// (group, head) over prefix and own keys together).
+static bool prefix_split_enabled() {
+  static const bool on = [] {
+    const char* e = getenv("PHOTON_PREFIX_SPLIT");
+    return !(e && e[0] == '0');
+  }();
+  return on;
+}
 
 static bool split_norm_enabled() {
   static const bool on = [] {
@@ -567,7 +581,10 @@ static void run_block(photon_model* m, const BlockW& w, float* x, const StackRun
   a.p0_dev = r.p0_dev;
   a.n_plan = r.n_plan;
   bool done = false;
-  if (r.q_len <= 4) done = launch_attn_decode(m->dt, a, b.attn_ws, b.attn_ws_bytes, b.err, s);
+  // with a shared prefix: the prefix once for all queries, then each group's own keys
+  if (r.kp && b.pre_ws && prefix_split_enabled())
+    done = launch_attn_prefix_split(m->dt, a, b.pre_ws, b.pre_ws_bytes, s);
+  if (!done && r.q_len <= 4) done = launch_attn_decode(m->dt, a, b.attn_ws, b.attn_ws_bytes, b.err, s);
   if (!done) launch_attn_prefill(m->dt, a, s);
 
   Epilogue eo = epi(EPI_ADD_F32, x, d);
@@ -668,6 +685,8 @@ static Bufs decode_bufs(photon_cache* c) {
   b.sn_x = c->sn_x;
   b.sn_ss = c->sn_ss;
   b.sn_cap = c->sn_x ? kSsqCap : 0;
+  b.pre_ws = c->pre_ws;
+  b.pre_ws_bytes = c->pre_ws_bytes;
   return b;
 }
 
@@ -895,6 +914,15 @@ int photon_prefill(photon_model* m, const photon_cache* prefix, const int32_t* d
     aw = std::max(aw, attn_ws_need(m->dt, rows_g, m->H, m->dh, i == 0 ? C1 : 1, C1 + i));
   c->attn_ws_bytes = aw;
   c->attn_ws = al.get<float>(aw);
+  if (prefix) {  // top step (1 query) and HierGen's level-1 re-encode (C2 queries) per sequence
+    AttnArgs pa;
+    pa.G = B;
+    pa.q_len = C2;
+    pa.H = m->H;
+    pa.dh = m->dh;
+    c->pre_ws_bytes = attn_prefix_split_bytes(pa);
+    c->pre_ws = al.get<float>(c->pre_ws_bytes);
+  }
   // top-encoder branch (B rows) of RecGen, run concurrently with the token decoder
   c->xn_t = al.get<void>((size_t)B * d * es);
   c->q_t = al.get<void>((size_t)B * d * es);
@@ -948,11 +976,24 @@ int photon_prefill(photon_model* m, const photon_cache* prefix, const int32_t* d
   pgw = std::max(pgw, gemm_ws_need(m, (int)rows1, d, C1 * d));
   pgw = std::max(pgw, gemm_ws_need(m, (int)rows2, d, C2 * d));
   float* pws = at.get<float>(pgw);
+  size_t ppb = 0;
+  float* ppw = nullptr;
+  if (prefix) {  // the level-1 stack has the most query rows
+    AttnArgs pa;
+    pa.G = B;
+    pa.q_len = N1_own;
+    pa.H = m->H;
+    pa.dh = m->dh;
+    ppb = attn_prefix_split_bytes(pa);
+    ppw = at.get<float>(ppb);
+  }
   if (at.err != cudaSuccess) {
     free_list(tmp, s);
     return bail(PHOTON_ERR_OOM);
   }
   Bufs pb{xn, q, att, hid, c->rope, pws, pgw, c->gemm_cnt, nullptr, 0, c->d_err};
+  pb.pre_ws = ppw;
+  pb.pre_ws_bytes = ppb;
 
   // a1: embedding; a2: Chunker_1 (concatenate C1 states, linear C1*d -> d)
   launch_embed(m->dt, d_tokens, m->ptr(m->i_embed), emb, (int)rows0, d, m->V, c->d_err, s);
