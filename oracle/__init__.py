@@ -15,6 +15,9 @@ Contents:
                 following the PHOTON pages step by step.
   sampling.py -- temperature sampling by the Gumbel-max rule with a
                 counter-based generator (SplitMix64 + MurmurHash3 fmix32).
+  vanilla.py -- a vanilla token-level Transformer of the same width, the
+                baseline of the pages' TPM comparison, built from the same
+                pinned blocks.
 
 Every oracle function is pinned by CPU tests (tests/test_oracle_*.py) to
 facts that do not come from the oracle itself: published SplitMix64 test
