@@ -316,6 +316,14 @@ def run_gpu(args) -> None:
     torch.cuda.synchronize()
     samp_dec_ms = sev[0].elapsed_time(sev[1])
 
+    # ---- same-kernel baseline: a vanilla token-level Transformer of the same
+    # width and total depth over the same prompts (its KV covers every token)
+    van = None
+    van_ms = 0.0
+    if not prefix_len and not args.no_vanilla and args.workload in ("c2", "c3"):
+        van = measure_vanilla(shape, toks, wl, stream)
+        van_ms = van.pop("_decode_ms")
+
     # ---- the decode's dominant kernel (its GEMM launches) and its attention,
     # alone, at the same shapes and launch configuration
     roof = measure_gemm_roofline(model, wl, dev, stream)
@@ -328,8 +336,8 @@ def run_gpu(args) -> None:
     if pre_cache is not None:
         pre_cache.free()
 
-    total_ms, prefill_ms, decode_ms, e2e_ms, hier_dec_ms, samp_dec_ms = max_over_ranks(
-        [total_ms, prefill_ms, decode_ms, e2e_ms, hier_dec_ms, samp_dec_ms], device=dev)
+    total_ms, prefill_ms, decode_ms, e2e_ms, hier_dec_ms, samp_dec_ms, van_ms = max_over_ranks(
+        [total_ms, prefill_ms, decode_ms, e2e_ms, hier_dec_ms, samp_dec_ms, van_ms], device=dev)
 
     dec_tokens = world * B * chunks * C * args.steps
     value = job_throughput(B * chunks * C * args.steps, world, decode_ms)
@@ -369,6 +377,7 @@ def run_gpu(args) -> None:
                     "resident_gib": round(hier_res / 2 ** 30, 4),
                     "tok_s_per_gib": round(B * chunks * C / (hier_dec_ms / 1e3) / (hier_res / 2 ** 30), 1),
                     "steps": 1},
+        "vanilla_baseline": vanilla_line(van, van_ms, world, value / world / gib) if van else None,
         "recgen_sampled": {"temperature": 1.0,
                            "decode_tok_s": round(job_throughput(B * chunks * C, world, samp_dec_ms), 1),
                            "decode_ms_per_chunk": round(samp_dec_ms / chunks, 4), "steps": 1},
@@ -432,6 +441,54 @@ def _with_traffic(roof: dict, key: str) -> dict:
 def _peak_gbs():
     peaks, src = _peaks()
     return peaks["hbm_gbs"], src
+
+
+def measure_vanilla(shape, toks, wl, stream) -> dict:
+    """The same prompts through a vanilla Transformer of the same width and
+    total depth (L1 + Ltop + Ld1 + Ld2 blocks) on the same kernels: prefill
+    of the first T-1 tokens, then one token per sequence per step for the
+    workload's decode length; the steps after the first (which captures the
+    step's graph) are timed.  Its prefill (one untimed pass, including the
+    first-use allocation of its KV cache) is not reported."""
+    import torch
+    import hierarchical_autoregressive_lm_b200 as hal
+    vshape = dict(vocab=shape["vocab"], d_model=shape["d_model"], n_heads=shape["n_heads"],
+                  head_dim=shape["head_dim"], layers=shape["L1"] + shape["Ltop"] + shape["Ld1"] + shape["Ld2"],
+                  mlp_mult=shape["mlp_mult"], dtype=shape["dtype"], init_std=shape["init_std"],
+                  rope_theta=shape["rope_theta"], norm_eps=shape["norm_eps"])
+    B, T = toks.shape
+    n = wl["decode_tokens"]
+    vm = hal.VanillaModel(vshape, WEIGHT_SEED)
+    out = torch.empty(B, dtype=torch.int32, device=toks.device)
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+    torch.cuda.synchronize()
+    ev[0].record(stream)
+    c = vm.prefill(toks, n)
+    ev[1].record(stream)
+    c.decode_step(out)
+    ev[2].record(stream)
+    for _ in range(n - 1):
+        c.decode_step(out)
+    ev[3].record(stream)
+    torch.cuda.synchronize()
+    info, minfo = c.info(), vm.info()
+    c.free()
+    vm.free()
+    resident = minfo["resident_bytes"] + info["kv_bytes"]
+    return {"model": f"vanilla Transformer, {vshape['layers']} layers, d={vshape['d_model']}, "
+                     f"{vshape['n_heads']}x{vshape['head_dim']} heads, vocab {vshape['vocab']}, {vshape['dtype']}",
+            "params_m": round(minfo["param_count"] / 1e6, 1),
+            "resident_gib": round(resident / 2 ** 30, 3), "kv_gib": round(info["kv_bytes"] / 2 ** 30, 3),
+            "graph_steps": info["graph_steps"], "tokens": B * (n - 1), "steps": n - 1,
+            "_decode_ms": ev[2].elapsed_time(ev[3])}
+
+
+def vanilla_line(van: dict, van_ms: float, world: int, photon_tpm: float) -> dict:
+    """The baseline's decode throughput (whole job), per GiB, and PHOTON's TPM over it."""
+    tok_s = world * van["tokens"] / (van_ms / 1e3)
+    tpm = tok_s / world / van["resident_gib"]
+    return dict(van, decode_tok_s=round(tok_s, 1), decode_ms_per_step=round(van_ms / van["steps"], 3),
+                tok_s_per_gib=round(tpm, 1), photon_over_vanilla_tpm=round(photon_tpm / tpm, 1))
 
 
 def measure_gemm_roofline(model, wl, dev, stream) -> dict:
@@ -684,6 +741,8 @@ def main() -> None:
     ap.add_argument("--impl", default="photon", choices=["photon", "reference"])
     ap.add_argument("--cpu-budget", type=float, default=20.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-vanilla", action="store_true",
+                    help="skip the same-kernel vanilla Transformer baseline")
     ap.add_argument("--decode-api", default="chunks", choices=["chunks", "steps"],
                     help="RecGen decode through one multi-chunk call (default) or per-chunk calls")
     ap.add_argument("--only-roofline", action="store_true",

@@ -32,8 +32,9 @@ EXPORTED = ("photon_init_weights", "photon_free_model", "photon_prefill",
             "photon_decode_rec_chunks",
             "photon_free_cache", "photon_cache_set_sampling", "photon_cache_info", "photon_model_info",
             "photon_export_weight", "photon_export_state", "photon_gemm", "photon_gemm_rmsnorm",
-            "photon_attn_decode", "photon_attn_decode_noalloc", "photon_launch_count",
-            "photon_last_error")
+            "photon_attn_decode", "photon_attn_decode_noalloc", "photon_vanilla_init",
+            "photon_vanilla_prefill", "photon_vanilla_decode_step", "photon_vanilla_cache_info",
+            "photon_vanilla_free_cache", "photon_launch_count", "photon_last_error")
 
 
 class PhotonError(RuntimeError):
@@ -67,6 +68,18 @@ class photon_model_stats(ctypes.Structure):
                 ("tcgen05_gemm", ctypes.c_int32)]
 
 
+class photon_vanilla_config(ctypes.Structure):
+    _fields_ = [("vocab", ctypes.c_int32), ("d_model", ctypes.c_int32), ("n_heads", ctypes.c_int32),
+                ("head_dim", ctypes.c_int32), ("layers", ctypes.c_int32), ("mlp_mult", ctypes.c_int32),
+                ("dtype", ctypes.c_int32), ("init_std", ctypes.c_float), ("rope_theta", ctypes.c_float),
+                ("norm_eps", ctypes.c_float)]
+
+
+class photon_vanilla_stats(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_int32) for n in ("B", "N", "capacity", "steps", "device_error", "graph_steps")] + \
+               [("kv_bytes", ctypes.c_uint64), ("workspace_bytes", ctypes.c_uint64)]
+
+
 _lib: Optional[ctypes.CDLL] = None
 
 
@@ -90,6 +103,11 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "photon_decode_rec_chunks": [P, P, I32, P, P],
         "photon_free_cache": [P],
         "photon_cache_set_sampling": [P, ctypes.c_float, U64],
+        "photon_vanilla_init": [ctypes.POINTER(photon_vanilla_config), U64, ctypes.POINTER(P)],
+        "photon_vanilla_prefill": [P, P, I32, I32, I32, P, ctypes.POINTER(P)],
+        "photon_vanilla_decode_step": [P, P, P, P, P, P],
+        "photon_vanilla_cache_info": [P, ctypes.POINTER(photon_vanilla_stats)],
+        "photon_vanilla_free_cache": [P],
         "photon_cache_info": [P, ctypes.POINTER(photon_cache_stats)],
         "photon_model_info": [P, ctypes.POINTER(photon_model_stats)],
         "photon_export_weight": [P, I32, P, SZ, ctypes.POINTER(SZ), P],
@@ -250,6 +268,65 @@ class Cache:
     def free(self) -> None:
         if self._h:
             _check(load_library().photon_free_cache(self._h))
+            self._h = None
+
+
+class VanillaModel(Model):
+    """Same-kernel baseline: a vanilla token-level Transformer (include/photon.h).
+
+    shape keys: vocab, d_model, n_heads, head_dim, layers, mlp_mult, dtype,
+    init_std, rope_theta, norm_eps."""
+
+    def __init__(self, shape: dict, seed: int):
+        L = load_library()
+        self.shape = dict(shape)
+        c = photon_vanilla_config()
+        c.vocab, c.d_model = shape["vocab"], shape["d_model"]
+        c.n_heads, c.head_dim, c.layers = shape["n_heads"], shape["head_dim"], shape["layers"]
+        c.mlp_mult = shape.get("mlp_mult", 4)
+        c.dtype = _DTYPES[shape["dtype"]]
+        c.init_std = shape.get("init_std", 0.02)
+        c.rope_theta = shape.get("rope_theta", 10000.0)
+        c.norm_eps = shape.get("norm_eps", 1e-6)
+        self.vcfg = c
+        h = ctypes.c_void_p()
+        _check(L.photon_vanilla_init(ctypes.byref(c), seed, ctypes.byref(h)))
+        self._h = h
+        self.vocab, self.d_model = shape["vocab"], shape["d_model"]
+
+    @property
+    def torch_dtype(self):
+        import torch
+        return torch.float32 if self.vcfg.dtype == 0 else torch.bfloat16
+
+    def prefill(self, tokens, max_new_tokens: int, stream=None) -> "VanillaCache":
+        """tokens: CUDA int32 [B, T]; the first T-1 enter the KV cache."""
+        B, T = tokens.shape
+        h = ctypes.c_void_p()
+        _check(load_library().photon_vanilla_prefill(self._h, _ptr(tokens), B, T, max_new_tokens,
+                                                     _stream(stream), ctypes.byref(h)))
+        return VanillaCache(self, h, B)
+
+
+class VanillaCache:
+    def __init__(self, model: VanillaModel, handle, B: int):
+        self.model, self._h, self.B = model, handle, B
+
+    def decode_step(self, out_tokens, out_logits=None, force_tokens=None, stream=None) -> None:
+        """One token per sequence: out_tokens CUDA int32 [B]; optional fp32 logits [B, vocab];
+        optional teacher-forced tokens [B] (entries < 0 not forced)."""
+        _check(load_library().photon_vanilla_decode_step(self.model._h, self._h, _ptr(out_tokens),
+                                                         _ptr(out_logits), _ptr(force_tokens),
+                                                         _stream(stream)))
+
+    def info(self) -> dict:
+        st = photon_vanilla_stats()
+        _check(load_library().photon_vanilla_cache_info(self._h, ctypes.byref(st)))
+        return {n: getattr(st, n) for n, _ in st._fields_}
+
+    def free(self) -> None:
+        if self._h:
+            _check(load_library().photon_vanilla_free_cache(self._h))
             self._h = None
 
 

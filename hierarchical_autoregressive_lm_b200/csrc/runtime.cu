@@ -82,6 +82,11 @@ struct photon_model {
   size_t es;
   uint64_t seed;
   int d, H, dh, V, C1, C2, C, f, L1, Ltop, Ld1, Ld2;
+  // same-kernel baseline: a vanilla token-level Transformer (embed, L_van
+  // blocks from i_van, final gain i_van_g, head i_head) instead of PHOTON
+  bool vanilla = false;
+  int i_van = 0, L_van = 0, i_van_g = 0;
+  bool graph_failed_van = false;  // the vanilla step could not be captured
   std::vector<TensorRec> t;
   size_t group_bytes[G_COUNT] = {0, 0, 0, 0};
   char* group_ptr[G_COUNT] = {nullptr, nullptr, nullptr, nullptr};
@@ -653,7 +658,7 @@ static size_t attn_ws_need(int dt, int G, int H, int dh, int q_len, int n_plan) 
 }
 
 // cos/sin table: entry [pos][i] = (cos, sin)(pos * theta^(-2i/dh)), computed in fp64.
-static int upload_rope(photon_model* m, photon_cache* c, Allocator& al, int positions) {
+static int upload_rope(photon_model* m, float2** out, Allocator& al, int positions) {
   const int half = m->dh / 2;
   std::vector<float2> host((size_t)positions * half);
   for (int p = 0; p < positions; ++p)
@@ -662,10 +667,9 @@ static int upload_rope(photon_model* m, photon_cache* c, Allocator& al, int posi
       const double ang = (double)p * inv;
       host[(size_t)p * half + i] = make_float2((float)std::cos(ang), (float)std::sin(ang));
     }
-  c->rope = al.get<float2>(host.size() * sizeof(float2));
-  if (!c->rope) return PHOTON_ERR_OOM;
-  CK(cudaMemcpyAsync(c->rope, host.data(), host.size() * sizeof(float2), cudaMemcpyHostToDevice,
-                     al.s));
+  *out = al.get<float2>(host.size() * sizeof(float2));
+  if (!*out) return PHOTON_ERR_OOM;
+  CK(cudaMemcpyAsync(*out, host.data(), host.size() * sizeof(float2), cudaMemcpyHostToDevice, al.s));
   return PHOTON_OK;
 }
 
@@ -807,6 +811,7 @@ int photon_prefill(photon_model* m, const photon_cache* prefix, const int32_t* d
   g_err.clear();
   if (!m || !out) return fail(PHOTON_ERR_ARG, "NULL model or out");
   *out = nullptr;
+  if (m->vanilla) return fail(PHOTON_ERR_ARG, "a vanilla baseline model takes the photon_vanilla_* calls");
   if (!d_tokens) return fail(PHOTON_ERR_ARG, "tokens pointer is NULL");
   if (B <= 0) return fail(PHOTON_ERR_ARG, "batch must be positive");
   if (T <= 0 || T % m->C) return fail(PHOTON_ERR_ARG, "T = %d is not a positive multiple of C1*C2 = %d", T, m->C);
@@ -953,7 +958,7 @@ int photon_prefill(photon_model* m, const photon_cache* prefix, const int32_t* d
     return bail(fail(PHOTON_ERR_CUDA, "stream/event creation failed"));
   const int positions =
       std::max(std::max(c->n_pre + c->Ncap, c->n1_pre + N1_own + C2 * max_new_chunks), 2 * C1 + C2) + 1;
-  rc = upload_rope(m, c, al, positions);
+  rc = upload_rope(m, &c->rope, al, positions);
   if (al.err != cudaSuccess || rc) return bail(PHOTON_ERR_OOM);
   if (cudaMemsetAsync(c->d_err, 0, 16, s) != cudaSuccess ||
       cudaMemsetAsync(c->gemm_cnt, 0, kGemmTileCounters * sizeof(int), s) != cudaSuccess ||
@@ -1894,6 +1899,381 @@ int photon_attn_decode(int32_t dtype, const void* d_q, const void* d_k, const vo
   if (ws) cudaFreeAsync(ws, s);
   if (!ok) return fail(PHOTON_ERR_ARG, "decode attention rejected the shape");
   CK(cudaGetLastError());
+  return PHOTON_OK;
+}
+
+}  // extern "C"
+
+// ============================================================== vanilla baseline
+// A vanilla token-level Transformer of PHOTON's width on the same kernels:
+// the baseline of the pages' throughput-per-memory comparison (explainer,
+// 475x section).  It is a photon_model with its own tensor list (embed,
+// L_van blocks, final gain, head), so weight generation, export, the block
+// stack and the GEMM/attention dispatch are shared.
+
+static void build_specs_vanilla(photon_model* m) {
+  const long long d = m->d, V = m->V, f = m->f;
+  auto add = [&](const std::string& n, int g, long long numel, bool gain) {
+    m->t.push_back(TensorRec{n, g, 0, numel, gain});
+  };
+  m->i_embed = (int)m->t.size();
+  add("embed", G_EMB, V * d, false);
+  m->i_van = (int)m->t.size();
+  for (int l = 0; l < m->L_van; ++l) {  // the layout BlockW expects (wq, wk, wv back to back)
+    const std::string p = "van." + std::to_string(l) + ".";
+    add(p + "g_attn", G_TOP, d, true);
+    add(p + "wq", G_TOP, d * d, false);
+    add(p + "wk", G_TOP, d * d, false);
+    add(p + "wv", G_TOP, d * d, false);
+    add(p + "wo", G_TOP, d * d, false);
+    add(p + "g_mlp", G_TOP, d, true);
+    add(p + "w1", G_TOP, f * d, false);
+    add(p + "w2", G_TOP, d * f, false);
+  }
+  m->i_van_g = (int)m->t.size();
+  add("van.g_final", G_TOP, d, true);
+  m->i_head = (int)m->t.size();
+  add("head", G_DEC, V * d, false);
+  for (auto& r : m->t) {
+    const size_t bytes = (size_t)r.numel * (r.gain ? 4 : m->es);
+    r.offset = m->group_bytes[r.group];
+    m->group_bytes[r.group] += (bytes + 255) & ~size_t(255);
+  }
+}
+
+struct photon_vanilla_cache {
+  photon_model* m = nullptr;
+  int B = 0, T = 0, N = 0, cap = 0, max_new = 0, steps = 0, graph_steps = 0;
+  cudaStream_t stream = nullptr;
+  cudaStream_t cap_s = nullptr;  // capture stream: only ever captured into
+  std::vector<void*> allocs;
+  size_t kv_bytes = 0, ws_bytes = 0;
+  char* kc = nullptr;
+  char* vc = nullptr;
+  size_t layer_bytes = 0;  // [B][H][cap][dh] per layer
+  float2* rope = nullptr;
+  float* x = nullptr;
+  void *xn = nullptr, *q = nullptr, *att = nullptr, *hid = nullptr, *hn = nullptr;
+  float* gemm_ws = nullptr;
+  size_t gemm_ws_bytes = 0;
+  int* gemm_cnt = nullptr;
+  float* attn_ws = nullptr;
+  size_t attn_ws_bytes = 0;
+  void* sn_x = nullptr;
+  float* sn_ss = nullptr;
+  unsigned long long* amax_part = nullptr;
+  int amax_tiles = 0;
+  float* logits = nullptr;     // head output when the argmax is not fused
+  int32_t* next_ids = nullptr; // [B] the token the next step feeds
+  int32_t* tok_out = nullptr;  // [B] choices of graph-replayed steps
+  int* d_err = nullptr;
+  int* d_pos = nullptr;        // {position of the next fed token, 0}
+};
+
+static Bufs vanilla_bufs(photon_vanilla_cache* c) {
+  Bufs b{c->xn, c->q, c->att, c->hid, c->rope, c->gemm_ws, c->gemm_ws_bytes, c->gemm_cnt, c->attn_ws,
+         c->attn_ws_bytes, c->d_err};
+  b.sn_x = c->sn_x;
+  b.sn_ss = c->sn_ss;
+  b.sn_cap = c->sn_x ? kSsqCap : 0;
+  return b;
+}
+
+// One decode step: embed the pending token, run the stack at the next
+// position (appending its KV), final norm, head and greedy choice.
+static void enqueue_vanilla(photon_model* m, photon_vanilla_cache* c, int32_t* out, float* logits,
+                            const int32_t* force, cudaStream_t s) {
+  const int B = c->B, d = m->d, V = m->V;
+  Bufs b = vanilla_bufs(c);
+  launch_embed_f32(m->dt, c->next_ids, m->ptr(m->i_embed), c->x, B, d, V, c->d_err, s);
+  StackRun r;
+  r.G = B;
+  r.q_len = 1;
+  r.kc = c->kc;
+  r.vc = c->vc;
+  r.layer_bytes = c->layer_bytes;
+  r.cap = c->cap;
+  r.p0_dev = c->d_pos;
+  r.n_plan = c->cap;
+  r.sn_rows = c->sn_x ? B : 0;
+  run_stack(m, m->i_van, m->L_van, c->x, r, b, s);
+  launch_rmsnorm(m->dt, c->x, (const float*)m->ptr(m->i_van_g), c->hn, B, d, 1, 0, m->cfg.norm_eps, s);
+  if (c->amax_tiles > 0 && !logits) {
+    Epilogue e = epi(EPI_ARGMAX, nullptr, V);
+    e.argmax_part = c->amax_part;
+    e.argmax_tiles = c->amax_tiles;
+    gemm(m, b, c->hn, d, m->ptr(m->i_head), d, B, V, d, e, s);
+    launch_argmax_partials(c->amax_part, c->amax_tiles, B, V, 0, 1, force, out, nullptr, c->next_ids,
+                           c->d_err, nullptr, s);
+  } else {
+    float* lg = logits ? logits : c->logits;
+    gemm(m, b, c->hn, d, m->ptr(m->i_head), d, B, V, d, epi(EPI_STORE_F32, lg, V), s);
+    launch_argmax(lg, V, B, V, 0, 1, force, out, nullptr, c->next_ids, c->d_err, SampleArgs{}, s);
+  }
+  launch_advance(c->d_pos, 1, 0, s);
+}
+
+extern "C" {
+
+int photon_vanilla_init(const photon_vanilla_config* cfg, uint64_t seed, photon_model** out) {
+  g_err.clear();
+  if (!out) return fail(PHOTON_ERR_ARG, "out is NULL");
+  *out = nullptr;
+  if (!cfg) return fail(PHOTON_ERR_ARG, "config is NULL");
+  if (cfg->vocab <= 0 || cfg->d_model <= 0 || cfg->n_heads <= 0 || cfg->head_dim <= 0 || cfg->layers < 1 ||
+      cfg->mlp_mult < 1)
+    return fail(PHOTON_ERR_ARG, "non-positive model dimension");
+  // the shared checks of the PHOTON config, on an equivalent one
+  photon_config pc = {};
+  pc.vocab = cfg->vocab;
+  pc.d_model = cfg->d_model;
+  pc.n_heads = cfg->n_heads;
+  pc.head_dim = cfg->head_dim;
+  pc.levels = 2;
+  pc.chunk[0] = pc.chunk[1] = 1;
+  pc.enc_layers[0] = 1;
+  pc.enc_layers[1] = cfg->layers;
+  pc.dec_layers[0] = pc.dec_layers[1] = 1;
+  pc.mlp_mult = cfg->mlp_mult;
+  pc.dtype = cfg->dtype;
+  pc.init_std = cfg->init_std;
+  pc.rope_theta = cfg->rope_theta;
+  pc.norm_eps = cfg->norm_eps;
+  RET(check_config(&pc));
+  photon_model* m = new photon_model();
+  m->cfg = pc;
+  m->vanilla = true;
+  m->L_van = cfg->layers;
+  m->dt = cfg->dtype;
+  m->es = dtype_size(m->dt);
+  m->seed = seed;
+  m->d = cfg->d_model;
+  m->H = cfg->n_heads;
+  m->dh = cfg->head_dim;
+  m->V = cfg->vocab;
+  m->C1 = m->C2 = m->C = 1;
+  m->f = cfg->mlp_mult * cfg->d_model;
+  m->L1 = m->Ltop = m->Ld1 = m->Ld2 = 0;
+  m->use_tc = (m->dt == DT_BF16) && tma_available();
+  build_specs_vanilla(m);
+  for (int g = 0; g < G_COUNT; ++g) {
+    if (m->group_bytes[g] == 0) continue;
+    cudaError_t e = cudaMalloc((void**)&m->group_ptr[g], m->group_bytes[g]);
+    if (e != cudaSuccess) {
+      cudaGetLastError();
+      for (int k = 0; k < g; ++k)
+        if (m->group_ptr[k]) cudaFree(m->group_ptr[k]);
+      delete m;
+      return fail(e == cudaErrorMemoryAllocation ? PHOTON_ERR_OOM : PHOTON_ERR_CUDA,
+                  "weight allocation failed: %s", cudaGetErrorString(e));
+    }
+    generate_group(m, g, nullptr);
+  }
+  cudaError_t e = cudaStreamSynchronize(nullptr);
+  if (e == cudaSuccess) e = cudaGetLastError();
+  if (e != cudaSuccess) {
+    for (int g = 0; g < G_COUNT; ++g)
+      if (m->group_ptr[g]) cudaFree(m->group_ptr[g]);
+    delete m;
+    return fail(PHOTON_ERR_CUDA, "weight generation failed: %s", cudaGetErrorString(e));
+  }
+  *out = m;
+  return PHOTON_OK;
+}
+
+int photon_vanilla_prefill(photon_model* m, const int32_t* d_tokens, int32_t B, int32_t T,
+                           int32_t max_new_tokens, void* stream, photon_vanilla_cache** out) {
+  g_err.clear();
+  if (!m || !out) return fail(PHOTON_ERR_ARG, "NULL model or out");
+  *out = nullptr;
+  if (!m->vanilla) return fail(PHOTON_ERR_ARG, "not a vanilla baseline model");
+  if (!d_tokens) return fail(PHOTON_ERR_ARG, "tokens pointer is NULL");
+  if (B <= 0 || T < 2 || max_new_tokens < 0) return fail(PHOTON_ERR_ARG, "need B > 0, T >= 2, max_new >= 0");
+  cudaStream_t s = (cudaStream_t)stream;
+  const int d = m->d, V = m->V, H = m->H, dh = m->dh, L = m->L_van;
+  const size_t es = m->es;
+  photon_vanilla_cache* c = new photon_vanilla_cache();
+  c->m = m;
+  c->B = B;
+  c->T = T;
+  c->N = T - 1;
+  c->cap = T - 1 + max_new_tokens;
+  c->max_new = max_new_tokens;
+  c->stream = s;
+  Allocator al{s, &c->allocs, &c->kv_bytes};
+  Allocator aw{s, &c->allocs, &c->ws_bytes};
+  auto bail = [&](int code) {
+    cudaGetLastError();
+    if (c->cap_s) cudaStreamDestroy(c->cap_s);
+    free_list(c->allocs, s);
+    cudaStreamSynchronize(s);
+    delete c;
+    return code == PHOTON_ERR_OOM ? fail(code, "device allocation failed during prefill") : code;
+  };
+  c->layer_bytes = (size_t)B * H * c->cap * dh * es;
+  c->kc = al.get<char>(c->layer_bytes * L);
+  c->vc = al.get<char>(c->layer_bytes * L);
+  if (upload_rope(m, &c->rope, aw, c->cap) != PHOTON_OK) return bail(PHOTON_ERR_OOM);
+  c->x = aw.get<float>((size_t)B * d * 4);
+  c->xn = aw.get<void>((size_t)B * d * es);
+  c->q = aw.get<void>((size_t)B * d * es);
+  c->att = aw.get<void>((size_t)B * d * es);
+  c->hn = aw.get<void>((size_t)B * d * es);
+  c->hid = aw.get<void>((size_t)B * m->f * es);
+  c->gemm_ws_bytes = std::max(block_ws_need(m, B), gemm_ws_need(m, B, V, d));
+  c->gemm_ws = aw.get<float>(c->gemm_ws_bytes);
+  c->gemm_cnt = aw.get<int>(kGemmTileCounters * sizeof(int));
+  c->attn_ws_bytes = attn_ws_need(m->dt, B, H, dh, 1, c->cap);
+  c->attn_ws = aw.get<float>(c->attn_ws_bytes);
+  c->amax_tiles = m->use_tc ? gemm_tc_argmax_tiles(B, V, d) : 0;
+  if (c->amax_tiles > 0)
+    c->amax_part = aw.get<unsigned long long>((size_t)B * c->amax_tiles * 8);
+  else
+    c->logits = aw.get<float>((size_t)B * V * 4);
+  if (m->use_tc && split_norm_enabled()) {
+    c->sn_x = aw.get<void>((size_t)B * d * es);
+    c->sn_ss = aw.get<float>((size_t)B * kSsqCap * sizeof(float));
+  }
+  c->next_ids = aw.get<int32_t>((size_t)B * 4);
+  c->tok_out = aw.get<int32_t>((size_t)B * 4);
+  c->d_err = aw.get<int>(16);
+  c->d_pos = aw.get<int>(16);
+  if (al.err != cudaSuccess || aw.err != cudaSuccess || !c->kc || !c->vc) return bail(PHOTON_ERR_OOM);
+  if (cudaStreamCreateWithFlags(&c->cap_s, cudaStreamNonBlocking) != cudaSuccess) c->cap_s = nullptr;
+  if (cudaMemsetAsync(c->d_err, 0, 16, s) != cudaSuccess ||
+      cudaMemsetAsync(c->gemm_cnt, 0, kGemmTileCounters * sizeof(int), s) != cudaSuccess)
+    return bail(PHOTON_ERR_CUDA);
+
+  // prefill of the first T-1 tokens (temporaries released at the end)
+  const long long rows = (long long)B * (T - 1);
+  std::vector<void*> tmp;
+  size_t tmp_bytes = 0;
+  Allocator at{s, &tmp, &tmp_bytes};
+  int32_t* ids = at.get<int32_t>((size_t)rows * 4);
+  float* x = at.get<float>((size_t)rows * d * 4);
+  void* xn = at.get<void>((size_t)rows * d * es);
+  void* q = at.get<void>((size_t)rows * d * es);
+  void* att = at.get<void>((size_t)rows * d * es);
+  void* hid = at.get<void>((size_t)rows * m->f * es);
+  const size_t pgw = block_ws_need(m, (int)rows);
+  float* pws = at.get<float>(pgw);
+  if (at.err != cudaSuccess) {
+    free_list(tmp, s);
+    return bail(PHOTON_ERR_OOM);
+  }
+  const size_t w_in = (size_t)T * sizeof(int32_t), w_pre = (size_t)(T - 1) * sizeof(int32_t);
+  const int pos[4] = {T - 1, 0, 0, 0};  // pageable source: staged before the call returns
+  if (cudaMemcpy2DAsync(ids, w_pre, d_tokens, w_in, w_pre, B, cudaMemcpyDeviceToDevice, s) != cudaSuccess ||
+      cudaMemcpy2DAsync(c->next_ids, sizeof(int32_t), d_tokens + (T - 1), w_in, sizeof(int32_t), B,
+                        cudaMemcpyDeviceToDevice, s) != cudaSuccess ||
+      cudaMemcpyAsync(c->d_pos, pos, sizeof(pos), cudaMemcpyHostToDevice, s) != cudaSuccess) {
+    free_list(tmp, s);
+    return bail(fail(PHOTON_ERR_CUDA, "token staging failed"));
+  }
+  launch_embed_f32(m->dt, ids, m->ptr(m->i_embed), x, (int)rows, d, V, c->d_err, s);
+  Bufs pb{xn, q, att, hid, c->rope, pws, pgw, c->gemm_cnt, nullptr, 0, c->d_err};
+  StackRun r;
+  r.G = B;
+  r.q_len = T - 1;
+  r.kc = c->kc;
+  r.vc = c->vc;
+  r.layer_bytes = c->layer_bytes;
+  r.cap = c->cap;
+  run_stack(m, m->i_van, L, x, r, pb, s);
+  cudaError_t le = cudaGetLastError();
+  free_list(tmp, s);
+  if (le != cudaSuccess) return bail(fail(PHOTON_ERR_CUDA, "prefill launch failed: %s", cudaGetErrorString(le)));
+  m->live_caches++;
+  *out = c;
+  return PHOTON_OK;
+}
+
+int photon_vanilla_decode_step(photon_model* m, photon_vanilla_cache* c, int32_t* d_out_tokens,
+                               float* d_out_logits, const int32_t* d_force_tokens, void* stream) {
+  g_err.clear();
+  if (!m || !c || c->m != m || !m->vanilla) return fail(PHOTON_ERR_ARG, "model/cache mismatch");
+  if (!d_out_tokens) return fail(PHOTON_ERR_ARG, "output token buffer is NULL");
+  if (c->steps >= c->max_new) return fail(PHOTON_ERR_CAPACITY, "cache is full (%d steps)", c->max_new);
+  cudaStream_t s = (cudaStream_t)stream;
+  c->stream = s;
+  // the plain step is captured once (on the cache's capture stream) and
+  // replayed; the model keeps the executable and updates it for new caches
+  const bool plain = !d_out_logits && !d_force_tokens;
+  bool replay = plain && c->cap_s != nullptr && graphs_enabled() && c->steps >= 1 && !m->graph_failed_van;
+  if (replay && m->graph_owner[0] != c) {
+    cudaGraph_t g = nullptr;
+    const unsigned long long n0 = launch_total();
+    bool ok = cudaStreamBeginCapture(c->cap_s, cudaStreamCaptureModeRelaxed) == cudaSuccess;
+    if (ok) {
+      enqueue_vanilla(m, c, c->tok_out, nullptr, nullptr, c->cap_s);
+      ok = cudaStreamEndCapture(c->cap_s, &g) == cudaSuccess && g;
+    }
+    const long long captured = (long long)(launch_total() - n0);
+    note_launch(-captured);
+    m->graph_kernels[0] = ok ? captured : 0;
+    if (ok && m->graph[0]) {
+      cudaGraphExecUpdateResultInfo info;
+      if (cudaGraphExecUpdate(m->graph[0], g, &info) != cudaSuccess) {
+        cudaGetLastError();
+        cudaGraphExecDestroy(m->graph[0]);
+        m->graph[0] = nullptr;
+      }
+    }
+    if (ok && !m->graph[0]) ok = cudaGraphInstantiate(&m->graph[0], g, 0) == cudaSuccess;
+    if (g) cudaGraphDestroy(g);
+    if (!ok) {
+      cudaGetLastError();
+      m->graph[0] = nullptr;
+      m->graph_owner[0] = nullptr;
+      m->graph_failed_van = true;
+      replay = false;
+    } else {
+      m->graph_owner[0] = c;
+    }
+  }
+  if (replay) {
+    CK(cudaGraphLaunch(m->graph[0], s));
+    note_launch(m->graph_kernels[0]);
+    c->graph_steps += 1;
+    if (d_out_tokens != c->tok_out)
+      CK(cudaMemcpyAsync(d_out_tokens, c->tok_out, (size_t)c->B * sizeof(int32_t), cudaMemcpyDeviceToDevice, s));
+  } else {
+    enqueue_vanilla(m, c, d_out_tokens, d_out_logits, d_force_tokens, s);
+  }
+  CK(cudaGetLastError());
+  c->N += 1;
+  c->steps += 1;
+  return PHOTON_OK;
+}
+
+int photon_vanilla_cache_info(photon_vanilla_cache* c, photon_vanilla_stats* out) {
+  g_err.clear();
+  if (!c || !out) return fail(PHOTON_ERR_ARG, "NULL argument");
+  memset(out, 0, sizeof(*out));
+  CK(cudaStreamSynchronize(c->stream));
+  int err = 0;
+  CK(cudaMemcpy(&err, c->d_err, sizeof(int), cudaMemcpyDeviceToHost));
+  out->B = c->B;
+  out->N = c->N;
+  out->capacity = c->cap;
+  out->steps = c->steps;
+  out->device_error = err;
+  out->graph_steps = c->graph_steps;
+  out->kv_bytes = c->kv_bytes;
+  out->workspace_bytes = c->ws_bytes;
+  return PHOTON_OK;
+}
+
+int photon_vanilla_free_cache(photon_vanilla_cache* c) {
+  g_err.clear();
+  if (!c) return fail(PHOTON_ERR_ARG, "cache is NULL");
+  photon_model* m = c->m;
+  if (m->graph_owner[0] == c) m->graph_owner[0] = nullptr;  // its buffers are going away
+  if (c->cap_s) cudaStreamDestroy(c->cap_s);                 // only ever captured into
+  free_list(c->allocs, c->stream);                             // stream-ordered
+  CK(cudaGetLastError());
+  m->live_caches--;
+  delete c;
   return PHOTON_OK;
 }
 

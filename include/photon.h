@@ -309,6 +309,71 @@ PHOTON_API int photon_attn_decode_noalloc(int32_t dtype, const void* d_q, const 
                                           int32_t cap, int32_t q_len, int32_t p0, void* d_o,
                                           void* stream);
 
+/* ------------------------------------------------------------------------
+ * Same-kernel baseline: a vanilla token-level Transformer.
+ *
+ * The explainer's decode-heavy table (475x section) compares PHOTON's
+ * throughput per memory with a vanilla Transformer of similar size.  This is
+ * that baseline built from the same kernels: one causal pre-norm stack over
+ * the token stream (PHOTON's block: RMSNorm, rotate-half RoPE per token
+ * position, full multi-head attention, erf-GELU MLP, no biases), a final
+ * RMSNorm and an untied head, with a KV cache over every token.  Weights use
+ * the same generator as photon_init_weights (tensor order: embed [V, d];
+ * per layer g_attn, Wq, Wk, Wv, Wo, g_mlp, W1, W2; final gain; head [V, d]),
+ * so photon_export_weight and photon_model_info work on it.  The PHOTON
+ * entry points reject a vanilla model and vice versa. */
+typedef struct photon_vanilla_cache photon_vanilla_cache; /* opaque, library-owned */
+
+typedef struct photon_vanilla_config {
+  int32_t vocab;
+  int32_t d_model;
+  int32_t n_heads;
+  int32_t head_dim;
+  int32_t layers;
+  int32_t mlp_mult;
+  int32_t dtype;   /* 0 fp32, 1 bf16 */
+  float init_std;
+  float rope_theta;
+  float norm_eps;
+} photon_vanilla_config;
+
+/* Model with weights drawn on the device.  Constraints as photon_init_weights
+ * (d_model == n_heads * head_dim, head_dim in {32, 64}, d_model % 64 == 0),
+ * layers >= 1.  Synchronising.  Errors: ERR_ARG, ERR_OOM, ERR_CUDA. */
+PHOTON_API int photon_vanilla_init(const photon_vanilla_config* cfg, uint64_t seed, photon_model** out);
+
+/* Prefill of B prompts d_tokens [B, T] (device, row-major, T >= 2): the
+ * first T-1 tokens of each prompt enter the KV cache; the last one is the
+ * input of the first decode step.  Room for max_new_tokens decode steps.
+ * Errors: ERR_ARG, ERR_OOM, ERR_CUDA. */
+PHOTON_API int photon_vanilla_prefill(photon_model* m, const int32_t* d_tokens, int32_t B, int32_t T,
+                                      int32_t max_new_tokens, void* stream, photon_vanilla_cache** out);
+
+/* One token per sequence: feeds the pending token (the last prompt token,
+ * then the previous step's choice, or d_force_tokens[b] if given and >= 0)
+ * at the next position and writes the greedy choice (lowest id on ties) to
+ * d_out_tokens [B].  d_out_logits (nullable) receives fp32 logits [B, V].
+ * Steps without logits or forcing replay a captured graph after the first.
+ * Errors: ERR_ARG, ERR_CAPACITY (more than max_new_tokens steps), ERR_CUDA. */
+PHOTON_API int photon_vanilla_decode_step(photon_model* m, photon_vanilla_cache* c, int32_t* d_out_tokens,
+                                          float* d_out_logits, const int32_t* d_force_tokens,
+                                          void* stream);
+
+typedef struct photon_vanilla_stats {
+  int32_t B, N;            /* sequences; positions in the KV cache */
+  int32_t capacity, steps; /* KV capacity; decode steps taken */
+  int32_t device_error;    /* device error word (0 = none) */
+  int32_t graph_steps;     /* decode steps replayed from the captured graph */
+  uint64_t kv_bytes;       /* KV cache bytes */
+  uint64_t workspace_bytes;
+} photon_vanilla_stats;
+
+/* Synchronises the cache's stream, then reports.  Errors: ERR_ARG, ERR_CUDA. */
+PHOTON_API int photon_vanilla_cache_info(photon_vanilla_cache* c, photon_vanilla_stats* out);
+
+/* Stream-ordered release (as photon_free_cache).  Errors: ERR_ARG, ERR_CUDA. */
+PHOTON_API int photon_vanilla_free_cache(photon_vanilla_cache* c);
+
 /* Number of kernels this library has launched in this process so far
  * (every launch of every entry point; host-side counter, no GPU access). */
 PHOTON_API uint64_t photon_launch_count(void);
