@@ -399,15 +399,16 @@ def run_gpu(args) -> None:
 
 
 def kernel_sources_sha256() -> str:
-    """sha256 over the relative path and bytes of every kernel source and
-    public header, sorted by path (the key under which profiled DRAM
-    traffic stays valid)."""
+    """sha256 over the relative path and bytes of the sources the three
+    roofline kernels are compiled from (their .cu files and every csrc
+    header), sorted by path: the key under which profiled DRAM traffic stays
+    valid.  Host-side orchestration (runtime.cu) and unrelated kernels do not
+    enter it."""
     import glob
     import hashlib
-    files = sorted(glob.glob(os.path.join(ROOT, "hierarchical_autoregressive_lm_b200", "csrc", "*.cu"))
-                   + glob.glob(os.path.join(ROOT, "hierarchical_autoregressive_lm_b200", "csrc", "*.cuh"))
-                   + glob.glob(os.path.join(ROOT, "hierarchical_autoregressive_lm_b200", "csrc", "*.h"))
-                   + glob.glob(os.path.join(ROOT, "include", "*.h")))
+    csrc = os.path.join(ROOT, "hierarchical_autoregressive_lm_b200", "csrc")
+    files = sorted([os.path.join(csrc, "k_gemm_tc.cu"), os.path.join(csrc, "k_attention.cu")]
+                   + glob.glob(os.path.join(csrc, "*.cuh")) + glob.glob(os.path.join(csrc, "*.h")))
     h = hashlib.sha256()
     for f in files:
         h.update(os.path.relpath(f, ROOT).encode())
