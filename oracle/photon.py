@@ -394,6 +394,38 @@ class PhotonOracle:
         st.steps += 1
         return StepResult(tokens=own, used=used, logits=logits, a_hat=a_hat, a=a, near_tie=tie)
 
+    # -- teacher-forced scoring -------------------------------------------------
+    def score(self, tokens):
+        """Log-probability of every token of chunks 1..N-1 of a prompt under
+        teacher forcing (explainer, quality section: the reported quality is
+        measured with teacher-forced HierGen).
+
+        The bottom-up pass encodes the true tokens; the top output o_k of
+        chunk k conditions chunk k+1 (R6); Decoder_2 and the token decoder
+        then read chunk k+1's true tokens as their inputs (R3, R4), so every
+        position's next-token distribution comes out at once.  The first
+        chunk has no top output before it and is not scored.  Returns
+        (log-probabilities [T - C], logits [T - C, V])."""
+        cfg, w = self.cfg, self.w
+        tokens = np.asarray(tokens, dtype=np.int64)
+        T = tokens.shape[0]
+        if T <= cfg.C or T % cfg.C:
+            raise ValueError("the prompt must be a multiple of C1*C2 longer than one chunk")
+        s1, _ = self.encode_level1(tokens, 0, None)
+        o_all, _ = self.top_encode(chunker(s1, w["chunker2"], cfg.C2), 0, None)
+        logits = []
+        for k in range(1, T // cfg.C):
+            a_hat = self.decode_chunk2(o_all[k - 1])
+            for j in range(cfg.C2):
+                cond = converter(a_hat[j], w["converter1"], cfg.C1)
+                base = k * cfg.C + j * cfg.C1
+                for i in range(cfg.C1):
+                    logits.append(self.token_decoder_logits(cond, [int(t) for t in tokens[base:base + i]]))
+        logits = np.stack(logits)
+        z = logits - logits.max(axis=1, keepdims=True)
+        logp = z - np.log(np.exp(z).sum(axis=1, keepdims=True))
+        return logp[np.arange(T - cfg.C), tokens[cfg.C:]], logits
+
     # -- full recomputation (used to pin the incremental paths) ---------------
     def full_hier(self, tokens: np.ndarray) -> SeqState:
         """HierGen state after all of `tokens`, computed from scratch."""
