@@ -32,7 +32,7 @@ EXPORTED = ("photon_init_weights", "photon_free_model", "photon_prefill",
             "photon_decode_rec_chunks",
             "photon_free_cache", "photon_cache_set_sampling", "photon_cache_info", "photon_model_info",
             "photon_export_weight", "photon_export_state", "photon_gemm", "photon_gemm_rmsnorm",
-            "photon_attn_decode", "photon_attn_decode_noalloc", "photon_vanilla_init",
+            "photon_attn_decode", "photon_attn_decode_noalloc", "photon_score", "photon_vanilla_init",
             "photon_vanilla_prefill", "photon_vanilla_decode_step", "photon_vanilla_cache_info",
             "photon_vanilla_free_cache", "photon_launch_count", "photon_last_error")
 
@@ -103,6 +103,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "photon_decode_rec_chunks": [P, P, I32, P, P],
         "photon_free_cache": [P],
         "photon_cache_set_sampling": [P, ctypes.c_float, U64],
+        "photon_score": [P, P, I32, I32, P, P],
         "photon_vanilla_init": [ctypes.POINTER(photon_vanilla_config), U64, ctypes.POINTER(P)],
         "photon_vanilla_prefill": [P, P, I32, I32, I32, P, ctypes.POINTER(P)],
         "photon_vanilla_decode_step": [P, P, P, P, P, P],
@@ -187,6 +188,16 @@ class Model:
         st = photon_model_stats()
         _check(load_library().photon_model_info(self._h, ctypes.byref(st)))
         return {n: getattr(st, n) for n, _ in st._fields_}
+
+    def score(self, tokens, out=None, stream=None):
+        """Teacher-forced log-probabilities of tokens[:, C:] (CUDA int32 [B, T]) as fp32
+        [B, T - C] (photon_score; synchronising)."""
+        import torch
+        B, T = tokens.shape
+        if out is None:
+            out = torch.empty(B, T - self.C, dtype=torch.float32, device=tokens.device)
+        _check(load_library().photon_score(self._h, _ptr(tokens), B, T, _ptr(out), _stream(stream)))
+        return out
 
     def export_weight(self, index: int, stream=None):
         """Stored values of parameter tensor `index` (generator order) as a flat tensor."""

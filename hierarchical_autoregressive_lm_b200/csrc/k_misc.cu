@@ -309,6 +309,50 @@ void launch_argmax(const float* logits, long long ld, int rows, int V, int i, in
                 samp);
 }
 
+// Log-probability of a target id under softmax(logits[row]): one CTA per
+// row reduces the row maximum and the sum of exp(l - max), then
+// out[row] = l[target] - max - log(sum).  An id outside the vocabulary
+// raises the error word and writes NaN.
+__global__ void k_logprob(const float* __restrict__ logits, int V, const int32_t* __restrict__ target,
+                          float* __restrict__ out, int rows, int* err) {
+  pdl_wait();
+  pdl_trigger();
+  const int row = blockIdx.x;
+  if (row >= rows) return;
+  const float* lr = logits + (long long)row * V;
+  __shared__ float red[32];
+  const int w = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
+  float mx = -INFINITY;
+  for (int c = threadIdx.x; c < V; c += blockDim.x) mx = fmaxf(mx, lr[c]);
+  mx = warp_max(mx);
+  if (lane == 0) red[w] = mx;
+  __syncthreads();
+  mx = red[0];
+  for (int k = 1; k < nw; ++k) mx = fmaxf(mx, red[k]);
+  __syncthreads();
+  float sm = 0.f;
+  for (int c = threadIdx.x; c < V; c += blockDim.x) sm += __expf(lr[c] - mx);
+  sm = warp_sum(sm);
+  if (lane == 0) red[w] = sm;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    float tot = 0.f;
+    for (int k = 0; k < nw; ++k) tot += red[k];
+    const int t = target[row];
+    if (t < 0 || t >= V) {
+      report_error(err, DEV_BAD_TOKEN);
+      out[row] = NAN;
+    } else {
+      out[row] = lr[t] - mx - logf(tot);
+    }
+  }
+}
+void launch_logprob(const float* logits, int V, const int32_t* target, float* out, int rows, int* err,
+                    cudaStream_t s) {
+  if (rows <= 0) return;
+  launch_kernel(k_logprob, rows, 256, 0, s, logits, V, target, out, rows, err);
+}
+
 // One warp per row: max over the row's tile partials, then the same token
 // bookkeeping as k_argmax.
 __global__ void k_argmax_partials(const unsigned long long* __restrict__ part, int tiles, int rows,

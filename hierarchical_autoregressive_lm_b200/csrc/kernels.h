@@ -161,6 +161,9 @@ void launch_argmax_embed_norm(int dt, const unsigned long long* part, int tiles,
                               int C1, const int32_t* force, int32_t* own, int32_t* used,
                               int32_t* next_ids, int* err, const void* E, float* x, const float* g,
                               void* xn, int d, float eps, cudaStream_t s);
+// out[r] = log softmax(logits[r, :V])[target[r]] (teacher-forced scoring).
+void launch_logprob(const float* logits, int V, const int32_t* target, float* out, int rows, int* err,
+                    cudaStream_t s);
 // chunk_ctr (nullable): incremented once, after the reduction (the chunk count
 // the sampling heads read).
 void launch_argmax_partials(const unsigned long long* part, int tiles, int rows, int V, int i,

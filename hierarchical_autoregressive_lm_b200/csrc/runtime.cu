@@ -806,8 +806,11 @@ int photon_export_weight(photon_model* m, int32_t index, void* d_dst, size_t dst
   return PHOTON_OK;
 }
 
-int photon_prefill(photon_model* m, const photon_cache* prefix, const int32_t* d_tokens, int32_t B,
-                   int32_t T, int32_t mode, int32_t max_new_chunks, void* stream, photon_cache** out) {
+// o_all (nullable): also the final-normed top output of every own position,
+// [B * T/C, d] in the storage type (teacher-forced scoring reads them all).
+static int prefill_impl(photon_model* m, const photon_cache* prefix, const int32_t* d_tokens, int32_t B,
+                        int32_t T, int32_t mode, int32_t max_new_chunks, void* stream, photon_cache** out,
+                        void* o_all) {
   g_err.clear();
   if (!m || !out) return fail(PHOTON_ERR_ARG, "NULL model or out");
   *out = nullptr;
@@ -1048,6 +1051,8 @@ int photon_prefill(photon_model* m, const photon_cache* prefix, const int32_t* d
   // pending output: final norm of the last top position of each sequence
   launch_rmsnorm(m->dt, x, (const float*)m->ptr(m->i_top_g), c->o, B, d, N_own, N_own - 1,
                  m->cfg.norm_eps, s);
+  if (o_all)
+    launch_rmsnorm(m->dt, x, (const float*)m->ptr(m->i_top_g), o_all, B * N_own, d, 1, 0, m->cfg.norm_eps, s);
   cudaError_t le = cudaGetLastError();
   free_list(tmp, s);
   if (le != cudaSuccess) {
@@ -1390,6 +1395,11 @@ static bool graphs_enabled() {
 }
 
 extern "C" {
+
+int photon_prefill(photon_model* m, const photon_cache* prefix, const int32_t* d_tokens, int32_t B,
+                   int32_t T, int32_t mode, int32_t max_new_chunks, void* stream, photon_cache** out) {
+  return prefill_impl(m, prefix, d_tokens, B, T, mode, max_new_chunks, stream, out, nullptr);
+}
 
 int photon_decode_step_ex(photon_model* m, photon_cache* c, int32_t mode, int32_t* d_out_tokens,
                           float* d_out_logits, const int32_t* d_force_tokens,
@@ -2274,6 +2284,140 @@ int photon_vanilla_free_cache(photon_vanilla_cache* c) {
   CK(cudaGetLastError());
   m->live_caches--;
   delete c;
+  return PHOTON_OK;
+}
+
+}  // extern "C"
+
+// ============================================================== teacher-forced scoring
+extern "C" {
+
+int photon_score(photon_model* m, const int32_t* d_tokens, int32_t B, int32_t T, float* d_out_logprob,
+                 void* stream) {
+  g_err.clear();
+  if (!m || !d_tokens || !d_out_logprob) return fail(PHOTON_ERR_ARG, "NULL argument");
+  if (m->vanilla) return fail(PHOTON_ERR_ARG, "a vanilla baseline model takes the photon_vanilla_* calls");
+  if (B <= 0 || T <= m->C || T % m->C)
+    return fail(PHOTON_ERR_ARG, "T = %d must be a multiple of C1*C2 = %d longer than one chunk", T, m->C);
+  cudaStream_t s = (cudaStream_t)stream;
+  const int d = m->d, V = m->V, C = m->C, C1 = m->C1, C2 = m->C2;
+  const size_t es = m->es, hd = (size_t)m->H * m->dh;
+  const float eps = m->cfg.norm_eps;
+  const int N = T / C, K = N - 1;
+  const long long G = (long long)B * K;  // scored chunks (chunk k conditions chunk k + 1)
+  const long long G2 = G * C2;           // their sub-chunks
+  const int P = 2 * C1 - 1;              // token-decoder positions per sub-chunk
+  const long long R = G2 * C1;           // scored tokens = B * (T - C)
+  const long long rows_x = G2 * P;
+
+  std::vector<void*> tmp;
+  size_t tmp_bytes = 0;
+  Allocator at{s, &tmp, &tmp_bytes};
+  void* o_all = at.get<void>((size_t)B * N * d * es);
+  if (at.err != cudaSuccess) {
+    free_list(tmp, s);
+    return fail(PHOTON_ERR_OOM, "device allocation failed during scoring");
+  }
+  // a1-a5 over the true tokens, keeping every top output
+  photon_cache* c = nullptr;
+  int rc = prefill_impl(m, nullptr, d_tokens, B, T, PHOTON_MODE_REC, 0, stream, &c, o_all);
+  if (rc != PHOTON_OK) {
+    free_list(tmp, s);
+    return rc;
+  }
+  void* o_sel = at.get<void>((size_t)G * d * es);
+  float* x2 = at.get<float>((size_t)G * C2 * d * 4);
+  void* ahat = at.get<void>((size_t)G * C2 * d * es);
+  float* c1 = at.get<float>((size_t)G2 * C1 * d * 4);
+  float* xd = at.get<float>((size_t)rows_x * d * 4);
+  int32_t* ids = C1 > 1 ? at.get<int32_t>((size_t)G2 * (C1 - 1) * 4) : nullptr;
+  float* emb = C1 > 1 ? at.get<float>((size_t)G2 * (C1 - 1) * d * 4) : nullptr;
+  void* xn = at.get<void>((size_t)rows_x * d * es);
+  void* q = at.get<void>((size_t)rows_x * d * es);
+  void* att = at.get<void>((size_t)rows_x * d * es);
+  void* hid = at.get<void>((size_t)rows_x * m->f * es);
+  void* hn = at.get<void>((size_t)rows_x * d * es);
+  void* hsel = at.get<void>((size_t)R * d * es);
+  int32_t* tg = at.get<int32_t>((size_t)R * 4);
+  const size_t l2 = (size_t)G * hd * C2 * es, l1 = (size_t)G2 * hd * P * es;
+  char* d2k = at.get<char>(l2 * m->Ld2);
+  char* d2v = at.get<char>(l2 * m->Ld2);
+  char* d1k = at.get<char>(l1 * m->Ld1);
+  char* d1v = at.get<char>(l1 * m->Ld1);
+  const long long S = std::min<long long>(R, 8192);  // head rows per slice
+  float* lg = at.get<float>((size_t)S * V * 4);
+  size_t gw = std::max(block_ws_need(m, (int)G * C2), block_ws_need(m, (int)rows_x));
+  gw = std::max(gw, gemm_ws_need(m, (int)G, C2 * d, d));
+  gw = std::max(gw, gemm_ws_need(m, (int)G2, C1 * d, d));
+  gw = std::max(gw, gemm_ws_need(m, (int)S, V, d));
+  float* pws = at.get<float>(gw);
+  int* cnt = at.get<int>(kGemmTileCounters * sizeof(int));
+  int* err = at.get<int>(16);
+  if (at.err != cudaSuccess) {
+    photon_free_cache(c);
+    free_list(tmp, s);
+    return fail(PHOTON_ERR_OOM, "device allocation failed during scoring");
+  }
+  CK(cudaMemsetAsync(cnt, 0, kGemmTileCounters * sizeof(int), s));
+  CK(cudaMemsetAsync(err, 0, 16, s));
+  Bufs b{xn, q, att, hid, c->rope, pws, gw, cnt, nullptr, 0, err};
+  const cudaMemcpyKind dd = cudaMemcpyDeviceToDevice;
+
+  // chunks 0..N-2 of every sequence condition chunks 1..N-1
+  CK(cudaMemcpy2DAsync(o_sel, (size_t)K * d * es, o_all, (size_t)N * d * es, (size_t)K * d * es, B, dd, s));
+  // a7, a8: Converter_2 and the level-2 decoder over its C2 positions -> A-hat
+  gemm(m, b, o_sel, d, m->ptr(m->i_cv2), d, (int)G, C2 * d, d, epi(EPI_STORE_F32, x2, (long long)C2 * d), s);
+  StackRun r2;
+  r2.G = (int)G;
+  r2.q_len = C2;
+  r2.kc = d2k;
+  r2.vc = d2v;
+  r2.layer_bytes = l2;
+  r2.cap = C2;
+  run_stack(m, m->i_dec2, m->Ld2, x2, r2, b, s);
+  launch_rmsnorm(m->dt, x2, (const float*)m->ptr(m->i_dec2_g), ahat, (int)(G * C2), d, 1, 0, eps, s);
+  // a9: Converter_1 -- C1 conditioning vectors per sub-chunk
+  gemm(m, b, ahat, d, m->ptr(m->i_cv1), d, (int)G2, C1 * d, d, epi(EPI_STORE_F32, c1, (long long)C1 * d), s);
+  // token-decoder sequence of a sub-chunk: its conditioning, then its first C1 - 1 true tokens
+  CK(cudaMemcpy2DAsync(xd, (size_t)P * d * 4, c1, (size_t)C1 * d * 4, (size_t)C1 * d * 4, G2, dd, s));
+  if (C1 > 1) {
+    for (int bb = 0; bb < B; ++bb)
+      CK(cudaMemcpy2DAsync(ids + (size_t)bb * K * C2 * (C1 - 1), (size_t)(C1 - 1) * 4,
+                           d_tokens + (size_t)bb * T + C, (size_t)C1 * 4, (size_t)(C1 - 1) * 4,
+                           (size_t)K * C2, dd, s));
+    launch_embed_f32(m->dt, ids, m->ptr(m->i_embed), emb, (int)(G2 * (C1 - 1)), d, V, err, s);
+    CK(cudaMemcpy2DAsync(xd + (size_t)C1 * d, (size_t)P * d * 4, emb, (size_t)(C1 - 1) * d * 4,
+                         (size_t)(C1 - 1) * d * 4, G2, dd, s));
+  }
+  // a10: the token decoder, one causal pass over the P positions of every sub-chunk
+  StackRun r1;
+  r1.G = (int)G2;
+  r1.q_len = P;
+  r1.kc = d1k;
+  r1.vc = d1v;
+  r1.layer_bytes = l1;
+  r1.cap = P;
+  run_stack(m, m->i_dec1, m->Ld1, xd, r1, b, s);
+  launch_rmsnorm(m->dt, xd, (const float*)m->ptr(m->i_dec1_g), hn, (int)rows_x, d, 1, 0, eps, s);
+  // rows C1-1 .. P-1 of a sub-chunk predict its C1 tokens; targets = tokens C .. T-1
+  CK(cudaMemcpy2DAsync(hsel, (size_t)C1 * d * es, (char*)hn + (size_t)(C1 - 1) * d * es, (size_t)P * d * es,
+                       (size_t)C1 * d * es, G2, dd, s));
+  CK(cudaMemcpy2DAsync(tg, (size_t)(T - C) * 4, d_tokens + C, (size_t)T * 4, (size_t)(T - C) * 4, B, dd, s));
+  // a11: head and log-softmax, a slice of rows at a time
+  for (long long r0 = 0; r0 < R; r0 += S) {
+    const int rows = (int)std::min<long long>(S, R - r0);
+    gemm(m, b, (char*)hsel + (size_t)r0 * d * es, d, m->ptr(m->i_head), d, rows, V, d,
+         epi(EPI_STORE_F32, lg, V), s);
+    launch_logprob(lg, V, tg + r0, d_out_logprob + r0, rows, err, s);
+  }
+  int herr = 0;
+  cudaError_t le = cudaGetLastError();
+  if (le == cudaSuccess) le = cudaMemcpyAsync(&herr, err, sizeof(int), cudaMemcpyDeviceToHost, s);
+  photon_free_cache(c);  // stream-ordered releases after the read above
+  free_list(tmp, s);
+  if (le == cudaSuccess) le = cudaStreamSynchronize(s);
+  if (le != cudaSuccess) return fail(PHOTON_ERR_CUDA, "scoring failed: %s", cudaGetErrorString(le));
+  if (herr) return fail(PHOTON_ERR_DEVICE_CHECK, "device check failed during scoring (code %d)", herr);
   return PHOTON_OK;
 }
 

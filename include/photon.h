@@ -309,6 +309,21 @@ PHOTON_API int photon_attn_decode_noalloc(int32_t dtype, const void* d_q, const 
                                           int32_t cap, int32_t q_len, int32_t p0, void* d_o,
                                           void* stream);
 
+/* Teacher-forced scoring (explainer, quality section: PHOTON's reported
+ * quality is measured with teacher-forced HierGen).  For prompts d_tokens
+ * [B, T] (device, row-major; T a multiple of C1*C2 and longer than one
+ * chunk) writes d_out_logprob [B, T - C1*C2] (device fp32): the natural-log
+ * probability of token t (t >= C1*C2) given the prompt before it.  The
+ * bottom-up pass encodes the true tokens; the top output of chunk k
+ * conditions chunk k + 1 through Converter_2, Decoder_2 and Converter_1, and
+ * the token decoder reads the chunk's true tokens (one causal pass per
+ * sub-chunk).  The first chunk has no conditioning and is not scored.
+ * Synchronising (it reports device checks).  Allocates its temporaries from
+ * the library's pool.  Errors: ERR_ARG, ERR_OOM, ERR_CUDA, ERR_DEVICE_CHECK
+ * (a token id outside the vocabulary). */
+PHOTON_API int photon_score(photon_model* m, const int32_t* d_tokens, int32_t B, int32_t T,
+                            float* d_out_logprob, void* stream);
+
 /* ------------------------------------------------------------------------
  * Same-kernel baseline: a vanilla token-level Transformer.
  *
