@@ -316,6 +316,20 @@ def run_gpu(args) -> None:
     torch.cuda.synchronize()
     samp_dec_ms = sev[0].elapsed_time(sev[1])
 
+    # ---- teacher-forced scoring (the pages' quality measurement) of a few of
+    # the prompts: log-probability of every token after the first chunk
+    sc_b = min(B, 4)
+    sc_ms = 0.0
+    if not prefix_len:
+        model.score(toks[:sc_b])                       # untimed first pass
+        se = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+        torch.cuda.synchronize()
+        se[0].record(stream)
+        model.score(toks[:sc_b])
+        se[1].record(stream)
+        torch.cuda.synchronize()
+        sc_ms = se[0].elapsed_time(se[1])
+
     # ---- same-kernel baseline: a vanilla token-level Transformer of the same
     # width and total depth over the same prompts (its KV covers every token)
     van = None
@@ -336,8 +350,8 @@ def run_gpu(args) -> None:
     if pre_cache is not None:
         pre_cache.free()
 
-    total_ms, prefill_ms, decode_ms, e2e_ms, hier_dec_ms, samp_dec_ms, van_ms = max_over_ranks(
-        [total_ms, prefill_ms, decode_ms, e2e_ms, hier_dec_ms, samp_dec_ms, van_ms], device=dev)
+    total_ms, prefill_ms, decode_ms, e2e_ms, hier_dec_ms, samp_dec_ms, van_ms, sc_ms = max_over_ranks(
+        [total_ms, prefill_ms, decode_ms, e2e_ms, hier_dec_ms, samp_dec_ms, van_ms, sc_ms], device=dev)
 
     dec_tokens = world * B * chunks * C * args.steps
     value = job_throughput(B * chunks * C * args.steps, world, decode_ms)
@@ -378,6 +392,11 @@ def run_gpu(args) -> None:
                     "tok_s_per_gib": round(B * chunks * C / (hier_dec_ms / 1e3) / (hier_res / 2 ** 30), 1),
                     "steps": 1},
         "vanilla_baseline": vanilla_line(van, van_ms, world, value / world / gib) if van else None,
+        "scoring": ({"sequences_per_gpu": sc_b, "scored_tokens_per_gpu": sc_b * (T - C),
+                     "tok_s": round(world * sc_b * (T - C) / (sc_ms / 1e3), 1), "ms": round(sc_ms, 3),
+                     "covers": "teacher-forced log-probabilities (photon_score): bottom-up pass, "
+                               "decoders over every chunk, vocabulary head for every token"}
+                    if sc_ms else None),
         "recgen_sampled": {"temperature": 1.0,
                            "decode_tok_s": round(job_throughput(B * chunks * C, world, samp_dec_ms), 1),
                            "decode_ms_per_chunk": round(samp_dec_ms / chunks, 4), "steps": 1},
