@@ -362,11 +362,7 @@ def run_gpu(args) -> None:
         "ms_per_step": round(total_ms / args.steps, 3), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": shape["dtype"],
         "data": "synthetic: seeded N(0,0.02)-like weights (SplitMix64 + Irwin-Hall), Zipf(1.1) prompt ids",
-        "config": {"workload": f"{args.workload}: PHOTON 600M-class L=2 C1=C2={shape['C1']}, "
-                               f"B={B} per GPU, prompt {T}"
-                               + (f" after a shared {prefix_len}-token prefix (prefilled once)"
-                                  if prefix_len else "")
-                               + f", RecGen decode {chunks * C} tokens",
+        "config": {"workload": workload_label(args.workload),
                    "batch_per_gpu": B, "prompt_len": T, "decode_tokens": chunks * C,
                    "parallelism": f"dp{world}", "l2": "working set > L2 (no flush)",
                    "decode_api": args.decode_api},
@@ -675,6 +671,15 @@ def measure_attn_roofline(model, wl, dev, stream) -> dict:
             "shape": f"B={B} H={H} dh={dh} keys={n_mid}"}
 
 
+def workload_label(workload: str) -> str:
+    """The workload a bench line is measured on (both arms print the same)."""
+    w = WORKLOADS[workload]
+    return (f"{workload}: PHOTON 600M-class L=2 C1=C2={w['C1']}, B={w['batch']} per GPU, "
+            f"prompt {w['prompt_len']}"
+            + (f" after a shared {w['prefix_len']}-token prefix (prefilled once)" if w.get("prefix_len") else "")
+            + f", RecGen decode {w['decode_tokens']} tokens")
+
+
 def oracle_prompt(workload: str):
     """Sequence 0's whole context: the shared prefix (if the workload has one)
     followed by its own prompt; the oracle's prefill of it equals prefilling
@@ -742,7 +747,7 @@ def run_reference(args) -> None:
         "n_gpus": world, "steps": len(per), "warmup": args.warmup,
         "ms_per_step": round(1e3 * secs / len(per), 3), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": args.workload, "batch_per_gpu": wl["batch"],
+        "config": {"workload": workload_label(args.workload), "batch_per_gpu": wl["batch"],
                    "prompt_len": wl["prompt_len"], "decode_tokens": wl["decode_tokens"],
                    "parallelism": "none (host cores)"},
         "cpu_baseline": {"value": round(value, 3), "unit": UNIT, "cores": cores, "kind": "oracle",
