@@ -329,9 +329,9 @@ class PhotonOracle:
 
         Sub-chunk j uses Converter_1(A-hat_j) as its conditioning; its tokens
         depend on nothing else (R4).  Greedy argmax, lowest index on ties (R12);
-        with `sample` = (temperature, seed, b) the token is drawn from
-        softmax(logits / temperature) instead (oracle/sampling.py), token
-        index first_t + j*C1 + i.  `force` (teacher forcing, entries < 0 = not
+        with `sample` = (temperature, seed, b[, top_p]) the token is drawn
+        from softmax(logits / temperature), optionally restricted to its top-p
+        nucleus (oracle/sampling.py), token index first_t + j*C1 + i.  `force` (teacher forcing, entries < 0 = not
         forced) replaces the token fed back, not the recorded choice."""
         cfg = self.cfg
         C1, C2, V = cfg.C1, cfg.C2, cfg.vocab
@@ -349,8 +349,10 @@ class PhotonOracle:
                 if sample is None:
                     own[t], z = int(np.argmax(lg)), lg
                 else:
-                    temperature, seed, b = sample
-                    own[t], z = draw(lg, temperature, seed, b, first_t + t)
+                    temperature, seed, b = sample[:3]
+                    top_p = sample[3] if len(sample) > 3 else 1.0
+                    own[t], z = draw(lg, temperature, seed, b, first_t + t, top_p)
+                    z = z[np.isfinite(z)]
                 srt = np.sort(z)
                 tie[t] = (srt[-1] - srt[-2]) < 1e-5 * (srt[-1] - srt[0])
                 used[t] = own[t] if force is None or force[t] < 0 else int(force[t])

@@ -29,6 +29,11 @@ b is the sequence's row in the batch, t the token's index among the tokens
 the cache has generated (chunk * C1*C2 + sub-chunk * C1 + position), v the
 vocabulary id.  Ties of the perturbed values go to the lowest id, as for
 greedy decoding.
+
+Nucleus (top-p) sampling, a common refinement the pages do not mention
+either, restricts the draw to the smallest set of most probable tokens whose
+probability reaches p (ties at its edge included) and renormalises; the
+Gumbel-max rule over that set has exactly that law.
 """
 from __future__ import annotations
 
@@ -77,11 +82,29 @@ def gumbel(key: np.uint32, V: int) -> np.ndarray:
     return -np.log(e)
 
 
-def sample(logits: np.ndarray, temperature: float, seed: int, b: int, t: int):
-    """Token drawn from softmax(logits / T) by the Gumbel-max rule.
+def nucleus(logits: np.ndarray, temperature: float, top_p: float) -> np.ndarray:
+    """Mask of the top-p nucleus of softmax(logits / T): the smallest set of
+    most probable tokens whose probability reaches top_p, with every token
+    tied with its least probable member (so it is {v : p_v >= theta})."""
+    z = np.asarray(logits, dtype=np.float64) / temperature
+    p = np.exp(z - z.max())
+    p /= p.sum()
+    order = np.argsort(-p, kind="stable")
+    cum = np.cumsum(p[order])
+    k = int(np.searchsorted(cum, top_p * (1.0 - 1e-12)))   # first index whose mass reaches top_p
+    theta = p[order[min(k, p.size - 1)]]
+    return p >= theta
 
-    Returns (token, perturbed values); T must be > 0."""
+
+def sample(logits: np.ndarray, temperature: float, seed: int, b: int, t: int, top_p: float = 1.0):
+    """Token drawn from softmax(logits / T) by the Gumbel-max rule; with
+    top_p < 1, from that distribution restricted to its top-p nucleus and
+    renormalised (the maximum runs over the nucleus only).
+
+    Returns (token, perturbed values, -inf outside the nucleus); T > 0."""
     if not temperature > 0:
         raise ValueError("temperature must be positive")
     z = np.asarray(logits, dtype=np.float64) / temperature + gumbel(row_key(seed, b, t), logits.shape[-1])
+    if top_p < 1.0:
+        z = np.where(nucleus(logits, temperature, top_p), z, -np.inf)
     return int(np.argmax(z)), z

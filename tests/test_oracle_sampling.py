@@ -91,3 +91,31 @@ def test_sampled_decode_step_reduces_to_greedy_and_is_reproducible():
         assert np.array_equal(h1.tokens, h2.tokens)
     # at T = 1 over a 256-way, nearly flat distribution the draws leave the greedy path
     assert hot1.tokens != greedy.tokens
+
+
+def test_nucleus_is_the_smallest_top_set_reaching_p():
+    lg = np.log(np.array([0.05, 0.4, 0.1, 0.3, 0.15]))
+    assert list(np.flatnonzero(S.nucleus(lg, 1.0, 0.5))) == [1, 3]          # 0.4 + 0.3 >= 0.5
+    assert list(np.flatnonzero(S.nucleus(lg, 1.0, 0.7))) == [1, 3]          # exactly 0.7
+    assert list(np.flatnonzero(S.nucleus(lg, 1.0, 0.71))) == [1, 3, 4]
+    assert S.nucleus(lg, 1.0, 1.0).all()
+    tie = np.log(np.array([0.3, 0.3, 0.2, 0.2]))
+    assert list(np.flatnonzero(S.nucleus(tie, 1.0, 0.55))) == [0, 1, 2, 3][:2]
+    assert list(np.flatnonzero(S.nucleus(tie, 1.0, 0.65))) == [0, 1, 2, 3]  # the tie at the edge joins
+
+
+def test_top_p_draws_follow_the_renormalised_nucleus():
+    logits = np.array([1.3, -0.2, 0.7, 2.1, 0.0, -1.5])
+    T, top_p, n = 1.0, 0.8, 30000
+    mask = S.nucleus(logits, T, top_p)
+    p = np.exp(logits / T - (logits / T).max())
+    p /= p.sum()
+    q = np.where(mask, p, 0.0)
+    q /= q.sum()
+    counts = np.zeros(logits.size)
+    for t in range(n):
+        counts[S.sample(logits, T, 5, 1, t, top_p)[0]] += 1
+    assert counts[~mask].sum() == 0
+    k = mask.sum()
+    chi2 = float(((counts[mask] - n * q[mask]) ** 2 / (n * q[mask])).sum())
+    assert chi2 < {1: 0.0, 2: 15.1, 3: 18.4, 4: 21.1, 5: 23.5}[k] + 1e-9, (chi2, counts / n, q)
