@@ -30,7 +30,8 @@ _ERRORS = {-1: "PHOTON_ERR_ARG", -2: "PHOTON_ERR_OOM", -3: "PHOTON_ERR_CUDA",
 EXPORTED = ("photon_init_weights", "photon_free_model", "photon_prefill",
             "photon_decode_step_hier", "photon_decode_step_rec", "photon_decode_step_ex",
             "photon_decode_rec_chunks",
-            "photon_free_cache", "photon_cache_set_sampling", "photon_cache_info", "photon_model_info",
+            "photon_free_cache", "photon_cache_set_sampling", "photon_cache_set_top_p",
+            "photon_sample_logits", "photon_cache_info", "photon_model_info",
             "photon_export_weight", "photon_export_state", "photon_gemm", "photon_gemm_rmsnorm",
             "photon_attn_decode", "photon_attn_decode_noalloc", "photon_score", "photon_vanilla_init",
             "photon_vanilla_prefill", "photon_vanilla_decode_step", "photon_vanilla_cache_info",
@@ -103,6 +104,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "photon_decode_rec_chunks": [P, P, I32, P, P],
         "photon_free_cache": [P],
         "photon_cache_set_sampling": [P, ctypes.c_float, U64],
+        "photon_cache_set_top_p": [P, ctypes.c_float],
+        "photon_sample_logits": [P, I32, I32, ctypes.c_float, ctypes.c_float, U64, P, I32, I32, I32, P, P],
         "photon_score": [P, P, I32, I32, P, P],
         "photon_vanilla_init": [ctypes.POINTER(photon_vanilla_config), U64, ctypes.POINTER(P)],
         "photon_vanilla_prefill": [P, P, I32, I32, I32, P, ctypes.POINTER(P)],
@@ -254,10 +257,13 @@ class Cache:
         _check(load_library().photon_decode_rec_chunks(self.model._h, self._h, n_chunks,
                                                        _ptr(out_tokens), _stream(stream)))
 
-    def set_sampling(self, temperature: float, seed: int = 0) -> None:
-        """Later tokens drawn from softmax(logits / temperature) (Gumbel-max with
-        counter-based noise, see photon.h); temperature 0 = greedy."""
-        _check(load_library().photon_cache_set_sampling(self._h, float(temperature), int(seed)))
+    def set_sampling(self, temperature: float, seed: int = 0, top_p: float = 1.0) -> None:
+        """Later tokens drawn from softmax(logits / temperature), optionally restricted to
+        its top-p nucleus (Gumbel-max with counter-based noise, see photon.h);
+        temperature 0 = greedy."""
+        L = load_library()
+        _check(L.photon_cache_set_sampling(self._h, float(temperature), int(seed)))
+        _check(L.photon_cache_set_top_p(self._h, float(top_p)))
 
     def info(self) -> dict:
         st = photon_cache_stats()
@@ -339,6 +345,14 @@ class VanillaCache:
         if self._h:
             _check(load_library().photon_vanilla_free_cache(self._h))
             self._h = None
+
+
+def sample_logits(logits, temperature: float, top_p: float, seed: int, chunk, C1: int, C2: int, i: int,
+                  out, stream=None) -> None:
+    """photon_sample_logits: logits CUDA fp32 [rows, V]; chunk CUDA int32 [1]; out int32 [rows]."""
+    rows, V = logits.shape
+    _check(load_library().photon_sample_logits(_ptr(logits), rows, V, float(temperature), float(top_p),
+                                               int(seed), _ptr(chunk), C1, C2, i, _ptr(out), _stream(stream)))
 
 
 def launch_count() -> int:

@@ -309,6 +309,111 @@ void launch_argmax(const float* logits, long long ld, int rows, int V, int i, in
                 samp);
 }
 
+// Nucleus (top-p) sampling of row `row` of logits: z = logit * inv_t,
+// p_v = exp(z_v - max z) (unnormalised, the largest is 1), S = sum p_v.  The
+// nucleus is {v : p_v >= theta} for the largest theta whose mass
+// sum_{p_v >= theta} p_v reaches top_p * S (the smallest set of most
+// probable tokens reaching top_p, ties at its edge included); theta is found
+// by bisection on (0, 1] until the bracket is two adjacent floats, every pass
+// recomputing p_v the same way, so the membership test is the one bisected.
+// The token is then the Gumbel-max draw over the nucleus (sampling.cuh), with
+// the same bookkeeping as k_argmax.
+__device__ __forceinline__ float block_sum256(float v, float* red) {
+  v = warp_sum(v);
+  const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  __syncthreads();
+  if (lane == 0) red[w] = v;
+  __syncthreads();
+  float t = 0.f;
+  for (int k = 0; k < (int)(blockDim.x >> 5); ++k) t += red[k];
+  return t;
+}
+__global__ void k_sample_topp(const float* __restrict__ logits, long long ld, int rows, int V, int step,
+                              int C1, SampleArgs sa, float top_p, const int32_t* __restrict__ force,
+                              int32_t* own, int32_t* used, int32_t* next_ids, int* err) {
+  pdl_wait();
+  pdl_trigger();
+  const int row = blockIdx.x;
+  if (row >= rows) return;
+  __shared__ float red[32];
+  __shared__ float sv[32];
+  __shared__ int si[32];
+  const float* lr = logits + (long long)row * ld;
+  const float it = sa.inv_t;
+  float mx = -INFINITY;
+  for (int c = threadIdx.x; c < V; c += blockDim.x) mx = fmaxf(mx, lr[c] * it);
+  mx = warp_max(mx);
+  {
+    const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (lane == 0) red[w] = mx;
+    __syncthreads();
+    mx = red[0];
+    for (int k = 1; k < (int)(blockDim.x >> 5); ++k) mx = fmaxf(mx, red[k]);
+  }
+  float part = 0.f;
+  for (int c = threadIdx.x; c < V; c += blockDim.x) part += __expf(lr[c] * it - mx);
+  const float target = top_p * block_sum256(part, red);
+  float lo = 0.f, hi = 1.0f;  // mass(lo) >= target; hi is above every p
+  hi = nextafterf(hi, 2.f);
+  for (int iter = 0; iter < 200; ++iter) {
+    const float mid = 0.5f * (lo + hi);
+    if (!(mid > lo && mid < hi)) break;  // adjacent floats
+    float mass = 0.f;
+    for (int c = threadIdx.x; c < V; c += blockDim.x) {
+      const float p = __expf(lr[c] * it - mx);
+      if (p >= mid) mass += p;
+    }
+    if (block_sum256(mass, red) >= target)
+      lo = mid;
+    else
+      hi = mid;
+  }
+  // Gumbel-max over the nucleus, lowest id on ties
+  const uint32_t key = sample_row_key(sa, row);
+  float bv = -INFINITY;
+  int bi = 0x7fffffff;
+  for (int c = threadIdx.x; c < V; c += blockDim.x) {
+    const float z = lr[c] * it;
+    if (__expf(z - mx) >= lo) better(bv, bi, z + sample_gumbel(key, c), c);
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+    const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
+    better(bv, bi, ov, oi);
+  }
+  const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (lane == 0) {
+    sv[w] = bv;
+    si[w] = bi;
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    for (int k = 1; k < (int)(blockDim.x >> 5); ++k) better(bv, bi, sv[k], si[k]);
+    if (bi < 0 || bi >= V) {
+      report_error(err, DEV_BAD_TOKEN);
+      bi = 0;
+    }
+    const long long slot = (long long)row * C1 + step;
+    int u = bi;
+    if (force) {
+      const int f = force[slot];
+      if (f >= 0) u = (f < V) ? f : 0;
+      if (f >= V) report_error(err, DEV_BAD_TOKEN);
+    }
+    if (own) own[slot] = bi;
+    if (used) used[slot] = u;
+    if (next_ids) next_ids[row] = u;
+  }
+}
+void launch_sample_topp(const float* logits, long long ld, int rows, int V, int i, int C1, const SampleArgs& sa,
+                        float top_p, const int32_t* force, int32_t* own, int32_t* used, int32_t* next_ids,
+                        int* err, cudaStream_t s) {
+  if (rows <= 0) return;
+  launch_kernel(k_sample_topp, rows, 256, 0, s, logits, ld, rows, V, i, C1, sa, top_p, force, own, used,
+                next_ids, err);
+}
+
 // Log-probability of a target id under softmax(logits[row]): one CTA per
 // row reduces the row maximum and the sum of exp(l - max), then
 // out[row] = l[target] - max - log(sum).  An id outside the vocabulary

@@ -161,6 +161,11 @@ void launch_argmax_embed_norm(int dt, const unsigned long long* part, int tiles,
                               int C1, const int32_t* force, int32_t* own, int32_t* used,
                               int32_t* next_ids, int* err, const void* E, float* x, const float* g,
                               void* xn, int d, float eps, cudaStream_t s);
+// Nucleus (top-p) draw per row of logits (Gumbel-max over the smallest set
+// of most probable tokens reaching top_p); outputs as launch_argmax.
+void launch_sample_topp(const float* logits, long long ld, int rows, int V, int i, int C1, const SampleArgs& sa,
+                        float top_p, const int32_t* force, int32_t* own, int32_t* used, int32_t* next_ids,
+                        int* err, cudaStream_t s);
 // out[r] = log softmax(logits[r, :V])[target[r]] (teacher-forced scoring).
 void launch_logprob(const float* logits, int V, const int32_t* target, float* out, int rows, int* err,
                     cudaStream_t s);

@@ -368,6 +368,7 @@ struct photon_cache {
   int* d_pos = nullptr;          // device {N, N1, chunks generated, 0} read by the decode kernels
   float samp_inv_t = 0.f;        // token sampling: 1 / temperature (0: greedy)
   unsigned long long samp_seed = 0;
+  float samp_top_p = 1.f;        // nucleus mass (1: the whole vocabulary)
   unsigned long long* amax_part = nullptr;  // [B*C2][amax_cap] head partials
   int amax_cap = 0;
   int32_t* tok_out = nullptr;    // [B, C] greedy tokens of the last graph-replayed step
@@ -1300,7 +1301,8 @@ static void enqueue_decode(photon_model* m, photon_cache* c, int mode, int32_t* 
     sa.C1 = C1;
     sa.C2 = C2;
     sa.i = i;
-    if (amax_tiles > 0 && amax_tiles <= c->amax_cap) {
+    const bool topp = c->samp_inv_t > 0.f && c->samp_top_p < 1.f;  // nucleus draws need the whole row
+    if (amax_tiles > 0 && amax_tiles <= c->amax_cap && !topp) {
       // tensor-core head with the greedy choice fused into its epilogue;
       // logits are written only when the caller asks for them
       Epilogue e = epi(EPI_ARGMAX, d_out_logits ? d_out_logits + (size_t)i * V : nullptr, ld);
@@ -1321,8 +1323,12 @@ static void enqueue_decode(photon_model* m, photon_cache* c, int mode, int32_t* 
     } else {
       float* lg = d_out_logits ? d_out_logits + (size_t)i * V : c->logits;
       gemm(m, bk, c->hn, d, m->ptr(m->i_head), d, G, V, d, epi(EPI_STORE_F32, lg, ld), ts);
-      launch_argmax(lg, ld, G, V, i, C1, d_force_tokens, d_out_tokens, c->used, c->next_ids,
-                    c->d_err, sa, ts);
+      if (topp)
+        launch_sample_topp(lg, ld, G, V, i, C1, sa, c->samp_top_p, d_force_tokens, d_out_tokens, c->used,
+                           c->next_ids, c->d_err, ts);
+      else
+        launch_argmax(lg, ld, G, V, i, C1, d_force_tokens, d_out_tokens, c->used, c->next_ids,
+                      c->d_err, sa, ts);
       if (i + 1 == C1) launch_advance(chunk_ctr, 1, 0, ts);  // count the chunk
     }
   };
@@ -1690,6 +1696,39 @@ int photon_cache_set_sampling(photon_cache* c, float temperature, uint64_t seed)
   for (int k = 0; k < 2; ++k)
     if (m->graph_owner[k] == c) m->graph_owner[k] = nullptr;
   if (m->pg_owner == c) m->pg_owner = nullptr;
+  return PHOTON_OK;
+}
+
+int photon_cache_set_top_p(photon_cache* c, float top_p) {
+  g_err.clear();
+  if (!c) return fail(PHOTON_ERR_ARG, "cache is NULL");
+  if (!(top_p > 0.f && top_p <= 1.f)) return fail(PHOTON_ERR_ARG, "top_p must be in (0, 1]");
+  c->samp_top_p = top_p;
+  photon_model* m = c->m;
+  for (int k = 0; k < 2; ++k)
+    if (m->graph_owner[k] == c) m->graph_owner[k] = nullptr;
+  if (m->pg_owner == c) m->pg_owner = nullptr;
+  return PHOTON_OK;
+}
+
+int photon_sample_logits(const float* d_logits, int32_t rows, int32_t V, float temperature, float top_p,
+                         uint64_t seed, const int32_t* d_chunk, int32_t C1, int32_t C2, int32_t i,
+                         int32_t* d_out, void* stream) {
+  g_err.clear();
+  if (!d_logits || !d_chunk || !d_out) return fail(PHOTON_ERR_ARG, "NULL buffer");
+  if (rows <= 0 || V <= 0 || C1 <= 0 || C2 <= 0 || i < 0 || i >= C1) return fail(PHOTON_ERR_ARG, "bad shape");
+  if (!(temperature > 0.f) || !std::isfinite(1.0f / temperature) || !(top_p > 0.f && top_p <= 1.f))
+    return fail(PHOTON_ERR_ARG, "need temperature > 0 and top_p in (0, 1]");
+  SampleArgs sa;
+  sa.inv_t = 1.0f / temperature;
+  sa.seed = seed;
+  sa.chunk = d_chunk;
+  sa.C1 = C1;
+  sa.C2 = C2;
+  sa.i = i;
+  launch_sample_topp(d_logits, V, rows, V, 0, 1, sa, top_p, nullptr, d_out, nullptr, nullptr, nullptr,
+                     (cudaStream_t)stream);
+  CK(cudaGetLastError());
   return PHOTON_OK;
 }
 

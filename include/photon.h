@@ -196,6 +196,25 @@ PHOTON_API int photon_free_cache(photon_cache* c);
  * subnormal-reciprocal temperature). */
 PHOTON_API int photon_cache_set_sampling(photon_cache* c, float temperature, uint64_t seed);
 
+/* Nucleus (top-p) restriction of the cache's temperature sampling: each
+ * draw runs over the smallest set of most probable tokens whose probability
+ * under softmax(logits / T) reaches top_p (ties at its edge included), i.e.
+ * {v : p_v >= theta} for the largest such theta, renormalised; the Gumbel
+ * noise is photon_cache_set_sampling's.  top_p = 1 (the default) turns it
+ * off; it has no effect while the temperature is 0.  Such heads write their
+ * logits and draw in a separate kernel instead of the fused epilogue.
+ * Host-only; the next decode call re-captures its graphs.  Errors: ERR_ARG
+ * (NULL cache, top_p outside (0, 1]). */
+PHOTON_API int photon_cache_set_top_p(photon_cache* c, float top_p);
+
+/* Kernel-level draw (tests): row r of d_logits [rows, V] (fp32) is a head
+ * row b*C2 + j emitting token j*C1 + i of chunk *d_chunk (device int32);
+ * d_out[r] receives its draw under (temperature, top_p, seed) exactly as a
+ * sampling decode step would.  Errors: ERR_ARG, ERR_CUDA. */
+PHOTON_API int photon_sample_logits(const float* d_logits, int32_t rows, int32_t V, float temperature,
+                                    float top_p, uint64_t seed, const int32_t* d_chunk, int32_t C1, int32_t C2,
+                                    int32_t i, int32_t* d_out, void* stream);
+
 typedef struct photon_cache_stats {
   int32_t B, T, mode;
   int32_t N;          /* top-level entries visible (prefix + own) */

@@ -146,3 +146,70 @@ def test_bf16_sampling_graphs_and_chunks_equal_eager_steps():
     for c in caches + [g, s]:
         c.free()
     model.free()
+
+
+@pytest.mark.parametrize("T,top_p", [(1.0, 0.9), (0.7, 0.5), (1.5, 0.99), (1.0, 1.0), (1.0, 0.02)])
+def test_topp_kernel_matches_oracle(T, top_p):
+    # logits with well-separated probabilities (a permuted geometric ladder:
+    # neighbours differ by 0.8 %), so the fp32 and fp64 nuclei agree unless
+    # the cumulative mass lands within 1e-5 of top_p (those rows are skipped)
+    from oracle import sampling as S
+    rows, V, C1, C2, i, chunk, seed = 12, 1000, 4, 4, 2, 5, 77
+    rng = np.random.default_rng(int(T * 100 + top_p * 1000))
+    lg = np.stack([8.0 * rng.permutation(V) / V for _ in range(rows)]).astype(np.float32)
+    out = torch.empty(rows, dtype=torch.int32, device="cuda")
+    hal.sample_logits(torch.from_numpy(lg).cuda(), T, top_p, seed,
+                      torch.tensor([chunk], dtype=torch.int32, device="cuda"), C1, C2, i, out)
+    torch.cuda.synchronize()
+    got = out.cpu().numpy()
+    compared = 0
+    for r in range(rows):
+        l64 = lg[r].astype(np.float64)
+        p = np.exp(l64 / T - (l64 / T).max())
+        cum = np.cumsum(np.sort(p)[::-1]) / p.sum()
+        if np.min(np.abs(cum - top_p)) < 1e-5 and top_p < 1.0:
+            continue
+        b, j = divmod(r, C2)
+        tok, z = S.sample(l64, T, seed, b, chunk * C1 * C2 + j * C1 + i, top_p)
+        top2 = np.sort(z[np.isfinite(z)])[-2:]
+        if top2.size == 2 and top2[1] - top2[0] < 1e-4:
+            continue
+        assert got[r] == tok, (r, got[r], tok)
+        if top_p < 1.0:
+            assert S.nucleus(l64, T, top_p)[got[r]]
+        compared += 1
+    assert compared >= rows - 2
+
+
+def test_bf16_topp_graphs_and_chunks_equal_eager_steps():
+    T, seed, top_p, n, B = 1.0, 31, 0.9, 4, 3
+    model = hal.Model(BF_SHAPE, 7)
+    toks = torch.from_numpy(np.random.default_rng(19).integers(0, BF_SHAPE["vocab"], size=(B, 336))
+                            .astype(np.int32)).cuda()
+    none = torch.full((B, BF_CFG.C), -1, dtype=torch.int32, device="cuda")
+    step = torch.empty(B, BF_CFG.C, dtype=torch.int32, device="cuda")
+    caches = [model.prefill(toks, hal.MODE_REC, n) for _ in range(4)]
+    for c in caches[:3]:
+        c.set_sampling(T, seed, top_p)
+    caches[3].set_sampling(T, seed)                   # the same noise without the nucleus
+    eager = torch.empty(B, n * BF_CFG.C, dtype=torch.int32, device="cuda")
+    graph = torch.empty_like(eager)
+    full = torch.empty_like(eager)
+    for k in range(n):
+        caches[0].decode_step(hal.MODE_REC, step, force_tokens=none)
+        eager[:, k * BF_CFG.C:(k + 1) * BF_CFG.C] = step
+        caches[1].step_rec(step)
+        graph[:, k * BF_CFG.C:(k + 1) * BF_CFG.C] = step
+    chunks = torch.empty_like(eager)
+    caches[2].decode_rec_chunks(n, chunks)
+    caches[3].decode_rec_chunks(n, full)
+    torch.cuda.synchronize()
+    assert torch.equal(graph, eager) and torch.equal(chunks, eager)
+    assert int(eager.min()) >= 0 and int(eager.max()) < BF_SHAPE["vocab"]
+    assert not torch.equal(eager, full)               # the nucleus changes some draws
+    assert caches[1].info()["device_error"] == 0
+    with pytest.raises(hal.PhotonError):
+        caches[0].set_sampling(T, seed, 0.0)
+    for c in caches:
+        c.free()
+    model.free()
