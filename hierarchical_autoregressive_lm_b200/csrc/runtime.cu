@@ -2397,13 +2397,17 @@ int photon_score(photon_model* m, const int32_t* d_tokens, int32_t B, int32_t T,
     free_list(tmp, s);
     return fail(PHOTON_ERR_OOM, "device allocation failed during scoring");
   }
-  CK(cudaMemsetAsync(cnt, 0, kGemmTileCounters * sizeof(int), s));
-  CK(cudaMemsetAsync(err, 0, 16, s));
+  cudaError_t ce = cudaSuccess;  // first failing call; work continues to the common release below
+  auto ck = [&](cudaError_t e) {
+    if (ce == cudaSuccess && e != cudaSuccess) ce = e;
+  };
+  ck(cudaMemsetAsync(cnt, 0, kGemmTileCounters * sizeof(int), s));
+  ck(cudaMemsetAsync(err, 0, 16, s));
   Bufs b{xn, q, att, hid, c->rope, pws, gw, cnt, nullptr, 0, err};
   const cudaMemcpyKind dd = cudaMemcpyDeviceToDevice;
 
   // chunks 0..N-2 of every sequence condition chunks 1..N-1
-  CK(cudaMemcpy2DAsync(o_sel, (size_t)K * d * es, o_all, (size_t)N * d * es, (size_t)K * d * es, B, dd, s));
+  ck(cudaMemcpy2DAsync(o_sel, (size_t)K * d * es, o_all, (size_t)N * d * es, (size_t)K * d * es, B, dd, s));
   // a7, a8: Converter_2 and the level-2 decoder over its C2 positions -> A-hat
   gemm(m, b, o_sel, d, m->ptr(m->i_cv2), d, (int)G, C2 * d, d, epi(EPI_STORE_F32, x2, (long long)C2 * d), s);
   StackRun r2;
@@ -2418,14 +2422,14 @@ int photon_score(photon_model* m, const int32_t* d_tokens, int32_t B, int32_t T,
   // a9: Converter_1 -- C1 conditioning vectors per sub-chunk
   gemm(m, b, ahat, d, m->ptr(m->i_cv1), d, (int)G2, C1 * d, d, epi(EPI_STORE_F32, c1, (long long)C1 * d), s);
   // token-decoder sequence of a sub-chunk: its conditioning, then its first C1 - 1 true tokens
-  CK(cudaMemcpy2DAsync(xd, (size_t)P * d * 4, c1, (size_t)C1 * d * 4, (size_t)C1 * d * 4, G2, dd, s));
+  ck(cudaMemcpy2DAsync(xd, (size_t)P * d * 4, c1, (size_t)C1 * d * 4, (size_t)C1 * d * 4, G2, dd, s));
   if (C1 > 1) {
     for (int bb = 0; bb < B; ++bb)
-      CK(cudaMemcpy2DAsync(ids + (size_t)bb * K * C2 * (C1 - 1), (size_t)(C1 - 1) * 4,
+      ck(cudaMemcpy2DAsync(ids + (size_t)bb * K * C2 * (C1 - 1), (size_t)(C1 - 1) * 4,
                            d_tokens + (size_t)bb * T + C, (size_t)C1 * 4, (size_t)(C1 - 1) * 4,
                            (size_t)K * C2, dd, s));
     launch_embed_f32(m->dt, ids, m->ptr(m->i_embed), emb, (int)(G2 * (C1 - 1)), d, V, err, s);
-    CK(cudaMemcpy2DAsync(xd + (size_t)C1 * d, (size_t)P * d * 4, emb, (size_t)(C1 - 1) * d * 4,
+    ck(cudaMemcpy2DAsync(xd + (size_t)C1 * d, (size_t)P * d * 4, emb, (size_t)(C1 - 1) * d * 4,
                          (size_t)(C1 - 1) * d * 4, G2, dd, s));
   }
   // a10: the token decoder, one causal pass over the P positions of every sub-chunk
@@ -2439,9 +2443,9 @@ int photon_score(photon_model* m, const int32_t* d_tokens, int32_t B, int32_t T,
   run_stack(m, m->i_dec1, m->Ld1, xd, r1, b, s);
   launch_rmsnorm(m->dt, xd, (const float*)m->ptr(m->i_dec1_g), hn, (int)rows_x, d, 1, 0, eps, s);
   // rows C1-1 .. P-1 of a sub-chunk predict its C1 tokens; targets = tokens C .. T-1
-  CK(cudaMemcpy2DAsync(hsel, (size_t)C1 * d * es, (char*)hn + (size_t)(C1 - 1) * d * es, (size_t)P * d * es,
+  ck(cudaMemcpy2DAsync(hsel, (size_t)C1 * d * es, (char*)hn + (size_t)(C1 - 1) * d * es, (size_t)P * d * es,
                        (size_t)C1 * d * es, G2, dd, s));
-  CK(cudaMemcpy2DAsync(tg, (size_t)(T - C) * 4, d_tokens + C, (size_t)T * 4, (size_t)(T - C) * 4, B, dd, s));
+  ck(cudaMemcpy2DAsync(tg, (size_t)(T - C) * 4, d_tokens + C, (size_t)T * 4, (size_t)(T - C) * 4, B, dd, s));
   // a11: head and log-softmax, a slice of rows at a time
   for (long long r0 = 0; r0 < R; r0 += S) {
     const int rows = (int)std::min<long long>(S, R - r0);
@@ -2450,7 +2454,8 @@ int photon_score(photon_model* m, const int32_t* d_tokens, int32_t B, int32_t T,
     launch_logprob(lg, V, tg + r0, d_out_logprob + r0, rows, err, s);
   }
   int herr = 0;
-  cudaError_t le = cudaGetLastError();
+  ck(cudaGetLastError());
+  cudaError_t le = ce;
   if (le == cudaSuccess) le = cudaMemcpyAsync(&herr, err, sizeof(int), cudaMemcpyDeviceToHost, s);
   photon_free_cache(c);  // stream-ordered releases after the read above
   free_list(tmp, s);
