@@ -18,6 +18,8 @@ Contents:
   vanilla.py -- a vanilla token-level Transformer of the same width, the
                 baseline of the pages' TPM comparison, built from the same
                 pinned blocks.
+  aggregate.py -- multi-query aggregation (majority vote, best-of-N by
+                teacher-forced log-likelihood) over groups of sampled rows.
 
 Every oracle function is pinned by CPU tests (tests/test_oracle_*.py) to
 facts that do not come from the oracle itself: published SplitMix64 test
