@@ -330,6 +330,11 @@ def run_gpu(args) -> None:
         torch.cuda.synchronize()
         sc_ms = se[0].elapsed_time(se[1])
 
+    # ---- multi-query aggregation: groups of nine sampled rows per prompt,
+    # majority vote and best-of-N (photon_multi_query)
+    mq = measure_multi_query(model, toks, chunks, stream, prefix=pre_cache)
+    mq_ms = [mq[k]["ms"] if isinstance(mq.get(k), dict) else 0.0 for k in ("vote", "best")]
+
     # ---- same-kernel baseline: a vanilla token-level Transformer of the same
     # width and total depth over the same prompts (its KV covers every token)
     van = None
@@ -350,8 +355,13 @@ def run_gpu(args) -> None:
     if pre_cache is not None:
         pre_cache.free()
 
-    total_ms, prefill_ms, decode_ms, e2e_ms, hier_dec_ms, samp_dec_ms, van_ms, sc_ms = max_over_ranks(
-        [total_ms, prefill_ms, decode_ms, e2e_ms, hier_dec_ms, samp_dec_ms, van_ms, sc_ms], device=dev)
+    total_ms, prefill_ms, decode_ms, e2e_ms, hier_dec_ms, samp_dec_ms, van_ms, sc_ms, *mq_ms = max_over_ranks(
+        [total_ms, prefill_ms, decode_ms, e2e_ms, hier_dec_ms, samp_dec_ms, van_ms, sc_ms, *mq_ms], device=dev)
+    for k, ms in zip(("vote", "best"), mq_ms):
+        if isinstance(mq.get(k), dict) and ms > 0:
+            q = mq["queries_per_gpu"]
+            mq[k].update(ms=round(ms, 3), answers_per_s=round(world * q / (ms / 1e3), 2),
+                         generated_tok_s=round(world * mq["rows"] * mq["new_tokens_per_row"] / (ms / 1e3), 1))
 
     dec_tokens = world * B * chunks * C * args.steps
     value = job_throughput(B * chunks * C * args.steps, world, decode_ms)
@@ -393,6 +403,9 @@ def run_gpu(args) -> None:
                      "covers": "teacher-forced log-probabilities (photon_score): bottom-up pass, "
                                "decoders over every chunk, vocabulary head for every token"}
                     if sc_ms else None),
+        "multi_query": dict(mq, covers="photon_multi_query: prefill of Q x N rows, RecGen decode with "
+                                           "temperature sampling, then majority vote (vote) or teacher-forced "
+                                           "scoring + best-of-N (best); whole job"),
         "recgen_sampled": {"temperature": 1.0,
                            "decode_tok_s": round(job_throughput(B * chunks * C, world, samp_dec_ms), 1),
                            "decode_ms_per_chunk": round(samp_dec_ms / chunks, 4), "steps": 1},
@@ -497,6 +510,43 @@ def measure_vanilla(shape, toks, wl, stream) -> dict:
             "resident_gib": round(resident / 2 ** 30, 3), "kv_gib": round(info["kv_bytes"] / 2 ** 30, 3),
             "graph_steps": info["graph_steps"], "tokens": B * (n - 1), "steps": n - 1,
             "_decode_ms": ev[2].elapsed_time(ev[3])}
+
+
+def measure_multi_query(model, toks, n_chunks: int, stream, N: int = 9, prefix=None,
+                        temperature: float = 1.0, seed: int = 7) -> dict:
+    """Multi-query aggregation (the explainer's answer to the single-query
+    quality gap): Q = rows // N groups, each group N copies of one prompt
+    that differ by their sampling noise.  Each mode runs once untimed and
+    once timed through photon_multi_query.  VOTE covers prefill, RecGen
+    decode and the vote.  BEST adds teacher-forced scoring of prompt +
+    continuation and the best-of-N pick, and is skipped after a shared
+    prefix, which the scorer does not take."""
+    import torch
+    import hierarchical_autoregressive_lm_b200 as hal
+    rows, T = toks.shape
+    Q = rows // N
+    if Q == 0:
+        return {"unavailable": f"fewer than N = {N} rows"}
+    grp = toks[:Q].repeat_interleave(N, dim=0).contiguous()
+    out = {"queries_per_gpu": Q, "n": N, "rows": Q * N, "prompt_len": T, "temperature": temperature,
+           "new_tokens_per_row": n_chunks * model.C}
+    for name, mode in (("vote", hal.AGG_VOTE), ("best", hal.AGG_BEST)):
+        if mode == hal.AGG_BEST and prefix is not None:
+            out[name] = None
+            continue
+        model.multi_query(grp, N, n_chunks, temperature, seed, mode=mode, prefix=prefix)   # untimed
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+        torch.cuda.synchronize()
+        ev[0].record(stream)
+        cand, win, score = model.multi_query(grp, N, n_chunks, temperature, seed, mode=mode, prefix=prefix)
+        ev[1].record(stream)
+        torch.cuda.synchronize()
+        ms = ev[0].elapsed_time(ev[1])
+        w = win.cpu()
+        out[name] = {"ms": round(ms, 3), "answers_per_s": round(Q / (ms / 1e3), 2),
+                     "generated_tok_s": round(Q * N * n_chunks * model.C / (ms / 1e3), 1),
+                     "winners_in_range": bool(((w >= 0) & (w < N)).all())}
+    return out
 
 
 def vanilla_line(van: dict, van_ms: float, world: int, photon_tpm: float) -> dict:

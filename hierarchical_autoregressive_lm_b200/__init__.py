@@ -16,11 +16,13 @@ import os
 from typing import Optional
 
 __all__ = ["PhotonError", "Model", "Cache", "load_library", "LIB_PATH", "MODE_HIER",
-           "MODE_REC", "STATE", "launch_count", "gemm", "gemm_rmsnorm", "attn_decode", "attn_decode_noalloc", "config_struct", "EXPORTED"]
+           "MODE_REC", "STATE", "launch_count", "gemm", "gemm_rmsnorm", "attn_decode", "attn_decode_noalloc", "config_struct", "EXPORTED",
+           "AGG_VOTE", "AGG_BEST", "aggregate"]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libphoton.so")
 
 MODE_HIER, MODE_REC = 0, 1
+AGG_VOTE, AGG_BEST = 0, 1
 STATE = {"top_k": 0, "top_v": 1, "l1_k": 2, "l1_v": 3, "pending_o": 4, "a_hat": 5, "a": 6}
 _DTYPES = {"fp32": 0, "bf16": 1}
 _ERRORS = {-1: "PHOTON_ERR_ARG", -2: "PHOTON_ERR_OOM", -3: "PHOTON_ERR_CUDA",
@@ -33,7 +35,8 @@ EXPORTED = ("photon_init_weights", "photon_free_model", "photon_prefill",
             "photon_free_cache", "photon_cache_set_sampling", "photon_cache_set_top_p",
             "photon_sample_logits", "photon_cache_info", "photon_model_info",
             "photon_export_weight", "photon_export_state", "photon_gemm", "photon_gemm_rmsnorm",
-            "photon_attn_decode", "photon_attn_decode_noalloc", "photon_score", "photon_vanilla_init",
+            "photon_attn_decode", "photon_attn_decode_noalloc", "photon_score", "photon_aggregate",
+            "photon_multi_query", "photon_vanilla_init",
             "photon_vanilla_prefill", "photon_vanilla_decode_step", "photon_vanilla_cache_info",
             "photon_vanilla_free_cache", "photon_launch_count", "photon_last_error")
 
@@ -107,6 +110,9 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "photon_cache_set_top_p": [P, ctypes.c_float],
         "photon_sample_logits": [P, I32, I32, ctypes.c_float, ctypes.c_float, U64, P, I32, I32, I32, P, P],
         "photon_score": [P, P, I32, I32, P, P],
+        "photon_aggregate": [I32, P, P, I32, I32, I32, I32, I32, P, P, P],
+        "photon_multi_query": [P, P, P, I32, I32, I32, I32, ctypes.c_float, ctypes.c_float, U64, I32, P, P,
+                               P, P],
         "photon_vanilla_init": [ctypes.POINTER(photon_vanilla_config), U64, ctypes.POINTER(P)],
         "photon_vanilla_prefill": [P, P, I32, I32, I32, P, ctypes.POINTER(P)],
         "photon_vanilla_decode_step": [P, P, P, P, P, P],
@@ -201,6 +207,25 @@ class Model:
             out = torch.empty(B, T - self.C, dtype=torch.float32, device=tokens.device)
         _check(load_library().photon_score(self._h, _ptr(tokens), B, T, _ptr(out), _stream(stream)))
         return out
+
+    def multi_query(self, prompts, N: int, n_chunks: int, temperature: float, seed: int = 0,
+                    top_p: float = 1.0, mode: int = AGG_VOTE, prefix: "Cache" = None, stream=None):
+        """photon_multi_query: prompts CUDA int32 [Q*N, T], groups of N consecutive rows.
+        Returns (candidates int32 [Q*N, n_chunks*C], winners int32 [Q], scores fp64 [Q*N])."""
+        import torch
+        assert prompts.is_cuda and prompts.dtype.itemsize == 4 and prompts.is_contiguous()
+        rows, T = prompts.shape
+        if N <= 0 or rows % N:
+            raise ValueError(f"{rows} rows do not form groups of N = {N}")
+        Q = rows // N
+        cand = torch.empty(rows, n_chunks * self.C, dtype=torch.int32, device=prompts.device)
+        choice = torch.empty(Q, dtype=torch.int32, device=prompts.device)
+        score = torch.empty(rows, dtype=torch.float64, device=prompts.device)
+        _check(load_library().photon_multi_query(self._h, None if prefix is None else prefix._h,
+                                                 _ptr(prompts), Q, N, T, n_chunks, float(temperature),
+                                                 float(top_p), int(seed), mode, _ptr(cand), _ptr(choice),
+                                                 _ptr(score), _stream(stream)))
+        return cand, choice, score
 
     def export_weight(self, index: int, stream=None):
         """Stored values of parameter tensor `index` (generator order) as a flat tensor."""
@@ -353,6 +378,21 @@ def sample_logits(logits, temperature: float, top_p: float, seed: int, chunk, C1
     rows, V = logits.shape
     _check(load_library().photon_sample_logits(_ptr(logits), rows, V, float(temperature), float(top_p),
                                                int(seed), _ptr(chunk), C1, C2, i, _ptr(out), _stream(stream)))
+
+
+def aggregate(mode: int, N: int, choice, cand=None, logprob=None, span_begin: int = 0,
+              span_len: Optional[int] = None, score=None, stream=None) -> None:
+    """photon_aggregate over groups of N consecutive rows of cand (CUDA int32 [Q*N, L],
+    AGG_VOTE) or logprob (CUDA fp32 [Q*N, L], AGG_BEST); choice int32 [Q]; optional
+    score fp64 [Q*N].  span_len defaults to the rest of the row."""
+    src = cand if cand is not None else logprob
+    rows, L = src.shape
+    if N <= 0 or rows % N:
+        raise ValueError(f"{rows} rows do not form groups of N = {N}")
+    if span_len is None:
+        span_len = L - span_begin
+    _check(load_library().photon_aggregate(mode, _ptr(cand), _ptr(logprob), rows // N, N, L, span_begin,
+                                           span_len, _ptr(choice), _ptr(score), _stream(stream)))
 
 
 def launch_count() -> int:

@@ -2466,3 +2466,113 @@ int photon_score(photon_model* m, const int32_t* d_tokens, int32_t B, int32_t T,
 }
 
 }  // extern "C"
+
+// ============================================================== multi-query aggregation
+// PHOTON explainer, quality section: several slightly varied queries, their
+// outputs combined by majority vote or best-of-N.  Kernels in k_aggregate.cu.
+namespace photon {
+void launch_vote(const int32_t* cand, int Q, int N, int L, int b0, int len, int32_t* choice, double* score,
+                 cudaStream_t s);
+void launch_best(const float* logprob, int Q, int N, int L, int b0, int len, int32_t* choice, double* score,
+                 cudaStream_t s);
+}  // namespace photon
+
+extern "C" {
+
+int photon_aggregate(int32_t mode, const int32_t* d_cand, const float* d_logprob, int32_t Q, int32_t N,
+                     int32_t L, int32_t span_begin, int32_t span_len, int32_t* d_choice, double* d_score,
+                     void* stream) {
+  g_err.clear();
+  if (mode != PHOTON_AGG_VOTE && mode != PHOTON_AGG_BEST) return fail(PHOTON_ERR_ARG, "unknown aggregation mode %d", mode);
+  if (Q < 0 || N <= 0 || L < 0 || span_begin < 0 || span_len < 0 || (long long)span_begin + span_len > L)
+    return fail(PHOTON_ERR_ARG, "bad shape: Q = %d, N = %d, L = %d, span [%d, %d + %d)", Q, N, L, span_begin,
+                span_begin, span_len);
+  if (Q == 0) return PHOTON_OK;
+  if (!d_choice) return fail(PHOTON_ERR_ARG, "d_choice is NULL");
+  cudaStream_t s = (cudaStream_t)stream;
+  if (mode == PHOTON_AGG_VOTE) {
+    if (!d_cand) return fail(PHOTON_ERR_ARG, "majority vote needs d_cand");
+    launch_vote(d_cand, Q, N, L, span_begin, span_len, d_choice, d_score, s);
+  } else {
+    if (!d_logprob) return fail(PHOTON_ERR_ARG, "best-of-N needs d_logprob");
+    launch_best(d_logprob, Q, N, L, span_begin, span_len, d_choice, d_score, s);
+  }
+  CK(cudaGetLastError());
+  return PHOTON_OK;
+}
+
+int photon_multi_query(photon_model* m, const photon_cache* prefix, const int32_t* d_prompts, int32_t Q,
+                       int32_t N, int32_t T, int32_t n_chunks, float temperature, float top_p, uint64_t seed,
+                       int32_t mode, int32_t* d_cand, int32_t* d_choice, double* d_score, void* stream) {
+  g_err.clear();
+  if (!m || !d_prompts || !d_cand || !d_choice) return fail(PHOTON_ERR_ARG, "NULL argument");
+  if (m->vanilla) return fail(PHOTON_ERR_ARG, "a vanilla baseline model takes the photon_vanilla_* calls");
+  if (mode != PHOTON_AGG_VOTE && mode != PHOTON_AGG_BEST) return fail(PHOTON_ERR_ARG, "unknown aggregation mode %d", mode);
+  if (Q <= 0 || N <= 0 || n_chunks <= 0 || (long long)Q * N > (1ll << 30))
+    return fail(PHOTON_ERR_ARG, "bad group shape: Q = %d, N = %d, n_chunks = %d", Q, N, n_chunks);
+  if (!(temperature >= 0.f) || !std::isfinite(temperature) ||
+      (temperature > 0.f && !std::isfinite(1.0f / temperature)))
+    return fail(PHOTON_ERR_ARG, "temperature must be finite, >= 0 and not subnormal");
+  if (!(top_p > 0.f && top_p <= 1.f)) return fail(PHOTON_ERR_ARG, "top_p must be in (0, 1]");
+  if (mode == PHOTON_AGG_BEST && prefix)
+    return fail(PHOTON_ERR_ARG, "best-of-N scores the whole context and takes no prefix cache");
+  if ((long long)n_chunks * m->C > (1ll << 30)) return fail(PHOTON_ERR_ARG, "n_chunks too large");
+  cudaStream_t s = (cudaStream_t)stream;
+  const int rows = Q * N, C = m->C, Lc = n_chunks * C;
+
+  // every row decodes n_chunks chunks in RecGen mode, drawing with its own row's noise
+  photon_cache* c = nullptr;
+  RET(prefill_impl(m, prefix, d_prompts, rows, T, PHOTON_MODE_REC, n_chunks, stream, &c, nullptr));
+  int rc = photon_cache_set_sampling(c, temperature, seed);
+  if (rc == PHOTON_OK) rc = photon_cache_set_top_p(c, top_p);
+  if (rc == PHOTON_OK) rc = photon_decode_rec_chunks(m, c, n_chunks, d_cand, stream);
+  int herr = 0;
+  cudaError_t le = cudaSuccess;
+  if (rc == PHOTON_OK) le = cudaMemcpyAsync(&herr, c->d_err, sizeof(int), cudaMemcpyDeviceToHost, s);
+  const std::string decode_msg = g_err;
+  const int frc = photon_free_cache(c);
+  if (rc != PHOTON_OK) {
+    g_err = decode_msg;
+    return rc;
+  }
+  if (frc != PHOTON_OK) return frc;
+  if (le == cudaSuccess) le = cudaStreamSynchronize(s);
+  if (le != cudaSuccess) return fail(PHOTON_ERR_CUDA, "multi-query decode failed: %s", cudaGetErrorString(le));
+  if (herr) return fail(PHOTON_ERR_DEVICE_CHECK, "device check failed during decode (code %d)", herr);
+
+  if (mode == PHOTON_AGG_VOTE) {
+    RET(photon_aggregate(PHOTON_AGG_VOTE, d_cand, nullptr, Q, N, Lc, 0, Lc, d_choice, d_score, stream));
+    CK(cudaStreamSynchronize(s));
+    return PHOTON_OK;
+  }
+  // best-of-N: teacher-forced log-probabilities of prompt + continuation,
+  // summed over the continuation (score index t covers token t + C)
+  const int Tf = T + Lc;
+  std::vector<void*> tmp;
+  size_t tmp_bytes = 0;
+  Allocator at{s, &tmp, &tmp_bytes};
+  int32_t* full = at.get<int32_t>((size_t)rows * Tf * sizeof(int32_t));
+  float* lp = at.get<float>((size_t)rows * (Tf - C) * sizeof(float));
+  if (at.err != cudaSuccess) {
+    free_list(tmp, s);
+    return fail(PHOTON_ERR_OOM, "device allocation failed during best-of-N scoring");
+  }
+  const cudaMemcpyKind dd = cudaMemcpyDeviceToDevice;
+  cudaError_t ce = cudaMemcpy2DAsync(full, (size_t)Tf * 4, d_prompts, (size_t)T * 4, (size_t)T * 4, rows, dd, s);
+  if (ce == cudaSuccess)
+    ce = cudaMemcpy2DAsync(full + T, (size_t)Tf * 4, d_cand, (size_t)Lc * 4, (size_t)Lc * 4, rows, dd, s);
+  rc = ce == cudaSuccess ? photon_score(m, full, rows, Tf, lp, stream) : PHOTON_OK;
+  if (ce == cudaSuccess && rc == PHOTON_OK)
+    rc = photon_aggregate(PHOTON_AGG_BEST, nullptr, lp, Q, N, Tf - C, T - C, Lc, d_choice, d_score, stream);
+  const std::string score_msg = g_err;
+  free_list(tmp, s);
+  if (ce != cudaSuccess) return fail(PHOTON_ERR_CUDA, "copying the scored rows failed: %s", cudaGetErrorString(ce));
+  if (rc != PHOTON_OK) {
+    g_err = score_msg;
+    return rc;
+  }
+  CK(cudaStreamSynchronize(s));
+  return PHOTON_OK;
+}
+
+}  // extern "C"

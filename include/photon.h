@@ -344,6 +344,62 @@ PHOTON_API int photon_score(photon_model* m, const int32_t* d_tokens, int32_t B,
                             float* d_out_logprob, void* stream);
 
 /* ------------------------------------------------------------------------
+ * Multi-query aggregation (explainer, quality section: the single-query
+ * quality gap is closed by running several slightly varied queries, about
+ * nine, and combining their outputs by majority vote or best-of-N).
+ *
+ * A query group is N consecutive rows of a batch.  The rows may hold
+ * different prompts (the caller's variations), and each row draws its own
+ * sampling noise (the generator is keyed by the row). */
+enum {
+  PHOTON_AGG_VOTE = 0, /* the row whose span equals the spans of the most rows */
+  PHOTON_AGG_BEST = 1  /* the row with the largest sum of log-probabilities over its span */
+};
+
+/* Picks one row per group.  Group q holds rows q*N .. q*N + N - 1 of
+ * d_cand [Q*N, L] (device int32, row-major; PHOTON_AGG_VOTE) or of
+ * d_logprob [Q*N, L] (device fp32; PHOTON_AGG_BEST).  Only positions
+ * [span_begin, span_begin + span_len) of a row take part.
+ *   VOTE: count[n] = the number of rows of the group whose span is identical
+ *         to row n's (row n included); the winner has the largest count.
+ *   BEST: sum[n] = the fp64 sum of row n's span; the winner has the largest
+ *         sum, and a NaN sum ranks below every number.
+ * Ties go to the lower row.  d_choice [Q] (device int32) receives the
+ * winner's index within its group (0 .. N-1).  d_score [Q*N] (device fp64,
+ * may be NULL) receives count[n] or sum[n] for every row.  The buffers are
+ * the caller's and must hold the sizes above.  Asynchronous on `stream`.
+ * One CTA per group.  The vote costs O(N^2 * span_len) reads, so it suits
+ * groups of a few dozen rows.  Q = 0 is a no-op.  Errors: ERR_ARG (unknown
+ * mode, N <= 0, Q < 0, a span outside [0, L], a NULL buffer that the mode
+ * reads or writes), ERR_CUDA. */
+PHOTON_API int photon_aggregate(int32_t mode, const int32_t* d_cand, const float* d_logprob, int32_t Q,
+                                int32_t N, int32_t L, int32_t span_begin, int32_t span_len,
+                                int32_t* d_choice, double* d_score, void* stream);
+
+/* The whole multi-query pass.  d_prompts [Q*N, T] (device int32; T a
+ * positive multiple of C1*C2) are prefilled in RecGen mode, after `prefix`
+ * if one is given.  Every row decodes n_chunks chunks with temperature /
+ * top-p sampling (photon_cache_set_sampling, photon_cache_set_top_p; a
+ * temperature of 0 is greedy).  Row r of d_cand [Q*N, n_chunks*C1*C2]
+ * (device int32) receives its continuation.  Each group then picks its
+ * winner over the whole continuation:
+ *   PHOTON_AGG_VOTE: photon_aggregate's vote over the continuation tokens.
+ *   PHOTON_AGG_BEST: photon_score over prompt + continuation.  The
+ *                    log-probabilities of the continuation's tokens are
+ *                    summed, i.e. each row's log-likelihood of its
+ *                    continuation given its own prompt.  No prefix.
+ * d_choice [Q] and d_score [Q*N] (may be NULL) are as in photon_aggregate.
+ * The cache and all temporaries come from the library's pool and are
+ * released before the call returns.  Synchronising (it reports device
+ * checks).  Errors: ERR_ARG (NULL buffer, bad shapes, temperature or top_p
+ * out of range, a prefix with PHOTON_AGG_BEST, a vanilla model), ERR_OOM,
+ * ERR_CUDA, ERR_DEVICE_CHECK (a token id outside the vocabulary). */
+PHOTON_API int photon_multi_query(photon_model* m, const photon_cache* prefix, const int32_t* d_prompts,
+                                  int32_t Q, int32_t N, int32_t T, int32_t n_chunks, float temperature,
+                                  float top_p, uint64_t seed, int32_t mode, int32_t* d_cand,
+                                  int32_t* d_choice, double* d_score, void* stream);
+
+/* ------------------------------------------------------------------------
  * Same-kernel baseline: a vanilla token-level Transformer.
  *
  * The explainer's decode-heavy table (475x section) compares PHOTON's

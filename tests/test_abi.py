@@ -54,3 +54,15 @@ def _load_missing(path):
         hal.load_library(path)
     finally:
         hal._lib = saved
+
+
+def test_aggregation_host_checks_without_a_device():
+    # the argument checks run on the host before any CUDA call
+    lib = hal.load_library()
+    assert lib.photon_aggregate(hal.AGG_VOTE, None, None, 0, 3, 4, 0, 4, None, None, None) == 0   # Q = 0
+    bad = [(2, 1, 3, 4, 0, 4), (hal.AGG_VOTE, 1, 0, 4, 0, 4), (hal.AGG_VOTE, 1, 3, 4, 2, 3),
+           (hal.AGG_VOTE, 1, 3, 4, -1, 1), (hal.AGG_VOTE, -1, 3, 4, 0, 4), (hal.AGG_BEST, 1, 3, 4, 0, 4)]
+    for mode, Q, N, L, b, n in bad:
+        assert lib.photon_aggregate(mode, None, None, Q, N, L, b, n, None, None, None) == -1, (mode, Q, N, L, b, n)
+        assert lib.photon_last_error() != b""
+    assert lib.photon_multi_query(None, None, None, 1, 9, 16, 1, 1.0, 1.0, 0, 0, None, None, None, None) == -1
