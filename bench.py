@@ -534,13 +534,17 @@ def measure_multi_query(model, toks, n_chunks: int, stream, N: int = 9, prefix=N
         if mode == hal.AGG_BEST and prefix is not None:
             out[name] = None
             continue
-        model.multi_query(grp, N, n_chunks, temperature, seed, mode=mode, prefix=prefix)   # untimed
-        ev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
-        torch.cuda.synchronize()
-        ev[0].record(stream)
-        cand, win, score = model.multi_query(grp, N, n_chunks, temperature, seed, mode=mode, prefix=prefix)
-        ev[1].record(stream)
-        torch.cuda.synchronize()
+        try:
+            model.multi_query(grp, N, n_chunks, temperature, seed, mode=mode, prefix=prefix)   # untimed
+            ev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+            torch.cuda.synchronize()
+            ev[0].record(stream)
+            cand, win, score = model.multi_query(grp, N, n_chunks, temperature, seed, mode=mode, prefix=prefix)
+            ev[1].record(stream)
+            torch.cuda.synchronize()
+        except hal.PhotonError as e:      # reported in the line; the rest of the bench goes on
+            out[name] = {"error": str(e)}
+            continue
         ms = ev[0].elapsed_time(ev[1])
         w = win.cpu()
         out[name] = {"ms": round(ms, 3), "answers_per_s": round(Q / (ms / 1e3), 2),

@@ -2331,13 +2331,9 @@ int photon_vanilla_free_cache(photon_vanilla_cache* c) {
 // ============================================================== teacher-forced scoring
 extern "C" {
 
-int photon_score(photon_model* m, const int32_t* d_tokens, int32_t B, int32_t T, float* d_out_logprob,
-                 void* stream) {
-  g_err.clear();
-  if (!m || !d_tokens || !d_out_logprob) return fail(PHOTON_ERR_ARG, "NULL argument");
-  if (m->vanilla) return fail(PHOTON_ERR_ARG, "a vanilla baseline model takes the photon_vanilla_* calls");
-  if (B <= 0 || T <= m->C || T % m->C)
-    return fail(PHOTON_ERR_ARG, "T = %d must be a multiple of C1*C2 = %d longer than one chunk", T, m->C);
+// Scores sequences [0, B) of d_tokens in one pass (arguments checked by photon_score).
+static int score_slice(photon_model* m, const int32_t* d_tokens, int32_t B, int32_t T, float* d_out_logprob,
+                       void* stream) {
   cudaStream_t s = (cudaStream_t)stream;
   const int d = m->d, V = m->V, C = m->C, C1 = m->C1, C2 = m->C2;
   const size_t es = m->es, hd = (size_t)m->H * m->dh;
@@ -2462,6 +2458,30 @@ int photon_score(photon_model* m, const int32_t* d_tokens, int32_t B, int32_t T,
   if (le == cudaSuccess) le = cudaStreamSynchronize(s);
   if (le != cudaSuccess) return fail(PHOTON_ERR_CUDA, "scoring failed: %s", cudaGetErrorString(le));
   if (herr) return fail(PHOTON_ERR_DEVICE_CHECK, "device check failed during scoring (code %d)", herr);
+  return PHOTON_OK;
+}
+
+int photon_score(photon_model* m, const int32_t* d_tokens, int32_t B, int32_t T, float* d_out_logprob,
+                 void* stream) {
+  g_err.clear();
+  if (!m || !d_tokens || !d_out_logprob) return fail(PHOTON_ERR_ARG, "NULL argument");
+  if (m->vanilla) return fail(PHOTON_ERR_ARG, "a vanilla baseline model takes the photon_vanilla_* calls");
+  if (B <= 0 || T <= m->C || T % m->C)
+    return fail(PHOTON_ERR_ARG, "T = %d must be a multiple of C1*C2 = %d longer than one chunk", T, m->C);
+  // The decoders run over (sequence, chunk, sub-chunk) groups, which the
+  // attention kernels index in a grid dimension of at most 65535 (times the
+  // query length where a split-K combine follows).  Whole sequences are
+  // scored a slice at a time so that a slice stays within it.
+  const long long K = T / m->C - 1, P = 2LL * m->C1 - 1;
+  const long long per_seq = K * m->C2 * std::max(1LL, std::min(P, 4LL));
+  constexpr long long kMaxGroups = 65535;
+  if (per_seq > kMaxGroups)
+    return fail(PHOTON_ERR_ARG, "T = %d is too long to score: at most %lld chunks per sequence", T,
+                kMaxGroups / ((long long)m->C2 * std::max(1LL, std::min(P, 4LL))) + 1);
+  const int bs = (int)std::min<long long>(B, kMaxGroups / per_seq);
+  for (int b0 = 0; b0 < B; b0 += bs)
+    RET(score_slice(m, d_tokens + (size_t)b0 * T, std::min(bs, B - b0), T,
+                    d_out_logprob + (size_t)b0 * (T - m->C), stream));
   return PHOTON_OK;
 }
 
