@@ -20,6 +20,9 @@ Contents:
                 pinned blocks.
   aggregate.py -- multi-query aggregation (majority vote, best-of-N by
                 teacher-forced log-likelihood) over groups of sampled rows.
+  hierarchy.py -- the same model for any number of levels L (L = 1: a
+                single-level block model; L = 2 reduces to photon.py; L >= 3:
+                deeper hierarchies), HierGen and RecGen.
 
 Every oracle function is pinned by CPU tests (tests/test_oracle_*.py) to
 facts that do not come from the oracle itself: published SplitMix64 test
