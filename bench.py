@@ -366,6 +366,19 @@ def run_gpu(args) -> None:
     dec_tokens = world * B * chunks * C * args.steps
     value = job_throughput(B * chunks * C * args.steps, world, decode_ms)
     gib = resident / 2 ** 30
+    # the method's own per-chunk roofline, and the fraction of it each measured rate reaches (per GPU)
+    peaks, peak_src = _peaks()
+    sroof = step_roofline(shape, wl, peaks)
+    sroof["recgen"]["frac"] = round(value / world / sroof["recgen"]["tok_s"], 4)
+    sroof["hiergen"]["frac"] = round(B * chunks * C / (hier_dec_ms / 1e3) / sroof["hiergen"]["tok_s"], 4)
+    sroof["prefill"]["frac"] = round(B * T * args.steps / (prefill_ms / 1e3) / sroof["prefill"]["tok_s"], 4)
+    sroof["peaks"]["source"] = peak_src
+    per_seq = (cinfo["kv_bytes"] + cinfo["workspace_bytes"]) / B
+    sroof["peak_batch"] = {"sequences": peak_batch(torch.cuda.get_device_properties(dev).total_memory,
+                                                   minfo["resident_bytes"], pre_kv, 0, per_seq),
+                           "bytes_per_sequence": int(per_seq),
+                           "covers": "device memory - resident weights - shared prefix, over one "
+                                     "sequence's RecGen KV and decode workspace"}
     line = {
         "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup,
@@ -387,6 +400,7 @@ def run_gpu(args) -> None:
                 "kv_gib": round((cinfo["kv_bytes"] + pre_kv) / 2 ** 30, 4),
                 "tok_s_per_gib_kv_only": round(value / world / ((cinfo["kv_bytes"] + pre_kv) / 2 ** 30), 1),
                 "per_gpu": True},
+        "step_roofline": sroof,
         "e2e": {"value": round(world * B * chunks * C * e2e_steps / (e2e_ms / 1e3), 1), "unit": UNIT,
                 "h2d_bytes_per_step": int(B * T * 4), "d2h_bytes_per_step": int(B * chunks * C * 4),
                 "covers": "H2D prompt + prefill + RecGen decode + D2H of the tokens"
@@ -424,6 +438,77 @@ def run_gpu(args) -> None:
     model.free()
     if world > 1:
         dist.destroy_process_group()
+
+
+def step_roofline(shape: dict, wl: dict, peaks: dict) -> dict:
+    """The method's own roofline per decode chunk and per prefill, counting
+    only the work the method has to do.
+
+    Bytes per RecGen chunk:
+    - every weight matrix a pass uses, once per pass.  That is the top step,
+      Chunker_2, both converters, Decoder_2, and C1 passes of the token
+      decoder and the head;
+    - the embedding rows the token decoder feeds back;
+    - the top KV read at the decode's mean key count, plus its append (a
+      shared prefix counts once).
+
+    HierGen adds the level-1 re-encode's weights and embedding rows and the
+    level-1 KV read and append.  Flops are 2*M*K*N over the GEMMs plus
+    4*rows*keys*d per attention layer of the coarse streams.  Prefill is
+    counted in flops, causal attention as half of the square.  Roofline time
+    is max(bytes / HBM, flops / sustained bf16 peak) from the measured
+    peaks.  Returns tok/s per GPU at that time and the terms behind it."""
+    V, d = shape["vocab"], shape["d_model"]
+    f = shape.get("mlp_mult", 4) * d
+    C1, C2 = shape["C1"], shape["C2"]
+    C = C1 * C2
+    L1, Lt, Ld1, Ld2 = shape["L1"], shape["Ltop"], shape["Ld1"], shape["Ld2"]
+    es = 2 if shape["dtype"] == "bf16" else 4
+    B, T = wl["batch"], wl["prompt_len"]
+    chunks = wl["decode_tokens"] // C
+    pre = wl.get("prefix_len", 0)
+    blk = 4 * d * d + 2 * f * d                      # weights of one block
+    bw, fl = peaks["hbm_gbs"] * 1e9, peaks["bf16_tflops_sustained"] * 1e12
+    w_rec = (Lt * blk + 2 * C2 * d * d + Ld2 * blk + C1 * d * d + C1 * (Ld1 * blk + V * d)) * es
+    w_rec += B * C2 * (C1 - 1) * d * es
+    n_top = T // C + (chunks + 1) / 2                # mean keys of a sequence's own top stream
+    kv_rec = 2 * Lt * (B * n_top + pre // C) * d * es + 2 * Lt * B * d * es
+    rows_tok = B * C2 * (2 * C1 - 1)                 # token-decoder rows over its C1 passes
+    f_rec = 2 * (B * blk * Lt + 2 * B * C2 * d * d + B * C2 * blk * Ld2 + B * C2 * C1 * d * d
+                 + rows_tok * blk * Ld1 + B * C * V * d) + 4 * B * (n_top + pre // C) * d * Lt
+    n_l1 = T // C1 + C2 * (chunks - 1) / 2 + (C2 + 1) / 2
+    b_hier = (C1 * d * d + L1 * blk) * es + B * C * d * es + 2 * L1 * (B * n_l1 + pre // C1) * d * es \
+        + 2 * L1 * B * C2 * d * es
+    f_hier = 2 * (B * C2 * C1 * d * d + B * C2 * blk * L1) + 4 * B * C2 * (n_l1 + pre // C1) * d * L1
+    n1, nt = T // C1, T // C
+    f_pre = (2 * B * T * d * d + 2 * B * n1 * blk * L1 + B * L1 * (2 * n1 * n1 + 4 * n1 * (pre // C1)) * d
+             + 2 * B * nt * C2 * d * d + 2 * B * nt * blk * Lt + B * Lt * (2 * nt * nt + 4 * nt * (pre // C)) * d)
+    b_pre = (B * T * d + C1 * d * d + L1 * blk + C2 * d * d + Lt * blk) * es \
+        + 2 * (L1 * B * n1 + Lt * B * nt) * d * es
+    t_rec = max((w_rec + kv_rec) / bw, f_rec / fl)
+    t_hier = max((w_rec + kv_rec + b_hier) / bw, (f_rec + f_hier) / fl)
+    t_pre = max(b_pre / bw, f_pre / fl)
+    return {
+        "recgen": {"bytes_per_chunk": int(w_rec + kv_rec), "weight_bytes": int(w_rec),
+                   "top_kv_read_bytes": int(kv_rec), "flops_per_chunk": int(f_rec),
+                   "bound": "hbm" if (w_rec + kv_rec) / bw >= f_rec / fl else "tensor",
+                   "tok_s": round(B * C / t_rec, 1)},
+        "hiergen": {"bytes_per_chunk": int(w_rec + kv_rec + b_hier), "flops_per_chunk": int(f_rec + f_hier),
+                    "coarse_kv_read_bytes": int(kv_rec + 2 * L1 * (B * n_l1 + pre // C1) * d * es),
+                    "bound": "hbm" if (w_rec + kv_rec + b_hier) / bw >= (f_rec + f_hier) / fl else "tensor",
+                    "tok_s": round(B * C / t_hier, 1)},
+        "prefill": {"flops": int(f_pre), "bytes": int(b_pre),
+                    "bound": "tensor" if f_pre / fl >= b_pre / bw else "hbm", "tok_s": round(B * T / t_pre, 1)},
+        "peaks": {"hbm_gbs": peaks["hbm_gbs"], "bf16_tflops_sustained": peaks["bf16_tflops_sustained"]},
+    }
+
+
+def peak_batch(hbm_bytes: int, weight_bytes: int, prefix_bytes: int, workspace_bytes: int,
+               per_sequence_bytes: float) -> int:
+    """Largest batch whose caches fit: (HBM - weights - shared prefix -
+    workspace) / bytes one sequence's cache holds."""
+    free = hbm_bytes - weight_bytes - prefix_bytes - workspace_bytes
+    return max(0, int(free // per_sequence_bytes)) if per_sequence_bytes > 0 else 0
 
 
 def kernel_sources_sha256() -> str:
