@@ -333,7 +333,7 @@ def run_gpu(args) -> None:
     # ---- multi-query aggregation: groups of nine sampled rows per prompt,
     # majority vote and best-of-N (photon_multi_query)
     mq = measure_multi_query(model, toks, chunks, stream, prefix=pre_cache)
-    mq_ms = [mq[k]["ms"] if isinstance(mq.get(k), dict) else 0.0 for k in ("vote", "best")]
+    mq_ms = [mq[k].get("ms", 0.0) if isinstance(mq.get(k), dict) else 0.0 for k in ("vote", "best")]
 
     # ---- same-kernel baseline: a vanilla token-level Transformer of the same
     # width and total depth over the same prompts (its KV covers every token)
