@@ -156,6 +156,24 @@ def _ptr(t) -> Optional[int]:
     return None if t is None else t.data_ptr()
 
 
+def _need(t, dtype, numel: int, name: str) -> None:
+    """Host-side check of a buffer handed to the library: a contiguous CUDA
+    tensor of `dtype` holding at least `numel` elements.  The C entry points
+    take raw pointers and sizes, so a wrong dtype or a short buffer would
+    otherwise be read or written out of bounds on the device."""
+    import torch
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name}: expected a torch tensor, got {type(t).__name__}")
+    if t.dtype != dtype:
+        raise ValueError(f"{name}: expected {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name}: must be contiguous")
+    if t.numel() < numel:
+        raise ValueError(f"{name}: holds {t.numel()} elements, needs {numel}")
+    if not t.is_cuda:
+        raise ValueError(f"{name}: must be a CUDA tensor")
+
+
 def config_struct(shape: dict) -> photon_config:
     """photon_config from a plain shape dict (keys of synth_inputs.MODEL_KEYS)."""
     c = photon_config()
@@ -203,8 +221,10 @@ class Model:
         [B, T - C] (photon_score; synchronising)."""
         import torch
         B, T = tokens.shape
+        _need(tokens, torch.int32, B * T, "tokens")
         if out is None:
-            out = torch.empty(B, T - self.C, dtype=torch.float32, device=tokens.device)
+            out = torch.empty(B, max(T - self.C, 0), dtype=torch.float32, device=tokens.device)
+        _need(out, torch.float32, B * max(T - self.C, 0), "out")
         _check(load_library().photon_score(self._h, _ptr(tokens), B, T, _ptr(out), _stream(stream)))
         return out
 
@@ -213,8 +233,8 @@ class Model:
         """photon_multi_query: prompts CUDA int32 [Q*N, T], groups of N consecutive rows.
         Returns (candidates int32 [Q*N, n_chunks*C], winners int32 [Q], scores fp64 [Q*N])."""
         import torch
-        assert prompts.is_cuda and prompts.dtype.itemsize == 4 and prompts.is_contiguous()
         rows, T = prompts.shape
+        _need(prompts, torch.int32, rows * T, "prompts")
         if N <= 0 or rows % N:
             raise ValueError(f"{rows} rows do not form groups of N = {N}")
         Q = rows // N
@@ -240,8 +260,9 @@ class Model:
     def prefill(self, tokens, mode: int, max_new_chunks: int, prefix: "Cache" = None,
                 stream=None) -> "Cache":
         """tokens: CUDA int32 tensor [B, T] (contiguous)."""
-        assert tokens.is_cuda and tokens.dtype.itemsize == 4 and tokens.is_contiguous()
+        import torch
         B, T = tokens.shape
+        _need(tokens, torch.int32, B * T, "tokens")
         h = ctypes.c_void_p()
         _check(load_library().photon_prefill(self._h, None if prefix is None else prefix._h,
                                              _ptr(tokens), B, T, mode, max_new_chunks,
@@ -264,21 +285,38 @@ class Cache:
                     force_a=None, stream=None) -> None:
         """One top-level chunk: out_tokens CUDA int32 [B, C1*C2]; optional fp32
         logits [B, C1*C2, vocab]; optional teacher-forced tokens / forced A."""
+        import torch
+        self._need_step(out_tokens, out_logits)
+        if force_tokens is not None:
+            _need(force_tokens, torch.int32, self.B * self.model.C, "force_tokens")
+        if force_a is not None:
+            _need(force_a, self.model.torch_dtype, self.B * self.model.C2 * self.model.d_model, "force_a")
         _check(load_library().photon_decode_step_ex(
             self.model._h, self._h, mode, _ptr(out_tokens), _ptr(out_logits),
             _ptr(force_tokens), _ptr(force_a), _stream(stream)))
 
+    def _need_step(self, out_tokens, out_logits) -> None:
+        import torch
+        C = self.model.C
+        _need(out_tokens, torch.int32, self.B * C, "out_tokens")
+        if out_logits is not None:
+            _need(out_logits, torch.float32, self.B * C * self.model.vocab, "out_logits")
+
     def step_rec(self, out_tokens, out_logits=None, stream=None) -> None:
+        self._need_step(out_tokens, out_logits)
         _check(load_library().photon_decode_step_rec(self.model._h, self._h, _ptr(out_tokens),
                                                      _ptr(out_logits), _stream(stream)))
 
     def step_hier(self, out_tokens, out_logits=None, stream=None) -> None:
+        self._need_step(out_tokens, out_logits)
         _check(load_library().photon_decode_step_hier(self.model._h, self._h, _ptr(out_tokens),
                                                       _ptr(out_logits), _stream(stream)))
 
     def decode_rec_chunks(self, n_chunks: int, out_tokens, stream=None) -> None:
         """n RecGen chunks in one call; out_tokens int32 [B, n_chunks * C] on the device
         (each chunk's token decoder overlapped with the next chunk's main chain)."""
+        import torch
+        _need(out_tokens, torch.int32, self.B * max(n_chunks, 0) * self.model.C, "out_tokens")
         _check(load_library().photon_decode_rec_chunks(self.model._h, self._h, n_chunks,
                                                        _ptr(out_tokens), _stream(stream)))
 
@@ -343,7 +381,9 @@ class VanillaModel(Model):
 
     def prefill(self, tokens, max_new_tokens: int, stream=None) -> "VanillaCache":
         """tokens: CUDA int32 [B, T]; the first T-1 enter the KV cache."""
+        import torch
         B, T = tokens.shape
+        _need(tokens, torch.int32, B * T, "tokens")
         h = ctypes.c_void_p()
         _check(load_library().photon_vanilla_prefill(self._h, _ptr(tokens), B, T, max_new_tokens,
                                                      _stream(stream), ctypes.byref(h)))
@@ -357,6 +397,12 @@ class VanillaCache:
     def decode_step(self, out_tokens, out_logits=None, force_tokens=None, stream=None) -> None:
         """One token per sequence: out_tokens CUDA int32 [B]; optional fp32 logits [B, vocab];
         optional teacher-forced tokens [B] (entries < 0 not forced)."""
+        import torch
+        _need(out_tokens, torch.int32, self.B, "out_tokens")
+        if out_logits is not None:
+            _need(out_logits, torch.float32, self.B * self.model.vocab, "out_logits")
+        if force_tokens is not None:
+            _need(force_tokens, torch.int32, self.B, "force_tokens")
         _check(load_library().photon_vanilla_decode_step(self.model._h, self._h, _ptr(out_tokens),
                                                          _ptr(out_logits), _ptr(force_tokens),
                                                          _stream(stream)))
@@ -375,7 +421,11 @@ class VanillaCache:
 def sample_logits(logits, temperature: float, top_p: float, seed: int, chunk, C1: int, C2: int, i: int,
                   out, stream=None) -> None:
     """photon_sample_logits: logits CUDA fp32 [rows, V]; chunk CUDA int32 [1]; out int32 [rows]."""
+    import torch
     rows, V = logits.shape
+    _need(logits, torch.float32, rows * V, "logits")
+    _need(chunk, torch.int32, 1, "chunk")
+    _need(out, torch.int32, rows, "out")
     _check(load_library().photon_sample_logits(_ptr(logits), rows, V, float(temperature), float(top_p),
                                                int(seed), _ptr(chunk), C1, C2, i, _ptr(out), _stream(stream)))
 
@@ -391,6 +441,14 @@ def aggregate(mode: int, N: int, choice, cand=None, logprob=None, span_begin: in
         raise ValueError(f"{rows} rows do not form groups of N = {N}")
     if span_len is None:
         span_len = L - span_begin
+    import torch
+    if cand is not None:
+        _need(cand, torch.int32, rows * L, "cand")
+    if logprob is not None:
+        _need(logprob, torch.float32, rows * L, "logprob")
+    _need(choice, torch.int32, rows // N, "choice")
+    if score is not None:
+        _need(score, torch.float64, rows, "score")
     _check(load_library().photon_aggregate(mode, _ptr(cand), _ptr(logprob), rows // N, N, L, span_begin,
                                            span_len, _ptr(choice), _ptr(score), _stream(stream)))
 

@@ -66,3 +66,25 @@ def test_aggregation_host_checks_without_a_device():
         assert lib.photon_aggregate(mode, None, None, Q, N, L, b, n, None, None, None) == -1, (mode, Q, N, L, b, n)
         assert lib.photon_last_error() != b""
     assert lib.photon_multi_query(None, None, None, 1, 9, 16, 1, 1.0, 1.0, 0, 0, None, None, None, None) == -1
+
+
+def test_binding_rejects_bad_buffers_on_the_host():
+    # dtype, layout and size are checked before any pointer reaches the library
+    import torch
+    need = hal._need
+    with pytest.raises(TypeError):
+        need([1, 2], torch.int32, 2, "x")
+    with pytest.raises(ValueError, match="expected torch.float32"):
+        need(torch.zeros(4, dtype=torch.float16), torch.float32, 4, "x")
+    with pytest.raises(ValueError, match="contiguous"):
+        need(torch.zeros(4, 4, dtype=torch.int32).t(), torch.int32, 16, "x")
+    with pytest.raises(ValueError, match="needs 5"):
+        need(torch.zeros(4, dtype=torch.int32), torch.int32, 5, "x")
+    with pytest.raises(ValueError, match="CUDA"):
+        need(torch.zeros(4, dtype=torch.int32), torch.int32, 4, "x")
+    with pytest.raises(ValueError, match="logprob: expected torch.float32"):
+        hal.aggregate(hal.AGG_BEST, 3, torch.zeros(2, dtype=torch.int32),
+                      logprob=torch.zeros(6, 4, dtype=torch.float16))
+    with pytest.raises(ValueError, match="groups of N"):
+        hal.aggregate(hal.AGG_VOTE, 4, torch.zeros(2, dtype=torch.int32),
+                      cand=torch.zeros(6, 4, dtype=torch.int32))
