@@ -236,6 +236,36 @@ class HierOracle:
         st.tokens.extend(int(t) for t in used)
         return HierStep(tokens=own, used=used, logits=logits, a_hat=a_hat, a=a)
 
+    # -- teacher-forced scoring -------------------------------------------------
+    def score(self, tokens):
+        """Log-probability of every token after the first top chunk under
+        teacher forcing (explainer, quality section).  The bottom-up pass
+        encodes the true tokens.  Top output o_k conditions top chunk k + 1
+        down every level, and each decoder reads the true tokens of its
+        sub-chunk.  Returns (log-probabilities [T - C], logits [T - C, V])."""
+        cfg = self.cfg
+        tokens = np.asarray(tokens, dtype=np.int64)
+        T = tokens.shape[0]
+        if T <= cfg.C or T % cfg.C:
+            raise ValueError("the prompt must be a multiple of C_1 * ... * C_L longer than one top chunk")
+        s = self.w["embed"][tokens]
+        for l in range(1, cfg.L + 1):
+            s, _ = self.encode(l, s, 0, None)
+        logits = []
+        for k in range(1, T // cfg.C):
+            force = tokens[k * cfg.C:(k + 1) * cfg.C]
+            out: list = []
+            if cfg.L == 1:
+                self._emit(1, s[k - 1], force, out)
+            else:
+                for row in self.reconstruct(cfg.L, s[k - 1]):
+                    self._emit(cfg.L - 1, row, force, out)
+            logits.extend(lg for _, _, lg in out)
+        logits = np.stack(logits)
+        z = logits - logits.max(axis=1, keepdims=True)
+        logp = z - np.log(np.exp(z).sum(axis=1, keepdims=True))
+        return logp[np.arange(T - cfg.C), tokens[cfg.C:]], logits
+
     # -- full recomputation (pins the incremental paths) --------------------------
     def full_top(self, top_inputs):
         """Top encoder over a whole list of coarse inputs, from scratch."""

@@ -166,3 +166,35 @@ def test_three_level_tokens_come_out_in_time_order():
             for i in range(C1):
                 lg = orc.token_logits(cond, [int(x) for x in step.used[base:base + i]])
                 np.testing.assert_allclose(step.logits[base + i], lg, rtol=0, atol=1e-12)
+
+
+def test_two_level_scoring_reduces_to_the_two_level_oracle():
+    h, p = HierOracle(TWO_H, 5), PhotonOracle(TWO, 5)
+    toks = _prompt(TWO.C, 4, 8)
+    lh, gh = h.score(toks)
+    lp, gp = p.score(toks)
+    np.testing.assert_allclose(gh, gp, rtol=0, atol=1e-12)
+    np.testing.assert_allclose(lh, lp, rtol=0, atol=1e-12)
+
+
+@pytest.mark.parametrize("cfg", [THREE, ONE], ids=["L3", "L1"])
+def test_scoring_follows_the_chain_rule_of_incremental_decoding(cfg):
+    # chunk k's scores = log-softmax of the decode step after a HierGen prefill of
+    # chunks 0..k-1, teacher-forced on chunk k's true tokens
+    orc = HierOracle(cfg, 14)
+    toks = _prompt(cfg.C, 4, 9)
+    lp, _ = orc.score(toks)
+    assert lp.shape == (3 * cfg.C,) and np.all(lp < 0)
+    for k in (1, 3):
+        st = orc.prefill(toks[:k * cfg.C], "hier")
+        chunk = toks[k * cfg.C:(k + 1) * cfg.C]
+        lg = orc.decode_step(st, "hier", force_tokens=chunk).logits
+        z = lg - lg.max(axis=1, keepdims=True)
+        ref = (z - np.log(np.exp(z).sum(axis=1, keepdims=True)))[np.arange(cfg.C), chunk]
+        np.testing.assert_allclose(lp[(k - 1) * cfg.C:k * cfg.C], ref, rtol=0, atol=1e-12)
+    # a token's score depends on the tokens before it only
+    q = toks.copy()
+    q[-1] = (q[-1] + 1) % cfg.vocab
+    lq, _ = orc.score(q)
+    np.testing.assert_array_equal(lq[:-1], lp[:-1])
+    assert lq[-1] != lp[-1]
