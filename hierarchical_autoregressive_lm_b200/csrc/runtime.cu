@@ -818,6 +818,10 @@ static int prefill_impl(photon_model* m, const photon_cache* prefix, const int32
   if (m->vanilla) return fail(PHOTON_ERR_ARG, "a vanilla baseline model takes the photon_vanilla_* calls");
   if (!d_tokens) return fail(PHOTON_ERR_ARG, "tokens pointer is NULL");
   if (B <= 0) return fail(PHOTON_ERR_ARG, "batch must be positive");
+  // the attention kernels index (sequence, sub-chunk) groups in a grid
+  // dimension of at most 65535
+  if ((long long)B * m->C2 > 65535)
+    return fail(PHOTON_ERR_ARG, "batch %d too large: B * C2 must be at most 65535", B);
   if (T <= 0 || T % m->C) return fail(PHOTON_ERR_ARG, "T = %d is not a positive multiple of C1*C2 = %d", T, m->C);
   if (mode != PHOTON_MODE_HIER && mode != PHOTON_MODE_REC) return fail(PHOTON_ERR_ARG, "unknown mode %d", mode);
   if (max_new_chunks < 0) return fail(PHOTON_ERR_ARG, "max_new_chunks must be >= 0");
@@ -2138,6 +2142,7 @@ int photon_vanilla_prefill(photon_model* m, const int32_t* d_tokens, int32_t B, 
   if (!m->vanilla) return fail(PHOTON_ERR_ARG, "not a vanilla baseline model");
   if (!d_tokens) return fail(PHOTON_ERR_ARG, "tokens pointer is NULL");
   if (B <= 0 || T < 2 || max_new_tokens < 0) return fail(PHOTON_ERR_ARG, "need B > 0, T >= 2, max_new >= 0");
+  if (B > 65535) return fail(PHOTON_ERR_ARG, "batch %d too large: at most 65535 (attention grid limit)", B);
   cudaStream_t s = (cudaStream_t)stream;
   const int d = m->d, V = m->V, H = m->H, dh = m->dh, L = m->L_van;
   const size_t es = m->es;

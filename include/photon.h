@@ -116,6 +116,7 @@ PHOTON_API int photon_free_model(photon_model* m);
  *         prefix must outlive it.
  *   out: receives the new cache.  Invalid token ids set the device error
  *         word (see photon_cache_info).
+ *   B * C2 must be at most 65535 (the attention kernels' grid limit).
  * Errors: ERR_ARG, ERR_OOM, ERR_CUDA. */
 PHOTON_API int photon_prefill(photon_model* m, const photon_cache* prefix, const int32_t* d_tokens,
                    int32_t B, int32_t T, int32_t mode, int32_t max_new_chunks, void* stream,
@@ -435,6 +436,7 @@ PHOTON_API int photon_vanilla_init(const photon_vanilla_config* cfg, uint64_t se
 /* Prefill of B prompts d_tokens [B, T] (device, row-major, T >= 2): the
  * first T-1 tokens of each prompt enter the KV cache; the last one is the
  * input of the first decode step.  Room for max_new_tokens decode steps.
+ * B must be at most 65535 (the attention kernels' grid limit).
  * Errors: ERR_ARG, ERR_OOM, ERR_CUDA. */
 PHOTON_API int photon_vanilla_prefill(photon_model* m, const int32_t* d_tokens, int32_t B, int32_t T,
                                       int32_t max_new_tokens, void* stream, photon_vanilla_cache** out);
