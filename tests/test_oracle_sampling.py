@@ -119,3 +119,24 @@ def test_top_p_draws_follow_the_renormalised_nucleus():
     k = mask.sum()
     chi2 = float(((counts[mask] - n * q[mask]) ** 2 / (n * q[mask])).sum())
     assert chi2 < {1: 0.0, 2: 15.1, 3: 18.4, 4: 21.1, 5: 23.5}[k] + 1e-9, (chi2, counts / n, q)
+
+
+def test_fmix32_is_murmurhash3s_finaliser():
+    # MurmurHash3_x86_32 of one 4-byte key is fmix32 applied to the mixed block
+    # xor the length; scikit-learn ships an independent implementation of it
+    from sklearn.utils import murmurhash3_32
+    M = 0xFFFFFFFF
+
+    def rotl(x, r):
+        return ((x << r) | (x >> (32 - r))) & M
+
+    def block(key, seed):            # the algorithm's body for a single 32-bit block
+        k = rotl((key * 0xCC9E2D51) & M, 15) * 0x1B873593 & M
+        return ((rotl(seed ^ k, 13) * 5 + 0xE6546B64) & M) ^ 4
+
+    rng = np.random.default_rng(3)
+    keys = [0, 1, 0x7FFFFFFF, 0x80000000, M] + [int(x) for x in rng.integers(0, 1 << 32, size=40)]
+    for key in keys:
+        for seed in (0, 1, 0x9747B28C):
+            want = murmurhash3_32(key - (1 << 32) if key >= 1 << 31 else key, seed=seed, positive=True)
+            assert int(S.fmix32(np.uint32(block(key, seed)))) == want, (key, seed)
