@@ -30,6 +30,11 @@ the cache has generated (chunk * C1*C2 + sub-chunk * C1 + position), v the
 vocabulary id.  Ties of the perturbed values go to the lowest id, as for
 greedy decoding.
 
+The hash finaliser is pinned to MurmurHash3 and the 64-bit mixes to SplitMix64
+(tests).  The fold of the 64-bit key to 32 bits is this project's own choice.
+Nothing outside the code fixes it (parity unpinned for that step); the GPU's
+draws are compared with it.
+
 Nucleus (top-p) sampling, a common refinement the pages do not mention
 either, restricts the draw to the smallest set of most probable tokens whose
 probability reaches p (ties at its edge included) and renormalises; the
