@@ -339,8 +339,12 @@ PHOTON_API int photon_attn_decode_noalloc(int32_t dtype, const void* d_q, const 
  * the token decoder reads the chunk's true tokens (one causal pass per
  * sub-chunk).  The first chunk has no conditioning and is not scored.
  * Synchronising (it reports device checks).  Allocates its temporaries from
- * the library's pool.  Errors: ERR_ARG, ERR_OOM, ERR_CUDA, ERR_DEVICE_CHECK
- * (a token id outside the vocabulary). */
+ * the library's pool.  Long batches are scored a slice of whole sequences at
+ * a time, so that the decoders' (sequence, chunk, sub-chunk) groups stay
+ * within the attention kernels' grid limit.  One sequence may hold at most
+ * 65535 / (C2 * min(2*C1 - 1, 4)) + 1 chunks.  Errors: ERR_ARG (including
+ * a longer sequence), ERR_OOM, ERR_CUDA, ERR_DEVICE_CHECK (a token id
+ * outside the vocabulary). */
 PHOTON_API int photon_score(photon_model* m, const int32_t* d_tokens, int32_t B, int32_t T,
                             float* d_out_logprob, void* stream);
 
