@@ -135,6 +135,24 @@ def test_c1_error_paths(model):
     assert model.info()["live_caches"] == 0
 
 
+def test_c1_empty_and_oversized_inputs(model):
+    # rejected on the host before any launch: an empty batch, an empty prompt,
+    # scoring either, and a batch past the attention grid limit (B * C2 > 65535)
+    for shape in ((0, 64), (1, 0)):
+        t = torch.zeros(shape, dtype=torch.int32, device="cuda")
+        with pytest.raises(hal.PhotonError) as e:
+            model.prefill(t, hal.MODE_REC, 1)
+        assert e.value.code == -1
+        with pytest.raises(hal.PhotonError) as e:
+            model.score(t)
+        assert e.value.code == -1
+    big = torch.zeros(65536 // CFG.C2, CFG.C, dtype=torch.int32, device="cuda")
+    with pytest.raises(hal.PhotonError) as e:
+        model.prefill(big, hal.MODE_REC, 1)
+    assert e.value.code == -1 and "65535" in str(e.value)
+    assert model.info()["live_caches"] == 0
+
+
 def test_c1_residency(model):
     toks = torch.from_numpy(prompt_tokens("c1")).cuda()
     r = model.prefill(toks, hal.MODE_REC, 1)

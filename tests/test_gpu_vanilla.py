@@ -111,3 +111,14 @@ def test_vanilla_graph_replay_equals_eager_and_kind_checks():
                                                      None, hal.ctypes.byref(hal.ctypes.c_void_p())))
     assert err.value.code == -1
     model.free()
+
+
+def test_vanilla_rejects_empty_and_oversized_batches():
+    model = hal.VanillaModel(F32, 5)
+    for shape in ((0, 40), (2, 1), (65536, 2)):
+        t = torch.zeros(shape, dtype=torch.int32, device="cuda")
+        with pytest.raises(hal.PhotonError) as e:
+            model.prefill(t, 4)
+        assert e.value.code == -1
+    assert model.info()["live_caches"] == 0
+    model.free()
