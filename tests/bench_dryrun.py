@@ -120,6 +120,11 @@ torch.cuda.get_device_properties = lambda dev: types.SimpleNamespace(uuid="fake"
 torch.cuda.nvtx.range_push = lambda *a, **k: None
 torch.cuda.nvtx.range_pop = lambda *a, **k: None
 torch.Tensor.pin_memory = lambda self: self
+# more than one rank (torchrun): the same collectives over gloo on the host
+import torch.distributed as dist  # noqa: E402
+_init = dist.init_process_group
+dist.init_process_group = lambda backend=None, **kw: _init(
+    "gloo", **{k: v for k, v in kw.items() if k != "device_id"})
 hal.Model = FakeModel
 hal.launch_count = lambda: 0
 roof = lambda *a, **k: {"bound": "hbm", "achieved": 1.0, "peak": 2.0, "unit": "GB/s", "frac": 0.5}
@@ -128,9 +133,11 @@ bench.measure_attn_roofline = roof
 bench.measure_prefill_roofline = roof
 bench.ClockSampler = FakeClock
 
-args = argparse.Namespace(gpus=1, steps=2, warmup=3, workload=WL, impl="photon", cpu_budget=1.0,
+args = argparse.Namespace(gpus=int(os.environ.get("WORLD_SIZE", "1")), steps=2, warmup=3, workload=WL, impl="photon", cpu_budget=1.0,
                           no_cpu_baseline=True, no_vanilla=True, decode_api="chunks", only_roofline=False)
 buf = io.StringIO()
 with contextlib.redirect_stdout(buf):
     bench.run_gpu(args)
-print(buf.getvalue().strip().splitlines()[-1])
+out = buf.getvalue().strip().splitlines()
+if out:                       # rank 0 prints the line; the other ranks print nothing
+    print(out[-1])

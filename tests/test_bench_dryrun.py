@@ -1,7 +1,8 @@
 """bench.py's GPU arm run on the CPU with the library and CUDA calls faked
 (tests/bench_dryrun.py, in a subprocess): the JSON line keeps the contract's
-keys, and a library error inside the multi-query measurement is recorded in
-the line instead of ending the run."""
+keys, a library error inside the multi-query measurement is recorded in the
+line instead of ending the run, and under torchrun with two gloo ranks the
+line reports the whole job (max over ranks) from rank 0 alone."""
 import json
 import os
 import subprocess
@@ -38,3 +39,24 @@ def test_bench_line_survives_a_library_error(mode, workload):
     for part in ("recgen", "hiergen", "prefill"):
         assert sr[part]["tok_s"] > 0 and sr[part]["frac"] > 0
     assert sr["peak_batch"]["sequences"] > 0 and sr["peaks"]["source"] in ("measured", "fallback")
+
+
+def test_bench_line_with_two_ranks():
+    # torchrun with two gloo ranks: max over ranks, whole-job throughput, one line from rank 0
+    import socket
+    s = socket.socket()
+    s.bind(("127.0.0.1", 0))
+    port = s.getsockname()[1]
+    s.close()
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes", "1", "--nproc-per-node", "2",
+           "--master-addr", "127.0.0.1", "--master-port", str(port),
+           os.path.join(HERE, "bench_dryrun.py"), "ok", "c2"]
+    r = subprocess.run(cmd, capture_output=True, text=True, timeout=300)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [l for l in r.stdout.splitlines() if l.startswith("{")]
+    assert len(lines) == 1
+    two = json.loads(lines[0])
+    one = _line("ok", "c2")
+    assert two["n_gpus"] == 2 and two["config"]["parallelism"] == "dp2"
+    assert abs(two["value"] / one["value"] - 2.0) < 1e-9            # the same per-rank work on each rank
+    assert two["multi_query"]["vote"]["answers_per_s"] == 2 * one["multi_query"]["vote"]["answers_per_s"]
