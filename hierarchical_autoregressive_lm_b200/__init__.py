@@ -16,7 +16,7 @@ import os
 from typing import Optional
 
 __all__ = ["PhotonError", "Model", "Cache", "load_library", "LIB_PATH", "MODE_HIER",
-           "MODE_REC", "STATE", "launch_count", "gemm", "gemm_rmsnorm", "attn_decode", "attn_decode_noalloc", "config_struct", "EXPORTED",
+           "MODE_REC", "STATE", "launch_count", "gemm", "gemm_rmsnorm", "attn_decode", "attn_decode_noalloc", "attn_decode_scratch_bytes", "config_struct", "EXPORTED",
            "AGG_VOTE", "AGG_BEST", "aggregate"]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libphoton.so")
@@ -35,7 +35,7 @@ EXPORTED = ("photon_init_weights", "photon_free_model", "photon_prefill",
             "photon_free_cache", "photon_cache_set_sampling", "photon_cache_set_top_p",
             "photon_sample_logits", "photon_cache_info", "photon_model_info",
             "photon_export_weight", "photon_export_state", "photon_gemm", "photon_gemm_rmsnorm",
-            "photon_attn_decode", "photon_attn_decode_noalloc", "photon_score", "photon_aggregate",
+            "photon_attn_decode", "photon_attn_decode_scratch_bytes", "photon_attn_decode_noalloc", "photon_score", "photon_aggregate",
             "photon_multi_query", "photon_vanilla_init",
             "photon_vanilla_prefill", "photon_vanilla_decode_step", "photon_vanilla_cache_info",
             "photon_vanilla_free_cache", "photon_launch_count", "photon_last_error")
@@ -124,8 +124,9 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "photon_export_state": [P, I32, I32, P, SZ, ctypes.POINTER(SZ), P],
         "photon_gemm": [I32, P, I64, P, I64, I32, I32, I32, P, I64, I32, I32, I32, P],
         "photon_gemm_rmsnorm": [P, I64, P, ctypes.c_float, P, I64, I32, I32, I32, P, I64, P],
-        "photon_attn_decode": [I32, P, P, P, I32, I32, I32, I32, I32, I32, P, P],
-        "photon_attn_decode_noalloc": [I32, P, P, P, I32, I32, I32, I32, I32, I32, P, P],
+        "photon_attn_decode": [I32, P, P, P, I32, I32, I32, I32, I32, I32, P, P, P],
+        "photon_attn_decode_noalloc": [I32, P, P, P, I32, I32, I32, I32, I32, I32, P, P, P],
+        "photon_attn_decode_scratch_bytes": [I32, I32, I32, I32, I32, I32, I32, P],
     }
     for name, args in sig.items():
         fn = getattr(L, name)
@@ -478,20 +479,45 @@ def gemm_rmsnorm(x, g, W, C, eps: float = 1e-6, stream=None) -> None:
                                               _stream(stream)))
 
 
-def attn_decode_noalloc(q, k, v, q_len: int, p0: int, out, stream=None) -> None:
+def _attn_bufs(q, k, v, q_len: int, out, err):
+    import torch
+    dt = 0 if q.dtype == torch.float32 else 1
+    if k.dim() != 4:
+        raise ValueError("k, v: expected [G, H, cap, head_dim]")
+    G, H, cap, dh = k.shape
+    _need(k, q.dtype, G * H * cap * dh, "k")
+    _need(v, q.dtype, G * H * cap * dh, "v")
+    _need(q, q.dtype, G * q_len * H * dh, "q")
+    _need(out, q.dtype, G * q_len * H * dh, "out")
+    if err is not None:
+        _need(err, torch.int32, 1, "err")
+    return dt, G, H, cap, dh
+
+
+def attn_decode_noalloc(q, k, v, q_len: int, p0: int, out, stream=None, err=None) -> None:
     """attn_decode through the allocation-free entry point (fixed 256 KiB scratch
-    inside the library; for callers whose memory is owned by someone else)."""
-    import torch
-    dt = 0 if q.dtype == torch.float32 else 1
-    G, H, cap, dh = k.shape
+    inside the library; for callers whose memory is owned by someone else).
+    err: optional int32 CUDA tensor that receives a nonzero code if a bounded
+    device wait runs out."""
+    dt, G, H, cap, dh = _attn_bufs(q, k, v, q_len, out, err)
     _check(load_library().photon_attn_decode_noalloc(dt, _ptr(q), _ptr(k), _ptr(v), G, H, dh,
-                                                     cap, q_len, p0, _ptr(out), _stream(stream)))
+                                                     cap, q_len, p0, _ptr(out), _ptr(err),
+                                                     _stream(stream)))
 
 
-def attn_decode(q, k, v, q_len: int, p0: int, out, stream=None) -> None:
-    """Split-K decode attention: k, v [G, H, cap, dh]; q, out [G*q_len, H*dh]."""
-    import torch
-    dt = 0 if q.dtype == torch.float32 else 1
-    G, H, cap, dh = k.shape
+def attn_decode(q, k, v, q_len: int, p0: int, out, stream=None, err=None) -> None:
+    """Split-K decode attention: k, v [G, H, cap, dh]; q, out [G*q_len, H*dh].
+    err: optional int32 CUDA tensor that receives a nonzero code if a bounded
+    device wait runs out."""
+    dt, G, H, cap, dh = _attn_bufs(q, k, v, q_len, out, err)
     _check(load_library().photon_attn_decode(dt, _ptr(q), _ptr(k), _ptr(v), G, H, dh, cap, q_len,
-                                             p0, _ptr(out), _stream(stream)))
+                                             p0, _ptr(out), _ptr(err), _stream(stream)))
+
+
+def attn_decode_scratch_bytes(dtype_code: int, G: int, H: int, head_dim: int, cap: int, q_len: int,
+                              p0: int) -> int:
+    """Split scratch (bytes) the decode attention plans for this shape; 0 when it needs none."""
+    out = ctypes.c_uint64(0)
+    _check(load_library().photon_attn_decode_scratch_bytes(dtype_code, G, H, head_dim, cap, q_len, p0,
+                                                           ctypes.byref(out)))
+    return int(out.value)

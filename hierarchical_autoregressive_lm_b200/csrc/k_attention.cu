@@ -559,16 +559,7 @@ DecPlan dec_plan(const AttnArgs& a) {
 // pairs leave SMs idle; the chunked path splits their keys instead), a long
 // cache (planned key count >= PHOTON_ATTN_STREAM_MIN_KEYS, default 768; 0
 // turns the path off), and 16-byte aligned rows for the bulk copies.
-static int sm_count() {
-  static int sms = 0;
-  if (!sms) {
-    int dev = 0;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    if (sms <= 0) sms = 1;
-  }
-  return sms;
-}
+static int sm_count() { return device_sm_count(); }
 static int stream_min_keys() {
   static const int v = [] {
     const char* e = getenv("PHOTON_ATTN_STREAM_MIN_KEYS");
@@ -588,13 +579,14 @@ bool stream_attn_ok(int dt, const AttnArgs& a) {
 template <int DH>
 void run_stream(const AttnArgs& a, int* err, cudaStream_t s) {
   constexpr int kSmem = (int)StreamCfg<DH>::kRing;
-  static int per_sm = 0;
-  if (!per_sm) {
+  static PerDevice cache;
+  const int per_sm = cache.get([] {
+    int per = 0;
     cudaFuncSetAttribute(k_attn_decode_stream<DH>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
-    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k_attn_decode_stream<DH>,
-                                                  32 * (kStreamWarps + 1), kSmem);
-    if (per_sm < 1) per_sm = 1;
-  }
+    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per, k_attn_decode_stream<DH>, 32 * (kStreamWarps + 1),
+                                                  kSmem);
+    return per < 1 ? 1 : per;
+  });
   // every CTA gets the same number of pairs (the last one possibly fewer)
   const long long pairs = (long long)a.G * a.H;
   const long long resident = (long long)sm_count() * per_sm;
@@ -607,12 +599,12 @@ void run_stream(const AttnArgs& a, int* err, cudaStream_t s) {
 template <typename T, int DH, int QMAX, int W>
 void run_decode_w(const AttnArgs& a, const DecPlan& p, float* part, int* err, cudaStream_t s) {
   constexpr int kRingBytes = W * kDecStages * 2 * kDecU * kDecSPL * 32 * 16;
-  static bool configured = false;
-  if (!configured) {
+  static PerDevice configured;
+  configured.get([] {
     cudaFuncSetAttribute(k_attn_decode<T, DH, QMAX, W>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                          kRingBytes);
-    configured = true;
-  }
+    return 1;
+  });
   dim3 grid(p.splits, a.H, a.G);
   launch_kernel(k_attn_decode<T, DH, QMAX, W>, grid, 32 * W, kRingBytes, s, a, p.chunk, p.splits,
                 part, err);

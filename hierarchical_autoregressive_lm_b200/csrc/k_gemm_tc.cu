@@ -1095,12 +1095,12 @@ void run_tc(const CUtensorMap& ma, const CUtensorMap& mb, int grid_a, int grid_b
             int M, int N, int nkb, int kbs, const Epilogue& ep, float* part, int* counters,
             const void* w_ptr, long long w_ld_bytes, int* err, cudaStream_t s) {
   using Cfg = TcCfg<BN, STAGES>;
-  static bool configured = false;
-  if (!configured) {
+  static PerDevice configured;
+  configured.get([] {
     cudaFuncSetAttribute(k_gemm_tc<BN, STAGES, SWAP, SAMPLE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                          Cfg::kSmemBytes);
-    configured = true;
-  }
+    return 1;
+  });
   dim3 grid(grid_a, grid_b, splits);
   launch_kernel(k_gemm_tc<BN, STAGES, SWAP, SAMPLE>, grid, 128, Cfg::kSmemBytes, s, ma, mb, M, N, nkb, kbs,
                 ep, part, counters, static_cast<const char*>(w_ptr), w_ld_bytes, err);
@@ -1110,15 +1110,13 @@ template <int BN, int STAGES, bool SAMPLE = false>
 void run_tc_persist(const CUtensorMap& ma, const CUtensorMap& mb, int M, int N, int nkb,
                     const Epilogue& ep, int nt_major, int* err, cudaStream_t s) {
   using Cfg = TcCfg<BN, STAGES>;
-  static int sms = 0;
-  if (!sms) {
+  static PerDevice configured;
+  configured.get([] {
     cudaFuncSetAttribute(k_gemm_tc_persist<BN, STAGES, SAMPLE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                          Cfg::kSmemBytes);
-    int dev = 0;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    if (sms <= 0) sms = 148;
-  }
+    return 1;
+  });
+  const int sms = device_sm_count();
   const int tiles_n = (N + BN - 1) / BN;
   const int n_tiles = ((M + kBM - 1) / kBM) * tiles_n;
   const int grid = n_tiles < sms ? n_tiles : sms;
@@ -1126,16 +1124,14 @@ void run_tc_persist(const CUtensorMap& ma, const CUtensorMap& mb, int M, int N, 
                 M, N, nkb, tiles_n, n_tiles, nt_major, ep, err);
 }
 
-// How many clusters of k_gemm_dec<BN, S, STAGES> can be resident at once
-// (0 if the cluster shape cannot be launched).  Host-side occupancy query,
-// made once per instance.
 // How many clusters of k_gemm_dec<BN, S, STAGES, NORM> can be resident at
 // once (0 if the cluster shape cannot be launched).  Host-side occupancy
-// query, made once per instance; it also sets the instance's attributes.
+// query, made once per instance and device; it also sets the instance's
+// attributes.
 template <int BN, int S, int STAGES, bool NORM>
 int dec_max_clusters() {
-  static int n = -1;
-  if (n < 0) {
+  static PerDevice cache;
+  return cache.get([] {
     using Cfg = DecCfg<BN, STAGES, NORM>;
     auto k = k_gemm_dec<BN, S, STAGES, NORM>;
     bool okf = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::kSmemBytes) ==
@@ -1161,12 +1157,12 @@ int dec_max_clusters() {
       if (cudaOccupancyMaxActiveClusters(&c, k, &cfg) != cudaSuccess) c = 0;
     }
     cudaGetLastError();
-    n = okf ? c : 0;
+    const int n = okf ? c : 0;
 #ifdef PHOTON_GEMM_DEBUG
     fprintf(stderr, "k_gemm_dec<%d,%d,%d,%d>: %d clusters resident\n", BN, S, STAGES, (int)NORM, n);
 #endif
-  }
-  return n;
+    return n;
+  });
 }
 
 template <int BN, int S, int STAGES, bool NORM>
@@ -1406,6 +1402,9 @@ bool persistent_enabled() {
 }  // namespace
 
 bool tma_available() { return encode_fn() != nullptr; }
+bool tma_map_bf16(CUtensorMap* m, const void* ptr, long long rows, int K, long long ld, int box_rows) {
+  return make_map(m, ptr, rows, K, ld, box_rows);
+}
 
 int gemm_tc_argmax_tiles(int M, int N, int K) {
   if (M <= 0 || N <= 0 || K <= 0 || K % kBK || N % 64) return 0;

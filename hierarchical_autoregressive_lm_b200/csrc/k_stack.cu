@@ -427,17 +427,15 @@ bool smap(CUtensorMap* m, const void* ptr, long long rows, int K, long long ld, 
 }
 
 int stack_grid() {
-  static int grid = [] {
-    int dev = 0, sms = 0, per = 0;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  static PerDevice cache;
+  return cache.get([] {
+    int per = 0;
     if (cudaFuncSetAttribute(k_stack_local, cudaFuncAttributeMaxDynamicSharedMemorySize, kSSmem) != cudaSuccess ||
         cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per, k_stack_local, kSThreads, kSSmem) != cudaSuccess)
       per = 0;
     cudaGetLastError();
-    return per >= 1 ? sms : 0;
-  }();
-  return grid;
+    return per >= 1 ? device_sm_count() : 0;
+  });
 }
 
 }  // namespace

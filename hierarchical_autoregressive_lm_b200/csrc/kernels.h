@@ -2,6 +2,7 @@
 // public C ABI; the runtime in runtime.cu is the only caller.
 #pragma once
 
+#include <cuda.h>  // CUtensorMap (type only)
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -212,6 +213,60 @@ size_t stack_local_scratch_bytes(int rows, int d);
 bool stack_local_supported(int rows, int d, int H, int dh, int f, int L, int p0, int cap);
 bool launch_stack_local(const StackLocalLaunch& s, cudaStream_t stream);
 
+// ---- persistent top-encoder decode step (k_top_step.cu) -------------------
+// Chunker_2 + all top-encoder blocks at one new position + the final norm, in
+// one launch.  ch_in: [B, C2*d] bf16 input rows (A-hat or A), row stride
+// ch_ld.  Buffers: x fp32 [B, d]; xs, q, att bf16 [B, d]; hid bf16 [B, f];
+// ssq fp32 [B, top_step_ssq_slots(d)]; part top_step_part_bytes; cnt
+// top_step_counters ints and bar 3 words, zero before the first launch (each
+// launch leaves them zero).  kc / vc: the top cache [L][B][H][cap][64]
+// (layer stride layer_elems elements), the new key at slot pos[0] - kv_off.
+// The launch advances pos[0] by 1 and pos[1] by dN1.
+constexpr int kTopMaxLayers = 16;
+struct TopStepLaunch {
+  const void* ch_in;
+  long long ch_ld;
+  const void* w_ch;
+  const void* wqkv[kTopMaxLayers];
+  const void* wo[kTopMaxLayers];
+  const void* w1[kTopMaxLayers];
+  const void* w2[kTopMaxLayers];
+  const float* g_attn[kTopMaxLayers];
+  const float* g_mlp[kTopMaxLayers];
+  const float* g_final;
+  float* x;
+  void* xs;
+  float* ssq;
+  void* q;
+  void* att;
+  void* hid;
+  void* kc;
+  void* vc;
+  long long layer_elems;
+  int cap, kv_off;
+  const float2* rope;
+  int* pos;
+  int dN1;
+  void* o_out;
+  float* part;
+  size_t part_bytes;
+  int* cnt;
+  unsigned* bar;
+  int* err;
+  int B, d, H, f, L, C2;
+  float eps, scale;
+};
+struct TopStepPlan;
+bool top_step_supported(int B, int d, int H, int dh, int f, int L, int C2, int cap);
+size_t top_step_part_bytes(int d, int f, int C2);
+int top_step_counters(int d);
+int top_step_ssq_slots(int d);
+// Builds the launch (tensor maps, work split) once; nullptr if the shape or
+// buffers are not supported.
+TopStepPlan* top_step_plan(const TopStepLaunch& s);
+void top_step_free(TopStepPlan* p);
+bool launch_top_step(const TopStepPlan* p, cudaStream_t stream);
+
 // ---- GEMM ----------------------------------------------------------------
 void launch_gemm(int dt, const GemmArgs& a, const GemmWorkspace& ws, int* err, cudaStream_t s);
 void launch_gemm_simt(int dt, const GemmArgs& a, cudaStream_t s);
@@ -259,5 +314,8 @@ unsigned long long launch_total();
 
 // ---- TMA descriptors -----------------------------------------------------
 bool tma_available();
+// 2-D bf16 tensor map over a row-major [rows, K] matrix (leading dimension ld
+// elements): box 64 (K) x box_rows, 128-byte swizzle, zero fill.
+bool tma_map_bf16(CUtensorMap* m, const void* ptr, long long rows, int K, long long ld, int box_rows);
 
 }  // namespace photon

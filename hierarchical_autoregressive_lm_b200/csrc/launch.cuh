@@ -12,9 +12,61 @@
 
 #include <cuda_runtime.h>
 
+#include <atomic>
+#include <climits>
+#include <mutex>
+
 #include "kernels.h"
 
 namespace photon {
+
+constexpr int kMaxDevices = 64;
+
+// A number computed once per device: kernel attributes set with
+// cudaFuncSetAttribute, occupancy queries and SM counts belong to the device
+// that was current when they were made, so a process that drives several
+// GPUs needs one copy per device.  get() runs `compute` with the caller's
+// current device on the first call for that device (under a lock) and
+// returns the cached value afterwards without locking.
+class PerDevice {
+ public:
+  PerDevice() {
+    for (auto& v : vals_) v.store(kUnset, std::memory_order_relaxed);
+  }
+  template <typename F>
+  int get(F&& compute) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+      cudaGetLastError();
+      return compute();
+    }
+    int v = vals_[dev].load(std::memory_order_acquire);
+    if (v != kUnset) return v;
+    std::lock_guard<std::mutex> lock(mu_);
+    v = vals_[dev].load(std::memory_order_relaxed);
+    if (v == kUnset) {
+      v = compute();
+      vals_[dev].store(v, std::memory_order_release);
+    }
+    return v;
+  }
+
+ private:
+  static constexpr int kUnset = INT_MIN;
+  std::atomic<int> vals_[kMaxDevices];
+  std::mutex mu_;
+};
+
+// SM count of the current device.
+inline int device_sm_count() {
+  static PerDevice cache;
+  return cache.get([] {
+    int dev = 0, sms = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    return sms > 0 ? sms : 1;
+  });
+}
 
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 __device__ __forceinline__ void pdl_trigger() {

@@ -19,7 +19,10 @@
 // last call left in it: calls whose GPU work overlaps (different streams
 // without ordering between them) race on it and must be serialised by the
 // caller.  Nothing in it needs to start at zero: every partial result the
-// combine pass reads is written by the same call's first pass.
+// combine pass reads is written by the same call's first pass.  A shape
+// that needs no split scratch (one chunk per pair, or the streamed kernel)
+// never looks the array up.
+#include <atomic>
 #include <cmath>
 #include <cstdio>
 #include <mutex>
@@ -34,23 +37,29 @@ constexpr int kMaxDevices = 64;
 
 static __device__ __align__(256) float g_noalloc_scratch[kNoAllocScratchBytes / sizeof(float)];
 
-float* g_scratch_addr[kMaxDevices] = {};
+std::atomic<float*> g_scratch_addr[kMaxDevices] = {};
 std::mutex g_scratch_mu;
 
-// Device address of the scratch array on the current device (looked up once).
+// Device address of the scratch array on the current device: looked up
+// under the lock on the first call for that device, read without it after.
 cudaError_t scratch_address(float** out) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
-  std::lock_guard<std::mutex> lock(g_scratch_mu);
-  if (!g_scratch_addr[dev]) {
-    void* p = nullptr;
-    e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
-    if (e != cudaSuccess) return e;
-    g_scratch_addr[dev] = static_cast<float*>(p);
+  float* p = g_scratch_addr[dev].load(std::memory_order_acquire);
+  if (!p) {
+    std::lock_guard<std::mutex> lock(g_scratch_mu);
+    p = g_scratch_addr[dev].load(std::memory_order_relaxed);
+    if (!p) {
+      void* sym = nullptr;
+      e = cudaGetSymbolAddress(&sym, g_noalloc_scratch);
+      if (e != cudaSuccess) return e;
+      p = static_cast<float*>(sym);
+      g_scratch_addr[dev].store(p, std::memory_order_release);
+    }
   }
-  *out = g_scratch_addr[dev];
+  *out = p;
   return cudaSuccess;
 }
 
@@ -60,7 +69,7 @@ extern "C" {
 
 int photon_attn_decode_noalloc(int32_t dtype, const void* d_q, const void* d_k, const void* d_v,
                                int32_t G, int32_t H, int32_t head_dim, int32_t cap, int32_t q_len,
-                               int32_t p0, void* d_o, void* stream) {
+                               int32_t p0, void* d_o, int32_t* d_err, void* stream) {
   using namespace photon;
   set_error_message("");
   if (dtype != 0 && dtype != 1) return set_error_message("dtype must be 0 or 1"), PHOTON_ERR_ARG;
@@ -93,12 +102,14 @@ int photon_attn_decode_noalloc(int32_t dtype, const void* d_q, const void* d_k, 
     return PHOTON_ERR_CAPACITY;
   }
   float* scratch = nullptr;
-  const cudaError_t e = scratch_address(&scratch);
-  if (e != cudaSuccess) {
-    set_error_message(cudaGetErrorString(e));
-    return PHOTON_ERR_CUDA;
+  if (need > 0) {
+    const cudaError_t e = scratch_address(&scratch);
+    if (e != cudaSuccess) {
+      set_error_message(cudaGetErrorString(e));
+      return PHOTON_ERR_CUDA;
+    }
   }
-  if (!launch_attn_decode(dtype, a, scratch, kNoAllocScratchBytes, nullptr, (cudaStream_t)stream))
+  if (!launch_attn_decode(dtype, a, scratch, need > 0 ? kNoAllocScratchBytes : 0, d_err, (cudaStream_t)stream))
     return set_error_message("decode attention rejected the shape"), PHOTON_ERR_ARG;
   const cudaError_t le = cudaGetLastError();
   if (le != cudaSuccess) return set_error_message(cudaGetErrorString(le)), PHOTON_ERR_CUDA;

@@ -372,6 +372,21 @@ struct photon_cache {
   unsigned long long* amax_part = nullptr;  // [B*C2][amax_cap] head partials
   int amax_cap = 0;
   int32_t* tok_out = nullptr;    // [B, C] greedy tokens of the last graph-replayed step
+  // persistent top-step kernel (k_top_step.cu): scratch shared by the top
+  // chains of this cache (at most one runs at a time) and the launch plans,
+  // one per (input rows, buffer set, mode)
+  bool tk_ok = false;
+  float* tk_part = nullptr;
+  size_t tk_part_bytes = 0;
+  int* tk_cnt = nullptr;
+  unsigned* tk_bar = nullptr;
+  struct TopPlanKey {
+    const void* src;
+    const void* xs;
+    int mode;
+    TopStepPlan* plan;
+  };
+  std::vector<TopPlanKey> tk_plans;
   // RecGen's top-encoder branch runs on its own stream with its own buffers
   cudaStream_t side = nullptr;
   cudaStream_t cap = nullptr;  // the decode step is captured here (any caller stream can replay it)
@@ -443,6 +458,16 @@ static bool split_norm_enabled() {
   static const bool on = [] {
     const char* e = getenv("PHOTON_SPLIT_NORM");
     return !(e && e[0] == '0');
+  }();
+  return on;
+}
+
+// Persistent top-step kernel for the top encoder's decode step
+// (PHOTON_TOP_MEGA=1; otherwise one kernel per projection).
+static bool top_mega_enabled() {
+  static const bool on = [] {
+    const char* e = getenv("PHOTON_TOP_MEGA");
+    return e && e[0] == '1';
   }();
   return on;
 }
@@ -955,6 +980,15 @@ static int prefill_impl(photon_model* m, const photon_cache* prefix, const int32
     c->stk_part = al.get<float>(stack_local_scratch_bytes(B * C2, d));
     c->stk_cnt = al.get<int>((size_t)c->stk_cnt_len * sizeof(int));
     c->stk_bar = al.get<unsigned int>(256);
+    if (top_mega_enabled() && !prefix &&
+        top_step_supported(B, d, m->H, m->dh, m->f, m->Ltop, C2, c->Ncap) &&
+        top_step_ssq_slots(d) <= kSsqCap) {
+      c->tk_part_bytes = top_step_part_bytes(d, m->f, C2);
+      c->tk_part = al.get<float>(c->tk_part_bytes);
+      c->tk_cnt = al.get<int>((size_t)top_step_counters(d) * sizeof(int));
+      c->tk_bar = al.get<unsigned>(64);
+      c->tk_ok = true;
+    }
   }
   c->attn_ws_t = al.get<float>(aw);
   if (cudaStreamCreateWithFlags(&c->side, cudaStreamNonBlocking) != cudaSuccess ||
@@ -971,7 +1005,9 @@ static int prefill_impl(photon_model* m, const photon_cache* prefix, const int32
   if (cudaMemsetAsync(c->d_err, 0, 16, s) != cudaSuccess ||
       cudaMemsetAsync(c->gemm_cnt, 0, kGemmTileCounters * sizeof(int), s) != cudaSuccess ||
       cudaMemsetAsync(c->gemm_cnt_t, 0, kGemmTileCounters * sizeof(int), s) != cudaSuccess ||
-      (c->stk_cnt && cudaMemsetAsync(c->stk_cnt, 0, (size_t)c->stk_cnt_len * sizeof(int), s) != cudaSuccess))
+      (c->stk_cnt && cudaMemsetAsync(c->stk_cnt, 0, (size_t)c->stk_cnt_len * sizeof(int), s) != cudaSuccess) ||
+      (c->tk_cnt && cudaMemsetAsync(c->tk_cnt, 0, (size_t)top_step_counters(d) * sizeof(int), s) != cudaSuccess) ||
+      (c->tk_bar && cudaMemsetAsync(c->tk_bar, 0, 64, s) != cudaSuccess))
     return bail(PHOTON_ERR_CUDA);
 
   // prefill workspace (released at the end of this call)
@@ -1225,6 +1261,68 @@ static void enqueue_decode(photon_model* m, photon_cache* c, int mode, int32_t* 
     launch_advance(c->d_pos, 1, mode == PHOTON_MODE_HIER ? C2 : 0, st);
   };
 
+  // a12 + a13: Chunker_2 of `src` ([B, C2*d] rows), the top step, its final
+  // norm into the pending output, and the position advance -- in one
+  // persistent launch when the cache has one planned, else kernel by kernel
+  auto top_chain = [&](const void* src, const Bufs& bb, cudaStream_t st) {
+    if (c->tk_ok) {
+      TopStepPlan* plan = nullptr;
+      for (auto& e : c->tk_plans)
+        if (e.src == src && e.xs == bb.sn_x && e.mode == mode) plan = e.plan;
+      if (!plan) {
+        TopStepLaunch t;
+        memset(&t, 0, sizeof(t));
+        t.ch_in = src;
+        t.ch_ld = (long long)C2 * d;
+        t.w_ch = m->ptr(m->i_ch2);
+        for (int l = 0; l < m->Ltop; ++l) {
+          const BlockW w = m->block(m->i_top, l);
+          t.wqkv[l] = w.wqkv;
+          t.wo[l] = w.wo;
+          t.w1[l] = w.w1;
+          t.w2[l] = w.w2;
+          t.g_attn[l] = w.g_attn;
+          t.g_mlp[l] = w.g_mlp;
+        }
+        t.g_final = (const float*)m->ptr(m->i_top_g);
+        t.x = c->xt;
+        t.xs = bb.sn_x;
+        t.ssq = bb.sn_ss;
+        t.q = bb.q;
+        t.att = bb.att;
+        t.hid = bb.hid;
+        t.kc = c->top_k;
+        t.vc = c->top_v;
+        t.layer_elems = (long long)(c->top_layer / m->es);
+        t.cap = c->Ncap;
+        t.kv_off = c->n_pre;
+        t.rope = c->rope;
+        t.pos = c->d_pos;
+        t.dN1 = mode == PHOTON_MODE_HIER ? C2 : 0;
+        t.o_out = c->o;
+        t.part = c->tk_part;
+        t.part_bytes = c->tk_part_bytes;
+        t.cnt = c->tk_cnt;
+        t.bar = c->tk_bar;
+        t.err = c->d_err;
+        t.B = B;
+        t.d = d;
+        t.H = m->H;
+        t.f = m->f;
+        t.L = m->Ltop;
+        t.C2 = C2;
+        t.eps = eps;
+        t.scale = 1.0f / sqrtf((float)m->dh);
+        plan = top_step_plan(t);
+        if (plan) c->tk_plans.push_back({src, bb.sn_x, mode, plan});
+      }
+      if (plan && launch_top_step(plan, st)) return;
+    }
+    gemm(m, bb, src, (long long)C2 * d, m->ptr(m->i_ch2), (long long)C2 * d, B, d, C2 * d,
+         epi(EPI_STORE_F32, c->xt, d), st);
+    top_step(c->xt, bb, st);
+  };
+
   if (part != DEC_TOK) {
   // a7: Converter_2 -- o [B, d] -> C2 conditioning vectors per sequence
   gemm(m, b, c->o, d, m->ptr(m->i_cv2), d, B, C2 * d, d, epi(EPI_STORE_F32, c->xd, (long long)C2 * d), s);
@@ -1242,9 +1340,7 @@ static void enqueue_decode(photon_model* m, photon_cache* c, int mode, int32_t* 
   if (part == DEC_MAIN) {
     // pipelined RecGen: the top encoder's next input follows at once; the
     // token branch of this A-hat runs as its own graph
-    gemm(m, b, ahat, (long long)C2 * d, m->ptr(m->i_ch2), (long long)C2 * d, B, d, C2 * d,
-         epi(EPI_STORE_F32, c->xt, d), s);
-    top_step(c->xt, b, s);
+    top_chain(ahat, b, s);
     return;
   }
   }
@@ -1267,9 +1363,7 @@ static void enqueue_decode(photon_model* m, photon_cache* c, int mode, int32_t* 
     bt.sn_x = c->sn_x_t;
     bt.sn_ss = c->sn_ss_t;
     const void* src = d_force_a ? d_force_a : ahat;
-    gemm(m, bt, src, (long long)C2 * d, m->ptr(m->i_ch2), (long long)C2 * d, B, d, C2 * d,
-         epi(EPI_STORE_F32, c->xt, d), c->side);
-    top_step(c->xt, bt, c->side);
+    top_chain(src, bt, c->side);
     cudaEventRecord(c->ev_join, c->side);
   }
   // the token branch: the caller's stream, or (optionally) a high-priority
@@ -1360,9 +1454,8 @@ static void enqueue_decode(photon_model* m, photon_cache* c, int mode, int32_t* 
   }
   if (mode == PHOTON_MODE_REC) {
     // RecGen without a side stream: Chunker_2(A-hat), no re-encoding
-    const void* src = d_force_a ? d_force_a : c->a_hat;
-    gemm(m, b, src, (long long)C2 * d, m->ptr(m->i_ch2), (long long)C2 * d, B, d, C2 * d,
-         epi(EPI_STORE_F32, c->xt, d), s);
+    top_chain(d_force_a ? d_force_a : c->a_hat, b, s);
+    return;
   } else {
     // HierGen: embed the written tokens, Chunker_1, level-1 encoder with its cache, Chunker_2
     launch_embed(m->dt, c->used, m->ptr(m->i_embed), c->embd, B * C, d, V, c->d_err, s);
@@ -1389,11 +1482,9 @@ static void enqueue_decode(photon_model* m, photon_cache* c, int mode, int32_t* 
     }
     run_stack(m, m->i_enc1, m->L1, c->x1, re, b, s);
     launch_rmsnorm(m->dt, c->x1, (const float*)m->ptr(m->i_enc1_g), c->a, G, d, 1, 0, eps, s);
-    gemm(m, b, c->a, (long long)C2 * d, m->ptr(m->i_ch2), (long long)C2 * d, B, d, C2 * d,
-         epi(EPI_STORE_F32, c->xt, d), s);
+    // a13: one top-encoder step at position N (KV append + decode attention)
+    top_chain(c->a, b, s);
   }
-  // a13: one top-encoder step at position N (KV append + decode attention)
-  top_step(c->xt, b, s);
 }
 
 static bool graphs_enabled() {
@@ -1682,6 +1773,7 @@ int photon_free_cache(photon_cache* c) {
   CK(cudaGetLastError());
   m->live_caches--;
   if (c->mode == PHOTON_MODE_HIER) m->hier_caches--;
+  for (auto& e : c->tk_plans) top_step_free(e.plan);  // host-side launch descriptions only
   delete c;
   return PHOTON_OK;
 }
@@ -1922,9 +2014,29 @@ int photon_gemm_rmsnorm(const float* d_x, int64_t ldx, const float* d_g, float e
   return PHOTON_OK;
 }
 
+int photon_attn_decode_scratch_bytes(int32_t dtype, int32_t G, int32_t H, int32_t head_dim, int32_t cap,
+                                     int32_t q_len, int32_t p0, uint64_t* out_bytes) {
+  g_err.clear();
+  if (!out_bytes) return fail(PHOTON_ERR_ARG, "out_bytes is NULL");
+  if (dtype != 0 && dtype != 1) return fail(PHOTON_ERR_ARG, "dtype must be 0 or 1");
+  if (G <= 0 || H <= 0 || (head_dim != 32 && head_dim != 64)) return fail(PHOTON_ERR_ARG, "bad shape");
+  if (q_len < 1 || q_len > 4 || p0 < 0 || p0 + q_len > cap) return fail(PHOTON_ERR_ARG, "bad q_len/p0/cap");
+  AttnArgs a;
+  a.q_ld = (long long)H * head_dim;
+  a.o_ld = a.q_ld;
+  a.cap = cap;
+  a.G = G;
+  a.H = H;
+  a.dh = head_dim;
+  a.q_len = q_len;
+  a.p0 = p0;
+  *out_bytes = attn_decode_workspace_bytes(dtype, a);
+  return PHOTON_OK;
+}
+
 int photon_attn_decode(int32_t dtype, const void* d_q, const void* d_k, const void* d_v, int32_t G,
                        int32_t H, int32_t head_dim, int32_t cap, int32_t q_len, int32_t p0, void* d_o,
-                       void* stream) {
+                       int32_t* d_err, void* stream) {
   g_err.clear();
   if (dtype != 0 && dtype != 1) return fail(PHOTON_ERR_ARG, "dtype must be 0 or 1");
   if (!d_q || !d_k || !d_v || !d_o) return fail(PHOTON_ERR_ARG, "NULL buffer");
@@ -1948,7 +2060,7 @@ int photon_attn_decode(int32_t dtype, const void* d_q, const void* d_k, const vo
   const size_t wsb = attn_decode_workspace_bytes(dtype, a);
   float* ws = nullptr;
   if (wsb) CK(pool_malloc((void**)&ws, wsb, s));
-  const bool ok = launch_attn_decode(dtype, a, ws, wsb, nullptr, s);
+  const bool ok = launch_attn_decode(dtype, a, ws, wsb, d_err, s);
   if (ws) cudaFreeAsync(ws, s);
   if (!ok) return fail(PHOTON_ERR_ARG, "decode attention rejected the shape");
   CK(cudaGetLastError());

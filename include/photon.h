@@ -305,10 +305,22 @@ PHOTON_API int photon_gemm_rmsnorm(const float* d_x, int64_t ldx, const float* d
  * p0..p0+q_len-1 attend causally over keys 0..p0+i of a cache
  * d_k/d_v [G][H][cap][head_dim] (storage type, post-RoPE keys);
  * d_q and d_o are [G*q_len][H*head_dim].  Scale 1/sqrt(head_dim).
+ * d_err (device int32, nullable): the kernels' error word.  A bounded wait
+ * that runs out (about 2 s; the long-cache streamed kernel waits on its bulk
+ * copies) leaves d_o unwritten and sets *d_err to a nonzero code, which the
+ * caller reads after the stream has synchronised (zero it before the call).
+ * With d_err NULL such a timeout goes unreported.
  * Allocates its split scratch internally.  Errors: ERR_ARG. */
 PHOTON_API int photon_attn_decode(int32_t dtype, const void* d_q, const void* d_k, const void* d_v, int32_t G,
                        int32_t H, int32_t head_dim, int32_t cap, int32_t q_len, int32_t p0,
-                       void* d_o, void* stream);
+                       void* d_o, int32_t* d_err, void* stream);
+
+/* Bytes of split scratch photon_attn_decode needs for this shape (0 when
+ * every (group, head) pair is one chunk, or the long-cache streamed kernel
+ * takes it); a host-side planning query that launches nothing.  Written to
+ * *out_bytes.  Errors: ERR_ARG. */
+PHOTON_API int photon_attn_decode_scratch_bytes(int32_t dtype, int32_t G, int32_t H, int32_t head_dim,
+                                                int32_t cap, int32_t q_len, int32_t p0, uint64_t* out_bytes);
 
 /* Allocation-free variant of photon_attn_decode (this entry point has no
  * counterpart in the PHOTON paper; it exists for callers that cannot let the
@@ -320,14 +332,16 @@ PHOTON_API int photon_attn_decode(int32_t dtype, const void* d_q, const void* d_
  * GPU that loads the library until the process exits); the call allocates
  * and frees nothing.  The array's device address is looked up during the
  * first call on each device, so make that first call before any stream
- * capture.  All calls share the array: calls whose GPU work may overlap
- * race on it and must be ordered by the caller.  Errors: ERR_ARG (bad
- * arguments), ERR_CAPACITY (the shape needs more than the 256 KiB of scratch;
- * the message says how much), ERR_CUDA. */
+ * capture.  A shape that needs no split scratch never looks it up.  All
+ * calls share the array: calls whose GPU work may overlap race on it and
+ * must be ordered by the caller.  d_err as for photon_attn_decode (a word
+ * the caller owns; NULL leaves wait timeouts unreported).  Errors: ERR_ARG
+ * (bad arguments), ERR_CAPACITY (the shape needs more than the 256 KiB of
+ * scratch; the message says how much), ERR_CUDA. */
 PHOTON_API int photon_attn_decode_noalloc(int32_t dtype, const void* d_q, const void* d_k,
                                           const void* d_v, int32_t G, int32_t H, int32_t head_dim,
                                           int32_t cap, int32_t q_len, int32_t p0, void* d_o,
-                                          void* stream);
+                                          int32_t* d_err, void* stream);
 
 /* Teacher-forced scoring (explainer, quality section: PHOTON's reported
  * quality is measured with teacher-forced HierGen).  For prompts d_tokens

@@ -80,8 +80,10 @@ def _attn_case(dtype, G, H, dh, cap, q_len, p0, seed):
     k = _rand((G, H, cap, dh), dtype, seed + 1)
     v = _rand((G, H, cap, dh), dtype, seed + 2)
     out = torch.zeros(G * q_len, H * dh, dtype=dtype, device="cuda")
-    hal.attn_decode(q.cuda(), k.cuda(), v.cuda(), q_len, p0, out)
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    hal.attn_decode(q.cuda(), k.cuda(), v.cuda(), q_len, p0, out, err=err)
     torch.cuda.synchronize()
+    assert int(err.item()) == 0
     got = out.float().cpu().numpy().reshape(G, q_len, H, dh)
     qd = q.double().numpy().reshape(G, q_len, H, dh)
     kd, vd = k.double().numpy(), v.double().numpy()
