@@ -16,7 +16,8 @@ import os
 from typing import Optional
 
 __all__ = ["PhotonError", "Model", "Cache", "load_library", "LIB_PATH", "MODE_HIER",
-           "MODE_REC", "STATE", "launch_count", "gemm", "gemm_rmsnorm", "attn_decode", "attn_decode_noalloc", "attn_decode_scratch_bytes", "config_struct", "EXPORTED",
+           "MODE_REC", "STATE", "launch_count", "gemm", "gemm_rmsnorm", "attn_decode", "attn_decode_noalloc", "attn_decode_scratch_bytes", "debug_fail_alloc",
+           "selftest_wait_timeout", "config_struct", "EXPORTED",
            "AGG_VOTE", "AGG_BEST", "aggregate"]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libphoton.so")
@@ -38,7 +39,8 @@ EXPORTED = ("photon_init_weights", "photon_free_model", "photon_prefill",
             "photon_attn_decode", "photon_attn_decode_scratch_bytes", "photon_attn_decode_noalloc", "photon_score", "photon_aggregate",
             "photon_multi_query", "photon_vanilla_init",
             "photon_vanilla_prefill", "photon_vanilla_decode_step", "photon_vanilla_cache_info",
-            "photon_vanilla_free_cache", "photon_launch_count", "photon_last_error")
+            "photon_vanilla_free_cache", "photon_launch_count", "photon_last_error",
+            "photon_debug_fail_alloc", "photon_selftest_wait_timeout")
 
 
 class PhotonError(RuntimeError):
@@ -127,6 +129,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "photon_attn_decode": [I32, P, P, P, I32, I32, I32, I32, I32, I32, P, P, P],
         "photon_attn_decode_noalloc": [I32, P, P, P, I32, I32, I32, I32, I32, I32, P, P, P],
         "photon_attn_decode_scratch_bytes": [I32, I32, I32, I32, I32, I32, I32, P],
+        "photon_debug_fail_alloc": [I64],
+        "photon_selftest_wait_timeout": [I64, P, P],
     }
     for name, args in sig.items():
         fn = getattr(L, name)
@@ -521,3 +525,16 @@ def attn_decode_scratch_bytes(dtype_code: int, G: int, H: int, head_dim: int, ca
     _check(load_library().photon_attn_decode_scratch_bytes(dtype_code, G, H, head_dim, cap, q_len, p0,
                                                            ctypes.byref(out)))
     return int(out.value)
+
+
+def debug_fail_alloc(n: int) -> None:
+    """Test hook: the n-th device allocation from now on fails as out of memory (0: off)."""
+    _check(load_library().photon_debug_fail_alloc(int(n)))
+
+
+def selftest_wait_timeout(limit_cycles: int, err, stream=None) -> None:
+    """Runs the bounded-wait self-test (raises PhotonError with PHOTON_ERR_DEVICE_CHECK
+    when the wait runs out, which is its expected outcome); err: int32 CUDA tensor."""
+    import torch
+    _need(err, torch.int32, 1, "err")
+    _check(load_library().photon_selftest_wait_timeout(int(limit_cycles), _ptr(err), _stream(stream)))

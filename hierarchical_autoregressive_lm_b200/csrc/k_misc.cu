@@ -7,6 +7,7 @@
 #include "epilogue.cuh"
 #include "kernels.h"
 #include "launch.cuh"
+#include "ptx_sm100.cuh"
 #include "sampling.cuh"
 
 namespace photon {
@@ -621,6 +622,22 @@ void launch_splitk_reduce(int dt, const float* part, int splits, int M, int N, c
     {
       launch_kernel(k_splitk_reduce<bf16>, (int)blocks, threads, 0, s, part, splits, M, N, ep);
     }
+}
+
+// Self-test of the bounded-wait path: one thread waits on an mbarrier that
+// nothing ever arrives on, through the same bounded wait every kernel uses,
+// and records the timeout in the error word once `limit` cycles pass.
+__global__ void k_wait_selftest(long long limit, int* err) {
+  __shared__ __align__(8) uint64_t bar;
+  if (threadIdx.x != 0) return;
+  ptx::mbar_init(ptx::smem_u32(&bar), 1);
+  ptx::fence_barrier_init();
+  if (!ptx::mbar_wait_limit(ptx::smem_u32(&bar), 0u, nullptr, limit)) report_error(err, DEV_WAIT_TIMEOUT_PRODUCER);
+}
+
+void launch_wait_selftest(long long limit, int* err, cudaStream_t s) {
+  k_wait_selftest<<<1, 32, 0, s>>>(limit, err);
+  note_launch();
 }
 
 }  // namespace photon

@@ -32,9 +32,15 @@
 //    each token row of its accumulator by 1 / rms, which is exact since
 //    RMSNorm(x) W^T = rstd * (x * g) W^T.
 //  * The attention phase streams each (sequence, head) pair's K and V rows
-//    through a 3-stage bulk-copy ring.  The first tiles hold only keys
-//    cached by earlier steps, so their copies are issued when the QKV phase
-//    starts; the tile that holds the new key follows the barrier.
+//    through a 9-stage bulk-copy ring (3 stages of its own, 6 borrowed from
+//    the idle weight buffer and token region).  The first tiles hold only
+//    keys cached by earlier steps, so their copies are issued during the QKV
+//    phase; the tile that holds the new key follows the barrier.
+//  * The next phase's weight copies are issued once the current phase's own
+//    token blocks have landed, so they never delay the critical path.
+//  * The grid barrier is two-level: the 4 CTAs of a cluster meet at a
+//    cluster barrier and one thread per cluster takes part in the global
+//    count (release add, acquire poll with backoff).
 //
 // Data written in one phase and read in a later one goes through L2 (TMA
 // and bulk copies, or ld.global.cg), with a proxy fence around each barrier
@@ -44,10 +50,12 @@
 // is left waiting on a peer that has stopped.
 #include <cuda.h>
 
+#include <cstdio>
 #include <cstdlib>
 #include <cstring>
 
 #include "common.cuh"
+#include "epilogue.cuh"
 #include "kernels.h"
 #include "launch.cuh"
 #include "ptx_sm100.cuh"
@@ -56,39 +64,68 @@ namespace photon {
 
 namespace {
 
-constexpr int kCS = 4;              // CTAs per cluster: the K split of one weight tile
-constexpr int kWorkers = 256;       // warps 0-7: MMA issue, TMEM drain, epilogue, attention
-constexpr int kThreads = kWorkers + 32;  // warp 8: TMA / bulk-copy producer
-constexpr int kProducer = kWorkers;      // its lane 0
+#ifdef PHOTON_TOP_TRACE
+// Diagnostic builds only: %globaltimer at each grid barrier of CTA 0, and at
+// points inside the phases of CTA 0, printed by CTA 0 for a few launches.
+__device__ unsigned long long g_top_trace[128];
+__device__ unsigned long long g_top_pts[128][8];
+__device__ unsigned int g_top_trace_launch;
+__device__ __forceinline__ unsigned long long gtimer() {
+  unsigned long long t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+#define TOP_PT(c, k)                                                                              \
+  do {                                                                                            \
+    if (blockIdx.x == 0 && (threadIdx.x == 0 || threadIdx.x == kIssuer) && (c).nbar < 128)          \
+      g_top_pts[(c).nbar][k] = gtimer();                                                          \
+  } while (0)
+#else
+#define TOP_PT(c, k) \
+  do {               \
+  } while (0)
+#endif
+
+constexpr int kCS = 4;                   // CTAs per cluster: the K split of one weight tile
+constexpr int kWorkers = 256;            // warps 0-7: TMEM drain, epilogue, attention
+constexpr int kThreads = kWorkers + 64;  // warp 8: TMA / bulk-copy producer; warp 9: MMA issue
+constexpr int kProducer = kWorkers;      // lane 0 of warp 8
+constexpr int kIssuer = kWorkers + 32;   // lane 0 of warp 9
 constexpr int kBM = 128, kBN = 64, kBK = 64;
-constexpr int kKbMax = 4;                       // K blocks of one CTA per unit
-constexpr int kWTile = kBM * kBK * 2;           // 16 KB weight block
-constexpr int kXTile = kBN * kBK * 2;           // 8 KB token block
-constexpr int kWBuf = kKbMax * kWTile;          // 64 KB
-constexpr int kLDP = kBN + 4;                   // partial-tile row stride (floats)
+constexpr int kKbMax = 4;               // K blocks of one CTA per unit
+constexpr int kWTile = kBM * kBK * 2;   // 16 KB weight block
+constexpr int kXTile = kBN * kBK * 2;   // 8 KB token block
+constexpr int kWBuf = kKbMax * kWTile;  // 64 KB
+constexpr int kLDP = kBN + 4;           // partial-tile row stride (floats)
 constexpr int kPBytes = kBM * kLDP * 4;
 constexpr int kXBytes = kKbMax * kXTile;
 constexpr int kXP = ((kPBytes > kXBytes ? kPBytes : kXBytes) + 1023) & ~1023;
-constexpr int kPU = 64 / kCS;                   // RoPE pairs of a tile owned by one CTA
-constexpr int kTK = 64;                         // keys per attention tile
-constexpr int kAStages = 3;
-constexpr int kATile = kTK * 128;               // 64 keys x 64 bf16
-constexpr int kAStage = 2 * kATile;             // K and V
+constexpr int kPU = 64 / kCS;   // RoPE pairs of a tile owned by one CTA
+constexpr int kMaxParts = 4;    // K parts of one tile
+constexpr int kMaxSlots = 32;   // split-RMSNorm slots per row
+constexpr int kTK = 64;         // keys per attention tile
+constexpr int kATile = kTK * 128;  // 64 keys x 64 bf16
+constexpr int kAStage = 2 * kATile;  // K and V
 constexpr int kAWarps = 8;
-constexpr int kOffW = 0;                        // two weight buffers
-constexpr int kOffX = 2 * kWBuf;                // token blocks / partial tile
-constexpr int kOffA = kOffX + kXP;              // attention ring
-constexpr int kOffCtrl = kOffA + kAStages * kAStage;
-// control block: barriers (16 x 8 B), TMEM slot, abort flag, ok flag, rstd[64],
-// attention merge buffers m/l [2][8] and acc [2][8][64]
-constexpr int kCtrlBar = 0, kCtrlMisc = 128, kCtrlRstd = 256, kCtrlM = 512, kCtrlL = 576,
-              kCtrlAcc = 640;
-constexpr int kCtrlBytes = kCtrlAcc + 2 * kAWarps * 64 * 4;
+// Attention ring: 3 stages of its own, 4 in the QKV/W1 weight buffer and 2
+// in the token region, the last 6 usable only inside the attention phase
+// (the weight buffer and token region are idle then).
+constexpr int kAOwn = 3;
+constexpr int kAStages = kAOwn + kWBuf / kAStage + (kXP / kAStage);
+constexpr int kMaxPairsPerCta = kAWarps;  // one worker warp per (sequence, head) pair
+constexpr int kOffW = 0;            // two weight buffers
+constexpr int kOffX = 2 * kWBuf;    // token blocks / partial tile
+constexpr int kOffA = kOffX + kXP;  // the ring's own stages
+constexpr int kOffCtrl = kOffA + kAOwn * kAStage;
+// control block: barriers, TMEM slot and flags, rstd[64], the CTA's query rows
+constexpr int kCtrlBar = 0, kCtrlMisc = 256, kCtrlRstd = 384, kCtrlQ = 640;
+constexpr int kCtrlBytes = kCtrlQ + kMaxPairsPerCta * 128;
 constexpr int kSmem = kOffCtrl + kCtrlBytes + 1024;
 static_assert(kSmem <= 227 * 1024, "shared memory budget");
 static_assert(kPU * (kBN / 4) == kWorkers, "one epilogue item per worker thread");
+static_assert(kAStages <= 16 && (4 + 2 * kAStages + 1) * 8 <= kCtrlMisc, "control block layout");
 
-enum PhaseKind { PK_CH = 0, PK_QKV = 1, PK_O = 2, PK_W1 = 3, PK_W2 = 4 };
+enum PhaseKind { PK_NONE = -1, PK_CH = 0, PK_QKV = 1, PK_O = 2, PK_W1 = 3, PK_W2 = 4 };
 
 struct TopArgs {
   CUtensorMap w_ch;
@@ -97,29 +134,28 @@ struct TopArgs {
   const float* g_attn[kTopMaxLayers];
   const float* g_mlp[kTopMaxLayers];
   const float* g_final;
-  float* x;      // [B, d] residual stream
-  bf16* xs;      // [B, d] bf16(x * g) of the next norm
-  float* ssq;    // [B, ssq_slots] partial sums of squares
-  bf16* q;       // [B, d]
-  bf16* att;     // [B, d]
-  bf16* hid;     // [B, f]
-  bf16* kc;      // top KV cache, [L][B][H][cap][64]
+  float* x;   // [B, d] residual stream
+  bf16* xs;   // [B, d] bf16(x * g) of the next norm
+  float* ssq;  // [B, ssq_slots] partial sums of squares
+  bf16* q;    // [B, d]
+  bf16* att;  // [B, d]
+  bf16* hid;  // [B, f]
+  bf16* kc;   // top KV cache, [L][B][H][cap][64]
   bf16* vc;
   long long layer_elems;
   int cap, kv_off;
   const float2* rope;
-  int* pos;      // pos[0]: position of the new key; advanced by 1 (pos[1] by dN1) at the end
+  int* pos;  // pos[0]: position of the new key; advanced by 1 (pos[1] by dN1) at the end
   int dN1;
-  bf16* o_out;   // [B, d]
-  float* part;   // K-part partial tiles
-  int* cnt;      // per (tile, rank) counters, zero before and after
-  unsigned* bar; // [0] barrier count, [1] exit count, [2] abort word: zero before and after
+  bf16* o_out;    // [B, d]
+  float* part;    // K-part partial tiles
+  int* cnt;       // per (tile, rank) counters, zero before and after
+  unsigned* bar;  // [0] barrier count, [1] exit count, [2] abort word: zero before and after
   int* err;
   int B, d, H, f, L, nkb_ch;
   int pk_ch, pk_o, pk_w2;
   int ssq_slots;
   float eps, scale;
-  int l2_prefetch;
 };
 
 struct Ctx {
@@ -130,16 +166,19 @@ struct Ctx {
   volatile int* ok_flag;    // set by each grid barrier: the launch is still live
   volatile int* last_flag;  // this CTA arrived last at a K-part counter
   float* rstd;
-  uint32_t wuse[2];  // times each weight buffer has been armed
+  uint32_t wuse[2];  // times each weight buffer has been armed (all threads)
   uint32_t xuse;     // times the token / done barriers have completed
-  uint32_t at;       // attention tiles issued (producer) or consumed (workers) so far
+  uint32_t quse;     // attention phases whose query rows were copied
+  uint32_t a_par;    // ring stage s: parity of its next full-barrier completion (bit s)
+  uint32_t a_used;   // ring stage s: used at least once (bit s)
   uint32_t pre;      // attention tiles issued before this layer's attention phase
   int nbar;          // grid barriers passed
   int rank, cluster, nclusters;
-  // exit drain after an abort: copies and MMAs still in flight
-  uint32_t x_armed;  // producer: token-block loads armed
-  uint32_t at_issued;  // producer: attention tiles issued
-  bool mma_open;     // thread 0: MMAs committed whose completion it has not seen
+  // producer only: copies actually issued (for the exit drain after an abort)
+  uint32_t w_issued[2], x_issued;
+  bool q_issued;
+  uint32_t a_pend, a_pend_par;  // ring stages with an issued copy; parity of its completion
+  bool mma_open;  // issuer: MMAs committed whose completion it has not seen
 };
 
 __device__ __forceinline__ uint32_t bar_w(const Ctx& c, int b) { return ptx::smem_u32(c.bars + b); }
@@ -148,6 +187,15 @@ __device__ __forceinline__ uint32_t bar_done(const Ctx& c) { return ptx::smem_u3
 __device__ __forceinline__ uint32_t bar_afull(const Ctx& c, int s) { return ptx::smem_u32(c.bars + 4 + s); }
 __device__ __forceinline__ uint32_t bar_aempty(const Ctx& c, int s) {
   return ptx::smem_u32(c.bars + 4 + kAStages + s);
+}
+__device__ __forceinline__ uint32_t bar_q(const Ctx& c) { return ptx::smem_u32(c.bars + 4 + 2 * kAStages); }
+
+// Shared-memory address of attention ring stage s (`abuf`: the weight buffer
+// the ring borrows during the attention phase).
+__device__ __forceinline__ uint8_t* ring_stage(const Ctx& c, int s, int abuf) {
+  if (s < kAOwn) return c.smem + kOffA + s * kAStage;
+  if (s < kAOwn + kWBuf / kAStage) return c.smem + kOffW + abuf * kWBuf + (s - kAOwn) * kAStage;
+  return c.smem + kOffX + (s - kAOwn - kWBuf / kAStage) * kAStage;
 }
 
 __device__ __forceinline__ bool aborted(const TopArgs& a) {
@@ -159,37 +207,61 @@ __device__ __forceinline__ void raise_abort(const TopArgs& a, Ctx& c, int code) 
   *c.abort_cta = 1;
 }
 
-// Grid-wide barrier over all CTAs of the launch.  Prior global writes of every
-// thread (generic proxy, and made visible to the async proxy) happen before
-// any access after the barrier.  Returns false once the launch is aborted.
+// Grid-wide barrier over all CTAs of the launch: thread 0 of every CTA adds
+// to a global count with release semantics (after __syncthreads, so the
+// whole CTA's writes are ordered before it) and polls the count with acquire
+// semantics.  Prior global writes of every thread (made visible to the async
+// proxy as well) happen before any access after the barrier.  Returns false
+// once the launch is aborted.
 __device__ bool grid_barrier(const TopArgs& a, Ctx& c) {
-  asm volatile("fence.proxy.async.global;" ::: "memory");
+  asm volatile("fence.proxy.async;" ::: "memory");
   __syncthreads();
+  TOP_PT(c, 7);
   c.nbar += 1;
   if (threadIdx.x == 0) {
-    bool ok = *c.abort_cta == 0;
-    if (ok) {
-      __threadfence();
-      atomicAdd(a.bar, 1u);
+    if (*c.abort_cta == 0 && !aborted(a)) {
+      asm volatile("red.release.gpu.global.add.u32 [%0], 1;" ::"l"(a.bar) : "memory");
       const unsigned target = (unsigned)c.nbar * gridDim.x;
       const long long t0 = clock64();
       while (true) {
         unsigned v;
         asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(a.bar) : "memory");
-        if (v >= target) break;
-        if (aborted(a) || clock64() - t0 > ptx::kWaitLimitCycles) {
-          if (!aborted(a)) raise_abort(a, c, DEV_WAIT_TIMEOUT_EPILOGUE);
-          *c.abort_cta = 1;
-          ok = false;
+        if (v >= target || aborted(a)) break;
+        if (clock64() - t0 > ptx::kWaitLimitCycles) {
+          raise_abort(a, c, DEV_WAIT_TIMEOUT_EPILOGUE);
           break;
         }
       }
     }
-    asm volatile("fence.proxy.async.global;" ::: "memory");
+    asm volatile("fence.proxy.async;" ::: "memory");
+    const bool ok = *c.abort_cta == 0 && !aborted(a);
+    if (!ok) *c.abort_cta = 1;
     *c.ok_flag = ok ? 1 : 0;
+#ifdef PHOTON_TOP_TRACE
+    if (blockIdx.x == 0 && c.nbar < 128) g_top_trace[c.nbar] = gtimer();
+#endif
   }
   __syncthreads();
   return *c.ok_flag != 0;
+}
+
+// Sum of n (a multiple of 4, at most kMaxSlots) partial sums of squares in
+// slot order, all loads issued before the first add.
+__device__ __forceinline__ float sum_slots(const float* p, int n) {
+  float4 v[kMaxSlots / 4];
+#pragma unroll
+  for (int j = 0; j < kMaxSlots / 4; ++j)
+    if (4 * j < n) v[j] = __ldcg(reinterpret_cast<const float4*>(p) + j);
+  float t = 0.f;
+#pragma unroll
+  for (int j = 0; j < kMaxSlots / 4; ++j)
+    if (4 * j < n) {
+      t += v[j].x;
+      t += v[j].y;
+      t += v[j].z;
+      t += v[j].w;
+    }
+  return t;
 }
 
 struct GemmPhase {
@@ -226,21 +298,25 @@ __device__ __forceinline__ void unit_kbs(const GemmPhase& g, int u, int rank, in
   nk = max(0, min(p1, kb0 + rb) - kb0);
 }
 
-// Producer: load this CTA's weight slice of round-0 unit of phase g into
-// buffer `buf` (returns whether the buffer was armed).
-__device__ bool issue_weights(const Ctx& c, const GemmPhase& g, int buf, int u) {
+// Whether this CTA has weight blocks in the round-0 unit of phase g.
+__device__ __forceinline__ bool has_weights(const Ctx& c, const GemmPhase& g) {
   const int units = (g.N / kBM) * g.pk;
-  if (u >= units) return false;
+  if (c.cluster >= units) return false;
+  int tile, kp, kb0, nk;
+  unit_kbs(g, c.cluster, c.rank, tile, kp, kb0, nk);
+  return nk > 0;
+}
+
+// Producer: load this CTA's weight slice of unit u of phase g into buffer buf.
+__device__ void load_weights(Ctx& c, const GemmPhase& g, int buf, int u) {
   int tile, kp, kb0, nk;
   unit_kbs(g, u, c.rank, tile, kp, kb0, nk);
-  if (nk <= 0) return false;
-  if (threadIdx.x == kProducer) {
-    ptx::mbar_arrive_expect_tx(bar_w(c, buf), (uint32_t)(nk * kWTile));
-    const uint32_t dst = ptx::smem_u32(c.smem + kOffW + buf * kWBuf);
-    for (int i = 0; i < nk; ++i)
-      ptx::tma_load_2d(dst + i * kWTile, g.wmap, (kb0 + i) * kBK, tile * kBM, bar_w(c, buf));
-  }
-  return true;
+  if (nk <= 0) return;
+  ptx::mbar_arrive_expect_tx(bar_w(c, buf), (uint32_t)(nk * kWTile));
+  const uint32_t dst = ptx::smem_u32(c.smem + kOffW + buf * kWBuf);
+  for (int i = 0; i < nk; ++i)
+    ptx::tma_load_2d(dst + i * kWTile, g.wmap, (kb0 + i) * kBK, tile * kBM, bar_w(c, buf));
+  c.w_issued[buf] += 1;
 }
 
 // Wait helper that records where it gave up.
@@ -251,9 +327,91 @@ __device__ __forceinline__ bool wait_or_abort(const TopArgs& a, Ctx& c, uint32_t
   return false;
 }
 
-// One GEMM phase.  `armed` says whether this CTA's round-0 weights were
-// loaded ahead into buffer `buf`.
-__device__ void run_gemm(const TopArgs& a, Ctx& c, const GemmPhase& g, int buf, bool armed) {
+// ---- attention: one query per (sequence, head) pair over keys 0..pos ------
+struct AttnPlan {
+  int pair0, npairs, tpp, n;
+};
+__device__ __forceinline__ AttnPlan attn_plan(const TopArgs& a, int pos) {
+  AttnPlan p;
+  const int pairs = a.B * a.H;
+  const int per = (pairs + gridDim.x - 1) / gridDim.x;
+  p.pair0 = blockIdx.x * per;
+  p.npairs = max(0, min(per, pairs - p.pair0));
+  p.n = pos + 1 - a.kv_off;  // keys in the cache, the new one included
+  p.tpp = (p.n + kTK - 1) / kTK;
+  return p;
+}
+
+// Tiles of a layer are issued in the order t = j * npairs + w (tile j of the
+// CTA's pair w), so the CTA's pairs advance together; tile t goes to ring
+// stage t % kAStages.  A stage's use count at tile t is its count at the
+// start of the layer (parity bit in a_par, used bit in a_used) plus t / kAStages.
+__device__ __forceinline__ uint32_t ring_parity(const Ctx& c, int st, int t) {
+  return ((c.a_par >> st) & 1u) ^ (uint32_t)((t / kAStages) & 1);
+}
+__device__ __forceinline__ bool ring_reused(const Ctx& c, int st, int t) {
+  return t >= kAStages || ((c.a_used >> st) & 1u);
+}
+// After a layer of `total` tiles: every stage's parity and used bits.
+__device__ __forceinline__ void ring_advance(Ctx& c, int total) {
+  for (int st = 0; st < kAStages; ++st) {
+    const int uses = total > st ? (total - st + kAStages - 1) / kAStages : 0;
+    if (uses & 1) c.a_par ^= 1u << st;
+    if (uses > 0) c.a_used |= 1u << st;
+  }
+}
+
+// Producer: issue attention tiles [from, to) of this CTA's run for layer l.
+__device__ void attn_issue(const TopArgs& a, Ctx& c, const AttnPlan& p, int l, int abuf, int from, int to) {
+  for (int t = from; t < to; ++t) {
+    const int st = t % kAStages;
+    if (ring_reused(c, st, t) &&
+        !wait_or_abort(a, c, bar_aempty(c, st), ring_parity(c, st, t) ^ 1u, DEV_WAIT_TIMEOUT_PRODUCER))
+      return;
+    const int w = t % p.npairs, j = t / p.npairs;
+    const int pair = p.pair0 + w;
+    const int k0 = j * kTK, rows = min(kTK, p.n - k0);
+    const long long row0 = (long long)pair * a.cap + k0;  // pair = g * H + h
+    const bf16* ks = a.kc + (long long)l * a.layer_elems + row0 * 64;
+    const bf16* vs = a.vc + (long long)l * a.layer_elems + row0 * 64;
+    const uint32_t bytes = (uint32_t)rows * 128u;
+    uint8_t* dst = ring_stage(c, st, abuf);
+    ptx::mbar_arrive_expect_tx(bar_afull(c, st), 2 * bytes);
+    ptx::bulk_load(ptx::smem_u32(dst), ks, bytes, bar_afull(c, st));
+    ptx::bulk_load(ptx::smem_u32(dst + kATile), vs, bytes, bar_afull(c, st));
+    c.a_pend |= 1u << st;
+    c.a_pend_par = (c.a_pend_par & ~(1u << st)) | (ring_parity(c, st, t) << st);
+  }
+}
+
+// Tiles at the start of the run that hold only keys of earlier steps (every
+// pair's last tile holds the new key) and go to the ring's own stages: safe
+// to copy while the QKV phase runs.
+__device__ __forceinline__ int attn_safe_tiles(const AttnPlan& p) {
+  if (p.npairs == 0) return 0;
+  return min(kAOwn, (p.tpp - 1) * p.npairs);
+}
+
+// Work the producer does once the phase's own token blocks have landed: the
+// next GEMM phase's weights, and (QKV phase) the first attention tiles.
+struct Deferred {
+  int wkind, wlayer, wbuf;  // weights to load (wkind PK_NONE: none)
+  int attn_layer, attn_abuf, attn_safe;
+  AttnPlan ap;
+};
+
+__device__ void run_deferred(const TopArgs& a, Ctx& c, const Deferred& df) {
+  if (*c.abort_cta) return;
+  if (df.wkind != PK_NONE) {
+    const GemmPhase g = gemm_phase(a, df.wkind, df.wlayer);
+    if (has_weights(c, g)) load_weights(c, g, df.wbuf, c.cluster);
+  }
+  if (df.attn_safe > 0) attn_issue(a, c, df.ap, df.attn_layer, df.attn_abuf, 0, df.attn_safe);
+}
+
+// One GEMM phase.  `armed`: this CTA's round-0 weights are in (or on their way
+// into) buffer `buf`.  The producer starts `df` once the token blocks are in.
+__device__ void run_gemm(const TopArgs& a, Ctx& c, const GemmPhase& g, int buf, bool armed, const Deferred& df) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int tid = threadIdx.x;
   const int units = (g.N / kBM) * g.pk;
@@ -264,32 +422,38 @@ __device__ void run_gemm(const TopArgs& a, Ctx& c, const GemmPhase& g, int buf, 
   const uint32_t xreg = ptx::smem_u32(c.smem + kOffX);
   float* P = reinterpret_cast<float*>(c.smem + kOffX);
   const int pos = (kind == PK_QKV) ? __ldcg(a.pos) : 0;
-
-  // 1 / rms of each token row from the producing phase's slots, in slot order
-  if (takes_rstd && tid < kBN) {
-    float tot = 0.f;
-    if (tid < a.B && *c.abort_cta == 0)
-      for (int s = 0; s < a.ssq_slots; ++s) tot += __ldcg(a.ssq + (long long)tid * a.ssq_slots + s);
-    c.rstd[tid] = 1.0f / sqrtf(tot / (float)a.d + a.eps);
-  }
+  bool deferred_done = false;
 
   for (int r = 0; r < rounds; ++r) {
     const int u = c.cluster + r * c.nclusters;
     const bool has = u < units;
     int tile = 0, kp = 0, kb0 = 0, nk = 0;
     if (has) unit_kbs(g, u, c.rank, tile, kp, kb0, nk);
-    const bool mine = has && nk > 0 && *c.abort_cta == 0;
-    if (r > 0 && mine) {
-      // later rounds reload the weight buffer (the previous round's MMAs are done)
-      issue_weights(c, g, buf, u);
-      c.wuse[buf] += 1;
-    }
+    const bool mine = has && nk > 0 && *c.ok_flag != 0;  // uniform within the CTA
+    if (r > 0 && mine) c.wuse[buf] += 1;                // later rounds reload the buffer
     const bool wready = (r == 0) ? armed : mine;
-    if (mine && tid == kProducer) {
-      asm volatile("fence.proxy.async.global;" ::: "memory");
-      ptx::mbar_arrive_expect_tx(bar_x(c), (uint32_t)(nk * kXTile));
-      for (int i = 0; i < nk; ++i) ptx::tma_load_2d(xreg + i * kXTile, g.xmap, (kb0 + i) * kBK, 0, bar_x(c));
-      c.x_armed += 1;
+    if (tid == kProducer) {
+      if (mine && *c.abort_cta == 0) {
+        if (r > 0) load_weights(c, g, buf, u);  // the previous round's MMAs are done
+        asm volatile("fence.proxy.async;" ::: "memory");
+        ptx::mbar_arrive_expect_tx(bar_x(c), (uint32_t)(nk * kXTile));
+        for (int i = 0; i < nk; ++i) ptx::tma_load_2d(xreg + i * kXTile, g.xmap, (kb0 + i) * kBK, 0, bar_x(c));
+        c.x_issued += 1;
+      }
+      if (!deferred_done) {
+        // the deferred copies follow the phase's own operands
+        if (mine) wait_or_abort(a, c, bar_x(c), c.xuse & 1u, DEV_WAIT_TIMEOUT_PRODUCER);
+        run_deferred(a, c, df);
+        deferred_done = true;
+      }
+    }
+    // 1 / rms of each token row from the producing phase's slots, in slot
+    // order (warps 2-3: the MMA thread in warp 0 goes straight to its waits)
+    if (r == 0 && takes_rstd && tid >= 64 && tid < 64 + kBN) {
+      const int row = tid - 64;
+      float tot = 0.f;
+      if (row < a.B && *c.abort_cta == 0) tot = sum_slots(a.ssq + (long long)row * a.ssq_slots, a.ssq_slots);
+      c.rstd[row] = 1.0f / sqrtf(tot / (float)a.d + a.eps);
     }
     // epilogue operands that do not depend on this phase: residual values or RoPE factors
     const int i = tid;  // workers only (tid < 256)
@@ -313,11 +477,13 @@ __device__ void run_gemm(const TopArgs& a, Ctx& c, const GemmPhase& g, int buf, 
         }
       }
     }
-    if (tid == 0 && mine) {
+    if (tid == kIssuer && mine) {
       // MMA issue: weights ready (buf), token blocks ready
       bool ok = true;
       if (wready) ok = wait_or_abort(a, c, bar_w(c, buf), (c.wuse[buf] - 1) & 1u, DEV_WAIT_TIMEOUT_MMA);
+      TOP_PT(c, 1);
       ok = ok && wait_or_abort(a, c, bar_x(c), c.xuse & 1u, DEV_WAIT_TIMEOUT_MMA);
+      TOP_PT(c, 2);
       if (ok) {
         ptx::tc_fence_after();
         constexpr uint32_t idesc = ptx::idesc_bf16_f32(kBM, kBN);
@@ -331,15 +497,15 @@ __device__ void run_gemm(const TopArgs& a, Ctx& c, const GemmPhase& g, int buf, 
       }
       ptx::mma_commit(bar_done(c));  // arrives once the MMAs (if any) are done
       c.mma_open = true;
+      TOP_PT(c, 0);
     }
-    __syncwarp();
-    if (mine) {
-      // every thread waits for the accumulator (a thread that gives up aborts the launch)
-      if (tid < kWorkers && wait_or_abort(a, c, bar_done(c), c.xuse & 1u, DEV_WAIT_TIMEOUT_EPILOGUE))
-        c.mma_open = false;
-      c.xuse += 1;
-    }
+    // the MMA thread waits for the accumulator; the other warps wait at the
+    // CTA barrier below (parked, not spinning)
+    if (tid == kIssuer && mine && wait_or_abort(a, c, bar_done(c), c.xuse & 1u, DEV_WAIT_TIMEOUT_EPILOGUE))
+      c.mma_open = false;
+    if (mine) c.xuse += 1;
     __syncthreads();
+    TOP_PT(c, 3);
     const bool live = mine && *c.abort_cta == 0;
     ptx::tc_fence_after();
     // accumulator -> partial tile in shared memory (row = feature, column = token)
@@ -376,6 +542,7 @@ __device__ void run_gemm(const TopArgs& a, Ctx& c, const GemmPhase& g, int buf, 
       }
     }
     ptx::cluster_arrive();  // done reading the peers' tiles
+    TOP_PT(c, 4);
     bool final_here = has;
     if (has && g.pk > 1) {
       // K parts of the same tile meet in global memory; the last to arrive sums them
@@ -385,33 +552,44 @@ __device__ void run_gemm(const TopArgs& a, Ctx& c, const GemmPhase& g, int buf, 
         *reinterpret_cast<float4*>(mine_part + (f0 + 32) * kBN + 4 * qd) =
             make_float4(s1[0], s1[1], s1[2], s1[3]);
       }
-      __threadfence();
       __syncthreads();
       if (tid == 0) {
-        const int old = atomicAdd(a.cnt + tile * kCS + c.rank, 1);
+        // release this CTA's partial, acquire the others' (whoever is last)
+        int old;
+        asm volatile("atom.acq_rel.gpu.global.add.s32 %0, [%1], 1;"
+                     : "=r"(old)
+                     : "l"(a.cnt + tile * kCS + c.rank)
+                     : "memory");
         const int last = old == g.pk - 1;
         if (last) a.cnt[tile * kCS + c.rank] = 0;  // ready for the next phase or launch
         *c.last_flag = last;
       }
       __syncthreads();
+      TOP_PT(c, 5);
       final_here = *c.last_flag != 0;
       if (final_here && tid < kWorkers) {
-        __threadfence();
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
           s0[e] = 0.f;
           s1[e] = 0.f;
         }
-        for (int p = 0; p < g.pk; ++p) {
-          const float* src = a.part + ((long long)(tile * g.pk + p) * kBM) * kBN;
-          const float4 x0 = __ldcg(reinterpret_cast<const float4*>(src + f0 * kBN + 4 * qd));
-          const float4 x1 = __ldcg(reinterpret_cast<const float4*>(src + (f0 + 32) * kBN + 4 * qd));
-          s0[0] += x0.x; s0[1] += x0.y; s0[2] += x0.z; s0[3] += x0.w;
-          s1[0] += x1.x; s1[1] += x1.y; s1[2] += x1.z; s1[3] += x1.w;
-        }
+        float4 x0[kMaxParts], x1[kMaxParts];
+#pragma unroll
+        for (int p = 0; p < kMaxParts; ++p)
+          if (p < g.pk) {
+            const float* src = a.part + ((long long)(tile * g.pk + p) * kBM) * kBN;
+            x0[p] = __ldcg(reinterpret_cast<const float4*>(src + f0 * kBN + 4 * qd));
+            x1[p] = __ldcg(reinterpret_cast<const float4*>(src + (f0 + 32) * kBN + 4 * qd));
+          }
+#pragma unroll
+        for (int p = 0; p < kMaxParts; ++p)
+          if (p < g.pk) {
+            s0[0] += x0[p].x; s0[1] += x0[p].y; s0[2] += x0[p].z; s0[3] += x0[p].w;
+            s1[0] += x1[p].x; s1[1] += x1[p].y; s1[2] += x1[p].z; s1[3] += x1[p].w;
+          }
       }
     }
-    // ---- epilogue of this CTA's item (a whole warp takes part: the sum of
+    // ---- epilogue of this CTA's item (every worker takes part: the sum of
     // squares below is a butterfly over the 16 lanes of a token quad)
     if (final_here && tid < kWorkers) {
       const bool ok = *c.abort_cta == 0;
@@ -457,7 +635,7 @@ __device__ void run_gemm(const TopArgs& a, Ctx& c, const GemmPhase& g, int buf, 
         // residual stream (CH: store; O, W2: add) + split-RMSNorm producer
         const float* gn = kind == PK_CH ? a.g_attn[0]
                           : kind == PK_O ? a.g_mlp[g.layer]
-                          : (g.layer + 1 < a.L ? a.g_attn[g.layer + 1] : a.g_final);
+                                         : (g.layer + 1 < a.L ? a.g_attn[g.layer + 1] : a.g_final);
         const float gn0 = gn[gf], gn1 = gn[gf + 32];
         float ss[4];
 #pragma unroll
@@ -487,94 +665,61 @@ __device__ void run_gemm(const TopArgs& a, Ctx& c, const GemmPhase& g, int buf, 
         }
       }
     }
+    TOP_PT(c, 6);
     ptx::cluster_wait();  // the peers are done reading this CTA's partial tile
   }
+  if (tid == kProducer && !deferred_done) run_deferred(a, c, df);
 }
 
-// ---- attention: one query per (sequence, head) pair over keys 0..pos ------
-struct AttnPlan {
-  int pair0, npairs, tpp, n;
-};
-__device__ __forceinline__ AttnPlan attn_plan(const TopArgs& a, int pos) {
-  AttnPlan p;
-  const int pairs = a.B * a.H;
-  const int per = (pairs + gridDim.x - 1) / gridDim.x;
-  p.pair0 = blockIdx.x * per;
-  p.npairs = max(0, min(per, pairs - p.pair0));
-  p.n = pos + 1 - a.kv_off;  // keys in the cache, the new one included
-  p.tpp = (p.n + kTK - 1) / kTK;
-  return p;
-}
-
-// Producer: issue attention tiles [from, to) of this CTA's run for layer l.
-__device__ void attn_issue(const TopArgs& a, Ctx& c, const AttnPlan& p, int l, int from, int to) {
-  for (int t = from; t < to; ++t) {
-    const uint32_t gt = c.at + (uint32_t)t;  // ring position
-    const int st = (int)(gt % kAStages);
-    const uint32_t ph = (gt / kAStages) & 1u;
-    if (gt >= kAStages && !wait_or_abort(a, c, bar_aempty(c, st), ph ^ 1u, DEV_WAIT_TIMEOUT_PRODUCER)) return;
-    const int pair = p.pair0 + t / p.tpp, j = t % p.tpp;
-    const int k0 = j * kTK, rows = min(kTK, p.n - k0);
-    const long long row0 = (long long)pair * a.cap + k0;  // pair = g * H + h
-    const bf16* ks = a.kc + (long long)l * a.layer_elems + row0 * 64;
-    const bf16* vs = a.vc + (long long)l * a.layer_elems + row0 * 64;
-    const uint32_t bytes = (uint32_t)rows * 128u;
-    ptx::mbar_arrive_expect_tx(bar_afull(c, st), 2 * bytes);
-    ptx::bulk_load(ptx::smem_u32(c.smem + kOffA + st * kAStage), ks, bytes, bar_afull(c, st));
-    ptx::bulk_load(ptx::smem_u32(c.smem + kOffA + st * kAStage + kATile), vs, bytes, bar_afull(c, st));
-    c.at_issued = gt + 1;
-  }
-}
-
-// Tiles at the start of the run that hold only keys of earlier steps (safe
-// to copy before this step's QKV phase has written the new key).
-__device__ __forceinline__ int attn_safe_tiles(const AttnPlan& p) {
-  const int total = p.npairs * p.tpp;
-  if (p.npairs == 0) return 0;
-  return min(min(kAStages, total), p.tpp - 1);
-}
-
-__device__ void run_attention(const TopArgs& a, Ctx& c, int l, int pos) {
+// One warp per (sequence, head) pair: warp w streams pair w's K and V tiles
+// (8 lanes per 128-byte row, 4 rows per access, 16 accesses per 64-row
+// tile), keeps its own online softmax and writes the pair's output; no
+// cross-warp merge.
+__device__ void run_attention(const TopArgs& a, Ctx& c, int l, int pos, int abuf) {
   const AttnPlan p = attn_plan(a, pos);
   const int total = p.npairs * p.tpp;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const bool qcopy = p.npairs > 0 && *c.ok_flag != 0;  // uniform
   if (threadIdx.x == kProducer) {
-    asm volatile("fence.proxy.async.global;" ::: "memory");
-    if (*c.abort_cta == 0) attn_issue(a, c, p, l, (int)c.pre, total);
+    asm volatile("fence.proxy.async;" ::: "memory");
+    if (qcopy && *c.abort_cta == 0) {
+      // the query rows of this CTA's consecutive pairs: one contiguous run
+      ptx::mbar_arrive_expect_tx(bar_q(c), (uint32_t)p.npairs * 128u);
+      ptx::bulk_load(ptx::smem_u32(c.smem + kOffCtrl + kCtrlQ), a.q + (long long)p.pair0 * 64,
+                     (uint32_t)p.npairs * 128u, bar_q(c));
+      c.q_issued = true;
+    }
+    if (*c.abort_cta == 0) attn_issue(a, c, p, l, abuf, (int)c.pre, total);
   }
-  if (threadIdx.x < kWorkers) {
-    constexpr int VEC = 8, TPK = 8, GPW = 4, KPW = kTK / kAWarps, U = KPW / GPW;
-    float* sm_m = reinterpret_cast<float*>(c.smem + kOffCtrl + kCtrlM);
-    float* sm_l = reinterpret_cast<float*>(c.smem + kOffCtrl + kCtrlL);
-    float* sm_acc = reinterpret_cast<float*>(c.smem + kOffCtrl + kCtrlAcc);
+  if (threadIdx.x < kWorkers && warp < p.npairs) {
+    constexpr int VEC = 8, TPK = 8, GPW = 4, G = kTK / GPW;  // 16 four-row groups per tile
     const int kg = lane / TPK, sl = lane % TPK;
-    float qv[VEC], acc[VEC], m = -INFINITY, lsum = 0.f;
+    const uint8_t* qrows = c.smem + kOffCtrl + kCtrlQ;
     bool ok = *c.abort_cta == 0;
-    for (int t = 0; t < total; ++t) {
-      const uint32_t gt = c.at + (uint32_t)t;
-      const int st = (int)(gt % kAStages);
-      const uint32_t ph = (gt / kAStages) & 1u;
-      const int pair = p.pair0 + t / p.tpp, j = t % p.tpp;
-      if (ok && !wait_or_abort(a, c, bar_afull(c, st), ph, DEV_WAIT_TIMEOUT_EPILOGUE)) ok = false;
-      const uint8_t* kt = c.smem + kOffA + st * kAStage;
-      const uint8_t* vt = kt + kATile;
-      if (j == 0) {
-        uint4 raw = make_uint4(0u, 0u, 0u, 0u);
-        if (ok) raw = __ldcg(reinterpret_cast<const uint4*>(a.q + (long long)pair * 64 + sl * VEC));
-        const bf16* qp = reinterpret_cast<const bf16*>(&raw);
+    if (qcopy && ok && !wait_or_abort(a, c, bar_q(c), c.quse & 1u, DEV_WAIT_TIMEOUT_EPILOGUE)) ok = false;
+    float qv[VEC], acc[VEC], m = -INFINITY, lsum = 0.f;
+    {
+      uint4 raw = make_uint4(0u, 0u, 0u, 0u);
+      if (ok) raw = *reinterpret_cast<const uint4*>(qrows + warp * 128 + sl * 16);
+      const bf16* qp = reinterpret_cast<const bf16*>(&raw);
 #pragma unroll
-        for (int e = 0; e < VEC; ++e) {
-          qv[e] = __bfloat162float(qp[e]) * a.scale;
-          acc[e] = 0.f;
-        }
-        m = -INFINITY;
-        lsum = 0.f;
+      for (int e = 0; e < VEC; ++e) {
+        qv[e] = __bfloat162float(qp[e]) * a.scale;
+        acc[e] = 0.f;
       }
+    }
+    for (int j = 0; j < p.tpp; ++j) {
+      const int t = j * p.npairs + warp;
+      const int st = t % kAStages;
+      if (ok && !wait_or_abort(a, c, bar_afull(c, st), ring_parity(c, st, t), DEV_WAIT_TIMEOUT_EPILOGUE)) ok = false;
+      const uint8_t* kt = ring_stage(c, st, abuf);
+      const uint8_t* vt = kt + kATile;
       const int rows = min(kTK, p.n - j * kTK);
-      float sc[U];
+      float sc[G];
+      float mx = -INFINITY;
 #pragma unroll
-      for (int u = 0; u < U; ++u) {
-        const int r = warp * KPW + u * GPW + kg;
+      for (int g = 0; g < G; ++g) {
+        const int r = g * GPW + kg;
         float dd = 0.f;
         if (ok) {
           const uint4 kraw = *reinterpret_cast<const uint4*>(kt + r * 128 + sl * 16);
@@ -584,89 +729,63 @@ __device__ void run_attention(const TopArgs& a, Ctx& c, int l, int pos) {
         }
 #pragma unroll
         for (int o = TPK / 2; o > 0; o >>= 1) dd += __shfl_xor_sync(0xffffffffu, dd, o);
-        sc[u] = (r < rows && ok) ? dd : -INFINITY;
+        sc[g] = (r < rows && ok) ? dd : -INFINITY;
+        mx = fmaxf(mx, sc[g]);
       }
-      float mx = sc[0];
 #pragma unroll
-      for (int u = 1; u < U; ++u) mx = fmaxf(mx, sc[u]);
+      for (int o = TPK; o < 32; o <<= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
       if (mx != -INFINITY) {
         const float mn = fmaxf(m, mx);
-        const float cf = __expf(m - mn);
-        float pe[U], ps = 0.f;
-#pragma unroll
-        for (int u = 0; u < U; ++u) {
-          pe[u] = __expf(sc[u] - mn);
-          ps += pe[u];
-        }
-        lsum = lsum * cf + ps;
+        const float cf = __expf(m - mn);  // 0 while m is -inf
+        float ps = 0.f;
 #pragma unroll
         for (int e = 0; e < VEC; ++e) acc[e] *= cf;
 #pragma unroll
-        for (int u = 0; u < U; ++u) {
-          if (sc[u] == -INFINITY) continue;
-          const int r = warp * KPW + u * GPW + kg;
-          const uint4 vraw = *reinterpret_cast<const uint4*>(vt + r * 128 + sl * 16);
-          const bf16* vp = reinterpret_cast<const bf16*>(&vraw);
+        for (int g = 0; g < G; ++g) {
+          const float pe = sc[g] == -INFINITY ? 0.f : __expf(sc[g] - mn);
+          ps += pe;
+          if (pe != 0.f) {
+            const uint4 vraw = *reinterpret_cast<const uint4*>(vt + (g * GPW + kg) * 128 + sl * 16);
+            const bf16* vp = reinterpret_cast<const bf16*>(&vraw);
 #pragma unroll
-          for (int e = 0; e < VEC; ++e) acc[e] = fmaf(pe[u], __bfloat162float(vp[e]), acc[e]);
+            for (int e = 0; e < VEC; ++e) acc[e] = fmaf(pe, __bfloat162float(vp[e]), acc[e]);
+          }
         }
+        // the 8 lanes of a row group hold the same scores: one group's sum per row
+#pragma unroll
+        for (int o = TPK; o < 32; o <<= 1) ps += __shfl_xor_sync(0xffffffffu, ps, o);
+        lsum = lsum * cf + ps;
         m = mn;
       }
       __syncwarp();
       if (lane == 0) ptx::mbar_arrive(bar_aempty(c, st));  // this warp is done with the stage
-      if (j == p.tpp - 1) {
-        const int buf = (t / p.tpp) & 1;
-        float M = m;
+    }
+    // the four row groups of the warp hold partial sums of the same output slice
 #pragma unroll
-        for (int o = TPK; o < 32; o <<= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
-        const float cf = (M == -INFINITY) ? 0.f : __expf(m - M);
-        float L = lsum * cf;
+    for (int e = 0; e < VEC; ++e) {
 #pragma unroll
-        for (int o = TPK; o < 32; o <<= 1) L += __shfl_xor_sync(0xffffffffu, L, o);
+      for (int o = TPK; o < 32; o <<= 1) acc[e] += __shfl_xor_sync(0xffffffffu, acc[e], o);
+    }
+    if (ok && kg == 0) {
+      const float inv = lsum > 0.f ? 1.0f / lsum : 0.f;
+      uint4 out;
+      uint32_t* ow = reinterpret_cast<uint32_t*>(&out);
 #pragma unroll
-        for (int e = 0; e < VEC; ++e) {
-          float v = acc[e] * cf;
-#pragma unroll
-          for (int o = TPK; o < 32; o <<= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-          if (lane < TPK) sm_acc[(buf * kAWarps + warp) * 64 + sl * VEC + e] = v;
-        }
-        if (lane == 0) {
-          sm_m[buf * kAWarps + warp] = M;
-          sm_l[buf * kAWarps + warp] = L;
-        }
-        asm volatile("bar.sync 1, %0;" ::"n"(kWorkers) : "memory");  // the 8 worker warps
-        const int dd = threadIdx.x;
-        if (dd < 64 && ok) {
-          float Mx = -INFINITY;
-#pragma unroll
-          for (int w = 0; w < kAWarps; ++w) Mx = fmaxf(Mx, sm_m[buf * kAWarps + w]);
-          float Ls = 0.f, v = 0.f;
-#pragma unroll
-          for (int w = 0; w < kAWarps; ++w) {
-            const float mw = sm_m[buf * kAWarps + w];
-            const float cw = (mw == -INFINITY) ? 0.f : __expf(mw - Mx);
-            Ls += cw * sm_l[buf * kAWarps + w];
-            v += cw * sm_acc[(buf * kAWarps + w) * 64 + dd];
-          }
-          st_f(a.att + (long long)pair * 64 + dd, Ls > 0.f ? v / Ls : 0.f);
-        }
-      }
+      for (int e = 0; e < VEC / 2; ++e) ow[e] = pack2_bf16(acc[2 * e] * inv, acc[2 * e + 1] * inv);
+      *reinterpret_cast<uint4*>(a.att + (long long)(p.pair0 + warp) * 64 + sl * VEC) = out;
     }
   }
-  c.at += (uint32_t)total;
+  if (qcopy) c.quse += 1;
+  ring_advance(c, total);
   c.pre = 0;
 }
 
 // Final norm of the residual stream: o = bf16(x * rstd * g_final), one row per CTA.
 __device__ void run_final_norm(const TopArgs& a, Ctx& c) {
-  if (*c.abort_cta) return;
   for (int row = blockIdx.x; row < a.B; row += gridDim.x) {
     __shared__ float s_rstd;
-    if (threadIdx.x == 0) {
-      float tot = 0.f;
-      for (int s = 0; s < a.ssq_slots; ++s) tot += __ldcg(a.ssq + (long long)row * a.ssq_slots + s);
-      s_rstd = 1.0f / sqrtf(tot / (float)a.d + a.eps);
-    }
+    if (threadIdx.x == 0) s_rstd = 1.0f / sqrtf(sum_slots(a.ssq + (long long)row * a.ssq_slots, a.ssq_slots) /
+                                                  (float)a.d + a.eps);
     __syncthreads();
     const float rs = s_rstd;
     for (int col = threadIdx.x; col < a.d; col += blockDim.x)
@@ -689,23 +808,29 @@ __global__ void __launch_bounds__(kThreads, 1) k_top_step(const __grid_constant_
   c.rstd = reinterpret_cast<float*>(ctrl + kCtrlRstd);
   c.wuse[0] = c.wuse[1] = 0;
   c.xuse = 0;
-  c.at = 0;
+  c.quse = 0;
+  c.a_par = 0;
+  c.a_used = 0;
   c.pre = 0;
   c.nbar = 0;
   c.rank = (int)ptx::cluster_ctarank();
   c.cluster = blockIdx.x / kCS;
   c.nclusters = gridDim.x / kCS;
-  c.x_armed = 0;
-  c.at_issued = 0;
+  c.w_issued[0] = c.w_issued[1] = 0;
+  c.x_issued = 0;
+  c.q_issued = false;
+  c.a_pend = c.a_pend_par = 0;
   c.mma_open = false;
   const int warp = threadIdx.x >> 5;
   if (threadIdx.x == 0) {
     for (int b = 0; b < 4; ++b) ptx::mbar_init(ptx::smem_u32(c.bars + b), 1);  // weights x2, tokens, done
     for (int st = 0; st < kAStages; ++st) {
       ptx::mbar_init(bar_afull(c, st), 1);
-      ptx::mbar_init(bar_aempty(c, st), kAWarps);  // one arrival per worker warp
+      ptx::mbar_init(bar_aempty(c, st), 1);  // the one warp that reads the tile
     }
+    ptx::mbar_init(bar_q(c), 1);
     *c.abort_cta = 0;
+    *c.ok_flag = 1;
     ptx::fence_barrier_init();
   }
   if (warp == 0) {
@@ -720,83 +845,128 @@ __global__ void __launch_bounds__(kThreads, 1) k_top_step(const __grid_constant_
   // Chunker_2's weights (buffer 0) and the first QKV's (buffer 1) before
   // waiting for the previous kernel: weights are never written by any kernel
   const GemmPhase g0 = gemm_phase(a, PK_CH, 0);
-  const bool armed0 = issue_weights(c, g0, 0, c.cluster);
+  const GemmPhase gq0 = gemm_phase(a, PK_QKV, 0);
+  const bool armed0 = has_weights(c, g0), armed1 = has_weights(c, gq0);
+  if (threadIdx.x == kProducer) {
+    if (armed0) load_weights(c, g0, 0, c.cluster);
+    if (armed1) load_weights(c, gq0, 1, c.cluster);
+  }
   if (armed0) c.wuse[0] += 1;
-  const bool armed1 = issue_weights(c, gemm_phase(a, PK_QKV, 0), 1, c.cluster);
   if (armed1) c.wuse[1] += 1;
   pdl_wait();
+#ifdef PHOTON_TOP_TRACE
+  if (threadIdx.x == 0 && blockIdx.x == 0) g_top_trace[0] = gtimer();
+#endif
 
   // Every phase function runs on every CTA even after an abort (they then
   // skip their work), so all CTAs of a cluster take the same cluster
-  // barriers and all CTAs the same grid barriers.
-  run_gemm(a, c, g0, 0, armed0);
+  // barriers and all CTAs the same grid barriers.  Weight buffers: the
+  // layer's QKV and W1 use `buf`, O and W2 `buf ^ 1`; each phase's producer
+  // loads the next phase's weights once its own token blocks are in.
+  const int buf = 1;
+  Deferred none;
+  none.wkind = PK_NONE;
+  none.attn_safe = 0;
+  run_gemm(a, c, g0, 0, armed0, none);
   grid_barrier(a, c);
   const int pos = __ldcg(a.pos);
-  int buf = 1;  // weight buffer of the layer's QKV (and W1); O and W2 use buf ^ 1
+  const AttnPlan ap = attn_plan(a, pos);
   bool armed_q = armed1;
   for (int l = 0; l < a.L; ++l) {
     const GemmPhase gq = gemm_phase(a, PK_QKV, l);
     const GemmPhase gop = gemm_phase(a, PK_O, l);
     const GemmPhase g1 = gemm_phase(a, PK_W1, l);
     const GemmPhase g2 = gemm_phase(a, PK_W2, l);
-    const bool live = *c.ok_flag != 0 && *c.abort_cta == 0;  // uniform: set by the last grid barrier
-    // ---- QKV; O's weights into the other buffer; the first attention tiles
-    const bool armed_o = live && issue_weights(c, gop, buf ^ 1, c.cluster);
+    // ---- QKV; then O's weights and the first attention tiles
+    bool live = *c.ok_flag != 0;  // uniform: set by the last grid barrier
+    Deferred dq;
+    dq.wkind = PK_O;
+    dq.wlayer = l;
+    dq.wbuf = buf ^ 1;
+    dq.attn_layer = l;
+    dq.attn_abuf = buf;
+    dq.attn_safe = live ? attn_safe_tiles(ap) : 0;
+    dq.ap = ap;
+    const bool armed_o = live && has_weights(c, gop);
     if (armed_o) c.wuse[buf ^ 1] += 1;
-    const AttnPlan ap = attn_plan(a, pos);
-    const int safe = live ? attn_safe_tiles(ap) : 0;
-    if (threadIdx.x == kProducer && safe > 0) attn_issue(a, c, ap, l, 0, safe);
-    c.pre = (uint32_t)safe;
-    run_gemm(a, c, gq, buf, armed_q);
+    c.pre = (uint32_t)dq.attn_safe;
+    run_gemm(a, c, gq, buf, armed_q, dq);
     grid_barrier(a, c);
-    // ---- attention; W1's weights into the QKV buffer (its MMAs are done)
-    const bool armed_w1 = *c.ok_flag != 0 && issue_weights(c, g1, buf, c.cluster);
+    // ---- attention (borrows buffer `buf` and the token region)
+    run_attention(a, c, l, pos, buf);
+    grid_barrier(a, c);
+    // ---- O; then W1's weights into `buf`
+    live = *c.ok_flag != 0;
+    Deferred d1;
+    d1.wkind = PK_W1;
+    d1.wlayer = l;
+    d1.wbuf = buf;
+    d1.attn_safe = 0;
+    const bool armed_w1 = live && has_weights(c, g1);
     if (armed_w1) c.wuse[buf] += 1;
-    run_attention(a, c, l, pos);
+    run_gemm(a, c, gop, buf ^ 1, armed_o, d1);
     grid_barrier(a, c);
-    // ---- O; the next layer's cached keys and values toward L2 meanwhile
-    if (a.l2_prefetch && l + 1 < a.L && threadIdx.x == kProducer && *c.ok_flag != 0) {
-      const int old = ap.n - 1;
-      if (old > 0)
-        for (int pp = 0; pp < ap.npairs; ++pp) {
-          const long long row0 = (long long)(ap.pair0 + pp) * a.cap;
-          ptx::bulk_prefetch_l2(a.kc + (long long)(l + 1) * a.layer_elems + row0 * 64, (uint32_t)old * 128u);
-          ptx::bulk_prefetch_l2(a.vc + (long long)(l + 1) * a.layer_elems + row0 * 64, (uint32_t)old * 128u);
-        }
-    }
-    run_gemm(a, c, gop, buf ^ 1, armed_o);
-    grid_barrier(a, c);
-    // ---- W1; W2's weights into the O buffer
-    const bool armed_w2 = *c.ok_flag != 0 && issue_weights(c, g2, buf ^ 1, c.cluster);
+    // ---- W1; then W2's weights
+    live = *c.ok_flag != 0;
+    Deferred d2;
+    d2.wkind = PK_W2;
+    d2.wlayer = l;
+    d2.wbuf = buf ^ 1;
+    d2.attn_safe = 0;
+    const bool armed_w2 = live && has_weights(c, g2);
     if (armed_w2) c.wuse[buf ^ 1] += 1;
-    run_gemm(a, c, g1, buf, armed_w1);
+    run_gemm(a, c, g1, buf, armed_w1, d2);
     grid_barrier(a, c);
-    // ---- W2; the next layer's QKV weights into the W1 buffer
-    armed_q = false;
-    if (l + 1 < a.L) {
-      armed_q = *c.ok_flag != 0 && issue_weights(c, gemm_phase(a, PK_QKV, l + 1), buf, c.cluster);
-      if (armed_q) c.wuse[buf] += 1;
-    }
-    run_gemm(a, c, g2, buf ^ 1, armed_w2);
+    // ---- W2; then the next layer's QKV weights
+    live = *c.ok_flag != 0;
+    Deferred dn;
+    dn.wkind = l + 1 < a.L ? PK_QKV : PK_NONE;
+    dn.wlayer = l + 1;
+    dn.wbuf = buf;
+    dn.attn_safe = 0;
+    armed_q = live && l + 1 < a.L && has_weights(c, gemm_phase(a, PK_QKV, l + 1));
+    if (armed_q) c.wuse[buf] += 1;
+    run_gemm(a, c, g2, buf ^ 1, armed_w2, dn);
     grid_barrier(a, c);
   }
-  const bool done_ok = *c.ok_flag != 0 && *c.abort_cta == 0;
+  const bool done_ok = *c.ok_flag != 0;
   // every CTA has passed its last read of the positions: advance them
   if (done_ok && blockIdx.x == 0 && threadIdx.x == 0) {
     a.pos[0] += 1;
     if (a.dN1) a.pos[1] += a.dN1;
   }
   if (done_ok) run_final_norm(a, c);
+#ifdef PHOTON_TOP_TRACE
+  if (blockIdx.x == 0 && threadIdx.x == 0) {
+    const unsigned int k = atomicAdd(&g_top_trace_launch, 1u);
+    if (k >= 4 && k < 7) {
+      const unsigned long long e = gtimer();
+      printf("top_step trace launch %u: total %.2f us; phases (us):", k, (e - g_top_trace[0]) * 1e-3);
+      for (int i = 1; i <= c.nbar && i < 128; ++i) printf(" %.2f", (g_top_trace[i] - g_top_trace[i - 1]) * 1e-3);
+      printf("\n");
+      for (int ph = 6; ph <= 10; ++ph) {
+        printf("  phase %d:", ph);
+        for (int k2 = 0; k2 < 8; ++k2)
+          if (g_top_pts[ph][k2] > g_top_trace[ph])
+            printf(" p%d=%.2f", k2, (g_top_pts[ph][k2] - g_top_trace[ph]) * 1e-3);
+        printf(" end=%.2f\n", (g_top_trace[ph + 1] - g_top_trace[ph]) * 1e-3);
+      }
+      for (int i = 0; i < 128; ++i)
+        for (int k2 = 0; k2 < 8; ++k2) g_top_pts[i][k2] = 0;
+    }
+  }
+#endif
   // after an abort, copies and MMAs still in flight land before the CTA exits
   if (*c.abort_cta) {
     if (threadIdx.x == kProducer) {
       for (int b = 0; b < 2; ++b)
-        if (c.wuse[b] > 0) ptx::mbar_wait(bar_w(c, b), (c.wuse[b] - 1) & 1u, nullptr);
-      if (c.x_armed > 0) ptx::mbar_wait(bar_x(c), (c.x_armed - 1) & 1u, nullptr);
-      for (uint32_t u = c.at_issued > kAStages ? c.at_issued - kAStages : 0; u < c.at_issued; ++u)
-        ptx::mbar_wait(bar_afull(c, (int)(u % kAStages)), (u / kAStages) & 1u, nullptr);
+        if (c.w_issued[b] > 0) ptx::mbar_wait(bar_w(c, b), (c.w_issued[b] - 1) & 1u, nullptr);
+      if (c.x_issued > 0) ptx::mbar_wait(bar_x(c), (c.x_issued - 1) & 1u, nullptr);
+      if (c.q_issued) ptx::mbar_wait(bar_q(c), (c.quse - 1) & 1u, nullptr);
+      for (int st = 0; st < kAStages; ++st)
+        if (c.a_pend & (1u << st)) ptx::mbar_wait(bar_afull(c, st), (c.a_pend_par >> st) & 1u, nullptr);
     }
-    if (threadIdx.x == 0 && c.mma_open) ptx::mbar_wait(bar_done(c), (c.xuse - 1) & 1u, nullptr);
+    if (threadIdx.x == kIssuer && c.mma_open) ptx::mbar_wait(bar_done(c), (c.xuse - 1) & 1u, nullptr);
   }
   pdl_trigger();
   ptx::tc_fence_before();
@@ -864,11 +1034,14 @@ static int kparts(int nkb) {
   return pk;
 }
 
+int top_step_ssq_slots(int d) { return (d / kBM) * kCS; }
+
 bool top_step_supported(int B, int d, int H, int dh, int f, int L, int C2, int cap) {
   if (B < 1 || B > kBN || dh != 64 || d != H * 64 || d % kBM || f % kBM || L < 1 || L > kTopMaxLayers) return false;
   if (d / kBK > kCS * kKbMax || cap < 1) return false;  // QKV and W1 take one K part
+  if (top_step_ssq_slots(d) > kMaxSlots || kparts(f / kBK) > kMaxParts || kparts(C2 * d / kBK) > kMaxParts)
+    return false;
   if (!tma_available() || top_clusters_resident() < 1) return false;
-  (void)C2;
   return true;
 }
 
@@ -886,13 +1059,18 @@ static int top_grid_clusters(int d, int f, int C2) {
 }
 
 size_t top_step_part_bytes(int d, int f, int C2) {
+  // a partial tile per unit of a K-split phase: at most one round of
+  // clusters, or the minimum K parts of every tile
   int pk = kparts(d / kBK);
   pk = pk > kparts(f / kBK) ? pk : kparts(f / kBK);
   pk = pk > kparts(C2 * d / kBK) ? pk : kparts(C2 * d / kBK);
-  return (size_t)(d / kBM) * pk * kBM * kBN * sizeof(float);
+  int units = (d / kBM) * pk;
+  const int nc = top_grid_clusters(d, f, C2);
+  units = units > nc ? units : nc;
+  return (size_t)units * kBM * kBN * sizeof(float);
 }
 int top_step_counters(int d) { return (3 * d / kBM > d / kBM ? 3 * d / kBM : d / kBM) * kCS + 64; }
-int top_step_ssq_slots(int d) { return (d / kBM) * kCS; }
+
 
 TopStepPlan* top_step_plan(const TopStepLaunch& s) {
   const int d = s.d, f = s.f, L = s.L, B = s.B;
@@ -947,17 +1125,22 @@ TopStepPlan* top_step_plan(const TopStepLaunch& s) {
   // when the grid has room (each CTA then holds fewer weight blocks)
   const int nc = top_grid_clusters(d, f, s.C2);
   auto widen = [&](int pk, int nkb) {
-    while ((d / kBM) * (pk + 1) <= nc && (nkb + pk) / (pk + 1) >= kCS && pk < 16) ++pk;
+    while ((d / kBM) * (pk + 1) <= nc && (nkb + pk) / (pk + 1) >= kCS && pk < kMaxParts) ++pk;
     return pk;
   };
-  a.pk_o = widen(a.pk_o, d / kBK);
-  a.pk_w2 = widen(a.pk_w2, f / kBK);
-  a.pk_ch = widen(a.pk_ch, a.nkb_ch);
+  if (env_int("PHOTON_TOP_WIDEN", 0)) {
+    a.pk_o = widen(a.pk_o, d / kBK);
+    a.pk_w2 = widen(a.pk_w2, f / kBK);
+    a.pk_ch = widen(a.pk_ch, a.nkb_ch);
+  }
   a.ssq_slots = top_step_ssq_slots(d);
   a.eps = s.eps;
   a.scale = s.scale;
-  a.l2_prefetch = env_int("PHOTON_TOP_L2_PREFETCH", 1);
   p->grid = nc * kCS;
+  if ((B * s.H + p->grid - 1) / p->grid > kMaxPairsPerCta) {  // the query rows of one CTA's pairs
+    delete p;
+    return nullptr;
+  }
   if (nc < 1 || (size_t)(d / kBM) * (a.pk_o > a.pk_w2 ? (a.pk_o > a.pk_ch ? a.pk_o : a.pk_ch)
                                                        : (a.pk_w2 > a.pk_ch ? a.pk_w2 : a.pk_ch)) *
                         kBM * kBN * sizeof(float) > s.part_bytes) {

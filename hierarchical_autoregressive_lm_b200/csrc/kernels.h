@@ -175,6 +175,9 @@ void launch_logprob(const float* logits, int V, const int32_t* target, float* ou
 void launch_argmax_partials(const unsigned long long* part, int tiles, int rows, int V, int i,
                             int C1, const int32_t* force, int32_t* own, int32_t* used,
                             int32_t* next_ids, int* err, int* chunk_ctr, cudaStream_t s);
+// One thread waits on an mbarrier nothing arrives on, with a budget of
+// `limit` cycles, through the kernels' bounded wait; sets *err on expiry.
+void launch_wait_selftest(long long limit, int* err, cudaStream_t s);
 // pos[0] += dN; pos[1] += dN1 (device-side decode positions).
 void launch_advance(int* pos, int dN, int dN1, cudaStream_t s);
 

@@ -46,14 +46,19 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 // Waits for the phase with the given parity to complete.  Returns false if
-// the budget runs out or *abort becomes non-zero (another role gave up).
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort) {
+// `limit` clock cycles pass or *abort becomes non-zero (another role gave up).
+__device__ __forceinline__ bool mbar_wait_limit(uint32_t bar, uint32_t parity, volatile int* abort,
+                                                long long limit) {
   const long long t0 = clock64();
   while (!mbar_try_wait(bar, parity)) {
     if (abort && *abort) return false;
-    if (clock64() - t0 > kWaitLimitCycles) return false;
+    if (clock64() - t0 > limit) return false;
   }
   return true;
+}
+// The kernels' bounded wait: mbar_wait_limit with the library's budget.
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort) {
+  return mbar_wait_limit(bar, parity, abort, kWaitLimitCycles);
 }
 
 // ---------------------------------------------------------------- TMA

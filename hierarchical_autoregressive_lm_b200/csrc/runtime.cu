@@ -12,6 +12,7 @@
 #include <cstdlib>
 #include <cstdio>
 #include <cstring>
+#include <atomic>
 #include <mutex>
 #include <string>
 #include <vector>
@@ -229,7 +230,22 @@ static cudaError_t library_pool(cudaMemPool_t* out) {
   return cudaSuccess;
 }
 
+// Test hook (photon_debug_fail_alloc): the n-th device allocation from now
+// on fails as if the device were out of memory; 0 = off.
+static std::atomic<long long> g_fail_alloc{0};
+static bool injected_alloc_failure() {
+  long long v = g_fail_alloc.load();
+  while (v > 0) {
+    if (g_fail_alloc.compare_exchange_weak(v, v - 1)) return v == 1;
+  }
+  return false;
+}
+
 static cudaError_t pool_malloc(void** p, size_t bytes, cudaStream_t s) {
+  if (injected_alloc_failure()) {
+    *p = nullptr;
+    return cudaErrorMemoryAllocation;
+  }
   cudaMemPool_t pool = nullptr;
   cudaError_t e = library_pool(&pool);
   if (e != cudaSuccess) return e;
@@ -725,6 +741,27 @@ extern "C" {
 
 const char* photon_last_error(void) { return g_err.c_str(); }
 
+int photon_debug_fail_alloc(int64_t n) {
+  g_err.clear();
+  if (n < 0) return fail(PHOTON_ERR_ARG, "n must be >= 0");
+  g_fail_alloc.store(n);
+  return PHOTON_OK;
+}
+
+int photon_selftest_wait_timeout(int64_t limit_cycles, int32_t* d_err, void* stream) {
+  g_err.clear();
+  if (!d_err || limit_cycles < 0) return fail(PHOTON_ERR_ARG, "bad arguments");
+  cudaStream_t s = (cudaStream_t)stream;
+  CK(cudaMemsetAsync(d_err, 0, sizeof(int32_t), s));
+  launch_wait_selftest((long long)limit_cycles, d_err, s);
+  CK(cudaGetLastError());
+  int32_t h = 0;
+  CK(cudaMemcpyAsync(&h, d_err, sizeof(int32_t), cudaMemcpyDeviceToHost, s));
+  CK(cudaStreamSynchronize(s));
+  if (h != 0) return fail(PHOTON_ERR_DEVICE_CHECK, "device wait timed out (code %d)", h);
+  return PHOTON_OK;
+}
+
 uint64_t photon_launch_count(void) { return (uint64_t)launch_total(); }
 
 int photon_init_weights(const photon_config* cfg, uint64_t seed, photon_model** out) {
@@ -755,7 +792,8 @@ int photon_init_weights(const photon_config* cfg, uint64_t seed, photon_model** 
   build_specs(m);
   cudaStream_t s = nullptr;
   for (int g = 0; g < G_COUNT; ++g) {
-    cudaError_t e = cudaMalloc((void**)&m->group_ptr[g], m->group_bytes[g]);
+    cudaError_t e = injected_alloc_failure() ? cudaErrorMemoryAllocation
+                                             : cudaMalloc((void**)&m->group_ptr[g], m->group_bytes[g]);
     if (e != cudaSuccess) {
       cudaGetLastError();
       for (int k = 0; k < g; ++k) cudaFree(m->group_ptr[k]);
@@ -2223,7 +2261,8 @@ int photon_vanilla_init(const photon_vanilla_config* cfg, uint64_t seed, photon_
   build_specs_vanilla(m);
   for (int g = 0; g < G_COUNT; ++g) {
     if (m->group_bytes[g] == 0) continue;
-    cudaError_t e = cudaMalloc((void**)&m->group_ptr[g], m->group_bytes[g]);
+    cudaError_t e = injected_alloc_failure() ? cudaErrorMemoryAllocation
+                                             : cudaMalloc((void**)&m->group_ptr[g], m->group_bytes[g]);
     if (e != cudaSuccess) {
       cudaGetLastError();
       for (int k = 0; k < g; ++k)

@@ -491,6 +491,24 @@ PHOTON_API uint64_t photon_launch_count(void);
 /* Message describing the last error on this thread ("" if none). */
 PHOTON_API const char* photon_last_error(void);
 
+/* Test hook for the failure paths (no counterpart in the paper): the n-th
+ * device allocation the library makes from now on (n = 1: the next one;
+ * model weights, caches, workspaces) fails as if the device were out of
+ * memory, so the call that makes it returns PHOTON_ERR_OOM and releases
+ * what it had allocated.  n = 0 turns the hook off.  Process-wide.
+ * Errors: ERR_ARG (n < 0). */
+PHOTON_API int photon_debug_fail_alloc(int64_t n);
+
+/* Self-test of the kernels' bounded waits (no counterpart in the paper):
+ * launches one thread that waits on a barrier nothing ever arrives on,
+ * through the same bounded wait the kernels use, with a budget of
+ * limit_cycles clock cycles.  When the budget runs out the kernel writes a
+ * nonzero code to d_err (device int32 the caller owns) and returns; the call
+ * synchronises the stream and reports it.  The context stays usable.
+ * Errors: ERR_DEVICE_CHECK (the wait ran out: the expected outcome),
+ * ERR_ARG, ERR_CUDA. */
+PHOTON_API int photon_selftest_wait_timeout(int64_t limit_cycles, int32_t* d_err, void* stream);
+
 #ifdef __cplusplus
 }
 #endif
