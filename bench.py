@@ -384,7 +384,7 @@ def run_gpu(args) -> None:
         "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": round(total_ms / args.steps, 3), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": shape["dtype"],
-        "data": "synthetic: seeded N(0,0.02)-like weights (SplitMix64 + Irwin-Hall), Zipf(1.1) prompt ids",
+        "data": "synthetic: seeded N(0,0.02) weights (SplitMix64 + polar method), Zipf(1.1) prompt ids",
         "config": {"workload": workload_label(args.workload),
                    "batch_per_gpu": B, "prompt_len": T, "decode_tokens": chunks * C,
                    "parallelism": f"dp{world}", "l2": "working set > L2 (no flush)",

@@ -90,17 +90,23 @@ __global__ void __launch_bounds__(32 * W, (QMAX == 1 ? 24 : 8) / W)
   __shared__ float sm_acc[W][QMAX][DH];
   extern __shared__ uint4 ring[];  // [warp][stage][K,V][U][SPL][lane]
 
-  pdl_wait();  // before any global access, including the device-side position
-  pdl_trigger();
   const int s = blockIdx.x, h = blockIdx.y, g = blockIdx.z;
   const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
   const int kgrp = lane / TPK, sl = lane % TPK;
-  const int p0 = a.p0_dev ? (*a.p0_dev + a.p0) : a.p0;
-  const int n = min(p0 + a.q_len, splits * chunk);
-  const int k0 = s * chunk, k1 = min(n, k0 + chunk);
-  const int nk = max(0, k1 - k0);
-  const int wc = (nk + W - 1) / W;
-  const int kw0 = k0 + warp * wc, kw1 = min(k1, kw0 + wc);
+  // Keys cached by earlier steps never change, and the device-side position
+  // is written at the end of a step, long before this kernel's predecessor
+  // (the projection that writes this step's queries and new keys) runs.  So
+  // the first ring stages, when they hold only such keys, are copied before
+  // waiting for the predecessor.  The position is read again after the wait;
+  // if it moved (its writer was the predecessor after all), the early copies
+  // are drained and the plan starts over.
+  int p0 = a.p0_dev ? (__ldcg(a.p0_dev) + a.p0) : a.p0;
+  int n = min(p0 + a.q_len, splits * chunk);
+  const int k0 = s * chunk;
+  int k1 = min(n, k0 + chunk);
+  int nk = max(0, k1 - k0);
+  int wc = (nk + W - 1) / W;
+  int kw0 = k0 + warp * wc, kw1 = min(k1, kw0 + wc);
   // per-lane row bases: row `key` of this (group, head) starts at base + key*DH.
   // Lane sl of a key group holds the 16-byte slices sl, sl + TPK, ... of the
   // row, so each warp-wide copy reads whole 32-byte sectors.
@@ -129,6 +135,34 @@ __global__ void __launch_bounds__(32 * W, (QMAX == 1 ? 24 : 8) / W)
     }
   };
 
+  // stages of keys below p0 only (the new keys sit at p0 and after)
+  int pre = 0;
+  {
+    const int nb0 = (kw1 - kw0 + STEP - 1) / STEP;
+    for (int st = 0; st < kDecStages - 1 && st < nb0; ++st) {
+      if (min(kw1, kw0 + (st + 1) * STEP) > p0) break;
+      issue(st, kw0 + st * STEP);
+      cp_async_commit_group();
+      ++pre;
+    }
+  }
+  pdl_wait();  // the predecessor's queries and new keys are visible from here on
+  pdl_trigger();
+  if (a.p0_dev) {
+    const int p0_now = *a.p0_dev + a.p0;
+    if (p0_now != p0) {
+      cp_async_wait_group<0>();
+      p0 = p0_now;
+      n = min(p0 + a.q_len, splits * chunk);
+      k1 = min(n, k0 + chunk);
+      nk = max(0, k1 - k0);
+      wc = (nk + W - 1) / W;
+      kw0 = k0 + warp * wc;
+      kw1 = min(k1, kw0 + wc);
+      pre = 0;
+    }
+  }
+
   float qv[QMAX][LV], m[QMAX], l[QMAX], acc[QMAX][LV];
 #pragma unroll
   for (int qi = 0; qi < QMAX; ++qi) {
@@ -152,8 +186,7 @@ __global__ void __launch_bounds__(32 * W, (QMAX == 1 ? 24 : 8) / W)
   }
 
   const int nb = (kw1 - kw0 + STEP - 1) / STEP;  // stages this warp consumes
-#pragma unroll
-  for (int st = 0; st < kDecStages - 1; ++st) {
+  for (int st = pre; st < kDecStages - 1; ++st) {
     if (st < nb) issue(st, kw0 + st * STEP);
     cp_async_commit_group();
   }

@@ -26,11 +26,19 @@ bool pdl_enabled() {
 }
 
 // ------------------------------------------------------------------ weights
-// Counter-based draw, defined independently of any other implementation:
-// z = SplitMix64 output for counter (e + 1) of the tensor's stream; S = sum
-// of the four 16-bit fields of z; w = fp64(S - 131070) * K (an Irwin-Hall(4)
-// sum of uniforms, centred; K = init_std * sqrt(3) / 65536 so std = init_std),
-// rounded to fp32 (nearest even) and then to the storage type.
+// Counter-based N(0, sigma^2) draw, defined independently of any other
+// implementation (every implementation that follows it gets the same bits):
+// the element's key is the SplitMix64 output for counter (e + 1) of the
+// tensor's stream; Marsaglia's polar method takes attempt a's two uniforms on
+// [-1, 1) from the outputs for counters 2a + 1 and 2a + 2 of the key's
+// stream (53 bits each) until 0 < s = x^2 + y^2 < 1 (at most 64 attempts,
+// else 0), and w = x * sqrt(-2 ln(s) / s) * sigma.  ln s is evaluated from
+// its definition: s = m * 2^k with m in [1, 2), halved above sqrt 2, and
+// ln m = 2 atanh((m - 1) / (m + 1)) by its power series (coefficients
+// 1 / (2i + 1), i < 12, Horner).  Every floating-point step is a separately
+// rounded IEEE fp64 operation (the _rn intrinsics keep the compiler from
+// fusing them).  w is rounded to fp32 (nearest even), then to the storage
+// type.
 __device__ __forceinline__ uint64_t splitmix_mix(uint64_t z) {
   z ^= z >> 30;
   z *= 0xBF58476D1CE4E5B9ull;
@@ -49,22 +57,52 @@ static uint64_t splitmix_mix_host(uint64_t z) {
 }
 constexpr uint64_t kGamma = 0x9E3779B97F4A7C15ull;
 
+// ln s for a positive normal fp64 s (the series definition above).
+__device__ __forceinline__ double draw_log(double s) {
+  const long long bits = __double_as_longlong(s);
+  int k = (int)((bits >> 52) & 0x7FF) - 1023;
+  double m = __longlong_as_double((bits & 0x000FFFFFFFFFFFFFll) | 0x3FF0000000000000ll);
+  if (m >= 0x1.6a09e667f3bcdp+0) {
+    m = __dmul_rn(m, 0.5);
+    k += 1;
+  }
+  const double f = __ddiv_rn(__dsub_rn(m, 1.0), __dadd_rn(m, 1.0));
+  const double f2 = __dmul_rn(f, f);
+  double p = __ddiv_rn(1.0, 23.0);
+#pragma unroll
+  for (int i = 10; i >= 0; --i) p = __dadd_rn(__dmul_rn(p, f2), __ddiv_rn(1.0, (double)(2 * i + 1)));
+  const double lnm = __dmul_rn(__dmul_rn(2.0, f), p);
+  return __dadd_rn(__dmul_rn((double)k, 0x1.62e42fefa39efp-1), lnm);
+}
+
+__device__ __forceinline__ double draw_pm1(uint64_t z) {
+  return __dsub_rn(__dmul_rn((double)(z >> 11), 0x1p-52), 1.0);
+}
+
 template <typename T>
-__global__ void k_init_normal(T* __restrict__ dst, long long n, uint64_t base, double K) {
+__global__ void k_init_normal(T* __restrict__ dst, long long n, uint64_t base, double sigma) {
   pdl_wait();
   pdl_trigger();
   for (long long e = blockIdx.x * (long long)blockDim.x + threadIdx.x; e < n;
        e += (long long)gridDim.x * blockDim.x) {
-    const uint64_t z = splitmix_mix(base + kGamma * (uint64_t)(e + 1));
-    const int S = (int)(z & 0xFFFFu) + (int)((z >> 16) & 0xFFFFu) + (int)((z >> 32) & 0xFFFFu) +
-                  (int)(z >> 48);
-    const double w = (double)(S - 131070) * K;
-    st_f(dst + e, __double2float_rn(w));
+    const uint64_t key = splitmix_mix(base + kGamma * (uint64_t)(e + 1));
+    double w = 0.0;
+    for (int att = 0; att < 64; ++att) {
+      const double x = draw_pm1(splitmix_mix(key + kGamma * (uint64_t)(2 * att + 1)));
+      const double y = draw_pm1(splitmix_mix(key + kGamma * (uint64_t)(2 * att + 2)));
+      const double s = __dadd_rn(__dmul_rn(x, x), __dmul_rn(y, y));
+      if (s > 0.0 && s < 1.0) {
+        const double r = __dsqrt_rn(__ddiv_rn(__dmul_rn(-2.0, draw_log(s)), s));
+        w = __dmul_rn(x, r);
+        break;
+      }
+    }
+    st_f(dst + e, __double2float_rn(__dmul_rn(w, sigma)));
   }
 }
 
 void launch_init_normal(int dt, void* dst, long long numel, uint64_t seed, int tensor_index,
-                        double K, cudaStream_t s) {
+                        double sigma, cudaStream_t s) {
   const uint64_t base = splitmix_mix_host(seed + kGamma * (uint64_t)(tensor_index + 1));
   const int threads = 256;
   long long blocks = (numel + threads - 1) / threads;
@@ -72,11 +110,11 @@ void launch_init_normal(int dt, void* dst, long long numel, uint64_t seed, int t
   if (blocks < 1) blocks = 1;
   if (dt == DT_F32)
     {
-      launch_kernel(k_init_normal<float>, (int)blocks, threads, 0, s, (float*)dst, numel, base, K);
+      launch_kernel(k_init_normal<float>, (int)blocks, threads, 0, s, (float*)dst, numel, base, sigma);
     }
   else
     {
-      launch_kernel(k_init_normal<bf16>, (int)blocks, threads, 0, s, (bf16*)dst, numel, base, K);
+      launch_kernel(k_init_normal<bf16>, (int)blocks, threads, 0, s, (bf16*)dst, numel, base, sigma);
     }
 }
 

@@ -131,8 +131,9 @@ struct AttnArgs {
 };
 
 // ---- weights -----------------------------------------------------------
+// N(0, sigma^2) draw of tensor `tensor_index` (definition in k_misc.cu).
 void launch_init_normal(int dt, void* dst, long long numel, uint64_t seed, int tensor_index,
-                        double K, cudaStream_t s);
+                        double sigma, cudaStream_t s);
 void launch_fill_f32(float* dst, long long n, float v, cudaStream_t s);
 void launch_to_f32(int dt, const void* src, float* dst, long long n, cudaStream_t s);
 

@@ -254,7 +254,7 @@ static cudaError_t pool_malloc(void** p, size_t bytes, cudaStream_t s) {
 
 // Draws (or fills) every tensor of one group into its buffer.
 static void generate_group(photon_model* m, int g, cudaStream_t s) {
-  const double K = ((double)m->cfg.init_std * 1.7320508075688772) / 65536.0;
+  const double K = (double)m->cfg.init_std;  // sigma of the normal draw (fp32 value)
   for (size_t i = 0; i < m->t.size(); ++i) {
     const TensorRec& r = m->t[i];
     if (r.group != g) continue;

@@ -185,9 +185,10 @@ PHOTON_API int photon_free_cache(photon_cache* c);
  * with standard Gumbel noise G_v = -ln(-ln u_v) from a counter-based
  * generator (a pure function of seed, the sequence's batch row b, the
  * token's index t among the tokens this cache has generated, and v):
- *   K   = mix64(mix64(seed + g*(b+1)) + g*(t+1)), k32 = (K >> 32) ^ (K & 0xFFFFFFFF)
+ *   K   = mix64(mix64(seed + g*(b+1)) + g*(t+1))
  *         (mix64: the SplitMix64 output function, g = 0x9E3779B97F4A7C15),
- *   h   = fmix32(k32 + 0x9E3779B9*(v+1) mod 2^32)  (MurmurHash3's finaliser),
+ *   h   = MurmurHash3_x86_32 with seed 0 of the 12-byte message K (8 bytes,
+ *         little-endian) followed by v (4 bytes, little-endian),
  *   u_v = (floor(h / 256) + 1/2) / 2^24.
  * The explainer's quality section (several varied queries per prompt)
  * motivates sampling; the pages do not fix the sampler.  Tokens written by

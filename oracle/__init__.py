@@ -9,8 +9,8 @@ is synth_inputs, which generates seeded prompt ids and holds none of the
 model's arithmetic.
 
 Contents:
-  weights.py -- the counter-based N(0, 0.02^2)-like weight generator, written
-                from its definition (SplitMix64 + Irwin-Hall), fp64.
+  weights.py -- the counter-based N(0, 0.02^2) weight generator, written
+                from its definition (SplitMix64 + polar method), fp64.
   photon.py  -- the model in plain fp64 NumPy, one sequence at a time,
                 following the PHOTON pages step by step.
   sampling.py -- temperature sampling by the Gumbel-max rule with a

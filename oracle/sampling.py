@@ -15,12 +15,13 @@ only on (seed, sequence, token position, vocabulary id):
 
   row key   K   = mix64(mix64(seed + gamma * (b + 1)) + gamma * (t + 1))
                   (mix64 = the SplitMix64 output function, gamma its
-                  Weyl increment 0x9E3779B97F4A7C15), folded to 32 bits as
-                  k32 = high 32 bits XOR low 32 bits;
-  element   h   = fmix32(k32 + 0x9E3779B9 * (v + 1))   (mod 2^32), fmix32 =
-                  the 32-bit finaliser of MurmurHash3 (xor-shift 16,
-                  multiply 0x85EBCA6B, xor-shift 13, multiply 0xC2B2AE35,
-                  xor-shift 16);
+                  Weyl increment 0x9E3779B97F4A7C15), a 64-bit word;
+  element   h   = MurmurHash3_x86_32 (seed 0) of the 12-byte message made of
+                  K's 8 bytes and v's 4 bytes, both little-endian (Austin
+                  Appleby's public hash: three 4-byte blocks, each mixed
+                  with the constants 0xCC9E2D51 and 0x1B873593 and folded in
+                  with rotate 13, times 5 plus 0xE6546B64; then the length 12
+                  is xored in and the 32-bit finaliser applied);
   uniform   u   = (floor(h / 256) + 1/2) / 2^24, in (0, 1);
   Gumbel    G   = -ln(-ln u), with -ln u evaluated as -log1p(-(1 - u)) so
                   that u near 1 keeps its precision.
@@ -28,12 +29,11 @@ only on (seed, sequence, token position, vocabulary id):
 b is the sequence's row in the batch, t the token's index among the tokens
 the cache has generated (chunk * C1*C2 + sub-chunk * C1 + position), v the
 vocabulary id.  Ties of the perturbed values go to the lowest id, as for
-greedy decoding.
+greedy decoding.  The first two blocks depend on the row only, so `row_key`
+returns the hash state after them and `uniforms` finishes the message per v.
 
-The hash finaliser is pinned to MurmurHash3 and the 64-bit mixes to SplitMix64
-(tests).  The fold of the 64-bit key to 32 bits is this project's own choice.
-Nothing outside the code fixes it (parity unpinned for that step); the GPU's
-draws are compared with it.
+The 64-bit mixes are pinned to SplitMix64's published vectors and the
+element hash to scikit-learn's independent MurmurHash3 (tests).
 
 Nucleus (top-p) sampling, a common refinement the pages do not mention
 either, restricts the draw to the smallest set of most probable tokens whose
@@ -48,7 +48,9 @@ from .weights import GAMMA, mix64
 
 _F1 = np.uint32(0x85EBCA6B)
 _F2 = np.uint32(0xC2B2AE35)
-_WEYL32 = np.uint32(0x9E3779B9)
+_MM_C1 = np.uint32(0xCC9E2D51)
+_MM_C2 = np.uint32(0x1B873593)
+_MM_ADD = np.uint32(0xE6546B64)
 
 
 def fmix32(h: np.ndarray) -> np.ndarray:
@@ -63,20 +65,43 @@ def fmix32(h: np.ndarray) -> np.ndarray:
     return h
 
 
+def _rotl32(x: np.ndarray, r: int) -> np.ndarray:
+    return (x << np.uint32(r)) | (x >> np.uint32(32 - r))
+
+
+def mm3_block(h, k) -> np.ndarray:
+    """One 4-byte block of MurmurHash3_x86_32 folded into the state h (uint32)."""
+    h = np.asarray(h, dtype=np.uint32)
+    k = np.asarray(k, dtype=np.uint32)
+    with np.errstate(over="ignore"):
+        k = k * _MM_C1
+        k = _rotl32(k, 15)
+        k = k * _MM_C2
+        h = h ^ k
+        h = _rotl32(h, 13)
+        h = h * np.uint32(5) + _MM_ADD
+    return h
+
+
 def row_key(seed: int, b: int, t: int) -> np.uint32:
-    """32-bit key of one (sequence, token position) draw."""
+    """Hash state after the row key K's two blocks (low word, then high word)."""
     with np.errstate(over="ignore"):
         k = mix64(np.uint64(seed) + GAMMA * np.uint64(b + 1))
         k = mix64(k + GAMMA * np.uint64(t + 1))
     k = int(k)
-    return np.uint32((k >> 32) ^ (k & 0xFFFFFFFF))
+    h = mm3_block(np.uint32(0), np.uint32(k & 0xFFFFFFFF))
+    return np.uint32(mm3_block(h, np.uint32(k >> 32)))
+
+
+def element_hash(key: np.uint32, V: int) -> np.ndarray:
+    """h_v for v = 0..V-1: the message's third block v, the length, the finaliser."""
+    v = np.arange(V, dtype=np.uint32)
+    return fmix32(mm3_block(np.uint32(key), v) ^ np.uint32(12))
 
 
 def uniforms(key: np.uint32, V: int) -> np.ndarray:
     """u_v for v = 0..V-1, exact binary fractions in (0, 1) (fp64)."""
-    v = np.arange(1, V + 1, dtype=np.uint32)
-    with np.errstate(over="ignore"):
-        h = fmix32(np.uint32(key) + _WEYL32 * v)
+    h = element_hash(key, V)
     return ((h >> np.uint32(8)).astype(np.float64) + 0.5) / float(1 << 24)
 
 

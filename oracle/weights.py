@@ -8,7 +8,9 @@ definition of that draw; the CUDA library implements the same definition on
 its own side, and the two are compared byte for byte through the library's
 tensor export.
 
-Definition (all integer arithmetic modulo 2^64):
+Definition (integer arithmetic modulo 2^64; floating point is IEEE fp64
+with round-to-nearest-even, every operation rounded on its own, no fused
+multiply-add):
 
   gamma = 0x9E3779B97F4A7C15
   mix(z):  z ^= z >> 30; z *= 0xBF58476D1CE4E5B9;
@@ -17,20 +19,29 @@ Definition (all integer arithmetic modulo 2^64):
 
   tensor t (0-based, in the order of `tensor_specs`) has key
       base_t = mix(seed + gamma * (t + 1))
-  element e (row-major index in the tensor's stated shape) draws
-      z = mix(base_t + gamma * (e + 1))
-      S = sum of the four 16-bit fields of z            (0 <= S <= 262140)
-      w = fp64(S - 131070) * K,   K = (init_std * 1.7320508075688772) / 65536
-  with init_std taken as its fp32 value (the type of the config field in
-  the library's C ABI) and K evaluated in fp64, left to right.
-
-  S/65536 - 2 is the Irwin-Hall sum of four uniforms on (0, 1) minus its
-  mean (variance 1/3), so w has mean 0 and standard deviation init_std,
-  a bounded bell-shaped stand-in for N(0, init_std^2).  Only exact integer
-  operations and one fp64 multiply are involved, so every implementation
-  produces the same bits.  w is then rounded to fp32 (round to nearest
-  even) and, for bf16 models, from fp32 to bf16 (round to nearest even).
-  RMSNorm gains are exactly 1.0 and consume a tensor index but no draws.
+  element e (row-major index in the tensor's stated shape) has key
+      key_e = mix(base_t + gamma * (e + 1))
+  and draws by Marsaglia's polar method: for attempt a = 0, 1, ..., 63
+      x = (mix(key_e + gamma * (2a + 1)) >> 11) * 2^-52 - 1      (exact, in [-1, 1))
+      y = (mix(key_e + gamma * (2a + 2)) >> 11) * 2^-52 - 1
+      s = x*x + y*y
+  until 0 < s < 1 (after 64 rejected attempts, which has probability
+  (1 - pi/4)^64 < 1e-42, w = 0); then
+      w = (x * sqrt((-2 * ln s) / s)) * sigma,   sigma = fp64 of the fp32 init_std
+  (the first variable of the polar pair, a standard normal times sigma).
+  ln s is evaluated as its own definition, not by a library routine:
+      s = m * 2^k with m in [1, 2) (the exponent and mantissa fields);
+      if m >= 0x1.6a09e667f3bcdp+0 (sqrt 2 rounded): m = m/2, k = k+1;
+      f = (m - 1) / (m + 1);  ln m = 2 * atanh(f) = 2f (1 + f^2/3 + f^4/5 + ...),
+      the series summed by Horner's rule over the coefficients 1/(2i+1),
+      i = 11 down to 0 (each the rounded quotient), as p = p * f^2 + c_i;
+      ln m = (2f) * p;   ln s = k * LN2 + ln m,   LN2 = 0x1.62e42fefa39efp-1.
+  With |f| <= 0.1716 the dropped terms are below 1e-20 of ln m.
+  Only exact integer steps and correctly rounded +, -, *, / and sqrt are
+  involved, so every implementation that follows the definition produces
+  the same bits.  w is then rounded to fp32 (round to nearest even) and, for
+  bf16 models, from fp32 to bf16 (round to nearest even).  RMSNorm gains are
+  exactly 1.0 and consume a tensor index but no draws.
 """
 from __future__ import annotations
 
@@ -42,7 +53,10 @@ import numpy as np
 GAMMA = np.uint64(0x9E3779B97F4A7C15)
 _M1 = np.uint64(0xBF58476D1CE4E5B9)
 _M2 = np.uint64(0x94D049BB133111EB)
-SQRT3 = 1.7320508075688772
+LN2 = float.fromhex("0x1.62e42fefa39efp-1")
+SQRT2 = float.fromhex("0x1.6a09e667f3bcdp+0")
+ATANH_COEF = [1.0 / (2 * i + 1) for i in range(12)]
+MAX_ATTEMPTS = 64
 
 
 def mix64(z: np.ndarray) -> np.ndarray:
@@ -116,25 +130,68 @@ def round_fp32_to_bf16(x32: np.ndarray) -> np.ndarray:
     return r.astype(np.uint32).view(np.float32)
 
 
+def log_series(s: np.ndarray) -> np.ndarray:
+    """ln s for positive normal fp64 s, by the exponent split and the atanh
+    series of the definition above (elementwise, fp64)."""
+    s = np.asarray(s, dtype=np.float64)
+    bits = s.view(np.int64)
+    k = ((bits >> 52) & 0x7FF) - 1023
+    m = ((bits & 0x000FFFFFFFFFFFFF) | 0x3FF0000000000000).view(np.float64)
+    big = m >= SQRT2
+    m = np.where(big, m * 0.5, m)
+    k = np.where(big, k + 1, k)
+    f = (m - 1.0) / (m + 1.0)
+    f2 = f * f
+    p = np.full_like(f, ATANH_COEF[-1])
+    for c in reversed(ATANH_COEF[:-1]):
+        p = p * f2
+        p = p + c
+    lnm = (2.0 * f) * p
+    return k.astype(np.float64) * LN2 + lnm
+
+
+def _uniform_pm1(z: np.ndarray) -> np.ndarray:
+    """(z >> 11) * 2^-52 - 1, exact."""
+    return (z >> np.uint64(11)).astype(np.float64) * (2.0 ** -52) - 1.0
+
+
+def polar_normal(keys: np.ndarray) -> np.ndarray:
+    """Standard normal variables of the definition for element keys (uint64)."""
+    n = keys.size
+    out = np.zeros(n, dtype=np.float64)
+    todo = np.arange(n)
+    for att in range(MAX_ATTEMPTS):
+        if todo.size == 0:
+            break
+        kk = keys[todo]
+        with np.errstate(over="ignore"):
+            x = _uniform_pm1(mix64(kk + GAMMA * np.uint64(2 * att + 1)))
+            y = _uniform_pm1(mix64(kk + GAMMA * np.uint64(2 * att + 2)))
+        s = x * x
+        s = s + y * y
+        ok = (s > 0.0) & (s < 1.0)
+        sa, xa = s[ok], x[ok]
+        r = np.sqrt((-2.0 * log_series(sa)) / sa)
+        out[todo[ok]] = xa * r
+        todo = todo[~ok]
+    return out
+
+
 def draw_tensor(seed: int, t: int, numel: int, init_std: float, dtype: str,
                 chunk: int = 1 << 18) -> np.ndarray:
     """Values of tensor t as float32 (already rounded to the storage precision)."""
-    K = (float(np.float32(init_std)) * SQRT3) / 65536.0
+    sigma = float(np.float32(init_std))
     with np.errstate(over="ignore"):
         base = mix64(np.uint64(seed) + GAMMA * np.uint64(t + 1))
     out = np.empty(numel, dtype=np.float32)
-    mask = np.uint64(0xFFFF)
 
     def fill(lo: int) -> None:
         # elements lo..hi-1; independent of every other range
         hi = min(numel, lo + chunk)
         e1 = np.arange(lo + 1, hi + 1, dtype=np.uint64)
         with np.errstate(over="ignore"):
-            z = mix64(base + GAMMA * e1)
-        s = ((z & mask) + ((z >> np.uint64(16)) & mask)
-             + ((z >> np.uint64(32)) & mask) + (z >> np.uint64(48)))
-        w64 = (s.astype(np.int64) - 131070).astype(np.float64) * K
-        out[lo:hi] = w64.astype(np.float32)
+            keys = mix64(base + GAMMA * e1)
+        out[lo:hi] = (polar_normal(keys) * sigma).astype(np.float32)
 
     starts = range(0, numel, chunk)
     if len(starts) > 1:

@@ -36,18 +36,54 @@ def test_splitmix64_published_vectors():
                    4593380528125082431, 16408922859458223821]
 
 
-def test_generator_moments_and_support():
-    # Irwin-Hall(4) centred and scaled by sqrt(3): mean 0, std = init_std,
-    # |w| <= 2*sqrt(3)*init_std.
-    w = oracle.draw_tensor(seed=7, t=3, numel=1 << 20, init_std=0.02, dtype="fp32")
+def test_generator_log_is_the_natural_log():
+    # the generator evaluates ln from its atanh series (so both sides can
+    # reproduce it bit for bit); against the C library's log it must agree
+    # to a few units in the last place over (0, 1) and at exact points
+    from oracle import weights as W
+    rng = np.random.default_rng(5)
+    s = np.concatenate([rng.random(100000), 2.0 ** -rng.integers(1, 100, 2000) * rng.random(2000),
+                        np.array([0.5, 0.25, 1 - 2 ** -52, 2 ** -104, W.SQRT2 / 2, W.SQRT2 / 2 * (1 + 2 ** -52)])])
+    s = s[s > 0]
+    got = W.log_series(s)
+    ref = np.array([math.log(v) for v in s])
+    assert np.max(np.abs(got - ref) / np.abs(ref)) < 4 * 2 ** -52
+    assert W.log_series(np.array([0.5]))[0] == -W.LN2
+
+
+def test_generator_draws_are_normal():
+    # Marsaglia's polar method: standard normal variables times init_std.
+    # Kolmogorov-Smirnov against the normal CDF (99.9 % critical value),
+    # the moments up to the fourth, and the tails (a bounded stand-in such
+    # as a sum of uniforms fails the 4-sigma check)
+    from scipy import stats
+    w = oracle.draw_tensor(seed=7, t=3, numel=1 << 20, init_std=0.02, dtype="fp32").astype(np.float64)
     n = w.size
-    assert abs(w.mean()) < 4 * 0.02 / math.sqrt(n)
-    assert abs(w.std() / 0.02 - 1) < 5e-3
-    assert np.abs(w).max() <= 2 * math.sqrt(3) * 0.02 + 1e-9
+    assert stats.kstest(w / 0.02, stats.norm.cdf).statistic < 1.95 / math.sqrt(n)
+    z = w / 0.02
+    assert abs(z.mean()) < 4 / math.sqrt(n)
+    assert abs(z.std() - 1) < 4 * math.sqrt(0.5 / n)
+    assert abs(stats.kurtosis(z, fisher=False) - 3) < 4 * math.sqrt(24 / n)
+    p3 = 2 * stats.norm.sf(3)
+    assert abs((np.abs(z) > 3).mean() - p3) < 5 * math.sqrt(p3 / n)
+    assert np.abs(z).max() > 4
     # distinct tensors and seeds give distinct streams
     w2 = oracle.draw_tensor(seed=7, t=4, numel=1024, init_std=0.02, dtype="fp32")
     w3 = oracle.draw_tensor(seed=8, t=3, numel=1024, init_std=0.02, dtype="fp32")
     assert not np.array_equal(w[:1024], w2) and not np.array_equal(w[:1024], w3)
+
+
+def test_generator_polar_attempts_accept_at_pi_over_4():
+    # an attempt's pair is uniform on the square [-1, 1)^2, accepted inside
+    # the unit disc: probability pi / 4
+    from oracle import weights as W
+    keys = oracle.mix64(np.arange(1, 400001, dtype=np.uint64) * W.GAMMA)
+    with np.errstate(over="ignore"):
+        x = W._uniform_pm1(oracle.mix64(keys + W.GAMMA))
+        y = W._uniform_pm1(oracle.mix64(keys + W.GAMMA * np.uint64(2)))
+    acc = ((x * x + y * y) < 1).mean()
+    assert abs(acc - math.pi / 4) < 5 * math.sqrt(0.25 * 0.75 / keys.size)
+    assert x.min() >= -1 and x.max() < 1
 
 
 def test_bf16_rounding_ties_to_even():

@@ -6,8 +6,9 @@ tests check that claim and the pieces it rests on against facts that do not
 come from the sampler itself: the standard Gumbel law's mean (the
 Euler-Mascheroni constant) and variance (pi^2 / 6), a multinomial
 goodness-of-fit against softmax probabilities computed independently, the
-greedy limit T -> 0, and exact properties of the hash (a bijection of 32-bit
-words, fixed point 0, uniforms on the 2^-24 grid's odd midpoints).
+greedy limit T -> 0, exact properties of the hash (a bijection of 32-bit
+words, fixed point 0, uniforms on the 2^-24 grid's odd midpoints), and the
+whole element hash against scikit-learn's MurmurHash3 of the same message.
 """
 import math
 
@@ -140,3 +141,21 @@ def test_fmix32_is_murmurhash3s_finaliser():
         for seed in (0, 1, 0x9747B28C):
             want = murmurhash3_32(key - (1 << 32) if key >= 1 << 31 else key, seed=seed, positive=True)
             assert int(S.fmix32(np.uint32(block(key, seed)))) == want, (key, seed)
+
+
+def test_element_hash_is_murmurhash3_of_the_whole_message():
+    # the uniform of vocabulary id v is MurmurHash3_x86_32 (seed 0) of the
+    # 12-byte message (row key K, 8 bytes little-endian; v, 4 bytes
+    # little-endian); scikit-learn's implementation computes it independently
+    # of the oracle's block-by-block evaluation
+    from sklearn.utils import murmurhash3_32
+    from oracle.weights import GAMMA, mix64
+    rng = np.random.default_rng(17)
+    for seed, b, t in [(0, 0, 0), (1, 3, 7), (0x9747B28C, 63, 511)] + \
+            [(int(rng.integers(0, 1 << 62)), int(rng.integers(0, 256)), int(rng.integers(0, 4096))) for _ in range(12)]:
+        with np.errstate(over="ignore"):
+            K = int(mix64(mix64(np.uint64(seed) + GAMMA * np.uint64(b + 1)) + GAMMA * np.uint64(t + 1)))
+        h = S.element_hash(S.row_key(seed, b, t), 32000)
+        for v in [0, 1, 2, 255, 256, 31999] + [int(x) for x in rng.integers(0, 32000, size=10)]:
+            msg = K.to_bytes(8, "little") + v.to_bytes(4, "little")
+            assert int(h[v]) == murmurhash3_32(msg, seed=0, positive=True), (seed, b, t, v)
