@@ -40,7 +40,7 @@ EXPORTED = ("photon_init_weights", "photon_free_model", "photon_prefill",
             "photon_multi_query", "photon_vanilla_init",
             "photon_vanilla_prefill", "photon_vanilla_decode_step", "photon_vanilla_cache_info",
             "photon_vanilla_free_cache", "photon_launch_count", "photon_last_error",
-            "photon_debug_fail_alloc", "photon_selftest_wait_timeout")
+            "photon_debug_fail_alloc", "photon_selftest_wait_timeout", "photon_init_weights_levels")
 
 
 class PhotonError(RuntimeError):
@@ -65,6 +65,18 @@ class photon_cache_stats(ctypes.Structure):
                  "max_new_chunks", "device_error", "l1_resident")] + \
                [("kv_bytes", ctypes.c_uint64), ("workspace_bytes", ctypes.c_uint64),
                 ("graph_steps", ctypes.c_int32), ("graph_kernels", ctypes.c_int32)]
+
+
+MAX_LEVELS = 4
+
+
+class photon_level_config(ctypes.Structure):
+    _fields_ = [("vocab", ctypes.c_int32), ("d_model", ctypes.c_int32), ("n_heads", ctypes.c_int32),
+                ("head_dim", ctypes.c_int32), ("levels", ctypes.c_int32),
+                ("chunk", ctypes.c_int32 * MAX_LEVELS), ("enc_layers", ctypes.c_int32 * MAX_LEVELS),
+                ("dec_layers", ctypes.c_int32 * MAX_LEVELS), ("mlp_mult", ctypes.c_int32),
+                ("dtype", ctypes.c_int32), ("init_std", ctypes.c_float), ("rope_theta", ctypes.c_float),
+                ("norm_eps", ctypes.c_float)]
 
 
 class photon_model_stats(ctypes.Structure):
@@ -130,6 +142,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "photon_attn_decode_noalloc": [I32, P, P, P, I32, I32, I32, I32, I32, I32, P, P, P],
         "photon_attn_decode_scratch_bytes": [I32, I32, I32, I32, I32, I32, I32, P],
         "photon_debug_fail_alloc": [I64],
+        "photon_init_weights_levels": [ctypes.POINTER(photon_level_config), U64, ctypes.POINTER(P)],
         "photon_selftest_wait_timeout": [I64, P, P],
     }
     for name, args in sig.items():
@@ -179,6 +192,26 @@ def _need(t, dtype, numel: int, name: str) -> None:
         raise ValueError(f"{name}: must be a CUDA tensor")
 
 
+def level_config_struct(shape: dict) -> photon_level_config:
+    """photon_level_config from a shape dict with per-level lists: chunks,
+    enc_layers, dec_layers (level 1 first; the last encoder is the top)."""
+    c = photon_level_config()
+    c.vocab, c.d_model = shape["vocab"], shape["d_model"]
+    c.n_heads, c.head_dim = shape["n_heads"], shape["head_dim"]
+    L = len(shape["chunks"])
+    if not (1 <= L <= MAX_LEVELS and len(shape["enc_layers"]) == L == len(shape["dec_layers"])):
+        raise ValueError("chunks, enc_layers and dec_layers need one entry per level (1..4 levels)")
+    c.levels = L
+    for i in range(L):
+        c.chunk[i], c.enc_layers[i], c.dec_layers[i] = shape["chunks"][i], shape["enc_layers"][i], shape["dec_layers"][i]
+    c.mlp_mult = shape.get("mlp_mult", 4)
+    c.dtype = _DTYPES[shape["dtype"]]
+    c.init_std = shape.get("init_std", 0.02)
+    c.rope_theta = shape.get("rope_theta", 10000.0)
+    c.norm_eps = shape.get("norm_eps", 1e-6)
+    return c
+
+
 def config_struct(shape: dict) -> photon_config:
     """photon_config from a plain shape dict (keys of synth_inputs.MODEL_KEYS)."""
     c = photon_config()
@@ -201,14 +234,26 @@ class Model:
     """A PHOTON model on the current CUDA device (weights drawn from `seed`)."""
 
     def __init__(self, shape: dict, seed: int):
+        """shape: the two-level keys (C1, C2, L1, Ltop, Ld1, Ld2, ...), or
+        per-level lists (chunks, enc_layers, dec_layers) for any number of levels."""
         L = load_library()
         self.shape = dict(shape)
-        self.cfg = config_struct(shape)
         h = ctypes.c_void_p()
-        _check(L.photon_init_weights(ctypes.byref(self.cfg), seed, ctypes.byref(h)))
+        if "chunks" in shape:
+            self.cfg = level_config_struct(shape)
+            _check(L.photon_init_weights_levels(ctypes.byref(self.cfg), seed, ctypes.byref(h)))
+            self.levels = len(shape["chunks"])
+            self.C1, self.C2 = shape["chunks"][0], shape["chunks"][-1]
+            self.C = 1
+            for c in shape["chunks"]:
+                self.C *= c
+        else:
+            self.cfg = config_struct(shape)
+            _check(L.photon_init_weights(ctypes.byref(self.cfg), seed, ctypes.byref(h)))
+            self.levels = 2
+            self.C1, self.C2 = shape["C1"], shape["C2"]
+            self.C = self.C1 * self.C2
         self._h = h
-        self.C1, self.C2 = shape["C1"], shape["C2"]
-        self.C = self.C1 * self.C2
         self.vocab, self.d_model = shape["vocab"], shape["d_model"]
 
     @property

@@ -677,9 +677,10 @@ __global__ void __launch_bounds__(128) k_attn_prefill(AttnArgs a) {
   const unsigned gmask = 0xFu << ((t & 31) & 28);
   const int qi = blockIdx.x * 32 + (t >> 2);
   const bool active = qi < a.q_len;
-  const int pos = a.p0 + (active ? qi : a.q_len - 1);
+  const int p0 = a.p0_dev ? (*a.p0_dev + a.p0) : a.p0;  // first query's position
+  const int pos = p0 + (active ? qi : a.q_len - 1);
   const int last_q = min(a.q_len, (blockIdx.x + 1) * 32) - 1;
-  const int n_keys = a.p0 + last_q + 1;
+  const int n_keys = p0 + last_q + 1;
   const T* Kown = reinterpret_cast<const T*>(a.K);
   const T* Vown = reinterpret_cast<const T*>(a.V);
   const T* Kpre = reinterpret_cast<const T*>(a.Kp);

@@ -111,6 +111,17 @@ struct photon_model {
   // weights since they were generated; their release waits on all of them
   std::vector<std::pair<cudaStream_t, cudaEvent_t>> enc_users;
 
+  // any-L models (photon_init_weights_levels): per level l (index l - 1)
+  // chunk size, encoder and decoder depth, and first tensor of each piece
+  bool general = false;
+  int NL = 2;
+  int Cl[PHOTON_MAX_LEVELS] = {}, El[PHOTON_MAX_LEVELS] = {}, Dl[PHOTON_MAX_LEVELS] = {};
+  int i_chl[PHOTON_MAX_LEVELS] = {}, i_encl[PHOTON_MAX_LEVELS] = {}, i_encl_g[PHOTON_MAX_LEVELS] = {};
+  int i_cvl[PHOTON_MAX_LEVELS] = {}, i_decl[PHOTON_MAX_LEVELS] = {}, i_decl_g[PHOTON_MAX_LEVELS] = {};
+  cudaGraphExec_t ggraph[2] = {nullptr, nullptr};  // captured any-L decode step per mode
+  const void* ggraph_owner[2] = {nullptr, nullptr};
+  long long ggraph_kernels[2] = {0, 0};
+
   const void* ptr(int idx) const { return group_ptr[t[idx].group] + t[idx].offset; }
   BlockW block(int first, int l) const {
     const int b = first + 8 * l;
@@ -118,6 +129,15 @@ struct photon_model {
                   ptr(b + 6), ptr(b + 7)};
   }
 };
+
+// any-L models (defined with their prefill and decode further down)
+static int gen_check(const photon_level_config* c);
+static void build_specs_levels(photon_model* m);
+struct GenCache;
+static int gen_prefill(photon_model* m, const int32_t* d_tokens, int B, int T, int mode, int max_new,
+                       cudaStream_t s, photon_cache** out);
+static int gen_decode_step(photon_model* m, photon_cache* c, int mode, int32_t* d_out_tokens, float* d_out_logits,
+                           const int32_t* d_force_tokens, const void* d_force_a, cudaStream_t s);
 
 static int check_config(const photon_config* c) {
   if (!c) return fail(PHOTON_ERR_ARG, "config is NULL");
@@ -416,6 +436,8 @@ struct photon_cache {
   std::vector<void*> allocs;
   size_t kv_bytes = 0, ws_bytes = 0;
   bool has_a_hat = false, has_a = false;
+  struct GenCache* gen = nullptr;  // any-L models: their per-level state
+  int32_t* gen_tok_out() const { return tok_out; }
 };
 
 struct Allocator {
@@ -736,6 +758,33 @@ static Bufs decode_bufs(photon_cache* c) {
   return b;
 }
 
+// Allocates the model's weight groups and draws every tensor (synchronising);
+// on failure releases them and the model.
+static int alloc_and_generate(photon_model* m) {
+  cudaStream_t s = nullptr;
+  for (int g = 0; g < G_COUNT; ++g) {
+    if (m->group_bytes[g] == 0) continue;
+    cudaError_t e = injected_alloc_failure() ? cudaErrorMemoryAllocation
+                                             : cudaMalloc((void**)&m->group_ptr[g], m->group_bytes[g]);
+    if (e != cudaSuccess) {
+      cudaGetLastError();
+      for (int k = 0; k < g; ++k) cudaFree(m->group_ptr[k]);
+      delete m;
+      return e == cudaErrorMemoryAllocation ? fail(PHOTON_ERR_OOM, "out of device memory for the weights")
+                                            : fail(PHOTON_ERR_CUDA, "weight allocation: %s", cudaGetErrorString(e));
+    }
+    generate_group(m, g, s);
+  }
+  cudaError_t e = cudaStreamSynchronize(s);
+  if (e == cudaSuccess) e = cudaGetLastError();
+  if (e != cudaSuccess) {
+    for (int g = 0; g < G_COUNT; ++g) cudaFree(m->group_ptr[g]);
+    delete m;
+    return fail(PHOTON_ERR_CUDA, "weight generation failed: %s", cudaGetErrorString(e));
+  }
+  return PHOTON_OK;
+}
+
 // ============================================================== C ABI
 extern "C" {
 
@@ -790,26 +839,65 @@ int photon_init_weights(const photon_config* cfg, uint64_t seed, photon_model** 
   m->Ld2 = cfg->dec_layers[1];
   m->use_tc = (m->dt == DT_BF16) && tma_available();
   build_specs(m);
-  cudaStream_t s = nullptr;
-  for (int g = 0; g < G_COUNT; ++g) {
-    cudaError_t e = injected_alloc_failure() ? cudaErrorMemoryAllocation
-                                             : cudaMalloc((void**)&m->group_ptr[g], m->group_bytes[g]);
-    if (e != cudaSuccess) {
-      cudaGetLastError();
-      for (int k = 0; k < g; ++k) cudaFree(m->group_ptr[k]);
-      delete m;
-      return fail(e == cudaErrorMemoryAllocation ? PHOTON_ERR_OOM : PHOTON_ERR_CUDA,
-                  "weight allocation failed: %s", cudaGetErrorString(e));
-    }
-    generate_group(m, g, s);
+  RET(alloc_and_generate(m));
+  *out = m;
+  return PHOTON_OK;
+}
+
+int photon_init_weights_levels(const photon_level_config* cfg, uint64_t seed, photon_model** out) {
+  g_err.clear();
+  if (!out) return fail(PHOTON_ERR_ARG, "out is NULL");
+  *out = nullptr;
+  RET(gen_check(cfg));
+  int dev = 0;
+  CK(cudaGetDevice(&dev));
+  photon_model* m = new photon_model();
+  // the two-level config fields describe the bottom and the top of the hierarchy
+  memset(&m->cfg, 0, sizeof(m->cfg));
+  m->cfg.vocab = cfg->vocab;
+  m->cfg.d_model = cfg->d_model;
+  m->cfg.n_heads = cfg->n_heads;
+  m->cfg.head_dim = cfg->head_dim;
+  m->cfg.levels = cfg->levels;
+  m->cfg.mlp_mult = cfg->mlp_mult;
+  m->cfg.dtype = cfg->dtype;
+  m->cfg.init_std = cfg->init_std;
+  m->cfg.rope_theta = cfg->rope_theta;
+  m->cfg.norm_eps = cfg->norm_eps;
+  m->general = true;
+  m->NL = cfg->levels;
+  m->dt = cfg->dtype;
+  m->es = dtype_size(m->dt);
+  m->seed = seed;
+  m->d = cfg->d_model;
+  m->H = cfg->n_heads;
+  m->dh = cfg->head_dim;
+  m->V = cfg->vocab;
+  m->f = cfg->mlp_mult * cfg->d_model;
+  m->C = 1;
+  for (int l = 0; l < m->NL; ++l) {
+    m->Cl[l] = cfg->chunk[l];
+    m->El[l] = cfg->enc_layers[l];
+    m->Dl[l] = cfg->dec_layers[l];
+    m->C *= m->Cl[l];
   }
-  cudaError_t e = cudaStreamSynchronize(s);
-  if (e == cudaSuccess) e = cudaGetLastError();
-  if (e != cudaSuccess) {
-    for (int g = 0; g < G_COUNT; ++g) cudaFree(m->group_ptr[g]);
-    delete m;
-    return fail(PHOTON_ERR_CUDA, "weight generation failed: %s", cudaGetErrorString(e));
-  }
+  const int L = m->NL;
+  m->C1 = m->Cl[0];
+  m->C2 = m->Cl[L - 1];
+  m->L1 = m->El[0];
+  m->Ltop = m->El[L - 1];
+  m->Ld1 = m->Dl[0];
+  m->Ld2 = m->Dl[L - 1];
+  m->use_tc = (m->dt == DT_BF16) && tma_available();
+  build_specs_levels(m);
+  // the top-level pieces under their two-level names (export, info)
+  m->i_top = m->i_encl[L - 1];
+  m->i_top_g = m->i_encl_g[L - 1];
+  m->i_ch2 = m->i_chl[L - 1];
+  m->i_cv1 = m->i_cvl[0];
+  m->i_dec1 = m->i_decl[0];
+  m->i_dec1_g = m->i_decl_g[0];
+  RET(alloc_and_generate(m));
   *out = m;
   return PHOTON_OK;
 }
@@ -823,6 +911,7 @@ int photon_free_model(photon_model* m) {
   m->enc_users.clear();
   for (int k = 0; k < 2; ++k) {
     if (m->graph[k]) cudaGraphExecDestroy(m->graph[k]);
+    if (m->ggraph[k]) cudaGraphExecDestroy(m->ggraph[k]);
     for (int p = 0; p < 2; ++p)
       if (m->pg[k][p]) cudaGraphExecDestroy(m->pg[k][p]);
   }
@@ -1533,10 +1622,514 @@ static bool graphs_enabled() {
   return on;
 }
 
+// ============================================================== any number of levels
+// The general hierarchy (photon_init_weights_levels): L levels, each with a
+// chunker and an encoder going up and a converter and a decoder coming
+// down (explainer, architecture section, module table written for a
+// general level l).  Runs on the same kernels as the two-level path;
+// eager launches, with the plain decode step captured into a graph per mode.
+struct GenCache {
+  int L = 0;
+  // encoder caches of levels 1..L ([E_l][B][H][cap][dh] per K and V); the
+  // lower ones only in HierGen mode
+  char* kc[PHOTON_MAX_LEVELS] = {};
+  char* vc[PHOTON_MAX_LEVELS] = {};
+  size_t layer[PHOTON_MAX_LEVELS] = {};
+  int cap[PHOTON_MAX_LEVELS] = {};
+  int n[PHOTON_MAX_LEVELS] = {};   // host copy of the entries per level
+  int* d_n = nullptr;               // device: entries per level, then the chunk counter at [PHOTON_MAX_LEVELS]
+  // top-down: per level l residual stream [G_l * C_l, d], reconstruction
+  // (l >= 2) and chunk-local decoder KV
+  float* xdec[PHOTON_MAX_LEVELS] = {};
+  void* ahat[PHOTON_MAX_LEVELS] = {};
+  char* dk[PHOTON_MAX_LEVELS] = {};
+  char* dv[PHOTON_MAX_LEVELS] = {};
+  size_t dlayer[PHOTON_MAX_LEVELS] = {};
+  int G[PHOTON_MAX_LEVELS] = {};    // groups of level l's decoder
+  // token decoder single-row steps and the head
+  float* xs = nullptr;
+  void* hn = nullptr;
+  float* logits = nullptr;
+  int32_t* next_ids = nullptr;
+  int32_t* used = nullptr;
+  int32_t* tok_out = nullptr;
+  // HierGen re-encode and the top input
+  void* emb = nullptr;
+  float* xre[PHOTON_MAX_LEVELS] = {};
+  void* sre[PHOTON_MAX_LEVELS] = {};
+  float* xt = nullptr;
+  Bufs b;
+  bool graph_failed[2] = {false, false};
+};
+
+static int gen_check(const photon_level_config* c) {
+  if (!c) return fail(PHOTON_ERR_ARG, "config is NULL");
+  if (c->levels < 1 || c->levels > PHOTON_MAX_LEVELS)
+    return fail(PHOTON_ERR_ARG, "levels must be 1..%d", PHOTON_MAX_LEVELS);
+  if (c->vocab <= 0 || c->d_model <= 0 || c->n_heads <= 0 || c->head_dim <= 0)
+    return fail(PHOTON_ERR_ARG, "non-positive model dimension");
+  if (c->d_model != c->n_heads * c->head_dim) return fail(PHOTON_ERR_ARG, "d_model must equal n_heads * head_dim");
+  if (c->head_dim != 32 && c->head_dim != 64) return fail(PHOTON_ERR_ARG, "head_dim must be 32 or 64");
+  if (c->d_model % 64) return fail(PHOTON_ERR_ARG, "d_model must be a multiple of 64");
+  for (int l = 0; l < c->levels; ++l) {
+    if (c->chunk[l] < 1 || c->chunk[l] > 4) return fail(PHOTON_ERR_ARG, "chunk sizes must be 1..4");
+    if (c->enc_layers[l] < 1 || c->dec_layers[l] < 1) return fail(PHOTON_ERR_ARG, "layer counts must be >= 1");
+  }
+  if (c->mlp_mult < 1) return fail(PHOTON_ERR_ARG, "mlp_mult must be >= 1");
+  if (c->dtype != 0 && c->dtype != 1) return fail(PHOTON_ERR_ARG, "dtype must be 0 (fp32) or 1 (bf16)");
+  if (!(c->norm_eps > 0.f) || !(c->rope_theta > 0.f) || !(c->init_std > 0.f))
+    return fail(PHOTON_ERR_ARG, "eps, theta and init_std must be positive");
+  return PHOTON_OK;
+}
+
+// Tensor list of an L-level model: embed; chunker_l and encoder_l for
+// l = 1..L (the last encoder is the top encoder); converter_l and decoder_l
+// for l = L..1; head.  For L = 2 this is the two-level list.
+static void build_specs_levels(photon_model* m) {
+  const long long d = m->d, V = m->V, f = m->f;
+  const int L = m->NL;
+  auto add = [&](const std::string& n, int g, long long numel, bool gain) {
+    m->t.push_back(TensorRec{n, g, 0, numel, gain});
+  };
+  auto blocks = [&](const std::string& p, int n, int g) {
+    for (int l = 0; l < n; ++l) {
+      const std::string s = p + "." + std::to_string(l) + ".";
+      add(s + "g_attn", g, d, true);
+      add(s + "wq", g, d * d, false);
+      add(s + "wk", g, d * d, false);
+      add(s + "wv", g, d * d, false);
+      add(s + "wo", g, d * d, false);
+      add(s + "g_mlp", g, d, true);
+      add(s + "w1", g, f * d, false);
+      add(s + "w2", g, d * f, false);
+    }
+  };
+  m->i_embed = (int)m->t.size();
+  add("embed", G_EMB, V * d, false);
+  for (int l = 1; l <= L; ++l) {
+    const int g = l == L ? G_TOP : G_ENC1;
+    const std::string name = l == L ? "top" : "enc" + std::to_string(l);
+    m->i_chl[l - 1] = (int)m->t.size();
+    add("chunker" + std::to_string(l), g, d * m->Cl[l - 1] * d, false);
+    m->i_encl[l - 1] = (int)m->t.size();
+    blocks(name, m->El[l - 1], g);
+    m->i_encl_g[l - 1] = (int)m->t.size();
+    add(name + ".g_final", g, d, true);
+  }
+  for (int l = L; l >= 1; --l) {
+    m->i_cvl[l - 1] = (int)m->t.size();
+    add("converter" + std::to_string(l), G_DEC, m->Cl[l - 1] * d * d, false);
+    m->i_decl[l - 1] = (int)m->t.size();
+    blocks("dec" + std::to_string(l), m->Dl[l - 1], G_DEC);
+    m->i_decl_g[l - 1] = (int)m->t.size();
+    add("dec" + std::to_string(l) + ".g_final", G_DEC, d, true);
+  }
+  m->i_head = (int)m->t.size();
+  add("head", G_DEC, V * d, false);
+  for (auto& r : m->t) {
+    const size_t bytes = (size_t)r.numel * (r.gain ? 4 : m->es);
+    r.offset = m->group_bytes[r.group];
+    m->group_bytes[r.group] += (bytes + 255) & ~size_t(255);
+  }
+}
+
+// Product C_1 * ... * C_l (P(0) = 1).
+static int gen_prod(const photon_model* m, int l) {
+  int p = 1;
+  for (int j = 0; j < l; ++j) p *= m->Cl[j];
+  return p;
+}
+
+static int gen_prefill(photon_model* m, const int32_t* d_tokens, int B, int T, int mode, int max_new,
+                       cudaStream_t s, photon_cache** out) {
+  const int L = m->NL, d = m->d, C = m->C, C1 = m->Cl[0], H = m->H, dh = m->dh;
+  const size_t es = m->es, hd = (size_t)H * dh;
+  const float eps = m->cfg.norm_eps;
+  if (mode == PHOTON_MODE_REC && L < 2) return fail(PHOTON_ERR_ARG, "RecGen needs at least two levels");
+  photon_cache* c = new photon_cache();
+  GenCache* g = new GenCache();
+  c->gen = g;
+  g->L = L;
+  c->m = m;
+  c->B = B;
+  c->T = T;
+  c->mode = mode;
+  c->max_new = max_new;
+  c->stream = s;
+  Allocator al{s, &c->allocs, &c->kv_bytes};
+  auto bail = [&](int code) {
+    cudaGetLastError();
+    if (c->cap) cudaStreamDestroy(c->cap);
+    free_list(c->allocs, s);
+    cudaStreamSynchronize(s);
+    delete g;
+    delete c;
+    return code == PHOTON_ERR_OOM ? fail(code, "device allocation failed during prefill") : code;
+  };
+  // encoder caches: level l holds T / P(l) entries after prefill and grows by
+  // C / P(l) per HierGen step (the top by one per step in both modes)
+  std::vector<void*> tmp;
+  size_t tmp_bytes = 0;
+  Allocator at{s, &tmp, &tmp_bytes};
+  for (int l = 1; l <= L; ++l) {
+    const int Tl = T / gen_prod(m, l);
+    const bool keep = l == L || mode == PHOTON_MODE_HIER;
+    const int grow = l == L ? 1 : C / gen_prod(m, l);
+    g->cap[l - 1] = Tl + (keep ? grow * max_new : 0);
+    g->layer[l - 1] = (size_t)B * hd * g->cap[l - 1] * es;
+    Allocator& A = keep ? al : at;
+    g->kc[l - 1] = A.get<char>(g->layer[l - 1] * m->El[l - 1]);
+    g->vc[l - 1] = A.get<char>(g->layer[l - 1] * m->El[l - 1]);
+    g->n[l - 1] = keep ? Tl : 0;
+  }
+  c->top_k = g->kc[L - 1];
+  c->top_v = g->vc[L - 1];
+  c->top_layer = g->layer[L - 1];
+  c->Ncap = g->cap[L - 1];
+  c->N = g->n[L - 1];
+  c->N1 = (L >= 2 && mode == PHOTON_MODE_HIER) ? g->n[0] : 0;
+  c->N1cap = L >= 2 ? g->cap[0] : 0;
+  if (L >= 2 && mode == PHOTON_MODE_HIER) {
+    c->l1_k = g->kc[0];
+    c->l1_v = g->vc[0];
+    c->l1_layer = g->layer[0];
+  }
+  // decode workspace
+  al.counter = &c->ws_bytes;
+  c->o = al.get<void>((size_t)B * d * es);
+  c->d_err = al.get<int>(16);
+  g->d_n = al.get<int>(64);
+  int rows_max = B * C;
+  int groups = B;
+  for (int l = L; l >= 1; --l) {
+    const int Cl = m->Cl[l - 1];
+    g->G[l - 1] = groups;
+    const int rows = groups * Cl;
+    g->xdec[l - 1] = al.get<float>((size_t)rows * d * 4);
+    if (l >= 2) g->ahat[l - 1] = al.get<void>((size_t)rows * d * es);
+    const int kv = l == 1 ? 2 * C1 : Cl;
+    g->dlayer[l - 1] = (size_t)groups * hd * kv * es;
+    g->dk[l - 1] = al.get<char>(g->dlayer[l - 1] * m->Dl[l - 1]);
+    g->dv[l - 1] = al.get<char>(g->dlayer[l - 1] * m->Dl[l - 1]);
+    groups = rows;
+  }
+  const int G1 = g->G[0];
+  g->xs = al.get<float>((size_t)G1 * d * 4);
+  g->hn = al.get<void>((size_t)G1 * d * es);
+  g->logits = al.get<float>((size_t)G1 * m->V * 4);
+  g->next_ids = al.get<int32_t>((size_t)G1 * 4);
+  g->used = al.get<int32_t>((size_t)B * C * 4);
+  g->tok_out = al.get<int32_t>((size_t)B * C * 4);
+  c->tok_out = g->tok_out;
+  g->emb = al.get<void>((size_t)B * C * d * es);
+  for (int l = 1; l < L; ++l) {
+    const int rows = B * (C / gen_prod(m, l));
+    g->xre[l - 1] = al.get<float>((size_t)rows * d * 4);
+    g->sre[l - 1] = al.get<void>((size_t)rows * d * es);
+  }
+  g->xt = al.get<float>((size_t)B * d * 4);
+  // workspaces of every GEMM and attention shape of a decode step
+  size_t gw = 0, aw = 0;
+  auto gneed = [&](int M, int N, int K) { gw = std::max(gw, gemm_ws_need(m, M, N, K)); };
+  auto aneed = [&](int G, int q, int n) { aw = std::max(aw, attn_ws_need(m->dt, G, H, dh, q, n)); };
+  gw = std::max(gw, block_ws_need(m, B));
+  gw = std::max(gw, block_ws_need(m, rows_max));
+  gneed(B, m->Cl[L - 1] * d, d);
+  gneed(B, d, m->Cl[L - 1] * d);
+  for (int l = L; l >= 1; --l) {
+    const int Gl = g->G[l - 1], Cl = m->Cl[l - 1];
+    gw = std::max(gw, block_ws_need(m, Gl * Cl));
+    gw = std::max(gw, block_ws_need(m, Gl));
+    gneed(Gl, Cl * d, d);
+    aneed(Gl, std::min(Cl, 4), l == 1 ? 2 * C1 : Cl);
+  }
+  gneed(G1, m->V, d);
+  for (int i = 0; i < C1; ++i) aneed(G1, i == 0 ? std::min(C1, 4) : 1, C1 + i);
+  aneed(B, 1, g->cap[L - 1]);
+  for (int l = 1; l < L; ++l) {
+    const int q = C / gen_prod(m, l), rows = B * q;
+    gw = std::max(gw, block_ws_need(m, rows));
+    gneed(rows, d, m->Cl[l - 1] * d);
+    if (q <= 4) aneed(B, q, g->cap[l - 1]);
+  }
+  Bufs& b = g->b;
+  b.xn = al.get<void>((size_t)rows_max * d * es);
+  b.q = al.get<void>((size_t)rows_max * d * es);
+  b.att = al.get<void>((size_t)rows_max * d * es);
+  b.hid = al.get<void>((size_t)rows_max * m->f * es);
+  b.gemm_ws_bytes = gw;
+  b.gemm_ws = al.get<float>(gw);
+  b.gemm_cnt = al.get<int>(kGemmTileCounters * sizeof(int));
+  b.attn_ws_bytes = aw;
+  b.attn_ws = al.get<float>(aw);
+  b.err = c->d_err;
+  int positions = 2 * C1 + 1;
+  for (int l = 0; l < L; ++l) positions = std::max(positions, std::max(g->cap[l], m->Cl[l]) + 1);
+  int rc = upload_rope(m, &c->rope, al, positions);
+  b.rope = c->rope;
+  if (al.err != cudaSuccess || rc) return bail(PHOTON_ERR_OOM);
+  if (cudaStreamCreateWithFlags(&c->cap, cudaStreamNonBlocking) != cudaSuccess)
+    return bail(fail(PHOTON_ERR_CUDA, "stream creation failed"));
+  std::vector<int> hn(PHOTON_MAX_LEVELS + 1, 0);
+  for (int l = 0; l < L; ++l) hn[l] = g->n[l];
+  if (cudaMemsetAsync(c->d_err, 0, 16, s) != cudaSuccess ||
+      cudaMemsetAsync(b.gemm_cnt, 0, kGemmTileCounters * sizeof(int), s) != cudaSuccess ||
+      cudaMemcpyAsync(g->d_n, hn.data(), hn.size() * sizeof(int), cudaMemcpyHostToDevice, s) != cudaSuccess ||
+      cudaStreamSynchronize(s) != cudaSuccess)  // the host copy of hn leaves scope
+    return bail(PHOTON_ERR_CUDA);
+
+  // prefill: bottom-up through every level
+  const long long rows0 = (long long)B * T, rows1 = rows0 / m->Cl[0];
+  void* emb = at.get<void>((size_t)rows0 * d * es);
+  float* x = at.get<float>((size_t)rows1 * d * 4);
+  void* sb = at.get<void>((size_t)rows1 * d * es);
+  size_t pgw = 0, paw = 0;
+  for (int l = 1; l <= L; ++l) {
+    const int rows = (int)(rows0 / gen_prod(m, l)), Tl = T / gen_prod(m, l);
+    pgw = std::max(pgw, block_ws_need(m, rows));
+    pgw = std::max(pgw, gemm_ws_need(m, rows, d, m->Cl[l - 1] * d));
+    if (Tl <= 4) paw = std::max(paw, attn_ws_need(m->dt, B, H, dh, Tl, Tl));
+  }
+  Bufs pb;
+  pb.xn = at.get<void>((size_t)rows1 * d * es);
+  pb.q = at.get<void>((size_t)rows1 * d * es);
+  pb.att = at.get<void>((size_t)rows1 * d * es);
+  pb.hid = at.get<void>((size_t)rows1 * m->f * es);
+  pb.rope = c->rope;
+  pb.gemm_ws = at.get<float>(pgw);
+  pb.gemm_ws_bytes = pgw;
+  pb.gemm_cnt = b.gemm_cnt;
+  pb.attn_ws = at.get<float>(paw);
+  pb.attn_ws_bytes = paw;
+  pb.err = c->d_err;
+  if (at.err != cudaSuccess) {
+    free_list(tmp, s);
+    return bail(PHOTON_ERR_OOM);
+  }
+  launch_embed(m->dt, d_tokens, m->ptr(m->i_embed), emb, (int)rows0, d, m->V, c->d_err, s);
+  const void* prev = emb;
+  for (int l = 1; l <= L; ++l) {
+    const int Cl = m->Cl[l - 1], Tl = T / gen_prod(m, l), rows = B * Tl;
+    gemm(m, pb, prev, (long long)Cl * d, m->ptr(m->i_chl[l - 1]), (long long)Cl * d, rows, d, Cl * d,
+         epi(EPI_STORE_F32, x, d), s);
+    StackRun r;
+    r.G = B;
+    r.q_len = Tl;
+    r.kc = g->kc[l - 1];
+    r.vc = g->vc[l - 1];
+    r.layer_bytes = g->layer[l - 1];
+    r.cap = g->cap[l - 1];
+    r.n_plan = Tl;
+    run_stack(m, m->i_encl[l - 1], m->El[l - 1], x, r, pb, s);
+    if (l < L) {
+      launch_rmsnorm(m->dt, x, (const float*)m->ptr(m->i_encl_g[l - 1]), sb, rows, d, 1, 0, eps, s);
+      prev = sb;
+    } else {
+      launch_rmsnorm(m->dt, x, (const float*)m->ptr(m->i_encl_g[l - 1]), c->o, B, d, Tl, Tl - 1, eps, s);
+    }
+  }
+  const cudaError_t e = cudaGetLastError();
+  free_list(tmp, s);
+  if (e != cudaSuccess) return bail(fail(PHOTON_ERR_CUDA, "prefill launch: %s", cudaGetErrorString(e)));
+  m->live_caches++;
+  if (mode == PHOTON_MODE_HIER) m->hier_caches++;
+  *out = c;
+  return PHOTON_OK;
+}
+
+// One decode step of an L-level model: top-down through every level (all
+// groups of a level at once), the token decoder and head, then the top
+// encoder's next input and its step.
+static void gen_enqueue(photon_model* m, photon_cache* c, int mode, int32_t* out_tokens, float* out_logits,
+                        const int32_t* force, const void* force_a, cudaStream_t s) {
+  GenCache* g = c->gen;
+  const int L = m->NL, B = c->B, d = m->d, C = m->C, C1 = m->Cl[0], V = m->V;
+  const float eps = m->cfg.norm_eps;
+  const Bufs& b = g->b;
+  const void* src = c->o;
+  for (int l = L; l >= 2; --l) {
+    const int Gl = g->G[l - 1], Cl = m->Cl[l - 1];
+    gemm(m, b, src, d, m->ptr(m->i_cvl[l - 1]), d, Gl, Cl * d, d, epi(EPI_STORE_F32, g->xdec[l - 1], (long long)Cl * d), s);
+    StackRun r;
+    r.G = Gl;
+    r.q_len = Cl;
+    r.kc = g->dk[l - 1];
+    r.vc = g->dv[l - 1];
+    r.layer_bytes = g->dlayer[l - 1];
+    r.cap = Cl;
+    run_stack(m, m->i_decl[l - 1], m->Dl[l - 1], g->xdec[l - 1], r, b, s);
+    launch_rmsnorm(m->dt, g->xdec[l - 1], (const float*)m->ptr(m->i_decl_g[l - 1]), g->ahat[l - 1], Gl * Cl, d, 1, 0,
+                   eps, s);
+    src = g->ahat[l - 1];
+  }
+  // token decoder over each group's C_1 conditioning vectors, then one row per token
+  const int G1 = g->G[0];
+  gemm(m, b, src, d, m->ptr(m->i_cvl[0]), d, G1, C1 * d, d, epi(EPI_STORE_F32, g->xdec[0], (long long)C1 * d), s);
+  StackRun r1;
+  r1.G = G1;
+  r1.q_len = C1;
+  r1.kc = g->dk[0];
+  r1.vc = g->dv[0];
+  r1.layer_bytes = g->dlayer[0];
+  r1.cap = 2 * C1;
+  run_stack(m, m->i_decl[0], m->Dl[0], g->xdec[0], r1, b, s);
+  SampleArgs sa;
+  sa.inv_t = c->samp_inv_t;
+  sa.seed = c->samp_seed;
+  sa.chunk = g->d_n + PHOTON_MAX_LEVELS;
+  sa.C1 = C1;
+  sa.C2 = C / C1;
+  for (int i = 0; i < C1; ++i) {
+    const float* x = i == 0 ? g->xdec[0] : g->xs;
+    launch_rmsnorm(m->dt, x, (const float*)m->ptr(m->i_decl_g[0]), g->hn, G1, d, i == 0 ? C1 : 1,
+                   i == 0 ? C1 - 1 : 0, eps, s);
+    const long long ld = out_logits ? (long long)C1 * V : V;
+    float* lg = out_logits ? out_logits + (size_t)i * V : g->logits;
+    gemm(m, b, g->hn, d, m->ptr(m->i_head), d, G1, V, d, epi(EPI_STORE_F32, lg, ld), s);
+    sa.i = i;
+    launch_argmax(lg, ld, G1, V, i, C1, force, out_tokens, g->used, g->next_ids, c->d_err, sa, s);
+    if (i + 1 < C1) {
+      launch_embed_f32(m->dt, g->next_ids, m->ptr(m->i_embed), g->xs, G1, d, V, c->d_err, s);
+      StackRun rs = r1;
+      rs.q_len = 1;
+      rs.p0 = C1 + i;
+      run_stack(m, m->i_decl[0], m->Dl[0], g->xs, rs, b, s);
+    }
+  }
+  launch_advance(g->d_n + PHOTON_MAX_LEVELS, 1, 0, s);  // chunks generated (sampling keys)
+  // the top encoder's next input
+  const int CL = m->Cl[L - 1];
+  const void* top_in;
+  if (mode == PHOTON_MODE_REC) {
+    top_in = force_a ? force_a : g->ahat[L - 1];
+  } else {
+    launch_embed(m->dt, g->used, m->ptr(m->i_embed), g->emb, B * C, d, V, c->d_err, s);
+    const void* prev = g->emb;
+    for (int l = 1; l < L; ++l) {
+      const int Cl = m->Cl[l - 1], q = C / gen_prod(m, l), rows = B * q;
+      gemm(m, b, prev, (long long)Cl * d, m->ptr(m->i_chl[l - 1]), (long long)Cl * d, rows, d, Cl * d,
+           epi(EPI_STORE_F32, g->xre[l - 1], d), s);
+      StackRun re;
+      re.G = B;
+      re.q_len = q;
+      re.p0_dev = g->d_n + (l - 1);
+      re.n_plan = g->cap[l - 1];
+      re.kc = g->kc[l - 1];
+      re.vc = g->vc[l - 1];
+      re.layer_bytes = g->layer[l - 1];
+      re.cap = g->cap[l - 1];
+      run_stack(m, m->i_encl[l - 1], m->El[l - 1], g->xre[l - 1], re, b, s);
+      launch_rmsnorm(m->dt, g->xre[l - 1], (const float*)m->ptr(m->i_encl_g[l - 1]), g->sre[l - 1], rows, d, 1, 0,
+                     eps, s);
+      prev = g->sre[l - 1];
+    }
+    top_in = prev;
+  }
+  gemm(m, b, top_in, (long long)CL * d, m->ptr(m->i_chl[L - 1]), (long long)CL * d, B, d, CL * d,
+       epi(EPI_STORE_F32, g->xt, d), s);
+  StackRun rt;
+  rt.G = B;
+  rt.q_len = 1;
+  rt.p0_dev = g->d_n + (L - 1);
+  rt.n_plan = g->cap[L - 1];
+  rt.kc = g->kc[L - 1];
+  rt.vc = g->vc[L - 1];
+  rt.layer_bytes = g->layer[L - 1];
+  rt.cap = g->cap[L - 1];
+  run_stack(m, m->i_encl[L - 1], m->El[L - 1], g->xt, rt, b, s);
+  launch_rmsnorm(m->dt, g->xt, (const float*)m->ptr(m->i_encl_g[L - 1]), c->o, B, d, 1, 0, eps, s);
+  // positions: the top grows by one entry; in HierGen level l by C / P(l)
+  launch_advance(g->d_n + (L - 1), 1, 0, s);
+  if (mode == PHOTON_MODE_HIER)
+    for (int l = 1; l < L; ++l) launch_advance(g->d_n + (l - 1), C / gen_prod(m, l), 0, s);
+}
+
+static int gen_decode_step(photon_model* m, photon_cache* c, int mode, int32_t* d_out_tokens, float* d_out_logits,
+                           const int32_t* d_force_tokens, const void* d_force_a, cudaStream_t s) {
+  GenCache* g = c->gen;
+  const int L = m->NL;
+  if (mode == PHOTON_MODE_REC && L < 2) return fail(PHOTON_ERR_ARG, "RecGen needs at least two levels");
+  if (mode == PHOTON_MODE_HIER && c->mode != PHOTON_MODE_HIER && L >= 2)
+    return fail(PHOTON_ERR_MODE, "HierGen needs the lower encoder caches, discarded by a RecGen prefill");
+  if (c->steps >= c->max_new) return fail(PHOTON_ERR_CAPACITY, "cache is full (%d steps)", c->max_new);
+  c->stream = s;
+  const bool plain = !d_out_logits && !d_force_tokens && !d_force_a;
+  bool replay = plain && graphs_enabled() && c->steps >= 1 && !g->graph_failed[mode];
+  if (replay && m->ggraph_owner[mode] != c) {
+    cudaGraph_t gr = nullptr;
+    const unsigned long long n0 = launch_total();
+    bool ok = cudaStreamBeginCapture(c->cap, cudaStreamCaptureModeRelaxed) == cudaSuccess;
+    if (ok) {
+      gen_enqueue(m, c, mode, g->tok_out, nullptr, nullptr, nullptr, c->cap);
+      ok = cudaStreamEndCapture(c->cap, &gr) == cudaSuccess && gr;
+    }
+    const long long captured = (long long)(launch_total() - n0);
+    note_launch(-captured);
+    m->ggraph_kernels[mode] = ok ? captured : 0;
+    if (ok && m->ggraph[mode]) {
+      cudaGraphExecUpdateResultInfo info;
+      if (cudaGraphExecUpdate(m->ggraph[mode], gr, &info) != cudaSuccess) {
+        cudaGetLastError();
+        cudaGraphExecDestroy(m->ggraph[mode]);
+        m->ggraph[mode] = nullptr;
+      }
+    }
+    if (ok && !m->ggraph[mode]) ok = cudaGraphInstantiate(&m->ggraph[mode], gr, 0) == cudaSuccess;
+    if (gr) cudaGraphDestroy(gr);
+    if (!ok) {
+      cudaGetLastError();
+      m->ggraph[mode] = nullptr;
+      m->ggraph_owner[mode] = nullptr;
+      g->graph_failed[mode] = true;
+      replay = false;
+    } else {
+      m->ggraph_owner[mode] = c;
+    }
+  }
+  if (replay) {
+    CK(cudaGraphLaunch(m->ggraph[mode], s));
+    note_launch(m->ggraph_kernels[mode]);
+    c->graph_steps += 1;
+    if (d_out_tokens != g->tok_out)
+      CK(cudaMemcpyAsync(d_out_tokens, g->tok_out, (size_t)c->B * m->C * sizeof(int32_t), cudaMemcpyDeviceToDevice,
+                         s));
+  } else {
+    gen_enqueue(m, c, mode, d_out_tokens, d_out_logits, d_force_tokens, d_force_a, s);
+  }
+  CK(cudaGetLastError());
+  g->n[L - 1] += 1;
+  if (mode == PHOTON_MODE_HIER)
+    for (int l = 1; l < L; ++l) g->n[l - 1] += m->C / gen_prod(m, l);
+  c->N = g->n[L - 1];
+  c->N1 = (L >= 2 && mode == PHOTON_MODE_HIER) ? g->n[0] : 0;
+  if (L >= 2) {
+    c->a_hat = g->ahat[L - 1];
+    c->ahat_latest = g->ahat[L - 1];
+    c->has_a_hat = true;
+    if (mode == PHOTON_MODE_HIER) {
+      c->a = g->sre[L - 2];
+      c->has_a = true;
+    }
+  }
+  c->steps += 1;
+  return PHOTON_OK;
+}
+
+
 extern "C" {
 
 int photon_prefill(photon_model* m, const photon_cache* prefix, const int32_t* d_tokens, int32_t B,
                    int32_t T, int32_t mode, int32_t max_new_chunks, void* stream, photon_cache** out) {
+  if (m && m->general) {
+    g_err.clear();
+    if (!out) return fail(PHOTON_ERR_ARG, "out is NULL");
+    *out = nullptr;
+    if (prefix) return fail(PHOTON_ERR_ARG, "shared prefixes are not supported for this model");
+    if (!d_tokens || B <= 0 || T <= 0 || T % m->C) return fail(PHOTON_ERR_ARG, "T must be a positive multiple of C");
+    if (mode != PHOTON_MODE_HIER && mode != PHOTON_MODE_REC) return fail(PHOTON_ERR_ARG, "unknown mode %d", mode);
+    if (max_new_chunks < 0) return fail(PHOTON_ERR_ARG, "max_new_chunks must be >= 0");
+    return gen_prefill(m, d_tokens, B, T, mode, max_new_chunks, (cudaStream_t)stream, out);
+  }
   return prefill_impl(m, prefix, d_tokens, B, T, mode, max_new_chunks, stream, out, nullptr);
 }
 
@@ -1547,6 +2140,8 @@ int photon_decode_step_ex(photon_model* m, photon_cache* c, int32_t mode, int32_
   if (!m || !c || c->m != m) return fail(PHOTON_ERR_ARG, "model/cache mismatch");
   if (!d_out_tokens) return fail(PHOTON_ERR_ARG, "output token buffer is NULL");
   if (mode != PHOTON_MODE_HIER && mode != PHOTON_MODE_REC) return fail(PHOTON_ERR_ARG, "unknown mode %d", mode);
+  if (m->general) return gen_decode_step(m, c, mode, d_out_tokens, d_out_logits, d_force_tokens, d_force_a,
+                                         (cudaStream_t)stream);
   if (mode == PHOTON_MODE_HIER && (c->mode != PHOTON_MODE_HIER || !c->l1_k))
     return fail(PHOTON_ERR_MODE, "HierGen needs the level-1 KV, discarded by a RecGen prefill");
   if (c->steps >= c->max_new) return fail(PHOTON_ERR_CAPACITY, "cache is full (%d steps)", c->max_new);
@@ -1715,6 +2310,14 @@ int photon_decode_rec_chunks(photon_model* m, photon_cache* c, int32_t n, int32_
                          cudaMemcpyDeviceToDevice, s));
     return PHOTON_OK;
   };
+  if (m->general) {  // any-L models: one (graph-replayed) step per chunk
+    for (int k = 0; k < n; ++k) {
+      RET(photon_decode_step_ex(m, c, PHOTON_MODE_REC, c->gen_tok_out(), nullptr, nullptr, nullptr, stream));
+      CK(cudaMemcpy2DAsync(d_out_tokens + (size_t)k * C, pitch, c->gen_tok_out(), w, w, B, cudaMemcpyDeviceToDevice,
+                           s));
+    }
+    return PHOTON_OK;
+  }
   if (c->steps == 0) {
     RET(one_step(0));
     t = 1;
@@ -1774,8 +2377,10 @@ int photon_free_cache(photon_cache* c) {
   if (!c) return fail(PHOTON_ERR_ARG, "cache is NULL");
   if (c->dependents) return fail(PHOTON_ERR_ARG, "%d caches still read this prefix", c->dependents);
   photon_model* m = c->m;
-  for (int k = 0; k < 2; ++k)
+  for (int k = 0; k < 2; ++k) {
     if (m->graph_owner[k] == c) m->graph_owner[k] = nullptr;  // its buffers are going away
+    if (m->ggraph_owner[k] == c) m->ggraph_owner[k] = nullptr;
+  }
   if (m->pg_owner == c) m->pg_owner = nullptr;
   // Stream-ordered release: the helper streams' pending work is joined into
   // the cache's stream, the buffers go back to the pool on that stream, and
@@ -1812,6 +2417,7 @@ int photon_free_cache(photon_cache* c) {
   m->live_caches--;
   if (c->mode == PHOTON_MODE_HIER) m->hier_caches--;
   for (auto& e : c->tk_plans) top_step_free(e.plan);  // host-side launch descriptions only
+  delete c->gen;
   delete c;
   return PHOTON_OK;
 }
@@ -1827,8 +2433,10 @@ int photon_cache_set_sampling(photon_cache* c, float temperature, uint64_t seed)
   c->samp_seed = seed;
   // captured steps carry the old parameters: capture again on the next step
   photon_model* m = c->m;
-  for (int k = 0; k < 2; ++k)
+  for (int k = 0; k < 2; ++k) {
     if (m->graph_owner[k] == c) m->graph_owner[k] = nullptr;
+    if (m->ggraph_owner[k] == c) m->ggraph_owner[k] = nullptr;
+  }
   if (m->pg_owner == c) m->pg_owner = nullptr;
   return PHOTON_OK;
 }
@@ -1888,7 +2496,9 @@ int photon_cache_info(photon_cache* c, photon_cache_stats* out) {
   out->kv_bytes = c->kv_bytes;
   out->workspace_bytes = c->ws_bytes;
   out->graph_steps = c->graph_steps;
-  out->graph_kernels = (c->mode >= 0 && c->mode < 2 && c->m->graph_owner[c->mode] == c)
+  out->graph_kernels = c->gen ? (int32_t)std::max(c->m->ggraph_owner[0] == c ? c->m->ggraph_kernels[0] : 0,
+                                                 c->m->ggraph_owner[1] == c ? c->m->ggraph_kernels[1] : 0)
+                       : (c->mode >= 0 && c->mode < 2 && c->m->graph_owner[c->mode] == c)
                            ? (int32_t)c->m->graph_kernels[c->mode]
                            : c->m->pg_owner == c ? (int32_t)(c->m->pg_kernels[0] + c->m->pg_kernels[1]) : 0;
   return PHOTON_OK;
@@ -2622,6 +3232,7 @@ int photon_score(photon_model* m, const int32_t* d_tokens, int32_t B, int32_t T,
   g_err.clear();
   if (!m || !d_tokens || !d_out_logprob) return fail(PHOTON_ERR_ARG, "NULL argument");
   if (m->vanilla) return fail(PHOTON_ERR_ARG, "a vanilla baseline model takes the photon_vanilla_* calls");
+  if (m->general) return fail(PHOTON_ERR_ARG, "teacher-forced scoring is available for two-level models only");
   if (B <= 0 || T <= m->C || T % m->C)
     return fail(PHOTON_ERR_ARG, "T = %d must be a multiple of C1*C2 = %d longer than one chunk", T, m->C);
   // The decoders run over (sequence, chunk, sub-chunk) groups, which the
@@ -2682,6 +3293,7 @@ int photon_multi_query(photon_model* m, const photon_cache* prefix, const int32_
                        int32_t mode, int32_t* d_cand, int32_t* d_choice, double* d_score, void* stream) {
   g_err.clear();
   if (!m || !d_prompts || !d_cand || !d_choice) return fail(PHOTON_ERR_ARG, "NULL argument");
+  if (m->general) return fail(PHOTON_ERR_ARG, "multi-query aggregation is available for two-level models only");
   if (m->vanilla) return fail(PHOTON_ERR_ARG, "a vanilla baseline model takes the photon_vanilla_* calls");
   if (mode != PHOTON_AGG_VOTE && mode != PHOTON_AGG_BEST) return fail(PHOTON_ERR_ARG, "unknown aggregation mode %d", mode);
   if (Q <= 0 || N <= 0 || n_chunks <= 0 || (long long)Q * N > (1ll << 30))

@@ -87,12 +87,14 @@ enum { PHOTON_MODE_HIER = 0, PHOTON_MODE_REC = 1 };
  * generator: tensor t (fixed order: embed, chunker1, level-1 encoder
  * blocks + final gain, chunker2, top blocks + final gain, converter2,
  * level-2 decoder blocks + gain, converter1, token decoder blocks + gain,
- * head; per block g_attn, wq, wk, wv, wo, g_mlp, w1, w2), element e: SplitMix64
- * key mix(seed + gamma*(t+1)), draw z = mix(key + gamma*(e+1)), S = sum of the
- * four 16-bit fields of z, w = fp64(S - 131070) * init_std*1.7320508075688772/65536,
- * rounded to fp32 then to the storage type; RMSNorm gains are 1.  Linear maps
- * are [out, in].  Synchronising.  Errors: ERR_ARG (bad config or out==NULL),
- * ERR_OOM, ERR_CUDA. */
+ * head; per block g_attn, wq, wk, wv, wo, g_mlp, w1, w2), element e: an
+ * N(0, init_std^2) variable by Marsaglia's polar method from the SplitMix64
+ * stream of key mix(mix(seed + gamma*(t+1)) + gamma*(e+1)) (attempt a takes
+ * the stream's outputs 2a+1 and 2a+2 as 53-bit uniforms on [-1, 1); ln by its
+ * atanh series; every fp64 step correctly rounded), rounded to fp32 then to
+ * the storage type; RMSNorm gains are 1.  Linear maps are [out, in].
+ * Synchronising.  Errors: ERR_ARG (bad config or out==NULL), ERR_OOM,
+ * ERR_CUDA. */
 PHOTON_API int photon_init_weights(const photon_config* cfg, uint64_t seed, photon_model** out);
 
 /* Frees a model.  Every cache built on it must have been freed first
@@ -362,6 +364,47 @@ PHOTON_API int photon_attn_decode_noalloc(int32_t dtype, const void* d_q, const 
  * outside the vocabulary). */
 PHOTON_API int photon_score(photon_model* m, const int32_t* d_tokens, int32_t B, int32_t T,
                             float* d_out_logprob, void* stream);
+
+/* ------------------------------------------------------------------------
+ * Any number of levels (explainer, architecture section: every module is
+ * written for a general level l; RecGen section: Theorem A.6 needs A-hat = A
+ * only at the L -> L-1 interface).  L = 1 is a single-level block model
+ * (token blocks of C_1 merged by one linear map, a causal encoder over the
+ * blocks, a block-local token decoder), the shape of the Block Transformer
+ * the explainer compares PHOTON against; L = 3 adds a middle level.
+ *
+ * Level l = 1..L has chunk size chunk[l-1], encoder depth enc_layers[l-1]
+ * (the last is the top encoder) and decoder depth dec_layers[l-1] (the first
+ * is the token decoder).  Tensor order: embed; for l = 1..L chunker_l and
+ * encoder_l (blocks + final gain); for l = L..1 converter_l and decoder_l
+ * (blocks + final gain); head -- for L = 2 the same tensors and draws as
+ * photon_init_weights.  A model made here runs through photon_prefill,
+ * photon_decode_step_hier / _rec / _ex, photon_decode_rec_chunks,
+ * photon_cache_info, photon_export_weight / _state and the free calls.
+ * Prefill encodes bottom-up through every level; a decode step goes
+ * top-down level by level (Converter_l, then Decoder_l over its C_l
+ * conditioning positions for every group at once), then the token decoder
+ * writes the chunk's C tokens; HierGen re-encodes them through levels
+ * 1..L-1 (whose caches grow) and RecGen (L >= 2) feeds Chunker_L(A-hat_L)
+ * to the top encoder, keeping only the top cache.  Every weight stays
+ * resident.  The two-level optimisations (the forked and pipelined RecGen
+ * branches, the persistent top step) are specific to photon_init_weights
+ * models; steps here are captured once per mode into a graph and replayed.
+ * Not supported on these models: shared prefixes, photon_score,
+ * photon_multi_query. */
+#define PHOTON_MAX_LEVELS 4
+typedef struct {
+  int32_t vocab, d_model, n_heads, head_dim;
+  int32_t levels;                         /* L, 1..PHOTON_MAX_LEVELS */
+  int32_t chunk[PHOTON_MAX_LEVELS];       /* C_1 .. C_L, each 1..4 */
+  int32_t enc_layers[PHOTON_MAX_LEVELS];  /* encoder depth of levels 1..L */
+  int32_t dec_layers[PHOTON_MAX_LEVELS];  /* decoder depth of levels 1..L */
+  int32_t mlp_mult, dtype;
+  float init_std, rope_theta, norm_eps;
+} photon_level_config;
+
+/* Errors: ERR_ARG (bad config), ERR_OOM, ERR_CUDA.  Synchronising. */
+PHOTON_API int photon_init_weights_levels(const photon_level_config* cfg, uint64_t seed, photon_model** out);
 
 /* ------------------------------------------------------------------------
  * Multi-query aggregation (explainer, quality section: the single-query

@@ -88,3 +88,32 @@ def test_binding_rejects_bad_buffers_on_the_host():
     with pytest.raises(ValueError, match="groups of N"):
         hal.aggregate(hal.AGG_VOTE, 4, torch.zeros(2, dtype=torch.int32),
                       cand=torch.zeros(6, 4, dtype=torch.int32))
+
+
+def test_level_config_layout_and_host_checks():
+    # photon_level_config: 5 ints, three arrays of 4, 2 ints, 3 floats; the
+    # configuration is checked on the host before any CUDA call
+    import ctypes
+    assert ctypes.sizeof(hal.photon_level_config) == 4 * (5 + 12 + 2 + 3)
+    base = {"vocab": 256, "d_model": 64, "n_heads": 2, "head_dim": 32, "dtype": "fp32"}
+    c = hal.level_config_struct(dict(base, chunks=[2, 2, 2], enc_layers=[1, 1, 2], dec_layers=[1, 1, 1]))
+    assert (c.levels, c.chunk[2], c.enc_layers[2], c.dec_layers[0]) == (3, 2, 2, 1)
+    with pytest.raises(ValueError):
+        hal.level_config_struct(dict(base, chunks=[2, 2], enc_layers=[1], dec_layers=[1, 1]))
+    lib = hal.load_library()
+    h = ctypes.c_void_p()
+    for bad in (dict(levels=0), dict(levels=5), dict(chunk=(5, 1, 1, 1)), dict(chunk=(0, 1, 1, 1)),
+                dict(enc=(0, 1, 1, 1)), dict(d_model=96)):
+        cfg = hal.level_config_struct(dict(base, chunks=[2, 2], enc_layers=[1, 1], dec_layers=[1, 1]))
+        if "levels" in bad:
+            cfg.levels = bad["levels"]
+        if "chunk" in bad:
+            for i, v in enumerate(bad["chunk"]):
+                cfg.chunk[i] = v
+        if "enc" in bad:
+            for i, v in enumerate(bad["enc"]):
+                cfg.enc_layers[i] = v
+        if "d_model" in bad:
+            cfg.d_model = bad["d_model"]
+        assert lib.photon_init_weights_levels(ctypes.byref(cfg), 1, ctypes.byref(h)) == -1, bad
+        assert lib.photon_last_error() != b""
