@@ -339,9 +339,22 @@ def run_gpu(args) -> None:
     # width and total depth over the same prompts (its KV covers every token)
     van = None
     van_ms = 0.0
+    blk = None
+    blk_ms = 0.0
     if not prefix_len and not args.no_vanilla and args.workload in ("c2", "c3"):
         van = measure_vanilla(shape, toks, wl, stream)
         van_ms = van.pop("_decode_ms")
+        # and a single-level block model (L = 1) of the same width and depth
+        blk = measure_block(shape, toks, wl, stream)
+        blk_ms = blk.pop("_decode_ms")
+
+    # ---- residency of the level-1 encoder weights: the timed prefills above
+    # restore them from a pinned host copy (the default policy); the same
+    # prefill with the weights kept resident shows what the restore costs
+    resid = measure_residency(model, toks, chunks, stream, pre_cache)
+    # ---- the long-context workload's coarse-KV traffic and resident memory in
+    # both modes (measured on its own batch with this model)
+    longctx = measure_long_context(model, stream, dev) if args.workload == "c2" and world == 1 else None
 
     # ---- the decode's dominant kernel (its GEMM launches) and its attention,
     # alone, at the same shapes and launch configuration
@@ -355,8 +368,9 @@ def run_gpu(args) -> None:
     if pre_cache is not None:
         pre_cache.free()
 
-    total_ms, prefill_ms, decode_ms, e2e_ms, hier_dec_ms, samp_dec_ms, van_ms, sc_ms, *mq_ms = max_over_ranks(
-        [total_ms, prefill_ms, decode_ms, e2e_ms, hier_dec_ms, samp_dec_ms, van_ms, sc_ms, *mq_ms], device=dev)
+    total_ms, prefill_ms, decode_ms, e2e_ms, hier_dec_ms, samp_dec_ms, van_ms, blk_ms, sc_ms, *mq_ms = max_over_ranks(
+        [total_ms, prefill_ms, decode_ms, e2e_ms, hier_dec_ms, samp_dec_ms, van_ms, blk_ms, sc_ms, *mq_ms],
+        device=dev)
     for k, ms in zip(("vote", "best"), mq_ms):
         if isinstance(mq.get(k), dict) and ms > 0:
             q = mq["queries_per_gpu"]
@@ -411,7 +425,12 @@ def run_gpu(args) -> None:
                     "resident_gib": round(hier_res / 2 ** 30, 4),
                     "tok_s_per_gib": round(B * chunks * C / (hier_dec_ms / 1e3) / (hier_res / 2 ** 30), 1),
                     "steps": 1},
+        "residency": resid,
+        "long_context": longctx,
         "vanilla_baseline": vanilla_line(van, van_ms, world, value / world / gib) if van else None,
+        "block_baseline": block_line(blk, blk_ms, world, value / world / gib,
+                                     vanilla_line(van, van_ms, world, value / world / gib) if van else None)
+                          if blk else None,
         "scoring": ({"sequences_per_gpu": sc_b, "scored_tokens_per_gpu": sc_b * (T - C),
                      "tok_s": round(world * sc_b * (T - C) / (sc_ms / 1e3), 1), "ms": round(sc_ms, 3),
                      "covers": "teacher-forced log-probabilities (photon_score): bottom-up pass, "
@@ -595,6 +614,117 @@ def measure_vanilla(shape, toks, wl, stream) -> dict:
             "resident_gib": round(resident / 2 ** 30, 3), "kv_gib": round(info["kv_bytes"] / 2 ** 30, 3),
             "graph_steps": info["graph_steps"], "tokens": B * (n - 1), "steps": n - 1,
             "_decode_ms": ev[2].elapsed_time(ev[3])}
+
+
+def measure_residency(model, toks, chunks: int, stream, prefix) -> dict:
+    """RecGen prefill time under the default residency policy (the level-1
+    encoder weights, released after the previous prefill, come back by a
+    host-to-device copy of a pinned host copy) against the same prefill with
+    the weights kept resident; two prefills each, the second timed."""
+    import torch
+    import hierarchical_autoregressive_lm_b200 as hal
+    out = {"policy": "restore from a pinned host copy after each RecGen prefill (default)",
+           "encoder_bytes": int(model.info()["encoder_bytes"])}
+    for name, policy in (("restore", hal.ENC_RESTORE), ("keep", hal.ENC_KEEP), ("restore_again", hal.ENC_RESTORE)):
+        model.set_encoder_residency(policy)
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+        model.prefill(toks, hal.MODE_REC, chunks, prefix=prefix).free()
+        torch.cuda.synchronize()
+        ev[0].record(stream)
+        model.prefill(toks, hal.MODE_REC, chunks, prefix=prefix).free()
+        ev[1].record(stream)
+        torch.cuda.synchronize()
+        out[f"prefill_ms_{name}"] = round(ev[0].elapsed_time(ev[1]), 3)
+    model.set_encoder_residency(hal.ENC_RESTORE)
+    out.pop("prefill_ms_restore_again", None)
+    return out
+
+
+def measure_long_context(model, stream, dev) -> dict:
+    """The long-context workload (16 sequences of 32768 tokens) with the same
+    model: per mode, a prefill, one eager decode chunk and two graph-replayed
+    ones (timed), the resident bytes (weights on the device + caches) and the
+    coarse-KV bytes a chunk reads by the method's accounting."""
+    import torch
+    import hierarchical_autoregressive_lm_b200 as hal
+    wl = WORKLOADS["c3"]
+    toks = torch.from_numpy(prompt_tokens("c3")).to(dev)
+    B = toks.shape[0]
+    acct = step_roofline(model.shape, wl, _peaks()[0])
+    out = {"workload": f"c3: batch {B}, prompt {toks.shape[1]}, decode steps timed after one eager step"}
+    step = torch.empty(B, model.C, dtype=torch.int32, device=toks.device)
+    for name, mode in (("recgen", hal.MODE_REC), ("hiergen", hal.MODE_HIER)):
+        c = model.prefill(toks, mode, 3)
+        c.decode_step(mode, step)
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+        torch.cuda.synchronize()
+        ev[0].record(stream)
+        for _ in range(2):
+            c.decode_step(mode, step)
+        ev[1].record(stream)
+        torch.cuda.synchronize()
+        info = c.info()
+        resident = model.info()["resident_bytes"] + info["kv_bytes"]
+        ms = ev[0].elapsed_time(ev[1]) / 2
+        kv_read = acct["recgen"]["top_kv_read_bytes"] if mode == hal.MODE_REC else acct["hiergen"]["coarse_kv_read_bytes"]
+        out[name] = {"decode_tok_s": round(B * model.C / (ms / 1e3), 1), "ms_per_chunk": round(ms, 4),
+                     "resident_gib": round(resident / 2 ** 30, 4), "kv_gib": round(info["kv_bytes"] / 2 ** 30, 4),
+                     "coarse_kv_bytes_per_chunk": int(kv_read),
+                     "tok_s_per_gib": round(B * model.C / (ms / 1e3) / (resident / 2 ** 30), 1)}
+        c.free()
+    return out
+
+
+def measure_block(shape, toks, wl, stream) -> dict:
+    """The same prompts through a single-level block model (L = 1) of the same
+    width and total depth on the same kernels: token blocks of C1 merged by
+    one linear map, a causal encoder over the blocks (L1 + Ltop layers) and a
+    block-local token decoder (Ld1 + Ld2 layers) -- the shape of the Block
+    Transformer the explainer compares PHOTON with.  HierGen decode (RecGen
+    needs two levels) for the workload's decode length, the steps after the
+    first (which captures the step's graph) timed."""
+    import torch
+    import hierarchical_autoregressive_lm_b200 as hal
+    bshape = dict(vocab=shape["vocab"], d_model=shape["d_model"], n_heads=shape["n_heads"],
+                  head_dim=shape["head_dim"], chunks=[shape["C1"]], enc_layers=[shape["L1"] + shape["Ltop"]],
+                  dec_layers=[shape["Ld1"] + shape["Ld2"]], mlp_mult=shape["mlp_mult"], dtype=shape["dtype"],
+                  init_std=shape["init_std"], rope_theta=shape["rope_theta"], norm_eps=shape["norm_eps"])
+    B, T = toks.shape
+    n = wl["decode_tokens"] // shape["C1"]
+    bm = hal.Model(bshape, WEIGHT_SEED)
+    out = torch.empty(B, shape["C1"], dtype=torch.int32, device=toks.device)
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+    c = bm.prefill(toks, hal.MODE_HIER, n)
+    c.decode_step(hal.MODE_HIER, out)
+    torch.cuda.synchronize()
+    ev[0].record(stream)
+    for _ in range(n - 1):
+        c.decode_step(hal.MODE_HIER, out)
+    ev[1].record(stream)
+    torch.cuda.synchronize()
+    info, minfo = c.info(), bm.info()
+    c.free()
+    bm.free()
+    resident = minfo["resident_bytes"] + info["kv_bytes"]
+    return {"model": f"single-level block model (L = 1, blocks of {shape['C1']}), encoder "
+                     f"{bshape['enc_layers'][0]} + token decoder {bshape['dec_layers'][0]} layers, "
+                     f"d={bshape['d_model']}, {bshape['dtype']}",
+            "params_m": round(minfo["param_count"] / 1e6, 1),
+            "resident_gib": round(resident / 2 ** 30, 3), "kv_gib": round(info["kv_bytes"] / 2 ** 30, 3),
+            "graph_steps": info["graph_steps"], "tokens": B * (n - 1) * shape["C1"], "steps": n - 1,
+            "_decode_ms": ev[0].elapsed_time(ev[1])}
+
+
+def block_line(blk: dict, blk_ms: float, world: int, photon_tpm: float, van_line) -> dict:
+    """The block model's decode throughput (whole job), per GiB, and the TPM
+    ratios PHOTON / block and block / vanilla."""
+    tok_s = world * blk["tokens"] / (blk_ms / 1e3)
+    tpm = tok_s / world / blk["resident_gib"]
+    out = dict(blk, decode_tok_s=round(tok_s, 1), decode_ms_per_step=round(blk_ms / blk["steps"], 3),
+               tok_s_per_gib=round(tpm, 1), photon_over_block_tpm=round(photon_tpm / tpm, 2))
+    if van_line:
+        out["block_over_vanilla_tpm"] = round(tpm / van_line["tok_s_per_gib"], 1)
+    return out
 
 
 def measure_multi_query(model, toks, n_chunks: int, stream, N: int = 9, prefix=None,

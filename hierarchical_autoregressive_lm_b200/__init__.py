@@ -18,12 +18,13 @@ from typing import Optional
 __all__ = ["PhotonError", "Model", "Cache", "load_library", "LIB_PATH", "MODE_HIER",
            "MODE_REC", "STATE", "launch_count", "gemm", "gemm_rmsnorm", "attn_decode", "attn_decode_noalloc", "attn_decode_scratch_bytes", "debug_fail_alloc",
            "selftest_wait_timeout", "config_struct", "EXPORTED",
-           "AGG_VOTE", "AGG_BEST", "aggregate"]
+           "AGG_VOTE", "AGG_BEST", "aggregate", "ENC_RESTORE", "ENC_REGENERATE", "ENC_KEEP"]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libphoton.so")
 
 MODE_HIER, MODE_REC = 0, 1
 AGG_VOTE, AGG_BEST = 0, 1
+ENC_RESTORE, ENC_REGENERATE, ENC_KEEP = 0, 1, 2
 STATE = {"top_k": 0, "top_v": 1, "l1_k": 2, "l1_v": 3, "pending_o": 4, "a_hat": 5, "a": 6}
 _DTYPES = {"fp32": 0, "bf16": 1}
 _ERRORS = {-1: "PHOTON_ERR_ARG", -2: "PHOTON_ERR_OOM", -3: "PHOTON_ERR_CUDA",
@@ -40,7 +41,8 @@ EXPORTED = ("photon_init_weights", "photon_free_model", "photon_prefill",
             "photon_multi_query", "photon_vanilla_init",
             "photon_vanilla_prefill", "photon_vanilla_decode_step", "photon_vanilla_cache_info",
             "photon_vanilla_free_cache", "photon_launch_count", "photon_last_error",
-            "photon_debug_fail_alloc", "photon_selftest_wait_timeout", "photon_init_weights_levels")
+            "photon_debug_fail_alloc", "photon_selftest_wait_timeout", "photon_init_weights_levels",
+            "photon_model_set_encoder_residency")
 
 
 class PhotonError(RuntimeError):
@@ -142,6 +144,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "photon_attn_decode_noalloc": [I32, P, P, P, I32, I32, I32, I32, I32, I32, P, P, P],
         "photon_attn_decode_scratch_bytes": [I32, I32, I32, I32, I32, I32, I32, P],
         "photon_debug_fail_alloc": [I64],
+        "photon_model_set_encoder_residency": [P, I32],
         "photon_init_weights_levels": [ctypes.POINTER(photon_level_config), U64, ctypes.POINTER(P)],
         "photon_selftest_wait_timeout": [I64, P, P],
     }
@@ -255,6 +258,11 @@ class Model:
             self.C = self.C1 * self.C2
         self._h = h
         self.vocab, self.d_model = shape["vocab"], shape["d_model"]
+
+    def set_encoder_residency(self, policy: int) -> None:
+        """How released level-1 encoder weights come back (ENC_RESTORE from a pinned
+        host copy, ENC_REGENERATE from the seed) or ENC_KEEP (never released)."""
+        _check(load_library().photon_model_set_encoder_residency(self._h, int(policy)))
 
     @property
     def torch_dtype(self):

@@ -110,6 +110,8 @@ struct photon_model {
   // one event per stream that has enqueued work reading the level-1 encoder
   // weights since they were generated; their release waits on all of them
   std::vector<std::pair<cudaStream_t, cudaEvent_t>> enc_users;
+  int enc_policy = PHOTON_ENC_RESTORE;  // how released encoder weights come back
+  void* enc_host = nullptr;             // their pinned host copy (PHOTON_ENC_RESTORE)
 
   // any-L models (photon_init_weights_levels): per level l (index l - 1)
   // chunk size, encoder and decoder depth, and first tensor of each piece
@@ -290,10 +292,22 @@ static void generate_group(photon_model* m, int g, cudaStream_t s) {
 // (RecGen section: during RecGen decode the encoder hierarchy is never
 // called).  They are released after a RecGen prefill when no HierGen cache
 // is alive, and regenerated from the seed when needed again.
+// Residency of the level-1 encoder and Chunker_1 weights (explainer, RecGen
+// section: during RecGen decoding only the decoders (and, by R15, the top
+// encoder) need to stay on the device).  After a RecGen prefill they are
+// released unless a HierGen cache needs them; the next prefill brings them
+// back: by a host-to-device copy from a pinned host copy made at the first
+// release (PHOTON_ENC_RESTORE, the default, what a trained model would do),
+// by drawing them again from the seed (PHOTON_ENC_REGENERATE), or they are
+// never released (PHOTON_ENC_KEEP).
 static int ensure_encoder(photon_model* m, cudaStream_t s) {
   if (m->group_ptr[G_ENC1]) return PHOTON_OK;
   CK(pool_malloc((void**)&m->group_ptr[G_ENC1], m->group_bytes[G_ENC1], s));
-  generate_group(m, G_ENC1, s);
+  if (m->enc_policy == PHOTON_ENC_RESTORE && m->enc_host) {
+    CK(cudaMemcpyAsync(m->group_ptr[G_ENC1], m->enc_host, m->group_bytes[G_ENC1], cudaMemcpyHostToDevice, s));
+  } else {
+    generate_group(m, G_ENC1, s);
+  }
   CK(cudaGetLastError());
   return PHOTON_OK;
 }
@@ -312,7 +326,17 @@ static int note_encoder_use(photon_model* m, cudaStream_t s) {
 }
 // Stream-ordered release on `s`, after every user stream's last recorded use.
 static int release_encoder(photon_model* m, cudaStream_t s) {
-  if (!m->group_ptr[G_ENC1]) return PHOTON_OK;
+  if (!m->group_ptr[G_ENC1] || m->enc_policy == PHOTON_ENC_KEEP) return PHOTON_OK;
+  if (m->enc_policy == PHOTON_ENC_RESTORE && !m->enc_host) {
+    // the pinned host copy, made once (the weights never change)
+    if (cudaMallocHost(&m->enc_host, m->group_bytes[G_ENC1]) != cudaSuccess) {
+      cudaGetLastError();
+      m->enc_host = nullptr;
+      return fail(PHOTON_ERR_OOM, "pinned host memory for the encoder weights");
+    }
+    CK(cudaMemcpyAsync(m->enc_host, m->group_ptr[G_ENC1], m->group_bytes[G_ENC1], cudaMemcpyDeviceToHost, s));
+    CK(cudaStreamSynchronize(s));
+  }
   for (auto& u : m->enc_users) {
     CK(cudaStreamWaitEvent(s, u.second, 0));
     cudaEventDestroy(u.second);
@@ -917,9 +941,19 @@ int photon_free_model(photon_model* m) {
   }
   for (int g = 0; g < G_COUNT; ++g)
     if (m->group_ptr[g]) cudaFree(m->group_ptr[g]);
+  if (m->enc_host) cudaFreeHost(m->enc_host);
   delete m;
   cudaMemPool_t pool = nullptr;
   if (library_pool(&pool) == cudaSuccess) cudaMemPoolTrimTo(pool, 0);
+  return PHOTON_OK;
+}
+
+int photon_model_set_encoder_residency(photon_model* m, int32_t policy) {
+  g_err.clear();
+  if (!m) return fail(PHOTON_ERR_ARG, "model is NULL");
+  if (policy != PHOTON_ENC_RESTORE && policy != PHOTON_ENC_REGENERATE && policy != PHOTON_ENC_KEEP)
+    return fail(PHOTON_ERR_ARG, "unknown residency policy %d", policy);
+  m->enc_policy = policy;
   return PHOTON_OK;
 }
 

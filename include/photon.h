@@ -252,6 +252,20 @@ typedef struct photon_model_stats {
 
 PHOTON_API int photon_model_info(const photon_model* m, photon_model_stats* out);
 
+/* Residency of the level-1 encoder and Chunker_1 weights (explainer, RecGen
+ * section: only the decoders, and the top encoder that RecGen feeds, have to
+ * stay on the device while decoding).  A RecGen prefill releases them when
+ * no HierGen cache is alive; the next prefill or HierGen step needs them
+ * back:
+ *   PHOTON_ENC_RESTORE (default): host-to-device copy from a pinned host copy
+ *     the library makes at the first release (a trained model's weights
+ *     would come back this way);
+ *   PHOTON_ENC_REGENERATE: drawn again on the device from the seed;
+ *   PHOTON_ENC_KEEP: never released (more resident memory, no restore).
+ * Affects later prefills.  Errors: ERR_ARG. */
+enum { PHOTON_ENC_RESTORE = 0, PHOTON_ENC_REGENERATE = 1, PHOTON_ENC_KEEP = 2 };
+PHOTON_API int photon_model_set_encoder_residency(photon_model* m, int32_t policy);
+
 /* Copies parameter tensor `index` (generator order) into d_dst as stored:
  * the storage type for drawn tensors, fp32 for RMSNorm gains; out_bytes
  * receives the size.  Call with d_dst = NULL to query the size.  The level-1

@@ -55,6 +55,9 @@ class FakeCache:
     def step_hier(self, out):
         out.zero_()
 
+    def decode_step(self, mode, out, logits=None, force_tokens=None, force_a=None):
+        out.zero_()
+
     def set_sampling(self, T, seed=0, top_p=1.0):
         pass
 
@@ -77,7 +80,11 @@ class FakeModel:
         return FakeCache(self, tokens.shape[0], mode)
 
     def info(self):
-        return {"resident_bytes": 600 * 2 ** 20, "param_count": 384_000_000}
+        return {"resident_bytes": 600 * 2 ** 20, "param_count": 384_000_000, "encoder_bytes": 109 * 2 ** 20,
+                "encoder_resident": 0}
+
+    def set_encoder_residency(self, policy):
+        assert policy in (hal.ENC_RESTORE, hal.ENC_REGENERATE, hal.ENC_KEEP)
 
     def score(self, tokens, out=None, stream=None):
         return torch.zeros(tokens.shape[0], tokens.shape[1] - self.C)
