@@ -33,23 +33,24 @@ __device__ __forceinline__ const T* key_row(const AttnArgs& a, const T* own, con
   return own + (((long long)g * a.H + h) * a.cap + (pos - a.n_pre)) * DH;
 }
 
-// Decode attention: one CTA (2 warps) per (key chunk, head, group).  Warp w
-// streams half of the chunk's keys: each 16-byte slice of a key row goes to
+// Decode attention: one CTA of W warps (kDecWarps for caches of 192 keys or
+// more, else 2) per (key chunk, head, group).  Warp w streams 1/W of the
+// chunk's keys: each 16-byte slice of a key row goes to
 // one lane (TPK lanes per row, 32/TPK rows per warp-wide load).  Every lane
 // keeps a private ring of kDecStages stages in shared memory and fills it
 // with cp.async copies of its own slices, kDecStages-1 batches ahead of
 // the batch it is using; since a lane only reads back what it copied itself,
 // no barrier or warp synchronisation is needed until the end.  Each key
 // group keeps its own online-softmax state; the key groups are merged with
-// shuffles inside a warp and through shared memory across the two warps.
+// shuffles inside a warp and through shared memory across the warps.
 // With several chunks per (group, head), partials (acc, max, sum) are
 // merged in chunk order by k_attn_combine.
 // Decode-attention tiling (compile-time; -D overrides exist for tuning sweeps).
 #ifndef PHOTON_DEC_WARPS
-#define PHOTON_DEC_WARPS 8
+#define PHOTON_DEC_WARPS 4
 #endif
 #ifndef PHOTON_DEC_STAGES
-#define PHOTON_DEC_STAGES 4
+#define PHOTON_DEC_STAGES 3
 #endif
 #ifndef PHOTON_DEC_U
 #define PHOTON_DEC_U 2
@@ -76,7 +77,14 @@ __device__ __forceinline__ void cp_async_wait_group() {
 }
 
 template <typename T, int DH, int QMAX, int W>
-__global__ void __launch_bounds__(32 * W, (QMAX == 1 ? 24 : 8) / W)
+// Resident warps per SM the one-query kernel is compiled for: 28 = seven
+// 4-warp CTAs (56 registers, a 24 KB ring each), so the 1024 (sequence,
+// head) CTAs of the 600M-class batch-64 decode run as one wave on 148 SMs
+// (eight-warp CTAs fit three to an SM: 2.3 waves, the last one a third full).
+#ifndef PHOTON_DEC_RESIDENT_WARPS
+#define PHOTON_DEC_RESIDENT_WARPS 28
+#endif
+__global__ void __launch_bounds__(32 * W, (QMAX == 1 ? PHOTON_DEC_RESIDENT_WARPS : 8) / W)
     k_attn_decode(AttnArgs a, int chunk, int splits, float* __restrict__ part, int* err) {
   constexpr int SPL = kDecSPL;
   constexpr int VEC = 16 / sizeof(T);          // elements per slice
