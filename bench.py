@@ -117,7 +117,8 @@ def run_gpu(args) -> None:
     import torch.distributed as dist
 
     import hierarchical_autoregressive_lm_b200 as hal
-    from hierarchical_autoregressive_lm_b200.dist import job_throughput, max_over_ranks, rank_rows
+    from hierarchical_autoregressive_lm_b200.dist import (broadcast_cache_state, job_throughput, max_over_ranks,
+                                                          rank_rows)
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -164,21 +165,34 @@ def run_gpu(args) -> None:
     step_out = torch.empty(B, C, dtype=torch.int32, device=dev)
     stream = torch.cuda.current_stream()
 
-    # multi-query serving (c5): every rank prefills the shared context once
-    # (HierGen mode keeps its level-1 cache for the queries' prefill); each
-    # step's queries are prefilled after it and read its top cache in place
+    # multi-query serving (c5): the shared context is prefilled once (HierGen
+    # mode keeps its level-1 cache for the queries' prefill); each step's
+    # queries are prefilled after it and read its top cache in place.  With
+    # several ranks only rank 0 prefills it: the others build a shell cache
+    # and receive its state buffers in one broadcast before any timing.
     prefix_len = wl.get("prefix_len", 0)
-    pre_cache, prefix_ms = None, 0.0
+    pre_cache, prefix_ms, pre_bcast = None, 0.0, None
     if prefix_len:
         pre_dev = torch.from_numpy(np.ascontiguousarray(prefix_tokens(args.workload))).to(dev)
         pe = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
-        model.prefill(pre_dev, hal.MODE_HIER, 0).free()          # untimed warm-up
-        torch.cuda.synchronize()
-        pe[0].record(stream)
-        pre_cache = model.prefill(pre_dev, hal.MODE_HIER, 0)
-        pe[1].record(stream)
-        torch.cuda.synchronize()
-        prefix_ms = pe[0].elapsed_time(pe[1])
+        if rank == 0:
+            model.prefill(pre_dev, hal.MODE_HIER, 0).free()          # untimed warm-up
+            torch.cuda.synchronize()
+            pe[0].record(stream)
+            pre_cache = model.prefill(pre_dev, hal.MODE_HIER, 0)
+            pe[1].record(stream)
+            torch.cuda.synchronize()
+            prefix_ms = pe[0].elapsed_time(pe[1])
+        else:
+            pre_cache = model.prefill_shell(pre_dev.shape[0], pre_dev.shape[1], hal.MODE_HIER, 0)
+        if world > 1:
+            torch.cuda.synchronize()
+            pe[0].record(stream)
+            nbytes = broadcast_cache_state(pre_cache.state_buffers(), src=0)
+            pe[1].record(stream)
+            torch.cuda.synchronize()
+            pre_bcast = {"bytes": nbytes, "ms": round(max_over_ranks([pe[0].elapsed_time(pe[1])], dev)[0], 3),
+                         "src_rank": 0}
 
     def one_step(ev=None, mark=False):
         # mark: NVTX ranges around the prefill and one middle decode chunk,
@@ -408,6 +422,7 @@ def run_gpu(args) -> None:
         "prefill_tok_s": round(world * B * T * args.steps / (prefill_ms / 1e3), 1),
         "prefill_ms_steps": [round(e[0].elapsed_time(e[1]), 3) for e in evs],
         "prefix_prefill_ms": round(prefix_ms, 3) if prefix_len else None,
+        "prefix_broadcast": pre_bcast,
         "job_tok_s": round(dec_tokens / (total_ms / 1e3), 1),
         "tpm": {"tok_s_per_gib": round(value / world / gib, 1), "resident_gib": round(gib, 4),
                 "weights_gib": round(minfo["resident_bytes"] / 2 ** 30, 4),

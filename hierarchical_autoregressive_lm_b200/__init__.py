@@ -42,7 +42,7 @@ EXPORTED = ("photon_init_weights", "photon_free_model", "photon_prefill",
             "photon_vanilla_prefill", "photon_vanilla_decode_step", "photon_vanilla_cache_info",
             "photon_vanilla_free_cache", "photon_launch_count", "photon_last_error",
             "photon_debug_fail_alloc", "photon_selftest_wait_timeout", "photon_init_weights_levels",
-            "photon_model_set_encoder_residency")
+            "photon_model_set_encoder_residency", "photon_prefill_shell", "photon_cache_state_buffer")
 
 
 class PhotonError(RuntimeError):
@@ -117,6 +117,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "photon_init_weights": [ctypes.POINTER(photon_config), U64, ctypes.POINTER(P)],
         "photon_free_model": [P],
         "photon_prefill": [P, P, P, I32, I32, I32, I32, P, ctypes.POINTER(P)],
+        "photon_prefill_shell": [P, P, I32, I32, I32, I32, P, ctypes.POINTER(P)],
+        "photon_cache_state_buffer": [P, I32, ctypes.POINTER(P), ctypes.POINTER(SZ)],
         "photon_decode_step_hier": [P, P, P, P, P],
         "photon_decode_step_rec": [P, P, P, P, P],
         "photon_decode_step_ex": [P, P, I32, P, P, P, P, P],
@@ -327,10 +329,29 @@ class Model:
                                              _stream(stream), ctypes.byref(h)))
         return Cache(self, h, B, prefix)
 
+    def prefill_shell(self, B: int, T: int, mode: int, max_new_chunks: int, prefix: "Cache" = None,
+                      stream=None) -> "Cache":
+        """A cache laid out as prefill(tokens[B, T], ...) would make it, its state
+        left for the caller to fill (see state_buffers)."""
+        h = ctypes.c_void_p()
+        _check(load_library().photon_prefill_shell(self._h, None if prefix is None else prefix._h,
+                                                   B, T, mode, max_new_chunks, _stream(stream),
+                                                   ctypes.byref(h)))
+        return Cache(self, h, B, prefix)
+
     def free(self) -> None:
         if self._h:
             _check(load_library().photon_free_model(self._h))
             self._h = None
+
+
+class _DeviceBytes:
+    """A device byte range in the CUDA array interface, so torch can view it
+    without a copy."""
+
+    def __init__(self, ptr: int, n: int):
+        self.__cuda_array_interface__ = {"shape": (n,), "typestr": "|u1", "data": (ptr, False),
+                                         "version": 3, "strides": None, "stream": None}
 
 
 class Cache:
@@ -402,6 +423,20 @@ class Cache:
         _check(L.photon_export_state(self._h, STATE[which], layer, _ptr(buf), n.value, None,
                                      _stream(stream)))
         return buf[:n.value]
+
+    def state_buffers(self) -> list:
+        """(name, uint8 CUDA tensor) views of the whole state buffers a prefill
+        writes, in a fixed order; the memory stays owned by the cache.
+        Buffers a RecGen prefill discarded are left out."""
+        import torch
+        L = load_library()
+        out = []
+        for name in ("top_k", "top_v", "l1_k", "l1_v", "pending_o"):
+            ptr, n = ctypes.c_void_p(), ctypes.c_size_t()
+            _check(L.photon_cache_state_buffer(self._h, STATE[name], ctypes.byref(ptr), ctypes.byref(n)))
+            if n.value:
+                out.append((name, torch.as_tensor(_DeviceBytes(ptr.value, n.value), device="cuda")))
+        return out
 
     def free(self) -> None:
         if self._h:

@@ -995,14 +995,17 @@ int photon_export_weight(photon_model* m, int32_t index, void* d_dst, size_t dst
 
 // o_all (nullable): also the final-normed top output of every own position,
 // [B * T/C, d] in the storage type (teacher-forced scoring reads them all).
+// shell: allocate and set up the cache as a prefill of T tokens would, but
+// compute nothing (its state is then filled by the caller, e.g. a broadcast
+// of another rank's prefilled cache).
 static int prefill_impl(photon_model* m, const photon_cache* prefix, const int32_t* d_tokens, int32_t B,
                         int32_t T, int32_t mode, int32_t max_new_chunks, void* stream, photon_cache** out,
-                        void* o_all) {
+                        void* o_all, bool shell = false) {
   g_err.clear();
   if (!m || !out) return fail(PHOTON_ERR_ARG, "NULL model or out");
   *out = nullptr;
   if (m->vanilla) return fail(PHOTON_ERR_ARG, "a vanilla baseline model takes the photon_vanilla_* calls");
-  if (!d_tokens) return fail(PHOTON_ERR_ARG, "tokens pointer is NULL");
+  if (!d_tokens && !shell) return fail(PHOTON_ERR_ARG, "tokens pointer is NULL");
   if (B <= 0) return fail(PHOTON_ERR_ARG, "batch must be positive");
   // the attention kernels index (sequence, sub-chunk) groups in a grid
   // dimension of at most 65535
@@ -1171,96 +1174,98 @@ static int prefill_impl(photon_model* m, const photon_cache* prefix, const int32
       (c->tk_bar && cudaMemsetAsync(c->tk_bar, 0, 64, s) != cudaSuccess))
     return bail(PHOTON_ERR_CUDA);
 
-  // prefill workspace (released at the end of this call)
-  std::vector<void*> tmp;
-  size_t tmp_bytes = 0;
-  Allocator at{s, &tmp, &tmp_bytes};
-  const long long rows1 = rows0 / C1, rows2 = rows0 / C;
-  void* emb = at.get<void>((size_t)rows0 * d * es);
-  float* x = at.get<float>((size_t)rows1 * d * 4);
-  void* xn = at.get<void>((size_t)rows1 * d * es);
-  void* q = at.get<void>((size_t)rows1 * d * es);
-  void* att = at.get<void>((size_t)rows1 * d * es);
-  void* hid = at.get<void>((size_t)rows1 * m->f * es);
-  size_t pgw = std::max(block_ws_need(m, (int)rows1), block_ws_need(m, (int)rows2));
-  pgw = std::max(pgw, gemm_ws_need(m, (int)rows1, d, C1 * d));
-  pgw = std::max(pgw, gemm_ws_need(m, (int)rows2, d, C2 * d));
-  float* pws = at.get<float>(pgw);
-  size_t ppb = 0;
-  float* ppw = nullptr;
-  if (prefix) {  // the level-1 stack has the most query rows
-    AttnArgs pa;
-    pa.G = B;
-    pa.q_len = N1_own;
-    pa.H = m->H;
-    pa.dh = m->dh;
-    ppb = attn_prefix_split_bytes(pa);
-    ppw = at.get<float>(ppb);
-  }
-  if (at.err != cudaSuccess) {
+  if (!shell) {
+    // prefill workspace (released at the end of this call)
+    std::vector<void*> tmp;
+    size_t tmp_bytes = 0;
+    Allocator at{s, &tmp, &tmp_bytes};
+    const long long rows1 = rows0 / C1, rows2 = rows0 / C;
+    void* emb = at.get<void>((size_t)rows0 * d * es);
+    float* x = at.get<float>((size_t)rows1 * d * 4);
+    void* xn = at.get<void>((size_t)rows1 * d * es);
+    void* q = at.get<void>((size_t)rows1 * d * es);
+    void* att = at.get<void>((size_t)rows1 * d * es);
+    void* hid = at.get<void>((size_t)rows1 * m->f * es);
+    size_t pgw = std::max(block_ws_need(m, (int)rows1), block_ws_need(m, (int)rows2));
+    pgw = std::max(pgw, gemm_ws_need(m, (int)rows1, d, C1 * d));
+    pgw = std::max(pgw, gemm_ws_need(m, (int)rows2, d, C2 * d));
+    float* pws = at.get<float>(pgw);
+    size_t ppb = 0;
+    float* ppw = nullptr;
+    if (prefix) {  // the level-1 stack has the most query rows
+      AttnArgs pa;
+      pa.G = B;
+      pa.q_len = N1_own;
+      pa.H = m->H;
+      pa.dh = m->dh;
+      ppb = attn_prefix_split_bytes(pa);
+      ppw = at.get<float>(ppb);
+    }
+    if (at.err != cudaSuccess) {
+      free_list(tmp, s);
+      return bail(PHOTON_ERR_OOM);
+    }
+    Bufs pb{xn, q, att, hid, c->rope, pws, pgw, c->gemm_cnt, nullptr, 0, c->d_err};
+    pb.pre_ws = ppw;
+    pb.pre_ws_bytes = ppb;
+
+    // a1: embedding; a2: Chunker_1 (concatenate C1 states, linear C1*d -> d)
+    launch_embed(m->dt, d_tokens, m->ptr(m->i_embed), emb, (int)rows0, d, m->V, c->d_err, s);
+    gemm(m, pb, emb, (long long)C1 * d, m->ptr(m->i_ch1), (long long)C1 * d, (int)rows1, d, C1 * d,
+         epi(EPI_STORE_F32, x, d), s);
+    // a3: level-1 encoder over T/C1 positions per sequence, writing the level-1 KV
+    StackRun r1;
+    r1.G = B;
+    r1.q_len = N1_own;
+    r1.p0 = c->n1_pre;
+    r1.kv_off = c->n1_pre;
+    r1.kc = c->l1_k;
+    r1.vc = c->l1_v;
+    r1.layer_bytes = c->l1_layer;
+    r1.cap = c->N1cap;
+    if (prefix) {
+      r1.kp = prefix->l1_k;
+      r1.vp = prefix->l1_v;
+      r1.pre_layer_bytes = prefix->l1_layer;
+      r1.cap_pre = prefix->N1cap;
+      r1.n_pre = c->n1_pre;
+    }
+    run_stack(m, m->i_enc1, m->L1, x, r1, pb, s);
+    launch_rmsnorm(m->dt, x, (const float*)m->ptr(m->i_enc1_g), xn, (int)rows1, d, 1, 0,
+                   m->cfg.norm_eps, s);
+    // a4: Chunker_2 on the level-1 states (x is reused for the top stream)
+    gemm(m, pb, xn, (long long)C2 * d, m->ptr(m->i_ch2), (long long)C2 * d, (int)rows2, d, C2 * d,
+         epi(EPI_STORE_F32, x, d), s);
+    // a5: top encoder over T/C positions, writing the top KV
+    StackRun rt;
+    rt.G = B;
+    rt.q_len = N_own;
+    rt.p0 = c->n_pre;
+    rt.kv_off = c->n_pre;
+    rt.kc = c->top_k;
+    rt.vc = c->top_v;
+    rt.layer_bytes = c->top_layer;
+    rt.cap = c->Ncap;
+    if (prefix) {
+      rt.kp = prefix->top_k;
+      rt.vp = prefix->top_v;
+      rt.pre_layer_bytes = prefix->top_layer;
+      rt.cap_pre = prefix->Ncap;
+      rt.n_pre = c->n_pre;
+    }
+    run_stack(m, m->i_top, m->Ltop, x, rt, pb, s);
+    // pending output: final norm of the last top position of each sequence
+    launch_rmsnorm(m->dt, x, (const float*)m->ptr(m->i_top_g), c->o, B, d, N_own, N_own - 1,
+                   m->cfg.norm_eps, s);
+    if (o_all)
+      launch_rmsnorm(m->dt, x, (const float*)m->ptr(m->i_top_g), o_all, B * N_own, d, 1, 0, m->cfg.norm_eps, s);
+    cudaError_t le = cudaGetLastError();
     free_list(tmp, s);
-    return bail(PHOTON_ERR_OOM);
-  }
-  Bufs pb{xn, q, att, hid, c->rope, pws, pgw, c->gemm_cnt, nullptr, 0, c->d_err};
-  pb.pre_ws = ppw;
-  pb.pre_ws_bytes = ppb;
+    if (le != cudaSuccess) {
+      return bail(fail(PHOTON_ERR_CUDA, "prefill launch failed: %s", cudaGetErrorString(le)));
+    }
 
-  // a1: embedding; a2: Chunker_1 (concatenate C1 states, linear C1*d -> d)
-  launch_embed(m->dt, d_tokens, m->ptr(m->i_embed), emb, (int)rows0, d, m->V, c->d_err, s);
-  gemm(m, pb, emb, (long long)C1 * d, m->ptr(m->i_ch1), (long long)C1 * d, (int)rows1, d, C1 * d,
-       epi(EPI_STORE_F32, x, d), s);
-  // a3: level-1 encoder over T/C1 positions per sequence, writing the level-1 KV
-  StackRun r1;
-  r1.G = B;
-  r1.q_len = N1_own;
-  r1.p0 = c->n1_pre;
-  r1.kv_off = c->n1_pre;
-  r1.kc = c->l1_k;
-  r1.vc = c->l1_v;
-  r1.layer_bytes = c->l1_layer;
-  r1.cap = c->N1cap;
-  if (prefix) {
-    r1.kp = prefix->l1_k;
-    r1.vp = prefix->l1_v;
-    r1.pre_layer_bytes = prefix->l1_layer;
-    r1.cap_pre = prefix->N1cap;
-    r1.n_pre = c->n1_pre;
   }
-  run_stack(m, m->i_enc1, m->L1, x, r1, pb, s);
-  launch_rmsnorm(m->dt, x, (const float*)m->ptr(m->i_enc1_g), xn, (int)rows1, d, 1, 0,
-                 m->cfg.norm_eps, s);
-  // a4: Chunker_2 on the level-1 states (x is reused for the top stream)
-  gemm(m, pb, xn, (long long)C2 * d, m->ptr(m->i_ch2), (long long)C2 * d, (int)rows2, d, C2 * d,
-       epi(EPI_STORE_F32, x, d), s);
-  // a5: top encoder over T/C positions, writing the top KV
-  StackRun rt;
-  rt.G = B;
-  rt.q_len = N_own;
-  rt.p0 = c->n_pre;
-  rt.kv_off = c->n_pre;
-  rt.kc = c->top_k;
-  rt.vc = c->top_v;
-  rt.layer_bytes = c->top_layer;
-  rt.cap = c->Ncap;
-  if (prefix) {
-    rt.kp = prefix->top_k;
-    rt.vp = prefix->top_v;
-    rt.pre_layer_bytes = prefix->top_layer;
-    rt.cap_pre = prefix->Ncap;
-    rt.n_pre = c->n_pre;
-  }
-  run_stack(m, m->i_top, m->Ltop, x, rt, pb, s);
-  // pending output: final norm of the last top position of each sequence
-  launch_rmsnorm(m->dt, x, (const float*)m->ptr(m->i_top_g), c->o, B, d, N_own, N_own - 1,
-                 m->cfg.norm_eps, s);
-  if (o_all)
-    launch_rmsnorm(m->dt, x, (const float*)m->ptr(m->i_top_g), o_all, B * N_own, d, 1, 0, m->cfg.norm_eps, s);
-  cudaError_t le = cudaGetLastError();
-  free_list(tmp, s);
-  if (le != cudaSuccess) {
-    return bail(fail(PHOTON_ERR_CUDA, "prefill launch failed: %s", cudaGetErrorString(le)));
-  }
-
   c->N = c->n_pre + N_own;
   c->N1 = c->n1_pre + N1_own;
   // a6: RecGen keeps only the top-level KV (RecGen section)
@@ -2165,6 +2170,46 @@ int photon_prefill(photon_model* m, const photon_cache* prefix, const int32_t* d
     return gen_prefill(m, d_tokens, B, T, mode, max_new_chunks, (cudaStream_t)stream, out);
   }
   return prefill_impl(m, prefix, d_tokens, B, T, mode, max_new_chunks, stream, out, nullptr);
+}
+
+int photon_prefill_shell(photon_model* m, const photon_cache* prefix, int32_t B, int32_t T, int32_t mode,
+                         int32_t max_new_chunks, void* stream, photon_cache** out) {
+  if (m && m->general) {
+    g_err.clear();
+    if (out) *out = nullptr;
+    return fail(PHOTON_ERR_ARG, "shell caches are built for two-level models only");
+  }
+  return prefill_impl(m, prefix, nullptr, B, T, mode, max_new_chunks, stream, out, nullptr, true);
+}
+
+int photon_cache_state_buffer(photon_cache* c, int32_t which, void** d_ptr, size_t* bytes) {
+  g_err.clear();
+  if (!c || !d_ptr || !bytes) return fail(PHOTON_ERR_ARG, "NULL cache or output pointer");
+  photon_model* m = c->m;
+  if (m->general) return fail(PHOTON_ERR_ARG, "state buffers are listed for two-level models only");
+  *d_ptr = nullptr;
+  *bytes = 0;
+  switch (which) {
+    case PHOTON_STATE_TOP_K:
+    case PHOTON_STATE_TOP_V:
+      *d_ptr = which == PHOTON_STATE_TOP_K ? c->top_k : c->top_v;
+      *bytes = c->top_layer * m->Ltop;
+      break;
+    case PHOTON_STATE_L1_K:
+    case PHOTON_STATE_L1_V:
+      if (c->l1_k) {
+        *d_ptr = which == PHOTON_STATE_L1_K ? c->l1_k : c->l1_v;
+        *bytes = c->l1_layer * m->L1;
+      }
+      break;
+    case PHOTON_STATE_PENDING_O:
+      *d_ptr = c->o;
+      *bytes = (size_t)c->B * m->d * m->es;
+      break;
+    default:
+      return fail(PHOTON_ERR_ARG, "state %d is not a prefill state buffer", which);
+  }
+  return PHOTON_OK;
 }
 
 int photon_decode_step_ex(photon_model* m, photon_cache* c, int32_t mode, int32_t* d_out_tokens,

@@ -4,9 +4,12 @@ Sequences are independent at every level of the hierarchy, so the batch is
 split over ranks and every rank decodes its own sequences with its own
 replica of the weights and its own caches: no collective runs on the data
 path.  What remains for the host is (1) deciding which prompts a rank owns,
-(2) timing the job as the slowest rank, and (3) turning per-rank counts into
-whole-job throughput.  These helpers hold that logic so it can be tested on
-CPU with the gloo backend.
+(2) timing the job as the slowest rank, (3) turning per-rank counts into
+whole-job throughput, and (4) for multi-query serving over one shared
+context, handing the prefilled prefix from the rank that computed it to the
+others once, before decoding (a broadcast of its state buffers, which is
+NVLink traffic under NCCL).  These helpers hold that logic so it can be
+tested on CPU with the gloo backend.
 """
 from __future__ import annotations
 
@@ -39,3 +42,31 @@ def job_throughput(units_per_rank: int, world: int, max_ms: float) -> float:
     if max_ms <= 0:
         raise ValueError("elapsed time must be positive")
     return units_per_rank * world / (max_ms / 1e3)
+
+
+def broadcast_cache_state(buffers: list, src: int = 0, group=None) -> int:
+    """Broadcast a cache's state buffers from rank `src` to every rank, in
+    place.  `buffers` is Cache.state_buffers() (a list of (name, tensor)):
+    on `src` the prefilled cache, elsewhere a shell cache made with the
+    same model, batch, length, mode and capacity.  All ranks first agree on
+    the names and sizes (a mismatch raises ValueError on every rank, before
+    any data moves), then broadcast each buffer in list order.  Returns the
+    bytes each rank received (or sent).  The caller orders the buffers'
+    producers before this call and their consumers after it (on the GPU: a
+    device synchronisation on both sides)."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size(group) == 1:
+        return 0
+    layout = [(str(n), int(t.numel()) * t.element_size()) for n, t in buffers]
+    every = [None] * dist.get_world_size(group)
+    dist.all_gather_object(every, layout, group=group)
+    if any(other != every[0] for other in every):
+        raise ValueError(f"cache state layouts differ across ranks: {every}")
+    total = 0
+    for _, t in buffers:
+        if not t.is_contiguous():
+            raise ValueError("state buffers must be contiguous")
+        dist.broadcast(t, src=src, group=group)
+        total += int(t.numel()) * t.element_size()
+    return total

@@ -284,6 +284,32 @@ enum {
   PHOTON_STATE_A = 6        /* [B*C2][d_model] last HierGen step's level-1 encoder states */
 };
 
+/* Data-parallel serving of a shared prefix (multi-query serving over one
+ * long context, the explainer's quality section): one rank prefills the
+ * prefix, the others receive its state instead of recomputing it.
+ *
+ * photon_prefill_shell allocates and sets up a cache exactly as
+ * photon_prefill(m, prefix, tokens, B, T, mode, max_new_chunks) would,
+ * positions included, but runs no kernel on its state: the top and level-1
+ * KV and the pending top output hold whatever the allocator returned until
+ * the caller fills them (e.g. with a broadcast of another rank's prefilled
+ * cache of the same model, B, T, mode and max_new_chunks).  Errors as
+ * photon_prefill; ERR_ARG for a model of other than two levels.
+ *
+ * photon_cache_state_buffer returns the device address and size in bytes
+ * of one whole state buffer a prefill writes, with every layer and the
+ * unused capacity included: which = PHOTON_STATE_TOP_K / TOP_V ([Ltop][B]
+ * [H][Ncap][head_dim]), L1_K / L1_V ([L1][B][H][N1cap][head_dim]; NULL and
+ * 0 once a RecGen prefill discarded them) or PENDING_O ([B][d_model]); all
+ * of the storage type.  Two caches built by the same calls on the same
+ * model have buffers of equal sizes, so copying each buffer from one to
+ * the other makes the second cache equal to the first.  The memory stays
+ * owned by the cache; the caller must order its writes after the
+ * cache's stream.  Errors: ERR_ARG (NULL pointers, another state). */
+PHOTON_API int photon_prefill_shell(photon_model* m, const photon_cache* prefix, int32_t B, int32_t T,
+                         int32_t mode, int32_t max_new_chunks, void* stream, photon_cache** out);
+PHOTON_API int photon_cache_state_buffer(photon_cache* c, int32_t which, void** d_ptr, size_t* bytes);
+
 /* Copies a piece of cache state (storage type) into d_dst, compacted to
  * the entries in use.  Call with d_dst = NULL to query the size.
  * Errors: ERR_ARG (unknown state, layer out of range, discarded level-1 KV,

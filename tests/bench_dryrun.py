@@ -41,9 +41,20 @@ class FakeEvent:
         return max(0.5, other.t - self.t)
 
 
+def _pattern(n):
+    return (torch.arange(n, dtype=torch.int64) * 7 % 251).to(torch.uint8)
+
+
 class FakeCache:
-    def __init__(self, model, B, mode):
+    # a prefilled cache's state buffers hold a pattern, a shell's hold zeros
+    SIZES = (("top_k", 4096), ("top_v", 4096), ("l1_k", 8192), ("l1_v", 8192), ("pending_o", 64))
+
+    def __init__(self, model, B, mode, shell=False):
         self.model, self.B, self.mode = model, B, mode
+        self.bufs = [(n, torch.zeros(k, dtype=torch.uint8) if shell else _pattern(k)) for n, k in self.SIZES]
+
+    def state_buffers(self):
+        return self.bufs
 
     def decode_rec_chunks(self, n, out):
         assert out.dtype == torch.int32 and out.numel() >= self.B * n * self.model.C
@@ -77,7 +88,13 @@ class FakeModel:
         self.vocab, self.d_model = shape["vocab"], shape["d_model"]
 
     def prefill(self, tokens, mode, max_new, prefix=None, stream=None):
+        if prefix is not None:   # a shared prefix is complete before any query reads it
+            for n, t in prefix.state_buffers():
+                assert torch.equal(t, _pattern(t.numel())), n
         return FakeCache(self, tokens.shape[0], mode)
+
+    def prefill_shell(self, B, T, mode, max_new, prefix=None, stream=None):
+        return FakeCache(self, B, mode, shell=True)
 
     def info(self):
         return {"resident_bytes": 600 * 2 ** 20, "param_count": 384_000_000, "encoder_bytes": 109 * 2 ** 20,

@@ -41,8 +41,7 @@ def test_bench_line_survives_a_library_error(mode, workload):
     assert sr["peak_batch"]["sequences"] > 0 and sr["peaks"]["source"] in ("measured", "fallback")
 
 
-def test_bench_line_with_two_ranks():
-    # torchrun with two gloo ranks: max over ranks, whole-job throughput, one line from rank 0
+def _two_ranks(workload):
     import socket
     s = socket.socket()
     s.bind(("127.0.0.1", 0))
@@ -50,13 +49,28 @@ def test_bench_line_with_two_ranks():
     s.close()
     cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes", "1", "--nproc-per-node", "2",
            "--master-addr", "127.0.0.1", "--master-port", str(port),
-           os.path.join(HERE, "bench_dryrun.py"), "ok", "c2"]
+           os.path.join(HERE, "bench_dryrun.py"), "ok", workload]
     r = subprocess.run(cmd, capture_output=True, text=True, timeout=300)
     assert r.returncode == 0, r.stderr[-2000:]
     lines = [l for l in r.stdout.splitlines() if l.startswith("{")]
     assert len(lines) == 1
-    two = json.loads(lines[0])
+    return json.loads(lines[0])
+
+
+def test_bench_line_with_two_ranks():
+    # torchrun with two gloo ranks: max over ranks, whole-job throughput, one line from rank 0
+    two = _two_ranks("c2")
     one = _line("ok", "c2")
     assert two["n_gpus"] == 2 and two["config"]["parallelism"] == "dp2"
     assert abs(two["value"] / one["value"] - 2.0) < 1e-9            # the same per-rank work on each rank
     assert two["multi_query"]["vote"]["answers_per_s"] == 2 * one["multi_query"]["vote"]["answers_per_s"]
+
+
+def test_shared_prefix_is_prefilled_once_and_broadcast():
+    # c5 on two ranks: rank 0 prefills the shared context, rank 1 builds a
+    # shell and receives its state buffers before any query is prefilled
+    # (the fake model asserts that); one rank broadcasts nothing
+    two = _two_ranks("c5")
+    assert two["prefix_broadcast"]["bytes"] == 4096 * 2 + 8192 * 2 + 64
+    assert two["prefix_broadcast"]["src_rank"] == 0 and two["prefix_prefill_ms"] > 0
+    assert _line("ok", "c5")["prefix_broadcast"] is None
