@@ -16,7 +16,7 @@ import os
 from typing import Optional
 
 __all__ = ["PhotonError", "Model", "Cache", "load_library", "LIB_PATH", "MODE_HIER",
-           "MODE_REC", "STATE", "launch_count", "gemm", "gemm_rmsnorm", "attn_decode", "attn_decode_noalloc", "attn_decode_scratch_bytes", "debug_fail_alloc",
+           "MODE_REC", "STATE", "launch_count", "gemm", "gemm_rmsnorm", "attn_decode", "attn_decode_noalloc", "attn_prefill", "attn_decode_scratch_bytes", "debug_fail_alloc",
            "selftest_wait_timeout", "config_struct", "EXPORTED",
            "AGG_VOTE", "AGG_BEST", "aggregate", "ENC_RESTORE", "ENC_REGENERATE", "ENC_KEEP"]
 
@@ -42,7 +42,8 @@ EXPORTED = ("photon_init_weights", "photon_free_model", "photon_prefill",
             "photon_vanilla_prefill", "photon_vanilla_decode_step", "photon_vanilla_cache_info",
             "photon_vanilla_free_cache", "photon_launch_count", "photon_last_error",
             "photon_debug_fail_alloc", "photon_selftest_wait_timeout", "photon_init_weights_levels",
-            "photon_model_set_encoder_residency", "photon_prefill_shell", "photon_cache_state_buffer")
+            "photon_model_set_encoder_residency", "photon_prefill_shell", "photon_cache_state_buffer",
+            "photon_attn_prefill")
 
 
 class PhotonError(RuntimeError):
@@ -144,6 +145,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "photon_gemm_rmsnorm": [P, I64, P, ctypes.c_float, P, I64, I32, I32, I32, P, I64, P],
         "photon_attn_decode": [I32, P, P, P, I32, I32, I32, I32, I32, I32, P, P, P],
         "photon_attn_decode_noalloc": [I32, P, P, P, I32, I32, I32, I32, I32, I32, P, P, P],
+        "photon_attn_prefill": [I32, P, P, P, P, P, I32, I32, I32, I32, I32, I32, I32, I32, I32, P, P, P],
         "photon_attn_decode_scratch_bytes": [I32, I32, I32, I32, I32, I32, I32, P],
         "photon_debug_fail_alloc": [I64],
         "photon_model_set_encoder_residency": [P, I32],
@@ -604,6 +606,24 @@ def attn_decode(q, k, v, q_len: int, p0: int, out, stream=None, err=None) -> Non
     dt, G, H, cap, dh = _attn_bufs(q, k, v, q_len, out, err)
     _check(load_library().photon_attn_decode(dt, _ptr(q), _ptr(k), _ptr(v), G, H, dh, cap, q_len,
                                              p0, _ptr(out), _ptr(err), _stream(stream)))
+
+
+def attn_prefill(q, k, v, q_len: int, p0: int, out, kp=None, vp=None, n_pre: int = 0, path: int = 0,
+                 stream=None, err=None) -> None:
+    """Causal prefill attention: k, v [G, H, cap, dh]; optional shared prefix kp, vp
+    [H, cap_pre, dh] holding positions 0..n_pre-1; q, out [G*q_len, H*dh].
+    path: 0 library's choice, 1 CUDA cores, 2 mma.sync, 3 tcgen05."""
+    dt, G, H, cap, dh = _attn_bufs(q, k, v, q_len, out, err)
+    cap_pre = 0
+    if n_pre > 0:
+        if kp is None or vp is None or kp.dim() != 3:
+            raise ValueError("kp, vp: expected [H, cap_pre, head_dim]")
+        cap_pre = kp.shape[1]
+        _need(kp, q.dtype, H * cap_pre * dh, "kp")
+        _need(vp, q.dtype, H * cap_pre * dh, "vp")
+    _check(load_library().photon_attn_prefill(dt, _ptr(q), _ptr(k), _ptr(v), _ptr(kp), _ptr(vp), G, H, dh, cap,
+                                              q_len, p0, cap_pre, n_pre, path, _ptr(out), _ptr(err),
+                                              _stream(stream)))
 
 
 def attn_decode_scratch_bytes(dtype_code: int, G: int, H: int, head_dim: int, cap: int, q_len: int,

@@ -1191,41 +1191,80 @@ size_t attn_prefix_split_bytes(const AttnArgs& a) {
   return (size_t)a.G * a.q_len * a.H * (a.dh + 2) * sizeof(float);
 }
 
-bool launch_attn_prefix_split(int dt, const AttnArgs& a, float* part, size_t part_bytes, cudaStream_t s) {
+bool launch_attn_prefix_split(int dt, const AttnArgs& a, float* part, size_t part_bytes, int* err,
+                              cudaStream_t s) {
   if (a.G <= 0 || a.q_len <= 0) return true;
   if (!(dt == DT_BF16 && a.dh == 64 && a.Kp != nullptr && a.n_pre > 0 && a.q_ld % 8 == 0 &&
         a.o_ld % 2 == 0 && !tc_attn_disabled() && part != nullptr && part_bytes >= attn_prefix_split_bytes(a)))
     return false;
+  // each pass on the tcgen05 kernel when its query space fills 128-row tiles
   const long long rows = (long long)a.G * a.q_len;
-  launch_kernel(k_attn_prefill_mma<SEG_PREFIX>, dim3((unsigned)((rows + 63) / 64), a.H, 1), 128, 0, s, a, part);
-  launch_kernel(k_attn_prefill_mma<SEG_OWN>, dim3((a.q_len + 63) / 64, a.H, a.G), 128, 0, s, a, part);
+  if (!launch_attn_prefix_tc(a, part, err, s))
+    launch_kernel(k_attn_prefill_mma<SEG_PREFIX>, dim3((unsigned)((rows + 63) / 64), a.H, 1), 128, 0, s, a, part);
+  if (!launch_attn_own_tc(a, part, err, s))
+    launch_kernel(k_attn_prefill_mma<SEG_OWN>, dim3((a.q_len + 63) / 64, a.H, a.G), 128, 0, s, a, part);
   return true;
 }
 
-void launch_attn_prefill(int dt, const AttnArgs& a, cudaStream_t s) {
+void launch_attn_prefill(int dt, const AttnArgs& a, int* err, cudaStream_t s) {
   if (a.G <= 0 || a.q_len <= 0) return;
+  if (dt == DT_BF16 && launch_attn_prefill_tc(a, err, s)) return;
   if (dt == DT_BF16 && a.dh == 64 && a.q_ld % 8 == 0 && a.o_ld % 2 == 0 && !tc_attn_disabled()) {
     dim3 g64((a.q_len + 63) / 64, a.H, a.G);
     launch_kernel(k_attn_prefill_mma<SEG_ALL>, g64, 128, 0, s, a, (float*)nullptr);
     return;
   }
+  launch_attn_prefill_simt(dt, a, s);
+}
+
+bool launch_attn_prefill_simt(int dt, const AttnArgs& a, cudaStream_t s) {
   dim3 grid((a.q_len + 31) / 32, a.H, a.G);
   if (dt == DT_BF16 && a.dh == 64)
-    {
-      launch_kernel(k_attn_prefill<bf16, 64>, grid, 128, 0, s, a);
-    }
+    launch_kernel(k_attn_prefill<bf16, 64>, grid, 128, 0, s, a);
   else if (dt == DT_F32 && a.dh == 32)
-    {
-      launch_kernel(k_attn_prefill<float, 32>, grid, 128, 0, s, a);
-    }
+    launch_kernel(k_attn_prefill<float, 32>, grid, 128, 0, s, a);
   else if (dt == DT_F32 && a.dh == 64)
-    {
-      launch_kernel(k_attn_prefill<float, 64>, grid, 128, 0, s, a);
-    }
+    launch_kernel(k_attn_prefill<float, 64>, grid, 128, 0, s, a);
   else if (dt == DT_BF16 && a.dh == 32)
-    {
-      launch_kernel(k_attn_prefill<bf16, 32>, grid, 128, 0, s, a);
-    }
+    launch_kernel(k_attn_prefill<bf16, 32>, grid, 128, 0, s, a);
+  else
+    return false;
+  return true;
+}
+
+bool launch_attn_prefill_path(int dt, const AttnArgs& a, int path, float* part, size_t part_bytes, int* err,
+                              cudaStream_t s) {
+  if (a.G <= 0 || a.q_len <= 0) return true;
+  const bool bf64 = dt == DT_BF16 && a.dh == 64 && a.q_ld % 8 == 0 && a.o_ld % 8 == 0;
+  const bool split = a.n_pre > 0 && a.Kp != nullptr;
+  if (split && (part == nullptr || part_bytes < attn_prefix_split_bytes(a)) && (path == 2 || path == 3))
+    return false;
+  switch (path) {
+    case 0:
+      if (split && launch_attn_prefix_split(dt, a, part, part_bytes, err, s)) return true;
+      launch_attn_prefill(dt, a, err, s);
+      return true;
+    case 1:
+      return launch_attn_prefill_simt(dt, a, s);
+    case 2:
+      if (!bf64) return false;
+      if (split) {
+        const long long rows = (long long)a.G * a.q_len;
+        launch_kernel(k_attn_prefill_mma<SEG_PREFIX>, dim3((unsigned)((rows + 63) / 64), a.H, 1), 128, 0, s, a,
+                      part);
+        launch_kernel(k_attn_prefill_mma<SEG_OWN>, dim3((a.q_len + 63) / 64, a.H, a.G), 128, 0, s, a, part);
+      } else {
+        launch_kernel(k_attn_prefill_mma<SEG_ALL>, dim3((a.q_len + 63) / 64, a.H, a.G), 128, 0, s, a,
+                      (float*)nullptr);
+      }
+      return true;
+    case 3:
+      if (!bf64) return false;
+      if (split) return launch_attn_prefix_tc(a, part, err, s) && launch_attn_own_tc(a, part, err, s);
+      return launch_attn_prefill_tc(a, err, s);
+    default:
+      return false;
+  }
 }
 
 }  // namespace photon

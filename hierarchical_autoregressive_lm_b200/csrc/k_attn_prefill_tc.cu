@@ -1,0 +1,455 @@
+// Causal attention of many new queries (prefill) on the Blackwell tensor
+// cores: the Encoder_1 layers over every level-1 position of a prompt and
+// the top encoder over every chunk (the explainer's architecture module
+// table; softmax(Q K^T / sqrt(dh)) V with a causal mask, one softmax per
+// (sequence, head)).
+//
+// One CTA takes 128 consecutive queries of one (group, head), the M = 128
+// rows of a tcgen05 tile, and walks the keys in blocks of 64:
+//
+//   warp 4 (one lane)  TMA: the Q tile once, then K and V blocks into a
+//                      3-stage ring (3-D tensor maps whose key extent is
+//                      the number of written keys, so rows past it arrive
+//                      as zeros and never carry stale data into P V);
+//   warp 5 (one lane)  tcgen05.mma: S = Q K^T (M 128, N 64, K 64) into
+//                      tensor memory, then O_j = P V (M 128, N 64, K 64)
+//                      with V read as an MN-major operand straight from its
+//                      row-major tile; S of block j + 1 is issued as soon as
+//                      the softmax warps have read S of block j;
+//   warps 0-3          the softmax, one query row per thread (tensor-memory
+//                      lane = row): read S, mask, online max and sum in log2
+//                      units, P = exp2(S - m) as bf16 into shared memory in
+//                      the swizzled K-major layout the MMA reads, and
+//                      O = O * exp2(m_old - m_new) + P V accumulated in
+//                      registers from each block's product.
+//
+// Two CTAs fit on an SM (80 KB of shared memory, 128 tensor-memory columns
+// each), so one CTA's softmax overlaps the other's MMAs.  Every wait is
+// bounded; a wait that runs out records an error word and ends the CTA.
+//
+// Key segments as in the mma.sync kernel: ALL (own keys, no prefix), PREFIX
+// (all queries of the batch stacked, against a shared prefix, writing fp32
+// partials: unnormalised accumulator, max in log2 units, sum) and OWN (own
+// keys, merged with the PREFIX partial of each row before the store).
+#include <cstdlib>
+
+#include "common.cuh"
+#include "kernels.h"
+#include "launch.cuh"
+#include "ptx_sm100.cuh"
+
+namespace photon {
+
+namespace {
+
+namespace ftc {
+constexpr int BM = 128;  // queries per CTA
+constexpr int BN = 64;   // keys per block
+constexpr int D = 64;    // head size
+constexpr int ST = 2;    // K/V ring stages
+constexpr int kQBytes = BM * D * 2;
+constexpr int kKVBytes = BN * D * 2;
+constexpr int kPBytes = BM * BN * 2;
+constexpr int kOffQ = 0;
+constexpr int kOffK = kOffQ + kQBytes;
+constexpr int kOffV = kOffK + ST * kKVBytes;
+constexpr int kOffP = kOffV + ST * kKVBytes;
+constexpr int kOffCtrl = kOffP + kPBytes;
+constexpr int kCtrlBytes = 256;
+constexpr int kSmemBytes = kOffCtrl + kCtrlBytes + 1024;  // + alignment slack
+constexpr int kThreads = 192;                             // softmax warps 0-3, TMA warp 4, MMA warp 5
+constexpr uint32_t kTmemCols = 128;                       // S: columns 0-63, O: 64-127
+constexpr uint32_t kColO = 64;
+// P is taken relative to a reference maximum that only moves when a block's
+// maximum passes it by more than this (log2 units), so P < 2^kRescale and O
+// is rescaled in tensor memory only when the reference moves.
+constexpr float kRescale = 8.f;
+}  // namespace ftc
+
+enum { TSEG_ALL = 0, TSEG_PREFIX = 1, TSEG_OWN = 2 };
+
+struct TcAttnParams {
+  int H = 0, q_len = 0, qrows = 0;  // qrows: the launch's query space (q_len, or G * q_len for PREFIX)
+  int p0 = 0, n_pre = 0;
+  long long o_ld = 0;
+  void* O = nullptr;
+  float* part = nullptr;
+  float sl2 = 0.f;  // scale * log2(e)
+  int* err = nullptr;
+};
+
+__device__ __forceinline__ float ex2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+  const __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<const uint32_t*>(&v);
+}
+
+template <int SEG>
+__global__ void __launch_bounds__(ftc::kThreads, 3)
+    k_attn_prefill_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                      const __grid_constant__ CUtensorMap tmV, TcAttnParams a) {
+  using namespace ftc;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kOffCtrl);
+  // barriers: 0 q_full, 1..ST kv_full, ST+1..2ST kv_empty, then s_full,
+  // s_free, p_full, pv_full, drain
+  const uint32_t q_full = ptx::smem_u32(bars);
+  auto kv_full = [&](int st) { return ptx::smem_u32(bars + 1 + st); };
+  auto kv_empty = [&](int st) { return ptx::smem_u32(bars + 1 + ST + st); };
+  const uint32_t s_full = ptx::smem_u32(bars + 1 + 2 * ST);
+  const uint32_t s_free = ptx::smem_u32(bars + 2 + 2 * ST);
+  const uint32_t p_full = ptx::smem_u32(bars + 3 + 2 * ST);
+  const uint32_t pv_full = ptx::smem_u32(bars + 4 + 2 * ST);
+  const uint32_t drain = ptx::smem_u32(bars + 5 + 2 * ST);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 6 + 2 * ST);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  static_assert((6 + 2 * ST) * 8 + 8 <= kCtrlBytes, "control block layout");
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int h = blockIdx.y, g = SEG == TSEG_PREFIX ? 0 : (int)blockIdx.z;
+  const int tile = (int)(gridDim.x - 1 - blockIdx.x);  // longest key ranges first
+  const int q0 = tile * BM;
+  const int nq = min(BM, a.qrows - q0);
+  const int last_pos = a.p0 + q0 + nq - 1;                       // ALL, OWN
+  const int key0 = SEG == TSEG_OWN ? a.n_pre : 0;                // first key position
+  const int key_end = SEG == TSEG_PREFIX ? a.n_pre : last_pos + 1;
+  const int nb = (key_end - key0 + BN - 1) / BN;
+  const int kv_z = SEG == TSEG_PREFIX ? h : g * a.H + h;          // tensor-map coordinates
+  const int q_y = q0, q_z = SEG == TSEG_PREFIX ? 0 : g;
+
+  if (threadIdx.x == 0) {
+    ptx::mbar_init(q_full, 1);
+    for (int st = 0; st < ST; ++st) {
+      ptx::mbar_init(kv_full(st), 1);
+      ptx::mbar_init(kv_empty(st), 1);
+    }
+    ptx::mbar_init(s_full, 1);
+    ptx::mbar_init(s_free, 4);
+    ptx::mbar_init(p_full, 4);
+    ptx::mbar_init(pv_full, 1);
+    ptx::mbar_init(drain, 1);
+    *abort_flag = 0;
+    ptx::fence_barrier_init();
+    ptx::prefetch_tmap(&tmQ);
+    ptx::prefetch_tmap(&tmK);
+    ptx::prefetch_tmap(&tmV);
+  }
+  if (warp == 5) {
+    ptx::tmem_alloc(ptx::smem_u32(tmem_slot), kTmemCols);
+    ptx::tmem_relinquish();
+  }
+  ptx::tc_fence_before();
+  __syncthreads();
+  ptx::tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  pdl_wait();  // Q, K and V are written by the kernels before this one
+  pdl_trigger();
+
+  if (warp == 4) {
+    // ---------------------------------------------------------------- TMA
+    if (lane == 0) {
+      ptx::mbar_arrive_expect_tx(q_full, (uint32_t)kQBytes);
+      ptx::tma_load_3d(ptx::smem_u32(smem + kOffQ), &tmQ, h * D, q_y, q_z, q_full);
+      const int slot0 = SEG == TSEG_PREFIX ? 0 : key0 - a.n_pre;  // own caches start at position n_pre
+      int issued = 0;
+      for (int j = 0; j < nb; ++j) {
+        const int st = j % ST;
+        const uint32_t ph = (uint32_t)(j / ST) & 1u;
+        if (!ptx::mbar_wait(kv_empty(st), ph ^ 1u, abort_flag)) {
+          report_error(a.err, DEV_WAIT_TIMEOUT_PRODUCER);
+          *abort_flag = 1;
+          break;
+        }
+        ptx::mbar_arrive_expect_tx(kv_full(st), (uint32_t)(2 * kKVBytes));
+        const int y = slot0 + j * BN;
+        ptx::tma_load_3d(ptx::smem_u32(smem + kOffK + st * kKVBytes), &tmK, 0, y, kv_z, kv_full(st));
+        ptx::tma_load_3d(ptx::smem_u32(smem + kOffV + st * kKVBytes), &tmV, 0, y, kv_z, kv_full(st));
+        issued = j + 1;
+      }
+      // no copy of this CTA may still be landing when it exits (matters
+      // only after an abort: otherwise every block has been consumed)
+      ptx::mbar_wait(q_full, 0, nullptr);
+      for (int j = issued > ST ? issued - ST : 0; j < issued; ++j)
+        ptx::mbar_wait(kv_full(j % ST), (uint32_t)(j / ST) & 1u, nullptr);
+    }
+  } else if (warp == 5) {
+    // ---------------------------------------------------------------- MMA
+    if (lane == 0) {
+      constexpr uint32_t idS = ptx::idesc_bf16_f32(BM, BN);
+      constexpr uint32_t idPV = ptx::idesc_bf16_f32_bmn(BM, D);
+      const uint64_t qd = ptx::sdesc_kmajor_sw128(ptx::smem_u32(smem + kOffQ));
+      const uint64_t pd = ptx::sdesc_kmajor_sw128(ptx::smem_u32(smem + kOffP));
+      bool ok = ptx::mbar_wait(q_full, 0, abort_flag);
+      // S_j = Q K_j^T once K_j has landed and S_{j-1} has been read
+      auto issue_s = [&](int j) {
+        const int st = j % ST;
+        if (!ptx::mbar_wait(kv_full(st), (uint32_t)(j / ST) & 1u, abort_flag)) return false;
+        if (j > 0 && !ptx::mbar_wait(s_free, (uint32_t)(j - 1) & 1u, abort_flag)) return false;
+        ptx::tc_fence_after();
+        const uint64_t kd = ptx::sdesc_kmajor_sw128(ptx::smem_u32(smem + kOffK + st * kKVBytes));
+#pragma unroll
+        for (int k = 0; k < D / 16; ++k) ptx::mma_bf16(tmem, qd + 2 * k, kd + 2 * k, idS, k > 0 ? 1u : 0u);
+        ptx::mma_commit(s_full);
+        return true;
+      };
+      if (ok) ok = issue_s(0);
+      for (int j = 0; ok && j < nb; ++j) {
+        if (j + 1 < nb && !issue_s(j + 1)) {
+          ok = false;
+          break;
+        }
+        // O += P_j V_j once the softmax warps have written P_j
+        if (!ptx::mbar_wait(p_full, (uint32_t)j & 1u, abort_flag)) {
+          ok = false;
+          break;
+        }
+        ptx::tc_fence_after();
+        const int st = j % ST;
+        const uint64_t vd = ptx::sdesc_kmajor_sw128(ptx::smem_u32(smem + kOffV + st * kKVBytes));
+#pragma unroll
+        for (int k = 0; k < BN / 16; ++k)
+          ptx::mma_bf16(tmem + kColO, pd + 2 * k, vd + 128 * k, idPV, (j > 0 || k > 0) ? 1u : 0u);
+        ptx::mma_commit(kv_empty(st));
+        ptx::mma_commit(pv_full);
+      }
+      if (!ok) {
+        report_error(a.err, DEV_WAIT_TIMEOUT_MMA);
+        *abort_flag = 1;
+      }
+      // nothing this thread issued may still run when the tensor memory is freed
+      ptx::mma_commit(drain);
+      if (!ptx::mbar_wait(drain, 0, nullptr)) report_error(a.err, DEV_WAIT_TIMEOUT_MMA);
+    }
+  } else {
+    // ---------------------------------------------------------------- softmax
+    const int r = threadIdx.x;                              // query row of the tile = TMEM lane
+    const uint32_t trow = tmem + ((uint32_t)(warp * 32) << 16);
+    const int qpos = a.p0 + q0 + r;                         // ALL, OWN
+    uint8_t* prow = smem + kOffP + r * 128;
+    // warp-uniform bounded wait (the tensor-memory accesses below are warp-collective)
+    auto wait_all = [&](uint32_t bar, uint32_t parity) {
+      return __all_sync(0xffffffffu, ptx::mbar_wait(bar, parity, abort_flag)) != 0;
+    };
+    float m = -INFINITY, l = 0.f;  // reference maximum (log2 units) and row sum
+    bool ok = true;
+    for (int j = 0; j < nb; ++j) {
+      if (!wait_all(s_full, (uint32_t)j & 1u)) {
+        ok = false;
+        break;
+      }
+      ptx::tc_fence_after();
+      float s[BN];
+      ptx::tmem_ld64(trow, s);
+      ptx::tc_fence_before();
+      __syncwarp();
+      if (lane == 0) ptx::mbar_arrive(s_free);
+      // mask: keys past the segment, and (own keys) keys after this query
+      const int kbase = key0 + j * BN;
+      const int lim = SEG == TSEG_PREFIX ? key_end - 1 - kbase : qpos - kbase;
+      if (lim < BN - 1) {
+#pragma unroll
+        for (int c = 0; c < BN; ++c) s[c] = c > lim ? -INFINITY : s[c];
+      }
+      // block maximum of the raw scores (8 independent partial maxima), in
+      // log2 units after scaling (the scale is positive)
+      float mp[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) mp[i] = s[i];
+#pragma unroll
+      for (int c = 8; c < BN; ++c) mp[c & 7] = fmaxf(mp[c & 7], s[c]);
+#pragma unroll
+      for (int w = 4; w > 0; w >>= 1)
+#pragma unroll
+        for (int i = 0; i < w; ++i) mp[i] = fmaxf(mp[i], mp[i + w]);
+      const float bm = mp[0] * a.sl2;
+      const bool grow = bm > m + kRescale;  // also the first finite block maximum
+      const float corr = grow ? ex2(m - bm) : 1.f;
+      // the previous P V product is complete: P's buffer is free, and O may
+      // be rescaled to the new reference
+      if (j > 0) {
+        if (!wait_all(pv_full, (uint32_t)(j - 1) & 1u)) {
+          ok = false;
+          break;
+        }
+        ptx::tc_fence_after();
+        if (__any_sync(0xffffffffu, grow)) {
+#pragma unroll 1
+          for (int hh = 0; hh < D; hh += 8) {
+            float ov[8];
+            ptx::tmem_ld8(trow + kColO + (uint32_t)hh, ov);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) ov[i] *= corr;
+            ptx::tmem_st8(trow + kColO + (uint32_t)hh, ov);
+          }
+        }
+      }
+      if (grow) m = bm;
+      l *= corr;
+      const float nmu = m == -INFINITY ? 0.f : -m;
+      // P = exp2(S * scale * log2(e) - m) as bf16, row by row into the
+      // 128-byte-swizzled K-major tile: 16-byte chunk u at u ^ (row % 8)
+      float rp[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        uint32_t pk[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float p0 = ex2(fmaf(s[8 * u + 2 * e], a.sl2, nmu));
+          const float p1 = ex2(fmaf(s[8 * u + 2 * e + 1], a.sl2, nmu));
+          rp[e] += p0 + p1;
+          pk[e] = pack_bf16x2(p0, p1);
+        }
+        *reinterpret_cast<uint4*>(prow + ((u ^ (r & 7)) << 4)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+      }
+      l += (rp[0] + rp[1]) + (rp[2] + rp[3]);
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      ptx::tc_fence_before();
+      __syncwarp();
+      if (lane == 0) ptx::mbar_arrive(p_full);
+    }
+    float o[D];
+#pragma unroll
+    for (int c = 0; c < D; ++c) o[c] = 0.f;
+    if (ok && nb > 0) {
+      if (wait_all(pv_full, (uint32_t)(nb - 1) & 1u)) {
+        ptx::tc_fence_after();
+        ptx::tmem_ld64(trow + kColO, o);
+      } else {
+        ok = false;
+      }
+    }
+    if (!ok) {
+      report_error(a.err, DEV_WAIT_TIMEOUT_EPILOGUE);
+      *abort_flag = 1;
+    }
+    ptx::tc_fence_before();
+    if (ok && r < nq) {
+      const long long fr = (SEG == TSEG_PREFIX ? 0 : (long long)g * a.q_len) + q0 + r;  // flattened row
+      if constexpr (SEG == TSEG_PREFIX) {
+        float* pp = a.part + (fr * a.H + h) * (D + 2);
+#pragma unroll
+        for (int c = 0; c < D; c += 2) *reinterpret_cast<float2*>(pp + c) = make_float2(o[c], o[c + 1]);
+        *reinterpret_cast<float2*>(pp + D) = make_float2(m, l);
+      } else {
+        if constexpr (SEG == TSEG_OWN) {
+          // merge with the prefix partial of this row at the common maximum
+          const float* pp = a.part + (fr * a.H + h) * (D + 2);
+          const float2 ml = *reinterpret_cast<const float2*>(pp + D);
+          const float M = fmaxf(m, ml.x);
+          const float co = ex2(m - M), cp = ex2(ml.x - M);
+          l = l * co + ml.y * cp;
+#pragma unroll
+          for (int c = 0; c < D; c += 2) {
+            const float2 pa = *reinterpret_cast<const float2*>(pp + c);
+            o[c] = o[c] * co + pa.x * cp;
+            o[c + 1] = o[c + 1] * co + pa.y * cp;
+          }
+        }
+        const float inv = l > 0.f ? 1.f / l : 0.f;
+        bf16* orow = reinterpret_cast<bf16*>(a.O) + fr * a.o_ld + h * D;
+#pragma unroll
+        for (int u = 0; u < D / 8; ++u)
+          reinterpret_cast<uint4*>(orow)[u] =
+              make_uint4(pack_bf16x2(o[8 * u] * inv, o[8 * u + 1] * inv), pack_bf16x2(o[8 * u + 2] * inv, o[8 * u + 3] * inv),
+                         pack_bf16x2(o[8 * u + 4] * inv, o[8 * u + 5] * inv), pack_bf16x2(o[8 * u + 6] * inv, o[8 * u + 7] * inv));
+      }
+    }
+  }
+  __syncthreads();
+  if (warp == 5) {
+    ptx::tc_fence_after();
+    ptx::tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+bool tc_prefill_disabled() {
+  static const bool off = [] {
+    const char* e = getenv("PHOTON_PREFILL_ATTN");
+    return e && (e[0] == 's' || e[0] == 'm');  // "simt" or "mma": the older kernels
+  }();
+  return off;
+}
+
+template <int SEG>
+bool launch_seg(const AttnArgs& a, float* part, int* err, cudaStream_t s) {
+  using namespace ftc;
+  static PerDevice configured;
+  if (configured.get([] {
+        return (int)cudaFuncSetAttribute(k_attn_prefill_tc<SEG>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         kSmemBytes);
+      }) != (int)cudaSuccess)
+    return false;
+  CUtensorMap mq, mk, mv;
+  const long long hd = (long long)a.H * D;
+  TcAttnParams p;
+  p.H = a.H;
+  p.q_len = a.q_len;
+  p.p0 = a.p0;
+  p.n_pre = a.n_pre;
+  p.O = a.O;
+  p.o_ld = a.o_ld;
+  p.part = part;
+  p.sl2 = a.scale * 1.4426950408889634f;
+  p.err = err;
+  if (SEG == TSEG_PREFIX) {
+    p.qrows = a.G * a.q_len;
+    // queries: every group's rows stacked; keys: the prefix [H][cap_pre][D], n_pre written
+    if (!tma_map_bf16_3d(&mq, a.Q, hd, (long long)a.G * a.q_len, 1, a.q_ld, (long long)a.G * a.q_len * a.q_ld, D, BM) ||
+        !tma_map_bf16_3d(&mk, a.Kp, D, a.n_pre, a.H, D, (long long)a.cap_pre * D, D, BN) ||
+        !tma_map_bf16_3d(&mv, a.Vp, D, a.n_pre, a.H, D, (long long)a.cap_pre * D, D, BN))
+      return false;
+  } else {
+    p.qrows = a.q_len;
+    // own keys [G*H][cap][D]: slots 0 .. p0 - n_pre + q_len - 1 are written
+    const long long own = (long long)a.p0 - a.n_pre + a.q_len;
+    if (!tma_map_bf16_3d(&mq, a.Q, hd, a.q_len, a.G, a.q_ld, (long long)a.q_len * a.q_ld, D, BM) ||
+        !tma_map_bf16_3d(&mk, a.K, D, own, (long long)a.G * a.H, D, (long long)a.cap * D, D, BN) ||
+        !tma_map_bf16_3d(&mv, a.V, D, own, (long long)a.G * a.H, D, (long long)a.cap * D, D, BN))
+      return false;
+  }
+  const dim3 grid((unsigned)((p.qrows + BM - 1) / BM), (unsigned)a.H, SEG == TSEG_PREFIX ? 1u : (unsigned)a.G);
+  launch_kernel(k_attn_prefill_tc<SEG>, grid, kThreads, kSmemBytes, s, mq, mk, mv, p);
+  return true;
+}
+
+bool args_ok(const AttnArgs& a) {
+  const auto al16 = [](const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; };
+  return a.dh == ftc::D && a.G > 0 && a.H > 0 && a.p0_dev == nullptr && a.q_ld % 8 == 0 &&
+         a.o_ld % 8 == 0 && al16(a.Q) && al16(a.O) && tma_available() && !tc_prefill_disabled();
+}
+
+}  // namespace
+
+// Tensor-core prefill attention for bf16, head size 64, at least 128 query
+// rows (a 128-row tile would mostly idle below that); returns false when
+// the shape is not supported (the caller then takes the mma.sync kernel).
+bool launch_attn_prefill_tc(const AttnArgs& a, int* err, cudaStream_t s) {
+  if (!args_ok(a) || a.q_len < ftc::BM || a.n_pre != 0 || a.Kp != nullptr) return false;
+  if (!(reinterpret_cast<uintptr_t>(a.K) % 16 == 0 && reinterpret_cast<uintptr_t>(a.V) % 16 == 0 &&
+        a.p0 + a.q_len <= a.cap && a.p0 >= 0))
+    return false;
+  return launch_seg<TSEG_ALL>(a, nullptr, err, s);
+}
+
+bool launch_attn_prefix_tc(const AttnArgs& a, float* part, int* err, cudaStream_t s) {
+  if (!args_ok(a) || (long long)a.G * a.q_len < ftc::BM || a.n_pre <= 0 || a.Kp == nullptr || !part) return false;
+  if (reinterpret_cast<uintptr_t>(a.Kp) % 16 || reinterpret_cast<uintptr_t>(a.Vp) % 16 || a.n_pre > a.cap_pre)
+    return false;
+  return launch_seg<TSEG_PREFIX>(a, part, err, s);
+}
+
+bool launch_attn_own_tc(const AttnArgs& a, float* part, int* err, cudaStream_t s) {
+  if (!args_ok(a) || a.q_len < ftc::BM || a.n_pre <= 0 || !part) return false;
+  if (reinterpret_cast<uintptr_t>(a.K) % 16 || reinterpret_cast<uintptr_t>(a.V) % 16 || a.p0 < a.n_pre ||
+      a.p0 - a.n_pre + a.q_len > a.cap)
+    return false;
+  return launch_seg<TSEG_OWN>(a, part, err, s);
+}
+
+}  // namespace photon

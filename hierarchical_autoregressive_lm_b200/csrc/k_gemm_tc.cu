@@ -1405,6 +1405,21 @@ bool tma_available() { return encode_fn() != nullptr; }
 bool tma_map_bf16(CUtensorMap* m, const void* ptr, long long rows, int K, long long ld, int box_rows) {
   return make_map(m, ptr, rows, K, ld, box_rows);
 }
+// 3-D bf16 map: extents d0 (contiguous) x d1 x d2, strides of dims 1 and 2 in
+// elements; box = box0 x box1 x 1, 128-byte swizzle, zero fill past every
+// extent.
+bool tma_map_bf16_3d(CUtensorMap* m, const void* ptr, long long d0, long long d1, long long d2,
+                     long long stride1, long long stride2, int box0, int box1) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn || d0 <= 0 || d1 <= 0 || d2 <= 0) return false;
+  cuuint64_t dims[3] = {(cuuint64_t)d0, (cuuint64_t)d1, (cuuint64_t)d2};
+  cuuint64_t strides[2] = {(cuuint64_t)stride1 * 2, (cuuint64_t)stride2 * 2};
+  cuuint32_t box[3] = {(cuuint32_t)box0, (cuuint32_t)box1, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
 
 int gemm_tc_argmax_tiles(int M, int N, int K) {
   if (M <= 0 || N <= 0 || K <= 0 || K % kBK || N % 64) return 0;

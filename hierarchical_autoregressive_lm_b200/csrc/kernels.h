@@ -300,13 +300,23 @@ size_t attn_decode_workspace_bytes(int dt, const AttnArgs& a);
 bool launch_attn_decode(int dt, const AttnArgs& a, float* part, size_t part_bytes, int* err,
                         cudaStream_t s);
 // Causal attention for many new queries per group (prefill).
-void launch_attn_prefill(int dt, const AttnArgs& a, cudaStream_t s);
+void launch_attn_prefill(int dt, const AttnArgs& a, int* err, cudaStream_t s);
 // Attention with a shared prefix as two passes (bf16, dh = 64): all query
 // rows against the prefix rows, then each group's own causal keys merged
 // with that partial.  part holds attn_prefix_split_bytes(a).  Returns false
 // (nothing launched) when the shape or the scratch does not fit.
 size_t attn_prefix_split_bytes(const AttnArgs& a);
-bool launch_attn_prefix_split(int dt, const AttnArgs& a, float* part, size_t part_bytes, cudaStream_t s);
+bool launch_attn_prefix_split(int dt, const AttnArgs& a, float* part, size_t part_bytes, int* err,
+                              cudaStream_t s);
+// The CUDA-core prefill kernel (any storage type, head size 32 or 64).
+bool launch_attn_prefill_simt(int dt, const AttnArgs& a, cudaStream_t s);
+// Prefill attention on a chosen kernel (0 the library's choice, 1 CUDA
+// cores, 2 mma.sync, 3 tcgen05); with a prefix (n_pre > 0) paths 2 and 3
+// take the two-pass split and need attn_prefix_split_bytes(a) of part.
+// Returns false (possibly after launching a first pass) when the path does
+// not take the shape.
+bool launch_attn_prefill_path(int dt, const AttnArgs& a, int path, float* part, size_t part_bytes, int* err,
+                              cudaStream_t s);
 
 // ---- error message of the calling thread (read by photon_last_error) ----
 void set_error_message(const char* msg);
@@ -321,5 +331,14 @@ bool tma_available();
 // 2-D bf16 tensor map over a row-major [rows, K] matrix (leading dimension ld
 // elements): box 64 (K) x box_rows, 128-byte swizzle, zero fill.
 bool tma_map_bf16(CUtensorMap* m, const void* ptr, long long rows, int K, long long ld, int box_rows);
+bool tma_map_bf16_3d(CUtensorMap* m, const void* ptr, long long d0, long long d1, long long d2,
+                     long long stride1, long long stride2, int box0, int box1);
+// Tensor-core (tcgen05) prefill attention, k_attn_prefill_tc.cu: bf16, head
+// size 64, at least 128 query rows; false when the shape is not supported.
+// ALL: own keys only (no prefix).  PREFIX: every query row against the
+// shared prefix, fp32 partials into part; OWN: own keys merged with them.
+bool launch_attn_prefill_tc(const AttnArgs& a, int* err, cudaStream_t s);
+bool launch_attn_prefix_tc(const AttnArgs& a, float* part, int* err, cudaStream_t s);
+bool launch_attn_own_tc(const AttnArgs& a, float* part, int* err, cudaStream_t s);
 
 }  // namespace photon

@@ -676,9 +676,9 @@ static void run_block(photon_model* m, const BlockW& w, float* x, const StackRun
   bool done = false;
   // with a shared prefix: the prefix once for all queries, then each group's own keys
   if (r.kp && b.pre_ws && prefix_split_enabled())
-    done = launch_attn_prefix_split(m->dt, a, b.pre_ws, b.pre_ws_bytes, s);
+    done = launch_attn_prefix_split(m->dt, a, b.pre_ws, b.pre_ws_bytes, b.err, s);
   if (!done && r.q_len <= 4) done = launch_attn_decode(m->dt, a, b.attn_ws, b.attn_ws_bytes, b.err, s);
-  if (!done) launch_attn_prefill(m->dt, a, s);
+  if (!done) launch_attn_prefill(m->dt, a, b.err, s);
 
   Epilogue eo = epi(EPI_ADD_F32, x, d);
   int slots_o = 0;
@@ -2790,6 +2790,49 @@ int photon_attn_decode(int32_t dtype, const void* d_q, const void* d_k, const vo
   const bool ok = launch_attn_decode(dtype, a, ws, wsb, d_err, s);
   if (ws) cudaFreeAsync(ws, s);
   if (!ok) return fail(PHOTON_ERR_ARG, "decode attention rejected the shape");
+  CK(cudaGetLastError());
+  return PHOTON_OK;
+}
+
+int photon_attn_prefill(int32_t dtype, const void* d_q, const void* d_k, const void* d_v, const void* d_kp,
+                        const void* d_vp, int32_t G, int32_t H, int32_t head_dim, int32_t cap, int32_t q_len,
+                        int32_t p0, int32_t cap_pre, int32_t n_pre, int32_t path, void* d_o, int32_t* d_err,
+                        void* stream) {
+  g_err.clear();
+  if (dtype != 0 && dtype != 1) return fail(PHOTON_ERR_ARG, "dtype must be 0 or 1");
+  if (!d_q || !d_k || !d_v || !d_o) return fail(PHOTON_ERR_ARG, "NULL buffer");
+  if (G <= 0 || H <= 0 || (head_dim != 32 && head_dim != 64)) return fail(PHOTON_ERR_ARG, "bad shape");
+  if (q_len < 1 || n_pre < 0 || p0 < n_pre || p0 - n_pre + q_len > cap)
+    return fail(PHOTON_ERR_ARG, "bad q_len/p0/n_pre/cap");
+  if (n_pre > 0 && (!d_kp || !d_vp || n_pre > cap_pre)) return fail(PHOTON_ERR_ARG, "bad prefix");
+  if (path < 0 || path > 3) return fail(PHOTON_ERR_ARG, "unknown path %d", path);
+  cudaStream_t s = (cudaStream_t)stream;
+  AttnArgs a;
+  a.Q = d_q;
+  a.q_ld = (long long)H * head_dim;
+  a.K = d_k;
+  a.V = d_v;
+  a.cap = cap;
+  if (n_pre > 0) {
+    a.Kp = d_kp;
+    a.Vp = d_vp;
+    a.cap_pre = cap_pre;
+    a.n_pre = n_pre;
+  }
+  a.G = G;
+  a.H = H;
+  a.dh = head_dim;
+  a.q_len = q_len;
+  a.p0 = p0;
+  a.O = d_o;
+  a.o_ld = (long long)H * head_dim;
+  a.scale = 1.0f / sqrtf((float)head_dim);
+  const size_t wsb = n_pre > 0 ? attn_prefix_split_bytes(a) : 0;
+  float* ws = nullptr;
+  if (wsb) CK(pool_malloc((void**)&ws, wsb, s));
+  const bool ok = launch_attn_prefill_path(dtype, a, path, ws, wsb, d_err, s);
+  if (ws) cudaFreeAsync(ws, s);
+  if (!ok) return fail(PHOTON_ERR_ARG, "path %d does not take this shape", path);
   CK(cudaGetLastError());
   return PHOTON_OK;
 }

@@ -343,6 +343,25 @@ PHOTON_API int photon_gemm_rmsnorm(const float* d_x, int64_t ldx, const float* d
                                    const void* d_W, int64_t ldw, int32_t M, int32_t N, int32_t K,
                                    float* d_C, int64_t ldc, void* stream);
 
+/* Kernel-level entry: causal prefill attention (Encoder_1 over the level-1
+ * positions of a prompt, the top encoder over its chunks).  For G groups x
+ * H heads, q_len new queries at positions p0..p0+q_len-1 attend to keys
+ * 0..p0+i: positions < n_pre from a shared prefix d_kp/d_vp [H][cap_pre]
+ * [head_dim] (the same for every group; NULL when n_pre = 0), later ones
+ * from d_k/d_v [G][H][cap][head_dim] at slot pos - n_pre (post-RoPE keys,
+ * storage type).  Slots past p0 - n_pre + q_len and prefix rows past n_pre
+ * are never read, whatever they hold.  d_q, d_o: [G*q_len][H*head_dim].
+ * Scale 1/sqrt(head_dim).  path: 0 = the library's choice, 1 = CUDA-core
+ * kernel, 2 = mma.sync tiles (bf16, head_dim 64), 3 = tcgen05 kernel (bf16,
+ * head_dim 64, q_len >= 128, and with a prefix G*q_len >= 128).  d_err as
+ * for photon_attn_decode.  Allocates the prefix pass's partials internally.
+ * Errors: ERR_ARG (bad arguments, or a path that does not take the shape). */
+PHOTON_API int photon_attn_prefill(int32_t dtype, const void* d_q, const void* d_k, const void* d_v,
+                                   const void* d_kp, const void* d_vp, int32_t G, int32_t H,
+                                   int32_t head_dim, int32_t cap, int32_t q_len, int32_t p0,
+                                   int32_t cap_pre, int32_t n_pre, int32_t path, void* d_o,
+                                   int32_t* d_err, void* stream);
+
 /* Kernel-level entry: split-K decode attention (the top-encoder decode
  * kernel).  For G groups x H heads, q_len <= 4 new queries at positions
  * p0..p0+q_len-1 attend causally over keys 0..p0+i of a cache
