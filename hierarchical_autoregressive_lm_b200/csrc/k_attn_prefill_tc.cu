@@ -7,25 +7,31 @@
 // One CTA takes 128 consecutive queries of one (group, head), the M = 128
 // rows of a tcgen05 tile, and walks the keys in blocks of 64:
 //
-//   warp 4 (one lane)  TMA: the Q tile once, then K and V blocks into a
-//                      3-stage ring (3-D tensor maps whose key extent is
-//                      the number of written keys, so rows past it arrive
-//                      as zeros and never carry stale data into P V);
+//   warp 4 (one lane)  TMA: the Q tile once, then K and V blocks into rings
+//                      of 3 and 2 stages, K one block ahead of V (a K block
+//                      is free as soon as its S is computed).  The 3-D
+//                      tensor maps stop at the number of written keys, so
+//                      rows past it arrive as zeros and never carry stale
+//                      data into P V;
 //   warp 5 (one lane)  tcgen05.mma: S = Q K^T (M 128, N 64, K 64) into
-//                      tensor memory, then O_j = P V (M 128, N 64, K 64)
-//                      with V read as an MN-major operand straight from its
-//                      row-major tile; S of block j + 1 is issued as soon as
-//                      the softmax warps have read S of block j;
+//                      tensor memory, and O += P V (M 128, N 64, K 64) into
+//                      a tensor-memory accumulator, V read as an MN-major
+//                      operand straight from its row-major tile; S of block
+//                      j + 1 is issued as soon as the softmax warps have
+//                      read S of block j;
 //   warps 0-3          the softmax, one query row per thread (tensor-memory
-//                      lane = row): read S, mask, online max and sum in log2
-//                      units, P = exp2(S - m) as bf16 into shared memory in
-//                      the swizzled K-major layout the MMA reads, and
-//                      O = O * exp2(m_old - m_new) + P V accumulated in
-//                      registers from each block's product.
+//                      lane = row): read S, mask, P = exp2(S - m) as bf16
+//                      into shared memory in the swizzled K-major layout
+//                      the MMA reads, row sums in fp32.  The reference
+//                      maximum m (log2 units) moves only when a block's
+//                      maximum passes it by more than 8, so P < 2^8 and O
+//                      is rescaled in tensor memory only then; O / l at the
+//                      end is the same softmax for any such reference.
 //
-// Two CTAs fit on an SM (80 KB of shared memory, 128 tensor-memory columns
-// each), so one CTA's softmax overlaps the other's MMAs.  Every wait is
-// bounded; a wait that runs out records an error word and ends the CTA.
+// Three CTAs fit on an SM (73 KB of shared memory, 96 registers a thread,
+// 128 tensor-memory columns each), so one CTA's softmax overlaps the
+// others' MMAs and loads.  Every wait is bounded; a wait that runs out
+// records an error word and ends the CTA.
 //
 // Key segments as in the mma.sync kernel: ALL (own keys, no prefix), PREFIX
 // (all queries of the batch stacked, against a shared prefix, writing fp32
@@ -43,27 +49,32 @@ namespace photon {
 namespace {
 
 namespace ftc {
-constexpr int BM = 128;  // queries per CTA
+constexpr int BM = 128;  // queries per tile
 constexpr int BN = 64;   // keys per block
 constexpr int D = 64;    // head size
-constexpr int ST = 2;    // K/V ring stages
+constexpr int KST = 3;   // K ring stages (a K block is free once S = Q K^T is done)
+constexpr int VST = 2;   // V ring stages (a V block is free once O += P V is done)
 constexpr int kQBytes = BM * D * 2;
 constexpr int kKVBytes = BN * D * 2;
 constexpr int kPBytes = BM * BN * 2;
-constexpr int kOffQ = 0;
-constexpr int kOffK = kOffQ + kQBytes;
-constexpr int kOffV = kOffK + ST * kKVBytes;
-constexpr int kOffP = kOffV + ST * kKVBytes;
-constexpr int kOffCtrl = kOffP + kPBytes;
 constexpr int kCtrlBytes = 256;
-constexpr int kSmemBytes = kOffCtrl + kCtrlBytes + 1024;  // + alignment slack
-constexpr int kThreads = 192;                             // softmax warps 0-3, TMA warp 4, MMA warp 5
-constexpr uint32_t kTmemCols = 128;                       // S: columns 0-63, O: 64-127
-constexpr uint32_t kColO = 64;
 // P is taken relative to a reference maximum that only moves when a block's
 // maximum passes it by more than this (log2 units), so P < 2^kRescale and O
 // is rescaled in tensor memory only when the reference moves.
 constexpr float kRescale = 8.f;
+// NT query tiles per CTA share every K and V block.
+template <int NT>
+struct Cfg {
+  static constexpr int kOffQ = 0;
+  static constexpr int kOffK = kOffQ + NT * kQBytes;
+  static constexpr int kOffV = kOffK + KST * kKVBytes;
+  static constexpr int kOffP = kOffV + VST * kKVBytes;
+  static constexpr int kOffCtrl = kOffP + NT * kPBytes;
+  static constexpr int kSmemBytes = kOffCtrl + kCtrlBytes + 1024;  // + alignment slack
+  static constexpr int kThreads = NT * 128 + 64;  // softmax warps 0..4NT-1, then TMA, then MMA
+  static constexpr int kMinBlocks = NT == 1 ? 3 : 2;
+  static constexpr uint32_t kTmemCols = NT * 128;  // tile t: S at 128 t, O at 128 t + 64
+};
 }  // namespace ftc
 
 enum { TSEG_ALL = 0, TSEG_PREFIX = 1, TSEG_OWN = 2 };
@@ -88,51 +99,67 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return *reinterpret_cast<const uint32_t*>(&v);
 }
 
-template <int SEG>
-__global__ void __launch_bounds__(ftc::kThreads, 3)
+template <int SEG, int NT>
+__global__ void __launch_bounds__(ftc::Cfg<NT>::kThreads, ftc::Cfg<NT>::kMinBlocks)
     k_attn_prefill_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                       const __grid_constant__ CUtensorMap tmV, TcAttnParams a) {
   using namespace ftc;
+  using C = Cfg<NT>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kOffCtrl);
-  // barriers: 0 q_full, 1..ST kv_full, ST+1..2ST kv_empty, then s_full,
-  // s_free, p_full, pv_full, drain
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kOffCtrl);
+  // barriers: q_full, k_full[KST], k_empty[KST], v_full[VST], v_empty[VST],
+  // then per tile s_full, s_free, p_full, pv_full, then drain
   const uint32_t q_full = ptx::smem_u32(bars);
-  auto kv_full = [&](int st) { return ptx::smem_u32(bars + 1 + st); };
-  auto kv_empty = [&](int st) { return ptx::smem_u32(bars + 1 + ST + st); };
-  const uint32_t s_full = ptx::smem_u32(bars + 1 + 2 * ST);
-  const uint32_t s_free = ptx::smem_u32(bars + 2 + 2 * ST);
-  const uint32_t p_full = ptx::smem_u32(bars + 3 + 2 * ST);
-  const uint32_t pv_full = ptx::smem_u32(bars + 4 + 2 * ST);
-  const uint32_t drain = ptx::smem_u32(bars + 5 + 2 * ST);
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 6 + 2 * ST);
+  auto k_full = [&](int st) { return ptx::smem_u32(bars + 1 + st); };
+  auto k_empty = [&](int st) { return ptx::smem_u32(bars + 1 + KST + st); };
+  auto v_full = [&](int st) { return ptx::smem_u32(bars + 1 + 2 * KST + st); };
+  auto v_empty = [&](int st) { return ptx::smem_u32(bars + 1 + 2 * KST + VST + st); };
+  constexpr int kB = 1 + 2 * KST + 2 * VST;
+  auto s_full = [&](int t) { return ptx::smem_u32(bars + kB + 4 * t); };
+  auto s_free = [&](int t) { return ptx::smem_u32(bars + kB + 4 * t + 1); };
+  auto p_full = [&](int t) { return ptx::smem_u32(bars + kB + 4 * t + 2); };
+  auto pv_full = [&](int t) { return ptx::smem_u32(bars + kB + 4 * t + 3); };
+  const uint32_t drain = ptx::smem_u32(bars + kB + 4 * NT);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + kB + 4 * NT + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-  static_assert((6 + 2 * ST) * 8 + 8 <= kCtrlBytes, "control block layout");
+  static_assert((kB + 4 * NT + 1) * 8 + 8 <= kCtrlBytes, "control block layout");
+  constexpr int kProducer = 4 * NT, kMma = 4 * NT + 1;  // warp indices
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int h = blockIdx.y, g = SEG == TSEG_PREFIX ? 0 : (int)blockIdx.z;
-  const int tile = (int)(gridDim.x - 1 - blockIdx.x);  // longest key ranges first
-  const int q0 = tile * BM;
-  const int nq = min(BM, a.qrows - q0);
-  const int last_pos = a.p0 + q0 + nq - 1;                       // ALL, OWN
+  const int q0 = (int)(gridDim.x - 1 - blockIdx.x) * (NT * BM);  // longest key ranges first
   const int key0 = SEG == TSEG_OWN ? a.n_pre : 0;                // first key position
-  const int key_end = SEG == TSEG_PREFIX ? a.n_pre : last_pos + 1;
-  const int nb = (key_end - key0 + BN - 1) / BN;
+  // key blocks of tile t (0 for a tile past the last query)
+  auto tile_blocks = [&](int t) {
+    const int nq = min(BM, a.qrows - (q0 + t * BM));
+    if (nq <= 0) return 0;
+    const int key_end = SEG == TSEG_PREFIX ? a.n_pre : a.p0 + q0 + t * BM + nq;
+    return (key_end - key0 + BN - 1) / BN;
+  };
+  int nb = 0;
+#pragma unroll
+  for (int t = 0; t < NT; ++t) nb = max(nb, tile_blocks(t));
   const int kv_z = SEG == TSEG_PREFIX ? h : g * a.H + h;          // tensor-map coordinates
-  const int q_y = q0, q_z = SEG == TSEG_PREFIX ? 0 : g;
+  const int q_z = SEG == TSEG_PREFIX ? 0 : g;
 
   if (threadIdx.x == 0) {
     ptx::mbar_init(q_full, 1);
-    for (int st = 0; st < ST; ++st) {
-      ptx::mbar_init(kv_full(st), 1);
-      ptx::mbar_init(kv_empty(st), 1);
+    for (int st = 0; st < KST; ++st) {
+      ptx::mbar_init(k_full(st), 1);
+      ptx::mbar_init(k_empty(st), 1);
     }
-    ptx::mbar_init(s_full, 1);
-    ptx::mbar_init(s_free, 4);
-    ptx::mbar_init(p_full, 4);
-    ptx::mbar_init(pv_full, 1);
+    for (int st = 0; st < VST; ++st) {
+      ptx::mbar_init(v_full(st), 1);
+      ptx::mbar_init(v_empty(st), 1);
+    }
+    for (int t = 0; t < NT; ++t) {
+      ptx::mbar_init(s_full(t), 1);
+      ptx::mbar_init(s_free(t), 4);
+      ptx::mbar_init(p_full(t), 4);
+      ptx::mbar_init(pv_full(t), 1);
+    }
     ptx::mbar_init(drain, 1);
     *abort_flag = 0;
     ptx::fence_barrier_init();
@@ -140,8 +167,8 @@ __global__ void __launch_bounds__(ftc::kThreads, 3)
     ptx::prefetch_tmap(&tmK);
     ptx::prefetch_tmap(&tmV);
   }
-  if (warp == 5) {
-    ptx::tmem_alloc(ptx::smem_u32(tmem_slot), kTmemCols);
+  if (warp == kMma) {
+    ptx::tmem_alloc(ptx::smem_u32(tmem_slot), C::kTmemCols);
     ptx::tmem_relinquish();
   }
   ptx::tc_fence_before();
@@ -151,51 +178,77 @@ __global__ void __launch_bounds__(ftc::kThreads, 3)
   pdl_wait();  // Q, K and V are written by the kernels before this one
   pdl_trigger();
 
-  if (warp == 4) {
+  if (warp == kProducer) {
     // ---------------------------------------------------------------- TMA
     if (lane == 0) {
-      ptx::mbar_arrive_expect_tx(q_full, (uint32_t)kQBytes);
-      ptx::tma_load_3d(ptx::smem_u32(smem + kOffQ), &tmQ, h * D, q_y, q_z, q_full);
+      ptx::mbar_arrive_expect_tx(q_full, (uint32_t)(NT * kQBytes));
+      for (int t = 0; t < NT; ++t)
+        ptx::tma_load_3d(ptx::smem_u32(smem + C::kOffQ + t * kQBytes), &tmQ, h * D, q0 + t * BM, q_z, q_full);
       const int slot0 = SEG == TSEG_PREFIX ? 0 : key0 - a.n_pre;  // own caches start at position n_pre
-      int issued = 0;
-      for (int j = 0; j < nb; ++j) {
-        const int st = j % ST;
-        const uint32_t ph = (uint32_t)(j / ST) & 1u;
-        if (!ptx::mbar_wait(kv_empty(st), ph ^ 1u, abort_flag)) {
-          report_error(a.err, DEV_WAIT_TIMEOUT_PRODUCER);
-          *abort_flag = 1;
-          break;
+      // K runs one block ahead of V: K_0, K_1, V_0, K_2, V_1, ...
+      int nk = 0, nv = 0;
+      bool ok = true;
+      for (int i = 0; ok && i <= nb; ++i) {
+        if (i < nb) {
+          const int st = i % KST;
+          if (!ptx::mbar_wait(k_empty(st), ((uint32_t)(i / KST) & 1u) ^ 1u, abort_flag)) {
+            ok = false;
+            break;
+          }
+          ptx::mbar_arrive_expect_tx(k_full(st), (uint32_t)kKVBytes);
+          ptx::tma_load_3d(ptx::smem_u32(smem + C::kOffK + st * kKVBytes), &tmK, 0, slot0 + i * BN, kv_z, k_full(st));
+          nk = i + 1;
         }
-        ptx::mbar_arrive_expect_tx(kv_full(st), (uint32_t)(2 * kKVBytes));
-        const int y = slot0 + j * BN;
-        ptx::tma_load_3d(ptx::smem_u32(smem + kOffK + st * kKVBytes), &tmK, 0, y, kv_z, kv_full(st));
-        ptx::tma_load_3d(ptx::smem_u32(smem + kOffV + st * kKVBytes), &tmV, 0, y, kv_z, kv_full(st));
-        issued = j + 1;
+        if (i >= 1) {
+          const int j = i - 1, st = j % VST;
+          if (!ptx::mbar_wait(v_empty(st), ((uint32_t)(j / VST) & 1u) ^ 1u, abort_flag)) {
+            ok = false;
+            break;
+          }
+          ptx::mbar_arrive_expect_tx(v_full(st), (uint32_t)kKVBytes);
+          ptx::tma_load_3d(ptx::smem_u32(smem + C::kOffV + st * kKVBytes), &tmV, 0, slot0 + j * BN, kv_z, v_full(st));
+          nv = j + 1;
+        }
+      }
+      if (!ok) {
+        report_error(a.err, DEV_WAIT_TIMEOUT_PRODUCER);
+        *abort_flag = 1;
       }
       // no copy of this CTA may still be landing when it exits (matters
       // only after an abort: otherwise every block has been consumed)
       ptx::mbar_wait(q_full, 0, nullptr);
-      for (int j = issued > ST ? issued - ST : 0; j < issued; ++j)
-        ptx::mbar_wait(kv_full(j % ST), (uint32_t)(j / ST) & 1u, nullptr);
+      for (int j = nk > KST ? nk - KST : 0; j < nk; ++j)
+        ptx::mbar_wait(k_full(j % KST), (uint32_t)(j / KST) & 1u, nullptr);
+      for (int j = nv > VST ? nv - VST : 0; j < nv; ++j)
+        ptx::mbar_wait(v_full(j % VST), (uint32_t)(j / VST) & 1u, nullptr);
     }
-  } else if (warp == 5) {
+  } else if (warp == kMma) {
     // ---------------------------------------------------------------- MMA
     if (lane == 0) {
       constexpr uint32_t idS = ptx::idesc_bf16_f32(BM, BN);
       constexpr uint32_t idPV = ptx::idesc_bf16_f32_bmn(BM, D);
-      const uint64_t qd = ptx::sdesc_kmajor_sw128(ptx::smem_u32(smem + kOffQ));
-      const uint64_t pd = ptx::sdesc_kmajor_sw128(ptx::smem_u32(smem + kOffP));
-      bool ok = ptx::mbar_wait(q_full, 0, abort_flag);
-      // S_j = Q K_j^T once K_j has landed and S_{j-1} has been read
-      auto issue_s = [&](int j) {
-        const int st = j % ST;
-        if (!ptx::mbar_wait(kv_full(st), (uint32_t)(j / ST) & 1u, abort_flag)) return false;
-        if (j > 0 && !ptx::mbar_wait(s_free, (uint32_t)(j - 1) & 1u, abort_flag)) return false;
-        ptx::tc_fence_after();
-        const uint64_t kd = ptx::sdesc_kmajor_sw128(ptx::smem_u32(smem + kOffK + st * kKVBytes));
+      int nbt[NT];
 #pragma unroll
-        for (int k = 0; k < D / 16; ++k) ptx::mma_bf16(tmem, qd + 2 * k, kd + 2 * k, idS, k > 0 ? 1u : 0u);
-        ptx::mma_commit(s_full);
+      for (int t = 0; t < NT; ++t) nbt[t] = tile_blocks(t);
+      bool ok = ptx::mbar_wait(q_full, 0, abort_flag);
+      // S_t(j) = Q_t K_j^T for every tile that uses block j, once K_j has
+      // landed and the tile's softmax has read S_t(j - 1)
+      auto issue_s = [&](int j) {
+        const int st = j % KST;
+        if (!ptx::mbar_wait(k_full(st), (uint32_t)(j / KST) & 1u, abort_flag)) return false;
+        const uint64_t kd = ptx::sdesc_kmajor_sw128(ptx::smem_u32(smem + C::kOffK + st * kKVBytes));
+#pragma unroll
+        for (int t = 0; t < NT; ++t) {
+          if (j >= nbt[t]) continue;
+          if (j > 0 && !ptx::mbar_wait(s_free(t), (uint32_t)(j - 1) & 1u, abort_flag)) return false;
+          ptx::tc_fence_after();
+          const uint64_t qd = ptx::sdesc_kmajor_sw128(ptx::smem_u32(smem + C::kOffQ + t * kQBytes));
+#pragma unroll
+          for (int k = 0; k < D / 16; ++k)
+            ptx::mma_bf16(tmem + 128u * t, qd + 2 * k, kd + 2 * k, idS, k > 0 ? 1u : 0u);
+          ptx::mma_commit(s_full(t));
+        }
+        ptx::mma_commit(k_empty(st));
         return true;
       };
       if (ok) ok = issue_s(0);
@@ -204,19 +257,29 @@ __global__ void __launch_bounds__(ftc::kThreads, 3)
           ok = false;
           break;
         }
-        // O += P_j V_j once the softmax warps have written P_j
-        if (!ptx::mbar_wait(p_full, (uint32_t)j & 1u, abort_flag)) {
+        // O_t += P_t(j) V_j once each tile's softmax has written P_t(j)
+        const int st = j % VST;
+        if (!ptx::mbar_wait(v_full(st), (uint32_t)(j / VST) & 1u, abort_flag)) {
           ok = false;
           break;
         }
-        ptx::tc_fence_after();
-        const int st = j % ST;
-        const uint64_t vd = ptx::sdesc_kmajor_sw128(ptx::smem_u32(smem + kOffV + st * kKVBytes));
+        const uint64_t vd = ptx::sdesc_kmajor_sw128(ptx::smem_u32(smem + C::kOffV + st * kKVBytes));
 #pragma unroll
-        for (int k = 0; k < BN / 16; ++k)
-          ptx::mma_bf16(tmem + kColO, pd + 2 * k, vd + 128 * k, idPV, (j > 0 || k > 0) ? 1u : 0u);
-        ptx::mma_commit(kv_empty(st));
-        ptx::mma_commit(pv_full);
+        for (int t = 0; t < NT; ++t) {
+          if (j >= nbt[t]) continue;
+          if (!ptx::mbar_wait(p_full(t), (uint32_t)j & 1u, abort_flag)) {
+            ok = false;
+            break;
+          }
+          ptx::tc_fence_after();
+          const uint64_t pd = ptx::sdesc_kmajor_sw128(ptx::smem_u32(smem + C::kOffP + t * kPBytes));
+#pragma unroll
+          for (int k = 0; k < BN / 16; ++k)
+            ptx::mma_bf16(tmem + 128u * t + 64u, pd + 2 * k, vd + 128 * k, idPV, (j > 0 || k > 0) ? 1u : 0u);
+          ptx::mma_commit(pv_full(t));
+        }
+        if (!ok) break;
+        ptx::mma_commit(v_empty(st));
       }
       if (!ok) {
         report_error(a.err, DEV_WAIT_TIMEOUT_MMA);
@@ -228,18 +291,24 @@ __global__ void __launch_bounds__(ftc::kThreads, 3)
     }
   } else {
     // ---------------------------------------------------------------- softmax
-    const int r = threadIdx.x;                              // query row of the tile = TMEM lane
-    const uint32_t trow = tmem + ((uint32_t)(warp * 32) << 16);
-    const int qpos = a.p0 + q0 + r;                         // ALL, OWN
-    uint8_t* prow = smem + kOffP + r * 128;
+    const int t = warp >> 2;                                // this warp's tile
+    const int r = threadIdx.x & 127;                        // query row of the tile = TMEM lane
+    const int tq0 = q0 + t * BM;                            // the tile's first query
+    const int nq = min(BM, a.qrows - tq0);
+    const int nbt = tile_blocks(t);
+    const int key_end = SEG == TSEG_PREFIX ? a.n_pre : a.p0 + tq0 + nq;
+    const uint32_t trow = tmem + 128u * t + ((uint32_t)((warp & 3) * 32) << 16);
+    const uint32_t s_full_t = s_full(t), s_free_t = s_free(t), p_full_t = p_full(t), pv_full_t = pv_full(t);
+    const int qpos = a.p0 + tq0 + r;                        // ALL, OWN
+    uint8_t* prow = smem + C::kOffP + t * kPBytes + r * 128;
     // warp-uniform bounded wait (the tensor-memory accesses below are warp-collective)
     auto wait_all = [&](uint32_t bar, uint32_t parity) {
       return __all_sync(0xffffffffu, ptx::mbar_wait(bar, parity, abort_flag)) != 0;
     };
     float m = -INFINITY, l = 0.f;  // reference maximum (log2 units) and row sum
     bool ok = true;
-    for (int j = 0; j < nb; ++j) {
-      if (!wait_all(s_full, (uint32_t)j & 1u)) {
+    for (int j = 0; j < nbt; ++j) {
+      if (!wait_all(s_full_t, (uint32_t)j & 1u)) {
         ok = false;
         break;
       }
@@ -248,7 +317,7 @@ __global__ void __launch_bounds__(ftc::kThreads, 3)
       ptx::tmem_ld64(trow, s);
       ptx::tc_fence_before();
       __syncwarp();
-      if (lane == 0) ptx::mbar_arrive(s_free);
+      if (lane == 0) ptx::mbar_arrive(s_free_t);
       // mask: keys past the segment, and (own keys) keys after this query
       const int kbase = key0 + j * BN;
       const int lim = SEG == TSEG_PREFIX ? key_end - 1 - kbase : qpos - kbase;
@@ -273,7 +342,7 @@ __global__ void __launch_bounds__(ftc::kThreads, 3)
       // the previous P V product is complete: P's buffer is free, and O may
       // be rescaled to the new reference
       if (j > 0) {
-        if (!wait_all(pv_full, (uint32_t)(j - 1) & 1u)) {
+        if (!wait_all(pv_full_t, (uint32_t)(j - 1) & 1u)) {
           ok = false;
           break;
         }
@@ -282,10 +351,10 @@ __global__ void __launch_bounds__(ftc::kThreads, 3)
 #pragma unroll 1
           for (int hh = 0; hh < D; hh += 8) {
             float ov[8];
-            ptx::tmem_ld8(trow + kColO + (uint32_t)hh, ov);
+            ptx::tmem_ld8(trow + 64u + (uint32_t)hh, ov);
 #pragma unroll
             for (int i = 0; i < 8; ++i) ov[i] *= corr;
-            ptx::tmem_st8(trow + kColO + (uint32_t)hh, ov);
+            ptx::tmem_st8(trow + 64u + (uint32_t)hh, ov);
           }
         }
       }
@@ -311,15 +380,15 @@ __global__ void __launch_bounds__(ftc::kThreads, 3)
       asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
       ptx::tc_fence_before();
       __syncwarp();
-      if (lane == 0) ptx::mbar_arrive(p_full);
+      if (lane == 0) ptx::mbar_arrive(p_full_t);
     }
     float o[D];
 #pragma unroll
     for (int c = 0; c < D; ++c) o[c] = 0.f;
-    if (ok && nb > 0) {
-      if (wait_all(pv_full, (uint32_t)(nb - 1) & 1u)) {
+    if (ok && nbt > 0) {
+      if (wait_all(pv_full_t, (uint32_t)(nbt - 1) & 1u)) {
         ptx::tc_fence_after();
-        ptx::tmem_ld64(trow + kColO, o);
+        ptx::tmem_ld64(trow + 64u, o);
       } else {
         ok = false;
       }
@@ -330,7 +399,7 @@ __global__ void __launch_bounds__(ftc::kThreads, 3)
     }
     ptx::tc_fence_before();
     if (ok && r < nq) {
-      const long long fr = (SEG == TSEG_PREFIX ? 0 : (long long)g * a.q_len) + q0 + r;  // flattened row
+      const long long fr = (SEG == TSEG_PREFIX ? 0 : (long long)g * a.q_len) + tq0 + r;  // flattened row
       if constexpr (SEG == TSEG_PREFIX) {
         float* pp = a.part + (fr * a.H + h) * (D + 2);
 #pragma unroll
@@ -362,9 +431,9 @@ __global__ void __launch_bounds__(ftc::kThreads, 3)
     }
   }
   __syncthreads();
-  if (warp == 5) {
+  if (warp == kMma) {
     ptx::tc_fence_after();
-    ptx::tmem_dealloc(tmem, kTmemCols);
+    ptx::tmem_dealloc(tmem, C::kTmemCols);
   }
 }
 
@@ -376,13 +445,14 @@ bool tc_prefill_disabled() {
   return off;
 }
 
-template <int SEG>
-bool launch_seg(const AttnArgs& a, float* part, int* err, cudaStream_t s) {
+template <int SEG, int NT>
+bool launch_nt(const AttnArgs& a, float* part, int* err, cudaStream_t s) {
   using namespace ftc;
+  using C = Cfg<NT>;
   static PerDevice configured;
   if (configured.get([] {
-        return (int)cudaFuncSetAttribute(k_attn_prefill_tc<SEG>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         kSmemBytes);
+        return (int)cudaFuncSetAttribute(k_attn_prefill_tc<SEG, NT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         C::kSmemBytes);
       }) != (int)cudaSuccess)
     return false;
   CUtensorMap mq, mk, mv;
@@ -413,9 +483,25 @@ bool launch_seg(const AttnArgs& a, float* part, int* err, cudaStream_t s) {
         !tma_map_bf16_3d(&mv, a.V, D, own, (long long)a.G * a.H, D, (long long)a.cap * D, D, BN))
       return false;
   }
-  const dim3 grid((unsigned)((p.qrows + BM - 1) / BM), (unsigned)a.H, SEG == TSEG_PREFIX ? 1u : (unsigned)a.G);
-  launch_kernel(k_attn_prefill_tc<SEG>, grid, kThreads, kSmemBytes, s, mq, mk, mv, p);
+  const dim3 grid((unsigned)((p.qrows + NT * BM - 1) / (NT * BM)), (unsigned)a.H,
+                  SEG == TSEG_PREFIX ? 1u : (unsigned)a.G);
+  launch_kernel(k_attn_prefill_tc<SEG, NT>, grid, C::kThreads, C::kSmemBytes, s, mq, mk, mv, p);
   return true;
+}
+
+// Tiles per CTA: PHOTON_PREFILL_ATTN_TILES=1 or 2 (default 2: two tiles
+// share each K and V block, four tiles resident per SM).
+int tiles_per_cta() {
+  static const int nt = [] {
+    const char* e = getenv("PHOTON_PREFILL_ATTN_TILES");
+    return (e && e[0] == '1') ? 1 : 2;
+  }();
+  return nt;
+}
+
+template <int SEG>
+bool launch_seg(const AttnArgs& a, float* part, int* err, cudaStream_t s) {
+  return tiles_per_cta() == 1 ? launch_nt<SEG, 1>(a, part, err, s) : launch_nt<SEG, 2>(a, part, err, s);
 }
 
 bool args_ok(const AttnArgs& a) {
