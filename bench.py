@@ -21,7 +21,9 @@ Reported (rank 0, one JSON line):
                GEMM launches of one decode chunk) against the measured HBM
                copy peak; roofline_attention the same for the decode attention;
                roofline_prefill the prefill's persistent GEMM against the
-               measured bf16 GEMM peak;
+               measured bf16 GEMM peak, roofline_prefill_attention its
+               causal attention against the same peak (and the SFU's exp2
+               rate);
   hiergen      HierGen decode of the same batch (one timed pass);
   cpu_baseline the CPU oracle timed on a bounded sample on the host cores.
 Between timed steps nothing is flushed: the step's working set (0.66 GB of
@@ -137,13 +139,15 @@ def run_gpu(args) -> None:
     B, T = wl["batch"], wl["prompt_len"]
     model = hal.Model(shape, WEIGHT_SEED)
     if args.only_roofline:
-        # the three roofline measurements alone (a few GB on the device): the
+        # the four roofline measurements alone (a few GB on the device): the
         # small case the kernel-level profiles are captured on
         stream = torch.cuda.current_stream()
         if rank == 0:
             print(json.dumps({"roofline": measure_gemm_roofline(model, wl, dev, stream),
                               "roofline_attention": measure_attn_roofline(model, wl, dev, stream),
-                              "roofline_prefill": measure_prefill_roofline(model, wl, dev, stream)}),
+                              "roofline_prefill": measure_prefill_roofline(model, wl, dev, stream),
+                              "roofline_prefill_attention": measure_prefill_attn_roofline(model, wl, dev,
+                                                                                          stream)}),
                   flush=True)
         model.free()
         if world > 1:
@@ -379,6 +383,7 @@ def run_gpu(args) -> None:
     else:
         roof_attn = measure_attn_roofline(model, wl, dev, stream)
     roof_prefill = measure_prefill_roofline(model, wl, dev, stream)
+    roof_pattn = measure_prefill_attn_roofline(model, wl, dev, stream)
     if pre_cache is not None:
         pre_cache.free()
 
@@ -463,6 +468,7 @@ def run_gpu(args) -> None:
         "roofline": _with_traffic(roof, "roofline"),
         "roofline_attention": _with_traffic(roof_attn, "roofline_attention"),
         "roofline_prefill": _with_traffic(roof_prefill, "roofline_prefill"),
+        "roofline_prefill_attention": _with_traffic(roof_pattn, "roofline_prefill_attention"),
         "clocks": clk.summary(),
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -546,7 +552,7 @@ def peak_batch(hbm_bytes: int, weight_bytes: int, prefix_bytes: int, workspace_b
 
 
 def kernel_sources_sha256() -> str:
-    """sha256 over the relative path and bytes of the sources the three
+    """sha256 over the relative path and bytes of the sources the four
     roofline kernels are compiled from (their .cu files and every csrc
     header), sorted by path: the key under which profiled DRAM traffic stays
     valid.  Host-side orchestration (runtime.cu) and unrelated kernels do not
@@ -554,7 +560,8 @@ def kernel_sources_sha256() -> str:
     import glob
     import hashlib
     csrc = os.path.join(ROOT, "hierarchical_autoregressive_lm_b200", "csrc")
-    files = sorted([os.path.join(csrc, "k_gemm_tc.cu"), os.path.join(csrc, "k_attention.cu")]
+    files = sorted([os.path.join(csrc, "k_gemm_tc.cu"), os.path.join(csrc, "k_attention.cu"),
+                    os.path.join(csrc, "k_attn_prefill_tc.cu")]
                    + glob.glob(os.path.join(csrc, "*.cuh")) + glob.glob(os.path.join(csrc, "*.h")))
     h = hashlib.sha256()
     for f in files:
@@ -897,6 +904,54 @@ def measure_prefill_roofline(model, wl, dev, stream) -> dict:
             "peak_source": f"{src} (cuBLAS bf16 GEMM, burst)", "traffic": None,
             "launches": len(shapes), "flops_per_launch": int(flops / len(shapes)),
             "us_per_launch": round(ms * 1e3 / len(shapes), 3)}
+
+
+def measure_prefill_attn_roofline(model, wl, dev, stream) -> dict:
+    """The prefill's causal attention alone at the level-1 encoder's shape (B
+    sequences x H heads x T/C1 positions, head size dh), on the library's
+    choice of kernel (the tcgen05 one for this shape).  Algorithmic flops
+    count the visible (query, key) pairs only: 4 * dh per pair (Q K^T and
+    P V), against the measured bf16 GEMM peak (burst).  Each pair also costs
+    one exp2 on the SFU, whose peak (16 a clock per SM, at the maximum SM
+    clock) is the other bound this kernel meets; both fractions are given."""
+    import torch
+    import hierarchical_autoregressive_lm_b200 as hal
+    s = model.shape
+    G, H, dh = wl["batch"], s["n_heads"], s["head_dim"]
+    n = wl["prompt_len"] // s["C1"]
+    g = torch.Generator(device=dev).manual_seed(17)
+    q = torch.randn(G * n, H * dh, device=dev, generator=g).to(torch.bfloat16)
+    k = torch.randn(G, H, n, dh, device=dev, generator=g).to(torch.bfloat16)
+    v = torch.randn(G, H, n, dh, device=dev, generator=g).to(torch.bfloat16)
+    o = torch.empty_like(q)
+    for _ in range(3):
+        hal.attn_prefill(q, k, v, n, 0, o)
+    torch.cuda.synchronize()
+    reps = 10
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    torch.cuda.nvtx.range_push("roofline_prefill_attention")
+    a.record()
+    for _ in range(reps):
+        hal.attn_prefill(q, k, v, n, 0, o)
+    b.record()
+    torch.cuda.nvtx.range_pop()
+    torch.cuda.synchronize()
+    ms = a.elapsed_time(b) / reps
+    pairs = G * H * n * (n + 1) // 2
+    flops = 4 * dh * pairs
+    peaks, src = _peaks()
+    tf = flops / (ms / 1e3) / 1e12
+    sms = torch.cuda.get_device_properties(dev).multi_processor_count
+    sfu_peak = 16 * sms * peaks.get("sm_max_mhz", 1965.0) * 1e6  # exp2 per second
+    del q, k, v, o
+    return {"kernel": f"k_attn_prefill_tc (causal, {G} sequences x {H} heads x {n} positions, head {dh})",
+            "bound": "tensor", "achieved": round(tf, 1), "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+            "frac": round(tf / peaks["bf16_tflops"], 4),
+            "peak_source": f"{src} (cuBLAS bf16 GEMM, burst)", "traffic": None,
+            "launches": 1, "flops_per_launch": int(flops), "us_per_launch": round(ms * 1e3, 3),
+            "sfu": {"exp2_per_launch": int(pairs), "peak_exp2_per_s": sfu_peak,
+                    "frac": round(pairs / (ms / 1e3) / sfu_peak, 4)}}
 
 
 def measure_attn_roofline(model, wl, dev, stream) -> dict:

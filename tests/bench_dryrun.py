@@ -155,6 +155,7 @@ roof = lambda *a, **k: {"bound": "hbm", "achieved": 1.0, "peak": 2.0, "unit": "G
 bench.measure_gemm_roofline = roof
 bench.measure_attn_roofline = roof
 bench.measure_prefill_roofline = roof
+bench.measure_prefill_attn_roofline = roof
 bench.ClockSampler = FakeClock
 
 args = argparse.Namespace(gpus=int(os.environ.get("WORLD_SIZE", "1")), steps=2, warmup=3, workload=WL, impl="photon", cpu_budget=1.0,
