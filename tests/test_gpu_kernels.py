@@ -40,8 +40,9 @@ TC_CASES = [
     # persistent warp-specialised kernel (>= 2 tiles per SM): BN 256 and 128, ragged M
     (8192, 2048, 512, 0, 0), (8000, 1152, 256, 0, 0),
     # automatic plan for few tokens: cluster split-K with the reduction in
-    # distributed shared memory; clusters of 16, 8 and 4, token tiles of
-    # 64 / 128 / 256, CTAs left without K slices (K = 18 and 10 slices)
+    # distributed shared memory (CTA pairs by default; the larger clusters in
+    # the subprocess test below), token tiles of 64 / 128 / 256, CTAs left
+    # without K slices (K = 18 and 10 slices)
     (64, 1024, 1024, 0, 1), (256, 1024, 4096, 0, 1), (64, 3072, 1024, 0, 1), (100, 384, 256, 0, 1),
     (256, 4096, 1024, 0, 1), (192, 1152, 1152, 0, 1), (1, 640, 640, 0, 1), (130, 2048, 2048, 0, 1),
 ]
@@ -121,6 +122,44 @@ def test_attn_decode_streamed_bf16(G, H, dh, cap, p0):
 def test_attn_decode_fp32(G, H, cap, q_len, p0):
     got, ref = _attn_case(torch.float32, G, H, 32, cap, q_len, p0, 20)
     np.testing.assert_allclose(got, ref, rtol=1e-5, atol=1e-5)
+
+
+_CLUSTER_SCRIPT = r"""
+import sys, numpy as np, torch
+import hierarchical_autoregressive_lm_b200 as hal
+cases = [(64, 1024, 1024), (256, 1024, 4096), (64, 3072, 1024), (100, 384, 256), (256, 4096, 1024),
+         (192, 1152, 1152), (1, 640, 640), (130, 2048, 2048)]
+worst = 0.0
+for i, (M, N, K) in enumerate(cases):
+    g = torch.Generator().manual_seed(100 + i)
+    A = torch.randn(M, K, generator=g).to(torch.bfloat16)
+    W = torch.randn(N, K, generator=g).to(torch.bfloat16)
+    C = torch.full((M, N), float("nan"), device="cuda")
+    hal.gemm(A.cuda(), W.cuda(), C, path=2, splits=0, swap=1)
+    torch.cuda.synchronize()
+    ref = A.double().numpy() @ W.double().numpy().T
+    got = C.cpu().double().numpy()
+    assert np.isfinite(got).all(), (M, N, K)
+    err = np.abs(got - ref).max() / (1e-5 * np.sqrt(K) * 4 * np.abs(ref).max() + 1e-4)
+    worst = max(worst, err)
+print(worst)
+"""
+
+
+@pytest.mark.parametrize("cmax", ["16", "8", "4"])
+def test_gemm_few_token_clusters_up_to(cmax):
+    # the planner's cluster cap is read once per process: larger clusters
+    # (16, 8, 4 CTAs, reduction through distributed shared memory) run in a
+    # child process with the cap raised
+    import os
+    import subprocess
+    import sys
+    env = dict(os.environ, PHOTON_GEMM_CLUSTER_MAX=cmax)
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    r = subprocess.run([sys.executable, "-c", _CLUSTER_SCRIPT], env=env, cwd=root, capture_output=True,
+                       text=True, timeout=300)
+    assert r.returncode == 0, r.stderr[-2000:]
+    assert float(r.stdout.strip().splitlines()[-1]) <= 1.0
 
 
 # (M, N, K): fused RMSNorm in the cluster kernel (clusters of 2..8, ragged M,
