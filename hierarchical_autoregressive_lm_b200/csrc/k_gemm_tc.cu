@@ -561,6 +561,184 @@ __global__ void __launch_bounds__(192, 1)
   if (warp == 0) ptx::tmem_dealloc(tmem, 2 * BN);
 }
 
+// ------------------------------------------------------------------ CTA-pair persistent kernel
+// Large-M GEMMs (prefill) on CTA pairs: a two-CTA cluster computes 256 x 256
+// output tiles with tcgen05.mma.cta_group::2 (M = 256, N = 256).  CTA r of
+// the pair loads rows r*128.. of the A tile and rows r*128.. of the B tile
+// (its half of N) into its own shared memory; the MMA, issued by CTA 0
+// alone, reads both CTAs' halves and writes each CTA's 128 output rows x 256
+// columns into that CTA's tensor memory.  Per SM and 64-wide K slice that is
+// 32 KB of operands for 128 x 256 outputs, where the single-CTA kernel loads
+// 48 KB for the same work: the operand traffic from L2 that bounds the
+// single-CTA kernel drops by a third.
+//
+// Barriers: a stage's full barrier lives in CTA 0 and counts both CTAs'
+// TMA bytes (CTA 0 arms it for both); its empty barrier lives in each CTA
+// and CTA 0's MMA commit arrives on both.  The accumulator-ready barriers
+// live in each CTA (the same multicast commit); the accumulator-free barrier
+// lives in CTA 0 and counts the epilogue warps of both CTAs.  Cluster
+// barriers after the set-up and before the exit keep every remote arrive
+// and every operand read inside both CTAs' lifetimes.  No TMA multicast.
+constexpr int kPairN = 256;                                     // output columns per pair tile
+constexpr int kPairStages = 6;
+constexpr int kPairBBytes = (kPairN / 2) * kBK * 2;             // this CTA's half of B
+constexpr int kPairStageBytes = kATileBytes + kPairBBytes;      // 32 KB
+constexpr int kPairRingBytes = kPairStages * kPairStageBytes;   // 192 KB
+constexpr int kPairSmemBytes = kPairRingBytes + 256 + 1024;     // + barriers + alignment slack
+
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
+    k_gemm_tc_pair(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, int M,
+                   int N, int nkb, int tiles_n, int n_tiles, Epilogue ep, int* err) {
+  constexpr int ST = kPairStages;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kPairRingBytes);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * ST + 4);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  static_assert((2 * ST + 4) * 8 + 8 <= 256, "control block layout");
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = ptx::cluster_ctarank();  // 0 or 1
+  const int pair = blockIdx.x >> 1, n_pairs = gridDim.x >> 1;
+
+  auto full_bar = [&](int st) { return ptx::smem_u32(bars + st); };        // used in CTA 0
+  auto empty_bar = [&](int st) { return ptx::smem_u32(bars + ST + st); };  // in each CTA
+  auto tfull_bar = [&](int b) { return ptx::smem_u32(bars + 2 * ST + b); };
+  auto tempty_bar = [&](int b) { return ptx::smem_u32(bars + 2 * ST + 2 + b); };  // used in CTA 0
+  auto a_tile = [&](int st) { return ptx::smem_u32(smem + st * kPairStageBytes); };
+  auto b_tile = [&](int st) { return ptx::smem_u32(smem + st * kPairStageBytes + kATileBytes); };
+
+  if (threadIdx.x == 0) {
+    for (int st = 0; st < ST; ++st) {
+      ptx::mbar_init(full_bar(st), 1);
+      ptx::mbar_init(empty_bar(st), 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      ptx::mbar_init(tfull_bar(b), 1);
+      ptx::mbar_init(tempty_bar(b), 8);  // four epilogue warps in each CTA
+    }
+    *abort_flag = 0;
+    ptx::fence_barrier_init();
+    ptx::prefetch_tmap(&tmA);
+    ptx::prefetch_tmap(&tmB);
+  }
+  __syncwarp();
+  if (warp == 0) {
+    ptx::tmem_alloc_pair(ptx::smem_u32(tmem_slot), 2 * kPairN);
+    ptx::tmem_relinquish_pair();
+  }
+  ptx::tc_fence_before();
+  ptx::cluster_sync();  // both CTAs' barriers are initialised before any remote arrive
+  ptx::tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  pdl_wait();  // every role touches global memory only after this point
+  pdl_trigger();
+
+  if (warp == 0) {
+    if (lane == 0) {  // ---- TMA producer (both CTAs)
+      int it = 0;
+      for (int tile = pair; tile < n_tiles && !*abort_flag; tile += n_pairs) {
+        const int mt = tile / tiles_n, nt = tile - mt * tiles_n;
+        for (int kb = 0; kb < nkb; ++kb, ++it) {
+          const int st = it % ST;
+          const uint32_t ph = (uint32_t)(it / ST) & 1u;
+          if (!ptx::mbar_wait(empty_bar(st), ph ^ 1u, abort_flag)) {
+            report_error(err, DEV_WAIT_TIMEOUT_PRODUCER);
+            *abort_flag = 1;
+            break;
+          }
+          const uint32_t full0 = ptx::map_shared_rank(full_bar(st), 0);
+          if (rank == 0) ptx::mbar_arrive_expect_tx(full_bar(st), (uint32_t)(2 * kPairStageBytes));
+          ptx::tma_load_2d_pair(a_tile(st), &tmA, kb * kBK, mt * (2 * kBM) + (int)rank * kBM, full0);
+          ptx::tma_load_2d_pair(b_tile(st), &tmB, kb * kBK, nt * kPairN + (int)rank * (kPairN / 2), full0);
+        }
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0 && rank == 0) {  // ---- MMA issuer (CTA 0 of the pair)
+      constexpr uint32_t idesc = ptx::idesc_bf16_f32(2 * kBM, kPairN);
+      int it = 0, local = 0;
+      for (int tile = pair; tile < n_tiles && !*abort_flag; tile += n_pairs, ++local) {
+        const int b = local & 1;
+        const uint32_t use = (uint32_t)(local >> 1);
+        if (!ptx::mbar_wait(tempty_bar(b), (use & 1u) ^ 1u, abort_flag)) {
+          report_error(err, DEV_WAIT_TIMEOUT_MMA);
+          *abort_flag = 1;
+          break;
+        }
+        ptx::tc_fence_after();
+        const uint32_t d = tmem + (uint32_t)(b * kPairN);
+        for (int kb = 0; kb < nkb; ++kb, ++it) {
+          const int st = it % ST;
+          const uint32_t ph = (uint32_t)(it / ST) & 1u;
+          if (!ptx::mbar_wait(full_bar(st), ph, abort_flag)) {
+            report_error(err, DEV_WAIT_TIMEOUT_MMA);
+            *abort_flag = 1;
+            break;
+          }
+          ptx::tc_fence_after();
+          const uint64_t ad = ptx::sdesc_kmajor_sw128(a_tile(st));
+          const uint64_t bd = ptx::sdesc_kmajor_sw128(b_tile(st));
+#pragma unroll
+          for (int k = 0; k < kBK / 16; ++k)
+            ptx::mma_bf16_pair(d, ad + 2 * k, bd + 2 * k, idesc, (kb > 0 || k > 0) ? 1u : 0u);
+          ptx::mma_commit_pair(empty_bar(st), (uint16_t)3);
+        }
+        if (*abort_flag) break;
+        ptx::mma_commit_pair(tfull_bar(b), (uint16_t)3);  // accumulator b complete in both CTAs
+      }
+    }
+  } else {
+    // ---- epilogue warps 2..5 (both CTAs): this CTA's 128 rows of the tile
+    const int q = warp & 3;
+    int local = 0;
+    for (int tile = pair; tile < n_tiles; tile += n_pairs, ++local) {
+      const int b = local & 1;
+      const uint32_t use = (uint32_t)(local >> 1);
+      if (!ptx::mbar_wait(tfull_bar(b), use & 1u, abort_flag)) {
+        if (lane == 0) report_error(err, DEV_WAIT_TIMEOUT_EPILOGUE);
+        *abort_flag = 1;
+        break;
+      }
+      ptx::tc_fence_after();
+      const int mt = tile / tiles_n, nt = tile - mt * tiles_n;
+      const long long grow = (long long)mt * (2 * kBM) + (long long)rank * kBM + q * 32 + lane;
+      const uint32_t trow = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(b * kPairN);
+      // split RMSNorm consumer: this row's 1 / rms from the producer's slots
+      float rs = 1.f;
+      if (ep.ssq_in != nullptr && grow < M) {
+        float tot = 0.f;
+        for (int sl = 0; sl < ep.ssq_slots; ++sl) tot += ep.ssq_in[grow * ep.ssq_slots + sl];
+        rs = 1.0f / sqrtf(tot / (float)ep.norm_d + ep.norm_eps);
+      }
+#pragma unroll 1
+      for (int j0 = 0; j0 < kPairN; j0 += 64) {
+        float lo[32], hi[32];
+        ptx::tmem_ld32(trow + (uint32_t)j0, lo);
+        ptx::tmem_ld32(trow + (uint32_t)(j0 + 32), hi);
+        if (ep.ssq_in != nullptr) {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            lo[i] *= rs;
+            hi[i] *= rs;
+          }
+        }
+        const int gc = nt * kPairN + j0;
+        if (grow >= M || gc >= N) continue;
+        epi_row64(ep, grow, gc, lo, hi);
+      }
+      ptx::tc_fence_before();
+      __syncwarp();
+      if (lane == 0) ptx::mbar_arrive_cluster(ptx::map_shared_rank(tempty_bar(b), 0));
+    }
+  }
+  ptx::tc_fence_before();
+  __syncthreads();
+  ptx::cluster_sync();  // no remote arrive or operand read outlives either CTA
+  ptx::tc_fence_after();
+  if (warp == 0) ptx::tmem_dealloc_pair(tmem, 2 * kPairN);
+}
+
 // ------------------------------------------------------------------ cluster split-K variant
 // Few-token GEMM in the swapped orientation (decode).  A 128 x BN output
 // tile (128 output features x BN tokens) is computed by the S CTAs of one
@@ -1124,6 +1302,36 @@ void run_tc_persist(const CUtensorMap& ma, const CUtensorMap& mb, int M, int N, 
                 M, N, nkb, tiles_n, n_tiles, nt_major, ep, err);
 }
 
+// CTA-pair persistent GEMM: as many pairs as fit at once (one CTA per SM).
+int pair_resident() {
+  static PerDevice cache;
+  return cache.get([] {
+    if (cudaFuncSetAttribute(k_gemm_tc_pair, cudaFuncAttributeMaxDynamicSharedMemorySize, kPairSmemBytes) !=
+        cudaSuccess) {
+      cudaGetLastError();
+      return 0;
+    }
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(2, 1, 1);
+    cfg.blockDim = dim3(192);
+    cfg.dynamicSmemBytes = kPairSmemBytes;
+    int c = 0;
+    if (cudaOccupancyMaxActiveClusters(&c, k_gemm_tc_pair, &cfg) != cudaSuccess) c = 0;
+    cudaGetLastError();
+    return c;
+  });
+}
+
+void run_tc_pair(const CUtensorMap& ma, const CUtensorMap& mb, int M, int N, int nkb, const Epilogue& ep,
+                 int* err, cudaStream_t s) {
+  const int tiles_n = (N + kPairN - 1) / kPairN;
+  const int n_tiles = ((M + 2 * kBM - 1) / (2 * kBM)) * tiles_n;
+  const int res = pair_resident();
+  const int pairs = n_tiles < res ? n_tiles : res;
+  launch_kernel(k_gemm_tc_pair, dim3(2 * pairs), dim3(192), kPairSmemBytes, s, ma, mb, M, N, nkb, tiles_n,
+                n_tiles, ep, err);
+}
+
 // How many clusters of k_gemm_dec<BN, S, STAGES, NORM> can be resident at
 // once (0 if the cluster shape cannot be launched).  Host-side occupancy
 // query, made once per instance and device; it also sets the instance's
@@ -1396,6 +1604,16 @@ int persist_min_tiles() {
   return v;
 }
 
+// CTA-pair kernel for the normal-orientation large-M GEMMs without a fused
+// argmax (PHOTON_GEMM_PAIR=0 keeps the single-CTA persistent kernel).
+bool pair_enabled() {
+  static const bool on = [] {
+    const char* e = getenv("PHOTON_GEMM_PAIR");
+    return !(e && e[0] == '0');
+  }();
+  return on;
+}
+
 bool persistent_enabled() {
   static const bool on = [] {
     const char* e = getenv("PHOTON_GEMM_PERSISTENT");
@@ -1505,6 +1723,13 @@ bool launch_gemm_tc(const GemmArgs& a, const GemmWorkspace& ws, int* err, cudaSt
     if (!make_map(&ma, a.A, M, K, a.lda, kBM) || !make_map(&mb, a.W, N, K, a.ldw, p.bn)) return false;
     if (a.ep.ssq_in != nullptr && !(p.splits == 1 && p.ga * p.gb >= persist_min_tiles() && persistent_enabled()))
       return false;
+    if (p.splits == 1 && !argmax && p.bn == 256 && p.ga * p.gb >= persist_min_tiles() && persistent_enabled() &&
+        pair_enabled() && N % kPairN == 0 && pair_resident() > 0) {
+      CUtensorMap mb2;
+      if (!make_map(&mb2, a.W, N, K, a.ldw, kPairN / 2)) return false;
+      run_tc_pair(ma, mb2, M, N, nkb, a.ep, err, s);
+      return true;
+    }
     if (p.splits == 1 && (argmax || p.ga * p.gb >= persist_min_tiles()) && persistent_enabled()) {
       const int nt_major = argmax ? 1 : 0;
       if (p.bn == 256)

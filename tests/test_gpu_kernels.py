@@ -37,8 +37,11 @@ TC_CASES = [
     (128, 128, 64, 1, 0), (256, 512, 1024, 1, 0), (300, 256, 512, 1, 0), (4096, 1024, 1024, 1, 0),
     (64, 1024, 1024, 1, 1), (64, 1024, 1024, 4, 1), (256, 3072, 1024, 2, 1), (100, 384, 256, 1, 1),
     (256, 32000, 1024, 1, 1), (1024, 4096, 1024, 1, 0), (512, 1024, 4096, 8, 0),
-    # persistent warp-specialised kernel (>= 2 tiles per SM): BN 256 and 128, ragged M
-    (8192, 2048, 512, 0, 0), (8000, 1152, 256, 0, 0),
+    # persistent warp-specialised kernels (>= 64 tiles): the CTA-pair kernel (256 x 256 tiles,
+    # tcgen05.mma.cta_group::2) where N % 256 == 0, ragged M included; the single-CTA kernel
+    # (BN 256 and 128) otherwise
+    (8192, 2048, 512, 0, 0), (8000, 1152, 256, 0, 0), (1000, 2048, 512, 0, 0), (12345, 1024, 256, 0, 0),
+    (16384, 3072, 1024, 0, 0),
     # automatic plan for few tokens: cluster split-K with the reduction in
     # distributed shared memory (CTA pairs by default; the larger clusters in
     # the subprocess test below), token tiles of 64 / 128 / 256, CTAs left
