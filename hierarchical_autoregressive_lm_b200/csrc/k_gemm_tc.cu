@@ -579,6 +579,10 @@ __global__ void __launch_bounds__(192, 1)
 // lives in CTA 0 and counts the epilogue warps of both CTAs.  Cluster
 // barriers after the set-up and before the exit keep every remote arrive
 // and every operand read inside both CTAs' lifetimes.  No TMA multicast.
+//
+// Work units: the first n_full - rem tiles whole, then the last rem tiles
+// as two 256 x 128 halves each (MMA N = 128, each CTA loading 64 rows of
+// B), so a last wave that would leave most pairs idle is half as long.
 constexpr int kPairN = 256;                                     // output columns per pair tile
 constexpr int kPairStages = 6;
 constexpr int kPairBBytes = (kPairN / 2) * kBK * 2;             // this CTA's half of B
@@ -586,9 +590,28 @@ constexpr int kPairStageBytes = kATileBytes + kPairBBytes;      // 32 KB
 constexpr int kPairRingBytes = kPairStages * kPairStageBytes;   // 192 KB
 constexpr int kPairSmemBytes = kPairRingBytes + 256 + 1024;     // + barriers + alignment slack
 
+struct PairUnit {
+  int mt, n0, width;  // row tile, first column, columns (256 or 128)
+};
+__device__ __forceinline__ PairUnit pair_unit(int u, int tiles_n, int n_full, int rem) {
+  const int whole = n_full - rem;
+  int t = u, half = -1;
+  if (u >= whole) {
+    t = whole + ((u - whole) >> 1);
+    half = (u - whole) & 1;
+  }
+  const int mt = t / tiles_n, nt = t - mt * tiles_n;
+  PairUnit r;
+  r.mt = mt;
+  r.n0 = nt * kPairN + (half > 0 ? kPairN / 2 : 0);
+  r.width = half < 0 ? kPairN : kPairN / 2;
+  return r;
+}
+
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
-    k_gemm_tc_pair(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, int M,
-                   int N, int nkb, int tiles_n, int n_tiles, Epilogue ep, int* err) {
+    k_gemm_tc_pair(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                   const __grid_constant__ CUtensorMap tmB64, int M, int N, int nkb, int tiles_n, int n_full,
+                   int rem, Epilogue ep, int* err) {
   constexpr int ST = kPairStages;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -600,6 +623,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t rank = ptx::cluster_ctarank();  // 0 or 1
   const int pair = blockIdx.x >> 1, n_pairs = gridDim.x >> 1;
+  const int n_units = n_full + rem;
 
   auto full_bar = [&](int st) { return ptx::smem_u32(bars + st); };        // used in CTA 0
   auto empty_bar = [&](int st) { return ptx::smem_u32(bars + ST + st); };  // in each CTA
@@ -621,6 +645,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
     ptx::fence_barrier_init();
     ptx::prefetch_tmap(&tmA);
     ptx::prefetch_tmap(&tmB);
+    ptx::prefetch_tmap(&tmB64);
   }
   __syncwarp();
   if (warp == 0) {
@@ -637,8 +662,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
   if (warp == 0) {
     if (lane == 0) {  // ---- TMA producer (both CTAs)
       int it = 0;
-      for (int tile = pair; tile < n_tiles && !*abort_flag; tile += n_pairs) {
-        const int mt = tile / tiles_n, nt = tile - mt * tiles_n;
+      for (int u = pair; u < n_units && !*abort_flag; u += n_pairs) {
+        const PairUnit w = pair_unit(u, tiles_n, n_full, rem);
+        const bool whole = w.width == kPairN;
+        const uint32_t bytes = 2u * (uint32_t)(kATileBytes + (whole ? kPairBBytes : kPairBBytes / 2));
         for (int kb = 0; kb < nkb; ++kb, ++it) {
           const int st = it % ST;
           const uint32_t ph = (uint32_t)(it / ST) & 1u;
@@ -648,17 +675,20 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
             break;
           }
           const uint32_t full0 = ptx::map_shared_rank(full_bar(st), 0);
-          if (rank == 0) ptx::mbar_arrive_expect_tx(full_bar(st), (uint32_t)(2 * kPairStageBytes));
-          ptx::tma_load_2d_pair(a_tile(st), &tmA, kb * kBK, mt * (2 * kBM) + (int)rank * kBM, full0);
-          ptx::tma_load_2d_pair(b_tile(st), &tmB, kb * kBK, nt * kPairN + (int)rank * (kPairN / 2), full0);
+          if (rank == 0) ptx::mbar_arrive_expect_tx(full_bar(st), bytes);
+          ptx::tma_load_2d_pair(a_tile(st), &tmA, kb * kBK, w.mt * (2 * kBM) + (int)rank * kBM, full0);
+          ptx::tma_load_2d_pair(b_tile(st), whole ? &tmB : &tmB64, kb * kBK, w.n0 + (int)rank * (w.width / 2),
+                                full0);
         }
       }
     }
   } else if (warp == 1) {
     if (lane == 0 && rank == 0) {  // ---- MMA issuer (CTA 0 of the pair)
-      constexpr uint32_t idesc = ptx::idesc_bf16_f32(2 * kBM, kPairN);
+      constexpr uint32_t idesc_whole = ptx::idesc_bf16_f32(2 * kBM, kPairN);
+      constexpr uint32_t idesc_half = ptx::idesc_bf16_f32(2 * kBM, kPairN / 2);
       int it = 0, local = 0;
-      for (int tile = pair; tile < n_tiles && !*abort_flag; tile += n_pairs, ++local) {
+      for (int u = pair; u < n_units && !*abort_flag; u += n_pairs, ++local) {
+        const uint32_t idesc = pair_unit(u, tiles_n, n_full, rem).width == kPairN ? idesc_whole : idesc_half;
         const int b = local & 1;
         const uint32_t use = (uint32_t)(local >> 1);
         if (!ptx::mbar_wait(tempty_bar(b), (use & 1u) ^ 1u, abort_flag)) {
@@ -692,7 +722,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
     // ---- epilogue warps 2..5 (both CTAs): this CTA's 128 rows of the tile
     const int q = warp & 3;
     int local = 0;
-    for (int tile = pair; tile < n_tiles; tile += n_pairs, ++local) {
+    for (int u = pair; u < n_units; u += n_pairs, ++local) {
       const int b = local & 1;
       const uint32_t use = (uint32_t)(local >> 1);
       if (!ptx::mbar_wait(tfull_bar(b), use & 1u, abort_flag)) {
@@ -701,8 +731,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
         break;
       }
       ptx::tc_fence_after();
-      const int mt = tile / tiles_n, nt = tile - mt * tiles_n;
-      const long long grow = (long long)mt * (2 * kBM) + (long long)rank * kBM + q * 32 + lane;
+      const PairUnit w = pair_unit(u, tiles_n, n_full, rem);
+      const long long grow = (long long)w.mt * (2 * kBM) + (long long)rank * kBM + q * 32 + lane;
       const uint32_t trow = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(b * kPairN);
       // split RMSNorm consumer: this row's 1 / rms from the producer's slots
       float rs = 1.f;
@@ -712,7 +742,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
         rs = 1.0f / sqrtf(tot / (float)ep.norm_d + ep.norm_eps);
       }
 #pragma unroll 1
-      for (int j0 = 0; j0 < kPairN; j0 += 64) {
+      for (int j0 = 0; j0 < w.width; j0 += 64) {
         float lo[32], hi[32];
         ptx::tmem_ld32(trow + (uint32_t)j0, lo);
         ptx::tmem_ld32(trow + (uint32_t)(j0 + 32), hi);
@@ -723,7 +753,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
             hi[i] *= rs;
           }
         }
-        const int gc = nt * kPairN + j0;
+        const int gc = w.n0 + j0;
         if (grow >= M || gc >= N) continue;
         epi_row64(ep, grow, gc, lo, hi);
       }
@@ -1322,14 +1352,22 @@ int pair_resident() {
   });
 }
 
-void run_tc_pair(const CUtensorMap& ma, const CUtensorMap& mb, int M, int N, int nkb, const Epilogue& ep,
-                 int* err, cudaStream_t s) {
+void run_tc_pair(const CUtensorMap& ma, const CUtensorMap& mb, const CUtensorMap& mb64, int M, int N, int nkb,
+                 const Epilogue& ep, int* err, cudaStream_t s) {
   const int tiles_n = (N + kPairN - 1) / kPairN;
-  const int n_tiles = ((M + 2 * kBM - 1) / (2 * kBM)) * tiles_n;
+  const int n_full = ((M + 2 * kBM - 1) / (2 * kBM)) * tiles_n;
   const int res = pair_resident();
-  const int pairs = n_tiles < res ? n_tiles : res;
-  launch_kernel(k_gemm_tc_pair, dim3(2 * pairs), dim3(192), kPairSmemBytes, s, ma, mb, M, N, nkb, tiles_n,
-                n_tiles, ep, err);
+  const int pairs = n_full < res ? n_full : res;
+  // a last wave of fewer than half the pairs runs as half-width tiles
+  // (PHOTON_GEMM_PAIR_SPLIT_TAIL=0: whole tiles only)
+  static const bool split_tail = [] {
+    const char* e = getenv("PHOTON_GEMM_PAIR_SPLIT_TAIL");
+    return !(e && e[0] == '0');
+  }();
+  const int tail = n_full % pairs;
+  const int rem = (split_tail && n_full > pairs && tail > 0 && 2 * tail <= pairs) ? tail : 0;
+  launch_kernel(k_gemm_tc_pair, dim3(2 * pairs), dim3(192), kPairSmemBytes, s, ma, mb, mb64, M, N, nkb, tiles_n,
+                n_full, rem, ep, err);
 }
 
 // How many clusters of k_gemm_dec<BN, S, STAGES, NORM> can be resident at
@@ -1725,9 +1763,10 @@ bool launch_gemm_tc(const GemmArgs& a, const GemmWorkspace& ws, int* err, cudaSt
       return false;
     if (p.splits == 1 && !argmax && p.bn == 256 && p.ga * p.gb >= persist_min_tiles() && persistent_enabled() &&
         pair_enabled() && N % kPairN == 0 && pair_resident() > 0) {
-      CUtensorMap mb2;
-      if (!make_map(&mb2, a.W, N, K, a.ldw, kPairN / 2)) return false;
-      run_tc_pair(ma, mb2, M, N, nkb, a.ep, err, s);
+      CUtensorMap mb2, mb64;
+      if (!make_map(&mb2, a.W, N, K, a.ldw, kPairN / 2) || !make_map(&mb64, a.W, N, K, a.ldw, kPairN / 4))
+        return false;
+      run_tc_pair(ma, mb2, mb64, M, N, nkb, a.ep, err, s);
       return true;
     }
     if (p.splits == 1 && (argmax || p.ga * p.gb >= persist_min_tiles()) && persistent_enabled()) {

@@ -42,6 +42,8 @@ TC_CASES = [
     # (BN 256 and 128) otherwise
     (8192, 2048, 512, 0, 0), (8000, 1152, 256, 0, 0), (1000, 2048, 512, 0, 0), (12345, 1024, 256, 0, 0),
     (16384, 3072, 1024, 0, 0),
+    # a last wave of fewer than half the pairs split into 256 x 128 halves (74 pairs on 148 SMs)
+    (16384, 1024, 512, 0, 0), (20000, 1024, 256, 0, 0),
     # automatic plan for few tokens: cluster split-K with the reduction in
     # distributed shared memory (CTA pairs by default; the larger clusters in
     # the subprocess test below), token tiles of 64 / 128 / 256, CTAs left
