@@ -4,22 +4,23 @@
 // table; softmax(Q K^T / sqrt(dh)) V with a causal mask, one softmax per
 // (sequence, head)).
 //
-// One CTA takes 128 consecutive queries of one (group, head), the M = 128
-// rows of a tcgen05 tile, and walks the keys in blocks of 64:
+// A CTA takes NT (default 2) tiles of 128 consecutive queries of one
+// (group, head), each tile the M = 128 rows of a tcgen05 tile, and walks the
+// keys in blocks of 64; the tiles share every K and V block:
 //
-//   warp 4 (one lane)  TMA: the Q tile once, then K and V blocks into rings
-//                      of 3 and 2 stages, K one block ahead of V (a K block
-//                      is free as soon as its S is computed).  The 3-D
-//                      tensor maps stop at the number of written keys, so
-//                      rows past it arrive as zeros and never carry stale
-//                      data into P V;
-//   warp 5 (one lane)  tcgen05.mma: S = Q K^T (M 128, N 64, K 64) into
-//                      tensor memory, and O += P V (M 128, N 64, K 64) into
-//                      a tensor-memory accumulator, V read as an MN-major
-//                      operand straight from its row-major tile; S of block
-//                      j + 1 is issued as soon as the softmax warps have
-//                      read S of block j;
-//   warps 0-3          the softmax, one query row per thread (tensor-memory
+//   one TMA lane       the Q tiles once, then K and V blocks into rings of 3
+//                      and 2 stages, K one block ahead of V (a K block is
+//                      free as soon as its S is computed).  The 3-D tensor
+//                      maps stop at the number of written keys, so rows
+//                      past it arrive as zeros and never carry stale data
+//                      into P V;
+//   one MMA lane       tcgen05.mma per tile t: S_t = Q_t K^T (M 128, N 64,
+//                      K 64) into tensor memory, and O_t += P_t V (M 128,
+//                      N 64, K 64) into a tensor-memory accumulator, V read
+//                      as an MN-major operand straight from its row-major
+//                      tile; S_t of block j + 1 is issued as soon as tile
+//                      t's softmax warps have read S_t of block j;
+//   4 warps per tile   the softmax, one query row per thread (tensor-memory
 //                      lane = row): read S, mask, P = exp2(S - m) as bf16
 //                      into shared memory in the swizzled K-major layout
 //                      the MMA reads, row sums in fp32.  The reference
@@ -28,9 +29,10 @@
 //                      is rescaled in tensor memory only then; O / l at the
 //                      end is the same softmax for any such reference.
 //
-// Three CTAs fit on an SM (73 KB of shared memory, 96 registers a thread,
-// 128 tensor-memory columns each), so one CTA's softmax overlaps the
-// others' MMAs and loads.  Every wait is bounded; a wait that runs out
+// With two tiles a CTA holds 104 KB of shared memory and 256 tensor-memory
+// columns, and two CTAs fit on an SM (96 registers a thread); with one tile
+// (PHOTON_PREFILL_ATTN_TILES=1), three.  One tile's softmax overlaps the
+// other tiles' MMAs and loads.  Every wait is bounded; a wait that runs out
 // records an error word and ends the CTA.
 //
 // Key segments as in the mma.sync kernel: ALL (own keys, no prefix), PREFIX
