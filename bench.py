@@ -858,7 +858,7 @@ def measure_gemm_roofline(model, wl, dev, stream) -> dict:
 
 
 def measure_prefill_roofline(model, wl, dev, stream) -> dict:
-    """The prefill's dominant kernel (the persistent tcgen05 GEMM) alone at
+    """The prefill's dominant kernel (the CTA-pair persistent tcgen05 GEMM) alone at
     the top encoder's prefill shapes: one block's QKV, O, W1 and W2
     projections over M = B*T/C rows, replayed from a captured graph.
     Algorithmic flops = 2*M*N*K per launch, against the measured bf16 GEMM
@@ -897,8 +897,8 @@ def measure_prefill_roofline(model, wl, dev, stream) -> dict:
     peaks, src = _peaks()
     tf = flops / (ms / 1e3) / 1e12
     del graph, bufs
-    return {"kernel": "k_gemm_tc_persist (prefill projections of one top-encoder block, "
-                      f"M={M})", "bound": "tensor", "achieved": round(tf, 1),
+    return {"kernel": "k_gemm_tc_pair (CTA-pair tcgen05 GEMM, 256 x 256 tiles; prefill projections of one "
+                      f"top-encoder block, M={M})", "bound": "tensor", "achieved": round(tf, 1),
             "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
             "frac": round(tf / peaks["bf16_tflops"], 4),
             "peak_source": f"{src} (cuBLAS bf16 GEMM, burst)", "traffic": None,
