@@ -659,6 +659,21 @@ def measure_residency(model, toks, chunks: int, stream, prefix) -> dict:
         out[f"prefill_ms_{name}"] = round(ev[0].elapsed_time(ev[1]), 3)
     model.set_encoder_residency(hal.ENC_RESTORE)
     out.pop("prefill_ms_restore_again", None)
+    # the restore's copy on its own: the same bytes from pinned host memory
+    nb = out["encoder_bytes"]
+    host = torch.empty(nb, dtype=torch.uint8).pin_memory()
+    dev = torch.empty(nb, dtype=torch.uint8, device=toks.device)
+    dev.copy_(host, non_blocking=True)
+    torch.cuda.synchronize()
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+    ev[0].record(stream)
+    dev.copy_(host, non_blocking=True)
+    ev[1].record(stream)
+    torch.cuda.synchronize()
+    ms = ev[0].elapsed_time(ev[1])
+    out["h2d_copy_ms"] = round(ms, 3)
+    out["h2d_gbs"] = round(nb / (ms / 1e3) / 1e9, 1)
+    del host, dev
     return out
 
 

@@ -86,7 +86,8 @@ class photon_model_stats(ctypes.Structure):
     _fields_ = [("param_count", ctypes.c_uint64), ("resident_bytes", ctypes.c_uint64),
                 ("encoder_bytes", ctypes.c_uint64), ("encoder_resident", ctypes.c_int32),
                 ("n_tensors", ctypes.c_int32), ("live_caches", ctypes.c_int32),
-                ("tcgen05_gemm", ctypes.c_int32)]
+                ("tcgen05_gemm", ctypes.c_int32), ("encoder_restores", ctypes.c_uint64),
+                ("encoder_regenerations", ctypes.c_uint64)]
 
 
 class photon_vanilla_config(ctypes.Structure):

@@ -112,6 +112,7 @@ struct photon_model {
   std::vector<std::pair<cudaStream_t, cudaEvent_t>> enc_users;
   int enc_policy = PHOTON_ENC_RESTORE;  // how released encoder weights come back
   void* enc_host = nullptr;             // their pinned host copy (PHOTON_ENC_RESTORE)
+  uint64_t enc_restores = 0, enc_regenerations = 0;  // how often they came back, by which route
 
   // any-L models (photon_init_weights_levels): per level l (index l - 1)
   // chunk size, encoder and decoder depth, and first tensor of each piece
@@ -305,8 +306,10 @@ static int ensure_encoder(photon_model* m, cudaStream_t s) {
   CK(pool_malloc((void**)&m->group_ptr[G_ENC1], m->group_bytes[G_ENC1], s));
   if (m->enc_policy == PHOTON_ENC_RESTORE && m->enc_host) {
     CK(cudaMemcpyAsync(m->group_ptr[G_ENC1], m->enc_host, m->group_bytes[G_ENC1], cudaMemcpyHostToDevice, s));
+    ++m->enc_restores;
   } else {
     generate_group(m, G_ENC1, s);
+    ++m->enc_regenerations;
   }
   CK(cudaGetLastError());
   return PHOTON_OK;
@@ -973,6 +976,8 @@ int photon_model_info(const photon_model* m, photon_model_stats* out) {
   out->n_tensors = (int32_t)m->t.size();
   out->live_caches = m->live_caches;
   out->tcgen05_gemm = m->use_tc ? 1 : 0;
+  out->encoder_restores = m->enc_restores;
+  out->encoder_regenerations = m->enc_regenerations;
   return PHOTON_OK;
 }
 

@@ -248,6 +248,8 @@ typedef struct photon_model_stats {
   int32_t n_tensors;
   int32_t live_caches;
   int32_t tcgen05_gemm;       /* 1 if the tcgen05/TMA GEMM path is available */
+  uint64_t encoder_restores;  /* times released encoder weights came back by a host-to-device copy */
+  uint64_t encoder_regenerations; /* ... by being drawn again (the first draw not counted) */
 } photon_model_stats;
 
 PHOTON_API int photon_model_info(const photon_model* m, photon_model_stats* out);

@@ -41,6 +41,10 @@ def test_residency_policies_give_identical_results():
         model = hal.Model(SHAPE, 7)
         model.set_encoder_residency(policy)
         results[name] = _run(model, toks)
+        # the second prefill brought the weights back by the policy's route
+        info = model.info()
+        assert (info["encoder_restores"], info["encoder_regenerations"]) == {
+            "restore": (1, 0), "regenerate": (0, 1), "keep": (0, 0)}[name], name
         # the released weights come back byte for byte
         idx = 1   # chunker1, a level-1 encoder tensor
         ref = hal.Model(SHAPE, 7)
