@@ -647,18 +647,24 @@ def measure_residency(model, toks, chunks: int, stream, prefix) -> dict:
     import hierarchical_autoregressive_lm_b200 as hal
     out = {"policy": "restore from a pinned host copy after each RecGen prefill (default)",
            "encoder_bytes": int(model.info()["encoder_bytes"])}
+    out["live_caches_before"] = int(model.info()["live_caches"])
     for name, policy in (("restore", hal.ENC_RESTORE), ("keep", hal.ENC_KEEP), ("restore_again", hal.ENC_RESTORE)):
         model.set_encoder_residency(policy)
         ev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
         model.prefill(toks, hal.MODE_REC, chunks, prefix=prefix).free()
         torch.cuda.synchronize()
+        info0 = model.info()
         ev[0].record(stream)
         model.prefill(toks, hal.MODE_REC, chunks, prefix=prefix).free()
         ev[1].record(stream)
         torch.cuda.synchronize()
         out[f"prefill_ms_{name}"] = round(ev[0].elapsed_time(ev[1]), 3)
+        # whether the timed prefill found the weights released, and restored them
+        out[f"{name}_found_released"] = not info0["encoder_resident"]
+        out[f"{name}_restores"] = int(model.info()["encoder_restores"] - info0["encoder_restores"])
     model.set_encoder_residency(hal.ENC_RESTORE)
-    out.pop("prefill_ms_restore_again", None)
+    for k in [k for k in out if k.startswith("restore_again") or k == "prefill_ms_restore_again"]:
+        out.pop(k)
     # the restore's copy on its own: the same bytes from pinned host memory
     nb = out["encoder_bytes"]
     host = torch.empty(nb, dtype=torch.uint8).pin_memory()

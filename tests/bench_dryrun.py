@@ -98,7 +98,7 @@ class FakeModel:
 
     def info(self):
         return {"resident_bytes": 600 * 2 ** 20, "param_count": 384_000_000, "encoder_bytes": 109 * 2 ** 20,
-                "encoder_resident": 0}
+                "encoder_resident": 0, "encoder_restores": 0, "live_caches": 0}
 
     def set_encoder_residency(self, policy):
         assert policy in (hal.ENC_RESTORE, hal.ENC_REGENERATE, hal.ENC_KEEP)
