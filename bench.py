@@ -589,7 +589,8 @@ def profiled_traffic() -> dict:
 
 
 def _with_traffic(roof: dict, key: str) -> dict:
-    roof["traffic"] = profiled_traffic().get(key)
+    if "unavailable" not in roof:
+        roof["traffic"] = profiled_traffic().get(key)
     return roof
 
 
