@@ -88,6 +88,11 @@ struct photon_model {
   bool vanilla = false;
   int i_van = 0, L_van = 0, i_van_g = 0;
   bool graph_failed_van = false;  // the vanilla step could not be captured
+  // RoPE tables (cos, sin per position and frequency), made once per model and
+  // grown when a cache needs more positions; caches point at the latest one,
+  // so every table stays until the model is freed
+  std::vector<float2*> rope_tables;
+  int rope_positions = 0;
   std::vector<TensorRec> t;
   size_t group_bytes[G_COUNT] = {0, 0, 0, 0};
   char* group_ptr[G_COUNT] = {nullptr, nullptr, nullptr, nullptr};
@@ -749,18 +754,36 @@ static size_t attn_ws_need(int dt, int G, int H, int dh, int q_len, int n_plan) 
 }
 
 // cos/sin table: entry [pos][i] = (cos, sin)(pos * theta^(-2i/dh)), computed in fp64.
-static int upload_rope(photon_model* m, float2** out, Allocator& al, int positions) {
-  const int half = m->dh / 2;
-  std::vector<float2> host((size_t)positions * half);
-  for (int p = 0; p < positions; ++p)
-    for (int i = 0; i < half; ++i) {
-      const double inv = std::pow((double)m->cfg.rope_theta, -2.0 * i / m->dh);
-      const double ang = (double)p * inv;
-      host[(size_t)p * half + i] = make_float2((float)std::cos(ang), (float)std::sin(ang));
+// The model's RoPE table for at least `positions` positions: (cos, sin) of
+// p * theta^(-2i/dh), evaluated in fp64 on the host and rounded to fp32.  It
+// is computed when a cache first needs more positions than the model's table
+// has (then for twice as many, so growth is rare), not once per prefill.
+static int upload_rope(photon_model* m, float2** out, int positions) {
+  if (positions > m->rope_positions) {
+    const int n = std::max(positions, 2 * m->rope_positions);
+    const int half = m->dh / 2;
+    std::vector<float2> host((size_t)n * half);
+    for (int p = 0; p < n; ++p)
+      for (int i = 0; i < half; ++i) {
+        const double inv = std::pow((double)m->cfg.rope_theta, -2.0 * i / m->dh);
+        const double ang = (double)p * inv;
+        host[(size_t)p * half + i] = make_float2((float)std::cos(ang), (float)std::sin(ang));
+      }
+    float2* d = nullptr;
+    const size_t bytes = host.size() * sizeof(float2);
+    if (injected_alloc_failure() || cudaMalloc((void**)&d, bytes) != cudaSuccess) {
+      cudaGetLastError();
+      return PHOTON_ERR_OOM;
     }
-  *out = al.get<float2>(host.size() * sizeof(float2));
-  if (!*out) return PHOTON_ERR_OOM;
-  CK(cudaMemcpyAsync(*out, host.data(), host.size() * sizeof(float2), cudaMemcpyHostToDevice, al.s));
+    if (cudaMemcpy(d, host.data(), bytes, cudaMemcpyHostToDevice) != cudaSuccess) {
+      cudaGetLastError();
+      cudaFree(d);
+      return fail(PHOTON_ERR_CUDA, "RoPE table upload failed");
+    }
+    m->rope_tables.push_back(d);
+    m->rope_positions = n;
+  }
+  *out = m->rope_tables.back();
   return PHOTON_OK;
 }
 
@@ -944,6 +967,7 @@ int photon_free_model(photon_model* m) {
   }
   for (int g = 0; g < G_COUNT; ++g)
     if (m->group_ptr[g]) cudaFree(m->group_ptr[g]);
+  for (float2* r : m->rope_tables) cudaFree(r);
   if (m->enc_host) cudaFreeHost(m->enc_host);
   delete m;
   cudaMemPool_t pool = nullptr;
@@ -1169,8 +1193,8 @@ static int prefill_impl(photon_model* m, const photon_cache* prefix, const int32
     return bail(fail(PHOTON_ERR_CUDA, "stream/event creation failed"));
   const int positions =
       std::max(std::max(c->n_pre + c->Ncap, c->n1_pre + N1_own + C2 * max_new_chunks), 2 * C1 + C2) + 1;
-  rc = upload_rope(m, &c->rope, al, positions);
-  if (al.err != cudaSuccess || rc) return bail(PHOTON_ERR_OOM);
+  rc = upload_rope(m, &c->rope, positions);
+  if (al.err != cudaSuccess || rc) return bail(rc ? rc : PHOTON_ERR_OOM);
   if (cudaMemsetAsync(c->d_err, 0, 16, s) != cudaSuccess ||
       cudaMemsetAsync(c->gemm_cnt, 0, kGemmTileCounters * sizeof(int), s) != cudaSuccess ||
       cudaMemsetAsync(c->gemm_cnt_t, 0, kGemmTileCounters * sizeof(int), s) != cudaSuccess ||
@@ -1909,9 +1933,9 @@ static int gen_prefill(photon_model* m, const int32_t* d_tokens, int B, int T, i
   b.err = c->d_err;
   int positions = 2 * C1 + 1;
   for (int l = 0; l < L; ++l) positions = std::max(positions, std::max(g->cap[l], m->Cl[l]) + 1);
-  int rc = upload_rope(m, &c->rope, al, positions);
+  int rc = upload_rope(m, &c->rope, positions);
   b.rope = c->rope;
-  if (al.err != cudaSuccess || rc) return bail(PHOTON_ERR_OOM);
+  if (al.err != cudaSuccess || rc) return bail(rc ? rc : PHOTON_ERR_OOM);
   if (cudaStreamCreateWithFlags(&c->cap, cudaStreamNonBlocking) != cudaSuccess)
     return bail(fail(PHOTON_ERR_CUDA, "stream creation failed"));
   std::vector<int> hn(PHOTON_MAX_LEVELS + 1, 0);
@@ -3055,7 +3079,7 @@ int photon_vanilla_prefill(photon_model* m, const int32_t* d_tokens, int32_t B, 
   c->layer_bytes = (size_t)B * H * c->cap * dh * es;
   c->kc = al.get<char>(c->layer_bytes * L);
   c->vc = al.get<char>(c->layer_bytes * L);
-  if (upload_rope(m, &c->rope, aw, c->cap) != PHOTON_OK) return bail(PHOTON_ERR_OOM);
+  if (upload_rope(m, &c->rope, c->cap) != PHOTON_OK) return bail(PHOTON_ERR_OOM);
   c->x = aw.get<float>((size_t)B * d * 4);
   c->xn = aw.get<void>((size_t)B * d * es);
   c->q = aw.get<void>((size_t)B * d * es);
