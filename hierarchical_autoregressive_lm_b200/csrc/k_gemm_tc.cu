@@ -574,11 +574,12 @@ __global__ void __launch_bounds__(192, 1)
 //
 // Barriers: a stage's full barrier lives in CTA 0 and counts both CTAs'
 // TMA bytes (CTA 0 arms it for both); its empty barrier lives in each CTA
-// and CTA 0's MMA commit arrives on both.  The accumulator-ready barriers
-// live in each CTA (the same multicast commit); the accumulator-free barrier
-// lives in CTA 0 and counts the epilogue warps of both CTAs.  Cluster
-// barriers after the set-up and before the exit keep every remote arrive
-// and every operand read inside both CTAs' lifetimes.  No TMA multicast.
+// and CTA 0's MMA thread commits to both.  The accumulator-ready barriers
+// live in each CTA (two commits again); the accumulator-free barrier lives
+// in CTA 0 and counts the epilogue warps of both CTAs.  Cluster barriers
+// after the set-up and before the exit keep every remote arrive and every
+// operand read inside both CTAs' lifetimes.  Each TMA load copies this
+// GPU's memory into the issuing CTA alone.
 //
 // Work units: the first n_full - rem tiles whole, then the last rem tiles
 // as two 256 x 128 halves each (MMA N = 128, each CTA loading 64 rows of
@@ -712,10 +713,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
 #pragma unroll
           for (int k = 0; k < kBK / 16; ++k)
             ptx::mma_bf16_pair(d, ad + 2 * k, bd + 2 * k, idesc, (kb > 0 || k > 0) ? 1u : 0u);
-          ptx::mma_commit_pair(empty_bar(st), (uint16_t)3);
+          ptx::mma_commit_pair(empty_bar(st));                            // this CTA's stage
+          ptx::mma_commit_pair(ptx::map_shared_rank(empty_bar(st), 1));  // the peer's
         }
         if (*abort_flag) break;
-        ptx::mma_commit_pair(tfull_bar(b), (uint16_t)3);  // accumulator b complete in both CTAs
+        // accumulator b complete in both CTAs
+        ptx::mma_commit_pair(tfull_bar(b));
+        ptx::mma_commit_pair(ptx::map_shared_rank(tfull_bar(b), 1));
       }
     }
   } else {

@@ -189,8 +189,9 @@ __device__ __forceinline__ void mma_bf16(uint32_t tmem_d, uint64_t adesc, uint64
 }
 // CTA-pair forms (cta_group::2): allocation by one warp of each CTA of the
 // pair (same warp index, same destination offset), the MMA issued by the
-// pair's first CTA over both CTAs' operand halves, and a commit that
-// arrives on the barrier at the same offset in every CTA of `mask`.
+// pair's first CTA over both CTAs' operand halves, and a commit that arrives
+// on a barrier given by its shared::cluster address (this CTA's or the
+// peer's) once the issued MMAs are complete.
 __device__ __forceinline__ void tmem_alloc_pair(uint32_t dst_smem, uint32_t ncols) {
   asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(dst_smem),
                "r"(ncols)
@@ -212,12 +213,9 @@ __device__ __forceinline__ void mma_bf16_pair(uint32_t tmem_d, uint64_t adesc, u
       "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
       : "memory");
 }
-__device__ __forceinline__ void mma_commit_pair(uint32_t bar, uint16_t mask) {
-  asm volatile(
-      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(
-          bar),
-      "h"(mask)
-      : "memory");
+__device__ __forceinline__ void mma_commit_pair(uint32_t bar_cluster) {
+  asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar_cluster)
+               : "memory");
 }
 // Arrive on `bar` once all previously issued tcgen05.mma of this thread finish.
 __device__ __forceinline__ void mma_commit(uint32_t bar) {
