@@ -570,7 +570,8 @@ __global__ void __launch_bounds__(192, 1)
 // columns into that CTA's tensor memory.  Per SM and 64-wide K slice that is
 // 32 KB of operands for 128 x 256 outputs, where the single-CTA kernel loads
 // 48 KB for the same work: the operand traffic from L2 that bounds the
-// single-CTA kernel drops by a third.
+// single-CTA kernel drops by a third.  A ring stage holds two 64-wide K
+// slices (64 KB, 3 stages), so each full barrier covers eight MMAs.
 //
 // Barriers: a stage's full barrier lives in CTA 0 and counts both CTAs'
 // TMA bytes (CTA 0 arms it for both); its empty barrier lives in each CTA
@@ -585,9 +586,9 @@ __global__ void __launch_bounds__(192, 1)
 // as two 256 x 128 halves each (MMA N = 128, each CTA loading 64 rows of
 // B), so a last wave that would leave most pairs idle is half as long.
 constexpr int kPairN = 256;                                     // output columns per pair tile
-constexpr int kPairStages = 6;
-constexpr int kPairBBytes = (kPairN / 2) * kBK * 2;             // this CTA's half of B
-constexpr int kPairStageBytes = kATileBytes + kPairBBytes;      // 32 KB
+constexpr int kPairStages = 3;
+constexpr int kPairBBytes = 2 * (kPairN / 2) * kBK * 2;         // this CTA's half of B, two K slices
+constexpr int kPairStageBytes = 2 * kATileBytes + kPairBBytes;  // 64 KB
 constexpr int kPairRingBytes = kPairStages * kPairStageBytes;   // 192 KB
 constexpr int kPairSmemBytes = kPairRingBytes + 256 + 1024;     // + barriers + alignment slack
 
@@ -631,7 +632,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
   auto tfull_bar = [&](int b) { return ptx::smem_u32(bars + 2 * ST + b); };
   auto tempty_bar = [&](int b) { return ptx::smem_u32(bars + 2 * ST + 2 + b); };  // used in CTA 0
   auto a_tile = [&](int st) { return ptx::smem_u32(smem + st * kPairStageBytes); };
-  auto b_tile = [&](int st) { return ptx::smem_u32(smem + st * kPairStageBytes + kATileBytes); };
+  auto b_tile = [&](int st) { return ptx::smem_u32(smem + st * kPairStageBytes + 2 * kATileBytes); };
 
   if (threadIdx.x == 0) {
     for (int st = 0; st < ST; ++st) {
@@ -666,8 +667,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
       for (int u = pair; u < n_units && !*abort_flag; u += n_pairs) {
         const PairUnit w = pair_unit(u, tiles_n, n_full, rem);
         const bool whole = w.width == kPairN;
-        const uint32_t bytes = 2u * (uint32_t)(kATileBytes + (whole ? kPairBBytes : kPairBBytes / 2));
-        for (int kb = 0; kb < nkb; ++kb, ++it) {
+        // both CTAs' A and B for two K slices (a K past the end reads zeros)
+        const uint32_t bytes = 2u * (uint32_t)(2 * kATileBytes + (whole ? kPairBBytes : kPairBBytes / 2));
+        for (int kb = 0; kb < nkb; kb += 2, ++it) {
           const int st = it % ST;
           const uint32_t ph = (uint32_t)(it / ST) & 1u;
           if (!ptx::mbar_wait(empty_bar(st), ph ^ 1u, abort_flag)) {
@@ -678,6 +680,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
           const uint32_t full0 = ptx::map_shared_rank(full_bar(st), 0);
           if (rank == 0) ptx::mbar_arrive_expect_tx(full_bar(st), bytes);
           ptx::tma_load_2d_pair(a_tile(st), &tmA, kb * kBK, w.mt * (2 * kBM) + (int)rank * kBM, full0);
+          ptx::tma_load_2d_pair(a_tile(st) + kATileBytes, &tmA, (kb + 1) * kBK, w.mt * (2 * kBM) + (int)rank * kBM, full0);
+          ptx::tma_load_2d_pair(b_tile(st) + (whole ? kPairBBytes / 2 : kPairBBytes / 4), whole ? &tmB : &tmB64, (kb + 1) * kBK,
+                                w.n0 + (int)rank * (w.width / 2), full0);
           ptx::tma_load_2d_pair(b_tile(st), whole ? &tmB : &tmB64, kb * kBK, w.n0 + (int)rank * (w.width / 2),
                                 full0);
         }
@@ -699,7 +704,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
         }
         ptx::tc_fence_after();
         const uint32_t d = tmem + (uint32_t)(b * kPairN);
-        for (int kb = 0; kb < nkb; ++kb, ++it) {
+        for (int kb = 0; kb < nkb; kb += 2, ++it) {
           const int st = it % ST;
           const uint32_t ph = (uint32_t)(it / ST) & 1u;
           if (!ptx::mbar_wait(full_bar(st), ph, abort_flag)) {
@@ -710,9 +715,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
           ptx::tc_fence_after();
           const uint64_t ad = ptx::sdesc_kmajor_sw128(a_tile(st));
           const uint64_t bd = ptx::sdesc_kmajor_sw128(b_tile(st));
+          // slice 1 of a stage sits one A tile (16 KB) and one B half (16 or 8 KB) further
+          const uint32_t bhalf = (uint32_t)(pair_unit(u, tiles_n, n_full, rem).width == kPairN ? kPairBBytes / 2
+                                                                                              : kPairBBytes / 4);
 #pragma unroll
-          for (int k = 0; k < kBK / 16; ++k)
-            ptx::mma_bf16_pair(d, ad + 2 * k, bd + 2 * k, idesc, (kb > 0 || k > 0) ? 1u : 0u);
+          for (int k = 0; k < 2 * kBK / 16; ++k) {
+            const uint64_t a_k = ad + (uint64_t)((k >> 2) * (kATileBytes >> 4)) + 2 * (k & 3);
+            const uint64_t b_k = bd + (uint64_t)((k >> 2) * (bhalf >> 4)) + 2 * (k & 3);
+            ptx::mma_bf16_pair(d, a_k, b_k, idesc, (kb > 0 || k > 0) ? 1u : 0u);
+          }
           ptx::mma_commit_pair(empty_bar(st));                            // this CTA's stage
           ptx::mma_commit_pair(ptx::map_shared_rank(empty_bar(st), 1));  // the peer's
         }
