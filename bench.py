@@ -373,6 +373,8 @@ def run_gpu(args) -> None:
     # ---- the long-context workload's coarse-KV traffic and resident memory in
     # both modes (measured on its own batch with this model)
     longctx = measure_long_context(model, stream, dev) if args.workload == "c2" and world == 1 else None
+    # ---- the same RecGen decode with the top KV in pages of a pool
+    paged = measure_paged(model, toks, chunks, stream, pre_cache, decode_ms / args.steps / chunks)
 
     # ---- the decode's dominant kernel (its GEMM launches) and its attention,
     # alone, at the same shapes and launch configuration
@@ -447,6 +449,7 @@ def run_gpu(args) -> None:
                     "steps": 1},
         "residency": resid,
         "long_context": longctx,
+        "paged_kv": paged,
         "vanilla_baseline": vanilla_line(van, van_ms, world, value / world / gib) if van else None,
         "block_baseline": block_line(blk, blk_ms, world, value / world / gib,
                                      vanilla_line(van, van_ms, world, value / world / gib) if van else None)
@@ -717,6 +720,51 @@ def measure_long_context(model, stream, dev) -> dict:
                      "tok_s_per_gib": round(B * model.C / (ms / 1e3) / (resident / 2 ** 30), 1)}
         c.free()
     return out
+
+
+def measure_paged(model, toks, chunks: int, stream, prefix, contiguous_ms_per_chunk: float,
+                  page_rows: int = 16) -> dict:
+    """RecGen prefill + multi-chunk decode of the timed batch with the top KV
+    in pages of page_rows positions (photon_prefill_paged), one untimed pass
+    then one timed; the pool holds exactly the pages the batch ends with.
+    Reported beside the contiguous cache's decode time and KV bytes."""
+    import torch
+    import hierarchical_autoregressive_lm_b200 as hal
+    B, T = toks.shape
+    n_own = T // model.C
+    pages = B * (-(-(n_own + chunks) // page_rows))
+    out = torch.empty(B, chunks * model.C, dtype=torch.int32, device=toks.device)
+    try:
+        model.set_kv_pages(page_rows, pages)
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+        for timed in (False, True):
+            torch.cuda.synchronize()
+            if timed:
+                ev[0].record(stream)
+            c = model.prefill_paged(toks, hal.MODE_REC, chunks, prefix=prefix)
+            if timed:
+                ev[1].record(stream)
+                prompt_kv = c.info()["kv_bytes"]
+            c.decode_rec_chunks(chunks, out)
+            if timed:
+                ev[2].record(stream)
+            torch.cuda.synchronize()
+            if timed:
+                final_kv = c.info()["kv_bytes"]
+                free_pages = model.info()["kv_free_pages"]
+            c.free()
+        info = model.info()
+        ms = ev[1].elapsed_time(ev[2]) / chunks
+        return {"page_rows": page_rows, "pool_pages": pages, "pool_gib": round(info["kv_pool_bytes"] / 2 ** 30, 4),
+                "pages_free_at_end": free_pages,
+                "prefill_ms": round(ev[0].elapsed_time(ev[1]), 3),
+                "decode_ms_per_chunk": round(ms, 4), "decode_tok_s": round(B * model.C / (ms / 1e3), 1),
+                "vs_contiguous_decode": round(contiguous_ms_per_chunk / ms, 4),
+                "cache_bytes_after_prefill": int(prompt_kv), "cache_bytes_at_end": int(final_kv)}
+    except hal.PhotonError as e:
+        return {"unavailable": str(e)}
+    finally:
+        model.set_kv_pages(0, 0)
 
 
 def measure_block(shape, toks, wl, stream) -> dict:

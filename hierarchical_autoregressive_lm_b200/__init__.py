@@ -43,7 +43,7 @@ EXPORTED = ("photon_init_weights", "photon_free_model", "photon_prefill",
             "photon_vanilla_free_cache", "photon_launch_count", "photon_last_error",
             "photon_debug_fail_alloc", "photon_selftest_wait_timeout", "photon_init_weights_levels",
             "photon_model_set_encoder_residency", "photon_prefill_shell", "photon_cache_state_buffer",
-            "photon_attn_prefill")
+            "photon_attn_prefill", "photon_model_set_kv_pages", "photon_prefill_paged")
 
 
 class PhotonError(RuntimeError):
@@ -87,7 +87,9 @@ class photon_model_stats(ctypes.Structure):
                 ("encoder_bytes", ctypes.c_uint64), ("encoder_resident", ctypes.c_int32),
                 ("n_tensors", ctypes.c_int32), ("live_caches", ctypes.c_int32),
                 ("tcgen05_gemm", ctypes.c_int32), ("encoder_restores", ctypes.c_uint64),
-                ("encoder_regenerations", ctypes.c_uint64)]
+                ("encoder_regenerations", ctypes.c_uint64), ("kv_page_rows", ctypes.c_int32),
+                ("kv_pool_pages", ctypes.c_int32), ("kv_free_pages", ctypes.c_int32),
+                ("kv_paged_caches", ctypes.c_int32), ("kv_pool_bytes", ctypes.c_uint64)]
 
 
 class photon_vanilla_config(ctypes.Structure):
@@ -120,6 +122,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "photon_free_model": [P],
         "photon_prefill": [P, P, P, I32, I32, I32, I32, P, ctypes.POINTER(P)],
         "photon_prefill_shell": [P, P, I32, I32, I32, I32, P, ctypes.POINTER(P)],
+        "photon_prefill_paged": [P, P, P, I32, I32, I32, I32, P, ctypes.POINTER(P)],
+        "photon_model_set_kv_pages": [P, I32, I32],
         "photon_cache_state_buffer": [P, I32, ctypes.POINTER(P), ctypes.POINTER(SZ)],
         "photon_decode_step_hier": [P, P, P, P, P],
         "photon_decode_step_rec": [P, P, P, P, P],
@@ -330,6 +334,23 @@ class Model:
         _check(load_library().photon_prefill(self._h, None if prefix is None else prefix._h,
                                              _ptr(tokens), B, T, mode, max_new_chunks,
                                              _stream(stream), ctypes.byref(h)))
+        return Cache(self, h, B, prefix)
+
+    def set_kv_pages(self, page_rows: int, pool_pages: int) -> None:
+        """A pool of pool_pages top-KV pages of page_rows positions for prefill_paged
+        ((0, 0) frees it)."""
+        _check(load_library().photon_model_set_kv_pages(self._h, int(page_rows), int(pool_pages)))
+
+    def prefill_paged(self, tokens, mode: int, max_new_chunks: int, prefix: "Cache" = None,
+                      stream=None) -> "Cache":
+        """prefill() with the top KV in pages of the model's pool, taken as positions arrive."""
+        import torch
+        B, T = tokens.shape
+        _need(tokens, torch.int32, B * T, "tokens")
+        h = ctypes.c_void_p()
+        _check(load_library().photon_prefill_paged(self._h, None if prefix is None else prefix._h,
+                                                   _ptr(tokens), B, T, mode, max_new_chunks,
+                                                   _stream(stream), ctypes.byref(h)))
         return Cache(self, h, B, prefix)
 
     def prefill_shell(self, B: int, T: int, mode: int, max_new_chunks: int, prefix: "Cache" = None,

@@ -20,6 +20,15 @@ __device__ __forceinline__ unsigned long long argmax_key(float v, int idx) {
   return ((unsigned long long)b << 32) | (unsigned long long)(0xFFFFFFFFu - (uint32_t)idx);
 }
 
+// Row index (head-size units) of KV slot s of (group g, head h): the
+// contiguous cache [G][H][cap][dh], or a page of a paged one (-1: not to be
+// written).
+__device__ __forceinline__ long long kv_cache_row(const Epilogue& ep, int g, int h, int s) {
+  if (ep.kv_table)
+    return paged_kv_row(ep.kv_table, ep.kv_tab_len, ep.kv_page_rows, ep.kv_pages, ep.H, g, h, s);
+  return ((long long)g * ep.H + h) * ep.cap + s;
+}
+
 template <typename T>
 __device__ __forceinline__ void epi_one(const Epilogue& ep, long long row, int col, float v) {
   switch (ep.kind) {
@@ -67,8 +76,9 @@ __device__ __forceinline__ void epi_pair(const Epilogue& ep, long long row, int 
     st_f(q, o0);
     st_f(q + half, o1);
   } else {
-    T* base = reinterpret_cast<T*>(which == 1 ? ep.k_cache : ep.v_cache) +
-              (((long long)g * ep.H + h) * ep.cap + (pos - ep.kv_off)) * dh + i;
+    const long long kr = kv_cache_row(ep, g, h, pos - ep.kv_off);
+    if (kr < 0) return;
+    T* base = reinterpret_cast<T*>(which == 1 ? ep.k_cache : ep.v_cache) + kr * dh + i;
     st_f(base, o0);
     st_f(base + half, o1);
   }
@@ -162,11 +172,13 @@ __device__ __forceinline__ void epi_row64(const Epilogue& ep, long long row, int
         }
       }
       bf16* o;
-      if (which == 0)
+      if (which == 0) {
         o = reinterpret_cast<bf16*>(ep.q_out) + row * d + within;
-      else
-        o = reinterpret_cast<bf16*>(which == 1 ? ep.k_cache : ep.v_cache) +
-            (((long long)g * ep.H + h) * ep.cap + (pos - ep.kv_off)) * 64;
+      } else {
+        const long long kr = kv_cache_row(ep, g, h, pos - ep.kv_off);
+        if (kr < 0) break;
+        o = reinterpret_cast<bf16*>(which == 1 ? ep.k_cache : ep.v_cache) + kr * 64;
+      }
       store32_bf16(o, lo);
       store32_bf16(o + 32, hi);
       break;

@@ -30,6 +30,10 @@ template <typename T, int DH>
 __device__ __forceinline__ const T* key_row(const AttnArgs& a, const T* own, const T* pre, int g,
                                             int h, int pos) {
   if (pos < a.n_pre) return pre + ((long long)h * a.cap_pre + pos) * DH;
+  if (a.kv_table) {  // paged own keys (an unmapped slot reads page 0 instead of leaving the arrays)
+    const long long row = paged_kv_row(a.kv_table, a.kv_tab_len, a.kv_page_rows, a.kv_pages, a.H, g, h, pos - a.n_pre);
+    return own + (row < 0 ? 0 : row) * DH;
+  }
   return own + (((long long)g * a.H + h) * a.cap + (pos - a.n_pre)) * DH;
 }
 
@@ -76,7 +80,7 @@ __device__ __forceinline__ void cp_async_wait_group() {
   asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
 }
 
-template <typename T, int DH, int QMAX, int W>
+template <typename T, int DH, int QMAX, int W, bool PAGED>
 // Resident warps per SM the one-query kernel is compiled for: 28 = seven
 // 4-warp CTAs (56 registers, a 24 KB ring each), so the 1024 (sequence,
 // head) CTAs of the 600M-class batch-64 decode run as one wave on 148 SMs
@@ -135,6 +139,14 @@ __global__ void __launch_bounds__(32 * W, (QMAX == 1 ? PHOTON_DEC_RESIDENT_WARPS
       const bool pre = key < a.n_pre;
       const T* kr = ok ? (pre ? kpre : kown) + (long long)key * DH : reinterpret_cast<const T*>(a.K);
       const T* vr = ok ? (pre ? vpre : vown) + (long long)key * DH : reinterpret_cast<const T*>(a.V);
+      if constexpr (PAGED) {  // own keys of a paged cache: the slot's page through the table
+        if (ok && !pre) {
+          long long row = paged_kv_row(a.kv_table, a.kv_tab_len, a.kv_page_rows, a.kv_pages, a.H, g, h, key - a.n_pre);
+          if (row < 0) row = 0;  // an unmapped slot reads page 0 instead of leaving the arrays
+          kr = reinterpret_cast<const T*>(a.K) + row * DH + sl * VEC;
+          vr = reinterpret_cast<const T*>(a.V) + row * DH + sl * VEC;
+        }
+      }
 #pragma unroll
       for (int sp = 0; sp < SPL; ++sp) {
         cp_async16_zfill(ptx::smem_u32(slot(st, 0, u, sp)), kr + (ok ? sp * TPK * VEC : 0), ok);
@@ -612,7 +624,7 @@ bool stream_attn_ok(int dt, const AttnArgs& a) {
   auto al16 = [](const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; };
   const int n = a.n_plan > 0 ? a.n_plan : a.p0 + a.q_len;
   return stream_min_keys() > 0 && n >= stream_min_keys() && dt == DT_BF16 && (a.dh == 64 || a.dh == 32) &&
-         a.q_len == 1 &&
+         a.q_len == 1 && a.kv_table == nullptr &&
          (long long)a.G * a.H >= sm_count() && a.q_ld % 8 == 0 && al16(a.Q) && al16(a.K) &&
          al16(a.V) && (a.n_pre == 0 || (al16(a.Kp) && al16(a.Vp)));
 }
@@ -637,18 +649,28 @@ void run_stream(const AttnArgs& a, int* err, cudaStream_t s) {
                 (size_t)kSmem, s, a, (int)per, err);
 }
 
-template <typename T, int DH, int QMAX, int W>
-void run_decode_w(const AttnArgs& a, const DecPlan& p, float* part, int* err, cudaStream_t s) {
+template <typename T, int DH, int QMAX, int W, bool PAGED>
+void run_decode_wp(const AttnArgs& a, const DecPlan& p, float* part, int* err, cudaStream_t s) {
   constexpr int kRingBytes = W * kDecStages * 2 * kDecU * kDecSPL * 32 * 16;
   static PerDevice configured;
   configured.get([] {
-    cudaFuncSetAttribute(k_attn_decode<T, DH, QMAX, W>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    cudaFuncSetAttribute(k_attn_decode<T, DH, QMAX, W, PAGED>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                          kRingBytes);
     return 1;
   });
   dim3 grid(p.splits, a.H, a.G);
-  launch_kernel(k_attn_decode<T, DH, QMAX, W>, grid, 32 * W, kRingBytes, s, a, p.chunk, p.splits,
+  launch_kernel(k_attn_decode<T, DH, QMAX, W, PAGED>, grid, 32 * W, kRingBytes, s, a, p.chunk, p.splits,
                 part, err);
+}
+
+// the paged variant only where the own keys sit in pages (the address of a
+// contiguous cache's row stays one multiply-add)
+template <typename T, int DH, int QMAX, int W>
+void run_decode_w(const AttnArgs& a, const DecPlan& p, float* part, int* err, cudaStream_t s) {
+  if (a.kv_table)
+    run_decode_wp<T, DH, QMAX, W, true>(a, p, part, err, s);
+  else
+    run_decode_wp<T, DH, QMAX, W, false>(a, p, part, err, s);
 }
 
 template <typename T, int DH, int QMAX>
@@ -1132,7 +1154,8 @@ __global__ void __launch_bounds__(32 * kLocalWarps) k_attn_local(AttnArgs a) {
 }
 
 bool local_attn_ok(const AttnArgs& a) {
-  return a.Kp == nullptr && a.p0_dev == nullptr && a.p0 + a.q_len <= kLocalMaxKeys && a.q_len <= 4 &&
+  return a.Kp == nullptr && a.kv_table == nullptr && a.p0_dev == nullptr && a.p0 + a.q_len <= kLocalMaxKeys &&
+         a.q_len <= 4 &&
          (a.dh == 32 || a.dh == 64);
 }
 

@@ -518,7 +518,8 @@ bool args_ok(const AttnArgs& a) {
 // rows (a 128-row tile would mostly idle below that); returns false when
 // the shape is not supported (the caller then takes the mma.sync kernel).
 bool launch_attn_prefill_tc(const AttnArgs& a, int* err, cudaStream_t s) {
-  if (!args_ok(a) || a.q_len < ftc::BM || a.n_pre != 0 || a.Kp != nullptr) return false;
+  // own keys through tensor maps of a contiguous cache (a paged one takes the mma.sync kernel)
+  if (!args_ok(a) || a.q_len < ftc::BM || a.n_pre != 0 || a.Kp != nullptr || a.kv_table) return false;
   if (!(reinterpret_cast<uintptr_t>(a.K) % 16 == 0 && reinterpret_cast<uintptr_t>(a.V) % 16 == 0 &&
         a.p0 + a.q_len <= a.cap && a.p0 >= 0))
     return false;
@@ -533,7 +534,7 @@ bool launch_attn_prefix_tc(const AttnArgs& a, float* part, int* err, cudaStream_
 }
 
 bool launch_attn_own_tc(const AttnArgs& a, float* part, int* err, cudaStream_t s) {
-  if (!args_ok(a) || a.q_len < ftc::BM || a.n_pre <= 0 || !part) return false;
+  if (!args_ok(a) || a.q_len < ftc::BM || a.n_pre <= 0 || !part || a.kv_table) return false;
   if (reinterpret_cast<uintptr_t>(a.K) % 16 || reinterpret_cast<uintptr_t>(a.V) % 16 || a.p0 < a.n_pre ||
       a.p0 - a.n_pre + a.q_len > a.cap)
     return false;

@@ -1239,7 +1239,9 @@ __global__ void __launch_bounds__(kDecThreads, 1)
           } else {
             const int g = (int)(t / ep.q_len);
             const int pos = qp0 + (int)(t - (long long)g * ep.q_len);
-            o = base + (((long long)g * ep.H + h) * ep.cap + (pos - ep.kv_off)) * 64;
+            const long long kr = kv_cache_row(ep, g, h, pos - ep.kv_off);
+            if (kr < 0) continue;
+            o = base + kr * 64;
           }
           st_f(o, o0);
           st_f(o + 32, o1);

@@ -44,6 +44,12 @@ struct Epilogue {
   void* k_cache = nullptr;
   void* v_cache = nullptr;
   int d = 0, H = 0, dh = 0, cap = 0, q_len = 1, p0 = 0, kv_off = 0;
+  // Paged KV (kv_table set): k_cache / v_cache are this layer's page arrays
+  // [kv_pages][H][kv_page_rows][dh]; slot s of group g is row s % rows of
+  // page kv_table[g * kv_tab_len + s / rows].  A slot outside the table or a
+  // page outside the arrays is not written.
+  const int* kv_table = nullptr;
+  int kv_tab_len = 0, kv_page_rows = 0, kv_pages = 0;
   const float2* rope = nullptr;
   // If set, the position of a group's first row is *p0_dev + p0 (read on the
   // device, so a captured decode step can be replayed at later positions).
@@ -128,7 +134,25 @@ struct AttnArgs {
   // chunking is planned for this count; chunks past the live keys write
   // empty partials.
   int n_plan = 0;
+  // Paged own keys (kv_table set): K / V are this layer's page arrays
+  // [kv_pages][H][kv_page_rows][dh] and own slot s of group g is row
+  // s % rows of page kv_table[g * kv_tab_len + s / rows]; a slot outside the
+  // table or a page outside the arrays reads row 0 of page 0 instead.
+  const int* kv_table = nullptr;
+  int kv_tab_len = 0, kv_page_rows = 0, kv_pages = 0;
 };
+
+// Row index (in head-size units) of own slot s of (group g, head h) in a
+// paged KV array, or -1 when the slot or its page is out of range.
+__host__ __device__ inline long long paged_kv_row(const int* table, int tab_len, int rows, int pages, int H, int g,
+                                                  int h, int s) {
+  if (s < 0 || rows <= 0) return -1;
+  const int lp = s / rows;
+  if (lp >= tab_len) return -1;
+  const int phys = table[(long long)g * tab_len + lp];
+  if (phys < 0 || phys >= pages) return -1;
+  return ((long long)phys * H + h) * rows + (s - lp * rows);
+}
 
 // ---- weights -----------------------------------------------------------
 // N(0, sigma^2) draw of tensor `tensor_index` (definition in k_misc.cu).

@@ -93,6 +93,15 @@ struct photon_model {
   // so every table stays until the model is freed
   std::vector<float2*> rope_tables;
   int rope_positions = 0;
+  // paged top KV (photon_model_set_kv_pages): page arrays
+  // [Ltop][K, V][kv_pool_pages][H][kv_page_rows][dh]; a page id names the
+  // same slot in every array, so one table entry maps a run of positions of
+  // one sequence in every layer.  Pages released by a cache become reusable
+  // once the work queued before the release has finished (its event).
+  int kv_page_rows = 0, kv_pool_pages = 0, kv_paged_caches = 0;
+  char* kv_pool = nullptr;
+  std::vector<int> kv_free;
+  std::vector<std::pair<cudaEvent_t, std::vector<int>>> kv_pending;
   std::vector<TensorRec> t;
   size_t group_bytes[G_COUNT] = {0, 0, 0, 0};
   char* group_ptr[G_COUNT] = {nullptr, nullptr, nullptr, nullptr};
@@ -392,6 +401,14 @@ struct photon_cache {
   cudaStream_t stream = nullptr;
   char *top_k = nullptr, *top_v = nullptr;
   size_t top_layer = 0;
+  // paged top KV: top_k / top_v are the model's layer-0 page arrays and
+  // top_layer the stride between layers; kv_table [B][kv_tab_len] maps a
+  // sequence's runs of kv_page_rows positions to pages (host mirror beside)
+  bool paged = false;
+  int* kv_table = nullptr;
+  std::vector<int> kv_table_host;
+  int kv_tab_len = 0, kv_mapped = 0;  // table length; runs mapped per sequence so far
+  std::vector<int> kv_held;
   char *l1_k = nullptr, *l1_v = nullptr;
   size_t l1_layer = 0;
   void* o = nullptr;
@@ -507,6 +524,11 @@ struct StackRun {
   int cap_pre = 0, n_pre = 0;
   const int* p0_dev = nullptr;  // device position of the first row (added to p0)
   int n_plan = 0;               // key count the decode attention is planned for
+  // paged own KV: kc / vc are the page arrays of layer 0, layer_bytes the
+  // stride between layers, and slot s of group g lives in page
+  // kv_table[g * kv_tab_len + s / kv_page_rows]
+  const int* kv_table = nullptr;
+  int kv_tab_len = 0, kv_page_rows = 0, kv_pages = 0;
   bool xn_ready = false;        // the first block's attention norm is already in b.xn
   int sn_rows = 0;              // rows the split-RMSNorm buffers of the Bufs hold (0: none)
 };
@@ -649,6 +671,10 @@ static void run_block(photon_model* m, const BlockW& w, float* x, const StackRun
   e.kv_off = r.kv_off;
   e.rope = b.rope;
   e.p0_dev = r.p0_dev;
+  e.kv_table = r.kv_table;
+  e.kv_tab_len = r.kv_tab_len;
+  e.kv_page_rows = r.kv_page_rows;
+  e.kv_pages = r.kv_pages;
   if (sn && sn_slots > 0) {
     e.ssq_in = b.sn_ss;
     e.ssq_slots = sn_slots;
@@ -681,6 +707,10 @@ static void run_block(photon_model* m, const BlockW& w, float* x, const StackRun
   a.scale = 1.0f / sqrtf((float)m->dh);
   a.p0_dev = r.p0_dev;
   a.n_plan = r.n_plan;
+  a.kv_table = r.kv_table;
+  a.kv_tab_len = r.kv_tab_len;
+  a.kv_page_rows = r.kv_page_rows;
+  a.kv_pages = r.kv_pages;
   bool done = false;
   // with a shared prefix: the prefix once for all queries, then each group's own keys
   if (r.kp && b.pre_ws && prefix_split_enabled())
@@ -968,6 +998,8 @@ int photon_free_model(photon_model* m) {
   for (int g = 0; g < G_COUNT; ++g)
     if (m->group_ptr[g]) cudaFree(m->group_ptr[g]);
   for (float2* r : m->rope_tables) cudaFree(r);
+  for (auto& p : m->kv_pending) cudaEventDestroy(p.first);
+  if (m->kv_pool) cudaFree(m->kv_pool);
   if (m->enc_host) cudaFreeHost(m->enc_host);
   delete m;
   cudaMemPool_t pool = nullptr;
@@ -1002,6 +1034,14 @@ int photon_model_info(const photon_model* m, photon_model_stats* out) {
   out->tcgen05_gemm = m->use_tc ? 1 : 0;
   out->encoder_restores = m->enc_restores;
   out->encoder_regenerations = m->enc_regenerations;
+  out->kv_page_rows = m->kv_page_rows;
+  out->kv_pool_pages = m->kv_pool_pages;
+  size_t held_back = 0;
+  for (const auto& p : m->kv_pending) held_back += p.second.size();
+  out->kv_free_pages = (int32_t)(m->kv_free.size() + held_back);
+  out->kv_paged_caches = m->kv_paged_caches;
+  out->kv_pool_bytes =
+      m->kv_pool ? (uint64_t)m->Ltop * 2 * m->kv_pool_pages * m->H * m->kv_page_rows * m->dh * m->es : 0;
   return PHOTON_OK;
 }
 
@@ -1022,6 +1062,91 @@ int photon_export_weight(photon_model* m, int32_t index, void* d_dst, size_t dst
   return PHOTON_OK;
 }
 
+// ============================================================== paged top KV
+static size_t kv_page_bytes(const photon_model* m) {
+  return (size_t)m->H * m->kv_page_rows * m->dh * m->es;
+}
+
+// n pages from the pool: released pages whose work has finished come back
+// first; if that is not enough, the oldest release is waited for.  False
+// when the pool cannot supply them.
+static bool kv_take(photon_model* m, int n, std::vector<int>& out) {
+  auto reclaim = [&](size_t i) {
+    m->kv_free.insert(m->kv_free.end(), m->kv_pending[i].second.begin(), m->kv_pending[i].second.end());
+    cudaEventDestroy(m->kv_pending[i].first);
+    m->kv_pending.erase(m->kv_pending.begin() + (long)i);
+  };
+  for (size_t i = 0; i < m->kv_pending.size();) {
+    if (cudaEventQuery(m->kv_pending[i].first) == cudaSuccess) {
+      reclaim(i);
+    } else {
+      cudaGetLastError();
+      ++i;
+    }
+  }
+  while ((int)m->kv_free.size() < n && !m->kv_pending.empty()) {
+    cudaEventSynchronize(m->kv_pending[0].first);
+    cudaGetLastError();
+    reclaim(0);
+  }
+  if ((int)m->kv_free.size() < n) return false;
+  out.assign(m->kv_free.end() - n, m->kv_free.end());
+  m->kv_free.resize(m->kv_free.size() - n);
+  return true;
+}
+
+// Releases a paged cache's pages: reusable once the work queued on s so far
+// has finished.
+static void kv_release(photon_model* m, photon_cache* c, cudaStream_t s) {
+  if (c->kv_held.empty()) return;
+  cudaEvent_t e = nullptr;
+  if (cudaEventCreateWithFlags(&e, cudaEventDisableTiming) == cudaSuccess && cudaEventRecord(e, s) == cudaSuccess) {
+    m->kv_pending.emplace_back(e, std::move(c->kv_held));
+  } else {  // cannot order the reuse after the pending work: wait for it
+    cudaGetLastError();
+    if (e) cudaEventDestroy(e);
+    cudaStreamSynchronize(s);
+    m->kv_free.insert(m->kv_free.end(), c->kv_held.begin(), c->kv_held.end());
+  }
+  c->kv_held.clear();
+}
+
+// Maps pages until own slot `slot` of every sequence has one (a new run of
+// kv_page_rows positions per sequence at a time).  The new table entries
+// reach the device on s, before the work that writes those slots; entries
+// are written once and never change while the cache lives.
+static int kv_map_through(photon_cache* c, int slot, cudaStream_t s) {
+  photon_model* m = c->m;
+  const int P = m->kv_page_rows;
+  const int need = slot / P + 1;
+  if (need <= c->kv_mapped) return PHOTON_OK;
+  if (need > c->kv_tab_len) return fail(PHOTON_ERR_CAPACITY, "paged cache is full (%d positions)", c->kv_tab_len * P);
+  const int add = need - c->kv_mapped;
+  std::vector<int> pages;
+  if (!kv_take(m, add * c->B, pages))
+    return fail(PHOTON_ERR_CAPACITY, "the KV page pool (%d pages) has no %d free pages", m->kv_pool_pages,
+                add * c->B);
+  size_t k = 0;
+  for (int lp = c->kv_mapped; lp < need; ++lp)
+    for (int b = 0; b < c->B; ++b) c->kv_table_host[(size_t)b * c->kv_tab_len + lp] = pages[k++];
+  c->kv_held.insert(c->kv_held.end(), pages.begin(), pages.end());
+  // columns kv_mapped .. need-1 of every row (pageable source: staged before the call returns)
+  const size_t pitch = (size_t)c->kv_tab_len * sizeof(int);
+  CK(cudaMemcpy2DAsync(c->kv_table + c->kv_mapped, pitch, c->kv_table_host.data() + c->kv_mapped, pitch,
+                       (size_t)add * sizeof(int), c->B, cudaMemcpyHostToDevice, s));
+  c->kv_mapped = need;
+  c->kv_bytes += (size_t)add * c->B * m->Ltop * 2 * kv_page_bytes(m);
+  return PHOTON_OK;
+}
+
+static void set_paged(StackRun& r, const photon_cache* c) {
+  if (!c->paged) return;
+  r.kv_table = c->kv_table;
+  r.kv_tab_len = c->kv_tab_len;
+  r.kv_page_rows = c->m->kv_page_rows;
+  r.kv_pages = c->m->kv_pool_pages;
+}
+
 // o_all (nullable): also the final-normed top output of every own position,
 // [B * T/C, d] in the storage type (teacher-forced scoring reads them all).
 // shell: allocate and set up the cache as a prefill of T tokens would, but
@@ -1029,7 +1154,7 @@ int photon_export_weight(photon_model* m, int32_t index, void* d_dst, size_t dst
 // of another rank's prefilled cache).
 static int prefill_impl(photon_model* m, const photon_cache* prefix, const int32_t* d_tokens, int32_t B,
                         int32_t T, int32_t mode, int32_t max_new_chunks, void* stream, photon_cache** out,
-                        void* o_all, bool shell = false) {
+                        void* o_all, bool shell = false, bool paged = false) {
   g_err.clear();
   if (!m || !out) return fail(PHOTON_ERR_ARG, "NULL model or out");
   *out = nullptr;
@@ -1049,6 +1174,7 @@ static int prefill_impl(photon_model* m, const photon_cache* prefix, const int32
       return fail(PHOTON_ERR_ARG, "prefix must be prefilled in HIER mode");
     if (prefix->B != 1) return fail(PHOTON_ERR_ARG, "prefix batch must be 1");
     if (prefix->prefix) return fail(PHOTON_ERR_ARG, "nested prefixes are not supported");
+    if (prefix->paged) return fail(PHOTON_ERR_ARG, "a paged cache cannot be a shared prefix");
   }
   const long long rows0 = (long long)B * T;
   if (rows0 > (1ll << 31) / 4) return fail(PHOTON_ERR_ARG, "B*T too large");
@@ -1072,6 +1198,7 @@ static int prefill_impl(photon_model* m, const photon_cache* prefix, const int32
   Allocator al{s, &c->allocs, &c->kv_bytes};
   auto bail = [&](int code) {
     cudaGetLastError();
+    kv_release(m, c, s);
     if (c->side) cudaStreamDestroy(c->side);
     if (c->cap) cudaStreamDestroy(c->cap);
     if (c->hi) cudaStreamDestroy(c->hi);
@@ -1087,13 +1214,31 @@ static int prefill_impl(photon_model* m, const photon_cache* prefix, const int32
   if (rc) return bail(rc);
 
   const size_t hd = (size_t)m->H * m->dh;
-  c->top_layer = (size_t)B * hd * c->Ncap * m->es;
-  c->top_k = al.get<char>(c->top_layer * m->Ltop);
-  c->top_v = al.get<char>(c->top_layer * m->Ltop);
+  if (paged) {
+    // top K / V in the model's pages, mapped run by run as positions arrive
+    c->paged = true;
+    c->kv_tab_len = (c->Ncap + m->kv_page_rows - 1) / m->kv_page_rows;
+    c->kv_table = al.get<int>((size_t)B * c->kv_tab_len * sizeof(int));
+    c->kv_table_host.assign((size_t)B * c->kv_tab_len, -1);
+    c->top_k = m->kv_pool;
+    c->top_v = m->kv_pool + (size_t)m->kv_pool_pages * kv_page_bytes(m);
+    c->top_layer = 2 * (size_t)m->kv_pool_pages * kv_page_bytes(m);
+  } else {
+    c->top_layer = (size_t)B * hd * c->Ncap * m->es;
+    c->top_k = al.get<char>(c->top_layer * m->Ltop);
+    c->top_v = al.get<char>(c->top_layer * m->Ltop);
+  }
   c->l1_layer = (size_t)B * hd * c->N1cap * m->es;
   c->l1_k = al.get<char>(c->l1_layer * m->L1);
   c->l1_v = al.get<char>(c->l1_layer * m->L1);
   if (al.err != cudaSuccess) return bail(PHOTON_ERR_OOM);
+  if (paged) {  // the table (unmapped runs: -1), then pages for the prompt's positions
+    if (cudaMemcpyAsync(c->kv_table, c->kv_table_host.data(), c->kv_table_host.size() * sizeof(int),
+                        cudaMemcpyHostToDevice, s) != cudaSuccess)
+      return bail(fail(PHOTON_ERR_CUDA, "page table upload failed"));
+    const int rc_map = kv_map_through(c, N_own - 1, s);
+    if (rc_map) return bail(rc_map);
+  }
 
   // decode workspace (kept for the cache's lifetime)
   al.counter = &c->ws_bytes;
@@ -1173,7 +1318,7 @@ static int prefill_impl(photon_model* m, const photon_cache* prefix, const int32
     c->stk_part = al.get<float>(stack_local_scratch_bytes(B * C2, d));
     c->stk_cnt = al.get<int>((size_t)c->stk_cnt_len * sizeof(int));
     c->stk_bar = al.get<unsigned int>(256);
-    if (top_mega_enabled() && !prefix &&
+    if (top_mega_enabled() && !prefix && !paged &&
         top_step_supported(B, d, m->H, m->dh, m->f, m->Ltop, C2, c->Ncap) &&
         top_step_ssq_slots(d) <= kSsqCap) {
       c->tk_part_bytes = top_step_part_bytes(d, m->f, C2);
@@ -1275,6 +1420,7 @@ static int prefill_impl(photon_model* m, const photon_cache* prefix, const int32
     rt.vc = c->top_v;
     rt.layer_bytes = c->top_layer;
     rt.cap = c->Ncap;
+    set_paged(rt, c);
     if (prefix) {
       rt.kp = prefix->top_k;
       rt.vp = prefix->top_v;
@@ -1322,6 +1468,7 @@ static int prefill_impl(photon_model* m, const photon_cache* prefix, const int32
     return bail(PHOTON_ERR_CUDA);
   m->live_caches++;
   if (mode == PHOTON_MODE_HIER) m->hier_caches++;
+  if (paged) m->kv_paged_caches++;
   if (prefix) prefix->dependents++;
   *out = c;
   return PHOTON_OK;
@@ -1444,6 +1591,7 @@ static void enqueue_decode(photon_model* m, photon_cache* c, int mode, int32_t* 
     rt.vc = c->top_v;
     rt.layer_bytes = c->top_layer;
     rt.cap = c->Ncap;
+    set_paged(rt, c);
     if (c->prefix) {
       rt.kp = c->prefix->top_k;
       rt.vp = c->prefix->top_v;
@@ -2211,6 +2359,49 @@ int photon_prefill_shell(photon_model* m, const photon_cache* prefix, int32_t B,
   return prefill_impl(m, prefix, nullptr, B, T, mode, max_new_chunks, stream, out, nullptr, true);
 }
 
+int photon_model_set_kv_pages(photon_model* m, int32_t page_rows, int32_t pool_pages) {
+  g_err.clear();
+  if (!m) return fail(PHOTON_ERR_ARG, "model is NULL");
+  if (m->general || m->vanilla) return fail(PHOTON_ERR_ARG, "paged top KV is built for two-level models only");
+  if (page_rows < 0 || pool_pages < 0 || (page_rows == 0) != (pool_pages == 0))
+    return fail(PHOTON_ERR_ARG, "page_rows and pool_pages must both be positive (or both 0 to drop the pool)");
+  if (m->kv_paged_caches) return fail(PHOTON_ERR_ARG, "%d paged caches still hold pages", m->kv_paged_caches);
+  const size_t page = (size_t)m->H * page_rows * m->dh * m->es;
+  const size_t total = (size_t)m->Ltop * 2 * (size_t)pool_pages * page;
+  if (pool_pages > 0 && total / pool_pages / 2 / m->Ltop != page) return fail(PHOTON_ERR_ARG, "pool size overflows");
+  // pages released by freed caches: their work has to finish before the arrays go
+  for (auto& p : m->kv_pending) {
+    cudaEventSynchronize(p.first);
+    cudaEventDestroy(p.first);
+  }
+  m->kv_pending.clear();
+  m->kv_free.clear();
+  if (m->kv_pool) CK(cudaFree(m->kv_pool));
+  m->kv_pool = nullptr;
+  m->kv_page_rows = m->kv_pool_pages = 0;
+  if (pool_pages == 0) return PHOTON_OK;
+  if (cudaMalloc(&m->kv_pool, total) != cudaSuccess) {
+    cudaGetLastError();
+    m->kv_pool = nullptr;
+    return fail(PHOTON_ERR_OOM, "KV page pool of %zu bytes does not fit", total);
+  }
+  m->kv_page_rows = page_rows;
+  m->kv_pool_pages = pool_pages;
+  m->kv_free.resize(pool_pages);
+  for (int i = 0; i < pool_pages; ++i) m->kv_free[i] = pool_pages - 1 - i;  // taken from the back: 0, 1, ...
+  return PHOTON_OK;
+}
+
+int photon_prefill_paged(photon_model* m, const photon_cache* prefix, const int32_t* d_tokens, int32_t B,
+                         int32_t T, int32_t mode, int32_t max_new_chunks, void* stream, photon_cache** out) {
+  g_err.clear();
+  if (out) *out = nullptr;
+  if (!m) return fail(PHOTON_ERR_ARG, "model is NULL");
+  if (m->general || m->vanilla) return fail(PHOTON_ERR_ARG, "paged top KV is built for two-level models only");
+  if (!m->kv_pool) return fail(PHOTON_ERR_ARG, "the model has no KV page pool (photon_model_set_kv_pages)");
+  return prefill_impl(m, prefix, d_tokens, B, T, mode, max_new_chunks, stream, out, nullptr, false, true);
+}
+
 int photon_cache_state_buffer(photon_cache* c, int32_t which, void** d_ptr, size_t* bytes) {
   g_err.clear();
   if (!c || !d_ptr || !bytes) return fail(PHOTON_ERR_ARG, "NULL cache or output pointer");
@@ -2221,6 +2412,7 @@ int photon_cache_state_buffer(photon_cache* c, int32_t which, void** d_ptr, size
   switch (which) {
     case PHOTON_STATE_TOP_K:
     case PHOTON_STATE_TOP_V:
+      if (c->paged) return fail(PHOTON_ERR_ARG, "a paged cache's top KV is not one buffer");
       *d_ptr = which == PHOTON_STATE_TOP_K ? c->top_k : c->top_v;
       *bytes = c->top_layer * m->Ltop;
       break;
@@ -2256,6 +2448,7 @@ int photon_decode_step_ex(photon_model* m, photon_cache* c, int32_t mode, int32_
   if (mode == PHOTON_MODE_HIER && !m->group_ptr[G_ENC1]) RET(ensure_encoder(m, (cudaStream_t)stream));
   cudaStream_t s = (cudaStream_t)stream;
   c->stream = s;
+  if (c->paged) RET(kv_map_through(c, c->N - c->n_pre, s));  // the top slot this step appends
   const int C2 = m->C2;
   // The plain step (no hooks, no logits) is captured once per mode, after
   // one eager step has configured every kernel, and replayed afterwards.
@@ -2408,6 +2601,7 @@ int photon_decode_rec_chunks(photon_model* m, photon_cache* c, int32_t n, int32_
   if (c->steps + n > c->max_new) return fail(PHOTON_ERR_CAPACITY, "cache is full (%d steps)", c->max_new);
   cudaStream_t s = (cudaStream_t)stream;
   c->stream = s;
+  if (c->paged) RET(kv_map_through(c, c->N - c->n_pre + n - 1, s));  // the top slots of all n chunks
   const int B = c->B, C = m->C;
   const size_t pitch = (size_t)n * C * sizeof(int32_t), w = (size_t)C * sizeof(int32_t);
   int t = 0;
@@ -2514,6 +2708,10 @@ int photon_free_cache(photon_cache* c) {
   if (c->ev_fork) cudaEventDestroy(c->ev_fork);
   if (c->ev_join_hi) cudaEventDestroy(c->ev_join_hi);
   if (c->ev_join) cudaEventDestroy(c->ev_join);
+  if (c->paged) {  // pages come back once the work queued so far has finished
+    kv_release(m, c, c->stream);
+    m->kv_paged_caches--;
+  }
   free_list(c->allocs, c->stream);
   // a cache built on a prefix may run on another stream than the prefix's
   // eventual free: finish its work before the prefix can be released
@@ -2627,6 +2825,21 @@ int photon_export_state(photon_cache* c, int32_t which, int32_t layer, void* d_d
       if (layer < 0 || layer >= m->Ltop) return fail(PHOTON_ERR_ARG, "layer out of range");
       const int n = c->N - c->n_pre;
       src = (which == PHOTON_STATE_TOP_K ? c->top_k : c->top_v) + layer * c->top_layer;
+      if (c->paged) {  // gathered page by page into [B][H][n][dh]
+        const size_t row = (size_t)m->dh * es, P = (size_t)m->kv_page_rows, bytes = (size_t)c->B * m->H * n * row;
+        if (out_bytes) *out_bytes = bytes;
+        if (!d_dst || bytes == 0) return PHOTON_OK;
+        if (dst_bytes < bytes) return fail(PHOTON_ERR_ARG, "destination holds %zu bytes, need %zu", dst_bytes, bytes);
+        for (int b = 0; b < c->B; ++b)
+          for (int lp = 0; (size_t)lp * P < (size_t)n; ++lp) {
+            const int phys = c->kv_table_host[(size_t)b * c->kv_tab_len + lp];
+            const size_t r = std::min(P, (size_t)n - lp * P);
+            CK(cudaMemcpy2DAsync((char*)d_dst + ((size_t)b * m->H * n + lp * P) * row, (size_t)n * row,
+                                 src + (size_t)phys * m->H * P * row, P * row, r * row, m->H,
+                                 cudaMemcpyDeviceToDevice, s));
+          }
+        return PHOTON_OK;
+      }
       rows = (size_t)c->B * m->H;
       width = (size_t)n * m->dh * es;
       pitch = (size_t)c->Ncap * m->dh * es;

@@ -250,6 +250,11 @@ typedef struct photon_model_stats {
   int32_t tcgen05_gemm;       /* 1 if the tcgen05/TMA GEMM path is available */
   uint64_t encoder_restores;  /* times released encoder weights came back by a host-to-device copy */
   uint64_t encoder_regenerations; /* ... by being drawn again (the first draw not counted) */
+  int32_t kv_page_rows;       /* paged top KV: positions per page (0: no page pool) */
+  int32_t kv_pool_pages;      /* pages in the pool */
+  int32_t kv_free_pages;      /* pages no live cache holds (released ones included) */
+  int32_t kv_paged_caches;    /* live caches built by photon_prefill_paged */
+  uint64_t kv_pool_bytes;     /* device bytes of the pool (every top layer, K and V) */
 } photon_model_stats;
 
 PHOTON_API int photon_model_info(const photon_model* m, photon_model_stats* out);
@@ -311,6 +316,36 @@ enum {
 PHOTON_API int photon_prefill_shell(photon_model* m, const photon_cache* prefix, int32_t B, int32_t T,
                          int32_t mode, int32_t max_new_chunks, void* stream, photon_cache** out);
 PHOTON_API int photon_cache_state_buffer(photon_cache* c, int32_t which, void** d_ptr, size_t* bytes);
+
+/* Paged top KV (the top encoder's cache grows by one entry per generated
+ * chunk, the explainer's RecGen and memory sections; many requests over one
+ * shared context, its quality section).  A cache built by
+ * photon_prefill_paged keeps its own top-level keys and values in pages of a
+ * pool the model owns instead of a [B][H][Ncap][head_dim] block sized for
+ * max_new_chunks up front: a page holds page_rows consecutive positions of
+ * one sequence, for every head, in every top layer (K and V); pages are
+ * taken when the prefill or a decode step first writes into them, and come
+ * back to the pool when the cache is freed (reusable once the work queued
+ * on the cache's stream before the free has finished).  The computation is
+ * the contiguous cache's: same kernels, same tokens.
+ *
+ * photon_model_set_kv_pages allocates the pool: pool_pages pages of
+ * page_rows positions, Ltop * 2 * pool_pages * n_heads * page_rows *
+ * head_dim elements of the storage type; (0, 0) frees it.  Replaces an
+ * existing pool; refused while a paged cache is live.  Errors: ERR_ARG
+ * (model of other than two levels, sizes, paged caches live), ERR_OOM.
+ *
+ * photon_prefill_paged takes photon_prefill's arguments and errors, plus
+ * ERR_ARG when the model has no pool and ERR_CAPACITY when the pool cannot
+ * supply the prompt's pages.  A decode step that needs a page the pool
+ * cannot supply fails with ERR_CAPACITY before running anything.  A paged
+ * cache may read a contiguous shared prefix but cannot be one, and has no
+ * single top-KV state buffer (photon_cache_state_buffer refuses TOP_K /
+ * TOP_V); photon_export_state gathers its pages. */
+PHOTON_API int photon_model_set_kv_pages(photon_model* m, int32_t page_rows, int32_t pool_pages);
+PHOTON_API int photon_prefill_paged(photon_model* m, const photon_cache* prefix, const int32_t* d_tokens,
+                                    int32_t B, int32_t T, int32_t mode, int32_t max_new_chunks, void* stream,
+                                    photon_cache** out);
 
 /* Copies a piece of cache state (storage type) into d_dst, compacted to
  * the entries in use.  Call with d_dst = NULL to query the size.

@@ -96,9 +96,18 @@ class FakeModel:
     def prefill_shell(self, B, T, mode, max_new, prefix=None, stream=None):
         return FakeCache(self, B, mode, shell=True)
 
+    def set_kv_pages(self, page_rows, pool_pages):
+        assert (page_rows > 0) == (pool_pages > 0)
+        self.pool = pool_pages
+
+    def prefill_paged(self, tokens, mode, max_new, prefix=None, stream=None):
+        assert getattr(self, "pool", 0) > 0
+        return self.prefill(tokens, mode, max_new, prefix, stream)
+
     def info(self):
         return {"resident_bytes": 600 * 2 ** 20, "param_count": 384_000_000, "encoder_bytes": 109 * 2 ** 20,
-                "encoder_resident": 0, "encoder_restores": 0, "live_caches": 0}
+                "encoder_resident": 0, "encoder_restores": 0, "live_caches": 0,
+                "kv_pool_bytes": getattr(self, "pool", 0) * 1024, "kv_free_pages": 0}
 
     def set_encoder_residency(self, policy):
         assert policy in (hal.ENC_RESTORE, hal.ENC_REGENERATE, hal.ENC_KEEP)
