@@ -734,6 +734,7 @@ def measure_paged(model, toks, chunks: int, stream, prefix, contiguous_ms_per_ch
     n_own = T // model.C
     pages = B * (-(-(n_own + chunks) // page_rows))
     out = torch.empty(B, chunks * model.C, dtype=torch.int32, device=toks.device)
+    c = None
     try:
         model.set_kv_pages(page_rows, pages)
         ev = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
@@ -753,6 +754,7 @@ def measure_paged(model, toks, chunks: int, stream, prefix, contiguous_ms_per_ch
                 final_kv = c.info()["kv_bytes"]
                 free_pages = model.info()["kv_free_pages"]
             c.free()
+            c = None
         info = model.info()
         ms = ev[1].elapsed_time(ev[2]) / chunks
         return {"page_rows": page_rows, "pool_pages": pages, "pool_gib": round(info["kv_pool_bytes"] / 2 ** 30, 4),
@@ -764,6 +766,8 @@ def measure_paged(model, toks, chunks: int, stream, prefix, contiguous_ms_per_ch
     except hal.PhotonError as e:
         return {"unavailable": str(e)}
     finally:
+        if c is not None:
+            c.free()
         model.set_kv_pages(0, 0)
 
 

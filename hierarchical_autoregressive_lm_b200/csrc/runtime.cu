@@ -2376,9 +2376,10 @@ int photon_model_set_kv_pages(photon_model* m, int32_t page_rows, int32_t pool_p
   }
   m->kv_pending.clear();
   m->kv_free.clear();
-  if (m->kv_pool) CK(cudaFree(m->kv_pool));
+  char* old_pool = m->kv_pool;
   m->kv_pool = nullptr;
   m->kv_page_rows = m->kv_pool_pages = 0;
+  if (old_pool) CK(cudaFree(old_pool));
   if (pool_pages == 0) return PHOTON_OK;
   if (cudaMalloc(&m->kv_pool, total) != cudaSuccess) {
     cudaGetLastError();
